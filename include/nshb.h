@@ -1,0 +1,182 @@
+/*
+ * nshb.h -- C ABI of the B200 (sm_100a) Muon / Hyperball optimizer step.
+ *
+ * One call performs one optimizer step for a set of 2-D weight matrices:
+ *
+ *   1. momentum   M <- beta M + (1 - beta) G;  U = (1 - beta) G + beta M  (Nesterov)
+ *                 ("Muon: the orthogonalized optimizer explained", momentum recap note
+ *                  and the Muon.step code);
+ *   2. msgn       O = NS_K(U): X = U / (||U||_F + eps) on the wide side, then K times
+ *                 A = X X^T, B = b A + c A^2, X <- a X + B X
+ *                 (same page, Newton-Schulz section and newton_schulz5);
+ *   3. a weight-update rule:
+ *        muon_step          W <- (1 - lr wd) W - lr max(1, m/n)^0.5 O    (Muon.step code)
+ *        hyperball_step     W <- rho (W - eta O/||O||) / ||W - eta O/||O|| ||
+ *                           ("Fantastic Pretraining Optimizers ... II: Hyperball
+ *                            Optimization", Method)
+ *        radial_brake_step  plain Muon step, then ||w|| <- ||w_prev|| + s (||w|| - ||w_prev||)
+ *                           ("Refactor of pre/post weight update hook functions", PR #224,
+ *                            RadialBrake description)
+ *      and two variants of step 2:
+ *        himuon_step        NS run independently on every T x T tile, then Hyperball
+ *                           ("Hierarchical Muon: Tiled Newton-Schulz Updates", abstract)
+ *        newton_muon_step   NS of U (Z Z^T + lambda I)^-1, then Hyperball
+ *                           ("The Newton-Muon Optimizer", abstract)
+ *
+ * Conventions shared by every entry point:
+ *   - Every data pointer (W, G, M, O_out, rho, Z, workspace, norms) is a DEVICE pointer
+ *     owned by the caller.  The library allocates no device or host memory.
+ *   - Matrices are row-major with leading dimension `ld` (elements, ld >= cols) shared by
+ *     W, G and M.  O_out, when given, is row-major with leading dimension `cols`.
+ *   - All work is enqueued on `stream`; no call synchronises with the host except
+ *     nshb_device_status.  Concurrent calls that share a workspace race.
+ *   - Argument errors are returned synchronously and nothing is enqueued.  Conditions met
+ *     on the device (fallbacks, non-finite values, bounded waits that ran out) set bits in a
+ *     status word kept in the workspace; each step clears it first and
+ *     nshb_device_status reads it.  Nothing aborts or traps.
+ */
+#ifndef NSHB_H
+#define NSHB_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *nshb_stream; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum { NSHB_BF16 = 0, NSHB_F32 = 1 } nshb_dtype;
+
+typedef enum {
+  NSHB_OK = 0,
+  NSHB_ERR_NULL = 1,           /* a required pointer is NULL                                 */
+  NSHB_ERR_SHAPE = 2,          /* rows/cols <= 0, ld < cols, misaligned pointer/ld for bf16  */
+  NSHB_ERR_DTYPE = 3,          /* unknown dtype or unsupported dtype combination              */
+  NSHB_ERR_PARAM = 4,          /* a scalar parameter out of range                             */
+  NSHB_ERR_WORKSPACE = 5,      /* workspace smaller than nshb_workspace_size or misaligned    */
+  NSHB_ERR_CUDA = 6,           /* a CUDA runtime call or a kernel launch failed               */
+  NSHB_ERR_DEVICE_TIMEOUT = 7, /* (device status) a bounded wait inside a kernel ran out      */
+  NSHB_ERR_NONFINITE = 8,      /* (device status) a NaN/Inf norm was met                      */
+  NSHB_ERR_ZERO_NORM = 9,      /* (device status) radius taken from a zero weight norm        */
+  NSHB_ERR_UNSUPPORTED = 10    /* operation/size not supported by this build                  */
+} nshb_status;
+
+/* Bits of the device status word (nshb_device_status). */
+#define NSHB_DEV_ZERO_NORM_FALLBACK 0x1u /* ||W - eta U_hat|| < hb_eps: step skipped, W kept on its sphere */
+#define NSHB_DEV_NONFINITE 0x2u          /* a momentum, update or weight norm was NaN/Inf                  */
+#define NSHB_DEV_TIMEOUT 0x4u            /* a bounded device wait ran out; results are not valid           */
+#define NSHB_DEV_ZERO_RADIUS 0x8u        /* rho <= 0 asked for the current norm, which was < hb_eps        */
+#define NSHB_DEV_NOT_SPD 0x10u           /* Newton-Muon: Z Z^T + lambda I not positive definite in fp32    */
+
+typedef enum {
+  NSHB_OP_MUON = 0,
+  NSHB_OP_HYPERBALL = 1,
+  NSHB_OP_RADIAL_BRAKE = 2,
+  NSHB_OP_HIMUON = 3,
+  NSHB_OP_NEWTON_MUON = 4
+} nshb_op;
+
+/* One weight matrix (rows x cols).  W is updated in place, G is read, M is the fp32
+ * momentum buffer (zero before the first step; the only state a step keeps).
+ * W and G share w_dtype.  For NSHB_BF16, W, G and M must be 16-byte aligned and ld a
+ * multiple of 8; for NSHB_F32 W/G/M need 16-byte alignment and ld a multiple of 4.
+ * O_out (optional, may be NULL) receives the orthogonalised update O = NS_K(U)
+ * (before any step-length or shape scaling), dtype w_dtype, leading dimension cols.
+ * z_index picks the layer input Z of newton_muon_step (ignored elsewhere). */
+typedef struct {
+  int64_t rows, cols, ld;
+  int32_t w_dtype; /* nshb_dtype */
+  int32_t z_index;
+  void *W;
+  const void *G;
+  float *M;
+  void *O_out;
+} nshb_matrix;
+
+/* Step parameters.  Defaults (nshb_default_params): beta 0.95, Nesterov, K = 5 with
+ * (a, b, c) = (3.4445, -4.7750, 2.0315), ns_eps 1e-7, bf16 tensor-core NS, lr 0.02,
+ * wd 0, eta 0.02, rho NULL, hb_eps 1e-8, brake 0.5 / 1.0, tile 256, ridge_rel 1e-3. */
+typedef struct {
+  float beta;            /* momentum coefficient, [0, 1)                                    */
+  int32_t nesterov;      /* 1: U = (1-beta) G + beta M; 0: U = M                             */
+  int32_t ns_steps;      /* K >= 1 (<= 32)                                                   */
+  int32_t ns_precision;  /* NSHB_BF16: bf16 tensor cores, fp32 accumulate; NSHB_F32: fp32     */
+  const float *coeffs;   /* HOST pointer to ns_steps x 3 (a, b, c) rows, or NULL for the      */
+                         /* constant quintic (3.4445, -4.7750, 2.0315)                        */
+  float ns_eps;          /* additive eps of the NS normalisation, > 0                         */
+  float lr;              /* muon_step / radial_brake_step learning rate                       */
+  float weight_decay;    /* muon_step decoupled weight decay                                  */
+  float eta;             /* Hyperball step length (absolute Frobenius length), >= 0           */
+  const float *rho;      /* DEVICE array [n_mats] of radii; entry <= 0, or rho == NULL, means */
+                         /* "use the current ||W||_F" (radius=None in the hook)               */
+  float hb_eps;          /* numerical-zero threshold for norms, > 0                           */
+  float brake_out;       /* RadialBrake outward factor in [0, 1]                              */
+  float brake_in;        /* RadialBrake inward factor in [0, 1]                               */
+  int32_t tile;          /* HiMuon tile size T: 128, 256 or 512                               */
+  float ridge_rel;       /* Newton-Muon: lambda = ridge_rel * tr(Z Z^T) / d_in, >= 0          */
+  uint32_t debug_flags;  /* 0 in normal use; bit 0 shortens the device wait limit (tests)     */
+} nshb_params;
+
+/* Fills *p with the defaults listed above.  Returns NSHB_ERR_NULL if p is NULL. */
+nshb_status nshb_default_params(nshb_params *p);
+
+/* Bytes of device workspace that a step of kind `op` on these matrices needs.
+ * `n_tokens` and the Z rows matter only for NSHB_OP_NEWTON_MUON (pass 0 / NULL otherwise).
+ * Host-only: touches no device memory.  The workspace must be 256-byte aligned. */
+nshb_status nshb_workspace_size(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p,
+                                int32_t op, const int64_t *z_rows, int32_t n_z, size_t *bytes);
+
+/* Muon step (Muon.step code): momentum, NS, W <- (1 - lr wd) W - lr max(1, m/n)^0.5 O. */
+nshb_status muon_step(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, void *ws,
+                      size_t ws_bytes, nshb_stream stream);
+
+/* Muon step wrapped by Hyperball (Hyperball paper, Method):
+ * W <- rho (W - eta U_hat) / ||W - eta U_hat||_F with U_hat = O / max(||O||_F, hb_eps).
+ * If ||W - eta U_hat|| < hb_eps the step is skipped and W <- rho W / ||W||
+ * (NSHB_DEV_ZERO_NORM_FALLBACK).  Shape scaling and weight decay do not apply. */
+nshb_status hyperball_step(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, void *ws,
+                           size_t ws_bytes, nshb_stream stream);
+
+/* Muon step followed by the RadialBrake hook (PR #224): w = w_prev - lr max(1,m/n)^0.5 O,
+ * then w <- w (||w_prev|| + s (||w|| - ||w_prev||)) / ||w||, s = brake_out if the norm grew,
+ * else brake_in; w is left as is when ||w|| < hb_eps.  weight_decay must be 0. */
+nshb_status radial_brake_step(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p,
+                              void *ws, size_t ws_bytes, nshb_stream stream);
+
+/* Hierarchical Muon wrapped by Hyperball: U is cut into T x T tiles anchored at (0, 0)
+ * (edge tiles are the remainder), every tile gets its own normalisation and NS map,
+ * then the Hyperball rule acts on the whole matrix.  bf16 NS only. */
+nshb_status himuon_step(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, void *ws,
+                        size_t ws_bytes, nshb_stream stream);
+
+/* Newton-Muon wrapped by Hyperball: P = U (Z Z^T + lambda I)^-1 with
+ * lambda = ridge_rel tr(Z Z^T) / d_in, solved through an fp32 Cholesky factorisation,
+ * then O = NS_K(P) and the Hyperball rule.  Z[j] is a DEVICE pointer to a bf16 row-major
+ * z_rows[j] x n_tokens matrix (leading dimension n_tokens, 16-byte aligned, n_tokens a
+ * multiple of 64); matrix i uses Z[mats[i].z_index], which needs z_rows == cols.
+ * Z and z_rows are HOST arrays of n_z entries. */
+nshb_status newton_muon_step(const nshb_matrix *mats, int32_t n_mats, const void *const *Z,
+                             const int64_t *z_rows, int32_t n_z, int64_t n_tokens,
+                             const nshb_params *p, void *ws, size_t ws_bytes, nshb_stream stream);
+
+/* out[i] = ||W_i||_F (fp32) into the DEVICE array out (n_mats floats), e.g. rho = ||W0||.
+ * Needs a workspace of nshb_workspace_size(..., NSHB_OP_MUON, ...) bytes. */
+nshb_status nshb_fro_norms(const nshb_matrix *mats, int32_t n_mats, float *out, void *ws,
+                           size_t ws_bytes, nshb_stream stream);
+
+/* Synchronises `stream`, then copies the device status word of the last step that used
+ * this workspace into *flags (NSHB_DEV_* bits).  The one call that blocks the host. */
+nshb_status nshb_device_status(const void *ws, nshb_stream stream, uint32_t *flags);
+
+/* Static, NUL-terminated name of a status code. */
+const char *nshb_status_string(int32_t status);
+
+/* ABI version (major * 10000 + minor * 100 + patch). */
+int32_t nshb_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NSHB_H */

@@ -1,0 +1,189 @@
+"""B200 (sm_100a) Muon / Hyperball optimizer step.
+
+Python binding of libnshb.so (C ABI in include/nshb.h).  This module only marshals
+arguments: the step itself -- momentum, Newton-Schulz, the weight-update rule -- runs in
+the library's CUDA kernels.  PyTorch is used for device memory and streams only.
+
+    import newton_schulz_hyperball_b200 as nshb
+    mats = nshb.matrices(W_list, G_list, M_list)
+    p = nshb.params(eta=0.02, rho=rho_dev)
+    ws = nshb.workspace(mats, p, nshb.NSHB_OP_HYPERBALL)
+    nshb.hyperball_step(mats, p, ws)
+"""
+from __future__ import annotations
+
+import ctypes
+
+from . import _abi
+from ._abi import (  # noqa: F401  (re-exported constants)
+    NSHB_BF16, NSHB_F32, NSHB_OK, NSHB_ERR_NULL, NSHB_ERR_SHAPE, NSHB_ERR_DTYPE, NSHB_ERR_PARAM,
+    NSHB_ERR_WORKSPACE, NSHB_ERR_CUDA, NSHB_ERR_DEVICE_TIMEOUT, NSHB_ERR_NONFINITE, NSHB_ERR_ZERO_NORM,
+    NSHB_ERR_UNSUPPORTED, NSHB_DEV_ZERO_NORM_FALLBACK, NSHB_DEV_NONFINITE, NSHB_DEV_TIMEOUT,
+    NSHB_DEV_ZERO_RADIUS, NSHB_DEV_NOT_SPD, NSHB_OP_MUON, NSHB_OP_HYPERBALL, NSHB_OP_RADIAL_BRAKE,
+    NSHB_OP_HIMUON, NSHB_OP_NEWTON_MUON, nshb_matrix, nshb_params,
+)
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libnshb.so (raises ImportError if it was not built)."""
+    global _LIB
+    if _LIB is None:
+        _LIB = _abi.load()
+    return _LIB
+
+
+class NshbError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lib().nshb_status_string(status).decode()}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != NSHB_OK:
+        raise NshbError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return NSHB_BF16
+    if t.dtype == torch.float32:
+        return NSHB_F32
+    raise TypeError(f"unsupported weight dtype {t.dtype}")
+
+
+def matrices(W, G, M, O_out=None, z_index=None):
+    """ctypes array of nshb_matrix for lists of 2-D CUDA tensors (row-major, unit column stride)."""
+    n = len(W)
+    arr = (nshb_matrix * max(n, 1))()
+    for i in range(n):
+        w, g, m = W[i], G[i], M[i]
+        if w.dim() != 2 or w.stride(1) != 1 or g.stride() != w.stride() or m.stride() != w.stride():
+            raise ValueError("W, G and M must be 2-D with equal strides and unit column stride")
+        arr[i].rows, arr[i].cols = w.shape
+        arr[i].ld = w.stride(0)
+        arr[i].w_dtype = _dtype_code(w)
+        arr[i].z_index = -1 if z_index is None else int(z_index[i])
+        arr[i].W, arr[i].G, arr[i].M = _ptr(w), _ptr(g), _ptr(m)
+        arr[i].O_out = _ptr(O_out[i]) if O_out is not None else None
+    arr._n = n
+    arr._keep = (W, G, M, O_out)
+    return arr
+
+
+def params(**kw) -> nshb_params:
+    """nshb_params with the library defaults, overridden by keyword.  `coeffs` may be a
+    list of (a, b, c) rows; `rho` a CUDA float32 tensor (or a raw device pointer)."""
+    p = nshb_params()
+    _check(lib().nshb_default_params(ctypes.byref(p)), "nshb_default_params")
+    keep = []
+    for k, v in kw.items():
+        if k == "coeffs":
+            if v is None:
+                p.coeffs = None
+            else:
+                flat = [float(x) for row in v for x in row]
+                buf = (ctypes.c_float * len(flat))(*flat)
+                keep.append(buf)
+                p.coeffs = ctypes.cast(buf, ctypes.POINTER(ctypes.c_float))
+        elif k == "rho":
+            keep.append(v)
+            p.rho = _ptr(v)
+        elif k == "nesterov":
+            p.nesterov = 1 if v else 0
+        else:
+            if not hasattr(p, k):
+                raise KeyError(k)
+            setattr(p, k, v)
+    p._keep = keep
+    return p
+
+
+def _n(mats) -> int:
+    return getattr(mats, "_n", len(mats))
+
+
+def workspace_size(mats, p, op: int, z_rows=None) -> int:
+    out = ctypes.c_size_t(0)
+    zr, nz = None, 0
+    if z_rows is not None:
+        nz = len(z_rows)
+        zr = (ctypes.c_int64 * max(nz, 1))(*[int(x) for x in z_rows])
+    _check(lib().nshb_workspace_size(mats, _n(mats), ctypes.byref(p), op, zr, nz, ctypes.byref(out)),
+           "nshb_workspace_size")
+    return out.value
+
+
+def workspace(mats, p, op: int, device=None, z_rows=None):
+    """A device workspace (torch uint8 tensor, 256-byte aligned by the caching allocator)."""
+    import torch
+    nbytes = workspace_size(mats, p, op, z_rows)
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _ws(ws):
+    if isinstance(ws, tuple):
+        return ws
+    return ws.data_ptr(), ws.numel() * ws.element_size()
+
+
+def _step(name, mats, p, ws, stream):
+    ptr, nbytes = _ws(ws)
+    fn = getattr(lib(), name)
+    _check(fn(mats, _n(mats), ctypes.byref(p), ptr, nbytes, _stream(stream)), name)
+
+
+def muon_step(mats, p, ws, stream=None):
+    _step("muon_step", mats, p, ws, stream)
+
+
+def hyperball_step(mats, p, ws, stream=None):
+    _step("hyperball_step", mats, p, ws, stream)
+
+
+def radial_brake_step(mats, p, ws, stream=None):
+    _step("radial_brake_step", mats, p, ws, stream)
+
+
+def himuon_step(mats, p, ws, stream=None):
+    _step("himuon_step", mats, p, ws, stream)
+
+
+def newton_muon_step(mats, Z, n_tokens: int, p, ws, stream=None):
+    ptr, nbytes = _ws(ws)
+    nz = len(Z)
+    zp = (ctypes.c_void_p * max(nz, 1))(*[_ptr(z) for z in Z])
+    zr = (ctypes.c_int64 * max(nz, 1))(*[int(z.shape[0]) for z in Z])
+    _check(lib().newton_muon_step(mats, _n(mats), zp, zr, nz, int(n_tokens), ctypes.byref(p), ptr, nbytes,
+                                  _stream(stream)), "newton_muon_step")
+
+
+def fro_norms(mats, out, ws, stream=None):
+    ptr, nbytes = _ws(ws)
+    _check(lib().nshb_fro_norms(mats, _n(mats), _ptr(out), ptr, nbytes, _stream(stream)), "nshb_fro_norms")
+
+
+def device_status(ws, stream=None) -> int:
+    ptr, _ = _ws(ws)
+    v = ctypes.c_uint32(0)
+    _check(lib().nshb_device_status(ptr, _stream(stream), ctypes.byref(v)), "nshb_device_status")
+    return v.value

@@ -1,0 +1,612 @@
+// C ABI of the optimizer step: argument validation, workspace planning and the launch
+// sequence.  Host code only; every step of the path runs in the kernels of this library.
+//
+// Launch sequence of a step (all on the caller's stream, no host synchronisation):
+//   memset(status) -> momentum -> norm finalize -> K x {Gram, Poly, Update} GEMMs
+//   -> [reduce -> finalize -> exact norm -> finalize] -> apply
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "../../include/nshb.h"
+#include "nshb_internal.h"
+
+namespace nshb {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr long long kWaitLimit = 4000000000LL;  // ~2 s of SM clock per mbarrier phase
+constexpr long long kWaitLimitTest = 2000000LL; // ~1 ms (debug_flags bit 0)
+constexpr float kKeller[3] = {3.4445f, -4.7750f, 2.0315f};
+
+size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+struct MatPlan {
+  int64_t m = 0, n = 0, ld = 0;
+  bool tall = false;
+  int64_t r = 0, s = 0;          // wide-side dims of X
+  int64_t Rp = 0, Sp = 0;        // bf16: padded X dims (panel height, columns)
+  int flags = 0;
+  int64_t x0 = 0, x1 = 0, a = 0, b = 0;   // workspace offsets
+  int T = 0, tiles_r = 0, tiles_c = 0, ntiles = 0;
+  int seg_begin = 0, nseg = 0;
+  int pr = 0, pc = 0;            // momentum block domain (W coordinates)
+  int k1_blocks = 0, k1_begin = 0;
+  int w_blocks = 0, w_begin = 0;
+};
+
+struct Plan {
+  int op = 0;
+  bool f32ns = false;
+  bool tiled = false;
+  int bn = 256;
+  std::vector<MatPlan> mp;
+  size_t scal_off = 0, scale_off = 0, nu_off = 0, k1part_off = 0, wpart_off = 0, total = 0;
+  int nseg = 0, k1_total = 0, w_total = 0;
+};
+
+nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p, int op, Plan &pl) {
+  if (!p) return NSHB_ERR_NULL;
+  if (n_mats < 0) return NSHB_ERR_SHAPE;
+  if (n_mats > 0 && !mats) return NSHB_ERR_NULL;
+  if (op < NSHB_OP_MUON || op > NSHB_OP_NEWTON_MUON) return NSHB_ERR_PARAM;
+  if (!(p->beta >= 0.f && p->beta < 1.f)) return NSHB_ERR_PARAM;
+  if (p->ns_steps < 1 || p->ns_steps > 32) return NSHB_ERR_PARAM;
+  if (!(p->ns_eps > 0.f) || !std::isfinite(p->ns_eps)) return NSHB_ERR_PARAM;
+  if (!(p->hb_eps > 0.f) || !std::isfinite(p->hb_eps)) return NSHB_ERR_PARAM;
+  if (!std::isfinite(p->lr) || !std::isfinite(p->weight_decay) || !std::isfinite(p->eta) || p->eta < 0.f)
+    return NSHB_ERR_PARAM;
+  if (op == NSHB_OP_RADIAL_BRAKE) {
+    if (!(p->brake_out >= 0.f && p->brake_out <= 1.f && p->brake_in >= 0.f && p->brake_in <= 1.f))
+      return NSHB_ERR_PARAM;
+    if (p->weight_decay != 0.f) return NSHB_ERR_PARAM;
+  }
+  if (p->ns_precision != NSHB_BF16 && p->ns_precision != NSHB_F32) return NSHB_ERR_DTYPE;
+  if (p->coeffs)
+    for (int i = 0; i < 3 * p->ns_steps; ++i)
+      if (!std::isfinite(p->coeffs[i])) return NSHB_ERR_PARAM;
+  pl.op = op;
+  pl.f32ns = p->ns_precision == NSHB_F32;
+  pl.tiled = op == NSHB_OP_HIMUON;
+  if (pl.tiled) {
+    if (pl.f32ns) return NSHB_ERR_UNSUPPORTED;
+    if (p->tile != 128 && p->tile != 256 && p->tile != 512) return NSHB_ERR_PARAM;
+    pl.bn = p->tile == 128 ? 128 : 256;
+  }
+  if (op == NSHB_OP_NEWTON_MUON) {
+    if (!(p->ridge_rel >= 0.f) || !std::isfinite(p->ridge_rel)) return NSHB_ERR_PARAM;
+  }
+  pl.mp.resize(n_mats);
+  for (int i = 0; i < n_mats; ++i) {
+    const nshb_matrix &d = mats[i];
+    MatPlan &m = pl.mp[i];
+    if (d.rows <= 0 || d.cols <= 0 || d.ld < d.cols) return NSHB_ERR_SHAPE;
+    if (d.rows > (1LL << 20) || d.cols > (1LL << 20) || d.ld > (1LL << 30)) return NSHB_ERR_UNSUPPORTED;
+    if (!d.W || !d.G || !d.M) return NSHB_ERR_NULL;
+    if (d.w_dtype != NSHB_BF16 && d.w_dtype != NSHB_F32) return NSHB_ERR_DTYPE;
+    m.m = d.rows;
+    m.n = d.cols;
+    m.ld = d.ld;
+    const bool wf32 = d.w_dtype == NSHB_F32;
+    const size_t esz = wf32 ? 4 : 2;
+    const bool vec = ((uintptr_t)d.W % 16 == 0) && ((uintptr_t)d.G % 16 == 0) && ((uintptr_t)d.M % 16 == 0) &&
+                     ((d.ld * esz) % 16 == 0) && ((d.ld * 4) % 16 == 0);
+    if (d.O_out && ((uintptr_t)d.O_out % esz) != 0) return NSHB_ERR_SHAPE;
+    m.flags = (vec ? kVec : 0) | (wf32 ? kWF32 : 0) | (pl.f32ns ? kNsF32 : 0);
+    if (pl.tiled) {
+      m.flags |= kTiled;
+      m.T = p->tile;
+      m.tiles_r = (int)((m.m + m.T - 1) / m.T);
+      m.tiles_c = (int)((m.n + m.T - 1) / m.T);
+      m.ntiles = m.tiles_r * m.tiles_c;
+      m.pr = m.tiles_r * m.T;
+      m.pc = m.tiles_c * m.T;
+      m.nseg = m.ntiles;
+    } else {
+      m.tall = m.m > m.n;
+      if (m.tall) m.flags |= kTall;
+      m.r = m.tall ? m.n : m.m;
+      m.s = m.tall ? m.m : m.n;
+      if (pl.f32ns) {
+        m.pr = (int)round_up(m.m, kBlk);
+        m.pc = (int)round_up(m.n, kBlk);
+      } else {
+        m.Rp = round_up(m.r, 256);
+        m.Sp = round_up(m.s, 256);
+        m.pr = (int)(m.tall ? m.Sp : m.Rp);
+        m.pc = (int)(m.tall ? m.Rp : m.Sp);
+      }
+      m.nseg = 1;
+    }
+    m.k1_blocks = (m.pr / kBlk) * (m.pc / kBlk);
+    m.w_blocks = (int)(((m.m + kBlk - 1) / kBlk) * ((m.n + kBlk - 1) / kBlk));
+  }
+  // Workspace layout.
+  size_t off = kAlign;  // [0, 256): device status word
+  pl.scal_off = off;
+  off = align_up(off + sizeof(MatScalars) * (size_t)n_mats);
+  pl.nseg = 0;
+  pl.k1_total = 0;
+  pl.w_total = 0;
+  for (auto &m : pl.mp) {
+    m.seg_begin = pl.nseg;
+    pl.nseg += m.nseg;
+    m.k1_begin = pl.k1_total;
+    pl.k1_total += m.k1_blocks;
+    m.w_begin = pl.w_total;
+    pl.w_total += m.w_blocks;
+  }
+  pl.scale_off = off;
+  off = align_up(off + sizeof(float) * (size_t)pl.nseg);
+  pl.nu_off = off;
+  off = align_up(off + sizeof(double) * (size_t)pl.nseg);
+  pl.k1part_off = off;
+  off = align_up(off + sizeof(double) * (size_t)pl.k1_total);
+  pl.wpart_off = off;
+  off = align_up(off + 3 * sizeof(double) * (size_t)pl.w_total);
+  for (auto &m : pl.mp) {
+    size_t xb, ab;
+    if (pl.tiled) {
+      xb = (size_t)m.ntiles * m.T * m.T * 2;
+      ab = xb;
+    } else if (pl.f32ns) {
+      xb = (size_t)m.r * m.s * 4;
+      ab = (size_t)m.r * m.r * 4;
+    } else {
+      xb = (size_t)m.Rp * m.Sp * 2;
+      ab = (size_t)m.Rp * m.Rp * 2;
+    }
+    m.x0 = off; off = align_up(off + xb);
+    m.x1 = off; off = align_up(off + xb);
+    m.a = off;  off = align_up(off + ab);
+    m.b = off;  off = align_up(off + ab);
+  }
+  pl.total = off;
+  return NSHB_OK;
+}
+
+MatDesc make_desc(const nshb_matrix &d, const MatPlan &m, int idx, int64_t o_off, int blk_begin, bool k1) {
+  MatDesc r;
+  std::memset(&r, 0, sizeof(r));
+  r.W = d.W;
+  r.G = d.G;
+  r.M = d.M;
+  r.O_out = d.O_out;
+  r.x_off = m.x0;
+  r.o_off = o_off;
+  r.m = (int)m.m;
+  r.n = (int)m.n;
+  r.ld = (int)m.ld;
+  r.flags = m.flags;
+  if (m.flags & kTiled) r.ph = m.T;
+  else if (m.flags & kNsF32) r.ph = (int)m.s;
+  else r.ph = (int)m.Rp;
+  if (k1) {
+    r.pr = m.pr;
+    r.pc = m.pc;
+    if (m.flags & kTiled) r.flags |= kTileMajor;  // momentum blocks walk tile by tile
+  } else {
+    r.pr = (int)round_up(m.m, kBlk);
+    r.pc = (int)round_up(m.n, kBlk);
+  }
+  r.blk_begin = blk_begin;
+  r.seg_begin = m.seg_begin;
+  r.tiles_c = m.tiles_c;
+  r.mat = idx;
+  return r;
+}
+
+int device_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+#define NSHB_CHECK_CUDA(x)                 \
+  do {                                     \
+    if ((x) != cudaSuccess) {              \
+      (void)cudaGetLastError();            \
+      return NSHB_ERR_CUDA;                \
+    }                                      \
+  } while (0)
+
+// momentum + per-segment norms
+nshb_status run_momentum(const nshb_matrix *mats, const Plan &pl, const nshb_params *p, char *ws,
+                         cudaStream_t st) {
+  const int n = (int)pl.mp.size();
+  double *k1part = reinterpret_cast<double *>(ws + pl.k1part_off);
+  for (int c0 = 0; c0 < n; c0 += kMaxMats) {
+    const int c1 = std::min(n, c0 + kMaxMats);
+    MomentumParams mp;
+    std::memset(&mp, 0, sizeof(mp));
+    mp.ws = ws;
+    mp.partials = k1part + pl.mp[c0].k1_begin;
+    mp.status = reinterpret_cast<uint32_t *>(ws);
+    mp.beta = p->beta;
+    mp.nesterov = p->nesterov ? 1 : 0;
+    mp.nmat = c1 - c0;
+    int nb = 0;
+    for (int i = c0; i < c1; ++i) {
+      mp.mats[i - c0] = make_desc(mats[i], pl.mp[i], i, 0, nb, true);
+      nb += pl.mp[i].k1_blocks;
+    }
+    mp.total_blocks = nb;
+    NSHB_CHECK_CUDA(launch_momentum(mp, st));
+
+    NormFinParams nf;
+    std::memset(&nf, 0, sizeof(nf));
+    nf.partials = k1part + pl.mp[c0].k1_begin;
+    const int seg0 = pl.mp[c0].seg_begin;
+    nf.scales = reinterpret_cast<float *>(ws + pl.scale_off) + seg0;
+    nf.nus = reinterpret_cast<double *>(ws + pl.nu_off) + seg0;
+    nf.status = reinterpret_cast<uint32_t *>(ws);
+    nf.ns_eps = p->ns_eps;
+    nf.nmat = c1 - c0;
+    int segs = 0, blks = 0;
+    for (int i = c0; i < c1; ++i) {
+      const MatPlan &m = pl.mp[i];
+      nf.seg_begin[i - c0] = segs;
+      nf.blk_begin[i - c0] = blks;
+      nf.bps[i - c0] = m.k1_blocks / m.nseg;
+      segs += m.nseg;
+      blks += m.k1_blocks;
+    }
+    nf.seg_begin[c1 - c0] = segs;
+    NSHB_CHECK_CUDA(launch_norm_finalize(nf, segs, st));
+  }
+  return NSHB_OK;
+}
+
+void coeffs_for(const nshb_params *p, int it, float &a, float &b, float &c) {
+  if (p->coeffs) {
+    a = p->coeffs[3 * it];
+    b = p->coeffs[3 * it + 1];
+    c = p->coeffs[3 * it + 2];
+  } else {
+    a = kKeller[0];
+    b = kKeller[1];
+    c = kKeller[2];
+  }
+}
+
+// K iterations of the three NS phases.  Returns the offset of each matrix's O in `o_off`.
+nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t st, std::vector<int64_t> &o_off) {
+  const int n = (int)pl.mp.size();
+  o_off.resize(n);
+  const float *scales = reinterpret_cast<const float *>(ws + pl.scale_off);
+  uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+  const long long limit = (p->debug_flags & 1u) ? kWaitLimitTest : kWaitLimit;
+  for (int it = 0; it < p->ns_steps; ++it) {
+    float ca, cb, cc;
+    coeffs_for(p, it, ca, cb, cc);
+    for (int phase = 0; phase < 3; ++phase) {
+      const int mode = phase == 0 ? kGram : phase == 1 ? kPoly : kUpdate;
+      if (pl.f32ns) {
+        for (int c0 = 0; c0 < n; c0 += kMaxProb) {
+          const int c1 = std::min(n, c0 + kMaxProb);
+          F32Params fp;
+          std::memset(&fp, 0, sizeof(fp));
+          fp.ws = ws;
+          fp.scales = scales;
+          fp.mode = mode;
+          fp.ca = ca; fp.cb = cb; fp.cc = cc;
+          int tiles = 0;
+          for (int i = c0; i < c1; ++i) {
+            const MatPlan &m = pl.mp[i];
+            const int64_t xin = (it % 2 == 0) ? m.x0 : m.x1, xout = (it % 2 == 0) ? m.x1 : m.x0;
+            F32Prob &q = fp.prob[i - c0];
+            if (mode == kGram) {
+              q.a_off = xin; q.b_off = xin; q.c_off = m.a; q.d_off = m.a;
+              q.M = (int)m.r; q.N = (int)m.r; q.K = (int)m.s;
+              q.lda = (int)m.s; q.ldb = (int)m.s; q.ldc = (int)m.r; q.b_trans = 1;
+            } else if (mode == kPoly) {
+              q.a_off = m.a; q.b_off = m.a; q.c_off = m.a; q.d_off = m.b;
+              q.M = (int)m.r; q.N = (int)m.r; q.K = (int)m.r;
+              q.lda = (int)m.r; q.ldb = (int)m.r; q.ldc = (int)m.r; q.b_trans = 0;
+            } else {
+              q.a_off = m.b; q.b_off = xin; q.c_off = xin; q.d_off = xout;
+              q.M = (int)m.r; q.N = (int)m.s; q.K = (int)m.r;
+              q.lda = (int)m.r; q.ldb = (int)m.s; q.ldc = (int)m.s; q.b_trans = 0;
+            }
+            q.scale_idx = (it == 0 && mode != kPoly) ? m.seg_begin : -1;
+            q.tiles_n = (q.N + 63) / 64;
+            q.tile_begin = tiles;
+            tiles += ((q.M + 63) / 64) * q.tiles_n;
+          }
+          fp.nprob = c1 - c0;
+          fp.total_tiles = tiles;
+          NSHB_CHECK_CUDA(launch_gemm_f32(fp, st));
+        }
+      } else {
+        for (int c0 = 0; c0 < n; c0 += kMaxProb) {
+          const int c1 = std::min(n, c0 + kMaxProb);
+          GemmParams gp;
+          std::memset(&gp, 0, sizeof(gp));
+          gp.ws = ws;
+          gp.scales = scales;
+          gp.status = status;
+          gp.wait_limit = limit;
+          gp.mode = mode;
+          gp.ca = ca; gp.cb = cb; gp.cc = cc;
+          // Longest-k problems first, so the static tile walk ends evenly.
+          std::vector<std::pair<int64_t, int>> ord;
+          for (int i = c0; i < c1; ++i) {
+            const MatPlan &m = pl.mp[i];
+            const int64_t kext = pl.tiled ? m.T : (mode == kGram ? m.Sp : m.Rp);
+            ord.push_back({-kext, i});
+          }
+          std::stable_sort(ord.begin(), ord.end());
+          int tiles = 0, k = 0;
+          for (auto &e : ord) {
+            const int i = e.second;
+            const MatPlan &m = pl.mp[i];
+            const int64_t xin = (it % 2 == 0) ? m.x0 : m.x1, xout = (it % 2 == 0) ? m.x1 : m.x0;
+            GemmProb &q = gp.prob[k++];
+            int64_t R, S;
+            int batch;
+            int64_t xbs, abs_;
+            if (pl.tiled) {
+              R = m.T; S = m.T; batch = m.ntiles;
+              xbs = (int64_t)m.T * m.T * 2;
+              abs_ = xbs;
+            } else {
+              R = m.Rp; S = m.Sp; batch = 1;
+              xbs = 0; abs_ = 0;
+            }
+            q.batch = batch;
+            q.a_ph = q.b_ph = q.d_ph = (int)R;
+            q.mt = (int)(R / 128);
+            if (mode == kGram) {
+              q.a_off = xin; q.b_off = xin; q.c_off = m.a; q.d_off = m.a;
+              q.a_bs = xbs; q.b_bs = xbs; q.c_bs = abs_; q.d_bs = abs_;
+              q.nt = (int)(R / pl.bn); q.kt = (int)(S / 64);
+            } else if (mode == kPoly) {
+              q.a_off = m.a; q.b_off = m.a; q.c_off = m.a; q.d_off = m.b;
+              q.a_bs = abs_; q.b_bs = abs_; q.c_bs = abs_; q.d_bs = abs_;
+              q.nt = (int)(R / pl.bn); q.kt = (int)(R / 64);
+            } else {
+              q.a_off = m.b; q.b_off = xin; q.c_off = xin; q.d_off = xout;
+              q.a_bs = abs_; q.b_bs = xbs; q.c_bs = xbs; q.d_bs = xbs;
+              q.nt = (int)(S / pl.bn); q.kt = (int)(R / 64);
+            }
+            if (mode == kUpdate) {
+              q.tiles_per_batch = q.mt * q.nt;
+            } else {
+              int cnt = 0;
+              for (int mi = 0; mi < q.mt; ++mi) cnt += std::min(q.nt, (128 * mi + 127) / pl.bn + 1);
+              q.tiles_per_batch = cnt;
+            }
+            q.scale_idx = (it == 0 && mode != kPoly) ? m.seg_begin : -1;
+            q.tile_begin = tiles;
+            tiles += q.tiles_per_batch * q.batch;
+          }
+          gp.nprob = k;
+          gp.total_tiles = tiles;
+          NSHB_CHECK_CUDA(launch_gemm_tc(gp, pl.bn, device_sms(), st));
+        }
+      }
+    }
+  }
+  for (int i = 0; i < n; ++i) o_off[i] = (p->ns_steps % 2 == 0) ? pl.mp[i].x0 : pl.mp[i].x1;
+  return NSHB_OK;
+}
+
+nshb_status run_apply(const nshb_matrix *mats, const Plan &pl, const nshb_params *p, int apply_op, char *ws,
+                      cudaStream_t st, const std::vector<int64_t> &o_off, float *norms_out) {
+  const int n = (int)pl.mp.size();
+  MatScalars *scal = reinterpret_cast<MatScalars *>(ws + pl.scal_off);
+  double *wpart = reinterpret_cast<double *>(ws + pl.wpart_off);
+  uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+  for (int c0 = 0; c0 < n; c0 += kMaxMats) {
+    const int c1 = std::min(n, c0 + kMaxMats);
+    ApplyParams ap;
+    std::memset(&ap, 0, sizeof(ap));
+    ap.ws = ws;
+    ap.scal = scal;
+    ap.status = status;
+    ap.op = apply_op;
+    ap.nmat = c1 - c0;
+    ApplyFinParams fp;
+    std::memset(&fp, 0, sizeof(fp));
+    fp.scal = scal;
+    fp.status = status;
+    fp.rho = p->rho;
+    fp.norms_out = norms_out;
+    fp.op = apply_op;
+    fp.lr = p->lr;
+    fp.weight_decay = p->weight_decay;
+    fp.eta = p->eta;
+    fp.hb_eps = p->hb_eps;
+    fp.brake_out = p->brake_out;
+    fp.brake_in = p->brake_in;
+    fp.nmat = c1 - c0;
+    int nb = 0;
+    for (int i = c0; i < c1; ++i) {
+      const MatPlan &m = pl.mp[i];
+      ap.mats[i - c0] = make_desc(mats[i], m, i, o_off.empty() ? 0 : o_off[i], nb, false);
+      fp.blk_begin[i - c0] = nb;
+      fp.mat[i - c0] = i;
+      fp.m[i - c0] = (int)m.m;
+      fp.n[i - c0] = (int)m.n;
+      nb += m.w_blocks;
+    }
+    fp.blk_begin[c1 - c0] = nb;
+    ap.total_blocks = nb;
+    ap.partials = wpart;
+    fp.partials = wpart;
+    if (apply_op != kOpMuon) {
+      NSHB_CHECK_CUDA(launch_reduce(ap, st));
+    }
+    fp.stage = 0;
+    NSHB_CHECK_CUDA(launch_apply_finalize(fp, st));
+    if (apply_op == kOpNorms) continue;
+    if (apply_op == kOpHyperball || apply_op == kOpBrake) {
+      NSHB_CHECK_CUDA(launch_exact_norm(ap, st));
+      fp.stage = 1;
+      NSHB_CHECK_CUDA(launch_apply_finalize(fp, st));
+    }
+    NSHB_CHECK_CUDA(launch_apply(ap, st));
+  }
+  return NSHB_OK;
+}
+
+nshb_status check_ws(const Plan &pl, void *ws, size_t ws_bytes) {
+  if (!ws) return NSHB_ERR_NULL;
+  if ((uintptr_t)ws % kAlign != 0) return NSHB_ERR_WORKSPACE;
+  if (ws_bytes < pl.total) return NSHB_ERR_WORKSPACE;
+  return NSHB_OK;
+}
+
+nshb_status do_step(const nshb_matrix *mats, int n_mats, const nshb_params *p, int op, void *ws, size_t ws_bytes,
+                    cudaStream_t st) {
+  Plan pl;
+  nshb_status e = plan_step(mats, n_mats, p, op, pl);
+  if (e != NSHB_OK) return e;
+  if (n_mats == 0) return NSHB_OK;
+  e = check_ws(pl, ws, ws_bytes);
+  if (e != NSHB_OK) return e;
+  char *w = static_cast<char *>(ws);
+  NSHB_CHECK_CUDA(cudaMemsetAsync(w, 0, sizeof(uint32_t), st));
+  e = run_momentum(mats, pl, p, w, st);
+  if (e != NSHB_OK) return e;
+  std::vector<int64_t> o_off;
+  e = run_ns(pl, p, w, st, o_off);
+  if (e != NSHB_OK) return e;
+  const int aop = op == NSHB_OP_MUON ? kOpMuon : op == NSHB_OP_RADIAL_BRAKE ? kOpBrake : kOpHyperball;
+  return run_apply(mats, pl, p, aop, w, st, o_off, nullptr);
+}
+
+}  // namespace
+}  // namespace nshb
+
+using namespace nshb;
+
+extern "C" {
+
+nshb_status nshb_default_params(nshb_params *p) {
+  if (!p) return NSHB_ERR_NULL;
+  std::memset(p, 0, sizeof(*p));
+  p->beta = 0.95f;
+  p->nesterov = 1;
+  p->ns_steps = 5;
+  p->ns_precision = NSHB_BF16;
+  p->coeffs = nullptr;
+  p->ns_eps = 1e-7f;
+  p->lr = 0.02f;
+  p->weight_decay = 0.f;
+  p->eta = 0.02f;
+  p->rho = nullptr;
+  p->hb_eps = 1e-8f;
+  p->brake_out = 0.5f;
+  p->brake_in = 1.0f;
+  p->tile = 256;
+  p->ridge_rel = 1e-3f;
+  p->debug_flags = 0;
+  return NSHB_OK;
+}
+
+nshb_status nshb_workspace_size(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, int32_t op,
+                                const int64_t *z_rows, int32_t n_z, size_t *bytes) {
+  if (!bytes) return NSHB_ERR_NULL;
+  (void)z_rows;
+  (void)n_z;
+  Plan pl;
+  nshb_status e = plan_step(mats, n_mats, p, op, pl);
+  if (e != NSHB_OK) return e;
+  *bytes = pl.total;
+  return NSHB_OK;
+}
+
+nshb_status muon_step(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, void *ws, size_t ws_bytes,
+                      nshb_stream stream) {
+  return do_step(mats, n_mats, p, NSHB_OP_MUON, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+nshb_status hyperball_step(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, void *ws,
+                           size_t ws_bytes, nshb_stream stream) {
+  return do_step(mats, n_mats, p, NSHB_OP_HYPERBALL, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+nshb_status radial_brake_step(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, void *ws,
+                              size_t ws_bytes, nshb_stream stream) {
+  return do_step(mats, n_mats, p, NSHB_OP_RADIAL_BRAKE, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+nshb_status himuon_step(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, void *ws, size_t ws_bytes,
+                        nshb_stream stream) {
+  return do_step(mats, n_mats, p, NSHB_OP_HIMUON, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+nshb_status newton_muon_step(const nshb_matrix *mats, int32_t n_mats, const void *const *Z, const int64_t *z_rows,
+                             int32_t n_z, int64_t n_tokens, const nshb_params *p, void *ws, size_t ws_bytes,
+                             nshb_stream stream) {
+  (void)mats; (void)n_mats; (void)Z; (void)z_rows; (void)n_z; (void)n_tokens; (void)p; (void)ws;
+  (void)ws_bytes; (void)stream;
+  return NSHB_ERR_UNSUPPORTED;
+}
+
+nshb_status nshb_fro_norms(const nshb_matrix *mats, int32_t n_mats, float *out, void *ws, size_t ws_bytes,
+                           nshb_stream stream) {
+  if (!out && n_mats > 0) return NSHB_ERR_NULL;
+  nshb_params p;
+  nshb_default_params(&p);
+  Plan pl;
+  nshb_status e = plan_step(mats, n_mats, &p, NSHB_OP_MUON, pl);
+  if (e != NSHB_OK) return e;
+  if (n_mats == 0) return NSHB_OK;
+  e = check_ws(pl, ws, ws_bytes);
+  if (e != NSHB_OK) return e;
+  char *w = static_cast<char *>(ws);
+  cudaStream_t st = (cudaStream_t)stream;
+  NSHB_CHECK_CUDA(cudaMemsetAsync(w, 0, sizeof(uint32_t), st));
+  std::vector<int64_t> none;
+  return run_apply(mats, pl, &p, kOpNorms, w, st, none, out);
+}
+
+nshb_status nshb_device_status(const void *ws, nshb_stream stream, uint32_t *flags) {
+  if (!ws || !flags) return NSHB_ERR_NULL;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(st) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return NSHB_ERR_CUDA;
+  }
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return NSHB_ERR_CUDA;
+  }
+  *flags = v;
+  return NSHB_OK;
+}
+
+const char *nshb_status_string(int32_t s) {
+  switch (s) {
+    case NSHB_OK: return "NSHB_OK";
+    case NSHB_ERR_NULL: return "NSHB_ERR_NULL";
+    case NSHB_ERR_SHAPE: return "NSHB_ERR_SHAPE";
+    case NSHB_ERR_DTYPE: return "NSHB_ERR_DTYPE";
+    case NSHB_ERR_PARAM: return "NSHB_ERR_PARAM";
+    case NSHB_ERR_WORKSPACE: return "NSHB_ERR_WORKSPACE";
+    case NSHB_ERR_CUDA: return "NSHB_ERR_CUDA";
+    case NSHB_ERR_DEVICE_TIMEOUT: return "NSHB_ERR_DEVICE_TIMEOUT";
+    case NSHB_ERR_NONFINITE: return "NSHB_ERR_NONFINITE";
+    case NSHB_ERR_ZERO_NORM: return "NSHB_ERR_ZERO_NORM";
+    case NSHB_ERR_UNSUPPORTED: return "NSHB_ERR_UNSUPPORTED";
+    default: return "NSHB_ERR_UNKNOWN";
+  }
+}
+
+int32_t nshb_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,154 @@
+// Launch-parameter layouts shared by the host planner and the kernels.
+// Everything a kernel needs travels by value in its parameter block (up to a few
+// tens of KB, allowed on sm_70+ since CUDA 12.1), so a step needs no host->device
+// copies and the whole launch sequence can be captured in a CUDA graph.
+#pragma once
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace nshb {
+
+constexpr int kMaxMats = 192;   // matrices per launch of a streaming kernel (host splits larger sets)
+constexpr int kMaxProb = 192;   // GEMM problems per launch
+constexpr int kBlk = 64;        // streaming kernels work on 64 x 64 blocks
+
+// Matrix flags.
+constexpr int kTall = 1;        // rows > cols: the NS works on U^T (wide side)
+constexpr int kVec = 2;         // 16-byte vector access is legal for W/G/M rows
+constexpr int kWF32 = 4;        // W and G are fp32 (else bf16)
+constexpr int kTiled = 8;       // Hierarchical Muon: X is a grid of T x T tiles
+constexpr int kNsF32 = 16;      // NS in fp32, X row-major fp32 (else bf16 panel layout)
+constexpr int kTileMajor = 32;  // block list enumerates tile by tile (momentum of tiled matrices)
+
+// Per-matrix record of a streaming launch (momentum, reductions, apply).
+struct MatDesc {
+  void *W;
+  const void *G;
+  float *M;
+  void *O_out;
+  int64_t x_off;     // workspace byte offset of X0 (where U is written)
+  int64_t o_off;     // workspace byte offset of the final O
+  int32_t m, n, ld;  // W shape and leading dimension
+  int32_t flags;
+  int32_t ph;        // bf16: panel height of X (padded rows); fp32: row stride of X; tiled: T
+  int32_t pr, pc;    // block domain of this launch in W coordinates (padded extents)
+  int32_t blk_begin; // first 64x64 block of this matrix in the launch's block list
+  int32_t seg_begin; // first norm segment (matrix, or first tile when tiled)
+  int32_t tiles_c;   // tiled: tiles per tile-row of the padded grid
+  int32_t mat;       // index of the matrix in the whole call
+  int32_t pad_;
+};
+
+// Momentum + U + per-block ||U||^2 partials.
+struct MomentumParams {
+  char *ws;
+  double *partials;  // one per block of the launch
+  uint32_t *status;
+  float beta;
+  int32_t nesterov;
+  int32_t nmat, total_blocks;
+  MatDesc mats[kMaxMats];
+};
+
+// Per-segment ||U||^2 -> scale 1 / (sqrt(nu) + eps).
+struct NormFinParams {
+  const double *partials;
+  float *scales;
+  double *nus;
+  uint32_t *status;
+  float ns_eps;
+  int32_t nmat;
+  int32_t seg_begin[kMaxMats + 1];  // segment prefix (segments of one matrix are contiguous)
+  int32_t blk_begin[kMaxMats];      // partial index of each matrix's first block
+  int32_t bps[kMaxMats];            // blocks per segment
+};
+
+// Per-matrix scalars kept in the workspace between the reduce, finalize and apply kernels.
+struct MatScalars {
+  double omega, delta, pi;  // ||O||^2, <W, O>, ||W||^2
+  double t;                 // eta / ||O|| (Hyperball) or lr * shape scale (RadialBrake)
+  float alpha, beta;        // W_new = alpha W + beta O
+  int32_t need_exact;       // closed-form ||W - t O|| lost too many digits; recompute it
+  int32_t pad_;
+  double vv;                // exact ||W - t O||^2 when need_exact
+  double pad2_;
+};
+
+// Reductions over (W, O) blocks and the streaming update W <- alpha W + beta O.
+enum ApplyOp { kOpMuon = 0, kOpHyperball = 1, kOpBrake = 2, kOpNorms = 3 };
+struct ApplyParams {
+  char *ws;
+  double *partials;        // 3 doubles per block (reduce) or 1 (exact norm)
+  MatScalars *scal;        // indexed by MatDesc::mat
+  uint32_t *status;
+  int32_t op;
+  int32_t nmat, total_blocks;
+  MatDesc mats[kMaxMats];
+};
+struct ApplyFinParams {
+  const double *partials;
+  MatScalars *scal;
+  uint32_t *status;
+  const float *rho;        // device radii or NULL
+  float *norms_out;        // kOpNorms: ||W|| per matrix
+  int32_t op, stage;       // stage 0: after the reduce; stage 1: after the exact-norm pass
+  float lr, weight_decay, eta, hb_eps, brake_out, brake_in;
+  int32_t nmat;
+  int32_t blk_begin[kMaxMats + 1];
+  int32_t mat[kMaxMats];
+  int32_t m[kMaxMats], n[kMaxMats];
+};
+
+// One bf16 GEMM problem of a Newton-Schulz phase (possibly a batch of equal problems).
+// Operands live in the workspace in the panel layout (see panel_chunk_off).
+struct GemmProb {
+  int64_t a_off, b_off, c_off, d_off;  // byte offsets of batch 0
+  int64_t a_bs, b_bs, c_bs, d_bs;      // byte strides between batches
+  int32_t a_ph, b_ph, d_ph;            // panel heights (C shares D's)
+  int32_t mt, nt, kt;                  // 128-row tiles, BN-column tiles, 64-deep k blocks
+  int32_t batch, tiles_per_batch, tile_begin;
+  int32_t scale_idx;                   // scale of batch 0 in GemmParams::scales, or -1
+};
+enum GemmMode { kGram = 0, kPoly = 1, kUpdate = 2, kPlain = 3 };
+struct GemmParams {
+  char *ws;
+  const float *scales;
+  uint32_t *status;
+  long long wait_limit;   // clock cycles a role may wait on one mbarrier phase
+  int32_t mode;           // kGram: D = s^2 acc (lower triangle + mirror)
+                          // kPoly: D = cb C + cc acc (lower triangle + mirror)
+                          // kUpdate: D = s (ca C + acc), B operand MN-major
+  float ca, cb, cc;
+  int32_t nprob, total_tiles;
+  GemmProb prob[kMaxProb];
+};
+
+// fp32 SIMT GEMM problem (row-major fp32 operands in the workspace).
+struct F32Prob {
+  int64_t a_off, b_off, c_off, d_off;
+  int32_t M, N, K;
+  int32_t lda, ldb, ldc;   // ldd = ldc
+  int32_t b_trans;         // 1: B element (k, j) at b[j * ldb + k]; 0: at b[k * ldb + j]
+  int32_t tiles_n, tile_begin;
+  int32_t scale_idx;
+};
+struct F32Params {
+  char *ws;
+  const float *scales;
+  int32_t mode;            // as GemmMode (no symmetry exploited)
+  float ca, cb, cc;
+  int32_t nprob, total_tiles;
+  F32Prob prob[kMaxProb];
+};
+
+// Launchers (defined in the .cu files); each returns cudaGetLastError().
+cudaError_t launch_momentum(const MomentumParams &p, cudaStream_t s);
+cudaError_t launch_norm_finalize(const NormFinParams &p, int nseg_total, cudaStream_t s);
+cudaError_t launch_reduce(const ApplyParams &p, cudaStream_t s);
+cudaError_t launch_exact_norm(const ApplyParams &p, cudaStream_t s);
+cudaError_t launch_apply_finalize(const ApplyFinParams &p, cudaStream_t s);
+cudaError_t launch_apply(const ApplyParams &p, cudaStream_t s);
+cudaError_t launch_gemm_tc(const GemmParams &p, int bn, int num_sms, cudaStream_t s);
+cudaError_t launch_gemm_f32(const F32Params &p, cudaStream_t s);
+
+}  // namespace nshb

@@ -1,0 +1,145 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+function include/nshb.h declares, and rejects bad arguments synchronously, before any
+CUDA call is made."""
+import ctypes
+import pathlib
+import re
+
+import pytest
+
+import newton_schulz_hyperball_b200 as nshb
+from newton_schulz_hyperball_b200 import _abi
+
+HEADER = pathlib.Path(__file__).resolve().parents[1] / "include" / "nshb.h"
+
+
+def declared_functions():
+    text = HEADER.read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([a-z_][a-z0-9_]*)\s*\(",
+                                 text, flags=re.M)))
+
+
+def test_library_exports_every_declared_function():
+    lib = nshb.lib()
+    names = declared_functions()
+    assert {"muon_step", "hyperball_step", "radial_brake_step", "himuon_step", "newton_muon_step",
+            "nshb_workspace_size", "nshb_fro_norms", "nshb_device_status", "nshb_status_string"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_abi.SIGNATURES)
+
+
+def test_struct_layouts_match_header():
+    assert ctypes.sizeof(_abi.nshb_matrix) == 64
+    assert ctypes.sizeof(_abi.nshb_params) == 72
+    assert _abi.nshb_params.coeffs.offset == 16 and _abi.nshb_params.rho.offset == 40
+
+
+def test_defaults_and_strings():
+    p = nshb.params()
+    assert abs(p.beta - 0.95) < 1e-7 and p.nesterov == 1 and p.ns_steps == 5
+    assert abs(p.ns_eps - 1e-7) < 1e-12 and abs(p.hb_eps - 1e-8) < 1e-13
+    assert p.ns_precision == nshb.NSHB_BF16 and p.tile == 256
+    assert nshb.lib().nshb_status_string(nshb.NSHB_ERR_WORKSPACE) == b"NSHB_ERR_WORKSPACE"
+    assert nshb.lib().nshb_version() >= 100
+
+
+def fake_mats(shapes, dtype=nshb.NSHB_BF16, ld=None):
+    arr = (nshb.nshb_matrix * len(shapes))()
+    for i, (r, c) in enumerate(shapes):
+        arr[i].rows, arr[i].cols = r, c
+        arr[i].ld = c if ld is None else ld
+        arr[i].w_dtype = dtype
+        arr[i].z_index = -1
+        base = 0x10000000 * (i + 1)
+        arr[i].W, arr[i].G, arr[i].M = base, base + 0x4000000, base + 0x8000000
+    arr._n = len(shapes)
+    return arr
+
+
+def ws_size(mats, p, op):
+    return nshb.workspace_size(mats, p, op)
+
+
+def test_workspace_size_grows_with_matrices_and_orientation():
+    p = nshb.params()
+    a = ws_size(fake_mats([(768, 768)]), p, nshb.NSHB_OP_HYPERBALL)
+    b = ws_size(fake_mats([(768, 768), (3072, 768)]), p, nshb.NSHB_OP_HYPERBALL)
+    c = ws_size(fake_mats([(768, 768), (768, 3072)]), p, nshb.NSHB_OP_HYPERBALL)
+    assert 0 < a < b and b == c      # tall and wide matrices use the same wide-side buffers
+    # bf16 NS keeps X twice (ping-pong) and the two r x r Gram/polynomial matrices.
+    assert a >= 2 * 768 * 768 * 2 * 2
+    f = nshb.params(ns_precision=nshb.NSHB_F32)
+    assert ws_size(fake_mats([(768, 768)], nshb.NSHB_F32), f, nshb.NSHB_OP_HYPERBALL) >= 4 * 768 * 768 * 4
+
+
+@pytest.mark.parametrize("shape,code", [((0, 5), nshb.NSHB_ERR_SHAPE), ((5, -1), nshb.NSHB_ERR_SHAPE)])
+def test_bad_shapes(shape, code):
+    with pytest.raises(nshb.NshbError) as e:
+        ws_size(fake_mats([shape]), nshb.params(), nshb.NSHB_OP_MUON)
+    assert e.value.status == code
+
+
+def test_ld_smaller_than_cols():
+    with pytest.raises(nshb.NshbError) as e:
+        ws_size(fake_mats([(8, 16)], ld=8), nshb.params(), nshb.NSHB_OP_MUON)
+    assert e.value.status == nshb.NSHB_ERR_SHAPE
+
+
+def test_null_pointers():
+    m = fake_mats([(8, 8)])
+    m[0].G = None
+    with pytest.raises(nshb.NshbError) as e:
+        ws_size(m, nshb.params(), nshb.NSHB_OP_MUON)
+    assert e.value.status == nshb.NSHB_ERR_NULL
+    lib = nshb.lib()
+    assert lib.muon_step(fake_mats([(8, 8)]), 1, None, None, 0, None) == nshb.NSHB_ERR_NULL
+    assert lib.nshb_device_status(None, None, None) == nshb.NSHB_ERR_NULL
+
+
+def test_bad_dtype():
+    with pytest.raises(nshb.NshbError) as e:
+        ws_size(fake_mats([(8, 8)], dtype=7), nshb.params(), nshb.NSHB_OP_MUON)
+    assert e.value.status == nshb.NSHB_ERR_DTYPE
+    with pytest.raises(nshb.NshbError) as e:
+        ws_size(fake_mats([(8, 8)]), nshb.params(ns_precision=3), nshb.NSHB_OP_MUON)
+    assert e.value.status == nshb.NSHB_ERR_DTYPE
+
+
+@pytest.mark.parametrize("kw,op", [
+    (dict(beta=1.0), nshb.NSHB_OP_MUON),
+    (dict(beta=-0.1), nshb.NSHB_OP_MUON),
+    (dict(ns_steps=0), nshb.NSHB_OP_MUON),
+    (dict(ns_steps=33), nshb.NSHB_OP_MUON),
+    (dict(ns_eps=0.0), nshb.NSHB_OP_MUON),
+    (dict(hb_eps=0.0), nshb.NSHB_OP_HYPERBALL),
+    (dict(eta=-1.0), nshb.NSHB_OP_HYPERBALL),
+    (dict(brake_out=1.5), nshb.NSHB_OP_RADIAL_BRAKE),
+    (dict(brake_in=-0.1), nshb.NSHB_OP_RADIAL_BRAKE),
+    (dict(weight_decay=0.1), nshb.NSHB_OP_RADIAL_BRAKE),
+    (dict(tile=100), nshb.NSHB_OP_HIMUON),
+    (dict(ridge_rel=-1.0), nshb.NSHB_OP_NEWTON_MUON),
+    (dict(coeffs=[(float("nan"), 0, 0)] * 5), nshb.NSHB_OP_MUON),
+])
+def test_bad_params(kw, op):
+    with pytest.raises(nshb.NshbError) as e:
+        ws_size(fake_mats([(8, 8)]), nshb.params(**kw), op)
+    assert e.value.status == nshb.NSHB_ERR_PARAM
+
+
+def test_workspace_too_small_or_misaligned_is_rejected_before_launch():
+    lib = nshb.lib()
+    m = fake_mats([(64, 64)])
+    p = nshb.params()
+    need = ws_size(m, p, nshb.NSHB_OP_HYPERBALL)
+    for fn in (lib.muon_step, lib.hyperball_step, lib.radial_brake_step):
+        assert fn(m, 1, ctypes.byref(p), 0x20000000, need - 256, None) == nshb.NSHB_ERR_WORKSPACE
+        assert fn(m, 1, ctypes.byref(p), 0x20000010, need, None) == nshb.NSHB_ERR_WORKSPACE
+        assert fn(m, 1, ctypes.byref(p), None, need, None) == nshb.NSHB_ERR_NULL
+
+
+def test_zero_matrices_is_a_no_op():
+    lib = nshb.lib()
+    p = nshb.params()
+    assert lib.hyperball_step(None, 0, ctypes.byref(p), None, 0, None) == nshb.NSHB_OK

@@ -1,0 +1,224 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 CPU oracle on the same
+seeded inputs.
+
+Tolerances (written per test):
+  * fp32 NS path: relative Frobenius error of O and of the weight change <= 1e-4;
+  * bf16 tensor-core NS path: relative Frobenius error of O <= 2e-2;
+  * momentum buffer (fp32): relative error <= 1e-6;
+  * radius: | ||W|| - rho | / rho <= 1e-5 for fp32 weights; for bf16 weights the stored
+    value carries the bf16 rounding of every element, so the bound is 1e-5 plus six
+    standard deviations of that rounding's effect on the norm (2^-9/sqrt(3) per element,
+    relative), computed from the weights themselves.
+"""
+import math
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a GPU", allow_module_level=True)
+
+from newton_schulz_hyperball_b200 import workloads as wl  # noqa: E402
+from oracle import nshb_oracle as o  # noqa: E402
+import newton_schulz_hyperball_b200 as nshb  # noqa: E402
+from gpu_harness import GpuSet, rel_fro  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+
+def radius_tol(W, bf16):
+    if not bf16:
+        return 1e-5
+    w2 = np.sum(W * W)
+    return 1e-5 + 6 * (2.0 ** -9 / math.sqrt(3)) * math.sqrt(np.sum(W ** 4)) / w2
+
+
+def bf16_w_tol(W_ref, eta):
+    """Frobenius bound on W_gpu - W_ref for bf16 weights: half an ulp per element of
+    storage rounding plus the 2e-2 relative error of the unit update direction."""
+    a = np.abs(W_ref)
+    e = np.floor(np.log2(np.maximum(a, 1e-38)))
+    half_ulp = np.where(a > 0, 2.0 ** (e - 8), 0.0)
+    return float(np.linalg.norm(half_ulp)) + 2 * 2e-2 * eta + 1e-6 * float(np.linalg.norm(W_ref))
+
+
+# ------------------------------------------------------------------ fp32 path
+def test_fp32_single_matrix_hyperball_10_steps():
+    """256x256 fp32, W0 ~ N(0, 0.02^2), G ~ N(0, 1e-2^2) fresh each step, beta 0.95 Nesterov,
+    K = 5, Hyperball rho = ||W0||, eta = 0.02, 10 steps."""
+    cfg = wl.CFG_SINGLE_F32
+    W = wl.init_weight(cfg, 0, 256, 256, bf16=False).astype(np.float64)
+    rho = o.fro(W)
+    gs = GpuSet([W], bf16=False)
+    rho_dev = torch.tensor([rho], dtype=torch.float32, device="cuda")
+    p = nshb.params(ns_precision=nshb.NSHB_F32, eta=0.02, rho=rho_dev)
+    Wr, Mr = W.copy(), np.zeros_like(W)
+    for step in range(10):
+        G = wl.plain_gradient(cfg, 0, step, 256, 256, 1e-2, bf16=False)
+        gs.set_grads([G])
+        W_prev = Wr.copy()
+        flags = gs.step("hyperball", p)
+        assert flags == 0
+        Wr, Mr, Or, _ = o.hyperball_step(Wr, G, Mr, eta=0.02, rho=rho)
+        Wg, Mg, Og = gs.host()
+        assert rel_fro(Mg[0], Mr) <= 1e-6
+        assert rel_fro(Og[0], Or) <= 1e-4
+        assert rel_fro(Wg[0] - W_prev, Wr - W_prev) <= 1e-4
+        assert abs(o.fro(Wg[0]) - rho) / rho <= 1e-5
+        # continue the oracle from the GPU's weights? No: each side keeps its own state.
+
+
+@pytest.mark.parametrize("shape", [(96, 200), (200, 96), (5, 7), (7, 5), (1, 9), (9, 1), (130, 130)])
+def test_fp32_shapes_muon_and_hyperball(shape):
+    cfg = 11
+    m, n = shape
+    W = wl.init_weight(cfg, 1, m, n, bf16=False).astype(np.float64)
+    G = wl.gradient(cfg, 1, 0, m, n, bf16=False)
+    for kind in ("muon", "hyperball"):
+        gs = GpuSet([W], bf16=False)
+        gs.set_grads([G])
+        p = nshb.params(ns_precision=nshb.NSHB_F32, eta=0.01, lr=0.05, weight_decay=0.1)
+        flags = gs.step(kind, p)
+        assert flags == 0
+        Wg, Mg, Og = gs.host()
+        if kind == "muon":
+            Wr, Mr, Or = o.muon_step(W, G, np.zeros_like(W), lr=0.05, weight_decay=0.1)
+        else:
+            Wr, Mr, Or, _ = o.hyperball_step(W, G, np.zeros_like(W), eta=0.01, rho=None)
+            assert abs(o.fro(Wg[0]) - o.fro(W)) / o.fro(W) <= 1e-5
+        assert rel_fro(Mg[0], Mr) <= 1e-6
+        assert rel_fro(Og[0], Or) <= 1e-4
+        assert rel_fro(Wg[0] - W, Wr - W) <= 1e-4
+
+
+# ------------------------------------------------------------------ bf16 path
+PHASE_SHAPES = [(256, 256), (256, 512), (512, 256), (300, 700), (700, 300), (5, 7), (128, 1000)]
+
+
+@pytest.mark.parametrize("coeffs", [(1.0, 0.0, 0.0), (0.0, 1.0, 0.0), (0.0, 0.0, 1.0), (0.5, -0.25, 0.125)])
+@pytest.mark.parametrize("shape", PHASE_SHAPES)
+def test_bf16_single_iteration_phases(shape, coeffs):
+    """One NS iteration with chosen (a, b, c) isolates the Gram (b), polynomial (c) and
+    update (a) phases of the tensor-core chain."""
+    cfg = 12
+    m, n = shape
+    W = wl.init_weight(cfg, 2, m, n, bf16=True).astype(np.float64)
+    G = wl.gradient(cfg, 2, 0, m, n, bf16=True).astype(np.float64)
+    gs = GpuSet([W], bf16=True)
+    gs.set_grads([G])
+    p = nshb.params(ns_steps=1, coeffs=[coeffs], lr=0.0)
+    assert gs.step("muon", p) == 0
+    _, Mg, Og = gs.host()
+    _, U = o.momentum(np.zeros_like(G), G, 0.95, True)
+    Or = o.newton_schulz(U, 1, coeffs=[coeffs])
+    assert rel_fro(Mg[0], (1 - 0.95) * G) <= 1e-6
+    assert rel_fro(Og[0], Or) <= 1e-2
+
+
+@pytest.mark.parametrize("shape", PHASE_SHAPES + [(768, 768), (3072, 768), (768, 3072)])
+def test_bf16_ns_five_steps(shape):
+    cfg = 13
+    m, n = shape
+    W = wl.init_weight(cfg, 3, m, n, bf16=True).astype(np.float64)
+    G = wl.gradient(cfg, 3, 0, m, n, bf16=True).astype(np.float64)
+    gs = GpuSet([W], bf16=True)
+    gs.set_grads([G])
+    p = nshb.params(lr=0.0)
+    assert gs.step("muon", p) == 0
+    Wg, _, Og = gs.host()
+    _, U = o.momentum(np.zeros_like(G), G, 0.95, True)
+    assert rel_fro(Og[0], o.newton_schulz(U)) <= 2e-2
+    assert np.array_equal(Wg[0], W)     # lr = 0 leaves W bit-exact
+
+
+def gpt2_layer(cfg, layer, step):
+    shapes = wl.gpt2_small_shapes(1)
+    Ws, Gs = [], []
+    for k, (_, r, c) in enumerate(shapes):
+        idx = layer * 6 + k
+        Ws.append(wl.init_weight(cfg, idx, r, c, bf16=True).astype(np.float64))
+        Gs.append(wl.gradient(cfg, idx, step, r, c, bf16=True).astype(np.float64))
+    return Ws, Gs
+
+
+def test_bf16_hyperball_gpt2_layer_two_steps():
+    cfg = wl.CFG_GPT2_SMALL
+    Ws, _ = gpt2_layer(cfg, 0, 0)
+    rhos = [o.fro(w) for w in Ws]
+    gs = GpuSet(Ws, bf16=True)
+    rho_dev = torch.tensor(rhos, dtype=torch.float32, device="cuda")
+    p = nshb.params(eta=0.02, rho=rho_dev)
+    Wr = [w.copy() for w in Ws]
+    Mr = [np.zeros_like(w) for w in Ws]
+    for step in range(2):
+        _, Gs = gpt2_layer(cfg, 0, step)
+        gs.set_grads(Gs)
+        assert gs.step("hyperball", p) == 0
+        Wg, Mg, Og = gs.host()
+        for i in range(len(Ws)):
+            # Oracle step from the GPU's current state, so bf16 rounding does not compound.
+            W_in = Wr[i]
+            Wn, Mn, On, _ = o.hyperball_step(W_in, Gs[i], Mr[i], eta=0.02, rho=rhos[i])
+            assert rel_fro(Mg[i], Mn) <= 1e-6
+            assert rel_fro(Og[i], On) <= 2e-2, i
+            assert np.linalg.norm(Wg[i] - Wn) <= bf16_w_tol(Wn, 0.02), i
+            assert abs(o.fro(Wg[i]) - rhos[i]) / rhos[i] <= radius_tol(Wg[i], True), i
+            Wr[i], Mr[i] = Wg[i], Mg[i]
+
+
+def test_bf16_muon_and_brake_steps():
+    cfg = 14
+    shapes = [(256, 512), (512, 256), (300, 300)]
+    Ws = [wl.init_weight(cfg, i, r, c, bf16=True).astype(np.float64) for i, (r, c) in enumerate(shapes)]
+    Gs = [wl.gradient(cfg, i, 0, r, c, bf16=True).astype(np.float64) for i, (r, c) in enumerate(shapes)]
+    for kind in ("muon", "brake"):
+        gs = GpuSet(Ws, bf16=True)
+        gs.set_grads(Gs)
+        p = nshb.params(lr=0.02, weight_decay=0.0, brake_out=0.5, brake_in=1.0)
+        assert gs.step(kind, p) == 0
+        Wg, _, Og = gs.host()
+        for i, W in enumerate(Ws):
+            if kind == "muon":
+                Wr, _, Or = o.muon_step(W, Gs[i], np.zeros_like(W), lr=0.02)
+            else:
+                Wr, _, Or = o.radial_brake_step(W, Gs[i], np.zeros_like(W), lr=0.02, outward=0.5, inward=1.0)
+            assert rel_fro(Og[i], Or) <= 2e-2
+            step_len = 0.02 * o.shape_scale(*W.shape) * o.fro(Or)
+            assert np.linalg.norm(Wg[i] - Wr) <= bf16_w_tol(Wr, step_len)
+
+
+# ---------------------------------------------------- page pins on the GPU
+def test_bf16_768_five_directions_page_pin():
+    """Muon explainer, code section: bf16 NS of a 768x768 matrix with singular values
+    0.9, 0.3, 0.1, 0.01, 0.001 and the rest about 0.011 lands within 0.005 of the scalar
+    polynomial."""
+    import json, pathlib
+    g = json.loads((pathlib.Path(__file__).parent / "golden" / "page_values.json").read_text())["bf16_768_example"]
+    n = g["n"]
+    sig = np.array(g["sigma_top"] + [g["bulk_sigma"]] * (n - 5))
+    U = wl.spectrum_matrix(5, n, n, sig).astype(np.float64)
+    U = wl.round_to_bf16(U.astype(np.float32)).astype(np.float64)
+    # Feed U as the Nesterov update: with M = 0 and beta = 0 (no momentum), U = G.
+    gs = GpuSet([np.zeros((n, n))], bf16=True)
+    gs.set_grads([U])
+    p = nshb.params(beta=0.0, lr=0.0)
+    assert gs.step("muon", p) == 0
+    _, _, Og = gs.host()
+    s_in = np.linalg.svd(U, compute_uv=False)
+    expect = o.scalar_ns(s_in / (np.sqrt(np.sum(s_in ** 2)) + o.NS_EPS), 5)
+    s_out = np.linalg.svd(Og[0], compute_uv=False)
+    assert np.max(np.abs(np.sort(s_out) - np.sort(expect))) <= g["abs_tol"]
+
+
+def test_bf16_random_3072x768_band_page_pin():
+    import json, pathlib
+    g = json.loads((pathlib.Path(__file__).parent / "golden" / "page_values.json").read_text())["random_3072x768_band"]
+    rng = np.random.default_rng(7)
+    U = wl.round_to_bf16(rng.standard_normal((g["rows"], g["cols"])).astype(np.float32)).astype(np.float64)
+    gs = GpuSet([np.zeros_like(U)], bf16=True)
+    gs.set_grads([U])
+    assert gs.step("muon", nshb.params(beta=0.0, lr=0.0)) == 0
+    _, _, Og = gs.host()
+    s = np.linalg.svd(Og[0], compute_uv=False)
+    assert s.min() >= g["lo"] - 0.01 and s.max() <= g["hi"] + 0.01
