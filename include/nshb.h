@@ -52,7 +52,7 @@ typedef enum { NSHB_BF16 = 0, NSHB_F32 = 1 } nshb_dtype;
 typedef enum {
   NSHB_OK = 0,
   NSHB_ERR_NULL = 1,           /* a required pointer is NULL                                 */
-  NSHB_ERR_SHAPE = 2,          /* rows/cols <= 0, ld < cols, misaligned pointer/ld for bf16  */
+  NSHB_ERR_SHAPE = 2,          /* rows/cols <= 0, ld < cols, misaligned O_out                */
   NSHB_ERR_DTYPE = 3,          /* unknown dtype or unsupported dtype combination              */
   NSHB_ERR_PARAM = 4,          /* a scalar parameter out of range                             */
   NSHB_ERR_WORKSPACE = 5,      /* workspace smaller than nshb_workspace_size or misaligned    */
@@ -80,8 +80,9 @@ typedef enum {
 
 /* One weight matrix (rows x cols).  W is updated in place, G is read, M is the fp32
  * momentum buffer (zero before the first step; the only state a step keeps).
- * W and G share w_dtype.  For NSHB_BF16, W, G and M must be 16-byte aligned and ld a
- * multiple of 8; for NSHB_F32 W/G/M need 16-byte alignment and ld a multiple of 4.
+ * W and G share w_dtype.  Rows are read and written with 16-byte vector accesses when
+ * W, G and M are 16-byte aligned and ld * sizeof(element) and ld * 4 are multiples of 16;
+ * other layouts take a slower element-wise path.  O_out needs element alignment.
  * O_out (optional, may be NULL) receives the orthogonalised update O = NS_K(U)
  * (before any step-length or shape scaling), dtype w_dtype, leading dimension cols.
  * z_index picks the layer input Z of newton_muon_step (ignored elsewhere). */
@@ -97,7 +98,8 @@ typedef struct {
 
 /* Step parameters.  Defaults (nshb_default_params): beta 0.95, Nesterov, K = 5 with
  * (a, b, c) = (3.4445, -4.7750, 2.0315), ns_eps 1e-7, bf16 tensor-core NS, lr 0.02,
- * wd 0, eta 0.02, rho NULL, hb_eps 1e-8, brake 0.5 / 1.0, tile 256, ridge_rel 1e-3. */
+ * wd 0, eta 0.02, rho NULL, hb_eps 1e-8, brake 0.5 / 1.0, tile 256, ridge_rel 1e-3,
+ * ns_compensated 2. */
 typedef struct {
   float beta;            /* momentum coefficient, [0, 1)                                    */
   int32_t nesterov;      /* 1: U = (1-beta) G + beta M; 0: U = M                             */
@@ -116,6 +118,9 @@ typedef struct {
   float brake_in;        /* RadialBrake inward factor in [0, 1]                               */
   int32_t tile;          /* HiMuon tile size T: 128, 256 or 512                               */
   float ridge_rel;       /* Newton-Muon: lambda = ridge_rel * tr(Z Z^T) / d_in, >= 0          */
+  int32_t ns_compensated;/* bf16 NS: leading iterations whose a*X term reads X as a bf16 hi/lo */
+                         /* pair (about fp32 accuracy); 0 = plain bf16 chain; default 2;      */
+                         /* values above ns_steps act as ns_steps; range [0, 32]             */
   uint32_t debug_flags;  /* 0 in normal use; bit 0 shortens the device wait limit (tests)     */
 } nshb_params;
 

@@ -67,6 +67,7 @@ class nshb_params(ctypes.Structure):
         ("brake_in", ctypes.c_float),
         ("tile", ctypes.c_int32),
         ("ridge_rel", ctypes.c_float),
+        ("ns_compensated", ctypes.c_int32),
         ("debug_flags", ctypes.c_uint32),
     ]
 

@@ -32,6 +32,7 @@ struct MatPlan {
   int64_t Rp = 0, Sp = 0;        // bf16: padded X dims (panel height, columns)
   int flags = 0;
   int64_t x0 = 0, x1 = 0, a = 0, b = 0;   // workspace offsets
+  int64_t xl0 = -1, xl1 = -1;             // bf16 low parts of X0 / X1 (compensated iterations)
   int T = 0, tiles_r = 0, tiles_c = 0, ntiles = 0;
   int seg_begin = 0, nseg = 0;
   int pr = 0, pc = 0;            // momentum block domain (W coordinates)
@@ -44,6 +45,7 @@ struct Plan {
   bool f32ns = false;
   bool tiled = false;
   int bn = 256;
+  int comp = 0;                  // compensated (hi/lo) iterations of the bf16 chain
   std::vector<MatPlan> mp;
   size_t scal_off = 0, scale_off = 0, nu_off = 0, k1part_off = 0, wpart_off = 0, total = 0;
   int nseg = 0, k1_total = 0, w_total = 0;
@@ -66,12 +68,14 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
     if (p->weight_decay != 0.f) return NSHB_ERR_PARAM;
   }
   if (p->ns_precision != NSHB_BF16 && p->ns_precision != NSHB_F32) return NSHB_ERR_DTYPE;
+  if (p->ns_compensated < 0 || p->ns_compensated > 32) return NSHB_ERR_PARAM;
   if (p->coeffs)
     for (int i = 0; i < 3 * p->ns_steps; ++i)
       if (!std::isfinite(p->coeffs[i])) return NSHB_ERR_PARAM;
   pl.op = op;
   pl.f32ns = p->ns_precision == NSHB_F32;
   pl.tiled = op == NSHB_OP_HIMUON;
+  pl.comp = pl.f32ns ? 0 : std::min(p->ns_compensated, p->ns_steps);
   if (pl.tiled) {
     if (pl.f32ns) return NSHB_ERR_UNSUPPORTED;
     if (p->tile != 128 && p->tile != 256 && p->tile != 512) return NSHB_ERR_PARAM;
@@ -164,6 +168,10 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
     m.x1 = off; off = align_up(off + xb);
     m.a = off;  off = align_up(off + ab);
     m.b = off;  off = align_up(off + ab);
+    if (pl.comp > 0) {
+      m.xl0 = off; off = align_up(off + xb);
+      if (pl.comp > 1) { m.xl1 = off; off = align_up(off + xb); }
+    }
   }
   pl.total = off;
   return NSHB_OK;
@@ -177,6 +185,7 @@ MatDesc make_desc(const nshb_matrix &d, const MatPlan &m, int idx, int64_t o_off
   r.M = d.M;
   r.O_out = d.O_out;
   r.x_off = m.x0;
+  r.xlo_off = m.xl0;
   r.o_off = o_off;
   r.m = (int)m.m;
   r.n = (int)m.n;
@@ -367,6 +376,12 @@ nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t 
             q.batch = batch;
             q.a_ph = q.b_ph = q.d_ph = (int)R;
             q.mt = (int)(R / 128);
+            q.c_lo = -1;
+            q.d_lo = -1;
+            if (mode == kUpdate && it < pl.comp) {
+              q.c_lo = (it % 2 == 0) ? m.xl0 : m.xl1;
+              if (it + 1 < pl.comp) q.d_lo = (it % 2 == 0) ? m.xl1 : m.xl0;
+            }
             if (mode == kGram) {
               q.a_off = xin; q.b_off = xin; q.c_off = m.a; q.d_off = m.a;
               q.a_bs = xbs; q.b_bs = xbs; q.c_bs = abs_; q.d_bs = abs_;
@@ -512,6 +527,7 @@ nshb_status nshb_default_params(nshb_params *p) {
   p->brake_in = 1.0f;
   p->tile = 256;
   p->ridge_rel = 1e-3f;
+  p->ns_compensated = 2;
   p->debug_flags = 0;
   return NSHB_OK;
 }

@@ -226,6 +226,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       const float s2 = s * s;
       const char *cbase = p.ws + q.c_off + (int64_t)t.batch * q.c_bs;
       char *dbase = p.ws + q.d_off + (int64_t)t.batch * q.d_bs;
+      const char *clo = q.c_lo >= 0 ? p.ws + q.c_lo + (int64_t)t.batch * q.c_bs : nullptr;
+      char *dlo = q.d_lo >= 0 ? p.ws + q.d_lo + (int64_t)t.batch * q.d_bs : nullptr;
       const int64_t i = t.m0 + row;
       const bool sym = (p.mode == kGram || p.mode == kPoly);
       const int ra = (int)(i >> 6);
@@ -247,13 +249,17 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
           const float ks = (p.mode == kPoly) ? 1.0f : s;
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
-            const uint4 c4 = *reinterpret_cast<const uint4 *>(cbase + panel_chunk_off(i, col0 + 8 * g, q.d_ph));
-            const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              v[8 * g + 2 * h] = ks * fmaf(kc, bf16lo(cw[h]), ka * __uint_as_float(r[8 * g + 2 * h]));
-              v[8 * g + 2 * h + 1] = ks * fmaf(kc, bf16hi(cw[h]), ka * __uint_as_float(r[8 * g + 2 * h + 1]));
+            const size_t off = panel_chunk_off(i, col0 + 8 * g, q.d_ph);
+            const uint4 c4 = *reinterpret_cast<const uint4 *>(cbase + off);
+            float cv[8] = {bf16lo(c4.x), bf16hi(c4.x), bf16lo(c4.y), bf16hi(c4.y),
+                           bf16lo(c4.z), bf16hi(c4.z), bf16lo(c4.w), bf16hi(c4.w)};
+            if (clo) {   // C carried as a hi + lo pair
+              const uint4 l4 = *reinterpret_cast<const uint4 *>(clo + off);
+              cv[0] += bf16lo(l4.x); cv[1] += bf16hi(l4.x); cv[2] += bf16lo(l4.y); cv[3] += bf16hi(l4.y);
+              cv[4] += bf16lo(l4.z); cv[5] += bf16hi(l4.z); cv[6] += bf16lo(l4.w); cv[7] += bf16hi(l4.w);
             }
+#pragma unroll
+            for (int h = 0; h < 8; ++h) v[8 * g + h] = ks * fmaf(kc, cv[h], ka * __uint_as_float(r[8 * g + h]));
           }
         }
 #pragma unroll
@@ -263,7 +269,16 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
           o.y = pack_bf16(v[8 * g + 2], v[8 * g + 3]);
           o.z = pack_bf16(v[8 * g + 4], v[8 * g + 5]);
           o.w = pack_bf16(v[8 * g + 6], v[8 * g + 7]);
-          *reinterpret_cast<uint4 *>(dbase + panel_chunk_off(i, col0 + 8 * g, q.d_ph)) = o;
+          const size_t off = panel_chunk_off(i, col0 + 8 * g, q.d_ph);
+          *reinterpret_cast<uint4 *>(dbase + off) = o;
+          if (dlo) {   // keep the rounding residual as a second bf16
+            uint4 l;
+            l.x = pack_bf16(v[8 * g + 0] - bf16lo(o.x), v[8 * g + 1] - bf16hi(o.x));
+            l.y = pack_bf16(v[8 * g + 2] - bf16lo(o.y), v[8 * g + 3] - bf16hi(o.y));
+            l.z = pack_bf16(v[8 * g + 4] - bf16lo(o.z), v[8 * g + 5] - bf16hi(o.z));
+            l.w = pack_bf16(v[8 * g + 6] - bf16lo(o.w), v[8 * g + 7] - bf16hi(o.w));
+            *reinterpret_cast<uint4 *>(dlo + off) = l;
+          }
         }
         if (sym && ca < ra) {
           // Mirror: element (i, col0 + e) also lands at (col0 + e, i).

@@ -27,6 +27,7 @@ struct MatDesc {
   float *M;
   void *O_out;
   int64_t x_off;     // workspace byte offset of X0 (where U is written)
+  int64_t xlo_off;   // workspace byte offset of U's bf16 low part, or -1
   int64_t o_off;     // workspace byte offset of the final O
   int32_t m, n, ld;  // W shape and leading dimension
   int32_t flags;
@@ -103,6 +104,7 @@ struct ApplyFinParams {
 // Operands live in the workspace in the panel layout (see panel_chunk_off).
 struct GemmProb {
   int64_t a_off, b_off, c_off, d_off;  // byte offsets of batch 0
+  int64_t c_lo, d_lo;                  // kUpdate: bf16 low parts of C (read) / D (written), or -1
   int64_t a_bs, b_bs, c_bs, d_bs;      // byte strides between batches
   int32_t a_ph, b_ph, d_ph;            // panel heights (C shares D's)
   int32_t mt, nt, kt;                  // 128-row tiles, BN-column tiles, 64-deep k blocks
@@ -117,7 +119,8 @@ struct GemmParams {
   long long wait_limit;   // clock cycles a role may wait on one mbarrier phase
   int32_t mode;           // kGram: D = s^2 acc (lower triangle + mirror)
                           // kPoly: D = cb C + cc acc (lower triangle + mirror)
-                          // kUpdate: D = s (ca C + acc), B operand MN-major
+                          // kUpdate: D = s (ca C + acc), B operand MN-major; C may be a
+                          //          hi + lo pair and D may be written as one
   float ca, cb, cc;
   int32_t nprob, total_tiles;
   GemmProb prob[kMaxProb];

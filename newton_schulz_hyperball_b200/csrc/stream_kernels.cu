@@ -201,6 +201,7 @@ __device__ __forceinline__ void load_x16(const char *xbase, const MatDesc &d, in
 // ------------------------------------------------------------------------- momentum
 __global__ void __launch_bounds__(kThreads) momentum_kernel(const __grid_constant__ MomentumParams p) {
   __shared__ float sT[kBlk][kBlk + 1];
+  __shared__ float sL[kBlk][kBlk + 1];
   __shared__ double red[kThreads / 32];
   const int blk = blockIdx.x;
   const MatDesc &d = p.mats[find_mat(p, blk)];
@@ -210,8 +211,9 @@ __global__ void __launch_bounds__(kThreads) momentum_kernel(const __grid_constan
   const int i = r0 + rr, j = c0 + cg;
   const bool f32 = d.flags & kWF32, vec = d.flags & kVec;
   const bool round_bf16 = !(d.flags & kNsF32);
+  const bool lo_part = round_bf16 && d.xlo_off >= 0;
 
-  float g[16], mm[16], u[16];
+  float g[16], mm[16], u[16], ul[16];
   load16(d.G, d.ld, i, j, d.m, d.n, f32, vec, g);
   loadM(d.M, d.ld, i, j, d.m, d.n, vec, mm);
   const float beta = p.beta, omb = 1.0f - p.beta;
@@ -220,25 +222,38 @@ __global__ void __launch_bounds__(kThreads) momentum_kernel(const __grid_constan
   for (int e = 0; e < 16; ++e) {
     const float mnew = fmaf(beta, mm[e], omb * g[e]);
     mm[e] = mnew;
-    float uu = p.nesterov ? fmaf(omb, g[e], beta * mnew) : mnew;
-    if (round_bf16) uu = bf16_round(uu);
-    u[e] = (i < d.m && j + e < d.n) ? uu : 0.f;
-    acc = fmaf(u[e], u[e], acc);
+    float uf = p.nesterov ? fmaf(omb, g[e], beta * mnew) : mnew;
+    if (!(i < d.m && j + e < d.n)) uf = 0.f;
+    const float uh = round_bf16 ? bf16_round(uf) : uf;
+    u[e] = uh;
+    ul[e] = uf - uh;                       // exact in fp32; stored as bf16 when kept
+    const float un = lo_part ? uf : uh;    // the norm of what the first iteration reads
+    acc = fmaf(un, un, acc);
   }
   store16(d.M, d.ld, i, j, d.m, d.n, true, vec, mm);
 
   char *xbase = p.ws + d.x_off;
+  char *lbase = lo_part ? p.ws + d.xlo_off : nullptr;
   if (d.flags & kTall && !(d.flags & kTiled)) {
     // X = U^T: stage the block and write it transposed.
 #pragma unroll
-    for (int e = 0; e < 16; ++e) sT[rr][cg + e] = u[e];
+    for (int e = 0; e < 16; ++e) {
+      sT[rr][cg + e] = u[e];
+      sL[rr][cg + e] = ul[e];
+    }
     __syncthreads();
     float v[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) v[e] = sT[cg + e][rr];
     store_x16(xbase, d, c0 + rr, r0 + cg, v);
+    if (lo_part) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v[e] = sL[cg + e][rr];
+      store_x16(lbase, d, c0 + rr, r0 + cg, v);
+    }
   } else {
     store_x16(xbase, d, i, j, u);
+    if (lo_part) store_x16(lbase, d, i, j, ul);
   }
 
   double s[1] = {(double)acc};

@@ -32,7 +32,7 @@ def test_library_exports_every_declared_function():
 
 def test_struct_layouts_match_header():
     assert ctypes.sizeof(_abi.nshb_matrix) == 64
-    assert ctypes.sizeof(_abi.nshb_params) == 72
+    assert ctypes.sizeof(_abi.nshb_params) == 80
     assert _abi.nshb_params.coeffs.offset == 16 and _abi.nshb_params.rho.offset == 40
 
 
@@ -40,7 +40,7 @@ def test_defaults_and_strings():
     p = nshb.params()
     assert abs(p.beta - 0.95) < 1e-7 and p.nesterov == 1 and p.ns_steps == 5
     assert abs(p.ns_eps - 1e-7) < 1e-12 and abs(p.hb_eps - 1e-8) < 1e-13
-    assert p.ns_precision == nshb.NSHB_BF16 and p.tile == 256
+    assert p.ns_precision == nshb.NSHB_BF16 and p.tile == 256 and p.ns_compensated == 2
     assert nshb.lib().nshb_status_string(nshb.NSHB_ERR_WORKSPACE) == b"NSHB_ERR_WORKSPACE"
     assert nshb.lib().nshb_version() >= 100
 
@@ -121,6 +121,8 @@ def test_bad_dtype():
     (dict(tile=100), nshb.NSHB_OP_HIMUON),
     (dict(ridge_rel=-1.0), nshb.NSHB_OP_NEWTON_MUON),
     (dict(coeffs=[(float("nan"), 0, 0)] * 5), nshb.NSHB_OP_MUON),
+    (dict(ns_compensated=-1), nshb.NSHB_OP_MUON),
+    (dict(ns_compensated=33), nshb.NSHB_OP_MUON),
 ])
 def test_bad_params(kw, op):
     with pytest.raises(nshb.NshbError) as e:

@@ -132,6 +132,25 @@ def test_bf16_ns_five_steps(shape):
     assert np.array_equal(Wg[0], W)     # lr = 0 leaves W bit-exact
 
 
+def test_bf16_compensated_iterations_beat_plain_chain():
+    """The plain bf16 chain (every X rounded to bf16, as newton_schulz5 does) loses the
+    small singular directions of a spiked gradient to the rounding of U; carrying X as a
+    hi/lo pair through the first two a*X terms recovers them."""
+    cfg = 13
+    W = wl.init_weight(cfg, 3, 256, 256, bf16=True).astype(np.float64)
+    G = wl.gradient(cfg, 3, 0, 256, 256, bf16=True).astype(np.float64)
+    _, U = o.momentum(np.zeros_like(G), G, 0.95, True)
+    ref = o.newton_schulz(U)
+    errs = {}
+    for comp in (0, 1, 2, 5):
+        gs = GpuSet([W], bf16=True)
+        gs.set_grads([G])
+        assert gs.step("muon", nshb.params(lr=0.0, ns_compensated=comp)) == 0
+        errs[comp] = rel_fro(gs.host()[2][0], ref)
+    assert errs[2] <= 1e-2 and errs[5] <= 1e-2
+    assert errs[2] < errs[1] < errs[0]
+
+
 def gpt2_layer(cfg, layer, step):
     shapes = wl.gpt2_small_shapes(1)
     Ws, Gs = [], []
