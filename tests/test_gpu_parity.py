@@ -66,7 +66,6 @@ def test_fp32_single_matrix_hyperball_10_steps():
         assert rel_fro(Og[0], Or) <= 1e-4
         assert rel_fro(Wg[0] - W_prev, Wr - W_prev) <= 1e-4
         assert abs(o.fro(Wg[0]) - rho) / rho <= 1e-5
-        # continue the oracle from the GPU's weights? No: each side keeps its own state.
 
 
 @pytest.mark.parametrize("shape", [(96, 200), (200, 96), (5, 7), (7, 5), (1, 9), (9, 1), (130, 130)])
@@ -176,14 +175,13 @@ def test_bf16_hyperball_gpt2_layer_two_steps():
         assert gs.step("hyperball", p) == 0
         Wg, Mg, Og = gs.host()
         for i in range(len(Ws)):
-            # Oracle step from the GPU's current state, so bf16 rounding does not compound.
-            W_in = Wr[i]
-            Wn, Mn, On, _ = o.hyperball_step(W_in, Gs[i], Mr[i], eta=0.02, rho=rhos[i])
-            assert rel_fro(Mg[i], Mn) <= 1e-6
+            # Each side keeps its own state: the oracle in fp64, the GPU in bf16 / fp32.
+            Wr[i], Mr[i], On, _ = o.hyperball_step(Wr[i], Gs[i], Mr[i], eta=0.02, rho=rhos[i])
+            assert rel_fro(Mg[i], Mr[i]) <= 1e-6
             assert rel_fro(Og[i], On) <= 2e-2, i
-            assert np.linalg.norm(Wg[i] - Wn) <= bf16_w_tol(Wn, 0.02), i
+            # bf16 storage rounding accumulates once per step.
+            assert np.linalg.norm(Wg[i] - Wr[i]) <= (step + 1) * bf16_w_tol(Wr[i], 0.02), i
             assert abs(o.fro(Wg[i]) - rhos[i]) / rhos[i] <= radius_tol(Wg[i], True), i
-            Wr[i], Mr[i] = Wg[i], Mg[i]
 
 
 def test_bf16_muon_and_brake_steps():
