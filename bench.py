@@ -1,0 +1,387 @@
+"""Benchmark of the Muon-Hyperball optimizer step on B200.
+
+Workload (one step = the whole hot path over one batch of synthetic input): the GPT-2-small
+matrix set -- 12 layers x {Wq, Wk, Wv, Wo 768x768; W_fc 3072x768; W_proj 768x3072}, 72
+matrices, 84,934,656 parameters -- with bf16 weights and gradients, fp32 momentum, Nesterov
+beta = 0.95, K = 5 quintic Newton-Schulz iterations on the tensor cores, and the Hyperball
+rule with rho = ||W0||_F per matrix and eta = 0.02.  Gradients are seeded N(0, sigma^2) noise
+plus a rank-8 spike of RMS 10 sigma, sigma log-uniform in [1e-4, 1e-2] per matrix; four
+gradient sets rotate so every step sees a fresh one.  Inputs (W + G + M, 680 MB) are larger
+than the 126 MB L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+One JSON line is printed by rank 0.  Under torchrun (N > 1) every rank runs its own replica
+of the matrix set on its own GPU (weak scaling, no collective on the data path); the time is
+the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Muon-H optimizer step ms; NS TFLOP/s (% bf16 peak); fused-kernel HBM GB/s"
+WORKLOAD = "gpt2-small matrix set, MuonH step (72 bf16 matrices, fp32 momentum, K=5, Hyperball)"
+ETA = 0.02
+N_GRAD_SETS = 4
+DEFAULT_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def shapes():
+    from newton_schulz_hyperball_b200 import workloads as wl
+    return [(r, c) for _, r, c in wl.gpt2_small_shapes(12)]
+
+
+def ns_flops(shp, K=5):
+    """Algorithmic NS work per step: K (3 r^2 s + r^3), symmetric products counted once."""
+    tot = 0.0
+    for r, c in shp:
+        rr, ss = min(r, c), max(r, c)
+        tot += K * (3.0 * rr * rr * ss + rr ** 3)
+    return tot
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(DEFAULT_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        names = {
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_power_brake": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for k, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ workload
+def build_inputs(dev, rank: int):
+    """Host-side seeded inputs (bf16 values as float32 arrays) for the 72 matrices."""
+    import numpy as np
+    from newton_schulz_hyperball_b200 import workloads as wl
+    cfg = wl.CFG_GPT2_SMALL
+    shp = shapes()
+    W0 = [wl.init_weight(cfg, i, r, c, bf16=True) for i, (r, c) in enumerate(shp)]
+    G = [[wl.gradient(cfg, i, s, r, c, bf16=True) for i, (r, c) in enumerate(shp)] for s in range(N_GRAD_SETS)]
+    return W0, G
+
+
+def run_cuda(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import newton_schulz_hyperball_b200 as nshb
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    shp = shapes()
+    W0, Gh = build_inputs(dev, rank)
+    W = [torch.from_numpy(w).to(dev).to(torch.bfloat16) for w in W0]
+    Gd = [[torch.from_numpy(g).to(dev).to(torch.bfloat16) for g in gs] for gs in Gh]
+    M = [torch.zeros(w.shape, dtype=torch.float32, device=dev) for w in W]
+    rho = torch.tensor([float(np.linalg.norm(w.astype(np.float64))) for w in W0], dtype=torch.float32, device=dev)
+    p = nshb.params(eta=ETA, rho=rho)
+    mats = [nshb.matrices(W, Gd[s], M) for s in range(N_GRAD_SETS)]
+    ws = nshb.workspace(mats[0], p, nshb.NSHB_OP_HYPERBALL, device=dev)
+    n_params = sum(r * c for r, c in shp)
+
+    def step(k):
+        nshb.hyperball_step(mats[k % N_GRAD_SETS], p, ws, stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # warm-up
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    flags = nshb.device_status(ws, stream)
+
+    # ---- timed region: device-resident inputs
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        e0.record(stream)
+        for k in range(args.steps):
+            step(k)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+
+    # ---- per-kernel times (same step, events around each launch)
+    nshb.profile_enable(True)
+    nshb.profile_read()
+    kp = max(10, min(args.steps, 50))
+    for k in range(kp):
+        step(k)
+    torch.cuda.synchronize()
+    prof = nshb.profile_read()
+    nshb.profile_enable(False)
+    launches_per_step = sum(c for _, c in prof.values()) / kp
+
+    # ---- end to end through the public API with host buffers: H2D of the step's
+    # gradients from pinned memory, the step, D2H of the device status word.
+    Gpin = [[torch.from_numpy(g).to(torch.bfloat16).pin_memory() for g in gs] for gs in Gh[:2]]
+    Gdst = [torch.empty_like(g) for g in Gd[0]]
+    mats_e = nshb.matrices(W, Gdst, M)
+    st_host = torch.empty(1, dtype=torch.int32).pin_memory()
+    h2d = sum(g.numel() * g.element_size() for g in Gpin[0])
+    ke = max(5, min(args.steps, 30))
+    torch.cuda.synchronize()
+    barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(ke):
+        for d, s in zip(Gdst, Gpin[k % 2]):
+            d.copy_(s, non_blocking=True)
+        nshb.hyperball_step(mats_e, p, ws, stream)
+        st_host.copy_(ws[:4].view(torch.int32), non_blocking=True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1)) / ke
+
+    return dict(ms=ms, prof=prof, kp=kp, launches_per_step=launches_per_step, flags=flags,
+                clocks=clk.summary(), e2e_ms=e2e_ms, h2d=h2d, d2h=4, n_params=n_params, shp=shp)
+
+
+# --------------------------------------------------------------- CPU baseline
+def oracle_sample(layers=1, steps=1):
+    """Times the fp64 oracle on `layers` of the 12 GPT-2 layers for `steps` steps and returns
+    (seconds per full 72-matrix step extrapolated by NS flops, sample description)."""
+    import numpy as np
+    from newton_schulz_hyperball_b200 import workloads as wl
+    from oracle import nshb_oracle as o
+    cfg = wl.CFG_GPT2_SMALL
+    shp = shapes()
+    idx = list(range(6 * layers))
+    Ws = {i: wl.init_weight(cfg, i, *shp[i], bf16=True).astype(np.float64) for i in idx}
+    Ms = {i: np.zeros(shp[i]) for i in idx}
+    rho = {i: o.fro(Ws[i]) for i in idx}
+    Gs = [{i: wl.gradient(cfg, i, s, *shp[i], bf16=True).astype(np.float64) for i in idx} for s in range(steps)]
+    t0 = time.perf_counter()
+    for s in range(steps):
+        for i in idx:
+            Ws[i], Ms[i], _, _ = o.hyperball_step(Ws[i], Gs[s][i], Ms[i], eta=ETA, rho=rho[i])
+    dt = (time.perf_counter() - t0) / steps
+    full = dt * ns_flops(shp) / ns_flops([shp[i] for i in idx])
+    return full, f"{len(idx)} of 72 matrices (GPT-2 layer 0..{layers - 1}), {steps} step(s), extrapolated by NS flops"
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, rank, world):
+    """The oracle on the host cores, on this workload (bounded sample per step)."""
+    if rank != 0:
+        return None
+    for _ in range(args.warmup):
+        oracle_sample(1, 1)
+    times = []
+    desc = None
+    for _ in range(args.steps):
+        full, desc = oracle_sample(1, 1)
+        times.append(full)
+    ms = 1e3 * statistics.median(times)
+    return dict(ms=ms, desc=desc)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if world > 1 and rank != 0:
+            return 0
+        steps = min(args.steps, 20)
+        args.steps = steps
+        args.warmup = min(args.warmup, 3)
+        r = run_reference(args, rank, world)
+        line = {"metric": METRIC, "value": round(r["ms"], 3), "unit": "ms", "n_gpus": args.gpus, "steps": steps,
+                "warmup": args.warmup, "ms_per_step": round(r["ms"], 3), "higher_is_better": False,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "impl": "reference",
+                "config": {"workload": WORKLOAD, "matrices": 72, "params": 84934656},
+                "cpu_baseline": {"value": round(r["ms"], 3), "unit": "ms", "cores": cpu_cores(), "kind": "oracle",
+                                 "sample": r["desc"]},
+                "e2e": {"value": round(r["ms"], 3), "unit": "ms", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+
+    r = run_cuda(args, rank, world, local_rank)
+    peaks, peak_src = load_peaks()
+    shp = r["shp"]
+    flops = ns_flops(shp)
+    prof = r["prof"]
+    kp = r["kp"]
+    gemm_ms = sum(prof.get(k, (0.0, 0))[0] for k in ("gram", "poly", "update")) / kp
+    gemm_launches = sum(prof.get(k, (0.0, 0))[1] for k in ("gram", "poly", "update")) / kp
+    ns_tflops = flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
+    n = r["n_params"]
+    # Algorithmic HBM bytes of the fused streaming kernels: momentum 12 B/elem
+    # (G 2 + M 4 + 4 + U 2), apply 6 B/elem (W 2 + 2, O 2).
+    mom_ms = prof.get("momentum", (0.0, 0))[0] / kp
+    apply_ms = prof.get("apply", (0.0, 0))[0] / kp
+    red_ms = prof.get("reduce", (0.0, 0))[0] / kp
+    fused_bytes = 18.0 * n
+    fused_ms = mom_ms + apply_ms + red_ms
+    fused_gbs = fused_bytes / (fused_ms * 1e-3) / 1e9 if fused_ms > 0 else None
+    mom_gbs = 12.0 * n / (mom_ms * 1e-3) / 1e9 if mom_ms > 0 else None
+    peak_tf = peaks.get("bf16_tflops", DEFAULT_PEAKS["bf16_tflops"])
+    peak_bw = peaks.get("hbm_gbs", DEFAULT_PEAKS["hbm_gbs"])
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t0 = time.perf_counter()
+        full, desc = oracle_sample(1, 1)
+        cpu = {"value": round(full * 1e3, 3), "unit": "ms", "cores": cpu_cores(), "kind": "oracle",
+               "sample": desc + f" ({time.perf_counter() - t0:.1f} s of CPU work)"}
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC,
+        "value": round(r["ms"], 4),
+        "unit": "ms",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(r["ms"], 4),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded W0 ~ N(0, 0.02^2), spiked Gaussian gradients; no dataset)",
+        "config": {"workload": WORKLOAD, "matrices": len(shp), "params": n, "ns_steps": 5,
+                   "optimizer": "MuonH (Nesterov 0.95, eta 0.02, rho = ||W0||)",
+                   "l2": "inputs larger than L2 (W+G+M = 680 MB per step, 4 rotating gradient sets)",
+                   "parallelism": f"replica per GPU x{world}"},
+        "throughput": {"value": round(world * n / (r["ms"] * 1e-3), 1), "unit": "params/s"},
+        "ns_tflops": None if ns_tflops is None else round(ns_tflops, 1),
+        "ns_frac_of_bf16_peak": None if ns_tflops is None else round(ns_tflops / peak_tf, 4),
+        "fused_gbs": None if fused_gbs is None else round(fused_gbs, 1),
+        "fused_frac_of_hbm": None if fused_gbs is None else round(fused_gbs / peak_bw, 4),
+        "roofline": {"bound": "tensor", "kernel": "gemm_tc_kernel (NS Gram/poly/update)",
+                     "achieved": None if ns_tflops is None else round(ns_tflops, 1),
+                     "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": None if ns_tflops is None else round(ns_tflops / peak_tf, 4),
+                     "traffic": None, "peak_source": f"{peak_src} bf16 burst",
+                     "per_launch_ms": round(gemm_ms / max(gemm_launches, 1), 5)},
+        "kernels_ms_per_step": {k: round(v[0] / kp, 5) for k, v in prof.items()},
+        "momentum_gbs": None if mom_gbs is None else round(mom_gbs, 1),
+        "gpu_launches": int(round(r["launches_per_step"] * args.steps)),
+        "device_status": r["flags"],
+        "clocks": r["clocks"],
+        "e2e": {"value": round(r["e2e_ms"], 4), "unit": "ms", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"]},
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -178,6 +178,26 @@ nshb_status nshb_device_status(const void *ws, nshb_stream stream, uint32_t *fla
 /* Static, NUL-terminated name of a status code. */
 const char *nshb_status_string(int32_t status);
 
+/* Measurement aid.  While enabled (process-wide switch), every kernel launch of a step is
+ * bracketed by two CUDA events recorded on the step's stream.  nshb_profile_read waits for
+ * the recorded events, writes the summed kernel time (ms) and the launch count of each
+ * kind (NSHB_PROF_*) into ms[0..n_kinds) / launches[0..n_kinds), and clears the record.
+ * The events are created by the library on first use and reused afterwards. */
+#define NSHB_PROF_MOMENTUM 0 /* momentum + U + norm partials                  */
+#define NSHB_PROF_NORM 1     /* per-matrix / per-tile normalisation scales    */
+#define NSHB_PROF_GRAM 2     /* tensor-core A = s^2 X X^T                      */
+#define NSHB_PROF_POLY 3     /* tensor-core B = b A + c A^2                    */
+#define NSHB_PROF_UPDATE 4   /* tensor-core X' = s (a X + B X)                 */
+#define NSHB_PROF_REDUCE 5   /* ||O||^2, <W,O>, ||W||^2 partials               */
+#define NSHB_PROF_FINALIZE 6 /* per-matrix update coefficients                 */
+#define NSHB_PROF_EXACT 7    /* element-wise ||W - tO||^2 for cancelling steps */
+#define NSHB_PROF_APPLY 8    /* W <- alpha W + beta O                          */
+#define NSHB_PROF_F32GEMM 9  /* fp32 NS GEMMs (all three phases)               */
+#define NSHB_PROF_NEWTON 10  /* Newton-Muon Gram, Cholesky and solves          */
+#define NSHB_PROF_KINDS 12
+nshb_status nshb_profile_enable(int32_t on);
+nshb_status nshb_profile_read(int32_t n_kinds, float *ms, int32_t *launches);
+
 /* ABI version (major * 10000 + minor * 100 + patch). */
 int32_t nshb_version(void);
 

@@ -187,3 +187,16 @@ def device_status(ws, stream=None) -> int:
     v = ctypes.c_uint32(0)
     _check(lib().nshb_device_status(ptr, _stream(stream), ctypes.byref(v)), "nshb_device_status")
     return v.value
+
+
+def profile_enable(on: bool = True) -> None:
+    _check(lib().nshb_profile_enable(1 if on else 0), "nshb_profile_enable")
+
+
+def profile_read() -> dict:
+    """{kind: (ms, launches)} summed since the last read (waits for the recorded events)."""
+    n = _abi.NSHB_PROF_KINDS
+    ms = (ctypes.c_float * n)()
+    cnt = (ctypes.c_int32 * n)()
+    _check(lib().nshb_profile_read(n, ms, cnt), "nshb_profile_read")
+    return {_abi.NSHB_PROF_NAMES[k]: (ms[k], cnt[k]) for k in range(n) if cnt[k]}

@@ -29,6 +29,10 @@ NSHB_DEV_TIMEOUT = 0x4
 NSHB_DEV_ZERO_RADIUS = 0x8
 NSHB_DEV_NOT_SPD = 0x10
 
+NSHB_PROF_NAMES = ["momentum", "norm", "gram", "poly", "update", "reduce", "finalize", "exact", "apply",
+                   "f32gemm", "newton", "spare"]
+NSHB_PROF_KINDS = 12
+
 NSHB_OP_MUON = 0
 NSHB_OP_HYPERBALL = 1
 NSHB_OP_RADIAL_BRAKE = 2
@@ -92,6 +96,9 @@ SIGNATURES = {
     "nshb_device_status": (ctypes.c_int32, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "nshb_status_string": (ctypes.c_char_p, [ctypes.c_int32]),
     "nshb_version": (ctypes.c_int32, []),
+    "nshb_profile_enable": (ctypes.c_int32, [ctypes.c_int32]),
+    "nshb_profile_read": (ctypes.c_int32, [ctypes.c_int32, ctypes.POINTER(ctypes.c_float),
+                                           ctypes.POINTER(ctypes.c_int32)]),
 }
 
 

@@ -9,6 +9,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "../../include/nshb.h"
@@ -230,6 +231,62 @@ int device_sms() {
     }                                      \
   } while (0)
 
+
+// ---------------------------------------------------------------- phase timing
+// Opt-in measurement aid: when enabled, every kernel launch of a step is bracketed by two
+// CUDA events on the caller's stream; nshb_profile_read sums the elapsed times per kind.
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  struct Rec {
+    cudaEvent_t a, b;
+    int kind;
+  };
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+  }
+};
+Profiler &prof() {
+  static Profiler p;
+  return p;
+}
+struct ProfScope {
+  cudaEvent_t a = nullptr;
+  int kind;
+  cudaStream_t st;
+  ProfScope(int k, cudaStream_t s) : kind(k), st(s) {
+    Profiler &p = prof();
+    if (!p.on) return;
+    std::lock_guard<std::mutex> g(p.mu);
+    a = p.get();
+    if (a) cudaEventRecord(a, st);
+  }
+  ~ProfScope() {
+    if (!a) return;
+    Profiler &p = prof();
+    std::lock_guard<std::mutex> g(p.mu);
+    cudaEvent_t b = p.get();
+    if (!b) return;
+    cudaEventRecord(b, st);
+    p.recs.push_back({a, b, kind});
+  }
+};
+
+#define NSHB_LAUNCH(kind, call)   \
+  do {                            \
+    ProfScope ps_(kind, st);      \
+    NSHB_CHECK_CUDA(call);        \
+  } while (0)
+
 // momentum + per-segment norms
 nshb_status run_momentum(const nshb_matrix *mats, const Plan &pl, const nshb_params *p, char *ws,
                          cudaStream_t st) {
@@ -251,7 +308,7 @@ nshb_status run_momentum(const nshb_matrix *mats, const Plan &pl, const nshb_par
       nb += pl.mp[i].k1_blocks;
     }
     mp.total_blocks = nb;
-    NSHB_CHECK_CUDA(launch_momentum(mp, st));
+    NSHB_LAUNCH(NSHB_PROF_MOMENTUM, launch_momentum(mp, st));
 
     NormFinParams nf;
     std::memset(&nf, 0, sizeof(nf));
@@ -272,7 +329,7 @@ nshb_status run_momentum(const nshb_matrix *mats, const Plan &pl, const nshb_par
       blks += m.k1_blocks;
     }
     nf.seg_begin[c1 - c0] = segs;
-    NSHB_CHECK_CUDA(launch_norm_finalize(nf, segs, st));
+    NSHB_LAUNCH(NSHB_PROF_NORM, launch_norm_finalize(nf, segs, st));
   }
   return NSHB_OK;
 }
@@ -335,7 +392,7 @@ nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t 
           }
           fp.nprob = c1 - c0;
           fp.total_tiles = tiles;
-          NSHB_CHECK_CUDA(launch_gemm_f32(fp, st));
+          NSHB_LAUNCH(NSHB_PROF_F32GEMM, launch_gemm_f32(fp, st));
         }
       } else {
         for (int c0 = 0; c0 < n; c0 += kMaxProb) {
@@ -408,7 +465,7 @@ nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t 
           }
           gp.nprob = k;
           gp.total_tiles = tiles;
-          NSHB_CHECK_CUDA(launch_gemm_tc(gp, pl.bn, device_sms(), st));
+          NSHB_LAUNCH(NSHB_PROF_GRAM + mode, launch_gemm_tc(gp, pl.bn, device_sms(), st));
         }
       }
     }
@@ -461,17 +518,17 @@ nshb_status run_apply(const nshb_matrix *mats, const Plan &pl, const nshb_params
     ap.partials = wpart;
     fp.partials = wpart;
     if (apply_op != kOpMuon) {
-      NSHB_CHECK_CUDA(launch_reduce(ap, st));
+      NSHB_LAUNCH(NSHB_PROF_REDUCE, launch_reduce(ap, st));
     }
     fp.stage = 0;
-    NSHB_CHECK_CUDA(launch_apply_finalize(fp, st));
+    NSHB_LAUNCH(NSHB_PROF_FINALIZE, launch_apply_finalize(fp, st));
     if (apply_op == kOpNorms) continue;
     if (apply_op == kOpHyperball || apply_op == kOpBrake) {
-      NSHB_CHECK_CUDA(launch_exact_norm(ap, st));
+      NSHB_LAUNCH(NSHB_PROF_EXACT, launch_exact_norm(ap, st));
       fp.stage = 1;
-      NSHB_CHECK_CUDA(launch_apply_finalize(fp, st));
+      NSHB_LAUNCH(NSHB_PROF_FINALIZE, launch_apply_finalize(fp, st));
     }
-    NSHB_CHECK_CUDA(launch_apply(ap, st));
+    NSHB_LAUNCH(NSHB_PROF_APPLY, launch_apply(ap, st));
   }
   return NSHB_OK;
 }
@@ -621,6 +678,39 @@ const char *nshb_status_string(int32_t s) {
     case NSHB_ERR_UNSUPPORTED: return "NSHB_ERR_UNSUPPORTED";
     default: return "NSHB_ERR_UNKNOWN";
   }
+}
+
+nshb_status nshb_profile_enable(int32_t on) {
+  Profiler &p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  p.on = on != 0;
+  return NSHB_OK;
+}
+
+nshb_status nshb_profile_read(int32_t n_kinds, float *ms, int32_t *launches) {
+  if (n_kinds < 0 || (n_kinds > 0 && (!ms || !launches))) return NSHB_ERR_NULL;
+  Profiler &p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  for (int k = 0; k < n_kinds; ++k) {
+    ms[k] = 0.f;
+    launches[k] = 0;
+  }
+  nshb_status st = NSHB_OK;
+  for (auto &r : p.recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) {
+      (void)cudaGetLastError();
+      st = NSHB_ERR_CUDA;
+    }
+    if (r.kind >= 0 && r.kind < n_kinds) {
+      ms[r.kind] += t;
+      launches[r.kind] += 1;
+    }
+    p.pool.push_back(r.a);
+    p.pool.push_back(r.b);
+  }
+  p.recs.clear();
+  return st;
 }
 
 int32_t nshb_version(void) { return 100; }

@@ -126,11 +126,12 @@ def layer_input(cfg: int, zidx: int, d_in: int, n_tokens: int, lo: float = 0.1, 
     return round_to_bf16(np.exp(u) * e)
 
 
-def spectrum_matrix(seed: int, rows: int, cols: int, sigma) -> np.ndarray:
+def spectrum_matrix(seed: int, rows: int, cols: int, sigma, factors: bool = False):
     """A rows x cols float32 matrix Q1 diag(sigma) Q2^T with random orthonormal factors
-    (singular values given; the rest zero)."""
+    (singular values given; the rest zero).  With factors=True also returns (Q1, Q2)."""
     rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([99, seed])))
     k = len(sigma)
     q1, _ = np.linalg.qr(rng.standard_normal((rows, k)))
     q2, _ = np.linalg.qr(rng.standard_normal((cols, k)))
-    return ((q1 * np.asarray(sigma, dtype=np.float64)) @ q2.T).astype(np.float32)
+    m = ((q1 * np.asarray(sigma, dtype=np.float64)) @ q2.T).astype(np.float32)
+    return (m, q1, q2) if factors else m

@@ -208,24 +208,26 @@ def test_bf16_muon_and_brake_steps():
 # ---------------------------------------------------- page pins on the GPU
 def test_bf16_768_five_directions_page_pin():
     """Muon explainer, code section: bf16 NS of a 768x768 matrix with singular values
-    0.9, 0.3, 0.1, 0.01, 0.001 and the rest about 0.011 lands within 0.005 of the scalar
-    polynomial."""
+    0.9, 0.3, 0.1, 0.01, 0.001 (the other 763 about 0.011) lands within 0.005 of the scalar
+    polynomial.  Read as: the stretch along each of the five named singular directions,
+    u_k^T O v_k, is within 0.005 of phi^5 applied to that direction's normalised input
+    stretch (the 763 filler values are degenerate, so their order is not defined)."""
     import json, pathlib
     g = json.loads((pathlib.Path(__file__).parent / "golden" / "page_values.json").read_text())["bf16_768_example"]
     n = g["n"]
     sig = np.array(g["sigma_top"] + [g["bulk_sigma"]] * (n - 5))
-    U = wl.spectrum_matrix(5, n, n, sig).astype(np.float64)
-    U = wl.round_to_bf16(U.astype(np.float32)).astype(np.float64)
-    # Feed U as the Nesterov update: with M = 0 and beta = 0 (no momentum), U = G.
+    U32, q1, q2 = wl.spectrum_matrix(5, n, n, sig, factors=True)
+    U = wl.round_to_bf16(U32).astype(np.float64)
+    # With M = 0 and beta = 0 the Nesterov update is U = G.
     gs = GpuSet([np.zeros((n, n))], bf16=True)
     gs.set_grads([U])
-    p = nshb.params(beta=0.0, lr=0.0)
-    assert gs.step("muon", p) == 0
-    _, _, Og = gs.host()
-    s_in = np.linalg.svd(U, compute_uv=False)
-    expect = o.scalar_ns(s_in / (np.sqrt(np.sum(s_in ** 2)) + o.NS_EPS), 5)
-    s_out = np.linalg.svd(Og[0], compute_uv=False)
-    assert np.max(np.abs(np.sort(s_out) - np.sort(expect))) <= g["abs_tol"]
+    assert gs.step("muon", nshb.params(beta=0.0, lr=0.0)) == 0
+    O = gs.host()[2][0]
+    nrm = np.sqrt(np.sum(U * U)) + o.NS_EPS
+    for k in range(5):
+        d_in = q1[:, k] @ U @ q2[:, k]
+        d_out = q1[:, k] @ O @ q2[:, k]
+        assert abs(d_out - o.scalar_ns(d_in / nrm, 5)) <= g["abs_tol"], k
 
 
 def test_bf16_random_3072x768_band_page_pin():
