@@ -549,7 +549,7 @@ nshb_status do_step(const nshb_matrix *mats, int n_mats, const nshb_params *p, i
   e = check_ws(pl, ws, ws_bytes);
   if (e != NSHB_OK) return e;
   char *w = static_cast<char *>(ws);
-  NSHB_CHECK_CUDA(cudaMemsetAsync(w, 0, sizeof(uint32_t), st));
+  NSHB_CHECK_CUDA(cudaMemsetAsync(w, 0, 2 * sizeof(uint32_t), st));  // status word, exact-pass counter
   e = run_momentum(mats, pl, p, w, st);
   if (e != NSHB_OK) return e;
   std::vector<int64_t> o_off;
@@ -642,7 +642,7 @@ nshb_status nshb_fro_norms(const nshb_matrix *mats, int32_t n_mats, float *out, 
   if (e != NSHB_OK) return e;
   char *w = static_cast<char *>(ws);
   cudaStream_t st = (cudaStream_t)stream;
-  NSHB_CHECK_CUDA(cudaMemsetAsync(w, 0, sizeof(uint32_t), st));
+  NSHB_CHECK_CUDA(cudaMemsetAsync(w, 0, 2 * sizeof(uint32_t), st));  // status word, exact-pass counter
   std::vector<int64_t> none;
   return run_apply(mats, pl, &p, kOpNorms, w, st, none, out);
 }

@@ -339,6 +339,7 @@ __global__ void __launch_bounds__(kThreads) exact_norm_kernel(const __grid_const
   __shared__ float sO[kBlk][kBlk + 1];
   __shared__ double red[kThreads / 32];
   const int t = threadIdx.x, rr = t >> 2, cg = (t & 3) * 16;
+  if (*(volatile uint32_t *)(p.status + 1) == 0) return;  // no matrix of this call needs it
   for (int mi = 0; mi < p.nmat; ++mi) {
     const MatDesc &d = p.mats[mi];
     const MatScalars &sc = p.scal[d.mat];
@@ -400,25 +401,38 @@ __device__ void brake_coeffs(MatScalars &s, double vv, double pi, const ApplyFin
   s.beta = (float)(-f * s.t);
 }
 
+// One warp per matrix: the lanes sum the block partials in a fixed order, lane 0 derives
+// the coefficients.
 __global__ void apply_finalize_kernel(const __grid_constant__ ApplyFinParams p) {
-  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  const int k = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (k >= p.nmat) return;
   MatScalars &s = p.scal[p.mat[k]];
   const int m = p.m[k], n = p.n[k];
   const double sshape = sqrt(fmax(1.0, (double)m / (double)n));
   if (p.op == kOpMuon) {
-    s.alpha = (float)(1.0 - (double)p.lr * (double)p.weight_decay);
-    s.beta = (float)(-(double)p.lr * sshape);
-    s.need_exact = 0;
+    if (lane == 0) {
+      s.alpha = (float)(1.0 - (double)p.lr * (double)p.weight_decay);
+      s.beta = (float)(-(double)p.lr * sshape);
+      s.need_exact = 0;
+    }
     return;
   }
+  double om = 0.0, de = 0.0, pi = 0.0, ex = 0.0;
   if (p.stage == 0) {
-    double om = 0.0, de = 0.0, pi = 0.0;
-    for (int b = p.blk_begin[k]; b < p.blk_begin[k + 1]; ++b) {
+    for (int b = p.blk_begin[k] + lane; b < p.blk_begin[k + 1]; b += 32) {
       om += p.partials[3 * (int64_t)b];
       de += p.partials[3 * (int64_t)b + 1];
       pi += p.partials[3 * (int64_t)b + 2];
     }
+    om = warp_sum(om);
+    de = warp_sum(de);
+    pi = warp_sum(pi);
+  } else if (s.need_exact) {
+    for (int b = p.blk_begin[k] + lane; b < p.blk_begin[k + 1]; b += 32) ex += p.partials[b];
+    ex = warp_sum(ex);
+  }
+  if (lane != 0) return;
+  if (p.stage == 0) {
     s.omega = om; s.delta = de; s.pi = pi;
     s.need_exact = 0;
     if (p.op == kOpNorms) {
@@ -443,14 +457,13 @@ __global__ void apply_finalize_kernel(const __grid_constant__ ApplyFinParams p) 
     // fp32-accumulated partials; recompute ||W - tO||^2 element-wise instead.
     if (vv < 1e-2 * (pi + tw)) {
       s.need_exact = 1;
+      atomicAdd(p.status + 1, 1u);   // tells the exact-norm pass that it has work
       return;
     }
     s.vv = vv;
   } else {
     if (!s.need_exact) return;
-    double vv = 0.0;
-    for (int b = p.blk_begin[k]; b < p.blk_begin[k + 1]; ++b) vv += p.partials[b];
-    s.vv = vv;
+    s.vv = ex;
     s.need_exact = 0;
   }
   if (p.op == kOpHyperball) {
@@ -516,7 +529,7 @@ cudaError_t launch_exact_norm(const ApplyParams &p, cudaStream_t s) {
   return cudaGetLastError();
 }
 cudaError_t launch_apply_finalize(const ApplyFinParams &p, cudaStream_t s) {
-  if (p.nmat > 0) apply_finalize_kernel<<<(p.nmat + 127) / 128, 128, 0, s>>>(p);
+  if (p.nmat > 0) apply_finalize_kernel<<<(p.nmat + 3) / 4, 128, 0, s>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_apply(const ApplyParams &p, cudaStream_t s) {
