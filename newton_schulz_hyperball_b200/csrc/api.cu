@@ -403,6 +403,7 @@ nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t 
           gp.scales = scales;
           gp.status = status;
           gp.wait_limit = limit;
+          gp.test_stall = (p->debug_flags & 2u) ? 1 : 0;
           gp.mode = mode;
           gp.ca = ca; gp.cb = cb; gp.cc = cc;
           // Longest-k problems first, so the static tile walk ends evenly.

@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
             phase ^= 1u;
           }
         }
-        if (ok) tc_commit(tfull_bar(buf));
+        if (ok && !(p.test_stall && tl == 0)) tc_commit(tfull_bar(buf));
       }
     }
   } else {

@@ -123,6 +123,8 @@ struct GemmParams {
                           //          hi + lo pair and D may be written as one
   float ca, cb, cc;
   int32_t nprob, total_tiles;
+  int32_t test_stall;     // tests only: the MMA warp withholds its first accumulator commit,
+                          // so the epilogue's bounded wait runs out (NSHB_DEV_TIMEOUT)
   GemmProb prob[kMaxProb];
 };
 
