@@ -121,7 +121,10 @@ typedef struct {
   int32_t ns_compensated;/* bf16 NS: leading iterations whose a*X term reads X as a bf16 hi/lo */
                          /* pair (about fp32 accuracy); 0 = plain bf16 chain; default 2;      */
                          /* values above ns_steps act as ns_steps; range [0, 32]             */
-  uint32_t debug_flags;  /* 0 in normal use; bit 0 shortens the device wait limit (tests)     */
+  uint32_t debug_flags;  /* 0 in normal use.  Tests only: bit 0 shortens every device wait    */
+                         /* limit to ~1 ms; bit 1 makes the tensor-core GEMM withhold one     */
+                         /* accumulator hand-off so that a bounded wait runs out and the step */
+                         /* reports NSHB_DEV_TIMEOUT (results then are not valid)             */
 } nshb_params;
 
 /* Fills *p with the defaults listed above.  Returns NSHB_ERR_NULL if p is NULL. */
@@ -170,6 +173,19 @@ nshb_status newton_muon_step(const nshb_matrix *mats, int32_t n_mats, const void
  * Needs a workspace of nshb_workspace_size(..., NSHB_OP_MUON, ...) bytes. */
 nshb_status nshb_fro_norms(const nshb_matrix *mats, int32_t n_mats, float *out, void *ws,
                            size_t ws_bytes, nshb_stream stream);
+
+/* No counterpart in the papers: an allocation-free variant of nshb_fro_norms for callers
+ * that cannot allocate device memory (e.g. a hook running inside a framework whose caching
+ * allocator owns the device memory, or a C tool with no allocator) and so cannot pass a
+ * workspace.  out[i] = ||W_i||_F (fp32, DEVICE array of n_mats floats); only W, rows, cols,
+ * ld and w_dtype of each matrix are read.  Scratch is a fixed NSHB_STATIC_SCRATCH_BYTES
+ * device array inside the library, held by every GPU that loads it until exit.  The first
+ * call on a device looks up that array's address (make it before any stream capture).
+ * Limits: n_mats <= 192 and sum over matrices of ceil(rows/64) * ceil(cols/64) <= 174,240
+ * (about 7.1e8 elements); larger requests return NSHB_ERR_WORKSPACE before any work is
+ * queued.  Calls share the array, so calls that overlap on the GPU race. */
+#define NSHB_STATIC_SCRATCH_BYTES (4u << 20)
+nshb_status nshb_fro_norms_static(const nshb_matrix *mats, int32_t n_mats, float *out, nshb_stream stream);
 
 /* Synchronises `stream`, then copies the device status word of the last step that used
  * this workspace into *flags (NSHB_DEV_* bits).  The one call that blocks the host. */

@@ -182,6 +182,11 @@ def fro_norms(mats, out, ws, stream=None):
     _check(lib().nshb_fro_norms(mats, _n(mats), _ptr(out), ptr, nbytes, _stream(stream)), "nshb_fro_norms")
 
 
+def fro_norms_static(mats, out, stream=None):
+    """||W_i||_F into `out` without a workspace (scratch is a fixed array in the library)."""
+    _check(lib().nshb_fro_norms_static(mats, _n(mats), _ptr(out), _stream(stream)), "nshb_fro_norms_static")
+
+
 def device_status(ws, stream=None) -> int:
     ptr, _ = _ws(ws)
     v = ctypes.c_uint32(0)

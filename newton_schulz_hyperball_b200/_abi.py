@@ -93,6 +93,7 @@ SIGNATURES = {
                                           ctypes.POINTER(ctypes.c_int64), ctypes.c_int32, ctypes.c_int64,
                                           _PAR, _P, ctypes.c_size_t, _P]),
     "nshb_fro_norms": (ctypes.c_int32, [_MATS, ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]),
+    "nshb_fro_norms_static": (ctypes.c_int32, [_MATS, ctypes.c_int32, _P, _P]),
     "nshb_device_status": (ctypes.c_int32, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "nshb_status_string": (ctypes.c_char_p, [ctypes.c_int32]),
     "nshb_version": (ctypes.c_int32, []),
