@@ -131,10 +131,12 @@ typedef struct {
 nshb_status nshb_default_params(nshb_params *p);
 
 /* Bytes of device workspace that a step of kind `op` on these matrices needs.
- * `n_tokens` and the Z rows matter only for NSHB_OP_NEWTON_MUON (pass 0 / NULL otherwise).
- * Host-only: touches no device memory.  The workspace must be 256-byte aligned. */
+ * z_rows (HOST array of n_z), n_z and n_tokens matter only for NSHB_OP_NEWTON_MUON
+ * (pass NULL / 0 / 0 otherwise).  Host-only: touches no device memory.  The workspace must
+ * be 256-byte aligned. */
 nshb_status nshb_workspace_size(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p,
-                                int32_t op, const int64_t *z_rows, int32_t n_z, size_t *bytes);
+                                int32_t op, const int64_t *z_rows, int32_t n_z, int64_t n_tokens,
+                                size_t *bytes);
 
 /* Muon step (Muon.step code): momentum, NS, W <- (1 - lr wd) W - lr max(1, m/n)^0.5 O. */
 nshb_status muon_step(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, void *ws,
@@ -161,10 +163,12 @@ nshb_status himuon_step(const nshb_matrix *mats, int32_t n_mats, const nshb_para
 
 /* Newton-Muon wrapped by Hyperball: P = U (Z Z^T + lambda I)^-1 with
  * lambda = ridge_rel tr(Z Z^T) / d_in, solved through an fp32 Cholesky factorisation,
- * then O = NS_K(P) and the Hyperball rule.  Z[j] is a DEVICE pointer to a bf16 row-major
- * z_rows[j] x n_tokens matrix (leading dimension n_tokens, 16-byte aligned, n_tokens a
- * multiple of 64); matrix i uses Z[mats[i].z_index], which needs z_rows == cols.
- * Z and z_rows are HOST arrays of n_z entries. */
+ * then O = NS_K(P) and the Hyperball rule (U is the Nesterov momentum update).  Z[j] is a
+ * DEVICE pointer to a bf16 row-major z_rows[j] x n_tokens matrix (leading dimension
+ * n_tokens, 16-byte aligned); n_tokens and every z_rows[j] must be multiples of 64 (up to
+ * 16384 rows); matrix i uses Z[mats[i].z_index], which needs z_rows == cols.  Z and z_rows
+ * are HOST arrays of n_z entries (n_z <= 192).  A pivot that is not positive in fp32 sets
+ * NSHB_DEV_NOT_SPD.  bf16 NS only. */
 nshb_status newton_muon_step(const nshb_matrix *mats, int32_t n_mats, const void *const *Z,
                              const int64_t *z_rows, int32_t n_z, int64_t n_tokens,
                              const nshb_params *p, void *ws, size_t ws_bytes, nshb_stream stream);

@@ -113,21 +113,21 @@ def _n(mats) -> int:
     return getattr(mats, "_n", len(mats))
 
 
-def workspace_size(mats, p, op: int, z_rows=None) -> int:
+def workspace_size(mats, p, op: int, z_rows=None, n_tokens: int = 0) -> int:
     out = ctypes.c_size_t(0)
     zr, nz = None, 0
     if z_rows is not None:
         nz = len(z_rows)
         zr = (ctypes.c_int64 * max(nz, 1))(*[int(x) for x in z_rows])
-    _check(lib().nshb_workspace_size(mats, _n(mats), ctypes.byref(p), op, zr, nz, ctypes.byref(out)),
-           "nshb_workspace_size")
+    _check(lib().nshb_workspace_size(mats, _n(mats), ctypes.byref(p), op, zr, nz, int(n_tokens),
+                                     ctypes.byref(out)), "nshb_workspace_size")
     return out.value
 
 
-def workspace(mats, p, op: int, device=None, z_rows=None):
+def workspace(mats, p, op: int, device=None, z_rows=None, n_tokens: int = 0):
     """A device workspace (torch uint8 tensor, 256-byte aligned by the caching allocator)."""
     import torch
-    nbytes = workspace_size(mats, p, op, z_rows)
+    nbytes = workspace_size(mats, p, op, z_rows, n_tokens)
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device or "cuda")
 
 

@@ -83,7 +83,7 @@ _PAR = ctypes.POINTER(nshb_params)
 SIGNATURES = {
     "nshb_default_params": (ctypes.c_int32, [_PAR]),
     "nshb_workspace_size": (ctypes.c_int32, [_MATS, ctypes.c_int32, _PAR, ctypes.c_int32,
-                                             ctypes.POINTER(ctypes.c_int64), ctypes.c_int32,
+                                             ctypes.POINTER(ctypes.c_int64), ctypes.c_int32, ctypes.c_int64,
                                              ctypes.POINTER(ctypes.c_size_t)]),
     "muon_step": (ctypes.c_int32, [_MATS, ctypes.c_int32, _PAR, _P, ctypes.c_size_t, _P]),
     "hyperball_step": (ctypes.c_int32, [_MATS, ctypes.c_int32, _PAR, _P, ctypes.c_size_t, _P]),

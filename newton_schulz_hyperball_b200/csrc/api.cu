@@ -48,6 +48,16 @@ struct Plan {
   int bn = 256;
   int comp = 0;                  // compensated (hi/lo) iterations of the bf16 chain
   std::vector<MatPlan> mp;
+  // Newton-Muon: per layer input Z
+  struct ZPlan {
+    int64_t d = 0, Dp = 0;
+    const void *src = nullptr;
+    int64_t zp = 0, s = 0, inv = 0;   // panel copy of Z, S / L (fp32 Dp x Dp), diagonal-block inverses
+  };
+  std::vector<ZPlan> zp;
+  int64_t n_tokens = 0;
+  std::vector<int64_t> r_off;         // per matrix: fp32 m x n buffer for U -> Y -> P
+  std::vector<int> zidx;
   size_t scal_off = 0, scale_off = 0, nu_off = 0, k1part_off = 0, wpart_off = 0, total = 0;
   int nseg = 0, k1_total = 0, w_total = 0;
 };
@@ -178,6 +188,41 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
   return NSHB_OK;
 }
 
+// Extends a plan with the Newton-Muon buffers (layer inputs, Gram / Cholesky factors, the
+// fp32 right-hand sides of the triangular solves).
+nshb_status plan_newton(const nshb_matrix *mats, int n_mats, const void *const *Z, const int64_t *z_rows, int n_z,
+                        int64_t n_tokens, Plan &pl) {
+  if (n_z <= 0 || n_z > kMaxMats || !z_rows) return n_z <= 0 || !z_rows ? NSHB_ERR_NULL : NSHB_ERR_UNSUPPORTED;
+  if (n_tokens <= 0 || n_tokens % 64 != 0 || n_tokens > (1LL << 24)) return NSHB_ERR_SHAPE;
+  if (pl.f32ns) return NSHB_ERR_UNSUPPORTED;
+  pl.n_tokens = n_tokens;
+  pl.zp.resize(n_z);
+  size_t off = pl.total;
+  for (int j = 0; j < n_z; ++j) {
+    Plan::ZPlan &z = pl.zp[j];
+    z.d = z_rows[j];
+    if (z.d <= 0 || z.d % 64 != 0 || z.d > 16384) return NSHB_ERR_SHAPE;
+    z.src = Z ? Z[j] : nullptr;
+    if (Z && (!z.src || (uintptr_t)z.src % 16 != 0)) return !z.src ? NSHB_ERR_NULL : NSHB_ERR_SHAPE;
+    z.Dp = round_up(z.d, 256);
+    z.zp = off; off = align_up(off + (size_t)z.Dp * n_tokens * 2);
+    z.s = off;  off = align_up(off + (size_t)z.Dp * z.Dp * 4);
+    z.inv = off; off = align_up(off + (size_t)(z.d / 64) * 64 * 64 * 4);
+  }
+  pl.r_off.resize(n_mats);
+  pl.zidx.resize(n_mats);
+  for (int i = 0; i < n_mats; ++i) {
+    const int zi = mats[i].z_index;
+    if (zi < 0 || zi >= n_z) return NSHB_ERR_PARAM;
+    if (pl.zp[zi].d != mats[i].cols) return NSHB_ERR_SHAPE;
+    pl.zidx[i] = zi;
+    pl.r_off[i] = off;
+    off = align_up(off + (size_t)mats[i].rows * mats[i].cols * 4);
+  }
+  pl.total = off;
+  return NSHB_OK;
+}
+
 MatDesc make_desc(const nshb_matrix &d, const MatPlan &m, int idx, int64_t o_off, int blk_begin, bool k1) {
   MatDesc r;
   std::memset(&r, 0, sizeof(r));
@@ -187,6 +232,7 @@ MatDesc make_desc(const nshb_matrix &d, const MatPlan &m, int idx, int64_t o_off
   r.O_out = d.O_out;
   r.x_off = m.x0;
   r.xlo_off = m.xl0;
+  r.u_off = 0;
   r.o_off = o_off;
   r.m = (int)m.m;
   r.n = (int)m.n;
@@ -289,7 +335,7 @@ struct ProfScope {
 
 // momentum + per-segment norms
 nshb_status run_momentum(const nshb_matrix *mats, const Plan &pl, const nshb_params *p, char *ws,
-                         cudaStream_t st) {
+                         cudaStream_t st, bool from_p = false) {
   const int n = (int)pl.mp.size();
   double *k1part = reinterpret_cast<double *>(ws + pl.k1part_off);
   for (int c0 = 0; c0 < n; c0 += kMaxMats) {
@@ -305,6 +351,10 @@ nshb_status run_momentum(const nshb_matrix *mats, const Plan &pl, const nshb_par
     int nb = 0;
     for (int i = c0; i < c1; ++i) {
       mp.mats[i - c0] = make_desc(mats[i], pl.mp[i], i, 0, nb, true);
+      if (from_p) {
+        mp.mats[i - c0].flags |= kFromP;
+        mp.mats[i - c0].u_off = pl.r_off[i];
+      }
       nb += pl.mp[i].k1_blocks;
     }
     mp.total_blocks = nb;
@@ -534,6 +584,190 @@ nshb_status run_apply(const nshb_matrix *mats, const Plan &pl, const nshb_params
   return NSHB_OK;
 }
 
+// F32 GEMM problem helper.
+F32Prob f32prob(int64_t a, int lda, int64_t b, int ldb, int bt, int64_t c, int64_t d, int ldc, int M, int N, int K) {
+  F32Prob q;
+  std::memset(&q, 0, sizeof(q));
+  q.a_off = a; q.lda = lda;
+  q.b_off = b; q.ldb = ldb; q.b_trans = bt;
+  q.c_off = c; q.d_off = d; q.ldc = ldc;
+  q.M = M; q.N = N; q.K = K;
+  q.scale_idx = -1;
+  q.tiles_n = (N + 63) / 64;
+  return q;
+}
+
+// Launches the fp32 GEMM on a list of problems (split into launches of kMaxProb).
+nshb_status run_f32(const std::vector<F32Prob> &probs, int mode, char *ws, cudaStream_t st) {
+  for (size_t c0 = 0; c0 < probs.size(); c0 += kMaxProb) {
+    const size_t c1 = std::min(probs.size(), c0 + kMaxProb);
+    F32Params fp;
+    std::memset(&fp, 0, sizeof(fp));
+    fp.ws = ws;
+    fp.mode = mode;
+    int tiles = 0;
+    for (size_t i = c0; i < c1; ++i) {
+      F32Prob q = probs[i];
+      q.tile_begin = tiles;
+      tiles += ((q.M + 63) / 64) * q.tiles_n;
+      fp.prob[i - c0] = q;
+    }
+    fp.nprob = (int)(c1 - c0);
+    fp.total_tiles = tiles;
+    NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_gemm_f32(fp, st));
+  }
+  return NSHB_OK;
+}
+
+// P = U (Z Z^T + lambda I)^-1 for every matrix; leaves P (fp32, m x n) at pl.r_off[i].
+nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const nshb_params *p, char *ws,
+                               cudaStream_t st) {
+  const int n = (int)pl.mp.size(), nz = (int)pl.zp.size();
+  uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+  const long long limit = (p->debug_flags & 1u) ? kWaitLimitTest : kWaitLimit;
+  // 1. momentum, U in fp32 row-major
+  for (int c0 = 0; c0 < n; c0 += kMaxMats) {
+    const int c1 = std::min(n, c0 + kMaxMats);
+    MomentumParams mp;
+    std::memset(&mp, 0, sizeof(mp));
+    mp.ws = ws;
+    mp.partials = reinterpret_cast<double *>(ws + pl.k1part_off);
+    mp.status = status;
+    mp.beta = p->beta;
+    mp.nesterov = p->nesterov ? 1 : 0;
+    mp.nmat = c1 - c0;
+    int nb = 0;
+    for (int i = c0; i < c1; ++i) {
+      MatDesc d = make_desc(mats[i], pl.mp[i], i, 0, nb, false);
+      d.flags = (d.flags & (kVec | kWF32)) | kURow;
+      d.u_off = pl.r_off[i];
+      mp.mats[i - c0] = d;
+      nb += pl.mp[i].w_blocks;
+    }
+    mp.total_blocks = nb;
+    NSHB_LAUNCH(NSHB_PROF_MOMENTUM, launch_momentum(mp, st));
+  }
+  // 2. Z -> panels, S = Z Z^T on the tensor cores (fp32 out), ridge
+  for (int c0 = 0; c0 < nz; c0 += kMaxMats) {
+    const int c1 = std::min(nz, c0 + kMaxMats);
+    PackParams pp;
+    std::memset(&pp, 0, sizeof(pp));
+    pp.ws = ws;
+    pp.n = c1 - c0;
+    int nb = 0;
+    for (int j = c0; j < c1; ++j) {
+      const Plan::ZPlan &z = pl.zp[j];
+      pp.src[j - c0] = z.src;
+      pp.dst_off[j - c0] = z.zp;
+      pp.rows[j - c0] = (int)z.d;
+      pp.cols[j - c0] = (int)pl.n_tokens;
+      pp.ld[j - c0] = (int)pl.n_tokens;
+      pp.ph[j - c0] = (int)z.Dp;
+      pp.blk_begin[j - c0] = nb;
+      nb += (int)(z.Dp / 64) * (int)(pl.n_tokens / 64);
+    }
+    pp.blk_begin[c1 - c0] = nb;
+    NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_pack_panels(pp, st));
+
+    GemmParams gp;
+    std::memset(&gp, 0, sizeof(gp));
+    gp.ws = ws;
+    gp.status = status;
+    gp.wait_limit = limit;
+    gp.test_stall = 0;
+    gp.mode = kGramF32;
+    int tiles = 0, k = 0;
+    for (int j = c0; j < c1; ++j) {
+      const Plan::ZPlan &z = pl.zp[j];
+      GemmProb &q = gp.prob[k++];
+      q.a_off = q.b_off = z.zp;
+      q.c_off = q.d_off = z.s;
+      q.c_lo = q.d_lo = -1;
+      q.a_ph = q.b_ph = (int)z.Dp;
+      q.d_ph = (int)z.Dp;
+      q.mt = (int)(z.Dp / 128);
+      q.nt = (int)(z.Dp / 256);
+      q.kt = (int)(pl.n_tokens / 64);
+      q.batch = 1;
+      int cnt = 0;
+      for (int mi = 0; mi < q.mt; ++mi) cnt += std::min(q.nt, (128 * mi + 127) / 256 + 1);
+      q.tiles_per_batch = cnt;
+      q.tile_begin = tiles;
+      q.scale_idx = -1;
+      tiles += cnt;
+    }
+    gp.nprob = k;
+    gp.total_tiles = tiles;
+    NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_gemm_tc(gp, 256, device_sms(), st));
+  }
+  // 3. blocked Cholesky, all layer inputs at once
+  int64_t dmax = 0;
+  for (auto &z : pl.zp) dmax = std::max(dmax, z.d);
+  for (int c0 = 0; c0 < nz; c0 += kMaxMats) {
+    const int c1 = std::min(nz, c0 + kMaxMats);
+    CholParams cp;
+    std::memset(&cp, 0, sizeof(cp));
+    cp.ws = ws;
+    cp.status = status;
+    cp.ridge_rel = p->ridge_rel;
+    cp.n = c1 - c0;
+    for (int j = c0; j < c1; ++j) {
+      cp.s_off[j - c0] = pl.zp[j].s;
+      cp.inv_off[j - c0] = pl.zp[j].inv;
+      cp.ld[j - c0] = (int)pl.zp[j].Dp;
+      cp.d[j - c0] = (int)pl.zp[j].d;
+    }
+    NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_ridge(cp, st));
+    for (int64_t k = 0; k < dmax; k += 64) {
+      cp.k = (int)k;
+      NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_potrf_block(cp, st));
+      std::vector<F32Prob> panel, trail;
+      for (int j = c0; j < c1; ++j) {
+        const Plan::ZPlan &z = pl.zp[j];
+        if (k + 64 >= z.d) continue;
+        const int ld = (int)z.Dp, rest = (int)(z.d - k - 64);
+        const int64_t pan = z.s + ((k + 64) * z.Dp + k) * 4;
+        panel.push_back(f32prob(pan, ld, z.inv + (k / 64) * 64 * 64 * 4, 64, 1, pan, pan, ld, rest, 64, 64));
+        const int64_t tr = z.s + ((k + 64) * z.Dp + (k + 64)) * 4;
+        trail.push_back(f32prob(pan, ld, pan, ld, 1, tr, tr, ld, rest, rest, 64));
+      }
+      nshb_status e = run_f32(panel, kPlain, ws, st);
+      if (e != NSHB_OK) return e;
+      e = run_f32(trail, kSub, ws, st);
+      if (e != NSHB_OK) return e;
+    }
+  }
+  // 4. P = U L^-T L^-1 by right-looking block solves, in place on the fp32 buffer
+  int max_blocks = 0;
+  for (int i = 0; i < n; ++i) max_blocks = std::max(max_blocks, (int)(pl.mp[i].n / 64));
+  for (int pass = 0; pass < 2; ++pass) {
+    for (int sidx = 0; sidx < max_blocks; ++sidx) {
+      std::vector<F32Prob> solve, upd;
+      for (int i = 0; i < n; ++i) {
+        const Plan::ZPlan &z = pl.zp[pl.zidx[i]];
+        const int d = (int)pl.mp[i].n, m = (int)pl.mp[i].m, nb = d / 64;
+        if (sidx >= nb) continue;
+        const int kb = pass == 0 ? sidx : nb - 1 - sidx;
+        const int64_t k = (int64_t)kb * 64;
+        const int64_t R = pl.r_off[i];
+        const int64_t inv = z.inv + (int64_t)kb * 64 * 64 * 4;
+        solve.push_back(f32prob(R + k * 4, d, inv, 64, pass == 0 ? 1 : 0, R + k * 4, R + k * 4, d, m, 64, 64));
+        if (pass == 0 && k + 64 < d) {
+          upd.push_back(f32prob(R + k * 4, d, z.s + ((k + 64) * z.Dp + k) * 4, (int)z.Dp, 1, R + (k + 64) * 4,
+                                R + (k + 64) * 4, d, m, (int)(d - k - 64), 64));
+        } else if (pass == 1 && k > 0) {
+          upd.push_back(f32prob(R + k * 4, d, z.s + (k * z.Dp) * 4, (int)z.Dp, 0, R, R, d, m, (int)k, 64));
+        }
+      }
+      nshb_status e = run_f32(solve, kPlain, ws, st);
+      if (e != NSHB_OK) return e;
+      e = run_f32(upd, kSub, ws, st);
+      if (e != NSHB_OK) return e;
+    }
+  }
+  return NSHB_OK;
+}
+
 nshb_status check_ws(const Plan &pl, void *ws, size_t ws_bytes) {
   if (!ws) return NSHB_ERR_NULL;
   if ((uintptr_t)ws % kAlign != 0) return NSHB_ERR_WORKSPACE;
@@ -591,13 +825,15 @@ nshb_status nshb_default_params(nshb_params *p) {
 }
 
 nshb_status nshb_workspace_size(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, int32_t op,
-                                const int64_t *z_rows, int32_t n_z, size_t *bytes) {
+                                const int64_t *z_rows, int32_t n_z, int64_t n_tokens, size_t *bytes) {
   if (!bytes) return NSHB_ERR_NULL;
-  (void)z_rows;
-  (void)n_z;
   Plan pl;
   nshb_status e = plan_step(mats, n_mats, p, op, pl);
   if (e != NSHB_OK) return e;
+  if (op == NSHB_OP_NEWTON_MUON && n_mats > 0) {
+    e = plan_newton(mats, n_mats, nullptr, z_rows, n_z, n_tokens, pl);
+    if (e != NSHB_OK) return e;
+  }
   *bytes = pl.total;
   return NSHB_OK;
 }
@@ -625,9 +861,26 @@ nshb_status himuon_step(const nshb_matrix *mats, int32_t n_mats, const nshb_para
 nshb_status newton_muon_step(const nshb_matrix *mats, int32_t n_mats, const void *const *Z, const int64_t *z_rows,
                              int32_t n_z, int64_t n_tokens, const nshb_params *p, void *ws, size_t ws_bytes,
                              nshb_stream stream) {
-  (void)mats; (void)n_mats; (void)Z; (void)z_rows; (void)n_z; (void)n_tokens; (void)p; (void)ws;
-  (void)ws_bytes; (void)stream;
-  return NSHB_ERR_UNSUPPORTED;
+  Plan pl;
+  nshb_status e = plan_step(mats, n_mats, p, NSHB_OP_NEWTON_MUON, pl);
+  if (e != NSHB_OK) return e;
+  if (n_mats == 0) return NSHB_OK;
+  if (!Z) return NSHB_ERR_NULL;
+  e = plan_newton(mats, n_mats, Z, z_rows, n_z, n_tokens, pl);
+  if (e != NSHB_OK) return e;
+  e = check_ws(pl, ws, ws_bytes);
+  if (e != NSHB_OK) return e;
+  char *w = static_cast<char *>(ws);
+  cudaStream_t st = (cudaStream_t)stream;
+  NSHB_CHECK_CUDA(cudaMemsetAsync(w, 0, 2 * sizeof(uint32_t), st));  // status word, exact-pass counter
+  e = run_newton_precond(mats, pl, p, w, st);
+  if (e != NSHB_OK) return e;
+  e = run_momentum(mats, pl, p, w, st, /*from_p=*/true);
+  if (e != NSHB_OK) return e;
+  std::vector<int64_t> o_off;
+  e = run_ns(pl, p, w, st, o_off);
+  if (e != NSHB_OK) return e;
+  return run_apply(mats, pl, p, kOpHyperball, w, st, o_off, nullptr);
 }
 
 nshb_status nshb_fro_norms(const nshb_matrix *mats, int32_t n_mats, float *out, void *ws, size_t ws_bytes,

@@ -7,8 +7,10 @@
 //   kPoly    B  = b A + c A A
 //   kUpdate  X' = s (a X + B X)
 // where s = 1 / (||U|| + eps) on the first iteration (the normalisation folded into the
-// first Gram and update epilogues) and 1 afterwards.  ("Muon: the orthogonalized optimizer
-// explained", Newton-Schulz section and newton_schulz5.)
+// first Gram and update epilogues) and 1 afterwards ("Muon: the orthogonalized optimizer
+// explained", Newton-Schulz section and newton_schulz5).  The same kernel also computes the
+// plain product D = A B and the update D = C - A B of the Newton-Muon Cholesky
+// factorisation and triangular solves.
 //
 // 64x64 output tiles, 16-deep k slices staged in shared memory, 256 threads with a 4x4
 // register tile each.  Deterministic: every output is one fixed-order fp32 dot product.
@@ -82,6 +84,7 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const __grid_constant__ F
       if (p.mode == kGram) v = (s * s) * acc[x][y];
       else if (p.mode == kPoly) v = fmaf(p.cb, C[o], p.cc * acc[x][y]);
       else if (p.mode == kUpdate) v = s * fmaf(p.ca, C[o], acc[x][y]);
+      else if (p.mode == kSub) v = C[o] - acc[x][y];
       else v = acc[x][y];
       D[o] = v;
     }

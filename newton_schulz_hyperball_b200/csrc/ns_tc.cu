@@ -68,7 +68,7 @@ __device__ __forceinline__ Tile decode(const GemmParams &p, int tile) {
   t.prob = lo;
   t.batch = lt / q.tiles_per_batch;
   int l = lt % q.tiles_per_batch;
-  if (p.mode == kGram || p.mode == kPoly) {
+  if (p.mode == kGram || p.mode == kPoly || p.mode == kGramF32) {
     int mi = 0;
     for (;; ++mi) {
       const int c = sym_cnt<BN>(mi, q.nt);
@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       const char *clo = q.c_lo >= 0 ? p.ws + q.c_lo + (int64_t)t.batch * q.c_bs : nullptr;
       char *dlo = q.d_lo >= 0 ? p.ws + q.d_lo + (int64_t)t.batch * q.d_bs : nullptr;
       const int64_t i = t.m0 + row;
-      const bool sym = (p.mode == kGram || p.mode == kPoly);
+      const bool sym = (p.mode == kGram || p.mode == kPoly || p.mode == kGramF32);
       const int ra = (int)(i >> 6);
 #pragma unroll 1
       for (int cc = 0; cc < BN / 32; ++cc) {
@@ -240,6 +240,21 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         tmem_ld32(tmem_base + (uint32_t)(buf * BN + cc * 32) + ((uint32_t)(quarter * 32) << 16), r);
         tmem_ld_wait();
         float v[32];
+        if (p.mode == kGramF32) {
+          // fp32 row-major output (row stride d_ph) for the Newton-Muon Gram S = Z Z^T.
+          float *drow = reinterpret_cast<float *>(dbase) + i * q.d_ph;
+#pragma unroll
+          for (int g = 0; g < 8; ++g)
+            *reinterpret_cast<float4 *>(drow + col0 + 4 * g) =
+                make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]), __uint_as_float(r[4 * g + 2]),
+                            __uint_as_float(r[4 * g + 3]));
+          if (ca < ra) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              reinterpret_cast<float *>(dbase)[(int64_t)(col0 + e) * q.d_ph + i] = __uint_as_float(r[e]);
+          }
+          continue;
+        }
         if (p.mode == kGram) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] = s2 * __uint_as_float(r[e]);

@@ -19,6 +19,8 @@ constexpr int kWF32 = 4;        // W and G are fp32 (else bf16)
 constexpr int kTiled = 8;       // Hierarchical Muon: X is a grid of T x T tiles
 constexpr int kNsF32 = 16;      // NS in fp32, X row-major fp32 (else bf16 panel layout)
 constexpr int kTileMajor = 32;  // block list enumerates tile by tile (momentum of tiled matrices)
+constexpr int kFromP = 64;      // momentum kernel: take U from an fp32 row-major matrix (no momentum)
+constexpr int kURow = 128;      // momentum kernel: write U as fp32 row-major only (Newton-Muon input)
 
 // Per-matrix record of a streaming launch (momentum, reductions, apply).
 struct MatDesc {
@@ -28,6 +30,7 @@ struct MatDesc {
   void *O_out;
   int64_t x_off;     // workspace byte offset of X0 (where U is written)
   int64_t xlo_off;   // workspace byte offset of U's bf16 low part, or -1
+  int64_t u_off;     // kURow / kFromP: workspace byte offset of the fp32 row-major m x n U / P
   int64_t o_off;     // workspace byte offset of the final O
   int32_t m, n, ld;  // W shape and leading dimension
   int32_t flags;
@@ -111,7 +114,7 @@ struct GemmProb {
   int32_t batch, tiles_per_batch, tile_begin;
   int32_t scale_idx;                   // scale of batch 0 in GemmParams::scales, or -1
 };
-enum GemmMode { kGram = 0, kPoly = 1, kUpdate = 2, kPlain = 3 };
+enum GemmMode { kGram = 0, kPoly = 1, kUpdate = 2, kPlain = 3, kSub = 4, kGramF32 = 5 };
 struct GemmParams {
   char *ws;
   const float *scales;
@@ -146,6 +149,26 @@ struct F32Params {
   F32Prob prob[kMaxProb];
 };
 
+// Newton-Muon helpers.
+struct PackParams {          // row-major bf16 (rows x cols, ld) -> panel layout (ph rows)
+  const void *src[kMaxMats];
+  int64_t dst_off[kMaxMats];
+  int32_t rows[kMaxMats], cols[kMaxMats], ld[kMaxMats], ph[kMaxMats];
+  int32_t blk_begin[kMaxMats + 1];
+  char *ws;
+  int32_t n;
+};
+struct CholParams {          // one blocked-Cholesky step (column block k) for a batch of matrices
+  char *ws;
+  uint32_t *status;
+  int64_t s_off[kMaxMats];   // fp32 row-major S / L (ld = ld[i])
+  int64_t inv_off[kMaxMats]; // fp32 64 x 64 inverse of each diagonal block, block b at +b*64*64
+  int32_t ld[kMaxMats], d[kMaxMats];
+  float ridge_rel;
+  int32_t k;                 // first column of the block
+  int32_t n;
+};
+
 // Launchers (defined in the .cu files); each returns cudaGetLastError().
 cudaError_t launch_momentum(const MomentumParams &p, cudaStream_t s);
 cudaError_t launch_norm_finalize(const NormFinParams &p, int nseg_total, cudaStream_t s);
@@ -155,5 +178,8 @@ cudaError_t launch_apply_finalize(const ApplyFinParams &p, cudaStream_t s);
 cudaError_t launch_apply(const ApplyParams &p, cudaStream_t s);
 cudaError_t launch_gemm_tc(const GemmParams &p, int bn, int num_sms, cudaStream_t s);
 cudaError_t launch_gemm_f32(const F32Params &p, cudaStream_t s);
+cudaError_t launch_pack_panels(const PackParams &p, cudaStream_t s);
+cudaError_t launch_ridge(const CholParams &p, cudaStream_t s);
+cudaError_t launch_potrf_block(const CholParams &p, cudaStream_t s);
 
 }  // namespace nshb

@@ -210,19 +210,30 @@ __global__ void __launch_bounds__(kThreads) momentum_kernel(const __grid_constan
   const int t = threadIdx.x, rr = t >> 2, cg = (t & 3) * 16;
   const int i = r0 + rr, j = c0 + cg;
   const bool f32 = d.flags & kWF32, vec = d.flags & kVec;
-  const bool round_bf16 = !(d.flags & kNsF32);
+  const bool round_bf16 = !(d.flags & (kNsF32 | kURow));
   const bool lo_part = round_bf16 && d.xlo_off >= 0;
 
   float g[16], mm[16], u[16], ul[16];
-  load16(d.G, d.ld, i, j, d.m, d.n, f32, vec, g);
-  loadM(d.M, d.ld, i, j, d.m, d.n, vec, mm);
+  const bool from_p = d.flags & kFromP;
+  if (from_p) {
+    // U is given (the Newton-Muon preconditioned update), fp32 row-major m x n.
+    load16(p.ws + d.u_off, d.n, i, j, d.m, d.n, true, (d.n % 4) == 0, g);
+  } else {
+    load16(d.G, d.ld, i, j, d.m, d.n, f32, vec, g);
+    loadM(d.M, d.ld, i, j, d.m, d.n, vec, mm);
+  }
   const float beta = p.beta, omb = 1.0f - p.beta;
   float acc = 0.f;
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
-    const float mnew = fmaf(beta, mm[e], omb * g[e]);
-    mm[e] = mnew;
-    float uf = p.nesterov ? fmaf(omb, g[e], beta * mnew) : mnew;
+    float uf;
+    if (from_p) {
+      uf = g[e];
+    } else {
+      const float mnew = fmaf(beta, mm[e], omb * g[e]);
+      mm[e] = mnew;
+      uf = p.nesterov ? fmaf(omb, g[e], beta * mnew) : mnew;
+    }
     if (!(i < d.m && j + e < d.n)) uf = 0.f;
     const float uh = round_bf16 ? bf16_round(uf) : uf;
     u[e] = uh;
@@ -230,7 +241,12 @@ __global__ void __launch_bounds__(kThreads) momentum_kernel(const __grid_constan
     const float un = lo_part ? uf : uh;    // the norm of what the first iteration reads
     acc = fmaf(un, un, acc);
   }
-  store16(d.M, d.ld, i, j, d.m, d.n, true, vec, mm);
+  if (!from_p) store16(d.M, d.ld, i, j, d.m, d.n, true, vec, mm);
+  if (d.flags & kURow) {
+    // Newton-Muon: U goes to an fp32 row-major buffer for the triangular solves.
+    store16(p.ws + d.u_off, d.n, i, j, d.m, d.n, true, (d.n % 4) == 0, u);
+    return;
+  }
 
   char *xbase = p.ws + d.x_off;
   char *lbase = lo_part ? p.ws + d.xlo_off : nullptr;

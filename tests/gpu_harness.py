@@ -54,3 +54,12 @@ def rel_fro(a, b) -> float:
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def newton_step(gs: "GpuSet", Zs, n_tokens: int, p):
+    """Runs newton_muon_step on a GpuSet whose matrices carry z_index; Zs are host arrays."""
+    Zd = [to_dev(z, True) for z in Zs]
+    need = nshb.workspace_size(gs.mats, p, nshb.NSHB_OP_NEWTON_MUON, [z.shape[0] for z in Zs], n_tokens)
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=DEV)
+    nshb.newton_muon_step(gs.mats, Zd, n_tokens, p, ws)
+    return nshb.device_status(ws)

@@ -349,3 +349,33 @@ def test_device_wait_limit_reports_timeout_without_faulting():
     _, _, Og = gs2.host()
     _, U = o.momentum(np.zeros_like(G), G, 0.95, True)
     assert rel_fro(Og[0], o.newton_schulz(U)) <= 2e-2
+
+
+# ---------------------------------------------------------------- Newton-Muon
+def test_bf16_newton_muon_small():
+    """P = U (Z Z^T + lambda I)^-1 through the tensor-core Gram, fp32 blocked Cholesky and
+    block solves, then bf16 NS and Hyperball; against the oracle's plain linear solve."""
+    from gpu_harness import newton_step
+    cfg = wl.CFG_NEWTON_GPT2
+    n_tok = 512
+    Zs = [wl.layer_input(cfg, 0, 128, n_tok), wl.layer_input(cfg, 1, 256, n_tok)]
+    shapes = [(192, 128), (128, 256), (320, 256), (64, 128)]
+    zi = [0, 1, 1, 0]
+    Ws = [wl.init_weight(cfg, 40 + i, r, c, bf16=True).astype(np.float64) for i, (r, c) in enumerate(shapes)]
+    Gs = [wl.gradient(cfg, 40 + i, 0, r, c, bf16=True).astype(np.float64) for i, (r, c) in enumerate(shapes)]
+    rhos = [o.fro(w) for w in Ws]
+    gs = GpuSet(Ws, bf16=True)
+    for k in range(len(shapes)):
+        gs.mats[k].z_index = zi[k]
+    gs.set_grads(Gs)
+    rho_dev = torch.tensor(rhos, dtype=torch.float32, device="cuda")
+    p = nshb.params(eta=0.02, rho=rho_dev, ridge_rel=1e-3)
+    assert newton_step(gs, Zs, n_tok, p) == 0
+    Wg, Mg, Og = gs.host()
+    for i, W in enumerate(Ws):
+        Wr, Mr, Or, _ = o.newton_muon_step(W, Gs[i], np.zeros_like(W), Zs[zi[i]].astype(np.float64),
+                                           ridge_rel=1e-3, eta=0.02, rho=rhos[i])
+        assert rel_fro(Mg[i], Mr) <= 1e-6
+        assert rel_fro(Og[i], Or) <= 2e-2, (i, rel_fro(Og[i], Or))
+        assert np.linalg.norm(Wg[i] - Wr) <= bf16_w_tol(Wr, 0.02)
+        assert abs(o.fro(Wg[i]) - rhos[i]) / rhos[i] <= radius_tol(Wg[i], True)
