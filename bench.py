@@ -172,6 +172,12 @@ def run_cuda(args, rank, world, local_rank):
         step(k)
     torch.cuda.synchronize()
     flags = nshb.device_status(ws, stream)
+    if args.ncu:
+        # profiling case: exactly `steps` more steps, nothing else
+        for k in range(args.steps):
+            step(args.warmup + k)
+        torch.cuda.synchronize()
+        return None
 
     # ---- timed region: device-resident inputs
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -276,8 +282,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ncu", action="store_true",
+                    help="profiling case: warm-up and `steps` steps only, no timing or report")
     args = ap.parse_args()
-    if args.warmup < 3:
+    if args.warmup < 3 and not args.ncu:
         args.warmup = 3
 
     rank = int(os.environ.get("RANK", "0"))
@@ -311,6 +319,9 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
 
     r = run_cuda(args, rank, world, local_rank)
+    if r is None:
+        print("ncu case done", flush=True)
+        return 0
     peaks, peak_src = load_peaks()
     shp = r["shp"]
     flops = ns_flops(shp)
