@@ -20,8 +20,9 @@
 //    contiguous copies and no tensor map is needed;
 //  * warp 1 issues tcgen05.mma (M=128, N=BN, K=16) into one of two TMEM accumulators and
 //    commits each stage back to the producer;
-//  * warps 2-5 drain the other accumulator (tcgen05.ld), apply the phase epilogue and
-//    store bf16, overlapping the next tile's main loop.
+//  * warps 2-9 drain the other accumulator (tcgen05.ld), apply the phase epilogue and
+//    store bf16, overlapping the next tile's main loop; the epilogue's C operand is
+//    fetched a chunk ahead (the first chunk before the accumulator is ready).
 // Every mbarrier wait is bounded; a wait that runs out sets NSHB_DEV_TIMEOUT and the role
 // returns, after which the CTA drains its copies and frees its tensor memory.
 #include <cuda_runtime.h>
@@ -34,6 +35,8 @@ namespace nshb {
 namespace {
 
 constexpr int BM = 128, BK = 64;
+constexpr int kEpiThreads = 256;              // eight epilogue warps
+constexpr int kThreads = 64 + kEpiThreads;   // + producer warp + MMA warp
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 template <int BN> struct Cfg {
   static constexpr int STAGES = BN == 256 ? 4 : 6;
@@ -85,7 +88,7 @@ __device__ __forceinline__ Tile decode(const GemmParams &p, int tile) {
 }
 
 template <int BN>
-__global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmParams p) {
   constexpr int STAGES = Cfg<BN>::STAGES, B_BYTES = Cfg<BN>::B_BYTES, STAGE_BYTES = Cfg<BN>::STAGE_BYTES;
   constexpr int TMEM_COLS = Cfg<BN>::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
@@ -107,7 +110,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), 128);
+      mbar_init(tempty_bar(b), kEpiThreads);
     }
     mbar_fence_init();
   }
@@ -209,19 +212,20 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     }
   } else {
     // -------------------------------------------------------------- epilogue
-    const int quarter = warp & 3;                 // TMEM lanes this warp may read
+    // Eight warps: warp w reads TMEM lane quarter (w % 4) -- the hardware restriction --
+    // and one half of the tile's columns, so each quarter is drained by two warps.
+    constexpr int NCH = BN / 64;                  // 32-column chunks per warp
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;          // row of the 128-row tile
+    const bool sym = (p.mode == kGram || p.mode == kPoly || p.mode == kGramF32);
+    const bool needc = (p.mode == kPoly || p.mode == kUpdate);
     int tl = 0;
     for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++tl) {
       const Tile t = decode<BN>(p, tile);
       const GemmProb &q = p.prob[t.prob];
       const int buf = tl & 1;
       const uint32_t tph = (uint32_t)(tl >> 1) & 1u;
-      if (!mbar_wait(tfull_bar(buf), tph, limit)) {
-        set_status(p.status, kTimeoutBit);
-        break;
-      }
-      tc_fence_after();
       const float s = q.scale_idx >= 0 ? p.scales[q.scale_idx + t.batch] : 1.0f;
       const float s2 = s * s;
       const char *cbase = p.ws + q.c_off + (int64_t)t.batch * q.c_bs;
@@ -229,13 +233,33 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       const char *clo = q.c_lo >= 0 ? p.ws + q.c_lo + (int64_t)t.batch * q.c_bs : nullptr;
       char *dlo = q.d_lo >= 0 ? p.ws + q.d_lo + (int64_t)t.batch * q.d_bs : nullptr;
       const int64_t i = t.m0 + row;
-      const bool sym = (p.mode == kGram || p.mode == kPoly || p.mode == kGramF32);
       const int ra = (int)(i >> 6);
+      const int cc_end = (half + 1) * NCH;
+      // chunk cc is processed unless it lies wholly above the diagonal (symmetric outputs)
+      auto live = [&](int cc) { return cc < cc_end && !(sym && ((t.n0 + cc * 32) >> 6) > ra); };
+      auto load_c = [&](int cc, uint4 (&h)[4], uint4 (&l)[4]) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const size_t off = panel_chunk_off(i, t.n0 + cc * 32 + 8 * g, q.d_ph);
+          h[g] = *reinterpret_cast<const uint4 *>(cbase + off);
+          l[g] = clo ? *reinterpret_cast<const uint4 *>(clo + off) : make_uint4(0, 0, 0, 0);
+        }
+      };
+      int cc = half * NCH;
+      uint4 ch[4], cl[4];
+      // C does not depend on the accumulator: fetch the first chunk before waiting for it.
+      if (needc && live(cc)) load_c(cc, ch, cl);
+      if (!mbar_wait(tfull_bar(buf), tph, limit)) {
+        set_status(p.status, kTimeoutBit);
+        break;
+      }
+      tc_fence_after();
 #pragma unroll 1
-      for (int cc = 0; cc < BN / 32; ++cc) {
+      for (; live(cc); ++cc) {
         const int col0 = t.n0 + cc * 32;
         const int ca = col0 >> 6;
-        if (sym && ca > ra) continue;            // upper-triangle block: filled by the mirror
+        uint4 nh[4], nl[4];
+        if (needc && live(cc + 1)) load_c(cc + 1, nh, nl);   // one chunk ahead
         uint32_t r[32];
         tmem_ld32(tmem_base + (uint32_t)(buf * BN + cc * 32) + ((uint32_t)(quarter * 32) << 16), r);
         tmem_ld_wait();
@@ -264,17 +288,16 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
           const float ks = (p.mode == kPoly) ? 1.0f : s;
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
-            const size_t off = panel_chunk_off(i, col0 + 8 * g, q.d_ph);
-            const uint4 c4 = *reinterpret_cast<const uint4 *>(cbase + off);
-            float cv[8] = {bf16lo(c4.x), bf16hi(c4.x), bf16lo(c4.y), bf16hi(c4.y),
-                           bf16lo(c4.z), bf16hi(c4.z), bf16lo(c4.w), bf16hi(c4.w)};
-            if (clo) {   // C carried as a hi + lo pair
-              const uint4 l4 = *reinterpret_cast<const uint4 *>(clo + off);
-              cv[0] += bf16lo(l4.x); cv[1] += bf16hi(l4.x); cv[2] += bf16lo(l4.y); cv[3] += bf16hi(l4.y);
-              cv[4] += bf16lo(l4.z); cv[5] += bf16hi(l4.z); cv[6] += bf16lo(l4.w); cv[7] += bf16hi(l4.w);
-            }
+            const uint32_t hw[4] = {ch[g].x, ch[g].y, ch[g].z, ch[g].w};
+            const uint32_t lw[4] = {cl[g].x, cl[g].y, cl[g].z, cl[g].w};
 #pragma unroll
-            for (int h = 0; h < 8; ++h) v[8 * g + h] = ks * fmaf(kc, cv[h], ka * __uint_as_float(r[8 * g + h]));
+            for (int h = 0; h < 4; ++h) {
+              // C carried as a hi + lo pair (lo is zero when not kept)
+              const float c0 = bf16lo(hw[h]) + bf16lo(lw[h]);
+              const float c1 = bf16hi(hw[h]) + bf16hi(lw[h]);
+              v[8 * g + 2 * h] = ks * fmaf(kc, c0, ka * __uint_as_float(r[8 * g + 2 * h]));
+              v[8 * g + 2 * h + 1] = ks * fmaf(kc, c1, ka * __uint_as_float(r[8 * g + 2 * h + 1]));
+            }
           }
         }
 #pragma unroll
@@ -305,6 +328,11 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
             *reinterpret_cast<__nv_bfloat16 *>(dbase + panel_chunk_off(col0 + e, ib, q.d_ph) + 2 * ie) = h;
           }
         }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          ch[g] = nh[g];
+          cl[g] = nl[g];
+        }
       }
       tc_fence_before();
       mbar_arrive(tempty_bar(buf));
@@ -330,7 +358,7 @@ cudaError_t launch_bn(const GemmParams &p, int num_sms, cudaStream_t s) {
     done_mask |= 1u << (dev & 31);
   }
   const int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
-  gemm_tc_kernel<BN><<<grid, 192, Cfg<BN>::SMEM_BYTES, s>>>(p);
+  gemm_tc_kernel<BN><<<grid, kThreads, Cfg<BN>::SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
 }
 
