@@ -47,6 +47,7 @@ struct Plan {
   bool tiled = false;
   int bn = 256;
   int comp = 0;                  // compensated (hi/lo) iterations of the bf16 chain
+  bool pair = true;              // bf16 GEMMs on CTA pairs (256-row tiles); single CTAs for T = 128
   std::vector<MatPlan> mp;
   // Newton-Muon: per layer input Z
   struct ZPlan {
@@ -91,6 +92,7 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
     if (pl.f32ns) return NSHB_ERR_UNSUPPORTED;
     if (p->tile != 128 && p->tile != 256 && p->tile != 512) return NSHB_ERR_PARAM;
     pl.bn = p->tile == 128 ? 128 : 256;
+    pl.pair = p->tile != 128;
   }
   if (op == NSHB_OP_NEWTON_MUON) {
     if (!(p->ridge_rel >= 0.f) || !std::isfinite(p->ridge_rel)) return NSHB_ERR_PARAM;
@@ -254,6 +256,16 @@ MatDesc make_desc(const nshb_matrix &d, const MatPlan &m, int idx, int64_t o_off
   r.tiles_c = m.tiles_c;
   r.mat = idx;
   return r;
+}
+
+// Output tiles of one GEMM problem: all mt x nt tiles, or for the symmetric phases only
+// those that touch the lower triangle (BM-row block mi needs the BN-wide column tiles
+// that start at or before its last row).
+int gemm_tiles(int mode, int mt, int nt, int bm, int bn) {
+  if (mode == kUpdate || mode == kPlain) return mt * nt;
+  int cnt = 0;
+  for (int mi = 0; mi < mt; ++mi) cnt += std::min(nt, (bm * mi + bm - 1) / bn + 1);
+  return cnt;
 }
 
 int device_sms() {
@@ -483,7 +495,7 @@ nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t 
             }
             q.batch = batch;
             q.a_ph = q.b_ph = q.d_ph = (int)R;
-            q.mt = (int)(R / 128);
+            q.mt = (int)(R / (pl.pair ? 256 : 128));
             q.c_lo = -1;
             q.d_lo = -1;
             if (mode == kUpdate && it < pl.comp) {
@@ -503,20 +515,19 @@ nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t 
               q.a_bs = abs_; q.b_bs = xbs; q.c_bs = xbs; q.d_bs = xbs;
               q.nt = (int)(S / pl.bn); q.kt = (int)(R / 64);
             }
-            if (mode == kUpdate) {
-              q.tiles_per_batch = q.mt * q.nt;
-            } else {
-              int cnt = 0;
-              for (int mi = 0; mi < q.mt; ++mi) cnt += std::min(q.nt, (128 * mi + 127) / pl.bn + 1);
-              q.tiles_per_batch = cnt;
-            }
+            q.tiles_per_batch = gemm_tiles(mode, q.mt, q.nt, pl.pair ? 256 : 128, pl.bn);
             q.scale_idx = (it == 0 && mode != kPoly) ? m.seg_begin : -1;
             q.tile_begin = tiles;
             tiles += q.tiles_per_batch * q.batch;
           }
           gp.nprob = k;
           gp.total_tiles = tiles;
-          NSHB_LAUNCH(NSHB_PROF_GRAM + mode, launch_gemm_tc(gp, pl.bn, device_sms(), st));
+          if (pl.pair) {
+            NSHB_CHECK_CUDA(encode_ws_tensor_map(&gp.tmap, ws, pl.total / 128 * 128));
+            NSHB_LAUNCH(NSHB_PROF_GRAM + mode, launch_gemm_tc2(gp, device_sms(), st));
+          } else {
+            NSHB_LAUNCH(NSHB_PROF_GRAM + mode, launch_gemm_tc(gp, pl.bn, device_sms(), st));
+          }
         }
       }
     }
@@ -685,12 +696,11 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
       q.c_lo = q.d_lo = -1;
       q.a_ph = q.b_ph = (int)z.Dp;
       q.d_ph = (int)z.Dp;
-      q.mt = (int)(z.Dp / 128);
+      q.mt = (int)(z.Dp / 256);
       q.nt = (int)(z.Dp / 256);
       q.kt = (int)(pl.n_tokens / 64);
       q.batch = 1;
-      int cnt = 0;
-      for (int mi = 0; mi < q.mt; ++mi) cnt += std::min(q.nt, (128 * mi + 127) / 256 + 1);
+      const int cnt = gemm_tiles(kGramF32, q.mt, q.nt, 256, 256);
       q.tiles_per_batch = cnt;
       q.tile_begin = tiles;
       q.scale_idx = -1;
@@ -698,7 +708,8 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
     }
     gp.nprob = k;
     gp.total_tiles = tiles;
-    NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_gemm_tc(gp, 256, device_sms(), st));
+    NSHB_CHECK_CUDA(encode_ws_tensor_map(&gp.tmap, ws, pl.total / 128 * 128));
+    NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_gemm_tc2(gp, device_sms(), st));
   }
   // 3. blocked Cholesky, all layer inputs at once
   int64_t dmax = 0;

@@ -1,0 +1,482 @@
+// Grouped bf16 Newton-Schulz GEMM on CTA pairs (tcgen05.mma.cta_group::2).
+//
+// Same phases and epilogues as the single-CTA kernel (ns_tc.cu): Gram A = s^2 X X^T and
+// polynomial B = b A + c A^2 (lower-triangle tiles + mirrored stores), update
+// X' = s (a X + B X) ("Muon: the orthogonalized optimizer explained", Newton-Schulz
+// section and newton_schulz5), plus the fp32 Gram of the Newton-Muon layer inputs.
+//
+// Why pairs: with single-CTA 128 x 256 tiles every SM must stream 96 bytes of operands
+// per clock to keep its tensor core busy, more than the L2 delivers per SM.  A pair of
+// CTAs on two SMs computes a 256 x 256 tile with one instruction stream: each CTA holds
+// 128 rows of A and 128 columns of B, and the tensor cores read the partner's half
+// directly, so each SM streams 64 bytes per clock for the same work.
+//
+// Roles per CTA (320 threads): warp 0 issues TMA loads of this CTA's halves into a
+// 6-stage ring; in the leader CTA (rank 0) warp 1 issues the MMAs for the pair and
+// multicasts each commit to both CTAs; warps 2-9 of both CTAs drain their own 128-row
+// accumulator (two TMEM buffers, so the epilogue overlaps the next tile).  Loads of both
+// CTAs complete on the leader's "full" barrier; the epilogues of both CTAs arrive on the
+// leader's "tmem empty" barrier.  No load is multicast.  Every wait is bounded.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "nshb_device.cuh"
+#include "nshb_internal.h"
+
+namespace nshb {
+namespace {
+
+constexpr int BM = 256, BN = 256, BK = 64, STAGES = 6;
+constexpr int HALF_BYTES = 128 * BK * 2;          // 16 KB: 128 rows x 64 bf16
+constexpr int STAGE_BYTES = 2 * HALF_BYTES;       // A half + B half of one CTA
+constexpr int TMEM_COLS = 2 * BN;                 // two 128 x 256 fp32 accumulators
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr uint32_t kTimeoutBit = 0x4u;
+constexpr uint32_t kPeerMask = 0xFEFFFFFFu;       // clears the CTA-rank bit of a cluster address
+
+__device__ __forceinline__ uint32_t cta_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t num_clusters() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// 2-D TMA load into this CTA's shared memory; the transaction bytes complete on the
+// barrier at cluster address `bar` (the leader's barrier).
+__device__ __forceinline__ void tma_load_2sm(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc2(uint32_t dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish2() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_mma2(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.u32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on the barrier at this shared offset in every CTA of `mask` when all
+// tcgen05.mma issued so far by this thread have completed.
+__device__ __forceinline__ void tc_commit2_mc(uint32_t bar, uint16_t mask) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::
+                   "r"(bar),
+               "h"(mask)
+               : "memory");
+}
+
+struct Tile {
+  int prob, batch, m0, n0;
+};
+
+__device__ __forceinline__ bool sym_mode(int mode) { return mode == kGram || mode == kPoly || mode == kGramF32; }
+
+__device__ __forceinline__ Tile decode2(const GemmParams &p, int tile) {
+  int lo = 0, hi = p.nprob - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (p.prob[mid].tile_begin <= tile) lo = mid; else hi = mid - 1;
+  }
+  const GemmProb &q = p.prob[lo];
+  const int lt = tile - q.tile_begin;
+  Tile t;
+  t.prob = lo;
+  t.batch = lt / q.tiles_per_batch;
+  int l = lt % q.tiles_per_batch;
+  if (sym_mode(p.mode)) {
+    // 256-row block mi needs the column tiles nj <= mi (lower triangle incl. diagonal)
+    int mi = 0;
+    for (;; ++mi) {
+      const int c = (mi + 1 < q.nt) ? mi + 1 : q.nt;
+      if (l < c) break;
+      l -= c;
+    }
+    t.m0 = mi * BM;
+    t.n0 = l * BN;
+  } else {
+    t.m0 = (l / q.nt) * BM;
+    t.n0 = (l % q.nt) * BN;
+  }
+  return t;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 4);
+  const uint32_t smem_base = smem_u32(smem);
+  const uint32_t bar_base = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + 2 + b); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cta_rank();
+  const bool leader = rank == 0;
+  const int cid = (int)cluster_id(), ncl = (int)num_clusters();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 2 * kEpiWarps);   // one arrive per epilogue warp of both CTAs
+    }
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc2(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish2();
+  }
+  tc_fence_before();
+  cluster_sync();                                  // barriers of both CTAs initialised
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const long long limit = p.wait_limit;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer (both CTAs)
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_parity[STAGES];
+      for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
+      bool ok = true;
+      for (int tile = cid; ok && tile < p.total_tiles; tile += ncl) {
+        const Tile t = decode2(p, tile);
+        const GemmProb &q = p.prob[t.prob];
+        const int64_t a_row = (q.a_off + (int64_t)t.batch * q.a_bs) >> 7;   // 128-byte rows
+        const int64_t b_row = (q.b_off + (int64_t)t.batch * q.b_bs) >> 7;
+        const int am = t.m0 + 128 * (int)rank;     // this CTA's A rows
+        const int bn = t.n0 + 128 * (int)rank;     // this CTA's B columns
+        for (int kb = 0; kb < q.kt; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, limit)) {
+            set_status(p.status, kTimeoutBit);
+            ok = false;
+            break;
+          }
+          const uint32_t sA = smem_base + stage * STAGE_BYTES, sB = sA + HALF_BYTES;
+          const uint32_t fb = full_bar(stage) & kPeerMask;   // the leader's barrier
+          if (leader) {
+            mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
+            last_parity[stage] = (int)phase;
+          }
+          const int64_t ya = a_row + (int64_t)kb * q.a_ph + am;
+          tma_load_2sm(sA, &p.tmap, 0, (int)ya, fb);
+          tma_load_2sm(sA + HALF_BYTES / 2, &p.tmap, 0, (int)(ya + 64), fb);
+          if (p.mode != kUpdate) {
+            const int64_t yb = b_row + (int64_t)kb * q.b_ph + bn;
+            tma_load_2sm(sB, &p.tmap, 0, (int)yb, fb);
+            tma_load_2sm(sB + HALF_BYTES / 2, &p.tmap, 0, (int)(yb + 64), fb);
+          } else {
+            // MN-major: the 128 columns are two 64-column panels, rows kb*64 .. +63
+            const int64_t y0 = b_row + (int64_t)(bn >> 6) * q.b_ph + (int64_t)kb * BK;
+            tma_load_2sm(sB, &p.tmap, 0, (int)y0, fb);
+            tma_load_2sm(sB + HALF_BYTES / 2, &p.tmap, 0, (int)(y0 + q.b_ph), fb);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Drain: every load of the pair that the leader armed must have landed.
+      if (leader)
+        for (int s = 0; s < STAGES; ++s)
+          if (last_parity[s] >= 0 && !mbar_wait(full_bar(s), (uint32_t)last_parity[s], limit))
+            set_status(p.status, kTimeoutBit);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------------------ MMA issuer (leader)
+      const uint32_t idesc = idesc_bf16(BM, BN, p.mode == kUpdate ? 1 : 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int tl = 0;
+      bool ok = true;
+      for (int tile = cid; ok && tile < p.total_tiles; tile += ncl, ++tl) {
+        const Tile t = decode2(p, tile);
+        const GemmProb &q = p.prob[t.prob];
+        const int buf = tl & 1;
+        const uint32_t tph = (uint32_t)(tl >> 1) & 1u;
+        if (!mbar_wait(tempty_bar(buf), tph ^ 1u, limit)) {
+          set_status(p.status, kTimeoutBit);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+        for (int kb = 0; kb < q.kt; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, limit)) {
+            set_status(p.status, kTimeoutBit);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sA = smem_base + stage * STAGE_BYTES, sB = sA + HALF_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = smem_desc_sw128(sA + 32u * k, 16, 1024);
+            const uint64_t bd = (p.mode == kUpdate) ? smem_desc_sw128(sB + 2048u * k, HALF_BYTES / 2, 1024)
+                                                    : smem_desc_sw128(sB + 32u * k, 16, 1024);
+            tc_mma2(d_tmem, ad, bd, idesc, (kb | k) != 0);
+          }
+          tc_commit2_mc(empty_bar(stage), 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok && !(p.test_stall && tl == 0)) tc_commit2_mc(tfull_bar(buf), 0x3);
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue (both CTAs)
+    constexpr int NCH = BN / 64;                  // 32-column chunks per warp (half the tile)
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row = 128 * (int)rank + quarter * 32 + lane;   // row of the 256-row tile
+    const bool sym = sym_mode(p.mode);
+    const bool needc = (p.mode == kPoly || p.mode == kUpdate);
+    int tl = 0;
+    for (int tile = cid; tile < p.total_tiles; tile += ncl, ++tl) {
+      const Tile t = decode2(p, tile);
+      const GemmProb &q = p.prob[t.prob];
+      const int buf = tl & 1;
+      const uint32_t tph = (uint32_t)(tl >> 1) & 1u;
+      const float s = q.scale_idx >= 0 ? p.scales[q.scale_idx + t.batch] : 1.0f;
+      const float s2 = s * s;
+      const char *cbase = p.ws + q.c_off + (int64_t)t.batch * q.c_bs;
+      char *dbase = p.ws + q.d_off + (int64_t)t.batch * q.d_bs;
+      const char *clo = q.c_lo >= 0 ? p.ws + q.c_lo + (int64_t)t.batch * q.c_bs : nullptr;
+      char *dlo = q.d_lo >= 0 ? p.ws + q.d_lo + (int64_t)t.batch * q.d_bs : nullptr;
+      const int64_t i = t.m0 + row;
+      const int ra = (int)(i >> 6);
+      const int cc_end = (half + 1) * NCH;
+      auto live = [&](int cc) { return cc < cc_end && !(sym && ((t.n0 + cc * 32) >> 6) > ra); };
+      auto load_c = [&](int cc, uint4 (&h)[4], uint4 (&l)[4]) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const size_t off = panel_chunk_off(i, t.n0 + cc * 32 + 8 * g, q.d_ph);
+          h[g] = *reinterpret_cast<const uint4 *>(cbase + off);
+          l[g] = clo ? *reinterpret_cast<const uint4 *>(clo + off) : make_uint4(0, 0, 0, 0);
+        }
+      };
+      int cc = half * NCH;
+      uint4 ch[4], cl[4];
+      if (needc && live(cc)) load_c(cc, ch, cl);
+      if (!mbar_wait(tfull_bar(buf), tph, limit)) {
+        set_status(p.status, kTimeoutBit);
+        break;
+      }
+      tc_fence_after();
+#pragma unroll 1
+      for (; live(cc); ++cc) {
+        const int col0 = t.n0 + cc * 32;
+        const int ca = col0 >> 6;
+        uint4 nh[4], nl[4];
+        if (needc && live(cc + 1)) load_c(cc + 1, nh, nl);
+        uint32_t r[32];
+        tmem_ld32(tmem_base + (uint32_t)(buf * BN + cc * 32) + ((uint32_t)(quarter * 32) << 16), r);
+        tmem_ld_wait();
+        float v[32];
+        if (p.mode == kGramF32) {
+          float *drow = reinterpret_cast<float *>(dbase) + i * q.d_ph;
+#pragma unroll
+          for (int g = 0; g < 8; ++g)
+            *reinterpret_cast<float4 *>(drow + col0 + 4 * g) =
+                make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]), __uint_as_float(r[4 * g + 2]),
+                            __uint_as_float(r[4 * g + 3]));
+          if (ca < ra) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              reinterpret_cast<float *>(dbase)[(int64_t)(col0 + e) * q.d_ph + i] = __uint_as_float(r[e]);
+          }
+          continue;
+        }
+        if (p.mode == kGram) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = s2 * __uint_as_float(r[e]);
+        } else {
+          const float kc = (p.mode == kPoly) ? p.cb : p.ca;
+          const float ka = (p.mode == kPoly) ? p.cc : 1.0f;
+          const float ks = (p.mode == kPoly) ? 1.0f : s;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const uint32_t hw[4] = {ch[g].x, ch[g].y, ch[g].z, ch[g].w};
+            const uint32_t lw[4] = {cl[g].x, cl[g].y, cl[g].z, cl[g].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float c0 = bf16lo(hw[h]) + bf16lo(lw[h]);
+              const float c1 = bf16hi(hw[h]) + bf16hi(lw[h]);
+              v[8 * g + 2 * h] = ks * fmaf(kc, c0, ka * __uint_as_float(r[8 * g + 2 * h]));
+              v[8 * g + 2 * h + 1] = ks * fmaf(kc, c1, ka * __uint_as_float(r[8 * g + 2 * h + 1]));
+            }
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint4 o;
+          o.x = pack_bf16(v[8 * g + 0], v[8 * g + 1]);
+          o.y = pack_bf16(v[8 * g + 2], v[8 * g + 3]);
+          o.z = pack_bf16(v[8 * g + 4], v[8 * g + 5]);
+          o.w = pack_bf16(v[8 * g + 6], v[8 * g + 7]);
+          const size_t off = panel_chunk_off(i, col0 + 8 * g, q.d_ph);
+          *reinterpret_cast<uint4 *>(dbase + off) = o;
+          if (dlo) {
+            uint4 l;
+            l.x = pack_bf16(v[8 * g + 0] - bf16lo(o.x), v[8 * g + 1] - bf16hi(o.x));
+            l.y = pack_bf16(v[8 * g + 2] - bf16lo(o.y), v[8 * g + 3] - bf16hi(o.y));
+            l.z = pack_bf16(v[8 * g + 4] - bf16lo(o.z), v[8 * g + 5] - bf16hi(o.z));
+            l.w = pack_bf16(v[8 * g + 6] - bf16lo(o.w), v[8 * g + 7] - bf16hi(o.w));
+            *reinterpret_cast<uint4 *>(dlo + off) = l;
+          }
+        }
+        if (sym && ca < ra) {
+          const int64_t ib = i & ~7LL;
+          const int ie = (int)(i & 7);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            __nv_bfloat16 h = __float2bfloat16_rn(v[e]);
+            *reinterpret_cast<__nv_bfloat16 *>(dbase + panel_chunk_off(col0 + e, ib, q.d_ph) + 2 * ie) = h;
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          ch[g] = nh[g];
+          cl[g] = nl[g];
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) remote_arrive(mapa(tempty_bar(buf), 0));   // the leader's barrier
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();                                  // no CTA leaves while its partner may still
+                                                   // read its shared memory or signal it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc2(tmem_base, TMEM_COLS);
+  }
+}
+
+std::mutex g_tmap_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+}  // namespace
+
+cudaError_t encode_ws_tensor_map(CUtensorMap *map, void *ws, size_t bytes) {
+  {
+    std::lock_guard<std::mutex> g(g_tmap_mu);
+    if (!g_encode) {
+      void *fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+      if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return e != cudaSuccess ? e : cudaErrorNotSupported;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  const cuuint64_t dims[2] = {64, (cuuint64_t)(bytes / 128)};
+  const cuuint64_t strides[1] = {128};
+  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gemm_tc2(const GemmParams &p, int num_sms, cudaStream_t s) {
+  static unsigned done_mask = 0;  // the attribute is set once per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(done_mask & (1u << (dev & 31)))) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    done_mask |= 1u << (dev & 31);
+  }
+  if (p.total_tiles <= 0) return cudaSuccess;
+  // Pairs that can be resident at once (a GPC with an odd number of free SMs leaves one
+  // idle), so that the persistent grid never spills into a second wave.
+  static int max_pairs[32] = {0};
+  int &mp = max_pairs[dev & 31];
+  if (!mp) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc2_kernel, &cfg) != cudaSuccess || n <= 0) {
+      (void)cudaGetLastError();
+      n = num_sms / 2;
+    }
+    mp = n < num_sms / 2 ? n : num_sms / 2;
+  }
+  const int clusters = p.total_tiles < mp ? p.total_tiles : mp;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc2_kernel, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace nshb

@@ -3,6 +3,7 @@
 // tens of KB, allowed on sm_70+ since CUDA 12.1), so a step needs no host->device
 // copies and the whole launch sequence can be captured in a CUDA graph.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -116,6 +117,8 @@ struct GemmProb {
 };
 enum GemmMode { kGram = 0, kPoly = 1, kUpdate = 2, kPlain = 3, kSub = 4, kGramF32 = 5 };
 struct GemmParams {
+  CUtensorMap tmap;       // 2-SM kernel: the workspace seen as rows of 128 bytes (64 bf16),
+                          // 64-row boxes, no swizzle (the data is stored pre-swizzled)
   char *ws;
   const float *scales;
   uint32_t *status;
@@ -177,6 +180,10 @@ cudaError_t launch_exact_norm(const ApplyParams &p, cudaStream_t s);
 cudaError_t launch_apply_finalize(const ApplyFinParams &p, cudaStream_t s);
 cudaError_t launch_apply(const ApplyParams &p, cudaStream_t s);
 cudaError_t launch_gemm_tc(const GemmParams &p, int bn, int num_sms, cudaStream_t s);
+// 2-SM (CTA pair) form: 256 x 256 tiles, tcgen05.mma.cta_group::2; p.tmap must be encoded.
+cudaError_t launch_gemm_tc2(const GemmParams &p, int num_sms, cudaStream_t s);
+// Encodes p.tmap for a workspace of `bytes` bytes at `ws` (host; driver entry point).
+cudaError_t encode_ws_tensor_map(CUtensorMap *map, void *ws, size_t bytes);
 cudaError_t launch_gemm_f32(const F32Params &p, cudaStream_t s);
 cudaError_t launch_pack_panels(const PackParams &p, cudaStream_t s);
 cudaError_t launch_ridge(const CholParams &p, cudaStream_t s);
