@@ -218,6 +218,10 @@ const char *nshb_status_string(int32_t status);
 nshb_status nshb_profile_enable(int32_t on);
 nshb_status nshb_profile_read(int32_t n_kinds, float *ms, int32_t *launches);
 
+/* The cudaError_t value behind the last NSHB_ERR_CUDA returned to this host thread
+ * (0 if none): a diagnostic for failed launches or runtime calls. */
+int32_t nshb_last_cuda_error(void);
+
 /* ABI version (major * 10000 + minor * 100 + patch). */
 int32_t nshb_version(void);
 

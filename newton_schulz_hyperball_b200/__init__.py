@@ -37,7 +37,10 @@ def lib() -> ctypes.CDLL:
 class NshbError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {lib().nshb_status_string(status).decode()}")
+        msg = f"{where}: {lib().nshb_status_string(status).decode()}"
+        if status == NSHB_ERR_CUDA:
+            msg += f" (cudaError {lib().nshb_last_cuda_error()})"
+        super().__init__(msg)
 
 
 def _check(status: int, where: str) -> None:

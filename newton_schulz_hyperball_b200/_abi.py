@@ -97,6 +97,7 @@ SIGNATURES = {
     "nshb_device_status": (ctypes.c_int32, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "nshb_status_string": (ctypes.c_char_p, [ctypes.c_int32]),
     "nshb_version": (ctypes.c_int32, []),
+    "nshb_last_cuda_error": (ctypes.c_int32, []),
     "nshb_profile_enable": (ctypes.c_int32, [ctypes.c_int32]),
     "nshb_profile_read": (ctypes.c_int32, [ctypes.c_int32, ctypes.POINTER(ctypes.c_float),
                                            ctypes.POINTER(ctypes.c_int32)]),

@@ -281,9 +281,13 @@ int device_sms() {
   return cache[dev];
 }
 
+thread_local int g_last_cuda_error = 0;   // last CUDA error seen by this thread's calls
+
 #define NSHB_CHECK_CUDA(x)                 \
   do {                                     \
-    if ((x) != cudaSuccess) {              \
+    cudaError_t e_ = (x);                  \
+    if (e_ != cudaSuccess) {               \
+      g_last_cuda_error = (int)e_;         \
       (void)cudaGetLastError();            \
       return NSHB_ERR_CUDA;                \
     }                                      \
@@ -977,6 +981,8 @@ nshb_status nshb_profile_read(int32_t n_kinds, float *ms, int32_t *launches) {
   p.recs.clear();
   return st;
 }
+
+int32_t nshb_last_cuda_error(void) { return g_last_cuda_error; }
 
 int32_t nshb_version(void) { return 100; }
 

@@ -40,7 +40,8 @@ constexpr int HALF_BYTES = 2 * SLICE_BYTES;       // one operand half: two 64-de
 constexpr int STAGE_BYTES = 2 * HALF_BYTES;       // A half + B half of one CTA (64 KB)
 constexpr int TMEM_COLS = 2 * BN;                 // two 128 x 256 fp32 accumulators
 constexpr int kEpiWarpsSmem = 8;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256 + kEpiWarpsSmem * 4096;   // + epilogue staging
+// [alignment slack <= 1 KB][operand stages][barriers, TMEM slot: 256 B][epilogue staging]
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256 + kEpiWarpsSmem * 4096;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTimeoutBit = 0x4u;
@@ -143,7 +144,7 @@ __device__ __forceinline__ Tile decode2(const GemmParams &p, int tile) {
   return t;
 }
 
-__global__ void __maxnreg__(200) gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
@@ -289,7 +290,7 @@ __global__ void __maxnreg__(200) gemm_tc2_kernel(const __grid_constant__ GemmPar
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
     const int ew = warp - 2;
-    uint8_t *stg = smem + STAGES * STAGE_BYTES + 1024 + 256 + ew * 4096;   // 4 KB, 1 KB aligned
+    uint8_t *stg = smem + STAGES * STAGE_BYTES + 256 + ew * 4096;   // 4 KB after the barriers
     const uint32_t stg_s = smem_u32(stg);
     const bool sym = sym_mode(p.mode);
     const bool needc = (p.mode == kPoly || p.mode == kUpdate);
@@ -319,13 +320,7 @@ __global__ void __maxnreg__(200) gemm_tc2_kernel(const __grid_constant__ GemmPar
         const int ca = c0 >> 6;
         if (sym && ca > ra) continue;                            // above the diagonal: mirrored
         const int tcol = half * 128 + pp * 64;                   // column inside the tile
-        uint32_t r0[32], r1[32];
-        {
-          const uint32_t ta = tmem_base + (uint32_t)(buf * BN + tcol) + ((uint32_t)(quarter * 32) << 16);
-          tmem_ld32(ta, r0);
-          tmem_ld32(ta + 32, r1);
-        }
-#define RACC(e) ((e) < 32 ? r0[(e)] : r1[(e) - 32])
+        const uint32_t ta = tmem_base + (uint32_t)(buf * BN + tcol) + ((uint32_t)(quarter * 32) << 16);
         // the panel block of rows rb..rb+31 as stored: 4 KB contiguous
         const size_t blk = panel_chunk_off(rb, c0, q.d_ph);     // (rb & 7) == 0: chunk 0 of row rb
         float cv[64];
@@ -362,34 +357,47 @@ __global__ void __maxnreg__(200) gemm_tc2_kernel(const __grid_constant__ GemmPar
             __syncwarp();
           }
         }
-        tmem_ld_wait();
         if (p.mode == kGramF32) {
           // fp32 row-major output (row stride d_ph) for the Newton-Muon Gram S = Z Z^T.
-          float *drow = reinterpret_cast<float *>(dbase) + i * q.d_ph;
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            uint32_t r[32];
+            tmem_ld32(ta + 32 * h, r);
+            tmem_ld_wait();
+            float *drow = reinterpret_cast<float *>(dbase) + i * q.d_ph + c0 + 32 * h;
 #pragma unroll
-          for (int g = 0; g < 16; ++g)
-            *reinterpret_cast<float4 *>(drow + c0 + 4 * g) =
-                make_float4(__uint_as_float(RACC(4 * g)), __uint_as_float(RACC(4 * g + 1)),
-                            __uint_as_float(RACC(4 * g + 2)), __uint_as_float(RACC(4 * g + 3)));
-          if (ca < ra) {
+            for (int g = 0; g < 8; ++g)
+              *reinterpret_cast<float4 *>(drow + 4 * g) =
+                  make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]), __uint_as_float(r[4 * g + 2]),
+                              __uint_as_float(r[4 * g + 3]));
+            if (ca < ra) {
 #pragma unroll
-            for (int e = 0; e < 64; ++e)
-              reinterpret_cast<float *>(dbase)[(int64_t)(c0 + e) * q.d_ph + i] = __uint_as_float(RACC(e));
+              for (int e = 0; e < 32; ++e)
+                reinterpret_cast<float *>(dbase)[(int64_t)(c0 + 32 * h + e) * q.d_ph + i] = __uint_as_float(r[e]);
+            }
           }
           continue;
         }
-        // v = the phase epilogue, computed in place over cv
+        // v = the phase epilogue, computed in place over cv, 32 accumulator columns at a time
         float *v = cv;
-        if (p.mode == kGram) {
-#pragma unroll
-          for (int e = 0; e < 64; ++e) v[e] = s2 * __uint_as_float(RACC(e));
-        } else {
+        {
           const float kc = (p.mode == kPoly) ? p.cb : p.ca;
           const float ka = (p.mode == kPoly) ? p.cc : 1.0f;
           const float ks = (p.mode == kPoly) ? 1.0f : s;
 #pragma unroll
-          for (int e = 0; e < 64; ++e) v[e] = ks * fmaf(kc, cv[e], ka * __uint_as_float(RACC(e)));
-#undef RACC
+          for (int h = 0; h < 2; ++h) {
+            uint32_t r[32];
+            tmem_ld32(ta + 32 * h, r);
+            tmem_ld_wait();
+            if (p.mode == kGram) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[32 * h + e] = s2 * __uint_as_float(r[e]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                v[32 * h + e] = ks * fmaf(kc, cv[32 * h + e], ka * __uint_as_float(r[e]));
+            }
+          }
         }
         // hi part: each lane writes its row (swizzled) into staging, then coalesced store
 #pragma unroll
