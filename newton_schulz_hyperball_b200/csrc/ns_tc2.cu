@@ -39,9 +39,7 @@ constexpr int SLICE_BYTES = 128 * 64 * 2;         // 16 KB: 128 rows x 64 bf16 (
 constexpr int HALF_BYTES = 2 * SLICE_BYTES;       // one operand half: two 64-deep k panels
 constexpr int STAGE_BYTES = 2 * HALF_BYTES;       // A half + B half of one CTA (64 KB)
 constexpr int TMEM_COLS = 2 * BN;                 // two 128 x 256 fp32 accumulators
-constexpr int kEpiWarpsSmem = 8;
-// [alignment slack <= 1 KB][operand stages][barriers, TMEM slot: 256 B][epilogue staging]
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256 + kEpiWarpsSmem * 4096;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTimeoutBit = 0x4u;
@@ -282,18 +280,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
     }
   } else {
     // -------------------------------------------------------------- epilogue (both CTAs)
-    // Warp w drains TMEM lane quarter (w % 4) -- 32 rows of this CTA -- over one half of
-    // the tile's columns.  Phases that read C (polynomial, update) load each thread's row
-    // directly, one 32-column chunk ahead, so the load latency hides behind the math.
-    // Store-only phases (Gram) go through a 4 KB per-warp staging buffer so that every
-    // store moves whole 128-byte rows (the panel image of 32 rows x 64 columns is one
-    // contiguous, pre-swizzled 4 KB block).  Mirrored (transposed) blocks of the symmetric
-    // phases are transposed in the staging buffer and stored as 64-byte row segments.
+    constexpr int NCH = BN / 64;                  // 32-column chunks per warp (half the tile)
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
-    const int ew = warp - 2;
-    uint8_t *stg = smem + STAGES * STAGE_BYTES + 256 + ew * 4096;   // 4 KB after the barriers
-    const uint32_t stg_s = smem_u32(stg);
+    const int row = 128 * (int)rank + quarter * 32 + lane;   // row of the 256-row tile
     const bool sym = sym_mode(p.mode);
     const bool needc = (p.mode == kPoly || p.mode == kUpdate);
     int tl = 0;
@@ -308,250 +298,102 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
       char *dbase = p.ws + q.d_off + (int64_t)t.batch * q.d_bs;
       const char *clo = q.c_lo >= 0 ? p.ws + q.c_lo + (int64_t)t.batch * q.c_bs : nullptr;
       char *dlo = q.d_lo >= 0 ? p.ws + q.d_lo + (int64_t)t.batch * q.d_bs : nullptr;
-      const int64_t rb = t.m0 + 128 * (int)rank + quarter * 32;   // first of this warp's 32 rows
-      const int64_t i = rb + lane;                                // this thread's row
-      const int ra = (int)(rb >> 6);
-      if (needc) {
-        // C-reading phases: direct row loads, fetched one chunk ahead
-        const int NCH = BN / 64;
-        int cc = half * NCH;
-        auto live = [&](int c) { return c < (half + 1) * NCH && !(sym && ((t.n0 + c * 32) >> 6) > ra); };
-        auto load_c = [&](int c, uint4 (&h)[4], uint4 (&l)[4]) {
+      const int64_t i = t.m0 + row;
+      const int ra = (int)(i >> 6);
+      const int cc_end = (half + 1) * NCH;
+      auto live = [&](int cc) { return cc < cc_end && !(sym && ((t.n0 + cc * 32) >> 6) > ra); };
+      auto load_c = [&](int cc, uint4 (&h)[4], uint4 (&l)[4]) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const size_t off = panel_chunk_off(i, t.n0 + cc * 32 + 8 * g, q.d_ph);
+          h[g] = *reinterpret_cast<const uint4 *>(cbase + off);
+          l[g] = clo ? *reinterpret_cast<const uint4 *>(clo + off) : make_uint4(0, 0, 0, 0);
+        }
+      };
+      int cc = half * NCH;
+      uint4 ch[4], cl[4];
+      if (needc && live(cc)) load_c(cc, ch, cl);
+      if (!mbar_wait(tfull_bar(buf), tph, limit)) {
+        set_status(p.status, kTimeoutBit);
+        break;
+      }
+      tc_fence_after();
+#pragma unroll 1
+      for (; live(cc); ++cc) {
+        const int col0 = t.n0 + cc * 32;
+        const int ca = col0 >> 6;
+        uint4 nh[4], nl[4];
+        if (needc && live(cc + 1)) load_c(cc + 1, nh, nl);
+        uint32_t r[32];
+        tmem_ld32(tmem_base + (uint32_t)(buf * BN + cc * 32) + ((uint32_t)(quarter * 32) << 16), r);
+        tmem_ld_wait();
+        float v[32];
+        if (p.mode == kGramF32) {
+          float *drow = reinterpret_cast<float *>(dbase) + i * q.d_ph;
+#pragma unroll
+          for (int g = 0; g < 8; ++g)
+            *reinterpret_cast<float4 *>(drow + col0 + 4 * g) =
+                make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]), __uint_as_float(r[4 * g + 2]),
+                            __uint_as_float(r[4 * g + 3]));
+          if (ca < ra) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              reinterpret_cast<float *>(dbase)[(int64_t)(col0 + e) * q.d_ph + i] = __uint_as_float(r[e]);
+          }
+          continue;
+        }
+        if (p.mode == kGram) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = s2 * __uint_as_float(r[e]);
+        } else {
+          const float kc = (p.mode == kPoly) ? p.cb : p.ca;
+          const float ka = (p.mode == kPoly) ? p.cc : 1.0f;
+          const float ks = (p.mode == kPoly) ? 1.0f : s;
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
-            const size_t off = panel_chunk_off(i, t.n0 + c * 32 + 8 * g, q.d_ph);
-            h[g] = *reinterpret_cast<const uint4 *>(cbase + off);
-            l[g] = clo ? *reinterpret_cast<const uint4 *>(clo + off) : make_uint4(0, 0, 0, 0);
-          }
-        };
-        uint4 ch[4], cl[4];
-        if (needc && live(cc)) load_c(cc, ch, cl);
-        if (!mbar_wait(tfull_bar(buf), tph, limit)) {
-          set_status(p.status, kTimeoutBit);
-          break;
-        }
-        tc_fence_after();
-  #pragma unroll 1
-        for (; live(cc); ++cc) {
-          const int col0 = t.n0 + cc * 32;
-          const int ca = col0 >> 6;
-          uint4 nh[4], nl[4];
-          if (needc && live(cc + 1)) load_c(cc + 1, nh, nl);
-          uint32_t r[32];
-          tmem_ld32(tmem_base + (uint32_t)(buf * BN + cc * 32) + ((uint32_t)(quarter * 32) << 16), r);
-          tmem_ld_wait();
-          float v[32];
-          if (p.mode == kGramF32) {
-            float *drow = reinterpret_cast<float *>(dbase) + i * q.d_ph;
+            const uint32_t hw[4] = {ch[g].x, ch[g].y, ch[g].z, ch[g].w};
+            const uint32_t lw[4] = {cl[g].x, cl[g].y, cl[g].z, cl[g].w};
 #pragma unroll
-            for (int g = 0; g < 8; ++g)
-              *reinterpret_cast<float4 *>(drow + col0 + 4 * g) =
-                  make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]), __uint_as_float(r[4 * g + 2]),
-                              __uint_as_float(r[4 * g + 3]));
-            if (ca < ra) {
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                reinterpret_cast<float *>(dbase)[(int64_t)(col0 + e) * q.d_ph + i] = __uint_as_float(r[e]);
+            for (int h = 0; h < 4; ++h) {
+              const float c0 = bf16lo(hw[h]) + bf16lo(lw[h]);
+              const float c1 = bf16hi(hw[h]) + bf16hi(lw[h]);
+              v[8 * g + 2 * h] = ks * fmaf(kc, c0, ka * __uint_as_float(r[8 * g + 2 * h]));
+              v[8 * g + 2 * h + 1] = ks * fmaf(kc, c1, ka * __uint_as_float(r[8 * g + 2 * h + 1]));
             }
-            continue;
-          }
-          if (p.mode == kGram) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = s2 * __uint_as_float(r[e]);
-          } else {
-            const float kc = (p.mode == kPoly) ? p.cb : p.ca;
-            const float ka = (p.mode == kPoly) ? p.cc : 1.0f;
-            const float ks = (p.mode == kPoly) ? 1.0f : s;
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              const uint32_t hw[4] = {ch[g].x, ch[g].y, ch[g].z, ch[g].w};
-              const uint32_t lw[4] = {cl[g].x, cl[g].y, cl[g].z, cl[g].w};
-#pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                const float c0 = bf16lo(hw[h]) + bf16lo(lw[h]);
-                const float c1 = bf16hi(hw[h]) + bf16hi(lw[h]);
-                v[8 * g + 2 * h] = ks * fmaf(kc, c0, ka * __uint_as_float(r[8 * g + 2 * h]));
-                v[8 * g + 2 * h + 1] = ks * fmaf(kc, c1, ka * __uint_as_float(r[8 * g + 2 * h + 1]));
-              }
-            }
-          }
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            uint4 o;
-            o.x = pack_bf16(v[8 * g + 0], v[8 * g + 1]);
-            o.y = pack_bf16(v[8 * g + 2], v[8 * g + 3]);
-            o.z = pack_bf16(v[8 * g + 4], v[8 * g + 5]);
-            o.w = pack_bf16(v[8 * g + 6], v[8 * g + 7]);
-            const size_t off = panel_chunk_off(i, col0 + 8 * g, q.d_ph);
-            *reinterpret_cast<uint4 *>(dbase + off) = o;
-            if (dlo) {
-              uint4 l;
-              l.x = pack_bf16(v[8 * g + 0] - bf16lo(o.x), v[8 * g + 1] - bf16hi(o.x));
-              l.y = pack_bf16(v[8 * g + 2] - bf16lo(o.y), v[8 * g + 3] - bf16hi(o.y));
-              l.z = pack_bf16(v[8 * g + 4] - bf16lo(o.z), v[8 * g + 5] - bf16hi(o.z));
-              l.w = pack_bf16(v[8 * g + 6] - bf16lo(o.w), v[8 * g + 7] - bf16hi(o.w));
-              *reinterpret_cast<uint4 *>(dlo + off) = l;
-            }
-          }
-          if (sym && ca < ra) {
-            // Mirror through the staging buffer: the 32 x 32 block (rows rb.., cols col0..)
-            // lands transposed at rows col0..col0+31, columns rb..rb+31 (64 bytes per row).
-            __nv_bfloat16 *T = reinterpret_cast<__nv_bfloat16 *>(stg);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) T[e * 32 + lane] = __float2bfloat16_rn(v[e]);
-            __syncwarp();
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int trow = k * 8 + (lane >> 2), qd = lane & 3;
-              const uint4 val = *reinterpret_cast<const uint4 *>(stg + trow * 64 + qd * 16);
-              *reinterpret_cast<uint4 *>(dbase + panel_chunk_off(col0 + trow, rb + 8 * qd, q.d_ph)) = val;
-            }
-            __syncwarp();
-          }
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            ch[g] = nh[g];
-            cl[g] = nl[g];
           }
         }
-
-      } else {
-        if (!mbar_wait(tfull_bar(buf), tph, limit)) {
-          set_status(p.status, kTimeoutBit);
-          break;
-        }
-        tc_fence_after();
-  #pragma unroll 1
-        for (int pp = 0; pp < 2; ++pp) {
-          const int c0 = t.n0 + half * 128 + pp * 64;              // first column of the panel
-          const int ca = c0 >> 6;
-          if (sym && ca > ra) continue;                            // above the diagonal: mirrored
-          const int tcol = half * 128 + pp * 64;                   // column inside the tile
-          const uint32_t ta = tmem_base + (uint32_t)(buf * BN + tcol) + ((uint32_t)(quarter * 32) << 16);
-          // the panel block of rows rb..rb+31 as stored: 4 KB contiguous
-          const size_t blk = panel_chunk_off(rb, c0, q.d_ph);     // (rb & 7) == 0: chunk 0 of row rb
-          float cv[64];
-          if (needc) {
-            // coalesced copy of the C block into the staging buffer, then each lane reads its row
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              *reinterpret_cast<uint4 *>(stg + k * 512 + lane * 16) =
-                  *reinterpret_cast<const uint4 *>(cbase + blk + k * 512 + lane * 16);
-            __syncwarp();
-#pragma unroll
-            for (int qd = 0; qd < 8; ++qd) {
-              const uint4 h = *reinterpret_cast<const uint4 *>(stg + lane * 128 + ((qd ^ (lane & 7)) << 4));
-              cv[8 * qd + 0] = bf16lo(h.x); cv[8 * qd + 1] = bf16hi(h.x);
-              cv[8 * qd + 2] = bf16lo(h.y); cv[8 * qd + 3] = bf16hi(h.y);
-              cv[8 * qd + 4] = bf16lo(h.z); cv[8 * qd + 5] = bf16hi(h.z);
-              cv[8 * qd + 6] = bf16lo(h.w); cv[8 * qd + 7] = bf16hi(h.w);
-            }
-            __syncwarp();
-            if (clo) {   // C carried as a hi + lo pair
-#pragma unroll
-              for (int k = 0; k < 8; ++k)
-                *reinterpret_cast<uint4 *>(stg + k * 512 + lane * 16) =
-                    *reinterpret_cast<const uint4 *>(clo + blk + k * 512 + lane * 16);
-              __syncwarp();
-#pragma unroll
-              for (int qd = 0; qd < 8; ++qd) {
-                const uint4 h = *reinterpret_cast<const uint4 *>(stg + lane * 128 + ((qd ^ (lane & 7)) << 4));
-                cv[8 * qd + 0] += bf16lo(h.x); cv[8 * qd + 1] += bf16hi(h.x);
-                cv[8 * qd + 2] += bf16lo(h.y); cv[8 * qd + 3] += bf16hi(h.y);
-                cv[8 * qd + 4] += bf16lo(h.z); cv[8 * qd + 5] += bf16hi(h.z);
-                cv[8 * qd + 6] += bf16lo(h.w); cv[8 * qd + 7] += bf16hi(h.w);
-              }
-              __syncwarp();
-            }
-          }
-          if (p.mode == kGramF32) {
-            // fp32 row-major output (row stride d_ph) for the Newton-Muon Gram S = Z Z^T.
-  #pragma unroll 1
-            for (int h = 0; h < 2; ++h) {
-              uint32_t r[32];
-              tmem_ld32(ta + 32 * h, r);
-              tmem_ld_wait();
-              float *drow = reinterpret_cast<float *>(dbase) + i * q.d_ph + c0 + 32 * h;
-#pragma unroll
-              for (int g = 0; g < 8; ++g)
-                *reinterpret_cast<float4 *>(drow + 4 * g) =
-                    make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]), __uint_as_float(r[4 * g + 2]),
-                                __uint_as_float(r[4 * g + 3]));
-              if (ca < ra) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                  reinterpret_cast<float *>(dbase)[(int64_t)(c0 + 32 * h + e) * q.d_ph + i] = __uint_as_float(r[e]);
-              }
-            }
-            continue;
-          }
-          // v = the phase epilogue, computed in place over cv, 32 accumulator columns at a time
-          float *v = cv;
-          {
-            const float kc = (p.mode == kPoly) ? p.cb : p.ca;
-            const float ka = (p.mode == kPoly) ? p.cc : 1.0f;
-            const float ks = (p.mode == kPoly) ? 1.0f : s;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              uint32_t r[32];
-              tmem_ld32(ta + 32 * h, r);
-              tmem_ld_wait();
-              if (p.mode == kGram) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) v[32 * h + e] = s2 * __uint_as_float(r[e]);
-              } else {
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                  v[32 * h + e] = ks * fmaf(kc, cv[32 * h + e], ka * __uint_as_float(r[e]));
-              }
-            }
-          }
-          // hi part: each lane writes its row (swizzled) into staging, then coalesced store
-#pragma unroll
-          for (int qd = 0; qd < 8; ++qd)
-            *reinterpret_cast<uint4 *>(stg + lane * 128 + ((qd ^ (lane & 7)) << 4)) =
-                make_uint4(pack_bf16(v[8 * qd + 0], v[8 * qd + 1]), pack_bf16(v[8 * qd + 2], v[8 * qd + 3]),
-                           pack_bf16(v[8 * qd + 4], v[8 * qd + 5]), pack_bf16(v[8 * qd + 6], v[8 * qd + 7]));
-          __syncwarp();
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            *reinterpret_cast<uint4 *>(dbase + blk + k * 512 + lane * 16) =
-                *reinterpret_cast<const uint4 *>(stg + k * 512 + lane * 16);
-          __syncwarp();
-          if (dlo) {   // rounding residual kept as a second bf16
-#pragma unroll
-            for (int qd = 0; qd < 8; ++qd) {
-              float w[8];
-#pragma unroll
-              for (int h = 0; h < 8; ++h) w[h] = v[8 * qd + h] - bf16_round(v[8 * qd + h]);
-              *reinterpret_cast<uint4 *>(stg + lane * 128 + ((qd ^ (lane & 7)) << 4)) =
-                  make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7]));
-            }
-            __syncwarp();
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              *reinterpret_cast<uint4 *>(dlo + blk + k * 512 + lane * 16) =
-                  *reinterpret_cast<const uint4 *>(stg + k * 512 + lane * 16);
-            __syncwarp();
-          }
-          if (sym && ca < ra) {
-            // Mirror: the 32 x 64 block (rows rb.., cols c0..) lands transposed at rows
-            // c0..c0+63, columns rb..rb+31 -- 64 bytes of each target row.  Transpose in
-            // staging ([64 rows][32 bf16]), then each target row is one 64-byte store group.
-            __nv_bfloat16 *T = reinterpret_cast<__nv_bfloat16 *>(stg);
-#pragma unroll
-            for (int e = 0; e < 64; ++e) T[e * 32 + lane] = __float2bfloat16_rn(v[e]);
-            __syncwarp();
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const int trow = k * 8 + (lane >> 2), qd = lane & 3;
-              const uint4 val = *reinterpret_cast<const uint4 *>(stg + trow * 64 + qd * 16);
-              *reinterpret_cast<uint4 *>(dbase + panel_chunk_off(c0 + trow, rb + 8 * qd, q.d_ph)) = val;
-            }
-            __syncwarp();
+        for (int g = 0; g < 4; ++g) {
+          uint4 o;
+          o.x = pack_bf16(v[8 * g + 0], v[8 * g + 1]);
+          o.y = pack_bf16(v[8 * g + 2], v[8 * g + 3]);
+          o.z = pack_bf16(v[8 * g + 4], v[8 * g + 5]);
+          o.w = pack_bf16(v[8 * g + 6], v[8 * g + 7]);
+          const size_t off = panel_chunk_off(i, col0 + 8 * g, q.d_ph);
+          *reinterpret_cast<uint4 *>(dbase + off) = o;
+          if (dlo) {
+            uint4 l;
+            l.x = pack_bf16(v[8 * g + 0] - bf16lo(o.x), v[8 * g + 1] - bf16hi(o.x));
+            l.y = pack_bf16(v[8 * g + 2] - bf16lo(o.y), v[8 * g + 3] - bf16hi(o.y));
+            l.z = pack_bf16(v[8 * g + 4] - bf16lo(o.z), v[8 * g + 5] - bf16hi(o.z));
+            l.w = pack_bf16(v[8 * g + 6] - bf16lo(o.w), v[8 * g + 7] - bf16hi(o.w));
+            *reinterpret_cast<uint4 *>(dlo + off) = l;
           }
         }
-
+        if (sym && ca < ra) {
+          const int64_t ib = i & ~7LL;
+          const int ie = (int)(i & 7);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            __nv_bfloat16 h = __float2bfloat16_rn(v[e]);
+            *reinterpret_cast<__nv_bfloat16 *>(dbase + panel_chunk_off(col0 + e, ib, q.d_ph) + 2 * ie) = h;
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          ch[g] = nh[g];
+          cl[g] = nl[g];
+        }
       }
       tc_fence_before();
       __syncwarp();
