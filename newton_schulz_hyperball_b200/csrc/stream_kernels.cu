@@ -200,8 +200,7 @@ __device__ __forceinline__ void load_x16(const char *xbase, const MatDesc &d, in
 
 // ------------------------------------------------------------------------- momentum
 __global__ void __launch_bounds__(kThreads) momentum_kernel(const __grid_constant__ MomentumParams p) {
-  __shared__ float sT[kBlk][kBlk + 1];
-  __shared__ float sL[kBlk][kBlk + 1];
+  __shared__ float sT[kBlk][kBlk + 1];   // transpose staging (tall matrices), hi then lo
   __shared__ double red[kThreads / 32];
   const int blk = blockIdx.x;
   const MatDesc &d = p.mats[find_mat(p, blk)];
@@ -251,20 +250,21 @@ __global__ void __launch_bounds__(kThreads) momentum_kernel(const __grid_constan
   char *xbase = p.ws + d.x_off;
   char *lbase = lo_part ? p.ws + d.xlo_off : nullptr;
   if (d.flags & kTall && !(d.flags & kTiled)) {
-    // X = U^T: stage the block and write it transposed.
+    // X = U^T: stage the block and write it transposed (hi, then lo through the same tile).
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      sT[rr][cg + e] = u[e];
-      sL[rr][cg + e] = ul[e];
-    }
+    for (int e = 0; e < 16; ++e) sT[rr][cg + e] = u[e];
     __syncthreads();
     float v[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) v[e] = sT[cg + e][rr];
     store_x16(xbase, d, c0 + rr, r0 + cg, v);
     if (lo_part) {
+      __syncthreads();
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = sL[cg + e][rr];
+      for (int e = 0; e < 16; ++e) sT[rr][cg + e] = ul[e];
+      __syncthreads();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v[e] = sT[cg + e][rr];
       store_x16(lbase, d, c0 + rr, r0 + cg, v);
     }
   } else {
@@ -296,6 +296,24 @@ __global__ void norm_finalize_kernel(const __grid_constant__ NormFinParams p, in
     p.nus[warp] = s;
     p.scales[warp] = (float)(1.0 / (sqrt(s) + (double)p.ns_eps));
   }
+}
+
+// This thread's 16 O values of W row r0 + t/4, columns c0 + 16 (t%4) .. +15.  Matrices
+// whose NS ran on the transpose go through the shared tile sO; the others read their
+// 16 values straight from the panel layout (two 16-byte chunks, no block barrier).
+__device__ __forceinline__ void load_o_block(const ApplyParams &p, const MatDesc &d, int r0, int c0,
+                                             float (&sO)[kBlk][kBlk + 1]);
+__device__ __forceinline__ void load_o16(const ApplyParams &p, const MatDesc &d, int r0, int c0,
+                                         float (&sO)[kBlk][kBlk + 1], float (&o)[16]) {
+  const int t = threadIdx.x, rr = t >> 2, cg = (t & 3) * 16;
+  const bool tr = (d.flags & kTall) && !(d.flags & kTiled);
+  if (!tr) {
+    load_x16(p.ws + d.o_off, d, r0 + rr, c0 + cg, o);
+    return;
+  }
+  load_o_block(p, d, r0, c0, sO);
+#pragma unroll
+  for (int e = 0; e < 16; ++e) o[e] = sO[rr][cg + e];
 }
 
 // Loads the O block of W block (r0, c0) into sO[w_row][w_col] (zero outside W).
@@ -331,10 +349,11 @@ __global__ void __launch_bounds__(kThreads) reduce_kernel(const __grid_constant_
   load16(d.W, d.ld, i, j, d.m, d.n, d.flags & kWF32, d.flags & kVec, w);
   float om = 0.f, de = 0.f, pi = 0.f;
   if (p.op != kOpNorms) {
-    load_o_block(p, d, r0, c0, sO);
+    float ov[16];
+    load_o16(p, d, r0, c0, sO, ov);
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-      const float o = (i < d.m && j + e < d.n) ? sO[rr][cg + e] : 0.f;
+      const float o = (i < d.m && j + e < d.n) ? ov[e] : 0.f;
       om = fmaf(o, o, om);
       de = fmaf(w[e], o, de);
     }
@@ -368,11 +387,12 @@ __global__ void __launch_bounds__(kThreads) exact_norm_kernel(const __grid_const
       const int i = r0 + rr, j = c0 + cg;
       float w[16];
       load16(d.W, d.ld, i, j, d.m, d.n, d.flags & kWF32, d.flags & kVec, w);
-      load_o_block(p, d, r0, c0, sO);
+      float ov[16];
+      load_o16(p, d, r0, c0, sO, ov);
       float acc = 0.f;
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        const float o = (i < d.m && j + e < d.n) ? sO[rr][cg + e] : 0.f;
+        const float o = (i < d.m && j + e < d.n) ? ov[e] : 0.f;
         const float v = fmaf(-tt, o, w[e]);
         acc = fmaf(v, v, acc);
       }
@@ -508,10 +528,8 @@ __global__ void __launch_bounds__(kThreads) apply_kernel(const __grid_constant__
   const int t = threadIdx.x, rr = t >> 2, cg = (t & 3) * 16;
   const int i = r0 + rr, j = c0 + cg;
   const bool f32 = d.flags & kWF32, vec = d.flags & kVec;
-  load_o_block(p, d, r0, c0, sO);
   float o[16];
-#pragma unroll
-  for (int e = 0; e < 16; ++e) o[e] = sO[rr][cg + e];
+  load_o16(p, d, r0, c0, sO, o);
   if (d.O_out) {
     const bool vo = ((uintptr_t)d.O_out % 16 == 0) && (d.n % (f32 ? 4 : 8) == 0);
     store16(d.O_out, d.n, i, j, d.m, d.n, f32, vo, o);
