@@ -35,6 +35,20 @@ WORKLOAD = "gpt2-small matrix set, MuonH step (72 bf16 matrices, fp32 momentum, 
 ETA = 0.02
 N_GRAD_SETS = 4
 DEFAULT_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM read + write per launch of the NS GEMM from the ncu capture summarised in
+# profiles/gemm_tc2_gpt2_small_ns_iteration1.md, valid only for the kernel source it was taken on.
+GEMM_SOURCE = os.path.join(ROOT, "newton_schulz_hyperball_b200", "csrc", "ns_tc2.cu")
+GEMM_TRAFFIC = {"sha256_prefix": "704a1a72938141d3", "bytes_per_launch": 368434517}
+
+
+def gemm_traffic():
+    import hashlib
+    try:
+        with open(GEMM_SOURCE, "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return GEMM_TRAFFIC["bytes_per_launch"] if h == GEMM_TRAFFIC["sha256_prefix"] else None
 
 
 def shapes():
@@ -372,11 +386,13 @@ def main():
         "ns_frac_of_bf16_peak": None if ns_tflops is None else round(ns_tflops / peak_tf, 4),
         "fused_gbs": None if fused_gbs is None else round(fused_gbs, 1),
         "fused_frac_of_hbm": None if fused_gbs is None else round(fused_gbs / peak_bw, 4),
-        "roofline": {"bound": "tensor", "kernel": "gemm_tc_kernel (NS Gram/poly/update)",
+        "roofline": {"bound": "tensor", "kernel": "gemm_tc2_kernel (NS Gram / polynomial / update, CTA pairs)",
                      "achieved": None if ns_tflops is None else round(ns_tflops, 1),
                      "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": None if ns_tflops is None else round(ns_tflops / peak_tf, 4),
-                     "traffic": None, "peak_source": f"{peak_src} bf16 burst",
+                     "traffic": gemm_traffic(),
+                     "peak_source": f"{peak_src} bf16 burst (sustained {peaks.get('bf16_tflops_sustained')})",
+                     "flops_per_launch": round(flops / max(gemm_launches, 1)),
                      "per_launch_ms": round(gemm_ms / max(gemm_launches, 1), 5)},
         "kernels_ms_per_step": {k: round(v[0] / kp, 5) for k, v in prof.items()},
         "momentum_gbs": None if mom_gbs is None else round(mom_gbs, 1),
