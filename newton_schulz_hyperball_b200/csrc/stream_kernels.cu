@@ -199,108 +199,6 @@ __device__ __forceinline__ void load_x16(const char *xbase, const MatDesc &d, in
 }
 
 // ------------------------------------------------------------------------- momentum
-// Common case: bf16 G, aligned rows, bf16 panel output, the whole 16-element segment
-// inside the matrix.  The loaded data stays packed and is consumed 8 elements at a time,
-// which keeps the register count low enough for six resident blocks per SM (the kernel
-// is bound by how many loads are in flight).  Returns this thread's ||U||^2 share.
-__device__ __forceinline__ float momentum_fast(const MomentumParams &p, const MatDesc &d, int r0, int c0,
-                                               __nv_bfloat16 (&tH)[kBlk][kBlk + 8],
-                                               __nv_bfloat16 (&tL)[kBlk][kBlk + 8]) {
-  const int t = threadIdx.x, rr = t >> 2, cg = (t & 3) * 16;
-  const int i = r0 + rr, j = c0 + cg;
-  const bool lo_part = d.xlo_off >= 0;
-  const bool tall = (d.flags & kTall) && !(d.flags & kTiled);
-  const __nv_bfloat16 *grow = static_cast<const __nv_bfloat16 *>(d.G) + (int64_t)i * d.ld + j;
-  float *mrow = d.M + (int64_t)i * d.ld + j;
-  const uint4 g0 = *reinterpret_cast<const uint4 *>(grow);
-  const uint4 g1 = *reinterpret_cast<const uint4 *>(grow + 8);
-  float4 m4[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) m4[q] = *reinterpret_cast<const float4 *>(mrow + 4 * q);
-  const float beta = p.beta, omb = 1.0f - p.beta;
-  char *xbase = p.ws + d.x_off;
-  char *lbase = lo_part ? p.ws + d.xlo_off : nullptr;
-  float acc = 0.f;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const uint4 gw = h ? g1 : g0;
-    const uint32_t gv[4] = {gw.x, gw.y, gw.z, gw.w};
-    float mv[8] = {m4[2 * h].x, m4[2 * h].y, m4[2 * h].z, m4[2 * h].w,
-                   m4[2 * h + 1].x, m4[2 * h + 1].y, m4[2 * h + 1].z, m4[2 * h + 1].w};
-    uint32_t hi[4], lo[4];
-#pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      const float ga = bf16lo(gv[e / 2]), gb = bf16hi(gv[e / 2]);
-      const float ma = fmaf(beta, mv[e], omb * ga), mb = fmaf(beta, mv[e + 1], omb * gb);
-      mv[e] = ma;
-      mv[e + 1] = mb;
-      const float ua = p.nesterov ? fmaf(omb, ga, beta * ma) : ma;
-      const float ub = p.nesterov ? fmaf(omb, gb, beta * mb) : mb;
-      hi[e / 2] = pack_bf16(ua, ub);
-      const float ha = bf16lo(hi[e / 2]), hb = bf16hi(hi[e / 2]);
-      lo[e / 2] = pack_bf16(ua - ha, ub - hb);
-      const float na = lo_part ? ua : ha, nb = lo_part ? ub : hb;
-      acc = fmaf(na, na, fmaf(nb, nb, acc));
-    }
-    *reinterpret_cast<float4 *>(mrow + 8 * h) = make_float4(mv[0], mv[1], mv[2], mv[3]);
-    *reinterpret_cast<float4 *>(mrow + 8 * h + 4) = make_float4(mv[4], mv[5], mv[6], mv[7]);
-    if (!tall) {
-      const int xr = i, xc = j + 8 * h;
-      char *hb = xbase;
-      char *lb = lbase;
-      int lr = xr, lc = xc;
-      if (d.flags & kTiled) {
-        hb = tile_base(xbase, d, xr, xc);
-        if (lbase) lb = tile_base(lbase, d, xr, xc);
-        lr = xr % d.ph;
-        lc = xc % d.ph;
-      }
-      const size_t off = panel_chunk_off(lr, lc, d.ph);
-      *reinterpret_cast<uint4 *>(hb + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      if (lb) *reinterpret_cast<uint4 *>(lb + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        *reinterpret_cast<uint32_t *>(&tH[rr][cg + 8 * h + 2 * e]) = hi[e];
-        *reinterpret_cast<uint32_t *>(&tL[rr][cg + 8 * h + 2 * e]) = lo[e];
-      }
-    }
-  }
-  if (tall) {
-    // X = U^T: write the block transposed; thread (rr, cg) now owns X row c0 + rr.
-    __syncthreads();
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint32_t hv[4], lv[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int a = cg + 8 * h + 2 * e;
-        hv[e] = (uint32_t)__bfloat16_as_ushort(tH[a][rr]) | ((uint32_t)__bfloat16_as_ushort(tH[a + 1][rr]) << 16);
-        lv[e] = (uint32_t)__bfloat16_as_ushort(tL[a][rr]) | ((uint32_t)__bfloat16_as_ushort(tL[a + 1][rr]) << 16);
-      }
-      const size_t off = panel_chunk_off(c0 + rr, r0 + cg + 8 * h, d.ph);
-      *reinterpret_cast<uint4 *>(xbase + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-      if (lbase) *reinterpret_cast<uint4 *>(lbase + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
-    }
-  }
-  return acc;
-}
-
-// Launched when every matrix of the launch takes the common case (the host checks: bf16
-// G and W, aligned rows, bf16 NS operands, no padding blocks in the launch's domain).
-__global__ void __launch_bounds__(kThreads, 6) momentum_fast_kernel(const __grid_constant__ MomentumParams p) {
-  __shared__ __nv_bfloat16 tH[kBlk][kBlk + 8];
-  __shared__ __nv_bfloat16 tL[kBlk][kBlk + 8];
-  __shared__ double red[kThreads / 32];
-  const int blk = blockIdx.x;
-  const MatDesc &d = p.mats[find_mat(p, blk)];
-  int r0, c0;
-  block_origin(d, blk - d.blk_begin, r0, c0);
-  double s[1] = {(double)momentum_fast(p, d, r0, c0, tH, tL)};
-  block_sum<1>(s, red);
-  if (threadIdx.x == 0) p.partials[blk] = s[0];
-}
-
 __global__ void __launch_bounds__(kThreads) momentum_kernel(const __grid_constant__ MomentumParams p) {
   __shared__ float sT[kBlk][kBlk + 1];   // transpose staging (tall matrices), hi then lo
   __shared__ double red[kThreads / 32];
@@ -649,15 +547,7 @@ __global__ void __launch_bounds__(kThreads) apply_kernel(const __grid_constant__
 }  // namespace
 
 cudaError_t launch_momentum(const MomentumParams &p, cudaStream_t s) {
-  if (p.total_blocks <= 0) return cudaSuccess;
-  bool fast = true;
-  for (int k = 0; k < p.nmat && fast; ++k) {
-    const MatDesc &d = p.mats[k];
-    // the block domain must be the matrix itself (no zero-padding blocks to write)
-    fast = !(d.flags & (kWF32 | kNsF32 | kFromP | kURow)) && (d.flags & kVec) && d.pr == d.m && d.pc == d.n;
-  }
-  if (fast) momentum_fast_kernel<<<p.total_blocks, kThreads, 0, s>>>(p);
-  else momentum_kernel<<<p.total_blocks, kThreads, 0, s>>>(p);
+  if (p.total_blocks > 0) momentum_kernel<<<p.total_blocks, kThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_norm_finalize(const NormFinParams &p, int nseg_total, cudaStream_t s) {
