@@ -379,3 +379,106 @@ def test_bf16_newton_muon_small():
         assert rel_fro(Og[i], Or) <= 2e-2, (i, rel_fro(Og[i], Or))
         assert np.linalg.norm(Wg[i] - Wr) <= bf16_w_tol(Wr, 0.02)
         assert abs(o.fro(Wg[i]) - rhos[i]) / rhos[i] <= radius_tol(Wg[i], True)
+
+
+# ------------------------------------------------- determinism, schedules, graphs
+def test_steps_are_bit_deterministic():
+    """Fixed-order reductions, no float atomics: two runs on the same inputs agree bit for bit."""
+    cfg = 21
+    shapes = [(768, 768), (3072, 768), (768, 3072), (300, 700)]
+    Ws = [wl.init_weight(cfg, i, r, c, bf16=True).astype(np.float64) for i, (r, c) in enumerate(shapes)]
+    Gs = [wl.gradient(cfg, i, 0, r, c, bf16=True).astype(np.float64) for i, (r, c) in enumerate(shapes)]
+    outs = []
+    for _ in range(2):
+        gs = GpuSet(Ws, bf16=True)
+        gs.set_grads(Gs)
+        assert gs.step("hyperball", nshb.params(eta=0.02)) == 0
+        outs.append(gs.host())
+    for a, b in zip(outs[0], outs[1]):
+        for x, y in zip(a, b):
+            assert np.array_equal(x, y)
+
+
+def test_radial_brake_page_targets_on_gpu():
+    """PR #224 test targets 7.5 and 9.0 with exactly representable norms: ||w_prev|| = 5 and
+    a plain step to ||w|| = 10 (outward 0.5 -> 7.5); ||w_prev|| = 10 to ||w|| = 8
+    (inward 0.5 -> 9.0).  The update is forced through O by a rank-1 gradient whose NS
+    output is known: with K = 1 and (a, b, c) = (1, 0, 0), O = U / (||U|| + eps)."""
+    import json, pathlib
+    g = json.loads((pathlib.Path(__file__).parent / "golden" / "page_values.json").read_text())["radial_brake_targets"]
+    for w_prev, w_new, s_out, s_in, target in (([3.0, 4.0], [6.0, 8.0], 0.5, 1.0, g["outward_target"]),
+                                               ([6.0, 8.0], [4.8, 6.4], 1.0, 0.5, g["inward_target"])):
+        W = np.zeros((8, 8))
+        W[0, :2] = w_prev
+        D = np.zeros((8, 8))
+        D[0, :2] = np.array(w_prev) - np.array(w_new)        # W - lr * O = w_new  =>  lr * O = D
+        lr = float(np.linalg.norm(D))                       # O = D / ||D|| (unit), so lr = ||D||
+        gs = GpuSet([W], bf16=False)
+        gs.set_grads([D])                                   # beta = 0: U = G = D
+        p = nshb.params(ns_precision=nshb.NSHB_F32, beta=0.0, ns_steps=1, coeffs=[(1.0, 0.0, 0.0)],
+                        lr=lr, brake_out=s_out, brake_in=s_in, ns_eps=1e-30)
+        assert gs.step("brake", p) == 0
+        assert abs(np.linalg.norm(gs.host()[0][0]) - target) <= 1e-5 * target
+
+
+def test_momentum_closed_form_on_gpu():
+    """Constant G from M0 = 0: after t steps M_t = (1 - beta^t) G (fp32 buffer)."""
+    G = wl.gradient(22, 0, 0, 256, 512, bf16=True).astype(np.float64)
+    W = wl.init_weight(22, 0, 256, 512, bf16=True).astype(np.float64)
+    gs = GpuSet([W], bf16=True)
+    gs.set_grads([G])
+    beta = 0.9
+    for t in range(1, 6):
+        assert gs.step("muon", nshb.params(beta=beta, lr=0.0)) == 0
+        assert rel_fro(gs.host()[1][0], (1 - beta ** t) * G) <= 1e-6
+
+
+def test_per_iteration_coefficient_schedule():
+    """Per-iteration (a, b, c) rows (the two-stage schedule of the Muon explainer: Keller's
+    coefficients, then (2, -1.5, 0.5)) on the tensor-core path."""
+    cfg = 23
+    table = [o.KELLER_ABC] * 3 + [o.SETTLE_ABC] * 2
+    for shape in [(768, 768), (3072, 768)]:
+        W = wl.init_weight(cfg, 0, *shape, bf16=True).astype(np.float64)
+        G = wl.gradient(cfg, 0, 0, *shape, bf16=True).astype(np.float64)
+        gs = GpuSet([W], bf16=True)
+        gs.set_grads([G])
+        assert gs.step("muon", nshb.params(lr=0.0, coeffs=table)) == 0
+        _, U = o.momentum(np.zeros_like(G), G, 0.95, True)
+        assert rel_fro(gs.host()[2][0], o.newton_schulz(U, 5, coeffs=table)) <= 2e-2
+
+
+def test_step_captures_in_a_cuda_graph():
+    """The step enqueues only kernels and one memset on the caller's stream: it can be
+    captured once and replayed; the replay equals a direct call on the same inputs."""
+    cfg = 24
+    shapes = [(768, 768), (768, 3072), (3072, 768)]
+    Ws = [wl.init_weight(cfg, i, r, c, bf16=True).astype(np.float64) for i, (r, c) in enumerate(shapes)]
+    Gs = [wl.gradient(cfg, i, 0, r, c, bf16=True).astype(np.float64) for i, (r, c) in enumerate(shapes)]
+    direct = GpuSet(Ws, bf16=True)
+    direct.set_grads(Gs)
+    assert direct.step("hyperball", nshb.params(eta=0.02)) == 0
+    graphed = GpuSet(Ws, bf16=True)
+    graphed.set_grads(Gs)
+    p = nshb.params(eta=0.02)
+    need = nshb.workspace_size(graphed.mats, p, nshb.NSHB_OP_HYPERBALL)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    nshb.hyperball_step(graphed.mats, p, ws)        # first call outside capture (module set-up)
+    torch.cuda.synchronize()
+    # reset state and capture
+    for w, w0 in zip(graphed.W, Ws):
+        w.copy_(torch.from_numpy(w0.astype(np.float32)).to("cuda").to(torch.bfloat16))
+    for m in graphed.M:
+        m.zero_()
+    s = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            nshb.hyperball_step(graphed.mats, p, ws, s)
+    # capture does not execute: the state is still initial; replay runs the step once
+    graph.replay()
+    torch.cuda.synchronize()
+    assert nshb.device_status(ws) == 0
+    for a, b in zip(direct.host(), graphed.host()):
+        for x, y in zip(a, b):
+            assert np.array_equal(x, y)
