@@ -14,8 +14,14 @@
 //                    closed form cancels (an update that nearly equals W).
 //  apply_kernel      W <- alpha W + beta O, one read of W and O, one write of W.
 //
-// Every kernel works on 64x64 blocks with 256 threads: thread t owns row t/4 and the 16
-// columns 16*(t%4) .. +15 of its block.  Reductions use fixed-order trees in fp64.
+// The work unit is a 64x64 block; thread t of 256 owns the 8 consecutive columns
+// 8 (t%8) .. +7 of the block rows t/8 and t/8 + 32, so one warp access covers four whole
+// 128-byte bf16 row segments (or four 128-byte panel rows of X).  The streaming kernels
+// are persistent: a grid of (SMs x resident CTAs) walks the block list with a stride of
+// the grid size, and every CTA issues the loads of its next block before it processes the
+// current one, so loads stay in flight through the block's arithmetic, its stores and its
+// reduction.  Partial sums are still one per block (fixed-order trees in fp64), so the
+// results do not depend on the grid size.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cmath>
@@ -27,6 +33,7 @@ namespace nshb {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
 
 template <typename P>
 __device__ __forceinline__ int find_mat(const P &p, int blk) {
@@ -36,6 +43,13 @@ __device__ __forceinline__ int find_mat(const P &p, int blk) {
     if (p.mats[mid].blk_begin <= blk) lo = mid; else hi = mid - 1;
   }
   return lo;
+}
+
+// The block list is walked in increasing order, so the owning matrix only moves forward.
+template <typename P>
+__device__ __forceinline__ int advance_mat(const P &p, int mi, int blk) {
+  while (mi + 1 < p.nmat && p.mats[mi + 1].blk_begin <= blk) ++mi;
+  return mi;
 }
 
 // Origin (W coordinates) of local block `lb` of a matrix.  Tiled matrices enumerate
@@ -54,227 +68,310 @@ __device__ __forceinline__ void block_origin(const MatDesc &d, int lb, int &r0, 
   }
 }
 
-// Load 16 consecutive W-or-G values of row i starting at column j (bounds-checked).
-__device__ __forceinline__ void load16(const void *base, int64_t ld, int i, int j, int m, int n, bool f32,
-                                       bool vec, float (&v)[16]) {
-  if (i >= m) {
+// Eight values of one row as loaded from memory: bf16 pairs in q[0..3], or fp32 bit
+// patterns in q[0..7].  Kept raw so that a prefetch does not wait for its data.
+struct Raw8 {
+  uint32_t q[8];
+};
+
+__device__ __forceinline__ void raw_zero(Raw8 &r) {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) v[e] = 0.f;
+  for (int e = 0; e < 8; ++e) r.q[e] = 0u;
+}
+
+// Row i, columns j..j+7 of a row-major bf16 or fp32 matrix (zero outside m x n).
+__device__ __forceinline__ void raw_load8(const void *base, int64_t ld, int i, int j, int m, int n, bool f32,
+                                          bool vec, Raw8 &r) {
+  if (i >= m || j >= n) {
+    raw_zero(r);
     return;
   }
   if (f32) {
-    const float *row = static_cast<const float *>(base) + (int64_t)i * ld;
-    if (vec && j + 15 < n) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float4 t = *reinterpret_cast<const float4 *>(row + j + 4 * q);
-        v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
-      }
+    const float *row = static_cast<const float *>(base) + (int64_t)i * ld + j;
+    if (vec && j + 7 < n) {
+      const uint4 a = *reinterpret_cast<const uint4 *>(row);
+      const uint4 b = *reinterpret_cast<const uint4 *>(row + 4);
+      r.q[0] = a.x; r.q[1] = a.y; r.q[2] = a.z; r.q[3] = a.w;
+      r.q[4] = b.x; r.q[5] = b.y; r.q[6] = b.z; r.q[7] = b.w;
     } else {
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = (j + e < n) ? row[j + e] : 0.f;
+      for (int e = 0; e < 8; ++e) r.q[e] = (j + e < n) ? __float_as_uint(row[e]) : 0u;
     }
   } else {
-    const __nv_bfloat16 *row = static_cast<const __nv_bfloat16 *>(base) + (int64_t)i * ld;
-    if (vec && j + 15 < n) {
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint4 t = *reinterpret_cast<const uint4 *>(row + j + 8 * q);
-        v[8 * q + 0] = bf16lo(t.x); v[8 * q + 1] = bf16hi(t.x);
-        v[8 * q + 2] = bf16lo(t.y); v[8 * q + 3] = bf16hi(t.y);
-        v[8 * q + 4] = bf16lo(t.z); v[8 * q + 5] = bf16hi(t.z);
-        v[8 * q + 6] = bf16lo(t.w); v[8 * q + 7] = bf16hi(t.w);
-      }
+    const unsigned short *row = static_cast<const unsigned short *>(base) + (int64_t)i * ld + j;
+    if (vec && j + 7 < n) {
+      const uint4 a = *reinterpret_cast<const uint4 *>(row);
+      r.q[0] = a.x; r.q[1] = a.y; r.q[2] = a.z; r.q[3] = a.w;
     } else {
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = (j + e < n) ? __bfloat162float(row[j + e]) : 0.f;
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t lo = (j + 2 * e < n) ? row[2 * e] : 0u;
+        const uint32_t hi = (j + 2 * e + 1 < n) ? row[2 * e + 1] : 0u;
+        r.q[e] = lo | (hi << 16);
+      }
     }
   }
 }
 
-__device__ __forceinline__ void store16(void *base, int64_t ld, int i, int j, int m, int n, bool f32, bool vec,
-                                        const float (&v)[16]) {
-  if (i >= m) return;
+__device__ __forceinline__ void raw_cvt8(const Raw8 &r, bool f32, float (&v)[8]) {
   if (f32) {
-    float *row = static_cast<float *>(base) + (int64_t)i * ld;
-    if (vec && j + 15 < n) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<float4 *>(row + j + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 16; ++e)
-        if (j + e < n) row[j + e] = v[e];
-    }
+    for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r.q[e]);
   } else {
-    __nv_bfloat16 *row = static_cast<__nv_bfloat16 *>(base) + (int64_t)i * ld;
-    if (vec && j + 15 < n) {
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint4 t;
-        t.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
-        t.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
-        t.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
-        t.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
-        *reinterpret_cast<uint4 *>(row + j + 8 * q) = t;
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 16; ++e)
-        if (j + e < n) row[j + e] = __float2bfloat16_rn(v[e]);
+    for (int e = 0; e < 4; ++e) {
+      v[2 * e] = bf16lo(r.q[e]);
+      v[2 * e + 1] = bf16hi(r.q[e]);
     }
   }
 }
 
-// Momentum buffer: always fp32.
-__device__ __forceinline__ void loadM(const float *M, int64_t ld, int i, int j, int m, int n, bool vec,
-                                      float (&v)[16]) {
-  load16(M, ld, i, j, m, n, true, vec, v);
+// Row i, columns j..j+7 of a row-major bf16 or fp32 matrix (bounds-checked).
+__device__ __forceinline__ void store8(void *base, int64_t ld, int i, int j, int m, int n, bool f32, bool vec,
+                                       const float (&v)[8]) {
+  if (i >= m || j >= n) return;
+  if (f32) {
+    float *row = static_cast<float *>(base) + (int64_t)i * ld + j;
+    if (vec && j + 7 < n) {
+      *reinterpret_cast<float4 *>(row) = make_float4(v[0], v[1], v[2], v[3]);
+      *reinterpret_cast<float4 *>(row + 4) = make_float4(v[4], v[5], v[6], v[7]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        if (j + e < n) row[e] = v[e];
+    }
+  } else {
+    __nv_bfloat16 *row = static_cast<__nv_bfloat16 *>(base) + (int64_t)i * ld + j;
+    if (vec && j + 7 < n) {
+      uint4 t;
+      t.x = pack_bf16(v[0], v[1]);
+      t.y = pack_bf16(v[2], v[3]);
+      t.z = pack_bf16(v[4], v[5]);
+      t.w = pack_bf16(v[6], v[7]);
+      *reinterpret_cast<uint4 *>(row) = t;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        if (j + e < n) row[e] = __float2bfloat16_rn(v[e]);
+    }
+  }
 }
 
 // Address of X element block for the tiled layout: tile (tr, tc) is a T x T panel matrix.
-__device__ __forceinline__ char *tile_base(char *xbase, const MatDesc &d, int r, int c) {
+__device__ __forceinline__ const char *tile_base(const char *xbase, const MatDesc &d, int r, int c) {
   const int64_t T = d.ph;
   const int64_t tl = (int64_t)(r / T) * d.tiles_c + (c / T);
   return xbase + tl * T * T * 2;
 }
 
-// Writes 16 values of X row xr, columns xc..xc+15, into the NS operand storage.
-__device__ __forceinline__ void store_x16(char *xbase, const MatDesc &d, int xr, int xc, const float (&v)[16]) {
-  if (d.flags & kNsF32) {
-    // fp32 row-major, unpadded: r x s with row stride ph.
-    const bool tall = d.flags & kTall;
-    const int rr = tall ? d.n : d.m, ss = tall ? d.m : d.n;
+// Byte offset (from xbase) of the 16-byte chunk holding X row xr, columns xc..xc+7 of a
+// bf16 X (panel layout, or a grid of T x T panel tiles when tiled).
+__device__ __forceinline__ const char *x_chunk(const char *xbase, const MatDesc &d, int xr, int xc) {
+  if (d.flags & kTiled) return tile_base(xbase, d, xr, xc) + panel_chunk_off(xr % d.ph, xc % d.ph, d.ph);
+  return xbase + panel_chunk_off(xr, xc, d.ph);
+}
+
+// fp32 X (kNsF32): unpadded r x s, row stride ph.
+__device__ __forceinline__ void xf32_dims(const MatDesc &d, int &rr, int &ss) {
+  const bool tall = d.flags & kTall;
+  rr = tall ? d.n : d.m;
+  ss = tall ? d.m : d.n;
+}
+
+// Writes X row xr, columns xc..xc+7 into the NS operand storage.
+__device__ __forceinline__ void x_store8(char *xbase, const MatDesc &d, int xr, int xc, const float (&v)[8],
+                                         bool allow_f32) {
+  if (allow_f32 && (d.flags & kNsF32)) {
+    int rr, ss;
+    xf32_dims(d, rr, ss);
     if (xr >= rr) return;
     float *row = reinterpret_cast<float *>(xbase) + (int64_t)xr * d.ph;
 #pragma unroll
-    for (int e = 0; e < 16; ++e)
+    for (int e = 0; e < 8; ++e)
       if (xc + e < ss) row[xc + e] = v[e];
     return;
   }
-  char *base = xbase;
-  int64_t ph = d.ph;
-  int lr = xr, lc = xc;
-  if (d.flags & kTiled) {
-    base = tile_base(xbase, d, xr, xc);
-    lr = xr % d.ph;
-    lc = xc % d.ph;
-  }
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    uint4 t;
-    t.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
-    t.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
-    t.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
-    t.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
-    *reinterpret_cast<uint4 *>(base + panel_chunk_off(lr, lc + 8 * q, ph)) = t;
-  }
+  uint4 t;
+  t.x = pack_bf16(v[0], v[1]);
+  t.y = pack_bf16(v[2], v[3]);
+  t.z = pack_bf16(v[4], v[5]);
+  t.w = pack_bf16(v[6], v[7]);
+  *reinterpret_cast<uint4 *>(const_cast<char *>(x_chunk(xbase, d, xr, xc))) = t;
 }
 
-// Reads 16 values of X row xr, columns xc..xc+15 (zero outside an fp32 X).
-__device__ __forceinline__ void load_x16(const char *xbase, const MatDesc &d, int xr, int xc, float (&v)[16]) {
-  if (d.flags & kNsF32) {
-    const bool tall = d.flags & kTall;
-    const int rr = tall ? d.n : d.m, ss = tall ? d.m : d.n;
+// Reads X row xr, columns xc..xc+7 raw (bf16 chunk, or fp32 values zero outside X).
+__device__ __forceinline__ void x_load8(const char *xbase, const MatDesc &d, int xr, int xc, Raw8 &r,
+                                        bool allow_f32) {
+  if (allow_f32 && (d.flags & kNsF32)) {
+    int rr, ss;
+    xf32_dims(d, rr, ss);
     const float *row = reinterpret_cast<const float *>(xbase) + (int64_t)xr * d.ph;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) v[e] = (xr < rr && xc + e < ss) ? row[xc + e] : 0.f;
+    for (int e = 0; e < 8; ++e) r.q[e] = (xr < rr && xc + e < ss) ? __float_as_uint(row[xc + e]) : 0u;
     return;
   }
-  const char *base = xbase;
-  int lr = xr, lc = xc;
-  if (d.flags & kTiled) {
-    base = tile_base(const_cast<char *>(xbase), d, xr, xc);
-    lr = xr % d.ph;
-    lc = xc % d.ph;
-  }
+  const uint4 a = *reinterpret_cast<const uint4 *>(x_chunk(xbase, d, xr, xc));
+  r.q[0] = a.x; r.q[1] = a.y; r.q[2] = a.z; r.q[3] = a.w;
+}
+
+// Fixed-order sum over the CTA of NV per-thread doubles; thread 0 gets the totals.
+// `red` holds two buffers used alternately (`parity`), so that back-to-back calls need
+// one barrier each: a buffer is rewritten only after the barrier of the call in between.
+template <int NV>
+__device__ __forceinline__ void cta_sum(double (&v)[NV], double (*red)[kWarps * NV], int parity) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    uint4 t = *reinterpret_cast<const uint4 *>(base + panel_chunk_off(lr, lc + 8 * q, d.ph));
-    v[8 * q + 0] = bf16lo(t.x); v[8 * q + 1] = bf16hi(t.x);
-    v[8 * q + 2] = bf16lo(t.y); v[8 * q + 3] = bf16hi(t.y);
-    v[8 * q + 4] = bf16lo(t.z); v[8 * q + 5] = bf16hi(t.z);
-    v[8 * q + 6] = bf16lo(t.w); v[8 * q + 7] = bf16hi(t.w);
+  for (int k = 0; k < NV; ++k) v[k] = warp_sum(v[k]);
+  if (lane == 0) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k) red[parity][warp * NV + k] = v[k];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+      double s = 0.0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) s += red[parity][w * NV + k];
+      v[k] = s;
+    }
   }
 }
 
 // ------------------------------------------------------------------------- momentum
-__global__ void __launch_bounds__(kThreads) momentum_kernel(const __grid_constant__ MomentumParams p) {
-  __shared__ float sT[kBlk][kBlk + 1];   // transpose staging (tall matrices), hi then lo
-  __shared__ double red[kThreads / 32];
-  const int blk = blockIdx.x;
-  const MatDesc &d = p.mats[find_mat(p, blk)];
-  int r0, c0;
-  block_origin(d, blk - d.blk_begin, r0, c0);
-  const int t = threadIdx.x, rr = t >> 2, cg = (t & 3) * 16;
-  const int i = r0 + rr, j = c0 + cg;
-  const bool f32 = d.flags & kWF32, vec = d.flags & kVec;
-  const bool round_bf16 = !(d.flags & (kNsF32 | kURow));
-  const bool lo_part = round_bf16 && d.xlo_off >= 0;
+// Inputs of one block as loaded: G (or the given U) and M for the thread's two rows.
+struct MomIn {
+  Raw8 g[2], m[2];
+};
 
-  float g[16], mm[16], u[16], ul[16];
-  const bool from_p = d.flags & kFromP;
-  if (from_p) {
-    // U is given (the Newton-Muon preconditioned update), fp32 row-major m x n.
-    load16(p.ws + d.u_off, d.n, i, j, d.m, d.n, true, (d.n % 4) == 0, g);
-  } else {
-    load16(d.G, d.ld, i, j, d.m, d.n, f32, vec, g);
-    loadM(d.M, d.ld, i, j, d.m, d.n, vec, mm);
+template <bool F32>
+__device__ __forceinline__ void momentum_load(const MomentumParams &p, const MatDesc &d, int r0, int c0,
+                                              MomIn &in) {
+  const int rq = threadIdx.x >> 3, cq = (threadIdx.x & 7) * 8;
+  const bool vec = d.flags & kVec;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int i = r0 + rq + 32 * h, j = c0 + cq;
+    if (F32 && (d.flags & kFromP)) {
+      // U is given (the Newton-Muon preconditioned update), fp32 row-major m x n.
+      raw_load8(p.ws + d.u_off, d.n, i, j, d.m, d.n, true, (d.n % 4) == 0, in.g[h]);
+      raw_zero(in.m[h]);
+    } else {
+      raw_load8(d.G, d.ld, i, j, d.m, d.n, F32 && (d.flags & kWF32), vec, in.g[h]);
+      raw_load8(d.M, d.ld, i, j, d.m, d.n, true, vec, in.m[h]);
+    }
   }
+}
+
+// One 64x64 block: momentum update, U into the NS operand storage, ||U||^2 partial.
+template <bool F32>
+__device__ __forceinline__ void momentum_block(const MomentumParams &p, const MatDesc &d, int cblk, int cr0,
+                                               int cc0, const MomIn &in, float (&sT)[2][kBlk][kBlk + 1],
+                                               double (*red)[kWarps], int &nred) {
+  const int rq = threadIdx.x >> 3, cq = (threadIdx.x & 7) * 8;
+  const bool f32 = F32 && (d.flags & kWF32), vec = d.flags & kVec;
+  const bool from_p = F32 && (d.flags & kFromP);
+  const bool urow = F32 && (d.flags & kURow);
+  const bool round_bf16 = !F32 || !(d.flags & (kNsF32 | kURow));
+  const bool lo_part = round_bf16 && d.xlo_off >= 0;
+  const bool tr = (d.flags & kTall) && !(d.flags & kTiled);
+  char *xbase = p.ws + d.x_off;
+  char *lbase = lo_part ? p.ws + d.xlo_off : nullptr;
   const float beta = p.beta, omb = 1.0f - p.beta;
   float acc = 0.f;
 #pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    float uf;
-    if (from_p) {
-      uf = g[e];
+  for (int h = 0; h < 2; ++h) {
+    const int i = cr0 + rq + 32 * h, j = cc0 + cq;
+    float g[8], mm[8], u[8], ul[8];
+    raw_cvt8(in.g[h], f32 || from_p, g);
+    raw_cvt8(in.m[h], true, mm);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float uf;
+      if (from_p) {
+        uf = g[e];
+      } else {
+        const float mnew = fmaf(beta, mm[e], omb * g[e]);
+        mm[e] = mnew;
+        uf = p.nesterov ? fmaf(omb, g[e], beta * mnew) : mnew;
+      }
+      if (!(i < d.m && j + e < d.n)) uf = 0.f;
+      const float uh = round_bf16 ? bf16_round(uf) : uf;
+      u[e] = uh;
+      ul[e] = uf - uh;                       // exact in fp32; stored as bf16 when kept
+      const float un = lo_part ? uf : uh;    // the norm of what the first iteration reads
+      acc = fmaf(un, un, acc);
+    }
+    if (!from_p) store8(d.M, d.ld, i, j, d.m, d.n, true, vec, mm);
+    if (urow) {
+      // Newton-Muon: U goes to an fp32 row-major buffer for the triangular solves.
+      store8(p.ws + d.u_off, d.n, i, j, d.m, d.n, true, (d.n % 4) == 0, u);
+    } else if (tr) {
+      // X = U^T: stage hi and lo parts; the previous readers of sT finished before the
+      // last cta_sum barrier.
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        sT[0][rq + 32 * h][cq + e] = u[e];
+        if (lo_part) sT[1][rq + 32 * h][cq + e] = ul[e];
+      }
     } else {
-      const float mnew = fmaf(beta, mm[e], omb * g[e]);
-      mm[e] = mnew;
-      uf = p.nesterov ? fmaf(omb, g[e], beta * mnew) : mnew;
+      x_store8(xbase, d, i, j, u, F32);
+      if (lo_part) x_store8(lbase, d, i, j, ul, F32);
     }
-    if (!(i < d.m && j + e < d.n)) uf = 0.f;
-    const float uh = round_bf16 ? bf16_round(uf) : uf;
-    u[e] = uh;
-    ul[e] = uf - uh;                       // exact in fp32; stored as bf16 when kept
-    const float un = lo_part ? uf : uh;    // the norm of what the first iteration reads
-    acc = fmaf(un, un, acc);
   }
-  if (!from_p) store16(d.M, d.ld, i, j, d.m, d.n, true, vec, mm);
-  if (d.flags & kURow) {
-    // Newton-Muon: U goes to an fp32 row-major buffer for the triangular solves.
-    store16(p.ws + d.u_off, d.n, i, j, d.m, d.n, true, (d.n % 4) == 0, u);
-    return;
-  }
-
-  char *xbase = p.ws + d.x_off;
-  char *lbase = lo_part ? p.ws + d.xlo_off : nullptr;
-  if (d.flags & kTall && !(d.flags & kTiled)) {
-    // X = U^T: stage the block and write it transposed (hi, then lo through the same tile).
-#pragma unroll
-    for (int e = 0; e < 16; ++e) sT[rr][cg + e] = u[e];
-    __syncthreads();
-    float v[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) v[e] = sT[cg + e][rr];
-    store_x16(xbase, d, c0 + rr, r0 + cg, v);
-    if (lo_part) {
+  if (!urow) {
+    if (tr) {
       __syncthreads();
 #pragma unroll
-      for (int e = 0; e < 16; ++e) sT[rr][cg + e] = ul[e];
-      __syncthreads();
+      for (int h = 0; h < 2; ++h) {
+        float v[8];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = sT[cg + e][rr];
-      store_x16(lbase, d, c0 + rr, r0 + cg, v);
+        for (int e = 0; e < 8; ++e) v[e] = sT[0][cq + e][rq + 32 * h];
+        x_store8(xbase, d, cc0 + rq + 32 * h, cr0 + cq, v, F32);
+        if (lo_part) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = sT[1][cq + e][rq + 32 * h];
+          x_store8(lbase, d, cc0 + rq + 32 * h, cr0 + cq, v, F32);
+        }
+      }
     }
-  } else {
-    store_x16(xbase, d, i, j, u);
-    if (lo_part) store_x16(lbase, d, i, j, ul);
+    double s[1] = {(double)acc};
+    cta_sum<1>(s, red, nred & 1);
+    ++nred;
+    if (threadIdx.x == 0) p.partials[cblk] = s[0];
   }
+}
 
-  double s[1] = {(double)acc};
-  block_sum<1>(s, red);
-  if (t == 0) p.partials[blk] = s[0];
+// The next block's inputs are prefetched into registers while the current one is
+// processed.  F32 = false: every matrix of the launch has bf16 W, G and X (the common
+// case; half the prefetch registers, three CTAs per SM).
+template <bool F32>
+__global__ void __launch_bounds__(kThreads, F32 ? 2 : 3) momentum_kernel(const __grid_constant__ MomentumParams p) {
+  __shared__ float sT[2][kBlk][kBlk + 1];   // transpose staging (tall matrices): hi, lo
+  __shared__ double red[2][kWarps];
+  int blk = blockIdx.x;
+  if (blk >= p.total_blocks) return;
+  int mi = find_mat(p, blk);
+  int r0, c0;
+  block_origin(p.mats[mi], blk - p.mats[mi].blk_begin, r0, c0);
+  MomIn nxt;
+  momentum_load<F32>(p, p.mats[mi], r0, c0, nxt);
+  int nred = 0;
+  for (;;) {
+    const MomIn in = nxt;
+    const int cblk = blk, cr0 = r0, cc0 = c0;
+    const MatDesc &d = p.mats[mi];
+    blk += gridDim.x;
+    const bool more = blk < p.total_blocks;
+    if (more) {
+      const int nmi = advance_mat(p, mi, blk);
+      block_origin(p.mats[nmi], blk - p.mats[nmi].blk_begin, r0, c0);
+      momentum_load<F32>(p, p.mats[nmi], r0, c0, nxt);
+      mi = nmi;
+    }
+    momentum_block<F32>(p, d, cblk, cr0, cc0, in, sT, red, nred);
+    if (!more) break;
+  }
 }
 
 // ---------------------------------------------------------------- norm finalize
@@ -298,83 +395,140 @@ __global__ void norm_finalize_kernel(const __grid_constant__ NormFinParams p, in
   }
 }
 
-// This thread's 16 O values of W row r0 + t/4, columns c0 + 16 (t%4) .. +15.  Matrices
-// whose NS ran on the transpose go through the shared tile sO; the others read their
-// 16 values straight from the panel layout (two 16-byte chunks, no block barrier).
-__device__ __forceinline__ void load_o_block(const ApplyParams &p, const MatDesc &d, int r0, int c0,
-                                             float (&sO)[kBlk][kBlk + 1]);
-__device__ __forceinline__ void load_o16(const ApplyParams &p, const MatDesc &d, int r0, int c0,
-                                         float (&sO)[kBlk][kBlk + 1], float (&o)[16]) {
-  const int t = threadIdx.x, rr = t >> 2, cg = (t & 3) * 16;
-  const bool tr = (d.flags & kTall) && !(d.flags & kTiled);
-  if (!tr) {
-    load_x16(p.ws + d.o_off, d, r0 + rr, c0 + cg, o);
-    return;
-  }
-  load_o_block(p, d, r0, c0, sO);
+// ------------------------------------------------------------ (W, O) streaming input
+// W and O of one block as loaded.  O is read in X coordinates: for a matrix whose NS ran
+// on the transpose, the thread loads X rows c0 + t/8 (+32) = W columns and turns the
+// block around in shared memory when it processes it.
+struct WoIn {
+  Raw8 w[2], o[2];
+};
+
+__device__ __forceinline__ bool o_transposed(const MatDesc &d) { return (d.flags & kTall) && !(d.flags & kTiled); }
+
+template <bool F32>
+__device__ __forceinline__ void wo_load(const ApplyParams &p, const MatDesc &d, int r0, int c0, bool want_o,
+                                        WoIn &in) {
+  const int rq = threadIdx.x >> 3, cq = (threadIdx.x & 7) * 8;
+  const bool tr = o_transposed(d);
+  const char *xbase = p.ws + d.o_off;
 #pragma unroll
-  for (int e = 0; e < 16; ++e) o[e] = sO[rr][cg + e];
+  for (int h = 0; h < 2; ++h) {
+    raw_load8(d.W, d.ld, r0 + rq + 32 * h, c0 + cq, d.m, d.n, F32 && (d.flags & kWF32), d.flags & kVec, in.w[h]);
+    if (want_o) {
+      if (tr) x_load8(xbase, d, c0 + rq + 32 * h, r0 + cq, in.o[h], F32);
+      else x_load8(xbase, d, r0 + rq + 32 * h, c0 + cq, in.o[h], F32);
+    }
+  }
 }
 
-// Loads the O block of W block (r0, c0) into sO[w_row][w_col] (zero outside W).
-__device__ __forceinline__ void load_o_block(const ApplyParams &p, const MatDesc &d, int r0, int c0,
-                                             float (&sO)[kBlk][kBlk + 1]) {
-  const int t = threadIdx.x, rr = t >> 2, cg = (t & 3) * 16;
-  const char *xbase = p.ws + d.o_off;
-  float v[16];
-  const bool tr = (d.flags & kTall) && !(d.flags & kTiled);
-  if (tr) {
-    load_x16(xbase, d, c0 + rr, r0 + cg, v);          // X row = W column
+// The thread's O values in W coordinates (rows r0 + t/8 (+32), columns c0 + 8 (t%8) ..),
+// zero outside W.  Transposed blocks go through sO and end with a barrier, after which
+// sO may be rewritten.
+template <bool F32>
+__device__ __forceinline__ void wo_values(const MatDesc &d, int r0, int c0, const WoIn &in,
+                                          float (&sO)[kBlk][kBlk + 1], float (&w)[2][8], float (&o)[2][8]) {
+  const int rq = threadIdx.x >> 3, cq = (threadIdx.x & 7) * 8;
+  const bool of32 = F32 && (d.flags & kNsF32);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) sO[cg + e][rr] = v[e];
+  for (int h = 0; h < 2; ++h) raw_cvt8(in.w[h], F32 && (d.flags & kWF32), w[h]);
+  if (o_transposed(d)) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float v[8];
+      raw_cvt8(in.o[h], of32, v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sO[cq + e][rq + 32 * h] = v[e];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[h][e] = sO[rq + 32 * h][cq + e];
+    __syncthreads();
   } else {
-    load_x16(xbase, d, r0 + rr, c0 + cg, v);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) sO[rr][cg + e] = v[e];
+    for (int h = 0; h < 2; ++h) raw_cvt8(in.o[h], of32, o[h]);
   }
-  __syncthreads();
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int i = r0 + rq + 32 * h, j = c0 + cq;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (!(i < d.m && j + e < d.n)) o[h][e] = 0.f;
+  }
 }
 
 // ------------------------------------------------------------ (W, O) reductions
-__global__ void __launch_bounds__(kThreads) reduce_kernel(const __grid_constant__ ApplyParams p) {
-  __shared__ float sO[kBlk][kBlk + 1];
-  __shared__ double red[3 * kThreads / 32];
-  const int blk = blockIdx.x;
-  const MatDesc &d = p.mats[find_mat(p, blk)];
-  int r0, c0;
-  block_origin(d, blk - d.blk_begin, r0, c0);
-  const int t = threadIdx.x, rr = t >> 2, cg = (t & 3) * 16;
-  const int i = r0 + rr, j = c0 + cg;
-  float w[16];
-  load16(d.W, d.ld, i, j, d.m, d.n, d.flags & kWF32, d.flags & kVec, w);
+template <bool F32>
+__device__ __forceinline__ void reduce_block(const ApplyParams &p, const MatDesc &d, int cblk, int cr0, int cc0,
+                                             const WoIn &in, float (&sO)[kBlk][kBlk + 1], double (*red)[3 * kWarps],
+                                             int &nred) {
+  float w[2][8], o[2][8];
   float om = 0.f, de = 0.f, pi = 0.f;
   if (p.op != kOpNorms) {
-    float ov[16];
-    load_o16(p, d, r0, c0, sO, ov);
+    wo_values<F32>(d, cr0, cc0, in, sO, w, o);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const float o = (i < d.m && j + e < d.n) ? ov[e] : 0.f;
-      om = fmaf(o, o, om);
-      de = fmaf(w[e], o, de);
-    }
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        om = fmaf(o[h][e], o[h][e], om);
+        de = fmaf(w[h][e], o[h][e], de);
+      }
+  } else {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) raw_cvt8(in.w[h], F32 && (d.flags & kWF32), w[h]);
   }
 #pragma unroll
-  for (int e = 0; e < 16; ++e) pi = fmaf(w[e], w[e], pi);
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) pi = fmaf(w[h][e], w[h][e], pi);
   double s[3] = {(double)om, (double)de, (double)pi};
-  block_sum<3>(s, red);
-  if (t == 0) {
-    p.partials[3 * (int64_t)blk + 0] = s[0];
-    p.partials[3 * (int64_t)blk + 1] = s[1];
-    p.partials[3 * (int64_t)blk + 2] = s[2];
+  cta_sum<3>(s, red, nred & 1);
+  ++nred;
+  if (threadIdx.x == 0) {
+    p.partials[3 * (int64_t)cblk + 0] = s[0];
+    p.partials[3 * (int64_t)cblk + 1] = s[1];
+    p.partials[3 * (int64_t)cblk + 2] = s[2];
+  }
+}
+
+// Register prefetch of the next block (F32 as for momentum_kernel).
+template <bool F32>
+__global__ void __launch_bounds__(kThreads, F32 ? 2 : 3) reduce_kernel(const __grid_constant__ ApplyParams p) {
+  __shared__ float sO[kBlk][kBlk + 1];
+  __shared__ double red[2][3 * kWarps];
+  const bool want_o = p.op != kOpNorms;
+  int blk = blockIdx.x;
+  if (blk >= p.total_blocks) return;
+  int mi = find_mat(p, blk);
+  int r0, c0;
+  block_origin(p.mats[mi], blk - p.mats[mi].blk_begin, r0, c0);
+  WoIn nxt;
+  wo_load<F32>(p, p.mats[mi], r0, c0, want_o, nxt);
+  int nred = 0;
+  for (;;) {
+    const WoIn in = nxt;
+    const int cblk = blk, cr0 = r0, cc0 = c0;
+    const MatDesc &d = p.mats[mi];
+    blk += gridDim.x;
+    const bool more = blk < p.total_blocks;
+    if (more) {
+      const int nmi = advance_mat(p, mi, blk);
+      block_origin(p.mats[nmi], blk - p.mats[nmi].blk_begin, r0, c0);
+      wo_load<F32>(p, p.mats[nmi], r0, c0, want_o, nxt);
+      mi = nmi;
+    }
+    reduce_block<F32>(p, d, cblk, cr0, cc0, in, sO, red, nred);
+    if (!more) break;
   }
 }
 
 // ||W - t O||^2 for matrices flagged need_exact; a persistent grid walks their blocks.
 __global__ void __launch_bounds__(kThreads) exact_norm_kernel(const __grid_constant__ ApplyParams p) {
   __shared__ float sO[kBlk][kBlk + 1];
-  __shared__ double red[kThreads / 32];
-  const int t = threadIdx.x, rr = t >> 2, cg = (t & 3) * 16;
+  __shared__ double red[2][kWarps];
   if (*(volatile uint32_t *)(p.status + 1) == 0) return;  // no matrix of this call needs it
+  int nred = 0;
   for (int mi = 0; mi < p.nmat; ++mi) {
     const MatDesc &d = p.mats[mi];
     const MatScalars &sc = p.scal[d.mat];
@@ -384,21 +538,22 @@ __global__ void __launch_bounds__(kThreads) exact_norm_kernel(const __grid_const
     for (int lb = blockIdx.x; lb < nb; lb += gridDim.x) {
       int r0, c0;
       block_origin(d, lb, r0, c0);
-      const int i = r0 + rr, j = c0 + cg;
-      float w[16];
-      load16(d.W, d.ld, i, j, d.m, d.n, d.flags & kWF32, d.flags & kVec, w);
-      float ov[16];
-      load_o16(p, d, r0, c0, sO, ov);
+      WoIn in;
+      wo_load<true>(p, d, r0, c0, true, in);
+      float w[2][8], o[2][8];
+      wo_values<true>(d, r0, c0, in, sO, w, o);
       float acc = 0.f;
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float o = (i < d.m && j + e < d.n) ? ov[e] : 0.f;
-        const float v = fmaf(-tt, o, w[e]);
-        acc = fmaf(v, v, acc);
-      }
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float v = fmaf(-tt, o[h][e], w[h][e]);
+          acc = fmaf(v, v, acc);
+        }
       double s[1] = {(double)acc};
-      block_sum<1>(s, red);
-      if (t == 0) p.partials[d.blk_begin + lb] = s[0];
+      cta_sum<1>(s, red, nred & 1);
+      ++nred;
+      if (threadIdx.x == 0) p.partials[d.blk_begin + lb] = s[0];
     }
   }
 }
@@ -518,36 +673,103 @@ __global__ void apply_finalize_kernel(const __grid_constant__ ApplyFinParams p) 
   }
 }
 
+
 // ------------------------------------------------------------------------ apply
-__global__ void __launch_bounds__(kThreads) apply_kernel(const __grid_constant__ ApplyParams p) {
-  __shared__ float sO[kBlk][kBlk + 1];
-  const int blk = blockIdx.x;
-  const MatDesc &d = p.mats[find_mat(p, blk)];
-  int r0, c0;
-  block_origin(d, blk - d.blk_begin, r0, c0);
-  const int t = threadIdx.x, rr = t >> 2, cg = (t & 3) * 16;
-  const int i = r0 + rr, j = c0 + cg;
-  const bool f32 = d.flags & kWF32, vec = d.flags & kVec;
-  float o[16];
-  load_o16(p, d, r0, c0, sO, o);
+template <bool F32>
+__device__ __forceinline__ void apply_block(const MatDesc &d, int cr0, int cc0, const WoIn &in, float a, float b,
+                                            float (&sO)[kBlk][kBlk + 1]) {
+  const int rq = threadIdx.x >> 3, cq = (threadIdx.x & 7) * 8;
+  const bool f32 = F32 && (d.flags & kWF32), vec = d.flags & kVec;
+  float w[2][8], o[2][8];
+  wo_values<F32>(d, cr0, cc0, in, sO, w, o);
   if (d.O_out) {
     const bool vo = ((uintptr_t)d.O_out % 16 == 0) && (d.n % (f32 ? 4 : 8) == 0);
-    store16(d.O_out, d.n, i, j, d.m, d.n, f32, vo, o);
-  }
-  const MatScalars &s = p.scal[d.mat];
-  const float a = s.alpha, b = s.beta;
-  if (a == 1.f && b == 0.f) return;
-  float w[16];
-  load16(d.W, d.ld, i, j, d.m, d.n, f32, vec, w);
 #pragma unroll
-  for (int e = 0; e < 16; ++e) w[e] = fmaf(a, w[e], b * o[e]);
-  store16(d.W, d.ld, i, j, d.m, d.n, f32, vec, w);
+    for (int h = 0; h < 2; ++h) store8(d.O_out, d.n, cr0 + rq + 32 * h, cc0 + cq, d.m, d.n, f32, vo, o[h]);
+  }
+  if (!(a == 1.f && b == 0.f)) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w[h][e] = fmaf(a, w[h][e], b * o[h][e]);
+      store8(d.W, d.ld, cr0 + rq + 32 * h, cc0 + cq, d.m, d.n, f32, vec, w[h]);
+    }
+  }
+}
+
+// Register prefetch of the next block (F32 as for momentum_kernel).
+template <bool F32>
+__global__ void __launch_bounds__(kThreads, F32 ? 2 : 3) apply_kernel(const __grid_constant__ ApplyParams p) {
+  __shared__ float sO[kBlk][kBlk + 1];
+  int blk = blockIdx.x;
+  if (blk >= p.total_blocks) return;
+  int mi = find_mat(p, blk);
+  int r0, c0;
+  block_origin(p.mats[mi], blk - p.mats[mi].blk_begin, r0, c0);
+  WoIn nxt;
+  wo_load<F32>(p, p.mats[mi], r0, c0, true, nxt);
+  float na = p.scal[p.mats[mi].mat].alpha, nb = p.scal[p.mats[mi].mat].beta;
+  for (;;) {
+    const WoIn in = nxt;
+    const int cr0 = r0, cc0 = c0;
+    const float a = na, b = nb;
+    const MatDesc &d = p.mats[mi];
+    blk += gridDim.x;
+    const bool more = blk < p.total_blocks;
+    if (more) {
+      const int nmi = advance_mat(p, mi, blk);
+      const MatDesc &dn = p.mats[nmi];
+      block_origin(dn, blk - dn.blk_begin, r0, c0);
+      wo_load<F32>(p, dn, r0, c0, true, nxt);
+      if (nmi != mi) {
+        na = p.scal[dn.mat].alpha;
+        nb = p.scal[dn.mat].beta;
+      }
+      mi = nmi;
+    }
+    apply_block<F32>(d, cr0, cc0, in, a, b, sO);
+    if (!more) break;
+  }
+}
+
+// Persistent grid: the SM count times the CTAs of `kernel` that fit on one SM with
+// `dyn_smem` bytes of dynamic shared memory, capped by the work.  Queried once per
+// kernel and device.
+template <typename K>
+int stream_grid(K kernel, int slot, int dyn_smem, int total_blocks) {
+  static int cached[8][64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  int g = cached[slot][dev];
+  if (g == 0) {
+    int sms = 0, per = 0;
+    if (dyn_smem > 0) cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kernel, kThreads, dyn_smem);
+    g = (sms > 0 ? sms : 148) * (per > 0 ? per : 1);
+    cached[slot][dev] = g;
+  }
+  return total_blocks < g ? total_blocks : g;
 }
 
 }  // namespace
 
+// The bf16 instances need every matrix of the launch in bf16 (W, G and X); anything
+// else (fp32 W or X, the Newton-Muon U/P buffers) takes the F32 instances.
+template <typename P>
+bool needs_f32(const P &p) {
+  for (int i = 0; i < p.nmat; ++i)
+    if (p.mats[i].flags & (kWF32 | kNsF32 | kFromP | kURow)) return true;
+  return false;
+}
+
 cudaError_t launch_momentum(const MomentumParams &p, cudaStream_t s) {
-  if (p.total_blocks > 0) momentum_kernel<<<p.total_blocks, kThreads, 0, s>>>(p);
+  if (p.total_blocks > 0) {
+    if (needs_f32(p))
+      momentum_kernel<true><<<stream_grid(momentum_kernel<true>, 0, 0, p.total_blocks), kThreads, 0, s>>>(p);
+    else
+      momentum_kernel<false><<<stream_grid(momentum_kernel<false>, 1, 0, p.total_blocks), kThreads, 0, s>>>(p);
+  }
   return cudaGetLastError();
 }
 cudaError_t launch_norm_finalize(const NormFinParams &p, int nseg_total, cudaStream_t s) {
@@ -555,7 +777,12 @@ cudaError_t launch_norm_finalize(const NormFinParams &p, int nseg_total, cudaStr
   return cudaGetLastError();
 }
 cudaError_t launch_reduce(const ApplyParams &p, cudaStream_t s) {
-  if (p.total_blocks > 0) reduce_kernel<<<p.total_blocks, kThreads, 0, s>>>(p);
+  if (p.total_blocks > 0) {
+    if (needs_f32(p))
+      reduce_kernel<true><<<stream_grid(reduce_kernel<true>, 2, 0, p.total_blocks), kThreads, 0, s>>>(p);
+    else
+      reduce_kernel<false><<<stream_grid(reduce_kernel<false>, 3, 0, p.total_blocks), kThreads, 0, s>>>(p);
+  }
   return cudaGetLastError();
 }
 cudaError_t launch_exact_norm(const ApplyParams &p, cudaStream_t s) {
@@ -567,7 +794,12 @@ cudaError_t launch_apply_finalize(const ApplyFinParams &p, cudaStream_t s) {
   return cudaGetLastError();
 }
 cudaError_t launch_apply(const ApplyParams &p, cudaStream_t s) {
-  if (p.total_blocks > 0) apply_kernel<<<p.total_blocks, kThreads, 0, s>>>(p);
+  if (p.total_blocks > 0) {
+    if (needs_f32(p))
+      apply_kernel<true><<<stream_grid(apply_kernel<true>, 4, 0, p.total_blocks), kThreads, 0, s>>>(p);
+    else
+      apply_kernel<false><<<stream_grid(apply_kernel<false>, 5, 0, p.total_blocks), kThreads, 0, s>>>(p);
+  }
   return cudaGetLastError();
 }
 
