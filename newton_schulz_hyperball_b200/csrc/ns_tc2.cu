@@ -107,6 +107,32 @@ __device__ __forceinline__ void tc_commit2_mc(uint32_t bar, uint16_t mask) {
                : "memory");
 }
 
+// The two logically adjacent 16-byte chunks (columns col .. col+15, col a multiple of
+// 16) of a panel row share one 32-byte sector: the 128-byte swizzle maps chunk c to
+// c ^ (row & 7), which keeps pairs {c, c+1} (c even) together and swaps them on odd rows.
+__device__ __forceinline__ size_t panel_pair_off(int64_t row, int64_t col, int64_t ph) {
+  return ((size_t)((col >> 6) * ph + row) << 7) + ((size_t)(((col >> 4) & 3) ^ ((row >> 1) & 3)) << 5);
+}
+// Memory order <-> logical order of a sector pair (its own inverse).
+__device__ __forceinline__ void unswizzle_pair(const uint32_t (&w)[8], bool odd, uint32_t *out) {
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    out[e] = odd ? w[4 + e] : w[e];
+    out[4 + e] = odd ? w[e] : w[4 + e];
+  }
+}
+// 32-byte global accesses (one sector per thread).
+__device__ __forceinline__ void ld_global_256(const void *p, uint32_t (&w)[8]) {
+  asm volatile("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+               : "l"(p));
+}
+__device__ __forceinline__ void st_global_256(void *p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+               "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
 struct Tile {
   int prob, batch, m0, n0;
 };
@@ -302,16 +328,26 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
       const int ra = (int)(i >> 6);
       const int cc_end = (half + 1) * NCH;
       auto live = [&](int cc) { return cc < cc_end && !(sym && ((t.n0 + cc * 32) >> 6) > ra); };
-      auto load_c = [&](int cc, uint4 (&h)[4], uint4 (&l)[4]) {
+      const bool odd = i & 1;
+      // C words of columns col0 .. col0+31 in logical order (two 32-byte sector reads).
+      auto load_c = [&](int cc, uint32_t (&h)[16], uint32_t (&l)[16]) {
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const size_t off = panel_chunk_off(i, t.n0 + cc * 32 + 8 * g, q.d_ph);
-          h[g] = *reinterpret_cast<const uint4 *>(cbase + off);
-          l[g] = clo ? *reinterpret_cast<const uint4 *>(clo + off) : make_uint4(0, 0, 0, 0);
+        for (int k = 0; k < 2; ++k) {
+          const size_t off = panel_pair_off(i, t.n0 + cc * 32 + 16 * k, q.d_ph);
+          uint32_t w[8];
+          ld_global_256(cbase + off, w);
+          unswizzle_pair(w, odd, h + 8 * k);
+          if (clo) {
+            ld_global_256(clo + off, w);
+            unswizzle_pair(w, odd, l + 8 * k);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) l[8 * k + e] = 0u;
+          }
         }
       };
       int cc = half * NCH;
-      uint4 ch[4], cl[4];
+      uint32_t ch[16], cl[16];
       if (needc && live(cc)) load_c(cc, ch, cl);
       if (!mbar_wait(tfull_bar(buf), tph, limit)) {
         set_status(p.status, kTimeoutBit);
@@ -322,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
       for (; live(cc); ++cc) {
         const int col0 = t.n0 + cc * 32;
         const int ca = col0 >> 6;
-        uint4 nh[4], nl[4];
+        uint32_t nh[16], nl[16];
         if (needc && live(cc + 1)) load_c(cc + 1, nh, nl);
         uint32_t r[32];
         tmem_ld32(tmem_base + (uint32_t)(buf * BN + cc * 32) + ((uint32_t)(quarter * 32) << 16), r);
@@ -351,33 +387,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
           const float ks = (p.mode == kPoly) ? 1.0f : s;
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
-            const uint32_t hw[4] = {ch[g].x, ch[g].y, ch[g].z, ch[g].w};
-            const uint32_t lw[4] = {cl[g].x, cl[g].y, cl[g].z, cl[g].w};
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-              const float c0 = bf16lo(hw[h]) + bf16lo(lw[h]);
-              const float c1 = bf16hi(hw[h]) + bf16hi(lw[h]);
+              const float c0 = bf16lo(ch[4 * g + h]) + bf16lo(cl[4 * g + h]);
+              const float c1 = bf16hi(ch[4 * g + h]) + bf16hi(cl[4 * g + h]);
               v[8 * g + 2 * h] = ks * fmaf(kc, c0, ka * __uint_as_float(r[8 * g + 2 * h]));
               v[8 * g + 2 * h + 1] = ks * fmaf(kc, c1, ka * __uint_as_float(r[8 * g + 2 * h + 1]));
             }
           }
         }
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          uint4 o;
-          o.x = pack_bf16(v[8 * g + 0], v[8 * g + 1]);
-          o.y = pack_bf16(v[8 * g + 2], v[8 * g + 3]);
-          o.z = pack_bf16(v[8 * g + 4], v[8 * g + 5]);
-          o.w = pack_bf16(v[8 * g + 6], v[8 * g + 7]);
-          const size_t off = panel_chunk_off(i, col0 + 8 * g, q.d_ph);
-          *reinterpret_cast<uint4 *>(dbase + off) = o;
+        for (int k = 0; k < 2; ++k) {
+          uint32_t o[8], w[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[e] = pack_bf16(v[16 * k + 2 * e], v[16 * k + 2 * e + 1]);
+          const size_t off = panel_pair_off(i, col0 + 16 * k, q.d_ph);
+          unswizzle_pair(o, odd, w);              // the same swap puts logical order back
+          st_global_256(dbase + off, w);
           if (dlo) {
-            uint4 l;
-            l.x = pack_bf16(v[8 * g + 0] - bf16lo(o.x), v[8 * g + 1] - bf16hi(o.x));
-            l.y = pack_bf16(v[8 * g + 2] - bf16lo(o.y), v[8 * g + 3] - bf16hi(o.y));
-            l.z = pack_bf16(v[8 * g + 4] - bf16lo(o.z), v[8 * g + 5] - bf16hi(o.z));
-            l.w = pack_bf16(v[8 * g + 6] - bf16lo(o.w), v[8 * g + 7] - bf16hi(o.w));
-            *reinterpret_cast<uint4 *>(dlo + off) = l;
+            uint32_t l[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              l[e] = pack_bf16(v[16 * k + 2 * e] - bf16lo(o[e]), v[16 * k + 2 * e + 1] - bf16hi(o[e]));
+            unswizzle_pair(l, odd, w);
+            st_global_256(dlo + off, w);
           }
         }
         if (sym && ca < ra) {
@@ -390,9 +423,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
           }
         }
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          ch[g] = nh[g];
-          cl[g] = nl[g];
+        for (int e = 0; e < 16; ++e) {
+          ch[e] = nh[e];
+          cl[e] = nl[e];
         }
       }
       tc_fence_before();
