@@ -123,6 +123,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const long long limit = p.wait_limit;
+  pdl_trigger();
+  pdl_wait();                                      // the previous kernel's outputs are visible
 
   if (warp == 0) {
     if (lane == 0) {
@@ -358,8 +360,7 @@ cudaError_t launch_bn(const GemmParams &p, int num_sms, cudaStream_t s) {
     done_mask |= 1u << (dev & 31);
   }
   const int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
-  gemm_tc_kernel<BN><<<grid, kThreads, Cfg<BN>::SMEM_BYTES, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(gemm_tc_kernel<BN>, grid, kThreads, Cfg<BN>::SMEM_BYTES, s, p);
 }
 
 }  // namespace

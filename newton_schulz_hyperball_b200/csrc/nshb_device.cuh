@@ -2,6 +2,7 @@
 // reductions, mbarriers, bulk async copies and the tcgen05 (5th-generation
 // tensor core) instructions, written as inline PTX.
 #pragma once
+#include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cstdint>
 
@@ -63,6 +64,31 @@ __device__ __forceinline__ void set_status(uint32_t *status, uint32_t bits) {
 // 16-byte chunk that holds (row, col..col+7), col a multiple of 8:
 __device__ __forceinline__ size_t panel_chunk_off(int64_t row, int64_t col, int64_t ph) {
   return ((size_t)((col >> 6) * ph + row) << 7) + ((((col >> 3) & 7) ^ (row & 7)) << 4);
+}
+
+// -------------------------------------------------- programmatic dependent launch
+// A kernel launched with the programmatic-serialization attribute (launch_pdl) may be
+// scheduled while the previous kernel of its stream is still draining.  pdl_wait blocks
+// until that kernel has completed and its memory operations are visible; every kernel
+// calls it before its first global access (it returns at once for a plain launch).
+// pdl_trigger allows the next kernel of the stream to be scheduled early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
 }
 
 // ------------------------------------------------------------ shared-memory addresses

@@ -347,6 +347,8 @@ __device__ __forceinline__ void momentum_block(const MomentumParams &p, const Ma
 // case; half the prefetch registers, three CTAs per SM).
 template <bool F32>
 __global__ void __launch_bounds__(kThreads, F32 ? 2 : 3) momentum_kernel(const __grid_constant__ MomentumParams p) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float sT[2][kBlk][kBlk + 1];   // transpose staging (tall matrices): hi, lo
   __shared__ double red[2][kWarps];
   int blk = blockIdx.x;
@@ -376,6 +378,8 @@ __global__ void __launch_bounds__(kThreads, F32 ? 2 : 3) momentum_kernel(const _
 
 // ---------------------------------------------------------------- norm finalize
 __global__ void norm_finalize_kernel(const __grid_constant__ NormFinParams p, int nseg_total) {
+  pdl_trigger();
+  pdl_wait();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= nseg_total) return;
   int lo = 0, hi = p.nmat - 1;
@@ -495,6 +499,8 @@ __device__ __forceinline__ void reduce_block(const ApplyParams &p, const MatDesc
 // Register prefetch of the next block (F32 as for momentum_kernel).
 template <bool F32>
 __global__ void __launch_bounds__(kThreads, F32 ? 2 : 3) reduce_kernel(const __grid_constant__ ApplyParams p) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float sO[kBlk][kBlk + 1];
   __shared__ double red[2][3 * kWarps];
   const bool want_o = p.op != kOpNorms;
@@ -525,6 +531,8 @@ __global__ void __launch_bounds__(kThreads, F32 ? 2 : 3) reduce_kernel(const __g
 
 // ||W - t O||^2 for matrices flagged need_exact; a persistent grid walks their blocks.
 __global__ void __launch_bounds__(kThreads) exact_norm_kernel(const __grid_constant__ ApplyParams p) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float sO[kBlk][kBlk + 1];
   __shared__ double red[2][kWarps];
   if (*(volatile uint32_t *)(p.status + 1) == 0) return;  // no matrix of this call needs it
@@ -595,6 +603,8 @@ __device__ void brake_coeffs(MatScalars &s, double vv, double pi, const ApplyFin
 // One warp per matrix: the lanes sum the block partials in a fixed order, lane 0 derives
 // the coefficients.
 __global__ void apply_finalize_kernel(const __grid_constant__ ApplyFinParams p) {
+  pdl_trigger();
+  pdl_wait();
   const int k = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (k >= p.nmat) return;
   MatScalars &s = p.scal[p.mat[k]];
@@ -700,6 +710,8 @@ __device__ __forceinline__ void apply_block(const MatDesc &d, int cr0, int cc0, 
 // Register prefetch of the next block (F32 as for momentum_kernel).
 template <bool F32>
 __global__ void __launch_bounds__(kThreads, F32 ? 2 : 3) apply_kernel(const __grid_constant__ ApplyParams p) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float sO[kBlk][kBlk + 1];
   int blk = blockIdx.x;
   if (blk >= p.total_blocks) return;
@@ -766,39 +778,40 @@ bool needs_f32(const P &p) {
 cudaError_t launch_momentum(const MomentumParams &p, cudaStream_t s) {
   if (p.total_blocks > 0) {
     if (needs_f32(p))
-      momentum_kernel<true><<<stream_grid(momentum_kernel<true>, 0, 0, p.total_blocks), kThreads, 0, s>>>(p);
+      return launch_pdl(momentum_kernel<true>, stream_grid(momentum_kernel<true>, 0, 0, p.total_blocks), kThreads, 0, s, p);
     else
-      momentum_kernel<false><<<stream_grid(momentum_kernel<false>, 1, 0, p.total_blocks), kThreads, 0, s>>>(p);
+      return launch_pdl(momentum_kernel<false>, stream_grid(momentum_kernel<false>, 1, 0, p.total_blocks), kThreads, 0, s,
+                        p);
   }
   return cudaGetLastError();
 }
 cudaError_t launch_norm_finalize(const NormFinParams &p, int nseg_total, cudaStream_t s) {
-  if (nseg_total > 0) norm_finalize_kernel<<<(nseg_total + 7) / 8, 256, 0, s>>>(p, nseg_total);
+  if (nseg_total > 0) return launch_pdl(norm_finalize_kernel, (nseg_total + 7) / 8, 256, 0, s, p, nseg_total);
   return cudaGetLastError();
 }
 cudaError_t launch_reduce(const ApplyParams &p, cudaStream_t s) {
   if (p.total_blocks > 0) {
     if (needs_f32(p))
-      reduce_kernel<true><<<stream_grid(reduce_kernel<true>, 2, 0, p.total_blocks), kThreads, 0, s>>>(p);
+      return launch_pdl(reduce_kernel<true>, stream_grid(reduce_kernel<true>, 2, 0, p.total_blocks), kThreads, 0, s, p);
     else
-      reduce_kernel<false><<<stream_grid(reduce_kernel<false>, 3, 0, p.total_blocks), kThreads, 0, s>>>(p);
+      return launch_pdl(reduce_kernel<false>, stream_grid(reduce_kernel<false>, 3, 0, p.total_blocks), kThreads, 0, s, p);
   }
   return cudaGetLastError();
 }
 cudaError_t launch_exact_norm(const ApplyParams &p, cudaStream_t s) {
-  if (p.total_blocks > 0) exact_norm_kernel<<<296, kThreads, 0, s>>>(p);
+  if (p.total_blocks > 0) return launch_pdl(exact_norm_kernel, 296, kThreads, 0, s, p);
   return cudaGetLastError();
 }
 cudaError_t launch_apply_finalize(const ApplyFinParams &p, cudaStream_t s) {
-  if (p.nmat > 0) apply_finalize_kernel<<<(p.nmat + 3) / 4, 128, 0, s>>>(p);
+  if (p.nmat > 0) return launch_pdl(apply_finalize_kernel, (p.nmat + 3) / 4, 128, 0, s, p);
   return cudaGetLastError();
 }
 cudaError_t launch_apply(const ApplyParams &p, cudaStream_t s) {
   if (p.total_blocks > 0) {
     if (needs_f32(p))
-      apply_kernel<true><<<stream_grid(apply_kernel<true>, 4, 0, p.total_blocks), kThreads, 0, s>>>(p);
+      return launch_pdl(apply_kernel<true>, stream_grid(apply_kernel<true>, 4, 0, p.total_blocks), kThreads, 0, s, p);
     else
-      apply_kernel<false><<<stream_grid(apply_kernel<false>, 5, 0, p.total_blocks), kThreads, 0, s>>>(p);
+      return launch_pdl(apply_kernel<false>, stream_grid(apply_kernel<false>, 5, 0, p.total_blocks), kThreads, 0, s, p);
   }
   return cudaGetLastError();
 }
