@@ -214,28 +214,37 @@ __device__ __forceinline__ void x_load8(const char *xbase, const MatDesc &d, int
   r.q[0] = a.x; r.q[1] = a.y; r.q[2] = a.z; r.q[3] = a.w;
 }
 
-// Fixed-order sum over the CTA of NV per-thread doubles; thread 0 gets the totals.
-// `red` holds two buffers used alternately (`parity`), so that back-to-back calls need
-// one barrier each: a buffer is rewritten only after the barrier of the call in between.
+// Fixed-order sum over the CTA of NV per-thread fp32 partials; thread 0 gets the totals
+// in fp64.  Lanes combine in fp32 (five tree levels on top of each thread's own partial,
+// which already sums 16 terms in fp32), warps in fp64.  `red` holds two buffers used
+// alternately (`parity`), so that back-to-back calls need one barrier each: a buffer is
+// rewritten only after the barrier of the call in between.
 template <int NV>
-__device__ __forceinline__ void cta_sum(double (&v)[NV], double (*red)[kWarps * NV], int parity) {
+__device__ __forceinline__ void cta_sum(const float (&v)[NV], double (&out)[NV], double (*red)[kWarps * NV],
+                                        int parity) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float w[NV];
 #pragma unroll
-  for (int k = 0; k < NV; ++k) v[k] = warp_sum(v[k]);
+  for (int k = 0; k < NV; ++k) w[k] = warp_sum(v[k]);
   if (lane == 0) {
 #pragma unroll
-    for (int k = 0; k < NV; ++k) red[parity][warp * NV + k] = v[k];
+    for (int k = 0; k < NV; ++k) red[parity][warp * NV + k] = (double)w[k];
   }
   __syncthreads();
   if (threadIdx.x == 0) {
 #pragma unroll
     for (int k = 0; k < NV; ++k) {
-      double s = 0.0;
+      double t = 0.0;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) s += red[parity][w * NV + k];
-      v[k] = s;
+      for (int q = 0; q < kWarps; ++q) t += red[parity][q * NV + k];
+      out[k] = t;
     }
   }
+}
+
+// True when the 64x64 block at (r0, c0) lies inside the m x n matrix.
+__device__ __forceinline__ bool full_block(const MatDesc &d, int r0, int c0) {
+  return r0 + kBlk <= d.m && c0 + kBlk <= d.n;
 }
 
 // ------------------------------------------------------------------------- momentum
@@ -278,6 +287,7 @@ __device__ __forceinline__ void momentum_block(const MomentumParams &p, const Ma
   char *xbase = p.ws + d.x_off;
   char *lbase = lo_part ? p.ws + d.xlo_off : nullptr;
   const float beta = p.beta, omb = 1.0f - p.beta;
+  const bool full = full_block(d, cr0, cc0);
   float acc = 0.f;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
@@ -295,7 +305,7 @@ __device__ __forceinline__ void momentum_block(const MomentumParams &p, const Ma
         mm[e] = mnew;
         uf = p.nesterov ? fmaf(omb, g[e], beta * mnew) : mnew;
       }
-      if (!(i < d.m && j + e < d.n)) uf = 0.f;
+      if (!full && !(i < d.m && j + e < d.n)) uf = 0.f;
       const float uh = round_bf16 ? bf16_round(uf) : uf;
       u[e] = uh;
       ul[e] = uf - uh;                       // exact in fp32; stored as bf16 when kept
@@ -335,8 +345,9 @@ __device__ __forceinline__ void momentum_block(const MomentumParams &p, const Ma
         }
       }
     }
-    double s[1] = {(double)acc};
-    cta_sum<1>(s, red, nred & 1);
+    const float a1[1] = {acc};
+    double s[1];
+    cta_sum<1>(a1, s, red, nred & 1);
     ++nred;
     if (threadIdx.x == 0) p.partials[cblk] = s[0];
   }
@@ -453,12 +464,14 @@ __device__ __forceinline__ void wo_values(const MatDesc &d, int r0, int c0, cons
 #pragma unroll
     for (int h = 0; h < 2; ++h) raw_cvt8(in.o[h], of32, o[h]);
   }
+  if (!full_block(d, r0, c0)) {
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int i = r0 + rq + 32 * h, j = c0 + cq;
+    for (int h = 0; h < 2; ++h) {
+      const int i = r0 + rq + 32 * h, j = c0 + cq;
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-      if (!(i < d.m && j + e < d.n)) o[h][e] = 0.f;
+      for (int e = 0; e < 8; ++e)
+        if (!(i < d.m && j + e < d.n)) o[h][e] = 0.f;
+    }
   }
 }
 
@@ -486,8 +499,9 @@ __device__ __forceinline__ void reduce_block(const ApplyParams &p, const MatDesc
   for (int h = 0; h < 2; ++h)
 #pragma unroll
     for (int e = 0; e < 8; ++e) pi = fmaf(w[h][e], w[h][e], pi);
-  double s[3] = {(double)om, (double)de, (double)pi};
-  cta_sum<3>(s, red, nred & 1);
+  const float a3[3] = {om, de, pi};
+  double s[3];
+  cta_sum<3>(a3, s, red, nred & 1);
   ++nred;
   if (threadIdx.x == 0) {
     p.partials[3 * (int64_t)cblk + 0] = s[0];
@@ -558,8 +572,9 @@ __global__ void __launch_bounds__(kThreads) exact_norm_kernel(const __grid_const
           const float v = fmaf(-tt, o[h][e], w[h][e]);
           acc = fmaf(v, v, acc);
         }
-      double s[1] = {(double)acc};
-      cta_sum<1>(s, red, nred & 1);
+      const float a1[1] = {acc};
+      double s[1];
+      cta_sum<1>(a1, s, red, nred & 1);
       ++nred;
       if (threadIdx.x == 0) p.partials[d.blk_begin + lb] = s[0];
     }
