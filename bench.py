@@ -38,7 +38,7 @@ DEFAULT_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustaine
 # DRAM read + write per launch of the NS GEMM from the ncu capture summarised in
 # profiles/gemm_tc2_gpt2_small_ns_iteration1.md, valid only for the kernel source it was taken on.
 GEMM_SOURCE = os.path.join(ROOT, "newton_schulz_hyperball_b200", "csrc", "ns_tc2.cu")
-GEMM_TRAFFIC = {"sha256_prefix": "704a1a72938141d3", "bytes_per_launch": 368434517}
+GEMM_TRAFFIC = {"sha256_prefix": "5487563383b5abda", "bytes_per_launch": 372400725}
 
 
 def gemm_traffic():
