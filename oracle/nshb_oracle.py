@@ -23,6 +23,11 @@ rules in their own order.  Sources (page title, then section):
   tiles, then reassembled.
 * "The Newton-Muon Optimizer" (arXiv 2604.01472) -- abstract: the update
   msgn(G (Z Z^T)^-1), "up to momentum and weight decay".
+* The same hook PR's file list -- the RelativeUpdate hook: a pre-update scaling
+  that matches the update's norm to the current weight norm.
+* The Hyperball paper, Method -- Hyperball wraps any base step, Adam's
+  preconditioned update among them (AdamH); Adam itself as in "Adam: A Method
+  for Stochastic Optimization" (Kingma and Ba, 2014), which the pages cite.
 
 Parity status: every public function here is pinned by ``tests/test_oracle_pins.py``
 against page-printed values, closed forms, library routines or invariants.
@@ -184,6 +189,42 @@ def radial_brake_apply(W, O, lr: float, outward: float, inward: float, eps: floa
     return w * ((n_prev + s * delta) / n_new)
 
 
+def relative_update_apply(W, O, lr: float, weight_decay: float = 0.0, eps: float = HB_EPS):
+    """RelativeUpdate hook (PR #224): before the Muon update is applied, rescale it to the
+    Frobenius norm of the current weight.  The update max(1, m/n)^0.5 * O has direction
+    O / ||O||, so its shape factor cancels:
+        W <- (1 - lr wd) W - lr * ||W||_F * O / max(||O||_F, eps)
+    (a zero update stays zero, as in the hooks' eps clamp)."""
+    W = _f64(W)
+    O = _f64(O)
+    return (1.0 - lr * weight_decay) * W - lr * fro(W) * O / max(fro(O), eps)
+
+
+# --------------------------------------------------------------------------
+# Adam (Kingma and Ba, 2014), the base step of AdamH (Hyperball paper, Method).
+# --------------------------------------------------------------------------
+ADAM_BETA1 = 0.9
+ADAM_BETA2 = 0.999
+ADAM_EPS = 1e-8
+
+
+def adam_update(M, V, G, t: int, beta1: float = ADAM_BETA1, beta2: float = ADAM_BETA2, eps: float = ADAM_EPS):
+    """Moments and the bias-corrected Adam direction of step t (t = 1 is the first step):
+        M <- beta1 M + (1 - beta1) G;   V <- beta2 V + (1 - beta2) G^2;
+        U~ = (M / (1 - beta1^t)) / (sqrt(V / (1 - beta2^t)) + eps).
+    Returns (M_new, V_new, U~)."""
+    if t < 1:
+        raise ValueError("Adam steps count from 1")
+    M = _f64(M)
+    V = _f64(V)
+    G = _f64(G)
+    M_new = beta1 * M + (1.0 - beta1) * G
+    V_new = beta2 * V + (1.0 - beta2) * G * G
+    m_hat = M_new / (1.0 - beta1 ** t)
+    v_hat = V_new / (1.0 - beta2 ** t)
+    return M_new, V_new, m_hat / (np.sqrt(v_hat) + eps)
+
+
 # --------------------------------------------------------------------------
 # Hierarchical Muon (arXiv 2606.27216, abstract / core claim).
 # --------------------------------------------------------------------------
@@ -256,3 +297,19 @@ def newton_muon_step(W, G, M, Z, *, ridge_rel, eta, rho, beta=0.95, nesterov=Tru
     O = newton_schulz(P, steps, ns_eps, coeffs)
     W_new, fb = hyperball_apply(W, O, eta, rho, hb_eps)
     return W_new, M_new, O, fb
+
+
+def relative_update_step(W, G, M, *, lr, weight_decay=0.0, beta=0.95, nesterov=True, steps=5,
+                         ns_eps=NS_EPS, coeffs=None, hb_eps=HB_EPS):
+    M_new, U = momentum(M, G, beta, nesterov)
+    O = newton_schulz(U, steps, ns_eps, coeffs)
+    return relative_update_apply(W, O, lr, weight_decay, hb_eps), M_new, O
+
+
+def adamh_step(W, G, M, V, *, t, eta, rho, beta1=ADAM_BETA1, beta2=ADAM_BETA2, adam_eps=ADAM_EPS,
+               hb_eps=HB_EPS):
+    """AdamH: the Adam direction of step t, wrapped by Hyperball.
+    Returns (W_new, M_new, V_new, U~, fallback_taken)."""
+    M_new, V_new, U = adam_update(M, V, G, t, beta1, beta2, adam_eps)
+    W_new, fb = hyperball_apply(W, U, eta, rho, hb_eps)
+    return W_new, M_new, V_new, U, fb

@@ -308,3 +308,82 @@ def test_newton_muon_isotropic_input_is_muon():
     P = o.newton_precondition(U, Z, 1e-3)
     assert np.allclose(P * (9.0 + 1e-3 * 9.0), U, atol=1e-12)
     assert np.allclose(o.newton_schulz(P), o.newton_schulz(U), atol=1e-6)
+
+
+# ------------------------------------------------------------------ RelativeUpdate hook
+def test_relative_update_step_length_is_lr_times_weight_norm():
+    """The hook matches the update's norm to ||W||: with wd = 0 the step W - W_new has
+    Frobenius norm lr * ||W|| exactly and points along O, whatever ||O|| and the shape."""
+    rng = np.random.default_rng(41)
+    for shape in [(6, 9), (9, 6), (5, 5)]:
+        W = rng.standard_normal(shape)
+        O = 7.5 * rng.standard_normal(shape)
+        Wn = o.relative_update_apply(W, O, lr=0.03)
+        step = W - Wn
+        assert abs(o.fro(step) - 0.03 * o.fro(W)) <= 1e-14 * o.fro(W)
+        cos = float(np.sum(step * O)) / (o.fro(step) * o.fro(O))
+        assert abs(cos - 1.0) <= 1e-14
+
+
+def test_relative_update_zero_update_and_weight_decay():
+    rng = np.random.default_rng(42)
+    W = rng.standard_normal((4, 7))
+    assert np.array_equal(o.relative_update_apply(W, np.zeros_like(W), lr=0.1), W)
+    O = rng.standard_normal((4, 7))
+    d = o.relative_update_apply(W, O, lr=0.1, weight_decay=0.2) - o.relative_update_apply(W, O, lr=0.1)
+    assert np.allclose(d, -0.1 * 0.2 * W, rtol=0, atol=1e-15)
+
+
+# ------------------------------------------------------------------ Adam / AdamH
+def test_adam_first_step_from_zero_state_is_g_over_abs_g():
+    """Bias correction makes step 1 exact: m_hat = g, v_hat = g^2, so U~ = g / (|g| + eps)."""
+    rng = np.random.default_rng(43)
+    G = rng.standard_normal((5, 8)) * 1e-3
+    Mn, Vn, U = o.adam_update(np.zeros_like(G), np.zeros_like(G), G, 1)
+    assert np.allclose(Mn, 0.1 * G, rtol=1e-13, atol=0)        # 1 - 0.9 and 1 - 0.999 in fp64
+    assert np.allclose(Vn, 0.001 * G * G, rtol=1e-13, atol=0)
+    assert np.allclose(U, G / (np.abs(G) + 1e-8), rtol=1e-12, atol=0)
+
+
+def test_adam_constant_gradient_keeps_the_first_direction():
+    """With a constant gradient the corrected moments stay m_hat = g, v_hat = g^2 at every t."""
+    G = np.array([[2.0, -0.5], [1e-3, -4.0]])
+    M = np.zeros_like(G)
+    V = np.zeros_like(G)
+    for t in range(1, 8):
+        M, V, U = o.adam_update(M, V, G, t)
+        assert np.allclose(U, G / (np.abs(G) + 1e-8), rtol=1e-12, atol=0), t
+
+
+def test_adam_two_steps_by_hand():
+    """g = 1 then g = -1 from zero state: m2 = -0.01, v2 = 0.001999, so m_hat = -0.01 / 0.19
+    = -1/19 and v_hat = 0.001999 / (1 - 0.999^2) = 1: U~2 = -(1/19) / (1 + 1e-8)."""
+    M, V, U1 = o.adam_update(np.zeros(1), np.zeros(1), np.ones(1), 1)
+    assert abs(U1[0] - 1.0 / (1.0 + 1e-8)) <= 1e-15
+    M, V, U2 = o.adam_update(M, V, -np.ones(1), 2)
+    assert abs(M[0] + 0.01) <= 1e-17 and abs(V[0] - 0.001999) <= 1e-17
+    assert abs(U2[0] + (1.0 / 19.0) / (1.0 + 1e-8)) <= 1e-14
+
+
+def test_adam_without_averaging_is_elementwise_sign():
+    """beta1 = beta2 = 0: U~ = g / (|g| + eps), the sign of g up to eps, for any history."""
+    rng = np.random.default_rng(44)
+    G = rng.standard_normal((3, 4))
+    _, _, U = o.adam_update(rng.standard_normal((3, 4)), rng.random((3, 4)), G, 5, beta1=0.0, beta2=0.0)
+    assert np.allclose(U, G / (np.abs(G) + 1e-8), rtol=1e-12, atol=0)
+
+
+def test_adamh_step_lands_on_the_sphere_along_the_adam_direction():
+    rng = np.random.default_rng(45)
+    W = 0.02 * rng.standard_normal((16, 24))
+    G = 1e-3 * rng.standard_normal((16, 24))
+    rho = o.fro(W)
+    Wn, Mn, Vn, U, fb = o.adamh_step(W, G, np.zeros_like(W), np.zeros_like(W), t=1, eta=0.02, rho=rho)
+    assert not fb
+    assert abs(o.fro(Wn) - rho) <= 1e-14 * rho
+    # W_new is W - eta * U / ||U|| rescaled: undo the scale and compare the step
+    V = W - 0.02 * U / o.fro(U)
+    assert np.allclose(Wn, rho * V / o.fro(V), rtol=0, atol=1e-15)
+    # first step: U~ = sign(G) up to eps / |g|, so the unit direction has equal-magnitude entries
+    tol = 4e-8 / float(np.min(np.abs(G)))
+    assert np.allclose(np.abs(U / o.fro(U)), 1.0 / np.sqrt(U.size), rtol=tol, atol=0)
