@@ -244,6 +244,140 @@ def run_cuda(args, rank, world, local_rank):
                 clocks=clk.summary(), e2e_ms=e2e_ms, h2d=h2d, d2h=4, n_params=n_params, shp=shp)
 
 
+# ---------------------------------------------------------------------- AdamH
+def run_adamh(args, rank, world, local_rank):
+    """AdamH step (Adam moments + Hyperball) on the same matrix set: timed like run_cuda."""
+    import numpy as np
+    import torch
+    import newton_schulz_hyperball_b200 as nshb
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    shp = shapes()
+    W0, Gh = build_inputs(dev, rank)
+    W = [torch.from_numpy(w).to(dev).to(torch.bfloat16) for w in W0]
+    Gd = [[torch.from_numpy(g).to(dev).to(torch.bfloat16) for g in gs] for gs in Gh]
+    M = [torch.zeros(w.shape, dtype=torch.float32, device=dev) for w in W]
+    V = [torch.zeros(w.shape, dtype=torch.float32, device=dev) for w in W]
+    rho = torch.tensor([float(np.linalg.norm(w.astype(np.float64))) for w in W0], dtype=torch.float32, device=dev)
+    p = nshb.params(eta=ETA, rho=rho)
+    mats = [nshb.matrices(W, Gd[s], M) for s in range(N_GRAD_SETS)]
+    ws = nshb.workspace(mats[0], p, nshb.NSHB_OP_ADAMH, device=dev)
+    n_params = sum(r * c for r, c in shp)
+    count = [0]
+
+    def step(k, m=None):
+        count[0] += 1
+        nshb.adamh_step(m if m is not None else mats[k % N_GRAD_SETS], V, nshb.adam_params(step=count[0]), p, ws,
+                        stream)
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    flags = nshb.device_status(ws, stream)
+    if args.ncu:
+        for k in range(args.steps):
+            step(args.warmup + k)
+        torch.cuda.synchronize()
+        return None
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        e0.record(stream)
+        for k in range(args.steps):
+            step(k)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    nshb.profile_enable(True)
+    nshb.profile_read()
+    kp = max(10, min(args.steps, 50))
+    for k in range(kp):
+        step(k)
+    torch.cuda.synchronize()
+    prof = nshb.profile_read()
+    nshb.profile_enable(False)
+    launches_per_step = sum(c for _, c in prof.values()) / kp
+    Gpin = [[torch.from_numpy(g).to(torch.bfloat16).pin_memory() for g in gs] for gs in Gh[:2]]
+    Gdst = [torch.empty_like(g) for g in Gd[0]]
+    mats_e = nshb.matrices(W, Gdst, M)
+    st_host = torch.empty(1, dtype=torch.int32).pin_memory()
+    h2d = sum(g.numel() * g.element_size() for g in Gpin[0])
+    ke = max(5, min(args.steps, 30))
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(ke):
+        for d, s_ in zip(Gdst, Gpin[k % 2]):
+            d.copy_(s_, non_blocking=True)
+        step(k, mats_e)
+        st_host.copy_(ws[:4].view(torch.int32), non_blocking=True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = t0.elapsed_time(t1) / ke
+    return dict(ms=ms, prof=prof, kp=kp, launches_per_step=launches_per_step, flags=flags,
+                clocks=clk.summary(), e2e_ms=e2e_ms, h2d=h2d, d2h=4, n_params=n_params, shp=shp)
+
+
+def oracle_adamh_sample(layers=1):
+    """Times the oracle's AdamH step on `layers` GPT-2 layers; extrapolated by element count."""
+    import numpy as np
+    from newton_schulz_hyperball_b200 import workloads as wl
+    from oracle import nshb_oracle as o
+    cfg = wl.CFG_GPT2_SMALL
+    shp = shapes()
+    idx = list(range(6 * layers))
+    Ws = {i: wl.init_weight(cfg, i, *shp[i], bf16=True).astype(np.float64) for i in idx}
+    Gs = {i: wl.gradient(cfg, i, 0, *shp[i], bf16=True).astype(np.float64) for i in idx}
+    t0 = time.perf_counter()
+    for i in idx:
+        z = np.zeros(shp[i])
+        o.adamh_step(Ws[i], Gs[i], z, z, t=1, eta=ETA, rho=o.fro(Ws[i]))
+    dt = time.perf_counter() - t0
+    n_all = sum(r * c for r, c in shp)
+    n_s = sum(shp[i][0] * shp[i][1] for i in idx)
+    return dt * n_all / n_s, f"{len(idx)} of 72 matrices (GPT-2 layer 0), 1 step, extrapolated by element count"
+
+
+def report_adamh(args, r, world):
+    peaks, peak_src = load_peaks()
+    prof, kp, n = r["prof"], r["kp"], r["n_params"]
+    adam_ms = prof.get("adam", (0.0, 0))[0] / kp
+    apply_ms = prof.get("apply", (0.0, 0))[0] / kp
+    peak_bw = peaks.get("hbm_gbs", DEFAULT_PEAKS["hbm_gbs"])
+    # Algorithmic HBM bytes: adam 22 B/elem (G 2, M 4+4, V 4+4, W 2, U~ 2), apply 6 (W 2+2, U~ 2).
+    adam_gbs = 22.0 * n / (adam_ms * 1e-3) / 1e9 if adam_ms > 0 else None
+    fused_gbs = 28.0 * n / ((adam_ms + apply_ms) * 1e-3) / 1e9 if adam_ms + apply_ms > 0 else None
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        full, desc = oracle_adamh_sample(1)
+        cpu = {"value": round(full * 1e3, 3), "unit": "ms", "cores": cpu_cores(), "kind": "oracle", "sample": desc}
+    return {
+        "metric": "AdamH optimizer step ms; fused HBM GB/s",
+        "value": round(r["ms"], 4), "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(r["ms"], 4), "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 (bf16 storage)",
+        "data": "synthetic (seeded W0 ~ N(0, 0.02^2), spiked Gaussian gradients; no dataset)",
+        "config": {"workload": "gpt2-small matrix set, AdamH step (72 bf16 matrices, fp32 moments, Hyperball)",
+                   "matrices": len(r["shp"]), "params": n,
+                   "optimizer": "AdamH (0.9, 0.999, 1e-8, eta 0.02, rho = ||W0||)",
+                   "l2": "inputs larger than L2 (W+G+M+V = 1.02 GB per step)", "parallelism": f"replica per GPU x{world}"},
+        "throughput": {"value": round(world * n / (r["ms"] * 1e-3), 1), "unit": "params/s"},
+        "fused_gbs": None if fused_gbs is None else round(fused_gbs, 1),
+        "roofline": {"bound": "hbm", "kernel": "adam_kernel (moments, U~, partials)",
+                     "achieved": None if adam_gbs is None else round(adam_gbs, 1), "peak": peak_bw, "unit": "GB/s",
+                     "frac": None if adam_gbs is None else round(adam_gbs / peak_bw, 4), "traffic": None,
+                     "peak_source": f"{peak_src} copy bandwidth"},
+        "kernels_ms_per_step": {k: round(v[0] / kp, 5) for k, v in prof.items()},
+        "gpu_launches": int(round(r["launches_per_step"] * args.steps)),
+        "device_status": r["flags"], "clocks": r["clocks"],
+        "e2e": {"value": round(r["e2e_ms"], 4), "unit": "ms", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"]},
+        "cpu_baseline": cpu,
+    }
+
+
 # --------------------------------------------------------------- CPU baseline
 def oracle_sample(layers=1, steps=1):
     """Times the fp64 oracle on `layers` of the 12 GPT-2 layers for `steps` steps and returns
@@ -296,6 +430,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--optimizer", default="muonh", choices=["muonh", "adamh"],
+                    help="muonh: the headline MuonH step; adamh: the AdamH step on the same matrices")
     ap.add_argument("--ncu", action="store_true",
                     help="profiling case: warm-up and `steps` steps only, no timing or report")
     args = ap.parse_args()
@@ -332,6 +468,16 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
 
+    if args.optimizer == "adamh":
+        if world > 1:
+            print("--optimizer adamh runs on one GPU", file=sys.stderr)
+            return 2
+        r = run_adamh(args, rank, world, local_rank)
+        if r is None:
+            print("ncu case done", flush=True)
+            return 0
+        print(json.dumps(report_adamh(args, r, world)), flush=True)
+        return 0
     r = run_cuda(args, rank, world, local_rank)
     if r is None:
         print("ncu case done", flush=True)

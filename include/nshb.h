@@ -75,7 +75,9 @@ typedef enum {
   NSHB_OP_HYPERBALL = 1,
   NSHB_OP_RADIAL_BRAKE = 2,
   NSHB_OP_HIMUON = 3,
-  NSHB_OP_NEWTON_MUON = 4
+  NSHB_OP_NEWTON_MUON = 4,
+  NSHB_OP_RELATIVE_UPDATE = 5,
+  NSHB_OP_ADAMH = 6
 } nshb_op;
 
 /* One weight matrix (rows x cols).  W is updated in place, G is read, M is the fp32
@@ -173,6 +175,39 @@ nshb_status newton_muon_step(const nshb_matrix *mats, int32_t n_mats, const void
                              const int64_t *z_rows, int32_t n_z, int64_t n_tokens,
                              const nshb_params *p, void *ws, size_t ws_bytes, nshb_stream stream);
 
+/* Muon step followed by the RelativeUpdate hook (PR #224 file list: a pre-update scaling that
+ * matches the update's norm to the current weight norm):
+ *   W <- (1 - lr wd) W - lr ||W||_F O / max(||O||_F, hb_eps)
+ * (the shape factor of the Muon update cancels in the rescaling; a zero O leaves W scaled by
+ * 1 - lr wd).  Same momentum, NS options and workspace as muon_step (op
+ * NSHB_OP_RELATIVE_UPDATE in nshb_workspace_size). */
+nshb_status relative_update_step(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, void *ws,
+                                 size_t ws_bytes, nshb_stream stream);
+
+/* Adam options of adamh_step.  Defaults (nshb_default_adam_params): the values of "Adam: A
+ * Method for Stochastic Optimization", beta1 0.9, beta2 0.999, eps 1e-8, step 1. */
+typedef struct {
+  float beta1;   /* first-moment coefficient, [0, 1)                                      */
+  float beta2;   /* second-moment coefficient, [0, 1)                                     */
+  float eps;     /* added to sqrt(v_hat), > 0                                             */
+  int32_t step;  /* t >= 1, the step being taken (bias corrections 1 - beta^t)            */
+} nshb_adam_params;
+
+/* Fills *a with the defaults listed above.  Returns NSHB_ERR_NULL if a is NULL. */
+nshb_status nshb_default_adam_params(nshb_adam_params *a);
+
+/* AdamH (Hyperball paper, Method: Hyperball around Adam's preconditioned update):
+ *   M <- beta1 M + (1 - beta1) G;  V <- beta2 V + (1 - beta2) G^2;
+ *   U~ = (M / (1 - beta1^t)) / (sqrt(V / (1 - beta2^t)) + eps);
+ *   W <- rho (W - eta U_hat) / ||W - eta U_hat||_F,  U_hat = U~ / max(||U~||_F, hb_eps),
+ * with the zero-norm fallback and status bits of hyperball_step.  mats[i].M is the fp32 first
+ * moment; V is a HOST array of n_mats DEVICE pointers to the fp32 second moments (same rows,
+ * cols and ld as W, zero before step 1).  U~ is formed in fp32 and kept in w_dtype for the
+ * Hyperball rule.  p supplies eta, rho and hb_eps (the NS fields are not used); O_out, when
+ * set, receives U~.  Workspace: nshb_workspace_size(..., NSHB_OP_ADAMH, ...). */
+nshb_status adamh_step(const nshb_matrix *mats, int32_t n_mats, float *const *V, const nshb_adam_params *a,
+                       const nshb_params *p, void *ws, size_t ws_bytes, nshb_stream stream);
+
 /* out[i] = ||W_i||_F (fp32) into the DEVICE array out (n_mats floats), e.g. rho = ||W0||.
  * Needs a workspace of nshb_workspace_size(..., NSHB_OP_MUON, ...) bytes. */
 nshb_status nshb_fro_norms(const nshb_matrix *mats, int32_t n_mats, float *out, void *ws,
@@ -214,6 +249,7 @@ const char *nshb_status_string(int32_t status);
 #define NSHB_PROF_APPLY 8    /* W <- alpha W + beta O                          */
 #define NSHB_PROF_F32GEMM 9  /* fp32 NS GEMMs (all three phases)               */
 #define NSHB_PROF_NEWTON 10  /* Newton-Muon Gram, Cholesky and solves          */
+#define NSHB_PROF_ADAM 11    /* AdamH moments, direction and partials         */
 #define NSHB_PROF_KINDS 12
 nshb_status nshb_profile_enable(int32_t on);
 nshb_status nshb_profile_read(int32_t n_kinds, float *ms, int32_t *launches);

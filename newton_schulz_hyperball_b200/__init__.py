@@ -20,7 +20,8 @@ from ._abi import (  # noqa: F401  (re-exported constants)
     NSHB_ERR_WORKSPACE, NSHB_ERR_CUDA, NSHB_ERR_DEVICE_TIMEOUT, NSHB_ERR_NONFINITE, NSHB_ERR_ZERO_NORM,
     NSHB_ERR_UNSUPPORTED, NSHB_DEV_ZERO_NORM_FALLBACK, NSHB_DEV_NONFINITE, NSHB_DEV_TIMEOUT,
     NSHB_DEV_ZERO_RADIUS, NSHB_DEV_NOT_SPD, NSHB_OP_MUON, NSHB_OP_HYPERBALL, NSHB_OP_RADIAL_BRAKE,
-    NSHB_OP_HIMUON, NSHB_OP_NEWTON_MUON, nshb_matrix, nshb_params,
+    NSHB_OP_HIMUON, NSHB_OP_NEWTON_MUON, NSHB_OP_RELATIVE_UPDATE, NSHB_OP_ADAMH, nshb_matrix, nshb_params,
+    nshb_adam_params,
 )
 
 _LIB = None
@@ -169,6 +170,30 @@ def radial_brake_step(mats, p, ws, stream=None):
 
 def himuon_step(mats, p, ws, stream=None):
     _step("himuon_step", mats, p, ws, stream)
+
+
+def relative_update_step(mats, p, ws, stream=None):
+    _step("relative_update_step", mats, p, ws, stream)
+
+
+def adam_params(**kw) -> "_abi.nshb_adam_params":
+    """nshb_adam_params with the library defaults (0.9, 0.999, 1e-8, step 1), overridden by keyword."""
+    a = _abi.nshb_adam_params()
+    _check(lib().nshb_default_adam_params(ctypes.byref(a)), "nshb_default_adam_params")
+    for k, v in kw.items():
+        if not hasattr(a, k):
+            raise KeyError(k)
+        setattr(a, k, v)
+    return a
+
+
+def adamh_step(mats, V, a, p, ws, stream=None):
+    """AdamH step; mats[i].M is the first moment, V[i] (CUDA fp32 tensor or pointer) the second."""
+    ptr, nbytes = _ws(ws)
+    n = _n(mats)
+    vp = (ctypes.c_void_p * max(n, 1))(*[_ptr(v) for v in V])
+    _check(lib().adamh_step(mats, n, vp, ctypes.byref(a), ctypes.byref(p), ptr, nbytes, _stream(stream)),
+           "adamh_step")
 
 
 def newton_muon_step(mats, Z, n_tokens: int, p, ws, stream=None):

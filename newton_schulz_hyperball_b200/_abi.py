@@ -30,7 +30,7 @@ NSHB_DEV_ZERO_RADIUS = 0x8
 NSHB_DEV_NOT_SPD = 0x10
 
 NSHB_PROF_NAMES = ["momentum", "norm", "gram", "poly", "update", "reduce", "finalize", "exact", "apply",
-                   "f32gemm", "newton", "spare"]
+                   "f32gemm", "newton", "adam"]
 NSHB_PROF_KINDS = 12
 
 NSHB_OP_MUON = 0
@@ -38,6 +38,8 @@ NSHB_OP_HYPERBALL = 1
 NSHB_OP_RADIAL_BRAKE = 2
 NSHB_OP_HIMUON = 3
 NSHB_OP_NEWTON_MUON = 4
+NSHB_OP_RELATIVE_UPDATE = 5
+NSHB_OP_ADAMH = 6
 
 
 class nshb_matrix(ctypes.Structure):
@@ -76,6 +78,15 @@ class nshb_params(ctypes.Structure):
     ]
 
 
+class nshb_adam_params(ctypes.Structure):
+    _fields_ = [
+        ("beta1", ctypes.c_float),
+        ("beta2", ctypes.c_float),
+        ("eps", ctypes.c_float),
+        ("step", ctypes.c_int32),
+    ]
+
+
 # name -> (restype, argtypes)
 _P = ctypes.c_void_p
 _MATS = ctypes.POINTER(nshb_matrix)
@@ -88,6 +99,10 @@ SIGNATURES = {
     "muon_step": (ctypes.c_int32, [_MATS, ctypes.c_int32, _PAR, _P, ctypes.c_size_t, _P]),
     "hyperball_step": (ctypes.c_int32, [_MATS, ctypes.c_int32, _PAR, _P, ctypes.c_size_t, _P]),
     "radial_brake_step": (ctypes.c_int32, [_MATS, ctypes.c_int32, _PAR, _P, ctypes.c_size_t, _P]),
+    "relative_update_step": (ctypes.c_int32, [_MATS, ctypes.c_int32, _PAR, _P, ctypes.c_size_t, _P]),
+    "nshb_default_adam_params": (ctypes.c_int32, [ctypes.POINTER(nshb_adam_params)]),
+    "adamh_step": (ctypes.c_int32, [_MATS, ctypes.c_int32, ctypes.POINTER(ctypes.c_void_p),
+                                    ctypes.POINTER(nshb_adam_params), _PAR, _P, ctypes.c_size_t, _P]),
     "himuon_step": (ctypes.c_int32, [_MATS, ctypes.c_int32, _PAR, _P, ctypes.c_size_t, _P]),
     "newton_muon_step": (ctypes.c_int32, [_MATS, ctypes.c_int32, ctypes.POINTER(ctypes.c_void_p),
                                           ctypes.POINTER(ctypes.c_int64), ctypes.c_int32, ctypes.c_int64,

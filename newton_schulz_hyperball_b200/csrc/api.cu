@@ -67,7 +67,7 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
   if (!p) return NSHB_ERR_NULL;
   if (n_mats < 0) return NSHB_ERR_SHAPE;
   if (n_mats > 0 && !mats) return NSHB_ERR_NULL;
-  if (op < NSHB_OP_MUON || op > NSHB_OP_NEWTON_MUON) return NSHB_ERR_PARAM;
+  if (op < NSHB_OP_MUON || op > NSHB_OP_RELATIVE_UPDATE) return NSHB_ERR_PARAM;
   if (!(p->beta >= 0.f && p->beta < 1.f)) return NSHB_ERR_PARAM;
   if (p->ns_steps < 1 || p->ns_steps > 32) return NSHB_ERR_PARAM;
   if (!(p->ns_eps > 0.f) || !std::isfinite(p->ns_eps)) return NSHB_ERR_PARAM;
@@ -541,7 +541,8 @@ nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t 
 }
 
 nshb_status run_apply(const nshb_matrix *mats, const Plan &pl, const nshb_params *p, int apply_op, char *ws,
-                      cudaStream_t st, const std::vector<int64_t> &o_off, float *norms_out) {
+                      cudaStream_t st, const std::vector<int64_t> &o_off, float *norms_out,
+                      bool have_partials = false) {
   const int n = (int)pl.mp.size();
   MatScalars *scal = reinterpret_cast<MatScalars *>(ws + pl.scal_off);
   double *wpart = reinterpret_cast<double *>(ws + pl.wpart_off);
@@ -581,9 +582,10 @@ nshb_status run_apply(const nshb_matrix *mats, const Plan &pl, const nshb_params
     }
     fp.blk_begin[c1 - c0] = nb;
     ap.total_blocks = nb;
-    ap.partials = wpart;
-    fp.partials = wpart;
-    if (apply_op != kOpMuon) {
+    // One region for the whole call: chunk c0 uses the partials of its own blocks.
+    ap.partials = wpart + 3 * (int64_t)pl.mp[c0].w_begin;
+    fp.partials = ap.partials;
+    if (apply_op != kOpMuon && !have_partials) {
       NSHB_LAUNCH(NSHB_PROF_REDUCE, launch_reduce(ap, st));
     }
     fp.stage = 0;
@@ -805,8 +807,91 @@ nshb_status do_step(const nshb_matrix *mats, int n_mats, const nshb_params *p, i
   std::vector<int64_t> o_off;
   e = run_ns(pl, p, w, st, o_off);
   if (e != NSHB_OK) return e;
-  const int aop = op == NSHB_OP_MUON ? kOpMuon : op == NSHB_OP_RADIAL_BRAKE ? kOpBrake : kOpHyperball;
+  const int aop = op == NSHB_OP_MUON              ? kOpMuon
+                  : op == NSHB_OP_RADIAL_BRAKE    ? kOpBrake
+                  : op == NSHB_OP_RELATIVE_UPDATE ? kOpRelative
+                                                  : kOpHyperball;
   return run_apply(mats, pl, p, aop, w, st, o_off, nullptr);
+}
+
+// AdamH: no NS.  Per matrix the Adam direction U~ in the layout the apply kernels read as O
+// (bf16 panels of round_up(rows, 64) rows, or fp32 row-major), block partials and the
+// per-matrix scalars.
+nshb_status plan_adamh(const nshb_matrix *mats, int n_mats, float *const *V, const nshb_adam_params *a,
+                       const nshb_params *p, Plan &pl) {
+  if (!p || !a) return NSHB_ERR_NULL;
+  if (n_mats < 0) return NSHB_ERR_SHAPE;
+  if (n_mats > 0 && (!mats || !V)) return NSHB_ERR_NULL;
+  if (!(a->beta1 >= 0.f && a->beta1 < 1.f) || !(a->beta2 >= 0.f && a->beta2 < 1.f)) return NSHB_ERR_PARAM;
+  if (!(a->eps > 0.f) || !std::isfinite(a->eps) || a->step < 1) return NSHB_ERR_PARAM;
+  if (!(p->hb_eps > 0.f) || !std::isfinite(p->hb_eps) || !std::isfinite(p->eta) || p->eta < 0.f)
+    return NSHB_ERR_PARAM;
+  pl.op = NSHB_OP_ADAMH;
+  pl.mp.resize(n_mats);
+  size_t off = kAlign;  // [0, 256): device status word
+  pl.scal_off = off;
+  off = align_up(off + sizeof(MatScalars) * (size_t)n_mats);
+  pl.w_total = 0;
+  for (int i = 0; i < n_mats; ++i) {
+    const nshb_matrix &d = mats[i];
+    MatPlan &m = pl.mp[i];
+    if (d.rows <= 0 || d.cols <= 0 || d.ld < d.cols) return NSHB_ERR_SHAPE;
+    if (d.rows > (1LL << 20) || d.cols > (1LL << 20) || d.ld > (1LL << 30)) return NSHB_ERR_UNSUPPORTED;
+    if (!d.W || !d.G || !d.M || !V[i]) return NSHB_ERR_NULL;
+    if (d.w_dtype != NSHB_BF16 && d.w_dtype != NSHB_F32) return NSHB_ERR_DTYPE;
+    const bool wf32 = d.w_dtype == NSHB_F32;
+    const size_t esz = wf32 ? 4 : 2;
+    const bool vec = ((uintptr_t)d.W % 16 == 0) && ((uintptr_t)d.G % 16 == 0) && ((uintptr_t)d.M % 16 == 0) &&
+                     ((uintptr_t)V[i] % 16 == 0) && ((d.ld * esz) % 16 == 0) && ((d.ld * 4) % 16 == 0);
+    if (d.O_out && ((uintptr_t)d.O_out % esz) != 0) return NSHB_ERR_SHAPE;
+    m.m = d.rows;
+    m.n = d.cols;
+    m.ld = d.ld;
+    m.flags = (vec ? kVec : 0) | (wf32 ? (kWF32 | kNsF32) : 0);   // never transposed
+    m.Rp = round_up(m.m, kBlk);   // bf16 U~: panel height
+    m.s = m.n;                    // fp32 U~: row stride
+    m.w_blocks = (int)(((m.m + kBlk - 1) / kBlk) * ((m.n + kBlk - 1) / kBlk));
+    m.w_begin = pl.w_total;
+    pl.w_total += m.w_blocks;
+  }
+  pl.wpart_off = off;
+  off = align_up(off + 3 * sizeof(double) * (size_t)pl.w_total);
+  for (auto &m : pl.mp) {
+    m.x0 = off;
+    const size_t ub = (m.flags & kWF32) ? (size_t)m.m * m.n * 4 : (size_t)m.Rp * round_up(m.n, kBlk) * 2;
+    off = align_up(off + ub);
+  }
+  pl.total = off;
+  return NSHB_OK;
+}
+
+nshb_status run_adam(const nshb_matrix *mats, const Plan &pl, float *const *V, const nshb_adam_params *a,
+                     char *ws, cudaStream_t st) {
+  const int n = (int)pl.mp.size();
+  double *wpart = reinterpret_cast<double *>(ws + pl.wpart_off);
+  for (int c0 = 0; c0 < n; c0 += kMaxMats) {
+    const int c1 = std::min(n, c0 + kMaxMats);
+    AdamParams ap;
+    std::memset(&ap, 0, sizeof(ap));
+    ap.ws = ws;
+    ap.partials = wpart + 3 * (int64_t)pl.mp[c0].w_begin;
+    ap.status = reinterpret_cast<uint32_t *>(ws);
+    ap.beta1 = a->beta1;
+    ap.beta2 = a->beta2;
+    ap.eps = a->eps;
+    ap.bc1 = (float)(1.0 / (1.0 - std::pow((double)a->beta1, (double)a->step)));
+    ap.bc2 = (float)(1.0 / (1.0 - std::pow((double)a->beta2, (double)a->step)));
+    ap.nmat = c1 - c0;
+    int nb = 0;
+    for (int i = c0; i < c1; ++i) {
+      ap.mats[i - c0] = make_desc(mats[i], pl.mp[i], i, pl.mp[i].x0, nb, false);
+      ap.V[i - c0] = V[i];
+      nb += pl.mp[i].w_blocks;
+    }
+    ap.total_blocks = nb;
+    NSHB_LAUNCH(NSHB_PROF_ADAM, launch_adam(ap, st));
+  }
+  return NSHB_OK;
 }
 
 }  // namespace
@@ -843,6 +928,17 @@ nshb_status nshb_workspace_size(const nshb_matrix *mats, int32_t n_mats, const n
                                 const int64_t *z_rows, int32_t n_z, int64_t n_tokens, size_t *bytes) {
   if (!bytes) return NSHB_ERR_NULL;
   Plan pl;
+  if (op == NSHB_OP_ADAMH) {
+    // The moments' pointers do not change the size: plan with stand-ins for V.
+    nshb_adam_params a;
+    nshb_default_adam_params(&a);
+    if (!p) return NSHB_ERR_NULL;
+    std::vector<float *> vs((size_t)std::max(n_mats, 1), reinterpret_cast<float *>(uintptr_t(256)));
+    nshb_status e = plan_adamh(mats, n_mats, vs.data(), &a, p, pl);
+    if (e != NSHB_OK) return e;
+    *bytes = pl.total;
+    return NSHB_OK;
+  }
   nshb_status e = plan_step(mats, n_mats, p, op, pl);
   if (e != NSHB_OK) return e;
   if (op == NSHB_OP_NEWTON_MUON && n_mats > 0) {
@@ -856,6 +952,38 @@ nshb_status nshb_workspace_size(const nshb_matrix *mats, int32_t n_mats, const n
 nshb_status muon_step(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, void *ws, size_t ws_bytes,
                       nshb_stream stream) {
   return do_step(mats, n_mats, p, NSHB_OP_MUON, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+nshb_status relative_update_step(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, void *ws,
+                                 size_t ws_bytes, nshb_stream stream) {
+  return do_step(mats, n_mats, p, NSHB_OP_RELATIVE_UPDATE, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+nshb_status nshb_default_adam_params(nshb_adam_params *a) {
+  if (!a) return NSHB_ERR_NULL;
+  a->beta1 = 0.9f;
+  a->beta2 = 0.999f;
+  a->eps = 1e-8f;
+  a->step = 1;
+  return NSHB_OK;
+}
+
+nshb_status adamh_step(const nshb_matrix *mats, int32_t n_mats, float *const *V, const nshb_adam_params *a,
+                       const nshb_params *p, void *ws, size_t ws_bytes, nshb_stream stream) {
+  Plan pl;
+  nshb_status e = plan_adamh(mats, n_mats, V, a, p, pl);
+  if (e != NSHB_OK) return e;
+  if (n_mats == 0) return NSHB_OK;
+  e = check_ws(pl, ws, ws_bytes);
+  if (e != NSHB_OK) return e;
+  char *w = static_cast<char *>(ws);
+  cudaStream_t st = (cudaStream_t)stream;
+  NSHB_CHECK_CUDA(cudaMemsetAsync(w, 0, 2 * sizeof(uint32_t), st));  // status word, exact-pass counter
+  e = run_adam(mats, pl, V, a, w, st);
+  if (e != NSHB_OK) return e;
+  std::vector<int64_t> u_off(n_mats);
+  for (int i = 0; i < n_mats; ++i) u_off[i] = pl.mp[i].x0;
+  return run_apply(mats, pl, p, kOpHyperball, w, st, u_off, nullptr, /*have_partials=*/true);
 }
 
 nshb_status hyperball_step(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, void *ws,

@@ -80,7 +80,7 @@ struct MatScalars {
 };
 
 // Reductions over (W, O) blocks and the streaming update W <- alpha W + beta O.
-enum ApplyOp { kOpMuon = 0, kOpHyperball = 1, kOpBrake = 2, kOpNorms = 3 };
+enum ApplyOp { kOpMuon = 0, kOpHyperball = 1, kOpBrake = 2, kOpNorms = 3, kOpRelative = 4 };
 struct ApplyParams {
   char *ws;
   double *partials;        // 3 doubles per block (reduce) or 1 (exact norm)
@@ -102,6 +102,20 @@ struct ApplyFinParams {
   int32_t blk_begin[kMaxMats + 1];
   int32_t mat[kMaxMats];
   int32_t m[kMaxMats], n[kMaxMats];
+};
+
+// AdamH first pass: Adam moments, the direction U~ (kept in the matrix's dtype where the
+// apply kernels read O: bf16 panels, or fp32 row-major with kNsF32) and the
+// (||U~||^2, <W, U~>, ||W||^2) partials of every block.
+struct AdamParams {
+  char *ws;
+  double *partials;        // 3 doubles per block
+  uint32_t *status;
+  float beta1, beta2, eps;
+  float bc1, bc2;          // 1 / (1 - beta1^t), 1 / (1 - beta2^t)
+  int32_t nmat, total_blocks;
+  MatDesc mats[kMaxMats];  // o_off: U~; M: first moment
+  float *V[kMaxMats];      // second moments (same ld as W)
 };
 
 // One bf16 GEMM problem of a Newton-Schulz phase (possibly a batch of equal problems).
@@ -179,6 +193,7 @@ cudaError_t launch_reduce(const ApplyParams &p, cudaStream_t s);
 cudaError_t launch_exact_norm(const ApplyParams &p, cudaStream_t s);
 cudaError_t launch_apply_finalize(const ApplyFinParams &p, cudaStream_t s);
 cudaError_t launch_apply(const ApplyParams &p, cudaStream_t s);
+cudaError_t launch_adam(const AdamParams &p, cudaStream_t s);
 cudaError_t launch_gemm_tc(const GemmParams &p, int bn, int num_sms, cudaStream_t s);
 // 2-SM (CTA pair) form: 256 x 256 tiles, tcgen05.mma.cta_group::2; p.tmap must be encoded.
 cudaError_t launch_gemm_tc2(const GemmParams &p, int num_sms, cudaStream_t s);

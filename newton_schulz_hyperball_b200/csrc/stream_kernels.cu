@@ -661,6 +661,12 @@ __global__ void apply_finalize_kernel(const __grid_constant__ ApplyFinParams p) 
       s.alpha = 1.f; s.beta = 0.f;
       return;
     }
+    if (p.op == kOpRelative) {
+      // RelativeUpdate: the update is rescaled to ||W||, so the step is lr ||W|| O / ||O||.
+      s.alpha = (float)(1.0 - (double)p.lr * (double)p.weight_decay);
+      s.beta = (float)(-(double)p.lr * sqrt(pi) / fmax(sqrt(om), (double)p.hb_eps));
+      return;
+    }
     if (p.op == kOpHyperball) {
       const double nO = fmax(sqrt(om), (double)p.hb_eps);
       s.t = (double)p.eta / nO;
@@ -759,6 +765,82 @@ __global__ void __launch_bounds__(kThreads, F32 ? 2 : 3) apply_kernel(const __gr
   }
 }
 
+// ------------------------------------------------------------------------- AdamH
+// Inputs of one block: G, M, V and W for the thread's two rows.
+struct AdamIn {
+  Raw8 g[2], m[2], v[2], w[2];
+};
+
+template <bool F32>
+__device__ __forceinline__ void adam_block(const AdamParams &p, const MatDesc &d, const float *V, int blk, int r0,
+                                           int c0, double (*red)[3 * kWarps], int &nred) {
+  const int rq = threadIdx.x >> 3, cq = (threadIdx.x & 7) * 8;
+  const bool f32 = F32 && (d.flags & kWF32), vec = d.flags & kVec;
+  AdamIn in;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int i = r0 + rq + 32 * h, j = c0 + cq;
+    raw_load8(d.G, d.ld, i, j, d.m, d.n, f32, vec, in.g[h]);
+    raw_load8(d.M, d.ld, i, j, d.m, d.n, true, vec, in.m[h]);
+    raw_load8(V, d.ld, i, j, d.m, d.n, true, vec, in.v[h]);
+    raw_load8(d.W, d.ld, i, j, d.m, d.n, f32, vec, in.w[h]);
+  }
+  const float b1 = p.beta1, b2 = p.beta2, omb1 = 1.0f - p.beta1, omb2 = 1.0f - p.beta2;
+  float om = 0.f, de = 0.f, pi = 0.f;
+  char *ubase = p.ws + d.o_off;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int i = r0 + rq + 32 * h, j = c0 + cq;
+    float g[8], mm[8], vv[8], w[8], u[8];
+    raw_cvt8(in.g[h], f32, g);
+    raw_cvt8(in.m[h], true, mm);
+    raw_cvt8(in.v[h], true, vv);
+    raw_cvt8(in.w[h], f32, w);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      // Outside the matrix g = m = v = 0, so u = 0 there without masking.
+      mm[e] = fmaf(b1, mm[e], omb1 * g[e]);
+      vv[e] = fmaf(b2, vv[e], omb2 * g[e] * g[e]);
+      const float uf = (mm[e] * p.bc1) / (sqrtf(vv[e] * p.bc2) + p.eps);
+      u[e] = uf;
+      const float us = f32 ? uf : bf16_round(uf);   // what the apply kernels will read
+      om = fmaf(us, us, om);
+      de = fmaf(w[e], us, de);
+      pi = fmaf(w[e], w[e], pi);
+    }
+    store8(d.M, d.ld, i, j, d.m, d.n, true, vec, mm);
+    store8(const_cast<float *>(V), d.ld, i, j, d.m, d.n, true, vec, vv);
+    x_store8(ubase, d, i, j, u, F32);
+  }
+  const float a3[3] = {om, de, pi};
+  double s[3];
+  cta_sum<3>(a3, s, red, nred & 1);
+  ++nred;
+  if (threadIdx.x == 0) {
+    p.partials[3 * (int64_t)blk + 0] = s[0];
+    p.partials[3 * (int64_t)blk + 1] = s[1];
+    p.partials[3 * (int64_t)blk + 2] = s[2];
+  }
+}
+
+template <bool F32>
+__global__ void __launch_bounds__(kThreads, 2) adam_kernel(const __grid_constant__ AdamParams p) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ double red[2][3 * kWarps];
+  int blk = blockIdx.x;
+  if (blk >= p.total_blocks) return;
+  int mi = find_mat(p, blk);
+  int nred = 0;
+  for (; blk < p.total_blocks; blk += gridDim.x) {
+    mi = advance_mat(p, mi, blk);
+    const MatDesc &d = p.mats[mi];
+    int r0, c0;
+    block_origin(d, blk - d.blk_begin, r0, c0);
+    adam_block<F32>(p, d, p.V[mi], blk, r0, c0, red, nred);
+  }
+}
+
 // Persistent grid: the SM count times the CTAs of `kernel` that fit on one SM with
 // `dyn_smem` bytes of dynamic shared memory, capped by the work.  Queried once per
 // kernel and device.
@@ -819,6 +901,15 @@ cudaError_t launch_exact_norm(const ApplyParams &p, cudaStream_t s) {
 }
 cudaError_t launch_apply_finalize(const ApplyFinParams &p, cudaStream_t s) {
   if (p.nmat > 0) return launch_pdl(apply_finalize_kernel, (p.nmat + 3) / 4, 128, 0, s, p);
+  return cudaGetLastError();
+}
+cudaError_t launch_adam(const AdamParams &p, cudaStream_t s) {
+  if (p.total_blocks > 0) {
+    if (needs_f32(p))
+      return launch_pdl(adam_kernel<true>, stream_grid(adam_kernel<true>, 6, 0, p.total_blocks), kThreads, 0, s, p);
+    else
+      return launch_pdl(adam_kernel<false>, stream_grid(adam_kernel<false>, 7, 0, p.total_blocks), kThreads, 0, s, p);
+  }
   return cudaGetLastError();
 }
 cudaError_t launch_apply(const ApplyParams &p, cudaStream_t s) {

@@ -145,3 +145,26 @@ def test_zero_matrices_is_a_no_op():
     lib = nshb.lib()
     p = nshb.params()
     assert lib.hyperball_step(None, 0, ctypes.byref(p), None, 0, None) == nshb.NSHB_OK
+
+
+def test_adam_params_layout_defaults_and_argument_errors():
+    assert ctypes.sizeof(_abi.nshb_adam_params) == 16
+    a = nshb.adam_params()
+    assert abs(a.beta1 - 0.9) < 1e-7 and abs(a.beta2 - 0.999) < 1e-7 and abs(a.eps - 1e-8) < 1e-13 and a.step == 1
+    mats = fake_mats([(64, 64), (100, 30)])
+    p = nshb.params()
+    n = nshb.workspace_size(mats, p, nshb.NSHB_OP_ADAMH)
+    assert n > 0
+    assert nshb.workspace_size(mats, p, nshb.NSHB_OP_RELATIVE_UPDATE) == nshb.workspace_size(mats, p, nshb.NSHB_OP_MUON)
+    V = [0x30000000, 0x31000000]
+    ws = (0x40000000, n)
+    for bad in (dict(step=0), dict(beta1=1.0), dict(beta2=-0.1), dict(eps=0.0)):
+        with pytest.raises(nshb.NshbError) as e:
+            nshb.adamh_step(mats, V, nshb.adam_params(**bad), p, ws, stream=0)
+        assert e.value.status == nshb.NSHB_ERR_PARAM
+    with pytest.raises(nshb.NshbError) as e:
+        nshb.adamh_step(mats, [0x30000000, None], a, p, ws, stream=0)
+    assert e.value.status == nshb.NSHB_ERR_NULL
+    with pytest.raises(nshb.NshbError) as e:
+        nshb.adamh_step(mats, V, a, p, (0x40000000, n - 256), stream=0)
+    assert e.value.status == nshb.NSHB_ERR_WORKSPACE
