@@ -208,6 +208,20 @@ nshb_status nshb_default_adam_params(nshb_adam_params *a);
 nshb_status adamh_step(const nshb_matrix *mats, int32_t n_mats, float *const *V, const nshb_adam_params *a,
                        const nshb_params *p, void *ws, size_t ws_bytes, nshb_stream stream);
 
+/* Memory-bounded steps (Hierarchical Muon's scaling note: the work is independent per tile, so
+ * it can be processed in pieces).  nshb_step_chunked runs the step of kind `op` (NSHB_OP_MUON,
+ * _HYPERBALL, _RADIAL_BRAKE, _HIMUON or _RELATIVE_UPDATE) over mats[0..n_mats) in consecutive
+ * chunks, each as long as fits in ws_bytes, one after the other on `stream`; p->rho (when set)
+ * is indexed like mats.  Every matrix's result is the one the unchunked call computes.  The
+ * step's device status word is that of the last chunk: read it per chunk, or use one chunk,
+ * when the flags matter.  *n_chunks (optional) receives the number of chunks.
+ * nshb_workspace_size_min gives the smallest workspace it accepts (the largest single-matrix
+ * need); a smaller one returns NSHB_ERR_WORKSPACE before anything is queued. */
+nshb_status nshb_workspace_size_min(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, int32_t op,
+                                    size_t *bytes);
+nshb_status nshb_step_chunked(int32_t op, const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, void *ws,
+                              size_t ws_bytes, nshb_stream stream, int32_t *n_chunks);
+
 /* out[i] = ||W_i||_F (fp32) into the DEVICE array out (n_mats floats), e.g. rho = ||W0||.
  * Needs a workspace of nshb_workspace_size(..., NSHB_OP_MUON, ...) bytes. */
 nshb_status nshb_fro_norms(const nshb_matrix *mats, int32_t n_mats, float *out, void *ws,

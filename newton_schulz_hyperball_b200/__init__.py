@@ -172,6 +172,23 @@ def himuon_step(mats, p, ws, stream=None):
     _step("himuon_step", mats, p, ws, stream)
 
 
+def workspace_size_min(mats, p, op: int) -> int:
+    """Smallest workspace step_chunked accepts for these matrices (the largest single matrix's need)."""
+    out = ctypes.c_size_t(0)
+    _check(lib().nshb_workspace_size_min(mats, _n(mats), ctypes.byref(p), op, ctypes.byref(out)),
+           "nshb_workspace_size_min")
+    return out.value
+
+
+def step_chunked(op: int, mats, p, ws, stream=None) -> int:
+    """The step of kind `op` over the matrices in chunks that fit the workspace; returns the chunk count."""
+    ptr, nbytes = _ws(ws)
+    n = ctypes.c_int32(0)
+    _check(lib().nshb_step_chunked(op, mats, _n(mats), ctypes.byref(p), ptr, nbytes, _stream(stream),
+                                   ctypes.byref(n)), "nshb_step_chunked")
+    return n.value
+
+
 def relative_update_step(mats, p, ws, stream=None):
     _step("relative_update_step", mats, p, ws, stream)
 

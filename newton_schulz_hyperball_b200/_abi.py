@@ -107,6 +107,10 @@ SIGNATURES = {
     "newton_muon_step": (ctypes.c_int32, [_MATS, ctypes.c_int32, ctypes.POINTER(ctypes.c_void_p),
                                           ctypes.POINTER(ctypes.c_int64), ctypes.c_int32, ctypes.c_int64,
                                           _PAR, _P, ctypes.c_size_t, _P]),
+    "nshb_workspace_size_min": (ctypes.c_int32, [_MATS, ctypes.c_int32, _PAR, ctypes.c_int32,
+                                                 ctypes.POINTER(ctypes.c_size_t)]),
+    "nshb_step_chunked": (ctypes.c_int32, [ctypes.c_int32, _MATS, ctypes.c_int32, _PAR, _P, ctypes.c_size_t, _P,
+                                           ctypes.POINTER(ctypes.c_int32)]),
     "nshb_fro_norms": (ctypes.c_int32, [_MATS, ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]),
     "nshb_fro_norms_static": (ctypes.c_int32, [_MATS, ctypes.c_int32, _P, _P]),
     "nshb_device_status": (ctypes.c_int32, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),

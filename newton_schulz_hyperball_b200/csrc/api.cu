@@ -1026,6 +1026,74 @@ nshb_status newton_muon_step(const nshb_matrix *mats, int32_t n_mats, const void
   return run_apply(mats, pl, p, kOpHyperball, w, st, o_off, nullptr);
 }
 
+static bool chunkable_op(int32_t op) {
+  return op == NSHB_OP_MUON || op == NSHB_OP_HYPERBALL || op == NSHB_OP_RADIAL_BRAKE || op == NSHB_OP_HIMUON ||
+         op == NSHB_OP_RELATIVE_UPDATE;
+}
+
+nshb_status nshb_workspace_size_min(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, int32_t op,
+                                    size_t *bytes) {
+  if (!bytes) return NSHB_ERR_NULL;
+  if (!chunkable_op(op)) return NSHB_ERR_PARAM;
+  size_t best = 0;
+  for (int i = 0; i < n_mats; ++i) {
+    Plan pl;
+    const nshb_status e = plan_step(mats + i, 1, p, op, pl);
+    if (e != NSHB_OK) return e;
+    best = std::max(best, pl.total);
+  }
+  if (n_mats == 0) {
+    Plan pl;
+    const nshb_status e = plan_step(mats, 0, p, op, pl);
+    if (e != NSHB_OK) return e;
+  }
+  *bytes = best;
+  return NSHB_OK;
+}
+
+nshb_status nshb_step_chunked(int32_t op, const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, void *ws,
+                              size_t ws_bytes, nshb_stream stream, int32_t *n_chunks) {
+  if (!chunkable_op(op)) return NSHB_ERR_PARAM;
+  Plan all;
+  nshb_status e = plan_step(mats, n_mats, p, op, all);   // validates every argument before any launch
+  if (e != NSHB_OK) return e;
+  if (!ws) return NSHB_ERR_NULL;
+  if ((uintptr_t)ws % kAlign != 0) return NSHB_ERR_WORKSPACE;
+  // Chunk boundaries first (host only), so that a workspace too small for some matrix
+  // is reported before anything is queued.
+  std::vector<int> starts;
+  auto fits = [&](int i, int k) {
+    Plan pl;
+    return plan_step(mats + i, k, p, op, pl) == NSHB_OK && pl.total <= ws_bytes;
+  };
+  for (int i = 0; i < n_mats;) {
+    if (!fits(i, 1)) return NSHB_ERR_WORKSPACE;
+    int lo = 1, hi = 1;                        // largest k with fits(i, k): doubling, then bisection
+    while (i + hi < n_mats && fits(i, std::min(2 * hi, n_mats - i))) hi = std::min(2 * hi, n_mats - i);
+    if (i + hi < n_mats) {
+      lo = hi;
+      int up = std::min(2 * hi, n_mats - i);   // fits(i, up) is false
+      while (up - lo > 1) {
+        const int mid = (lo + up) / 2;
+        if (fits(i, mid)) lo = mid; else up = mid;
+      }
+      hi = lo;
+    }
+    starts.push_back(i);
+    i += hi;
+  }
+  starts.push_back(n_mats);
+  if (n_chunks) *n_chunks = (int32_t)starts.size() - 1;
+  for (size_t c = 0; c + 1 < starts.size(); ++c) {
+    const int i = starts[c], k = starts[c + 1] - starts[c];
+    nshb_params pc = *p;
+    if (p->rho) pc.rho = p->rho + i;           // the radii of this chunk's matrices
+    e = do_step(mats + i, k, &pc, op, ws, ws_bytes, (cudaStream_t)stream);
+    if (e != NSHB_OK) return e;
+  }
+  return NSHB_OK;
+}
+
 nshb_status nshb_fro_norms(const nshb_matrix *mats, int32_t n_mats, float *out, void *ws, size_t ws_bytes,
                            nshb_stream stream) {
   if (!out && n_mats > 0) return NSHB_ERR_NULL;

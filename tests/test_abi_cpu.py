@@ -168,3 +168,23 @@ def test_adam_params_layout_defaults_and_argument_errors():
     with pytest.raises(nshb.NshbError) as e:
         nshb.adamh_step(mats, V, a, p, (0x40000000, n - 256), stream=0)
     assert e.value.status == nshb.NSHB_ERR_WORKSPACE
+
+
+def test_chunked_step_workspace_bounds_are_checked_before_any_launch():
+    mats = fake_mats([(768, 768), (3072, 768), (768, 3072), (256, 512)])
+    p = nshb.params()
+    full = nshb.workspace_size(mats, p, nshb.NSHB_OP_HYPERBALL)
+    least = nshb.workspace_size_min(mats, p, nshb.NSHB_OP_HYPERBALL)
+    assert 0 < least < full
+    one = [nshb.workspace_size(fake_mats([s]), p, nshb.NSHB_OP_HYPERBALL)
+           for s in [(768, 768), (3072, 768), (768, 3072), (256, 512)]]
+    assert least == max(one)
+    with pytest.raises(nshb.NshbError) as e:
+        nshb.step_chunked(nshb.NSHB_OP_HYPERBALL, mats, p, (0x40000000, least - 256), stream=0)
+    assert e.value.status == nshb.NSHB_ERR_WORKSPACE
+    with pytest.raises(nshb.NshbError) as e:
+        nshb.step_chunked(nshb.NSHB_OP_NEWTON_MUON, mats, p, (0x40000000, full), stream=0)
+    assert e.value.status == nshb.NSHB_ERR_PARAM
+    with pytest.raises(nshb.NshbError) as e:
+        nshb.workspace_size_min(mats, p, nshb.NSHB_OP_ADAMH)
+    assert e.value.status == nshb.NSHB_ERR_PARAM
