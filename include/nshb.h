@@ -60,7 +60,7 @@ typedef enum {
   NSHB_ERR_DEVICE_TIMEOUT = 7, /* (device status) a bounded wait inside a kernel ran out      */
   NSHB_ERR_NONFINITE = 8,      /* (device status) a NaN/Inf norm was met                      */
   NSHB_ERR_ZERO_NORM = 9,      /* (device status) radius taken from a zero weight norm        */
-  NSHB_ERR_UNSUPPORTED = 10    /* operation/size not supported by this build                  */
+  NSHB_ERR_UNSUPPORTED = 10    /* operation/size not supported by the library                */
 } nshb_status;
 
 /* Bits of the device status word (nshb_device_status). */
