@@ -24,6 +24,11 @@ constexpr long long kWaitLimitTest = 2000000LL; // ~1 ms (debug_flags bit 0)
 constexpr float kKeller[3] = {3.4445f, -4.7750f, 2.0315f};
 
 size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+// Matrices whose wide side has fewer rows than this run their NS in fp32 even on the bf16
+// path: the tensor-core chain would pad them to 256-row panels, and with so few singular
+// values the bf16 rounding of B (amplified by the a + B cancellation near sigma = 1) is not
+// averaged over a spectrum (a rank-1 input is 5 % off in bf16).
+constexpr int64_t kSmallNsF32 = 32;
 int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 struct MatPlan {
@@ -34,6 +39,7 @@ struct MatPlan {
   int flags = 0;
   int64_t x0 = 0, x1 = 0, a = 0, b = 0;   // workspace offsets
   int64_t xl0 = -1, xl1 = -1;             // bf16 low parts of X0 / X1 (compensated iterations)
+  bool f32 = false;              // NS in fp32 (CUDA cores) for this matrix
   int T = 0, tiles_r = 0, tiles_c = 0, ntiles = 0;
   int seg_begin = 0, nseg = 0;
   int pr = 0, pc = 0;            // momentum block domain (W coordinates)
@@ -113,7 +119,8 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
     const bool vec = ((uintptr_t)d.W % 16 == 0) && ((uintptr_t)d.G % 16 == 0) && ((uintptr_t)d.M % 16 == 0) &&
                      ((d.ld * esz) % 16 == 0) && ((d.ld * 4) % 16 == 0);
     if (d.O_out && ((uintptr_t)d.O_out % esz) != 0) return NSHB_ERR_SHAPE;
-    m.flags = (vec ? kVec : 0) | (wf32 ? kWF32 : 0) | (pl.f32ns ? kNsF32 : 0);
+    m.f32 = pl.f32ns || (!pl.tiled && std::min(d.rows, d.cols) < kSmallNsF32);
+    m.flags = (vec ? kVec : 0) | (wf32 ? kWF32 : 0) | (m.f32 ? kNsF32 : 0);
     if (pl.tiled) {
       m.flags |= kTiled;
       m.T = p->tile;
@@ -128,7 +135,7 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
       if (m.tall) m.flags |= kTall;
       m.r = m.tall ? m.n : m.m;
       m.s = m.tall ? m.m : m.n;
-      if (pl.f32ns) {
+      if (m.f32) {
         m.pr = (int)round_up(m.m, kBlk);
         m.pc = (int)round_up(m.n, kBlk);
       } else {
@@ -170,7 +177,7 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
     if (pl.tiled) {
       xb = (size_t)m.ntiles * m.T * m.T * 2;
       ab = xb;
-    } else if (pl.f32ns) {
+    } else if (m.f32) {
       xb = (size_t)m.r * m.s * 4;
       ab = (size_t)m.r * m.r * 4;
     } else {
@@ -181,7 +188,7 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
     m.x1 = off; off = align_up(off + xb);
     m.a = off;  off = align_up(off + ab);
     m.b = off;  off = align_up(off + ab);
-    if (pl.comp > 0) {
+    if (pl.comp > 0 && !m.f32) {
       m.xl0 = off; off = align_up(off + xb);
       if (pl.comp > 1) { m.xl1 = off; off = align_up(off + xb); }
     }
@@ -419,14 +426,17 @@ nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t 
   const float *scales = reinterpret_cast<const float *>(ws + pl.scale_off);
   uint32_t *status = reinterpret_cast<uint32_t *>(ws);
   const long long limit = (p->debug_flags & 1u) ? kWaitLimitTest : kWaitLimit;
+  std::vector<int> f32_idx, bf_idx;   // matrices whose NS runs in fp32 / on the bf16 tensor cores
+  for (int i = 0; i < n; ++i) (pl.mp[i].f32 ? f32_idx : bf_idx).push_back(i);
   for (int it = 0; it < p->ns_steps; ++it) {
     float ca, cb, cc;
     coeffs_for(p, it, ca, cb, cc);
     for (int phase = 0; phase < 3; ++phase) {
       const int mode = phase == 0 ? kGram : phase == 1 ? kPoly : kUpdate;
-      if (pl.f32ns) {
-        for (int c0 = 0; c0 < n; c0 += kMaxProb) {
-          const int c1 = std::min(n, c0 + kMaxProb);
+      {
+        const int nf = (int)f32_idx.size();
+        for (int c0 = 0; c0 < nf; c0 += kMaxProb) {
+          const int c1 = std::min(nf, c0 + kMaxProb);
           F32Params fp;
           std::memset(&fp, 0, sizeof(fp));
           fp.ws = ws;
@@ -434,10 +444,10 @@ nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t 
           fp.mode = mode;
           fp.ca = ca; fp.cb = cb; fp.cc = cc;
           int tiles = 0;
-          for (int i = c0; i < c1; ++i) {
-            const MatPlan &m = pl.mp[i];
+          for (int ii = c0; ii < c1; ++ii) {
+            const MatPlan &m = pl.mp[f32_idx[ii]];
             const int64_t xin = (it % 2 == 0) ? m.x0 : m.x1, xout = (it % 2 == 0) ? m.x1 : m.x0;
-            F32Prob &q = fp.prob[i - c0];
+            F32Prob &q = fp.prob[ii - c0];
             if (mode == kGram) {
               q.a_off = xin; q.b_off = xin; q.c_off = m.a; q.d_off = m.a;
               q.M = (int)m.r; q.N = (int)m.r; q.K = (int)m.s;
@@ -460,9 +470,11 @@ nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t 
           fp.total_tiles = tiles;
           NSHB_LAUNCH(NSHB_PROF_F32GEMM, launch_gemm_f32(fp, st));
         }
-      } else {
-        for (int c0 = 0; c0 < n; c0 += kMaxProb) {
-          const int c1 = std::min(n, c0 + kMaxProb);
+      }
+      {
+        const int nb = (int)bf_idx.size();
+        for (int c0 = 0; c0 < nb; c0 += kMaxProb) {
+          const int c1 = std::min(nb, c0 + kMaxProb);
           GemmParams gp;
           std::memset(&gp, 0, sizeof(gp));
           gp.ws = ws;
@@ -474,7 +486,8 @@ nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t 
           gp.ca = ca; gp.cb = cb; gp.cc = cc;
           // Longest-k problems first, so the static tile walk ends evenly.
           std::vector<std::pair<int64_t, int>> ord;
-          for (int i = c0; i < c1; ++i) {
+          for (int ii = c0; ii < c1; ++ii) {
+            const int i = bf_idx[ii];
             const MatPlan &m = pl.mp[i];
             const int64_t kext = pl.tiled ? m.T : (mode == kGram ? m.Sp : m.Rp);
             ord.push_back({-kext, i});

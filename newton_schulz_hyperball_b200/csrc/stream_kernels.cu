@@ -824,7 +824,7 @@ __device__ __forceinline__ void adam_block(const AdamParams &p, const MatDesc &d
 }
 
 template <bool F32>
-__global__ void __launch_bounds__(kThreads, 2) adam_kernel(const __grid_constant__ AdamParams p) {
+__global__ void __launch_bounds__(kThreads, F32 ? 2 : 3) adam_kernel(const __grid_constant__ AdamParams p) {
   pdl_trigger();
   pdl_wait();
   __shared__ double red[2][3 * kWarps];

@@ -505,3 +505,55 @@ def test_thirteen_shapes_in_one_call():
     assert single.step("muon", nshb.params(lr=0.0)) == 0
     for i in range(2):
         assert rel_fro(single.host()[2][i], Og[i]) <= 2e-2
+
+
+# ------------------------------------------------------------------ degenerate inputs
+@pytest.mark.parametrize("shape", [(1, 1), (1, 9), (9, 1), (1, 300), (300, 1)])
+def test_bf16_degenerate_shapes_hyperball(shape):
+    """Single rows, columns and scalars on the tensor-core path (padded to 256 inside): a
+    rank-1 U has one singular value, normalised to 1, mapped by the scalar polynomial."""
+    cfg = 26
+    W = wl.init_weight(cfg, 0, *shape, bf16=True).astype(np.float64)
+    G = wl.gradient(cfg, 0, 0, *shape, bf16=True).astype(np.float64)
+    rho = o.fro(W)
+    gs = GpuSet([W], bf16=True)
+    gs.set_grads([G])
+    rho_dev = torch.tensor([rho], dtype=torch.float32, device="cuda")
+    assert gs.step("hyperball", nshb.params(eta=0.02, rho=rho_dev)) == 0
+    Wg, Mg, Og = gs.host()
+    Wr, Mr, Or, fb = o.hyperball_step(W, G, np.zeros_like(W), eta=0.02, rho=rho)
+    assert rel_fro(Mg[0], Mr) <= 1e-6
+    assert rel_fro(Og[0], Or) <= 2e-2
+    assert np.linalg.norm(Wg[0] - Wr) <= bf16_w_tol(Wr, 0.02)
+    # the single stretch of a rank-1 U is the scalar map of ||U|| / (||U|| + eps)
+    _, U = o.momentum(np.zeros_like(G), G, 0.95, True)
+    s = np.linalg.svd(Og[0], compute_uv=False)[0]
+    assert abs(s - float(o.scalar_ns(o.fro(U) / (o.fro(U) + o.NS_EPS), 5))) <= 2e-2
+
+
+def test_zero_gradient_leaves_weights_on_their_sphere():
+    """G = 0: U = 0, the NS output is 0 (0 / (0 + eps)), U_hat = 0, and W <- rho W / ||W||."""
+    shapes = [(256, 256), (768, 3072), (5, 7)]
+    Ws = [wl.init_weight(27, i, r, c, bf16=True).astype(np.float64) for i, (r, c) in enumerate(shapes)]
+    gs = GpuSet(Ws, bf16=True)
+    gs.set_grads([np.zeros_like(w) for w in Ws])
+    rho = torch.tensor([o.fro(w) for w in Ws], dtype=torch.float32, device="cuda")
+    assert gs.step("hyperball", nshb.params(eta=0.02, rho=rho)) == 0
+    Wg, Mg, Og = gs.host()
+    for i, W in enumerate(Ws):
+        assert not np.any(Og[i]) and not np.any(Mg[i])
+        Wr, fb = o.hyperball_apply(W, np.zeros_like(W), 0.02, o.fro(W))
+        assert not fb
+        assert np.linalg.norm(Wg[i] - Wr) <= bf16_w_tol(Wr, 0.0), i
+
+
+def test_zero_weight_with_current_norm_as_radius_reports_zero_radius():
+    """rho taken from the current norm (NULL rho) of an all-zero W: the hook's error case;
+    here the status bit NSHB_DEV_ZERO_RADIUS is set and W stays zero."""
+    W = np.zeros((128, 256))
+    G = wl.gradient(28, 0, 0, 128, 256, bf16=True).astype(np.float64)
+    gs = GpuSet([W], bf16=True)
+    gs.set_grads([G])
+    flags = gs.step("hyperball", nshb.params(eta=0.02))
+    assert flags & nshb.NSHB_DEV_ZERO_RADIUS
+    assert not np.any(gs.host()[0][0])
