@@ -42,6 +42,22 @@ GEMM_SOURCE = os.path.join(ROOT, "newton_schulz_hyperball_b200", "csrc", "ns_tc2
 GEMM_TRAFFIC = {"sha256_prefix": "5487563383b5abda", "bytes_per_launch": 372400725}
 
 
+# DRAM read + write per launch of adam_kernel from the capture summarised in
+# profiles/adam_kernel_gpt2_small_step.md, valid only for the source it was taken on.
+STREAM_SOURCE = os.path.join(ROOT, "newton_schulz_hyperball_b200", "csrc", "stream_kernels.cu")
+ADAM_TRAFFIC = {"sha256_prefix": "df0ca9588b2f3a9d", "bytes_per_launch": 1814096720}
+
+
+def source_traffic(path, rec):
+    import hashlib
+    try:
+        with open(path, "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return rec["bytes_per_launch"] if h == rec["sha256_prefix"] else None
+
+
 def gemm_traffic():
     import hashlib
     try:
@@ -385,7 +401,8 @@ def report_adamh(args, r, world):
         "fused_gbs": None if fused_gbs is None else round(fused_gbs, 1),
         "roofline": {"bound": "hbm", "kernel": "adam_kernel (moments, U~, partials)",
                      "achieved": None if adam_gbs is None else round(adam_gbs, 1), "peak": peak_bw, "unit": "GB/s",
-                     "frac": None if adam_gbs is None else round(adam_gbs / peak_bw, 4), "traffic": None,
+                     "frac": None if adam_gbs is None else round(adam_gbs / peak_bw, 4),
+                     "traffic": source_traffic(STREAM_SOURCE, ADAM_TRAFFIC),
                      "peak_source": f"{peak_src} copy bandwidth"},
         "kernels_ms_per_step": {k: round(v[0] / kp, 5) for k, v in prof.items()},
         "gpu_launches": int(round(r["launches_per_step"] * args.steps)),
