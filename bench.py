@@ -413,6 +413,125 @@ def report_adamh(args, r, world):
     }
 
 
+# ------------------------------------------------------------ other configurations
+CONFIGS = {
+    "qwen3": "Qwen3-style 1.4B matrix set (196 matrices), MuonH step",
+    "himuon8b": "8B-width matrix set (224 matrices, 6.98B params), Hierarchical Muon T=256 + Hyperball step",
+    "newton": "GPT-2-small matrix set, Newton-Muon step (48 layer inputs of 8192 tokens) + Hyperball",
+}
+
+
+def device_set(shapes, cfg, dev, torch):
+    """W ~ N(0, 0.02^2) and G = sigma (E + (10/sqrt 8) A B^T) drawn on the device with a seeded
+    generator (sigma per matrix from the host recipe); bf16."""
+    from newton_schulz_hyperball_b200 import workloads as wl
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 + cfg)
+    W, G = [], []
+    for i, (r, c) in enumerate(shapes):
+        W.append((0.02 * torch.randn(r, c, device=dev, generator=g)).to(torch.bfloat16))
+        a = torch.randn(r, 8, device=dev, generator=g)
+        b = torch.randn(c, 8, device=dev, generator=g)
+        e = torch.randn(r, c, device=dev, generator=g)
+        G.append((wl.grad_sigma(cfg, i) * (e + (10 / 8 ** 0.5) * (a @ b.T))).to(torch.bfloat16))
+        del a, b, e
+    return W, G
+
+
+def run_config(args):
+    """One of the larger configurations: step ms and algorithmic tensor-core TFLOP/s (1 GPU)."""
+    import numpy as np
+    import torch
+    import newton_schulz_hyperball_b200 as nshb
+    from newton_schulz_hyperball_b200 import workloads as wl
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    Z = None
+    if args.config == "qwen3":
+        cfg = wl.CFG_QWEN3_1B
+        named = wl.qwen3_1b_shapes(28)
+        shp = [(r, c) for _, r, c in named]
+        op, fn, flops = nshb.NSHB_OP_HYPERBALL, "hyperball_step", ns_flops(shp)
+        extra = {}
+    elif args.config == "himuon8b":
+        cfg = wl.CFG_8B_WIDTH
+        named = wl.width_8b_shapes(32)
+        shp = [(r, c) for _, r, c in named]
+        T = 256
+        op, fn, flops = nshb.NSHB_OP_HIMUON, "himuon_step", sum(20.0 * r * c * T for r, c in shp)
+        extra = {"tile": T}
+    else:
+        cfg = wl.CFG_NEWTON_GPT2
+        named = wl.gpt2_small_shapes(12)
+        shp = [(r, c) for _, r, c in named]
+        zi, zrows = wl.newton_gpt2_z_index(named)
+        n_tok = 8192
+        g = torch.Generator(device=dev)
+        g.manual_seed(2000 + cfg)
+        Z = []
+        for d in zrows:     # Z = diag(e^u) E, u ~ U(ln 0.1, ln 10), E ~ N(0, 1)
+            u = torch.empty(d, 1, device=dev).uniform_(float(np.log(0.1)), float(np.log(10.0)), generator=g)
+            Z.append((torch.exp(u) * torch.randn(d, n_tok, device=dev, generator=g)).to(torch.bfloat16))
+        syrk = sum(float(d) * d * n_tok for d in zrows)   # Z Z^T, symmetric half
+        op, fn, flops = nshb.NSHB_OP_NEWTON_MUON, "newton_muon_step", ns_flops(shp) + syrk
+        extra = {"z_inputs": len(zrows), "tokens": n_tok, "syrk_tflop": round(syrk / 1e12, 3)}
+    W, G = device_set(shp, cfg, dev, torch)
+    M = [torch.zeros(w.shape, dtype=torch.float32, device=dev) for w in W]
+    rho = torch.stack([w.float().norm() for w in W])
+    mats = nshb.matrices(W, G, M, z_index=(zi if Z is not None else None))
+    p = nshb.params(eta=ETA, rho=rho, **extra_params(extra))
+    if Z is not None:
+        ws = nshb.workspace(mats, p, op, device=dev, z_rows=[z.shape[0] for z in Z], n_tokens=n_tok)
+        step = lambda: nshb.newton_muon_step(mats, Z, n_tok, p, ws, stream)   # noqa: E731
+    else:
+        ws = nshb.workspace(mats, p, op, device=dev)
+        step = lambda: getattr(nshb, fn)(mats, p, ws, stream)   # noqa: E731
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    flags = nshb.device_status(ws, stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    nshb.profile_enable(True)
+    nshb.profile_read()
+    kp = 3
+    for _ in range(kp):
+        step()
+    torch.cuda.synchronize()
+    prof = nshb.profile_read()
+    nshb.profile_enable(False)
+    peaks, peak_src = load_peaks()
+    peak_tf = peaks.get("bf16_tflops_sustained", DEFAULT_PEAKS["bf16_tflops_sustained"])
+    n = sum(r * c for r, c in shp)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {
+        "metric": "optimizer step ms; algorithmic tensor-core TFLOP/s over the whole step",
+        "value": round(ms, 3), "unit": "ms", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 3), "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded on the device: W0 ~ N(0, 0.02^2), spiked Gaussian gradients)",
+        "config": {"workload": CONFIGS[args.config], "matrices": len(shp), "params": n, **extra},
+        "throughput": {"value": round(n / (ms * 1e-3), 1), "unit": "params/s"},
+        "step_tflops": round(tf, 1),
+        "step_tflops_frac_of_sustained_bf16_peak": round(tf / peak_tf, 4),
+        "algorithmic_tflop_per_step": round(flops / 1e12, 3),
+        "peak_source": f"{peak_src} bf16 sustained",
+        "kernels_ms_per_step": {k: round(v[0] / kp, 4) for k, v in prof.items()},
+        "launches_per_step": {k: round(v[1] / kp, 1) for k, v in prof.items()},
+        "device_status": flags, "clocks": clk.summary(),
+    }
+
+
+def extra_params(extra):
+    return {"tile": extra["tile"]} if "tile" in extra else {}
+
+
 # --------------------------------------------------------------- CPU baseline
 def oracle_sample(layers=1, steps=1):
     """Times the fp64 oracle on `layers` of the 12 GPT-2 layers for `steps` steps and returns
@@ -465,6 +584,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--config", default="gpt2", choices=["gpt2"] + sorted(CONFIGS),
+                    help="gpt2: the headline workload; the others time one larger configuration (1 GPU)")
     ap.add_argument("--optimizer", default="muonh", choices=["muonh", "adamh"],
                     help="muonh: the headline MuonH step; adamh: the AdamH step on the same matrices")
     ap.add_argument("--ncu", action="store_true",
@@ -503,6 +624,12 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
 
+    if args.config != "gpt2":
+        if world > 1:
+            print("--config runs on one GPU", file=sys.stderr)
+            return 2
+        print(json.dumps(run_config(args)), flush=True)
+        return 0
     if args.optimizer == "adamh":
         if world > 1:
             print("--optimizer adamh runs on one GPU", file=sys.stderr)
