@@ -419,6 +419,41 @@ void coeffs_for(const nshb_params *p, int it, float &a, float &b, float &c) {
   }
 }
 
+// Hierarchical Muon with T = 256: every tile's whole chain in the tile-resident kernel.
+nshb_status run_himuon_tile(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t st) {
+  const int n = (int)pl.mp.size();
+  for (int c0 = 0; c0 < n; c0 += kMaxProb) {
+    const int c1 = std::min(n, c0 + kMaxProb);
+    HmParams hp;
+    std::memset(&hp, 0, sizeof(hp));
+    hp.ws = ws;
+    hp.scales = reinterpret_cast<const float *>(ws + pl.scale_off);
+    hp.status = reinterpret_cast<uint32_t *>(ws);
+    hp.wait_limit = (p->debug_flags & 1u) ? kWaitLimitTest : kWaitLimit;
+    hp.ns_steps = p->ns_steps;
+    hp.comp = pl.comp;
+    for (int it = 0; it < p->ns_steps; ++it) coeffs_for(p, it, hp.coef[it][0], hp.coef[it][1], hp.coef[it][2]);
+    int tiles = 0;
+    for (int i = c0; i < c1; ++i) {
+      const MatPlan &m = pl.mp[i];
+      HmProb &q = hp.prob[i - c0];
+      q.x0 = m.x0;
+      q.xo = (p->ns_steps % 2 == 0) ? m.x0 : m.x1;
+      q.xl0 = m.xl0;
+      q.xl1 = m.xl1;
+      q.tile_begin = tiles;
+      q.ntiles = m.ntiles;
+      q.seg_begin = m.seg_begin;
+      tiles += m.ntiles;
+    }
+    hp.nprob = c1 - c0;
+    hp.total_tiles = tiles;
+    NSHB_CHECK_CUDA(encode_ws_tensor_map(&hp.tmap, ws, pl.total / 128 * 128));
+    NSHB_LAUNCH(NSHB_PROF_GRAM, launch_himuon_tile(hp, device_sms(), st));
+  }
+  return NSHB_OK;
+}
+
 // K iterations of the three NS phases.  Returns the offset of each matrix's O in `o_off`.
 nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t st, std::vector<int64_t> &o_off) {
   const int n = (int)pl.mp.size();
@@ -426,6 +461,12 @@ nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t 
   const float *scales = reinterpret_cast<const float *>(ws + pl.scale_off);
   uint32_t *status = reinterpret_cast<uint32_t *>(ws);
   const long long limit = (p->debug_flags & 1u) ? kWaitLimitTest : kWaitLimit;
+  if (pl.tiled && pl.pair && p->tile == 256 && !p->debug_flags) {
+    const nshb_status e = run_himuon_tile(pl, p, ws, st);
+    if (e != NSHB_OK) return e;
+    for (int i = 0; i < n; ++i) o_off[i] = (p->ns_steps % 2 == 0) ? pl.mp[i].x0 : pl.mp[i].x1;
+    return NSHB_OK;
+  }
   std::vector<int> f32_idx, bf_idx;   // matrices whose NS runs in fp32 / on the bf16 tensor cores
   for (int i = 0; i < n; ++i) (pl.mp[i].f32 ? f32_idx : bf_idx).push_back(i);
   for (int it = 0; it < p->ns_steps; ++it) {

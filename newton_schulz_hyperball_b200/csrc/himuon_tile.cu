@@ -1,0 +1,501 @@
+// Hierarchical Muon with T = 256: the whole Newton-Schulz chain of one tile on one CTA
+// pair, with the tile resident in shared and tensor memory.
+// ("Hierarchical Muon: Tiled Newton-Schulz Updates", abstract: the same finite NS map
+//  run independently on every T x T tile; "Muon: the orthogonalized optimizer
+//  explained", Newton-Schulz section: A = X X^T, B = b A + c A^2, X <- a X + B X.)
+//
+// Why a separate kernel: with T = 256 one phase of one tile is about 1.5 us of
+// tensor-core work, but as three grouped GEMM launches per iteration every phase
+// reloads 128 KB of operands per CTA and writes its result back to memory, and a
+// tile-phase takes 5.5-8 us.  Here a pair loads X once and runs, per iteration:
+//   Gram    A = s^2 X X^T        -> TMEM columns [0, 256)   (operands: sXown, K-major)
+//   epi 1   A -> bf16 sA                                  (A stays in TMEM in fp32)
+//   poly    A^2 = A A            -> TMEM columns [256, 512) (operands: sA; A is symmetric)
+//   epi 2   B = b A + c A^2 from the fp32 accumulators -> bf16 sA
+//   update  B X                  -> TMEM columns [0, 256)   (sA K-major, sXcol MN-major)
+//   epi 3   X' = s (a X + B X) -> own rows of sXown, the own column half of sXcol, and
+//           the partner's column half of its sXcol (distributed shared memory).
+// Only the first X, the low parts of the compensated iterations and the final O touch
+// global memory.  The factor s (1 / (||tile|| + eps)) applies in the first iteration.
+//
+// Shared memory per CTA r (0 = leader): sXown 64 KB = X rows 128r .. 128r+127 (four
+// 64-column panels of 128 rows, the tensor core's 128-byte swizzled image), sXcol 64 KB =
+// X columns 128r .. 128r+127 over all 256 rows (two panels of 256 rows), sA 64 KB (this
+// CTA's 128 rows of A, then of B).  A cta_group::2 MMA reads the same shared-memory
+// offset in both CTAs, so each CTA keeps its own half at offset 0.
+//
+// Roles (320 threads per CTA): warp 0 loads X (TMA onto a local barrier, then tells the
+// leader), warp 1 of the leader issues the MMAs and multicasts each commit, warps 2-9 of
+// both CTAs run the epilogues on their 128 accumulator rows (lane quarter = warp % 4,
+// column half = (warp - 2) / 4) and report to the leader.  Tiles are walked statically
+// by the persistent grid.  Every wait is bounded; no load is multicast.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "nshb_device.cuh"
+#include "nshb_internal.h"
+
+namespace nshb {
+namespace {
+
+constexpr int T = 256;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kPanel128 = 128 * 128;            // 64 columns x 128 rows of bf16: 16 KB
+constexpr int kPanel256 = 256 * 128;            // 64 columns x 256 rows: 32 KB
+constexpr int kHalf = 4 * kPanel128;            // 64 KB
+constexpr int SMEM_BYTES = 3 * kHalf + 1024 + 256;
+constexpr uint32_t kTimeoutBit = 0x4u;
+
+__device__ __forceinline__ uint32_t cta_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t num_clusters() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// 2-D TMA load into this CTA's shared memory, completing on this CTA's barrier.
+__device__ __forceinline__ void tma_load_local(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc2(uint32_t dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish2() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_mma2(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.u32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit2_mc(uint32_t bar, uint16_t mask) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::
+                   "r"(bar),
+               "h"(mask)
+               : "memory");
+}
+// Generic-proxy shared-memory writes become visible to the tensor core (async proxy).
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async;" ::: "memory"); }
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t *w) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+               : "memory");
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, const uint32_t *w) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+               "r"(w[3])
+               : "memory");
+}
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t *w) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+               : "r"(addr)
+               : "memory");
+}
+// 32-byte global accesses of two logically adjacent 16-byte chunks of a panel row (the
+// 128-byte swizzle keeps chunks {c, c+1}, c even, in one sector, swapped on odd rows).
+__device__ __forceinline__ size_t panel_pair_off(int64_t row, int64_t col, int64_t ph) {
+  return ((size_t)((col >> 6) * ph + row) << 7) + ((size_t)(((col >> 4) & 3) ^ ((row >> 1) & 3)) << 5);
+}
+__device__ __forceinline__ void unswizzle_pair(const uint32_t (&w)[8], bool odd, uint32_t *out) {
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    out[e] = odd ? w[4 + e] : w[e];
+    out[4 + e] = odd ? w[e] : w[4 + e];
+  }
+}
+__device__ __forceinline__ void ld_global_256(const void *p, uint32_t (&w)[8]) {
+  asm volatile("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+               : "l"(p));
+}
+__device__ __forceinline__ void st_global_256(void *p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+               "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
+// Byte offset in a K-major half (sA, sXown: 128 rows, four 64-column panels) of the 16-byte
+// chunk holding row rl, columns j .. j+7.
+__device__ __forceinline__ uint32_t half_chunk(int rl, int j) {
+  return (uint32_t)((j >> 6) * kPanel128 + rl * 128 + ((((j >> 3) & 7) ^ (rl & 7)) << 4));
+}
+// ... and in a column half (sXcol: 256 rows, two panels), row g, columns jj .. jj+7 (jj < 128).
+__device__ __forceinline__ uint32_t col_chunk(int g, int jj) {
+  return (uint32_t)((jj >> 6) * kPanel256 + g * 128 + ((((jj >> 3) & 7) ^ (g & 7)) << 4));
+}
+
+__device__ __forceinline__ int find_prob(const HmParams &p, int tile) {
+  int lo = 0, hi = p.nprob - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.prob[mid].tile_begin <= tile) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_constant__ HmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sXown = smem_u32(smem), sXcol = sXown + kHalf, sA = sXcol + kHalf;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 3 * kHalf);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
+  const uint32_t bar_base = smem_u32(bars);
+  const uint32_t xfull = bar_base, xfree = bar_base + 8, mmadone = bar_base + 16;
+  const uint32_t xready = bar_base + 24, opnd = bar_base + 32;   // used in the leader only
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cta_rank();
+  const bool leader = rank == 0;
+  const int cid = (int)cluster_id(), ncl = (int)num_clusters();
+  if (threadIdx.x == 0) {
+    mbar_init(xfull, 1);
+    mbar_init(xfree, 1);
+    mbar_init(mmadone, 1);
+    mbar_init(xready, 2);                 // both producers
+    mbar_init(opnd, 2 * kEpiWarps);       // every epilogue warp of both CTAs
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc2(smem_u32(tmem_slot), 512);
+    tmem_relinquish2();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const long long limit = p.wait_limit;
+  pdl_trigger();
+  pdl_wait();                             // X0, its low part and the scales are written
+  const int K = p.ns_steps;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer (both CTAs)
+      uint32_t ph_f = 0, ph_x = 0;
+      for (int tile = cid; tile < p.total_tiles; tile += ncl) {
+        if (!mbar_wait(xfree, ph_f ^ 1u, limit)) {
+          set_status(p.status, kTimeoutBit);
+          break;
+        }
+        ph_f ^= 1u;
+        const HmProb &q = p.prob[find_prob(p, tile)];
+        const int64_t base = (q.x0 + (int64_t)(tile - q.tile_begin) * T * T * 2) >> 7;   // 128-byte rows
+        mbar_arrive_expect_tx(xfull, 2 * kHalf);
+#pragma unroll
+        for (int pnl = 0; pnl < 4; ++pnl)   // own rows, all four panels
+          tma_load_local(sXown + pnl * kPanel128, &p.tmap, 0, (int)(base + pnl * T + 128 * rank), xfull);
+#pragma unroll
+        for (int pp = 0; pp < 2; ++pp)      // own two panels, all rows
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+            tma_load_local(sXcol + pp * kPanel256 + hh * kPanel128, &p.tmap, 0,
+                           (int)(base + (2 * rank + pp) * T + 128 * hh), xfull);
+        if (!mbar_wait(xfull, ph_x, limit)) {
+          set_status(p.status, kTimeoutBit);
+          break;
+        }
+        ph_x ^= 1u;
+        remote_arrive(mapa(xready, 0));
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------------------ MMA issuer (leader)
+      const uint32_t idesc_k = idesc_bf16(2 * 128, T, 0), idesc_mn = idesc_bf16(2 * 128, T, 1);
+      uint32_t ph_r = 0, ph_o = 0;
+      bool ok = true;
+      auto wait_opnd = [&]() {
+        if (!mbar_wait(opnd, ph_o, limit)) {
+          set_status(p.status, kTimeoutBit);
+          ok = false;
+        }
+        ph_o ^= 1u;
+        tc_fence_after();
+      };
+      for (int tile = cid; ok && tile < p.total_tiles; tile += ncl) {
+        if (!mbar_wait(xready, ph_r, limit)) {
+          set_status(p.status, kTimeoutBit);
+          break;
+        }
+        ph_r ^= 1u;
+        tc_fence_after();
+        for (int it = 0; ok && it < K; ++it) {
+          if (it > 0) {
+            wait_opnd();   // epilogue 3 of the previous iteration wrote X'
+            if (!ok) break;
+          }
+#pragma unroll
+          for (int k = 0; k < T / 16; ++k) {   // Gram: A = X X^T
+            const uint32_t kofs = (uint32_t)(k >> 2) * kPanel128 + 32u * (k & 3);
+            const uint64_t d = smem_desc_sw128(sXown + kofs, 16, 1024);
+            tc_mma2(tmem_base, d, d, idesc_k, k != 0);
+          }
+          tc_commit2_mc(mmadone, 0x3);
+          wait_opnd();     // epilogue 1 wrote A to sA
+          if (!ok) break;
+#pragma unroll
+          for (int k = 0; k < T / 16; ++k) {   // A^2 = A A^T (A symmetric)
+            const uint32_t kofs = (uint32_t)(k >> 2) * kPanel128 + 32u * (k & 3);
+            const uint64_t d = smem_desc_sw128(sA + kofs, 16, 1024);
+            tc_mma2(tmem_base + T, d, d, idesc_k, k != 0);
+          }
+          tc_commit2_mc(mmadone, 0x3);
+          wait_opnd();     // epilogue 2 wrote B to sA
+          if (!ok) break;
+#pragma unroll
+          for (int k = 0; k < T / 16; ++k) {   // B X: B K-major, X MN-major (16 rows per step)
+            const uint32_t kofs = (uint32_t)(k >> 2) * kPanel128 + 32u * (k & 3);
+            const uint64_t ad = smem_desc_sw128(sA + kofs, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(sXcol + 2048u * k, kPanel256, 1024);
+            tc_mma2(tmem_base, ad, bd, idesc_mn, k != 0);
+          }
+          tc_commit2_mc(mmadone, 0x3);
+        }
+        if (!ok) break;
+        wait_opnd();       // the tile's last epilogue is done with sXown and the TMEM
+        if (!ok) break;
+        remote_arrive(mapa(xfree, 0));
+        remote_arrive(mapa(xfree, 1));
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogues (both CTAs)
+    const int quarter = warp & 3;                      // TMEM lanes 32 quarter .. +31
+    const int half = (warp - 2) >> 2;                  // columns 128 half .. +127
+    const int rl = quarter * 32 + lane;                // row within this CTA's half
+    const int g = 128 * (int)rank + rl;                // row within the tile
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const bool odd = g & 1;
+    const bool own_cols = half == (int)rank;           // sXcol columns of this half live here
+    uint32_t ph_x = 0, ph_m = 0;
+    bool ok = true;
+    auto wait_mma = [&]() {
+      if (!mbar_wait(mmadone, ph_m, limit)) {
+        if (lane == 0) set_status(p.status, kTimeoutBit);
+        ok = false;
+      }
+      ph_m ^= 1u;
+      tc_fence_after();
+    };
+    auto report = [&]() {
+      fence_proxy_async();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) remote_arrive(mapa(opnd, 0));
+    };
+    for (int tile = cid; ok && tile < p.total_tiles; tile += ncl) {
+      const HmProb &q = p.prob[find_prob(p, tile)];
+      const int t = tile - q.tile_begin;
+      const int64_t toff = (int64_t)t * T * T * 2;
+      const float s = p.scales[q.seg_begin + t];
+      if (!mbar_wait(xfull, ph_x, limit)) {            // sXown holds X0 (read by epilogue 3)
+        if (lane == 0) set_status(p.status, kTimeoutBit);
+        break;
+      }
+      ph_x ^= 1u;
+      for (int it = 0; ok && it < K; ++it) {
+        const float ca = p.coef[it][0], cb = p.coef[it][1], cc = p.coef[it][2];
+        const float s2 = it == 0 ? s * s : 1.0f, ks = it == 0 ? s : 1.0f;
+        // ---- epilogue 1: A -> sA (bf16)
+        wait_mma();
+        if (!ok) break;
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          const int j0 = 128 * half + 32 * ch;
+          uint32_t r[32];
+          tmem_ld32(tmem_base + (uint32_t)j0 + lane_off, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = pack_bf16(s2 * __uint_as_float(r[8 * c + 2 * e]), s2 * __uint_as_float(r[8 * c + 2 * e + 1]));
+            st_shared_v4(sA + half_chunk(rl, j0 + 8 * c), w);
+          }
+        }
+        report();
+        // ---- epilogue 2: B = b A + c A^2 -> sA (bf16), A and A^2 from TMEM in fp32
+        wait_mma();
+        if (!ok) break;
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          const int j0 = 128 * half + 32 * ch;
+          uint32_t ra[32], rq[32];
+          tmem_ld32(tmem_base + (uint32_t)j0 + lane_off, ra);
+          tmem_ld32(tmem_base + (uint32_t)(T + j0) + lane_off, rq);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i0 = 8 * c + 2 * e;
+              w[e] = pack_bf16(fmaf(cb * s2, __uint_as_float(ra[i0]), cc * __uint_as_float(rq[i0])),
+                               fmaf(cb * s2, __uint_as_float(ra[i0 + 1]), cc * __uint_as_float(rq[i0 + 1])));
+            }
+            st_shared_v4(sA + half_chunk(rl, j0 + 8 * c), w);
+          }
+        }
+        report();
+        // ---- epilogue 3: X' = s (a X + B X)
+        wait_mma();
+        if (!ok) break;
+        const bool last = it + 1 == K;
+        const char *clo = it < p.comp ? p.ws + ((it % 2 == 0) ? q.xl0 : q.xl1) + toff : nullptr;
+        char *dlo = (it + 1 < p.comp) ? p.ws + ((it % 2 == 0) ? q.xl1 : q.xl0) + toff : nullptr;
+        char *dout = last ? p.ws + q.xo + toff : nullptr;
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          const int j0 = 128 * half + 32 * ch;
+          uint32_t r[32];
+          tmem_ld32(tmem_base + (uint32_t)j0 + lane_off, r);
+          uint32_t xw[16], lw[16];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) ld_shared_v4(sXown + half_chunk(rl, j0 + 8 * c), xw + 4 * c);
+          if (clo) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              uint32_t w8[8];
+              ld_global_256(clo + panel_pair_off(g, j0 + 16 * k, T), w8);
+              unswizzle_pair(w8, odd, lw + 8 * k);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) lw[e] = 0u;
+          }
+          tmem_ld_wait();
+          uint32_t hw[16], low[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float x0 = bf16lo(xw[e]) + bf16lo(lw[e]), x1 = bf16hi(xw[e]) + bf16hi(lw[e]);
+            const float v0 = ks * fmaf(ca, x0, __uint_as_float(r[2 * e]));
+            const float v1 = ks * fmaf(ca, x1, __uint_as_float(r[2 * e + 1]));
+            hw[e] = pack_bf16(v0, v1);
+            low[e] = pack_bf16(v0 - bf16lo(hw[e]), v1 - bf16hi(hw[e]));
+          }
+          if (last) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              uint32_t in8[8], w8[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) in8[e] = hw[8 * k + e];
+              unswizzle_pair(in8, odd, w8);
+              st_global_256(dout + panel_pair_off(g, j0 + 16 * k, T), w8);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              st_shared_v4(sXown + half_chunk(rl, j0 + 8 * c), hw + 4 * c);
+              const uint32_t a = sXcol + col_chunk(g, j0 + 8 * c - 128 * half);
+              if (own_cols) st_shared_v4(a, hw + 4 * c);
+              else st_cluster_v4(mapa(a, rank ^ 1u), hw + 4 * c);
+            }
+            if (dlo) {
+#pragma unroll
+              for (int k = 0; k < 2; ++k) {
+                uint32_t in8[8], w8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) in8[e] = low[8 * k + e];
+                unswizzle_pair(in8, odd, w8);
+                st_global_256(dlo + panel_pair_off(g, j0 + 16 * k, T), w8);
+              }
+            }
+          }
+        }
+        report();
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();                         // no CTA leaves while its partner may still
+                                          // read or write its shared memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc2(tmem_base, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_himuon_tile(const HmParams &p, int num_sms, cudaStream_t s) {
+  static unsigned done_mask = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(done_mask & (1u << (dev & 31)))) {
+    cudaError_t e = cudaFuncSetAttribute(himuon_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    done_mask |= 1u << (dev & 31);
+  }
+  if (p.total_tiles <= 0) return cudaSuccess;
+  static int max_pairs[32] = {0};
+  int &mp = max_pairs[dev & 31];
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see pdl_wait
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  if (!mp) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, himuon_tile_kernel, &cfg) != cudaSuccess || n <= 0) {
+      (void)cudaGetLastError();
+      n = num_sms / 2;
+    }
+    mp = n < num_sms / 2 ? n : num_sms / 2;
+  }
+  const int clusters = p.total_tiles < mp ? p.total_tiles : mp;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, himuon_tile_kernel, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace nshb

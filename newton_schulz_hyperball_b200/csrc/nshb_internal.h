@@ -148,6 +148,28 @@ struct GemmParams {
   GemmProb prob[kMaxProb];
 };
 
+// Tile-resident Hierarchical Muon (T = 256): one record per tiled matrix; its tiles are
+// consecutive T x T panel matrices (128 KB each) from x0 on.
+struct HmProb {
+  int64_t x0;              // X0 of tile 0 (read once per tile)
+  int64_t xo;              // where the final O of tile 0 is written
+  int64_t xl0, xl1;        // low parts of X0 / X1 (compensated iterations), or -1
+  int32_t tile_begin;      // first tile of this matrix in the launch
+  int32_t ntiles;
+  int32_t seg_begin;       // scale of tile 0 in scales
+  int32_t pad_;
+};
+struct HmParams {
+  CUtensorMap tmap;        // the workspace as 128-byte rows, 128-row boxes (see GemmParams)
+  char *ws;
+  const float *scales;
+  uint32_t *status;
+  long long wait_limit;
+  int32_t ns_steps, comp, nprob, total_tiles;
+  float coef[32][3];       // (a, b, c) of every iteration
+  HmProb prob[kMaxProb];
+};
+
 // fp32 SIMT GEMM problem (row-major fp32 operands in the workspace).
 struct F32Prob {
   int64_t a_off, b_off, c_off, d_off;
@@ -197,6 +219,8 @@ cudaError_t launch_adam(const AdamParams &p, cudaStream_t s);
 cudaError_t launch_gemm_tc(const GemmParams &p, int bn, int num_sms, cudaStream_t s);
 // 2-SM (CTA pair) form: 256 x 256 tiles, tcgen05.mma.cta_group::2; p.tmap must be encoded.
 cudaError_t launch_gemm_tc2(const GemmParams &p, int num_sms, cudaStream_t s);
+// Tile-resident Hierarchical Muon for T = 256 (all iterations of a tile on one CTA pair).
+cudaError_t launch_himuon_tile(const HmParams &p, int num_sms, cudaStream_t s);
 // Encodes p.tmap for a workspace of `bytes` bytes at `ws` (host; driver entry point).
 cudaError_t encode_ws_tensor_map(CUtensorMap *map, void *ws, size_t bytes);
 cudaError_t launch_gemm_f32(const F32Params &p, cudaStream_t s);
