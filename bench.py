@@ -416,7 +416,7 @@ def report_adamh(args, r, world):
 # ------------------------------------------------------------ other configurations
 CONFIGS = {
     "qwen3": "Qwen3-style 1.4B matrix set (196 matrices), MuonH step",
-    "himuon8b": "8B-width matrix set (224 matrices, 6.98B params), Hierarchical Muon T=256 + Hyperball step",
+    "himuon8b": "8B-width matrix set (224 matrices, 6.98B params), Hierarchical Muon + Hyperball step",
     "newton": "GPT-2-small matrix set, Newton-Muon step (48 layer inputs of 8192 tokens) + Hyperball",
 }
 
@@ -458,7 +458,7 @@ def run_config(args):
         cfg = wl.CFG_8B_WIDTH
         named = wl.width_8b_shapes(32)
         shp = [(r, c) for _, r, c in named]
-        T = 256
+        T = args.tile
         op, fn, flops = nshb.NSHB_OP_HIMUON, "himuon_step", sum(20.0 * r * c * T for r, c in shp)
         extra = {"tile": T}
     else:
@@ -586,6 +586,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--config", default="gpt2", choices=["gpt2"] + sorted(CONFIGS),
                     help="gpt2: the headline workload; the others time one larger configuration (1 GPU)")
+    ap.add_argument("--tile", type=int, default=256, choices=[128, 256, 512], help="--config himuon8b: tile size T")
     ap.add_argument("--optimizer", default="muonh", choices=["muonh", "adamh"],
                     help="muonh: the headline MuonH step; adamh: the AdamH step on the same matrices")
     ap.add_argument("--ncu", action="store_true",

@@ -419,7 +419,7 @@ void coeffs_for(const nshb_params *p, int it, float &a, float &b, float &c) {
   }
 }
 
-// Hierarchical Muon with T = 256: every tile's whole chain in the tile-resident kernel.
+// Hierarchical Muon with T = 256 or 128: every tile's whole chain in a tile-resident kernel.
 nshb_status run_himuon_tile(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t st) {
   const int n = (int)pl.mp.size();
   for (int c0 = 0; c0 < n; c0 += kMaxProb) {
@@ -449,7 +449,8 @@ nshb_status run_himuon_tile(const Plan &pl, const nshb_params *p, char *ws, cuda
     hp.nprob = c1 - c0;
     hp.total_tiles = tiles;
     NSHB_CHECK_CUDA(encode_ws_tensor_map(&hp.tmap, ws, pl.total / 128 * 128));
-    NSHB_LAUNCH(NSHB_PROF_GRAM, launch_himuon_tile(hp, device_sms(), st));
+    if (p->tile == 128) NSHB_LAUNCH(NSHB_PROF_GRAM, launch_himuon_tile128(hp, device_sms(), st));
+    else NSHB_LAUNCH(NSHB_PROF_GRAM, launch_himuon_tile(hp, device_sms(), st));
   }
   return NSHB_OK;
 }
@@ -461,7 +462,7 @@ nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t 
   const float *scales = reinterpret_cast<const float *>(ws + pl.scale_off);
   uint32_t *status = reinterpret_cast<uint32_t *>(ws);
   const long long limit = (p->debug_flags & 1u) ? kWaitLimitTest : kWaitLimit;
-  if (pl.tiled && pl.pair && p->tile == 256 && !p->debug_flags) {
+  if (pl.tiled && (p->tile == 256 || p->tile == 128) && !p->debug_flags) {
     const nshb_status e = run_himuon_tile(pl, p, ws, st);
     if (e != NSHB_OK) return e;
     for (int i = 0; i < n; ++i) o_off[i] = (p->ns_steps % 2 == 0) ? pl.mp[i].x0 : pl.mp[i].x1;

@@ -450,6 +450,274 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
   }
 }
 
+// ---------------------------------------------------------------------------- T = 128
+// One CTA holds a whole 128 x 128 tile: sX (two 64-column panels of 128 rows, 32 KB)
+// serves as the K-major Gram operand and as the MN-major update operand; sA (32 KB) holds
+// A, then B; TMEM columns [0, 128) take A and then B X, [128, 256) take A^2, so B = b A +
+// c A^2 is formed from the fp32 accumulators.  Two CTAs share an SM (64 KB of shared
+// memory and 256 TMEM columns each), so one tile's epilogues overlap the other's MMAs
+// (three per SM, with A taken from its bf16 copy, measured no faster).  192 threads:
+// warp 0 loads X, warp 1 issues the MMAs, warps 2-5 run the epilogues (lane quarter =
+// warp % 4, all 128 columns).
+constexpr int T1 = 128;
+constexpr int kThreads1 = 64 + 32 * 4;
+constexpr int kTile1 = 2 * kPanel128;                 // 32 KB
+// 64 KB of operands are used; asking for 100 KB keeps a third CTA off the SM, whose TMEM
+// allocation would otherwise wait for a neighbour's whole tile loop.
+constexpr int SMEM_BYTES1 = 100 * 1024;
+constexpr int kCtasPerSm1 = 2;
+static_assert(2 * kTile1 + 1024 + 256 <= SMEM_BYTES1, "shared memory of the T = 128 kernel");
+
+__global__ void __launch_bounds__(kThreads1, kCtasPerSm1) himuon_tile128_kernel(const __grid_constant__ HmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sX = smem_u32(smem), sA = sX + kTile1;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 2 * kTile1);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
+  const uint32_t bar_base = smem_u32(bars);
+  const uint32_t xfull = bar_base, xfree = bar_base + 8, mmadone = bar_base + 16, opnd = bar_base + 24;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(xfull, 1);
+    mbar_init(xfree, 1);
+    mbar_init(mmadone, 1);
+    mbar_init(opnd, 4);                   // the four epilogue warps
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const long long limit = p.wait_limit;
+  pdl_trigger();
+  pdl_wait();
+  const int K = p.ns_steps;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t ph_f = 0;
+      for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
+        if (!mbar_wait(xfree, ph_f ^ 1u, limit)) {
+          set_status(p.status, kTimeoutBit);
+          break;
+        }
+        ph_f ^= 1u;
+        const HmProb &q = p.prob[find_prob(p, tile)];
+        const int64_t base = (q.x0 + (int64_t)(tile - q.tile_begin) * T1 * T1 * 2) >> 7;
+        mbar_arrive_expect_tx(xfull, kTile1);
+        tma_load_local(sX, &p.tmap, 0, (int)base, xfull);
+        tma_load_local(sX + kPanel128, &p.tmap, 0, (int)(base + T1), xfull);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc_k = idesc_bf16(T1, T1, 0), idesc_mn = idesc_bf16(T1, T1, 1);
+      uint32_t ph_x = 0, ph_o = 0;
+      bool ok = true;
+      auto wait_opnd = [&]() {
+        if (!mbar_wait(opnd, ph_o, limit)) {
+          set_status(p.status, kTimeoutBit);
+          ok = false;
+        }
+        ph_o ^= 1u;
+        tc_fence_after();
+      };
+      for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+        if (!mbar_wait(xfull, ph_x, limit)) {
+          set_status(p.status, kTimeoutBit);
+          break;
+        }
+        ph_x ^= 1u;
+        tc_fence_after();
+        for (int it = 0; ok && it < K; ++it) {
+          if (it > 0) {
+            wait_opnd();
+            if (!ok) break;
+          }
+#pragma unroll
+          for (int k = 0; k < T1 / 16; ++k) {
+            const uint32_t kofs = (uint32_t)(k >> 2) * kPanel128 + 32u * (k & 3);
+            const uint64_t d = smem_desc_sw128(sX + kofs, 16, 1024);
+            tc_mma(tmem_base, d, d, idesc_k, k != 0);
+          }
+          tc_commit(mmadone);
+          wait_opnd();
+          if (!ok) break;
+#pragma unroll
+          for (int k = 0; k < T1 / 16; ++k) {
+            const uint32_t kofs = (uint32_t)(k >> 2) * kPanel128 + 32u * (k & 3);
+            const uint64_t d = smem_desc_sw128(sA + kofs, 16, 1024);
+            tc_mma(tmem_base + T1, d, d, idesc_k, k != 0);
+          }
+          tc_commit(mmadone);
+          wait_opnd();
+          if (!ok) break;
+#pragma unroll
+          for (int k = 0; k < T1 / 16; ++k) {
+            const uint32_t kofs = (uint32_t)(k >> 2) * kPanel128 + 32u * (k & 3);
+            const uint64_t ad = smem_desc_sw128(sA + kofs, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(sX + 2048u * k, kPanel128, 1024);
+            tc_mma(tmem_base, ad, bd, idesc_mn, k != 0);
+          }
+          tc_commit(mmadone);
+        }
+        if (!ok) break;
+        wait_opnd();
+        if (!ok) break;
+        mbar_arrive(xfree);
+      }
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int rl = quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const bool odd = rl & 1;
+    uint32_t ph_x = 0, ph_m = 0;
+    bool ok = true;
+    auto wait_mma = [&]() {
+      if (!mbar_wait(mmadone, ph_m, limit)) {
+        if (lane == 0) set_status(p.status, kTimeoutBit);
+        ok = false;
+      }
+      ph_m ^= 1u;
+      tc_fence_after();
+    };
+    auto report = [&]() {
+      fence_proxy_async();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(opnd);
+    };
+    for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+      const HmProb &q = p.prob[find_prob(p, tile)];
+      const int t = tile - q.tile_begin;
+      const int64_t toff = (int64_t)t * T1 * T1 * 2;
+      const float s = p.scales[q.seg_begin + t];
+      if (!mbar_wait(xfull, ph_x, limit)) {
+        if (lane == 0) set_status(p.status, kTimeoutBit);
+        break;
+      }
+      ph_x ^= 1u;
+      for (int it = 0; ok && it < K; ++it) {
+        const float ca = p.coef[it][0], cb = p.coef[it][1], cc = p.coef[it][2];
+        const float s2 = it == 0 ? s * s : 1.0f, ks = it == 0 ? s : 1.0f;
+        wait_mma();
+        if (!ok) break;
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          const int j0 = 32 * ch;
+          uint32_t r[32];
+          tmem_ld32(tmem_base + (uint32_t)j0 + lane_off, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = pack_bf16(s2 * __uint_as_float(r[8 * c + 2 * e]), s2 * __uint_as_float(r[8 * c + 2 * e + 1]));
+            st_shared_v4(sA + half_chunk(rl, j0 + 8 * c), w);
+          }
+        }
+        report();
+        wait_mma();
+        if (!ok) break;
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          const int j0 = 32 * ch;
+          uint32_t ra[32], rq[32];
+          tmem_ld32(tmem_base + (uint32_t)j0 + lane_off, ra);
+          tmem_ld32(tmem_base + (uint32_t)(T1 + j0) + lane_off, rq);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i0 = 8 * c + 2 * e;
+              w[e] = pack_bf16(fmaf(cb * s2, __uint_as_float(ra[i0]), cc * __uint_as_float(rq[i0])),
+                               fmaf(cb * s2, __uint_as_float(ra[i0 + 1]), cc * __uint_as_float(rq[i0 + 1])));
+            }
+            st_shared_v4(sA + half_chunk(rl, j0 + 8 * c), w);
+          }
+        }
+        report();
+        wait_mma();
+        if (!ok) break;
+        const bool last = it + 1 == K;
+        const char *clo = it < p.comp ? p.ws + ((it % 2 == 0) ? q.xl0 : q.xl1) + toff : nullptr;
+        char *dlo = (it + 1 < p.comp) ? p.ws + ((it % 2 == 0) ? q.xl1 : q.xl0) + toff : nullptr;
+        char *dout = last ? p.ws + q.xo + toff : nullptr;
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          const int j0 = 32 * ch;
+          uint32_t r[32];
+          tmem_ld32(tmem_base + (uint32_t)j0 + lane_off, r);
+          uint32_t xw[16], lw[16];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) ld_shared_v4(sX + half_chunk(rl, j0 + 8 * c), xw + 4 * c);
+          if (clo) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              uint32_t w8[8];
+              ld_global_256(clo + panel_pair_off(rl, j0 + 16 * k, T1), w8);
+              unswizzle_pair(w8, odd, lw + 8 * k);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) lw[e] = 0u;
+          }
+          tmem_ld_wait();
+          uint32_t hw[16], low[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float x0 = bf16lo(xw[e]) + bf16lo(lw[e]), x1 = bf16hi(xw[e]) + bf16hi(lw[e]);
+            const float v0 = ks * fmaf(ca, x0, __uint_as_float(r[2 * e]));
+            const float v1 = ks * fmaf(ca, x1, __uint_as_float(r[2 * e + 1]));
+            hw[e] = pack_bf16(v0, v1);
+            low[e] = pack_bf16(v0 - bf16lo(hw[e]), v1 - bf16hi(hw[e]));
+          }
+          if (last) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              uint32_t in8[8], w8[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) in8[e] = hw[8 * k + e];
+              unswizzle_pair(in8, odd, w8);
+              st_global_256(dout + panel_pair_off(rl, j0 + 16 * k, T1), w8);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) st_shared_v4(sX + half_chunk(rl, j0 + 8 * c), hw + 4 * c);
+            if (dlo) {
+#pragma unroll
+              for (int k = 0; k < 2; ++k) {
+                uint32_t in8[8], w8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) in8[e] = low[8 * k + e];
+                unswizzle_pair(in8, odd, w8);
+                st_global_256(dlo + panel_pair_off(rl, j0 + 16 * k, T1), w8);
+              }
+            }
+          }
+        }
+        report();
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 256);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_himuon_tile(const HmParams &p, int num_sms, cudaStream_t s) {
@@ -496,6 +764,30 @@ cudaError_t launch_himuon_tile(const HmParams &p, int num_sms, cudaStream_t s) {
   cudaError_t e = cudaLaunchKernelEx(&cfg, himuon_tile_kernel, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+cudaError_t launch_himuon_tile128(const HmParams &p, int num_sms, cudaStream_t s) {
+  static unsigned done_mask = 0;
+  static int max_ctas[32] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(done_mask & (1u << (dev & 31)))) {
+    cudaError_t e =
+        cudaFuncSetAttribute(himuon_tile128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES1);
+    if (e != cudaSuccess) return e;
+    int per = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, himuon_tile128_kernel, kThreads1, SMEM_BYTES1) !=
+            cudaSuccess ||
+        per <= 0) {
+      (void)cudaGetLastError();
+      per = 1;
+    }
+    max_ctas[dev & 31] = num_sms * (per < kCtasPerSm1 ? per : kCtasPerSm1);   // TMEM: 256 columns per CTA
+    done_mask |= 1u << (dev & 31);
+  }
+  if (p.total_tiles <= 0) return cudaSuccess;
+  const int grid = p.total_tiles < max_ctas[dev & 31] ? p.total_tiles : max_ctas[dev & 31];
+  return launch_pdl(himuon_tile128_kernel, grid, kThreads1, SMEM_BYTES1, s, p);
 }
 
 }  // namespace nshb

@@ -221,6 +221,8 @@ cudaError_t launch_gemm_tc(const GemmParams &p, int bn, int num_sms, cudaStream_
 cudaError_t launch_gemm_tc2(const GemmParams &p, int num_sms, cudaStream_t s);
 // Tile-resident Hierarchical Muon for T = 256 (all iterations of a tile on one CTA pair).
 cudaError_t launch_himuon_tile(const HmParams &p, int num_sms, cudaStream_t s);
+// The same for T = 128, one tile per CTA, two CTAs per SM.
+cudaError_t launch_himuon_tile128(const HmParams &p, int num_sms, cudaStream_t s);
 // Encodes p.tmap for a workspace of `bytes` bytes at `ws` (host; driver entry point).
 cudaError_t encode_ws_tensor_map(CUtensorMap *map, void *ws, size_t bytes);
 cudaError_t launch_gemm_f32(const F32Params &p, cudaStream_t s);
