@@ -504,9 +504,9 @@ nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t 
               q.lda = (int)m.r; q.ldb = (int)m.s; q.ldc = (int)m.s; q.b_trans = 0;
             }
             q.scale_idx = (it == 0 && mode != kPoly) ? m.seg_begin : -1;
-            q.tiles_n = (q.N + 63) / 64;
+            q.tiles_n = (q.N + kF32Tile - 1) / kF32Tile;
             q.tile_begin = tiles;
-            tiles += ((q.M + 63) / 64) * q.tiles_n;
+            tiles += ((q.M + kF32Tile - 1) / kF32Tile) * q.tiles_n;
           }
           fp.nprob = c1 - c0;
           fp.total_tiles = tiles;
@@ -657,6 +657,15 @@ nshb_status run_apply(const nshb_matrix *mats, const Plan &pl, const nshb_params
 }
 
 // F32 GEMM problem helper.
+// Output tiles of an fp32 GEMM problem (all, or those on and below the diagonal).
+int f32_tiles(const F32Prob &q) {
+  const int tm = (q.M + kF32Tile - 1) / kF32Tile;
+  if (!q.lower) return tm * q.tiles_n;
+  int cnt = 0;
+  for (int mi = 0; mi < tm; ++mi) cnt += std::min(mi + 1, q.tiles_n);
+  return cnt;
+}
+
 F32Prob f32prob(int64_t a, int lda, int64_t b, int ldb, int bt, int64_t c, int64_t d, int ldc, int M, int N, int K) {
   F32Prob q;
   std::memset(&q, 0, sizeof(q));
@@ -665,7 +674,7 @@ F32Prob f32prob(int64_t a, int lda, int64_t b, int ldb, int bt, int64_t c, int64
   q.c_off = c; q.d_off = d; q.ldc = ldc;
   q.M = M; q.N = N; q.K = K;
   q.scale_idx = -1;
-  q.tiles_n = (N + 63) / 64;
+  q.tiles_n = (N + kF32Tile - 1) / kF32Tile;
   return q;
 }
 
@@ -681,7 +690,7 @@ nshb_status run_f32(const std::vector<F32Prob> &probs, int mode, char *ws, cudaS
     for (size_t i = c0; i < c1; ++i) {
       F32Prob q = probs[i];
       q.tile_begin = tiles;
-      tiles += ((q.M + 63) / 64) * q.tiles_n;
+      tiles += f32_tiles(q);
       fp.prob[i - c0] = q;
     }
     fp.nprob = (int)(c1 - c0);
@@ -802,6 +811,7 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
         panel.push_back(f32prob(pan, ld, z.inv + (k / 64) * 64 * 64 * 4, 64, 1, pan, pan, ld, rest, 64, 64));
         const int64_t tr = z.s + ((k + 64) * z.Dp + (k + 64)) * 4;
         trail.push_back(f32prob(pan, ld, pan, ld, 1, tr, tr, ld, rest, rest, 64));
+        trail.back().lower = 1;   // symmetric update: the factorisation reads the lower triangle only
       }
       nshb_status e = run_f32(panel, kPlain, ws, st);
       if (e != NSHB_OK) return e;

@@ -171,6 +171,7 @@ struct HmParams {
 };
 
 // fp32 SIMT GEMM problem (row-major fp32 operands in the workspace).
+constexpr int kF32Tile = 128;   // output tile of the fp32 GEMM (kF32Tile x kF32Tile)
 struct F32Prob {
   int64_t a_off, b_off, c_off, d_off;
   int32_t M, N, K;
@@ -178,6 +179,8 @@ struct F32Prob {
   int32_t b_trans;         // 1: B element (k, j) at b[j * ldb + k]; 0: at b[k * ldb + j]
   int32_t tiles_n, tile_begin;
   int32_t scale_idx;
+  int32_t lower;           // 1: only the output tiles on and below the diagonal
+  int32_t pad_;
 };
 struct F32Params {
   char *ws;
