@@ -456,7 +456,7 @@ def run_config(args):
         extra = {}
     elif args.config == "himuon8b":
         cfg = wl.CFG_8B_WIDTH
-        named = wl.width_8b_shapes(32)
+        named = wl.width_8b_shapes(args.layers)
         shp = [(r, c) for _, r, c in named]
         T = args.tile
         op, fn, flops = nshb.NSHB_OP_HIMUON, "himuon_step", sum(20.0 * r * c * T for r, c in shp)
@@ -491,6 +491,11 @@ def run_config(args):
         step()
     torch.cuda.synchronize()
     flags = nshb.device_status(ws, stream)
+    if args.ncu:
+        for _ in range(args.steps):
+            step()
+        torch.cuda.synchronize()
+        return None
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(0) as clk:
         e0.record(stream)
@@ -516,7 +521,8 @@ def run_config(args):
         "value": round(ms, 3), "unit": "ms", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms, 3), "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded on the device: W0 ~ N(0, 0.02^2), spiked Gaussian gradients)",
-        "config": {"workload": CONFIGS[args.config], "matrices": len(shp), "params": n, **extra},
+        "config": {"workload": CONFIGS[args.config], "matrices": len(shp), "params": n, **extra,
+                   **({"layers": args.layers} if args.config == "himuon8b" else {})},
         "throughput": {"value": round(n / (ms * 1e-3), 1), "unit": "params/s"},
         "step_tflops": round(tf, 1),
         "step_tflops_frac_of_sustained_bf16_peak": round(tf / peak_tf, 4),
@@ -587,6 +593,7 @@ def main():
     ap.add_argument("--config", default="gpt2", choices=["gpt2"] + sorted(CONFIGS),
                     help="gpt2: the headline workload; the others time one larger configuration (1 GPU)")
     ap.add_argument("--tile", type=int, default=256, choices=[128, 256, 512], help="--config himuon8b: tile size T")
+    ap.add_argument("--layers", type=int, default=32, help="--config himuon8b: layers of the 8B-width set")
     ap.add_argument("--optimizer", default="muonh", choices=["muonh", "adamh"],
                     help="muonh: the headline MuonH step; adamh: the AdamH step on the same matrices")
     ap.add_argument("--ncu", action="store_true",
@@ -629,7 +636,8 @@ def main():
         if world > 1:
             print("--config runs on one GPU", file=sys.stderr)
             return 2
-        print(json.dumps(run_config(args)), flush=True)
+        r = run_config(args)
+        print("ncu case done" if r is None else json.dumps(r), flush=True)
         return 0
     if args.optimizer == "adamh":
         if world > 1:
