@@ -106,8 +106,12 @@ __device__ __forceinline__ void tc_commit2_mc(uint32_t bar, uint16_t mask) {
                "h"(mask)
                : "memory");
 }
-// Generic-proxy shared-memory writes become visible to the tensor core (async proxy).
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async;" ::: "memory"); }
+// Generic-proxy shared-memory writes become visible to the tensor core (async proxy): this
+// CTA's shared memory, or any shared memory of the cluster (writes into the partner's).
+__device__ __forceinline__ void fence_proxy_async_cta() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_cluster() {
+  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t *w) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
                : "memory");
@@ -309,8 +313,8 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
       ph_m ^= 1u;
       tc_fence_after();
     };
-    auto report = [&]() {
-      fence_proxy_async();
+    auto report = [&](bool partner_smem) {
+      if (partner_smem) fence_proxy_async_cluster(); else fence_proxy_async_cta();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) remote_arrive(mapa(opnd, 0));
@@ -346,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
             st_shared_v4(sA + half_chunk(rl, j0 + 8 * c), w);
           }
         }
-        report();
+        report(false);
         // ---- epilogue 2: B = b A + c A^2 -> sA (bf16), A and A^2 from TMEM in fp32
         wait_mma();
         if (!ok) break;
@@ -369,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
             st_shared_v4(sA + half_chunk(rl, j0 + 8 * c), w);
           }
         }
-        report();
+        report(false);
         // ---- epilogue 3: X' = s (a X + B X)
         wait_mma();
         if (!ok) break;
@@ -435,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
             }
           }
         }
-        report();
+        report(!last);   // the partner's sXcol was written
       }
     }
   }
@@ -587,7 +591,7 @@ __global__ void __launch_bounds__(kThreads1, kCtasPerSm1) himuon_tile128_kernel(
       tc_fence_after();
     };
     auto report = [&]() {
-      fence_proxy_async();
+      fence_proxy_async_cta();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(opnd);
