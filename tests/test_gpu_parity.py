@@ -184,6 +184,30 @@ def test_bf16_hyperball_gpt2_layer_two_steps():
             assert abs(o.fro(Wg[i]) - rhos[i]) / rhos[i] <= radius_tol(Wg[i], True), i
 
 
+def test_bf16_hyperball_gpt2_two_layers_six_steps():
+    """Six MuonH steps on two GPT-2 layers (12 matrices), each side keeping its own state:
+    the deviation of W may grow by one step's bound per step, the momentum stays at fp32
+    accuracy, every step's O within the NS tolerance, and the radius after every step."""
+    cfg = wl.CFG_GPT2_SMALL
+    Ws = gpt2_layer(cfg, 0, 0)[0] + gpt2_layer(cfg, 1, 0)[0]
+    rhos = [o.fro(w) for w in Ws]
+    gs = GpuSet(Ws, bf16=True)
+    p = nshb.params(eta=0.02, rho=torch.tensor(rhos, dtype=torch.float32, device="cuda"))
+    Wr = [w.copy() for w in Ws]
+    Mr = [np.zeros_like(w) for w in Ws]
+    for step in range(6):
+        Gs = gpt2_layer(cfg, 0, step)[1] + gpt2_layer(cfg, 1, step)[1]
+        gs.set_grads(Gs)
+        assert gs.step("hyperball", p) == 0
+        Wg, Mg, Og = gs.host()
+        for i in range(len(Ws)):
+            Wr[i], Mr[i], On, _ = o.hyperball_step(Wr[i], Gs[i], Mr[i], eta=0.02, rho=rhos[i])
+            assert rel_fro(Mg[i], Mr[i]) <= 1e-6, (step, i)
+            assert rel_fro(Og[i], On) <= 2e-2, (step, i)
+            assert np.linalg.norm(Wg[i] - Wr[i]) <= (step + 1) * bf16_w_tol(Wr[i], 0.02), (step, i)
+            assert abs(o.fro(Wg[i]) - rhos[i]) / rhos[i] <= radius_tol(Wg[i], True), (step, i)
+
+
 def test_bf16_muon_and_brake_steps():
     cfg = 14
     shapes = [(256, 512), (512, 256), (300, 300)]
