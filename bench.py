@@ -707,6 +707,8 @@ def main():
                      "achieved": None if ns_tflops is None else round(ns_tflops, 1),
                      "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": None if ns_tflops is None else round(ns_tflops / peak_tf, 4),
+                     "frac_of_sustained": None if ns_tflops is None else round(
+                         ns_tflops / peaks.get("bf16_tflops_sustained", DEFAULT_PEAKS["bf16_tflops_sustained"]), 4),
                      "traffic": gemm_traffic(),
                      "peak_source": f"{peak_src} bf16 burst (sustained {peaks.get('bf16_tflops_sustained')})",
                      "flops_per_launch": round(flops / max(gemm_launches, 1)),
