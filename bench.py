@@ -354,8 +354,10 @@ def run_adamh(args, rank, world, local_rank):
                 clocks=clk.summary(), e2e_ms=e2e_ms, h2d=h2d, d2h=4, n_params=n_params, shp=shp)
 
 
-def oracle_adamh_sample(layers=1):
-    """Times the oracle's AdamH step on `layers` GPT-2 layers; extrapolated by element count."""
+def oracle_adamh_sample(layers=12, steps=5):
+    """Times the oracle's AdamH step on `layers` GPT-2 layers for `steps` steps and returns
+    (seconds per full 72-matrix step, extrapolated by element count when layers < 12,
+    sample description)."""
     import numpy as np
     from newton_schulz_hyperball_b200 import workloads as wl
     from oracle import nshb_oracle as o
@@ -363,15 +365,23 @@ def oracle_adamh_sample(layers=1):
     shp = shapes()
     idx = list(range(6 * layers))
     Ws = {i: wl.init_weight(cfg, i, *shp[i], bf16=True).astype(np.float64) for i in idx}
-    Gs = {i: wl.gradient(cfg, i, 0, *shp[i], bf16=True).astype(np.float64) for i in idx}
+    Ms = {i: np.zeros(shp[i]) for i in idx}
+    Vs = {i: np.zeros(shp[i]) for i in idx}
+    rho = {i: o.fro(Ws[i]) for i in idx}
+    Gs = [{i: wl.gradient(cfg, i, s, *shp[i], bf16=True).astype(np.float64) for i in idx} for s in range(steps)]
     t0 = time.perf_counter()
-    for i in idx:
-        z = np.zeros(shp[i])
-        o.adamh_step(Ws[i], Gs[i], z, z, t=1, eta=ETA, rho=o.fro(Ws[i]))
-    dt = time.perf_counter() - t0
+    for s in range(steps):
+        for i in idx:
+            Ws[i], Ms[i], Vs[i], _, _ = o.adamh_step(Ws[i], Gs[s][i], Ms[i], Vs[i], t=s + 1, eta=ETA, rho=rho[i])
+    timed = time.perf_counter() - t0
     n_all = sum(r * c for r, c in shp)
     n_s = sum(shp[i][0] * shp[i][1] for i in idx)
-    return dt * n_all / n_s, f"{len(idx)} of 72 matrices (GPT-2 layer 0), 1 step, extrapolated by element count"
+    return timed / steps * n_all / n_s, sample_desc(len(idx), layers, steps, timed, "element count")
+
+
+def sample_desc(n_mats, layers, steps, timed, scale_by):
+    what = f"{n_mats} of 72 matrices (GPT-2 layers 0..{layers - 1}), {steps} step(s), {timed:.1f} s timed"
+    return what if n_mats == 72 else what + f", extrapolated to 72 matrices by {scale_by}"
 
 
 def report_adamh(args, r, world):
@@ -385,7 +395,7 @@ def report_adamh(args, r, world):
     fused_gbs = 28.0 * n / ((adam_ms + apply_ms) * 1e-3) / 1e9 if adam_ms + apply_ms > 0 else None
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        full, desc = oracle_adamh_sample(1)
+        full, desc = oracle_adamh_sample()
         cpu = {"value": round(full * 1e3, 3), "unit": "ms", "cores": cpu_cores(), "kind": "oracle", "sample": desc}
     return {
         "metric": "AdamH optimizer step ms; fused HBM GB/s",
@@ -539,7 +549,7 @@ def extra_params(extra):
 
 
 # --------------------------------------------------------------- CPU baseline
-def oracle_sample(layers=1, steps=1):
+def oracle_sample(layers=12, steps=2):
     """Times the fp64 oracle on `layers` of the 12 GPT-2 layers for `steps` steps and returns
     (seconds per full 72-matrix step extrapolated by NS flops, sample description)."""
     import numpy as np
@@ -556,9 +566,9 @@ def oracle_sample(layers=1, steps=1):
     for s in range(steps):
         for i in idx:
             Ws[i], Ms[i], _, _ = o.hyperball_step(Ws[i], Gs[s][i], Ms[i], eta=ETA, rho=rho[i])
-    dt = (time.perf_counter() - t0) / steps
-    full = dt * ns_flops(shp) / ns_flops([shp[i] for i in idx])
-    return full, f"{len(idx)} of 72 matrices (GPT-2 layer 0..{layers - 1}), {steps} step(s), extrapolated by NS flops"
+    timed = time.perf_counter() - t0
+    full = timed / steps * ns_flops(shp) / ns_flops([shp[i] for i in idx])
+    return full, sample_desc(len(idx), layers, steps, timed, "NS flops")
 
 
 def cpu_cores():
@@ -675,10 +685,9 @@ def main():
     peak_bw = peaks.get("hbm_gbs", DEFAULT_PEAKS["hbm_gbs"])
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t0 = time.perf_counter()
-        full, desc = oracle_sample(1, 1)
+        full, desc = oracle_sample()
         cpu = {"value": round(full * 1e3, 3), "unit": "ms", "cores": cpu_cores(), "kind": "oracle",
-               "sample": desc + f" ({time.perf_counter() - t0:.1f} s of CPU work)"}
+               "sample": desc}
     if rank != 0:
         return 0
     line = {
