@@ -39,13 +39,13 @@ DEFAULT_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustaine
 # DRAM read + write per launch of the NS GEMM from the ncu capture summarised in
 # profiles/gemm_tc2_gpt2_small_ns_iteration1.md, valid only for the kernel source it was taken on.
 GEMM_SOURCE = os.path.join(ROOT, "newton_schulz_hyperball_b200", "csrc", "ns_tc2.cu")
-GEMM_TRAFFIC = {"sha256_prefix": "5487563383b5abda", "bytes_per_launch": 372400725}
+GEMM_TRAFFIC = {"sha256_prefix": "3b2c50016d8520e6", "bytes_per_launch": 372400725}
 
 
 # DRAM read + write per launch of adam_kernel from the capture summarised in
 # profiles/adam_kernel_gpt2_small_step.md, valid only for the source it was taken on.
 STREAM_SOURCE = os.path.join(ROOT, "newton_schulz_hyperball_b200", "csrc", "stream_kernels.cu")
-ADAM_TRAFFIC = {"sha256_prefix": "df0ca9588b2f3a9d", "bytes_per_launch": 1814096720}
+ADAM_TRAFFIC = {"sha256_prefix": "705031530c8503d1", "bytes_per_launch": 1814096720}
 
 
 def source_traffic(path, rec):

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -276,16 +277,15 @@ int gemm_tiles(int mode, int mt, int nt, int bm, int bn) {
 }
 
 int device_sms() {
-  static int cache[64] = {0};
+  static PerDevice cache;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (dev < 0 || dev >= 64) return 148;
-  if (!cache[dev]) {
-    int v = 0;
+  int v = cache.get(dev);
+  if (!v) {
     if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
-    cache[dev] = v;
+    cache.set(dev, v);
   }
-  return cache[dev];
+  return v;
 }
 
 thread_local int g_last_cuda_error = 0;   // last CUDA error seen by this thread's calls
@@ -306,7 +306,7 @@ thread_local int g_last_cuda_error = 0;   // last CUDA error seen by this thread
 // CUDA events on the caller's stream; nshb_profile_read sums the elapsed times per kind.
 struct Profiler {
   std::mutex mu;
-  bool on = false;
+  std::atomic<bool> on{false};   // read without the lock on every launch
   struct Rec {
     cudaEvent_t a, b;
     int kind;

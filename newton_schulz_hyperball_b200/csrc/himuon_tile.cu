@@ -725,17 +725,17 @@ __global__ void __launch_bounds__(kThreads1, kCtasPerSm1) himuon_tile128_kernel(
 }  // namespace
 
 cudaError_t launch_himuon_tile(const HmParams &p, int num_sms, cudaStream_t s) {
-  static unsigned done_mask = 0;
+  static PerDevice attr_set;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!(done_mask & (1u << (dev & 31)))) {
+  if (!attr_set.get(dev)) {
     cudaError_t e = cudaFuncSetAttribute(himuon_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    done_mask |= 1u << (dev & 31);
+    attr_set.set(dev, 1);
   }
   if (p.total_tiles <= 0) return cudaSuccess;
-  static int max_pairs[32] = {0};
-  int &mp = max_pairs[dev & 31];
+  static PerDevice max_pairs;
+  int mp = max_pairs.get(dev);
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -756,6 +756,7 @@ cudaError_t launch_himuon_tile(const HmParams &p, int num_sms, cudaStream_t s) {
       n = num_sms / 2;
     }
     mp = n < num_sms / 2 ? n : num_sms / 2;
+    max_pairs.set(dev, mp);
   }
   const int clusters = p.total_tiles < mp ? p.total_tiles : mp;
   cudaLaunchConfig_t cfg = {};
@@ -771,11 +772,11 @@ cudaError_t launch_himuon_tile(const HmParams &p, int num_sms, cudaStream_t s) {
 }
 
 cudaError_t launch_himuon_tile128(const HmParams &p, int num_sms, cudaStream_t s) {
-  static unsigned done_mask = 0;
-  static int max_ctas[32] = {0};
+  static PerDevice max_ctas;   // set after the attribute, so nonzero means both are done
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!(done_mask & (1u << (dev & 31)))) {
+  int mc = max_ctas.get(dev);
+  if (!mc) {
     cudaError_t e =
         cudaFuncSetAttribute(himuon_tile128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES1);
     if (e != cudaSuccess) return e;
@@ -786,11 +787,11 @@ cudaError_t launch_himuon_tile128(const HmParams &p, int num_sms, cudaStream_t s
       (void)cudaGetLastError();
       per = 1;
     }
-    max_ctas[dev & 31] = num_sms * (per < kCtasPerSm1 ? per : kCtasPerSm1);   // TMEM: 256 columns per CTA
-    done_mask |= 1u << (dev & 31);
+    mc = num_sms * (per < kCtasPerSm1 ? per : kCtasPerSm1);   // TMEM: 256 columns per CTA
+    max_ctas.set(dev, mc);
   }
   if (p.total_tiles <= 0) return cudaSuccess;
-  const int grid = p.total_tiles < max_ctas[dev & 31] ? p.total_tiles : max_ctas[dev & 31];
+  const int grid = p.total_tiles < mc ? p.total_tiles : mc;
   return launch_pdl(himuon_tile128_kernel, grid, kThreads1, SMEM_BYTES1, s, p);
 }
 

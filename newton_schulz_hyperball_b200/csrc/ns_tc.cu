@@ -350,14 +350,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 
 template <int BN>
 cudaError_t launch_bn(const GemmParams &p, int num_sms, cudaStream_t s) {
-  static unsigned done_mask = 0;  // the attribute is set once per device
+  static PerDevice attr_set;  // the attribute is set once per device
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!(done_mask & (1u << (dev & 31)))) {
+  if (!attr_set.get(dev)) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg<BN>::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    done_mask |= 1u << (dev & 31);
+    attr_set.set(dev, 1);
   }
   const int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
   return launch_pdl(gemm_tc_kernel<BN>, grid, kThreads, Cfg<BN>::SMEM_BYTES, s, p);

@@ -473,19 +473,19 @@ cudaError_t encode_ws_tensor_map(CUtensorMap *map, void *ws, size_t bytes) {
 }
 
 cudaError_t launch_gemm_tc2(const GemmParams &p, int num_sms, cudaStream_t s) {
-  static unsigned done_mask = 0;  // the attribute is set once per device
+  static PerDevice attr_set;  // the attribute is set once per device
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!(done_mask & (1u << (dev & 31)))) {
+  if (!attr_set.get(dev)) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    done_mask |= 1u << (dev & 31);
+    attr_set.set(dev, 1);
   }
   if (p.total_tiles <= 0) return cudaSuccess;
   // Pairs that can be resident at once (a GPC with an odd number of free SMs leaves one
   // idle), so that the persistent grid never spills into a second wave.
-  static int max_pairs[32] = {0};
-  int &mp = max_pairs[dev & 31];
+  static PerDevice max_pairs;
+  int mp = max_pairs.get(dev);
   if (!mp) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
@@ -504,6 +504,7 @@ cudaError_t launch_gemm_tc2(const GemmParams &p, int num_sms, cudaStream_t s) {
       n = num_sms / 2;
     }
     mp = n < num_sms / 2 ? n : num_sms / 2;
+    max_pairs.set(dev, mp);
   }
   const int clusters = p.total_tiles < mp ? p.total_tiles : mp;
   cudaLaunchConfig_t cfg = {};

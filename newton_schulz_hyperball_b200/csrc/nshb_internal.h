@@ -5,9 +5,22 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 
 namespace nshb {
+
+// A once-per-device fact of a launcher (a kernel attribute already set, the CTAs that fit
+// at once): 0 until set.  Relaxed atomics, since threads that race compute the same value
+// and a lost race only repeats the query; devices past kMaxDevices are never cached.
+constexpr int kMaxDevices = 64;
+struct PerDevice {
+  std::atomic<int> v[kMaxDevices];
+  int get(int dev) const { return dev >= 0 && dev < kMaxDevices ? v[dev].load(std::memory_order_relaxed) : 0; }
+  void set(int dev, int x) {
+    if (dev >= 0 && dev < kMaxDevices) v[dev].store(x, std::memory_order_relaxed);
+  }
+};
 
 constexpr int kMaxMats = 192;   // matrices per launch of a streaming kernel (host splits larger sets)
 constexpr int kMaxProb = 192;   // GEMM problems per launch

@@ -846,17 +846,17 @@ __global__ void __launch_bounds__(kThreads, F32 ? 2 : 3) adam_kernel(const __gri
 // kernel and device.
 template <typename K>
 int stream_grid(K kernel, int slot, int dyn_smem, int total_blocks) {
-  static int cached[8][64];
+  static PerDevice cached[8];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  int g = cached[slot][dev];
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  int g = cached[slot].get(dev);
   if (g == 0) {
     int sms = 0, per = 0;
     if (dyn_smem > 0) cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kernel, kThreads, dyn_smem);
     g = (sms > 0 ? sms : 148) * (per > 0 ? per : 1);
-    cached[slot][dev] = g;
+    cached[slot].set(dev, g);
   }
   return total_blocks < g ? total_blocks : g;
 }
