@@ -395,8 +395,9 @@ def report_adamh(args, r, world):
     fused_gbs = 28.0 * n / ((adam_ms + apply_ms) * 1e-3) / 1e9 if adam_ms + apply_ms > 0 else None
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        full, desc = oracle_adamh_sample()
-        cpu = {"value": round(full * 1e3, 3), "unit": "ms", "cores": cpu_cores(), "kind": "oracle", "sample": desc}
+        with OracleThreads() as th:
+            full, desc = oracle_adamh_sample()
+        cpu = {"value": round(full * 1e3, 3), "unit": "ms", "cores": th.cores, "kind": "oracle", "sample": desc}
     return {
         "metric": "AdamH optimizer step ms; fused HBM GB/s",
         "value": round(r["ms"], 4), "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -578,19 +579,37 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
+class OracleThreads:
+    """Lets the oracle's BLAS use every core this process may run on (torchrun starts its
+    workers with OMP_NUM_THREADS=1) and records the thread count in effect, which is what
+    `cores` reports."""
+
+    def __enter__(self):
+        import numpy  # noqa: F401  (threadpoolctl sees only BLAS libraries already loaded)
+        from threadpoolctl import threadpool_info, threadpool_limits
+        self._lim = threadpool_limits(limits=cpu_cores(), user_api="blas")
+        self._lim.__enter__()
+        self.cores = max([d["num_threads"] for d in threadpool_info() if d["user_api"] == "blas"] or [1])
+        return self
+
+    def __exit__(self, *exc):
+        return self._lim.__exit__(*exc)
+
+
 def run_reference(args, rank, world):
     """The oracle on the host cores, on this workload (bounded sample per step)."""
     if rank != 0:
         return None
-    for _ in range(args.warmup):
-        oracle_sample(1, 1)
     times = []
     desc = None
-    for _ in range(args.steps):
-        full, desc = oracle_sample(1, 1)
-        times.append(full)
+    with OracleThreads() as th:
+        for _ in range(args.warmup):
+            oracle_sample(1, 1)
+        for _ in range(args.steps):
+            full, desc = oracle_sample(1, 1)
+            times.append(full)
     ms = 1e3 * statistics.median(times)
-    return dict(ms=ms, desc=desc)
+    return dict(ms=ms, desc=desc, cores=th.cores)
 
 
 def main():
@@ -628,7 +647,7 @@ def main():
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "impl": "reference",
                 "config": {"workload": WORKLOAD, "matrices": 72, "params": 84934656},
-                "cpu_baseline": {"value": round(r["ms"], 3), "unit": "ms", "cores": cpu_cores(), "kind": "oracle",
+                "cpu_baseline": {"value": round(r["ms"], 3), "unit": "ms", "cores": r["cores"], "kind": "oracle",
                                  "sample": r["desc"]},
                 "e2e": {"value": round(r["ms"], 3), "unit": "ms", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
@@ -685,8 +704,9 @@ def main():
     peak_bw = peaks.get("hbm_gbs", DEFAULT_PEAKS["hbm_gbs"])
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        full, desc = oracle_sample()
-        cpu = {"value": round(full * 1e3, 3), "unit": "ms", "cores": cpu_cores(), "kind": "oracle",
+        with OracleThreads() as th:
+            full, desc = oracle_sample()
+        cpu = {"value": round(full * 1e3, 3), "unit": "ms", "cores": th.cores, "kind": "oracle",
                "sample": desc}
     if rank != 0:
         return 0
@@ -732,11 +752,19 @@ def main():
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
     return 0
 
 
+def run():
+    """main(), then every rank releases its process group, whichever way main returned."""
+    try:
+        return main()
+    finally:
+        if "torch.distributed" in sys.modules:
+            import torch.distributed as dist
+            if dist.is_available() and dist.is_initialized():
+                dist.destroy_process_group()
+
+
 if __name__ == "__main__":
-    sys.exit(main())
+    sys.exit(run())
