@@ -17,11 +17,15 @@
  *        radial_brake_step  plain Muon step, then ||w|| <- ||w_prev|| + s (||w|| - ||w_prev||)
  *                           ("Refactor of pre/post weight update hook functions", PR #224,
  *                            RadialBrake description)
+ *        relative_update_step  Muon step of length lr ||W||_F along O (same PR, RelativeUpdate)
  *      and two variants of step 2:
  *        himuon_step        NS run independently on every T x T tile, then Hyperball
  *                           ("Hierarchical Muon: Tiled Newton-Schulz Updates", abstract)
  *        newton_muon_step   NS of U (Z Z^T + lambda I)^-1, then Hyperball
  *                           ("The Newton-Muon Optimizer", abstract)
+ *      and one step without NS:
+ *        adamh_step         Adam's bias-corrected direction in place of O, then Hyperball
+ *                           (Hyperball paper, Method)
  *
  * Conventions shared by every entry point:
  *   - Every data pointer (W, G, M, O_out, rho, Z, workspace, norms) is a DEVICE pointer
