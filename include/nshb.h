@@ -91,7 +91,9 @@ typedef enum {
  * other layouts take a slower element-wise path.  O_out needs element alignment.
  * O_out (optional, may be NULL) receives the orthogonalised update O = NS_K(U)
  * (before any step-length or shape scaling), dtype w_dtype, leading dimension cols.
- * z_index picks the layer input Z of newton_muon_step (ignored elsewhere). */
+ * z_index picks the layer input Z of newton_muon_step (ignored elsewhere).
+ * Sizes: rows and cols up to 2^20 and ld up to 2^30; larger ones return
+ * NSHB_ERR_UNSUPPORTED. */
 typedef struct {
   int64_t rows, cols, ld;
   int32_t w_dtype; /* nshb_dtype */
@@ -171,9 +173,10 @@ nshb_status himuon_step(const nshb_matrix *mats, int32_t n_mats, const nshb_para
  * lambda = ridge_rel tr(Z Z^T) / d_in, solved through an fp32 Cholesky factorisation,
  * then O = NS_K(P) and the Hyperball rule (U is the Nesterov momentum update).  Z[j] is a
  * DEVICE pointer to a bf16 row-major z_rows[j] x n_tokens matrix (leading dimension
- * n_tokens, 16-byte aligned); n_tokens and every z_rows[j] must be multiples of 64 (up to
- * 16384 rows); matrix i uses Z[mats[i].z_index], which needs z_rows == cols.  Z and z_rows
- * are HOST arrays of n_z entries (n_z <= 192).  A pivot that is not positive in fp32 sets
+ * n_tokens, 16-byte aligned); n_tokens (up to 2^24) and every z_rows[j] (up to 16384) must be
+ * multiples of 64, else NSHB_ERR_SHAPE; matrix i uses Z[mats[i].z_index] (an index outside
+ * [0, n_z) is NSHB_ERR_PARAM), which needs z_rows == cols (else NSHB_ERR_SHAPE).  Z and z_rows
+ * are HOST arrays of n_z entries (1 <= n_z <= 192).  A pivot that is not positive in fp32 sets
  * NSHB_DEV_NOT_SPD.  bf16 NS only. */
 nshb_status newton_muon_step(const nshb_matrix *mats, int32_t n_mats, const void *const *Z,
                              const int64_t *z_rows, int32_t n_z, int64_t n_tokens,

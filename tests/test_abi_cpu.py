@@ -188,3 +188,59 @@ def test_chunked_step_workspace_bounds_are_checked_before_any_launch():
     with pytest.raises(nshb.NshbError) as e:
         nshb.workspace_size_min(mats, p, nshb.NSHB_OP_ADAMH)
     assert e.value.status == nshb.NSHB_ERR_PARAM
+
+
+@pytest.mark.parametrize("shape,ld", [(((1 << 20) + 1, 8), None), ((8, (1 << 20) + 1), None),
+                                      ((8, 8), (1 << 30) + 1)])
+def test_sizes_beyond_the_documented_limits_are_unsupported(shape, ld):
+    with pytest.raises(nshb.NshbError) as e:
+        ws_size(fake_mats([shape], ld=ld), nshb.params(), nshb.NSHB_OP_HYPERBALL)
+    assert e.value.status == nshb.NSHB_ERR_UNSUPPORTED
+
+
+def newton_mats(cols_list, z_index):
+    m = fake_mats([(768, c) for c in cols_list])
+    for i, zi in enumerate(z_index):
+        m[i].z_index = zi
+    return m
+
+
+@pytest.mark.parametrize("z_rows,n_tokens,z_index,code", [
+    ([768], 8100, [0], nshb.NSHB_ERR_SHAPE),          # tokens not a multiple of 64
+    ([768], 0, [0], nshb.NSHB_ERR_SHAPE),
+    ([768], (1 << 24) + 64, [0], nshb.NSHB_ERR_SHAPE),
+    ([760], 8192, [0], nshb.NSHB_ERR_SHAPE),          # Z rows not a multiple of 64
+    ([16384 + 64], 8192, [0], nshb.NSHB_ERR_SHAPE),
+    ([768], 8192, [1], nshb.NSHB_ERR_PARAM),          # z_index outside [0, n_z)
+    ([768], 8192, [-1], nshb.NSHB_ERR_PARAM),
+    ([1536], 8192, [0], nshb.NSHB_ERR_SHAPE),         # Z rows != cols of the matrix
+    ([], 8192, [0], nshb.NSHB_ERR_NULL),              # no Z at all
+])
+def test_newton_muon_argument_errors(z_rows, n_tokens, z_index, code):
+    with pytest.raises(nshb.NshbError) as e:
+        nshb.workspace_size(newton_mats([768], z_index), nshb.params(), nshb.NSHB_OP_NEWTON_MUON,
+                            z_rows=z_rows, n_tokens=n_tokens)
+    assert e.value.status == code
+
+
+def test_newton_muon_workspace_and_step_checks_before_launch():
+    p = nshb.params()
+    m = newton_mats([768, 768, 3072], [0, 0, 1])
+    a = nshb.workspace_size(m, p, nshb.NSHB_OP_NEWTON_MUON, z_rows=[768, 3072], n_tokens=4096)
+    b = nshb.workspace_size(m, p, nshb.NSHB_OP_NEWTON_MUON, z_rows=[768, 3072], n_tokens=8192)
+    # the bf16 panel copy of every Z grows with the token count: (768 + 3072) x 4096 x 2 bytes more
+    assert b - a >= (768 + 3072) * 4096 * 2
+    assert a > nshb.workspace_size(m, p, nshb.NSHB_OP_HYPERBALL)
+    with pytest.raises(nshb.NshbError) as e:   # Newton-Muon runs the bf16 NS only
+        nshb.workspace_size(m, nshb.params(ns_precision=nshb.NSHB_F32), nshb.NSHB_OP_NEWTON_MUON,
+                            z_rows=[768, 3072], n_tokens=4096)
+    assert e.value.status == nshb.NSHB_ERR_UNSUPPORTED
+    lib = nshb.lib()
+    zr = (ctypes.c_int64 * 2)(768, 3072)
+    zp = (ctypes.c_void_p * 2)(0x30000000, 0x30000010)
+    # Z NULL, a misaligned Z, a short workspace: all rejected before any CUDA call
+    assert lib.newton_muon_step(m, 3, None, zr, 2, 4096, ctypes.byref(p), 0x20000000, a, None) == nshb.NSHB_ERR_NULL
+    bad = (ctypes.c_void_p * 2)(0x30000000, 0x30000008)
+    assert lib.newton_muon_step(m, 3, bad, zr, 2, 4096, ctypes.byref(p), 0x20000000, a, None) == nshb.NSHB_ERR_SHAPE
+    assert lib.newton_muon_step(m, 3, zp, zr, 2, 4096, ctypes.byref(p), 0x20000000, a - 256, None) == \
+        nshb.NSHB_ERR_WORKSPACE
