@@ -73,12 +73,13 @@ def shapes():
     return [(r, c) for _, r, c in wl.gpt2_small_shapes(12)]
 
 
-def ns_flops(shp, K=5):
-    """Algorithmic NS work per step: K (3 r^2 s + r^3), symmetric products counted once."""
+def ns_flops(shp, K=5, dense=False):
+    """Algorithmic NS work per step: K (3 r^2 s + r^3), symmetric products counted once;
+    dense=True gives the dense-equivalent K (4 r^2 s + 2 r^3) of the full products."""
     tot = 0.0
     for r, c in shp:
         rr, ss = min(r, c), max(r, c)
-        tot += K * (3.0 * rr * rr * ss + rr ** 3)
+        tot += K * ((4.0 * rr * rr * ss + 2.0 * rr ** 3) if dense else (3.0 * rr * rr * ss + rr ** 3))
     return tot
 
 
@@ -397,7 +398,8 @@ def report_adamh(args, r, world):
     if world == 1 and not args.no_cpu_baseline:
         with OracleThreads() as th:
             full, desc = oracle_adamh_sample()
-        cpu = {"value": round(full * 1e3, 3), "unit": "ms", "cores": th.cores, "kind": "oracle", "sample": desc}
+        cpu = {"value": round(full * 1e3, 3), "unit": "ms", "cores": th.cores, "affinity_cores": th.affinity,
+               "kind": "oracle", "sample": desc}
     return {
         "metric": "AdamH optimizer step ms; fused HBM GB/s",
         "value": round(r["ms"], 4), "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -590,6 +592,7 @@ class OracleThreads:
         self._lim = threadpool_limits(limits=cpu_cores(), user_api="blas")
         self._lim.__enter__()
         self.cores = max([d["num_threads"] for d in threadpool_info() if d["user_api"] == "blas"] or [1])
+        self.affinity = cpu_cores()
         return self
 
     def __exit__(self, *exc):
@@ -609,7 +612,7 @@ def run_reference(args, rank, world):
             full, desc = oracle_sample(1, 1)
             times.append(full)
     ms = 1e3 * statistics.median(times)
-    return dict(ms=ms, desc=desc, cores=th.cores)
+    return dict(ms=ms, desc=desc, cores=th.cores, affinity=th.affinity)
 
 
 def main():
@@ -647,7 +650,8 @@ def main():
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "impl": "reference",
                 "config": {"workload": WORKLOAD, "matrices": 72, "params": 84934656},
-                "cpu_baseline": {"value": round(r["ms"], 3), "unit": "ms", "cores": r["cores"], "kind": "oracle",
+                "cpu_baseline": {"value": round(r["ms"], 3), "unit": "ms", "cores": r["cores"],
+                                 "affinity_cores": r["affinity"], "kind": "oracle",
                                  "sample": r["desc"]},
                 "e2e": {"value": round(r["ms"], 3), "unit": "ms", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
@@ -706,8 +710,8 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         with OracleThreads() as th:
             full, desc = oracle_sample()
-        cpu = {"value": round(full * 1e3, 3), "unit": "ms", "cores": th.cores, "kind": "oracle",
-               "sample": desc}
+        cpu = {"value": round(full * 1e3, 3), "unit": "ms", "cores": th.cores, "affinity_cores": th.affinity,
+               "kind": "oracle", "sample": desc}
     if rank != 0:
         return 0
     line = {
@@ -730,6 +734,7 @@ def main():
         "throughput": {"value": round(world * n / (r["ms"] * 1e-3), 1), "unit": "params/s"},
         "ns_tflops": None if ns_tflops is None else round(ns_tflops, 1),
         "ns_frac_of_bf16_peak": None if ns_tflops is None else round(ns_tflops / peak_tf, 4),
+        "ns_tflops_dense_equiv": None if gemm_ms <= 0 else round(ns_flops(shp, dense=True) / (gemm_ms * 1e-3) / 1e12, 1),
         "fused_gbs": None if fused_gbs is None else round(fused_gbs, 1),
         "fused_frac_of_hbm": None if fused_gbs is None else round(fused_gbs / peak_bw, 4),
         "roofline": {"bound": "tensor", "kernel": "gemm_tc2_kernel (NS Gram / polynomial / update, CTA pairs)",
