@@ -208,6 +208,29 @@ def test_bf16_hyperball_gpt2_two_layers_six_steps():
             assert abs(o.fro(Wg[i]) - rhos[i]) / rhos[i] <= radius_tol(Wg[i], True), (step, i)
 
 
+def test_bf16_hyperball_gpt2_full_set_three_steps():
+    """All 72 GPT-2-small matrices in one call per step, three MuonH steps, each side keeping
+    its own state: every matrix's O, M, W and radius after every step."""
+    cfg = wl.CFG_GPT2_SMALL
+    Ws = [w for layer in range(12) for w in gpt2_layer(cfg, layer, 0)[0]]
+    rhos = [o.fro(w) for w in Ws]
+    gs = GpuSet(Ws, bf16=True)
+    p = nshb.params(eta=0.02, rho=torch.tensor(rhos, dtype=torch.float32, device="cuda"))
+    Wr = [w.copy() for w in Ws]
+    Mr = [np.zeros_like(w) for w in Ws]
+    for step in range(3):
+        Gs = [wl.gradient(cfg, i, step, *w.shape, bf16=True).astype(np.float64) for i, w in enumerate(Ws)]
+        gs.set_grads(Gs)
+        assert gs.step("hyperball", p) == 0
+        Wg, Mg, Og = gs.host()
+        for i in range(len(Ws)):
+            Wr[i], Mr[i], On, _ = o.hyperball_step(Wr[i], Gs[i], Mr[i], eta=0.02, rho=rhos[i])
+            assert rel_fro(Mg[i], Mr[i]) <= 1e-6, (step, i)
+            assert rel_fro(Og[i], On) <= 2e-2, (step, i, rel_fro(Og[i], On))
+            assert np.linalg.norm(Wg[i] - Wr[i]) <= (step + 1) * bf16_w_tol(Wr[i], 0.02), (step, i)
+            assert abs(o.fro(Wg[i]) - rhos[i]) / rhos[i] <= radius_tol(Wg[i], True), (step, i)
+
+
 def test_bf16_muon_and_brake_steps():
     cfg = 14
     shapes = [(256, 512), (512, 256), (300, 300)]
