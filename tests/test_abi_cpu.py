@@ -244,3 +244,21 @@ def test_newton_muon_workspace_and_step_checks_before_launch():
     assert lib.newton_muon_step(m, 3, bad, zr, 2, 4096, ctypes.byref(p), 0x20000000, a, None) == nshb.NSHB_ERR_SHAPE
     assert lib.newton_muon_step(m, 3, zp, zr, 2, 4096, ctypes.byref(p), 0x20000000, a - 256, None) == \
         nshb.NSHB_ERR_WORKSPACE
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """Without libnshb.so there is no step at all: no CPU fallback, an ImportError that says so."""
+    with pytest.raises(ImportError, match="no fallback"):
+        _abi.load(str(tmp_path / "libnshb.so"))
+
+
+def test_package_never_reaches_the_oracle():
+    """The product package (binding, planner helpers, sharding) neither imports nor reads
+    anything under oracle/: the oracle is test infrastructure only."""
+    pkg = pathlib.Path(nshb.__file__).resolve().parent
+    for f in sorted(pkg.rglob("*")):
+        if f.suffix not in (".py", ".cu", ".cuh", ".h", ".cpp"):
+            continue
+        text = f.read_text()
+        assert not re.search(r"^\s*(from|import)\s+oracle\b", text, flags=re.M), f
+        assert "nshb_oracle" not in text, f
