@@ -133,6 +133,19 @@ def test_momentum_closed_form_constant_gradient():
         assert np.array_equal(U_plain, M)
 
 
+def test_plain_momentum_closed_form_constant_gradient():
+    """Without Nesterov the update is the new buffer itself: U_t = M_t = (1 - b^t) G for a
+    constant G from M0 = 0 (an update taken from the old buffer would give (1 - b^(t-1)) G)."""
+    rng = np.random.default_rng(9)
+    G = rng.standard_normal((4, 3))
+    beta = 0.9
+    M = np.zeros_like(G)
+    for t in range(1, 6):
+        M, U = o.momentum(M, G, beta, False)
+        assert np.allclose(U, (1 - beta ** t) * G, atol=1e-14)
+        assert np.array_equal(U, M)
+
+
 def test_sum_form_momentum_gives_same_update():
     """Keller's sum form M' = b M' + G is (1-b)^-1 times the EMA, so NS agrees (scale invariance)."""
     rng = np.random.default_rng(8)
