@@ -68,13 +68,16 @@ def all_gather_weights(weights, plan: ShardPlan, group=None) -> None:
 
     The owned matrices of each rank are packed into one flat buffer (padded to the
     largest rank's size) and exchanged with a single all_gather_into_tensor; each rank
-    then unpacks every other rank's matrices into place."""
+    then unpacks every other rank's matrices into place.  All weights share one dtype and
+    device (the buffer is of that dtype, so a mixed set would be rounded); any strides."""
     import torch.distributed as dist
     world = plan.world
-    if world == 1:
+    if world == 1 or not weights:
         return
     dtype = weights[0].dtype
     device = weights[0].device
+    if any(w.dtype != dtype or w.device != device for w in weights):
+        raise ValueError("all_gather_weights needs every weight in one dtype on one device")
     per_rank = [[i for i, r in enumerate(plan.owner) if r == k] for k in range(world)]
     sizes = [sum(weights[i].numel() for i in idx) for idx in per_rank]
     cap = max(sizes)
@@ -96,7 +99,7 @@ def all_gather_weights(weights, plan: ShardPlan, group=None) -> None:
         off = 0
         for i in per_rank[k]:
             n = weights[i].numel()
-            weights[i].reshape(-1).copy_(recv[base + off:base + off + n])
+            weights[i].copy_(recv[base + off:base + off + n].view(weights[i].shape))
             off += n
 
 

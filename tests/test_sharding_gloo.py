@@ -1,5 +1,5 @@
 """Multi-rank host logic on CPU: LPT ownership and the all-gather of updated weights,
-run as two gloo ranks (spawned processes).  Each rank steps only its own matrices with the
+run as two or three gloo ranks (spawned processes).  Each rank steps only its own matrices with the
 oracle; after the exchange every rank must hold exactly the single-process result."""
 import os
 import socket
@@ -45,6 +45,9 @@ def _worker(rank, world, port, shapes, out_dir):
     try:
         plan = sharding.make_plan(shapes, world, rank)
         W = [torch.from_numpy(wl.init_weight(31, i, r, c, bf16=False).astype(np.float64)) for i, (r, c) in enumerate(shapes)]
+        # matrix 0 held as a transposed view (non-contiguous storage), as a framework may hold it
+        W[0] = W[0].t().contiguous().t()
+        assert not W[0].is_contiguous()
         M = [torch.zeros_like(w) for w in W]
         rho = [float(torch.linalg.norm(w)) for w in W]
         for step in range(2):
@@ -62,10 +65,13 @@ def _worker(rank, world, port, shapes, out_dir):
         dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_match_single_process(tmp_path):
+@pytest.mark.parametrize("world,shapes", [
+    (2, [(24, 16), (16, 40), (32, 32), (8, 20), (48, 12)]),
+    (3, [(24, 16), (16, 40), (32, 32), (8, 20), (48, 12)]),   # uneven ownership
+    (3, [(24, 16), (16, 40)]),                                # one rank owns nothing
+])
+def test_gloo_ranks_match_single_process(tmp_path, world, shapes):
     from oracle import nshb_oracle as o
-    shapes = [(24, 16), (16, 40), (32, 32), (8, 20), (48, 12)]
-    world = 2
     mp.start_processes(_worker, args=(world, _free_port(), shapes, str(tmp_path)), nprocs=world,
                        start_method="spawn", join=True)
     got = [torch.load(tmp_path / f"w{r}.pt") for r in range(world)]
@@ -79,6 +85,13 @@ def test_two_gloo_ranks_match_single_process(tmp_path):
             W[i], M[i], _, _ = o.hyperball_step(W[i], G, M[i], eta=0.02, rho=rho[i])
     for i in range(len(shapes)):
         # every rank holds the owner's bits ...
-        assert torch.equal(got[0][i], got[1][i]), i
+        for r in range(1, world):
+            assert torch.equal(got[0][i], got[r][i]), (i, r)
         # ... which equal the single-process result up to BLAS summation order across processes
         assert float((got[0][i] - torch.from_numpy(W[i])).abs().max()) <= 1e-13, i
+
+
+def test_all_gather_rejects_mixed_dtypes():
+    plan = sharding.ShardPlan([0, 1], 2, 0)
+    with pytest.raises(ValueError):
+        sharding.all_gather_weights([torch.zeros(2, 2), torch.zeros(2, 2, dtype=torch.bfloat16)], plan)
