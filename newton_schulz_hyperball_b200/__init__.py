@@ -67,19 +67,38 @@ def _dtype_code(t) -> int:
 
 
 def matrices(W, G, M, O_out=None, z_index=None):
-    """ctypes array of nshb_matrix for lists of 2-D CUDA tensors (row-major, unit column stride)."""
+    """ctypes array of nshb_matrix for lists of 2-D CUDA tensors (row-major, unit column stride).
+
+    The library receives bare pointers and cannot see a tensor's size, so what the C
+    header requires is checked here: G of W's shape, dtype and strides; M float32 of W's
+    shape and strides; O_out[i] (when given, None entries allowed) contiguous with W's
+    shape and dtype; every tensor on W[0]'s CUDA device."""
+    import torch
     n = len(W)
+    if len(G) != n or len(M) != n or (O_out is not None and len(O_out) != n) or \
+            (z_index is not None and len(z_index) != n):
+        raise ValueError("W, G, M (and O_out, z_index when given) must have one entry per matrix")
     arr = (nshb_matrix * max(n, 1))()
+    dev = W[0].device if n else None
     for i in range(n):
         w, g, m = W[i], G[i], M[i]
-        if w.dim() != 2 or w.stride(1) != 1 or g.stride() != w.stride() or m.stride() != w.stride():
-            raise ValueError("W, G and M must be 2-D with equal strides and unit column stride")
+        if w.dim() != 2 or g.shape != w.shape or m.shape != w.shape:
+            raise ValueError(f"matrix {i}: W, G and M must be 2-D of one shape")
+        if w.stride(1) != 1 or g.stride() != w.stride() or m.stride() != w.stride():
+            raise ValueError(f"matrix {i}: W, G and M must have equal strides and unit column stride")
+        if g.dtype != w.dtype or m.dtype != torch.float32:
+            raise TypeError(f"matrix {i}: G must have W's dtype and M must be float32")
+        o = O_out[i] if O_out is not None else None
+        if o is not None and (o.shape != w.shape or o.dtype != w.dtype or not o.is_contiguous()):
+            raise ValueError(f"matrix {i}: O_out must be a contiguous tensor of W's shape and dtype")
+        if any(t.device != dev for t in (w, g, m) + ((o,) if o is not None else ())) or dev.type != "cuda":
+            raise ValueError(f"matrix {i}: every tensor must be on one CUDA device")
         arr[i].rows, arr[i].cols = w.shape
         arr[i].ld = w.stride(0)
         arr[i].w_dtype = _dtype_code(w)
         arr[i].z_index = -1 if z_index is None else int(z_index[i])
         arr[i].W, arr[i].G, arr[i].M = _ptr(w), _ptr(g), _ptr(m)
-        arr[i].O_out = _ptr(O_out[i]) if O_out is not None else None
+        arr[i].O_out = _ptr(o)
     arr._n = n
     arr._keep = (W, G, M, O_out)
     return arr

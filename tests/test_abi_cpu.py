@@ -262,3 +262,29 @@ def test_package_never_reaches_the_oracle():
         text = f.read_text()
         assert not re.search(r"^\s*(from|import)\s+oracle\b", text, flags=re.M), f
         assert "nshb_oracle" not in text, f
+
+
+def test_matrices_checks_what_the_library_cannot_see():
+    """The C ABI gets bare pointers, so the binding checks sizes, dtypes, strides and the
+    device before any pointer reaches the library (here with CPU tensors: every error is
+    raised before the device check, and a consistent CPU set is refused as not CUDA)."""
+    import torch
+    W = torch.zeros(8, 16, dtype=torch.bfloat16)
+    G = torch.zeros_like(W)
+    M = torch.zeros(8, 16)
+    cases = [
+        (ValueError, dict(G=[torch.zeros(4, 16, dtype=torch.bfloat16)])),          # G smaller than W
+        (ValueError, dict(M=[torch.zeros(8, 8)])),                                  # M of another shape
+        (TypeError, dict(G=[torch.zeros(8, 16)])),                                  # G fp32 with bf16 W
+        (TypeError, dict(M=[torch.zeros(8, 16, dtype=torch.bfloat16)])),            # M not fp32
+        (ValueError, dict(O=[torch.zeros(8, 8, dtype=torch.bfloat16)])),            # O_out too small
+        (ValueError, dict(O=[torch.zeros(8, 16)])),                                 # O_out of another dtype
+        (ValueError, dict(O=[torch.zeros(16, 8, dtype=torch.bfloat16).t()])),       # O_out not contiguous
+        (ValueError, dict(W=[torch.zeros(16, 8, dtype=torch.bfloat16).t()])),       # W column stride != 1
+        (ValueError, dict(G=[])),                                                   # list lengths differ
+        (ValueError, dict()),                                                       # CPU tensors
+    ]
+    for exc, kw in cases:
+        with pytest.raises(exc):
+            nshb.matrices(kw.get("W", [W]), kw.get("G", [G]), kw.get("M", [M]), kw.get("O"))
+    assert nshb.matrices([], [], [])._n == 0
