@@ -57,6 +57,28 @@ def _ptr(t):
     return t.data_ptr()
 
 
+def _device_arg(t, what: str, dtype=None, min_numel: int = 0) -> None:
+    """Checks a tensor that becomes a bare device pointer: on a CUDA device, contiguous, of
+    `dtype` and at least `min_numel` elements.  Raw pointers (ints) and None pass unchecked."""
+    if t is None or isinstance(t, int):
+        return
+    if t.device.type != "cuda":
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{what} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    if t.numel() < min_numel:
+        raise ValueError(f"{what} has {t.numel()} elements, needs {min_numel}")
+
+
+def _check_rho(p, n: int) -> None:
+    """p.rho is read for every matrix of the call: a tensor must have an entry per matrix."""
+    rn = getattr(p, "_rho_n", None)
+    if rn is not None and rn < n:
+        raise ValueError(f"rho has {rn} entries for {n} matrices")
+
+
 def _dtype_code(t) -> int:
     import torch
     if t.dtype == torch.bfloat16:
@@ -120,8 +142,11 @@ def params(**kw) -> nshb_params:
                 keep.append(buf)
                 p.coeffs = ctypes.cast(buf, ctypes.POINTER(ctypes.c_float))
         elif k == "rho":
+            import torch
+            _device_arg(v, "rho", torch.float32)
             keep.append(v)
             p.rho = _ptr(v)
+            p._rho_n = None if v is None or isinstance(v, int) else v.numel()
         elif k == "nesterov":
             p.nesterov = 1 if v else 0
         else:
@@ -166,10 +191,12 @@ def _stream(stream):
 def _ws(ws):
     if isinstance(ws, tuple):
         return ws
+    _device_arg(ws, "workspace")
     return ws.data_ptr(), ws.numel() * ws.element_size()
 
 
 def _step(name, mats, p, ws, stream):
+    _check_rho(p, _n(mats))
     ptr, nbytes = _ws(ws)
     fn = getattr(lib(), name)
     _check(fn(mats, _n(mats), ctypes.byref(p), ptr, nbytes, _stream(stream)), name)
@@ -201,6 +228,7 @@ def workspace_size_min(mats, p, op: int) -> int:
 
 def step_chunked(op: int, mats, p, ws, stream=None) -> int:
     """The step of kind `op` over the matrices in chunks that fit the workspace; returns the chunk count."""
+    _check_rho(p, _n(mats))
     ptr, nbytes = _ws(ws)
     n = ctypes.c_int32(0)
     _check(lib().nshb_step_chunked(op, mats, _n(mats), ctypes.byref(p), ptr, nbytes, _stream(stream),
@@ -224,15 +252,35 @@ def adam_params(**kw) -> "_abi.nshb_adam_params":
 
 
 def adamh_step(mats, V, a, p, ws, stream=None):
-    """AdamH step; mats[i].M is the first moment, V[i] (CUDA fp32 tensor or pointer) the second."""
-    ptr, nbytes = _ws(ws)
+    """AdamH step; mats[i].M is the first moment, V[i] (CUDA fp32 tensor or pointer) the second,
+    with W's shape and strides."""
+    import torch
     n = _n(mats)
+    if len(V) != n:
+        raise ValueError("V needs one entry per matrix")
+    W = getattr(mats, "_keep", (None,))[0]
+    for i, v in enumerate(V):
+        if v is None or isinstance(v, int):
+            continue
+        if v.device.type != "cuda" or v.dtype != torch.float32:
+            raise TypeError(f"V[{i}] must be a CUDA float32 tensor")
+        if W is not None and (v.shape != W[i].shape or v.stride() != W[i].stride()):
+            raise ValueError(f"V[{i}] must have W's shape and strides")
+    _check_rho(p, n)
+    ptr, nbytes = _ws(ws)
     vp = (ctypes.c_void_p * max(n, 1))(*[_ptr(v) for v in V])
     _check(lib().adamh_step(mats, n, vp, ctypes.byref(a), ctypes.byref(p), ptr, nbytes, _stream(stream)),
            "adamh_step")
 
 
 def newton_muon_step(mats, Z, n_tokens: int, p, ws, stream=None):
+    """Newton-Muon step; Z[j] a contiguous bf16 CUDA tensor of z_rows x n_tokens."""
+    import torch
+    for j, z in enumerate(Z):
+        _device_arg(z, f"Z[{j}]", torch.bfloat16)
+        if z.dim() != 2 or z.shape[1] != n_tokens:
+            raise ValueError(f"Z[{j}] must be 2-D with n_tokens = {n_tokens} columns")
+    _check_rho(p, _n(mats))
     ptr, nbytes = _ws(ws)
     nz = len(Z)
     zp = (ctypes.c_void_p * max(nz, 1))(*[_ptr(z) for z in Z])
@@ -242,12 +290,16 @@ def newton_muon_step(mats, Z, n_tokens: int, p, ws, stream=None):
 
 
 def fro_norms(mats, out, ws, stream=None):
+    import torch
+    _device_arg(out, "out", torch.float32, _n(mats))
     ptr, nbytes = _ws(ws)
     _check(lib().nshb_fro_norms(mats, _n(mats), _ptr(out), ptr, nbytes, _stream(stream)), "nshb_fro_norms")
 
 
 def fro_norms_static(mats, out, stream=None):
     """||W_i||_F into `out` without a workspace (scratch is a fixed array in the library)."""
+    import torch
+    _device_arg(out, "out", torch.float32, _n(mats))
     _check(lib().nshb_fro_norms_static(mats, _n(mats), _ptr(out), _stream(stream)), "nshb_fro_norms_static")
 
 

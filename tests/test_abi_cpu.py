@@ -288,3 +288,34 @@ def test_matrices_checks_what_the_library_cannot_see():
         with pytest.raises(exc):
             nshb.matrices(kw.get("W", [W]), kw.get("G", [G]), kw.get("M", [M]), kw.get("O"))
     assert nshb.matrices([], [], [])._n == 0
+
+
+def test_pointer_arguments_are_checked_before_the_library_sees_them():
+    """rho, V, Z, out and the workspace become bare device pointers: host tensors, wrong
+    dtypes, short arrays and mismatched lengths are refused by the binding."""
+    import torch
+    with pytest.raises(ValueError):
+        nshb.params(rho=torch.ones(3))                               # rho on the host
+    assert getattr(nshb.params(rho=0x30000000), "_rho_n", None) is None  # raw pointer: caller's word
+    mats = fake_mats([(64, 64), (100, 30), (8, 8)])
+    p = nshb.params()
+    p._rho_n = 2                                                     # a 2-entry rho for 3 matrices
+    ws = (0x40000000, nshb.workspace_size(mats, nshb.params(), nshb.NSHB_OP_HYPERBALL))
+    for fn in (nshb.hyperball_step, nshb.muon_step, nshb.himuon_step, nshb.relative_update_step):
+        with pytest.raises(ValueError, match="rho"):
+            fn(mats, p, ws, stream=0)
+    with pytest.raises(ValueError, match="rho"):
+        nshb.step_chunked(nshb.NSHB_OP_HYPERBALL, mats, p, ws, stream=0)
+    a = nshb.adam_params()
+    with pytest.raises(ValueError):
+        nshb.adamh_step(mats, [0x30000000], a, nshb.params(), ws, stream=0)          # V too short
+    with pytest.raises(TypeError):
+        nshb.adamh_step(mats, [torch.zeros(64, 64)] * 3, a, nshb.params(), ws, stream=0)  # V on the host
+    with pytest.raises(ValueError):
+        nshb.newton_muon_step(mats, [torch.zeros(64, 128, dtype=torch.bfloat16)], 128, nshb.params(), ws, stream=0)
+    with pytest.raises(ValueError):
+        nshb.fro_norms(mats, torch.zeros(3), ws, stream=0)           # out on the host
+    with pytest.raises(ValueError):
+        nshb.fro_norms_static(mats, torch.zeros(3), stream=0)
+    with pytest.raises(ValueError):
+        nshb.device_status(torch.zeros(256, dtype=torch.uint8))      # workspace on the host
