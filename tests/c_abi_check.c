@@ -1,6 +1,6 @@
 /* Calls the library through include/nshb.h from C (no GPU needed: argument checking and
  * workspace sizing only) and prints what tests/test_c_abi.py compares with the ctypes
- * binding.  Built with gcc -std=c11 -pedantic -Wall -Wextra -Werror. */
+ * binding.  Built as C11 and as C++17 with -pedantic -Wall -Wextra -Werror. */
 #include <stddef.h>
 #include <stdint.h>
 #include <stdio.h>

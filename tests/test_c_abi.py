@@ -1,4 +1,4 @@
-"""The boundary is a C ABI: a C11 program built against include/nshb.h and linked with
+"""The boundary is a C ABI: a program built against include/nshb.h (as C11 and as C++17) and linked with
 libnshb.so sees the same struct layouts, defaults, workspace sizes and argument errors as
 the ctypes binding (CPU only: nothing here launches a kernel)."""
 import ctypes
@@ -23,12 +23,15 @@ def fake(shapes):
     return arr
 
 
-@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
-def test_c_program_sees_the_same_abi(tmp_path):
+@pytest.mark.parametrize("compiler,std", [("gcc", "-std=c11"), ("g++", "-std=c++17")])
+def test_c_program_sees_the_same_abi(tmp_path, compiler, std):
+    if shutil.which(compiler) is None:
+        pytest.skip(f"needs {compiler}")
     lib_dir = pathlib.Path(_abi.LIB_PATH).parent
     exe = tmp_path / "c_abi_check"
-    subprocess.run(["gcc", "-std=c11", "-pedantic", "-Wall", "-Wextra", "-Werror", "-I", str(ROOT / "include"),
-                    str(ROOT / "tests" / "c_abi_check.c"), "-L", str(lib_dir), "-lnshb",
+    lang = ["-x", "c++"] if compiler == "g++" else []
+    subprocess.run([compiler, std, "-pedantic", "-Wall", "-Wextra", "-Werror", "-I", str(ROOT / "include"),
+                    *lang, str(ROOT / "tests" / "c_abi_check.c"), "-x", "none", "-L", str(lib_dir), "-lnshb",
                     f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], check=True, capture_output=True, text=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
     got = dict(line.split(" ", 1) for line in out.strip().splitlines())
