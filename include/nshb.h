@@ -219,9 +219,9 @@ nshb_status adamh_step(const nshb_matrix *mats, int32_t n_mats, float *const *V,
  * it can be processed in pieces).  nshb_step_chunked runs the step of kind `op` (NSHB_OP_MUON,
  * _HYPERBALL, _RADIAL_BRAKE, _HIMUON or _RELATIVE_UPDATE) over mats[0..n_mats) in consecutive
  * chunks, each as long as fits in ws_bytes, one after the other on `stream`; p->rho (when set)
- * is indexed like mats.  Every matrix's result is the one the unchunked call computes.  The
- * step's device status word is that of the last chunk: read it per chunk, or use one chunk,
- * when the flags matter.  *n_chunks (optional) receives the number of chunks.
+ * is indexed like mats.  Every matrix's result is the one the unchunked call computes, and
+ * the device status word holds the flags of every chunk (the call clears it once, before
+ * the first).  *n_chunks (optional) receives the number of chunks.
  * nshb_workspace_size_min gives the smallest workspace it accepts (the largest single-matrix
  * need); a smaller one returns NSHB_ERR_WORKSPACE before anything is queued. */
 nshb_status nshb_workspace_size_min(const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, int32_t op,

@@ -857,8 +857,10 @@ nshb_status check_ws(const Plan &pl, void *ws, size_t ws_bytes) {
   return NSHB_OK;
 }
 
+// keep_status: a later chunk of one chunked call, which adds its flags to the status word
+// the earlier chunks set (only the exact-pass counter starts again from zero).
 nshb_status do_step(const nshb_matrix *mats, int n_mats, const nshb_params *p, int op, void *ws, size_t ws_bytes,
-                    cudaStream_t st) {
+                    cudaStream_t st, bool keep_status = false) {
   Plan pl;
   nshb_status e = plan_step(mats, n_mats, p, op, pl);
   if (e != NSHB_OK) return e;
@@ -866,7 +868,10 @@ nshb_status do_step(const nshb_matrix *mats, int n_mats, const nshb_params *p, i
   e = check_ws(pl, ws, ws_bytes);
   if (e != NSHB_OK) return e;
   char *w = static_cast<char *>(ws);
-  NSHB_CHECK_CUDA(cudaMemsetAsync(w, 0, 2 * sizeof(uint32_t), st));  // status word, exact-pass counter
+  if (keep_status)
+    NSHB_CHECK_CUDA(cudaMemsetAsync(w + sizeof(uint32_t), 0, sizeof(uint32_t), st));  // exact-pass counter
+  else
+    NSHB_CHECK_CUDA(cudaMemsetAsync(w, 0, 2 * sizeof(uint32_t), st));  // status word, exact-pass counter
   e = run_momentum(mats, pl, p, w, st);
   if (e != NSHB_OK) return e;
   std::vector<int64_t> o_off;
@@ -1153,7 +1158,7 @@ nshb_status nshb_step_chunked(int32_t op, const nshb_matrix *mats, int32_t n_mat
     const int i = starts[c], k = starts[c + 1] - starts[c];
     nshb_params pc = *p;
     if (p->rho) pc.rho = p->rho + i;           // the radii of this chunk's matrices
-    e = do_step(mats + i, k, &pc, op, ws, ws_bytes, (cudaStream_t)stream);
+    e = do_step(mats + i, k, &pc, op, ws, ws_bytes, (cudaStream_t)stream, /*keep_status=*/c > 0);
     if (e != NSHB_OK) return e;
   }
   return NSHB_OK;
