@@ -56,7 +56,7 @@ typedef enum { NSHB_BF16 = 0, NSHB_F32 = 1 } nshb_dtype;
 typedef enum {
   NSHB_OK = 0,
   NSHB_ERR_NULL = 1,           /* a required pointer is NULL                                 */
-  NSHB_ERR_SHAPE = 2,          /* rows/cols <= 0, ld < cols, misaligned O_out                */
+  NSHB_ERR_SHAPE = 2,          /* rows/cols <= 0, ld < cols, a pointer not element-aligned  */
   NSHB_ERR_DTYPE = 3,          /* unknown dtype or unsupported dtype combination              */
   NSHB_ERR_PARAM = 4,          /* a scalar parameter out of range                             */
   NSHB_ERR_WORKSPACE = 5,      /* workspace smaller than nshb_workspace_size or misaligned    */
@@ -88,7 +88,8 @@ typedef enum {
  * momentum buffer (zero before the first step; the only state a step keeps).
  * W and G share w_dtype.  Rows are read and written with 16-byte vector accesses when
  * W, G and M are 16-byte aligned and ld * sizeof(element) and ld * 4 are multiples of 16;
- * other layouts take a slower element-wise path.  O_out needs element alignment.
+ * other layouts take a slower element-wise path.  W, G and O_out must be aligned to their
+ * element size and M (and AdamH's V) to 4 bytes, else NSHB_ERR_SHAPE.
  * O_out (optional, may be NULL) receives the orthogonalised update O = NS_K(U)
  * (before any step-length or shape scaling), dtype w_dtype, leading dimension cols.
  * z_index picks the layer input Z of newton_muon_step (ignored elsewhere).

@@ -120,6 +120,7 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
     const bool vec = ((uintptr_t)d.W % 16 == 0) && ((uintptr_t)d.G % 16 == 0) && ((uintptr_t)d.M % 16 == 0) &&
                      ((d.ld * esz) % 16 == 0) && ((d.ld * 4) % 16 == 0);
     if (d.O_out && ((uintptr_t)d.O_out % esz) != 0) return NSHB_ERR_SHAPE;
+    if ((uintptr_t)d.W % esz || (uintptr_t)d.G % esz || (uintptr_t)d.M % 4) return NSHB_ERR_SHAPE;
     m.f32 = pl.f32ns || (!pl.tiled && std::min(d.rows, d.cols) < kSmallNsF32);
     m.flags = (vec ? kVec : 0) | (wf32 ? kWF32 : 0) | (m.f32 ? kNsF32 : 0);
     if (pl.tiled) {
@@ -914,6 +915,8 @@ nshb_status plan_adamh(const nshb_matrix *mats, int n_mats, float *const *V, con
     const bool vec = ((uintptr_t)d.W % 16 == 0) && ((uintptr_t)d.G % 16 == 0) && ((uintptr_t)d.M % 16 == 0) &&
                      ((uintptr_t)V[i] % 16 == 0) && ((d.ld * esz) % 16 == 0) && ((d.ld * 4) % 16 == 0);
     if (d.O_out && ((uintptr_t)d.O_out % esz) != 0) return NSHB_ERR_SHAPE;
+    if ((uintptr_t)d.W % esz || (uintptr_t)d.G % esz || (uintptr_t)d.M % 4 || (uintptr_t)V[i] % 4)
+      return NSHB_ERR_SHAPE;
     m.m = d.rows;
     m.n = d.cols;
     m.ld = d.ld;

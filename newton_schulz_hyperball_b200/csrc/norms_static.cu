@@ -81,6 +81,7 @@ extern "C" nshb_status nshb_fro_norms_static(const nshb_matrix *mats, int32_t n_
     if (d.w_dtype != NSHB_BF16 && d.w_dtype != NSHB_F32) return NSHB_ERR_DTYPE;
     const bool wf32 = d.w_dtype == NSHB_F32;
     const size_t esz = wf32 ? 4 : 2;
+    if ((uintptr_t)d.W % esz) return NSHB_ERR_SHAPE;
     const bool vec = ((uintptr_t)d.W % 16 == 0) && ((d.ld * esz) % 16 == 0);
     MatDesc &md = ap.mats[i];
     md.W = d.W;

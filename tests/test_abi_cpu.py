@@ -319,3 +319,26 @@ def test_pointer_arguments_are_checked_before_the_library_sees_them():
         nshb.fro_norms_static(mats, torch.zeros(3), stream=0)
     with pytest.raises(ValueError):
         nshb.device_status(torch.zeros(256, dtype=torch.uint8))      # workspace on the host
+
+
+@pytest.mark.parametrize("field,offset", [("W", 1), ("G", 1), ("M", 2)])
+def test_pointers_not_element_aligned_are_refused(field, offset):
+    """A misaligned element pointer would fault on the device: every entry point that plans a
+    step refuses it with NSHB_ERR_SHAPE before anything is queued."""
+    m = fake_mats([(64, 64)])
+    setattr(m[0], field, getattr(m[0], field) + offset)
+    for op in (nshb.NSHB_OP_MUON, nshb.NSHB_OP_HYPERBALL, nshb.NSHB_OP_HIMUON, nshb.NSHB_OP_ADAMH):
+        with pytest.raises(nshb.NshbError) as e:
+            ws_size(m, nshb.params(), op)
+        assert e.value.status == nshb.NSHB_ERR_SHAPE, op
+    if field == "W":
+        assert nshb.lib().nshb_fro_norms_static(m, 1, 0x1000, None) == nshb.NSHB_ERR_SHAPE
+
+
+def test_adam_second_moment_not_float_aligned_is_refused():
+    m = fake_mats([(64, 64)])
+    p = nshb.params()
+    n = nshb.workspace_size(m, p, nshb.NSHB_OP_ADAMH)
+    with pytest.raises(nshb.NshbError) as e:
+        nshb.adamh_step(m, [0x30000002], nshb.adam_params(), p, (0x40000000, n), stream=0)
+    assert e.value.status == nshb.NSHB_ERR_SHAPE
