@@ -121,7 +121,8 @@ typedef struct {
   float weight_decay;    /* muon_step decoupled weight decay                                  */
   float eta;             /* Hyperball step length (absolute Frobenius length), >= 0           */
   const float *rho;      /* DEVICE array [n_mats] of radii; entry <= 0, or rho == NULL, means */
-                         /* "use the current ||W||_F" (radius=None in the hook)               */
+                         /* "use the current ||W||_F" (radius=None in the hook); 4-byte       */
+                         /* aligned, else NSHB_ERR_PARAM                                      */
   float hb_eps;          /* numerical-zero threshold for norms, > 0                           */
   float brake_out;       /* RadialBrake outward factor in [0, 1]                              */
   float brake_in;        /* RadialBrake inward factor in [0, 1]                               */

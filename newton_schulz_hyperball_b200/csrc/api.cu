@@ -91,6 +91,7 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
   if (p->coeffs)
     for (int i = 0; i < 3 * p->ns_steps; ++i)
       if (!std::isfinite(p->coeffs[i])) return NSHB_ERR_PARAM;
+  if ((uintptr_t)p->rho % sizeof(float)) return NSHB_ERR_PARAM;
   pl.op = op;
   pl.f32ns = p->ns_precision == NSHB_F32;
   pl.tiled = op == NSHB_OP_HIMUON;
@@ -897,6 +898,7 @@ nshb_status plan_adamh(const nshb_matrix *mats, int n_mats, float *const *V, con
   if (!(a->eps > 0.f) || !std::isfinite(a->eps) || a->step < 1) return NSHB_ERR_PARAM;
   if (!(p->hb_eps > 0.f) || !std::isfinite(p->hb_eps) || !std::isfinite(p->eta) || p->eta < 0.f)
     return NSHB_ERR_PARAM;
+  if ((uintptr_t)p->rho % sizeof(float)) return NSHB_ERR_PARAM;
   pl.op = NSHB_OP_ADAMH;
   pl.mp.resize(n_mats);
   size_t off = kAlign;  // [0, 256): device status word

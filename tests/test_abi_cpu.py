@@ -342,3 +342,11 @@ def test_adam_second_moment_not_float_aligned_is_refused():
     with pytest.raises(nshb.NshbError) as e:
         nshb.adamh_step(m, [0x30000002], nshb.adam_params(), p, (0x40000000, n), stream=0)
     assert e.value.status == nshb.NSHB_ERR_SHAPE
+
+
+def test_misaligned_rho_is_refused():
+    m = fake_mats([(64, 64)])
+    for op in (nshb.NSHB_OP_HYPERBALL, nshb.NSHB_OP_ADAMH):
+        with pytest.raises(nshb.NshbError) as e:
+            ws_size(m, nshb.params(rho=0x30000002), op)
+        assert e.value.status == nshb.NSHB_ERR_PARAM, op
