@@ -231,7 +231,8 @@ nshb_status nshb_workspace_size_min(const nshb_matrix *mats, int32_t n_mats, con
 nshb_status nshb_step_chunked(int32_t op, const nshb_matrix *mats, int32_t n_mats, const nshb_params *p, void *ws,
                               size_t ws_bytes, nshb_stream stream, int32_t *n_chunks);
 
-/* out[i] = ||W_i||_F (fp32) into the DEVICE array out (n_mats floats), e.g. rho = ||W0||.
+/* out[i] = ||W_i||_F (fp32) into the DEVICE array out (n_mats floats, 4-byte aligned, else
+ * NSHB_ERR_SHAPE), e.g. rho = ||W0||.
  * Needs a workspace of nshb_workspace_size(..., NSHB_OP_MUON, ...) bytes. */
 nshb_status nshb_fro_norms(const nshb_matrix *mats, int32_t n_mats, float *out, void *ws,
                            size_t ws_bytes, nshb_stream stream);

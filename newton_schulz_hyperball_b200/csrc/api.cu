@@ -1172,6 +1172,7 @@ nshb_status nshb_step_chunked(int32_t op, const nshb_matrix *mats, int32_t n_mat
 nshb_status nshb_fro_norms(const nshb_matrix *mats, int32_t n_mats, float *out, void *ws, size_t ws_bytes,
                            nshb_stream stream) {
   if (!out && n_mats > 0) return NSHB_ERR_NULL;
+  if ((uintptr_t)out % sizeof(float)) return NSHB_ERR_SHAPE;
   nshb_params p;
   nshb_default_params(&p);
   Plan pl;

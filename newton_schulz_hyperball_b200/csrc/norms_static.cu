@@ -67,6 +67,7 @@ extern "C" nshb_status nshb_fro_norms_static(const nshb_matrix *mats, int32_t n_
   if (n_mats < 0) return NSHB_ERR_SHAPE;
   if (n_mats == 0) return NSHB_OK;
   if (!mats || !out) return NSHB_ERR_NULL;
+  if ((uintptr_t)out % sizeof(float)) return NSHB_ERR_SHAPE;
   if (n_mats > kMaxMats) return NSHB_ERR_WORKSPACE;
   ApplyParams ap;
   ApplyFinParams fp;

@@ -350,3 +350,10 @@ def test_misaligned_rho_is_refused():
         with pytest.raises(nshb.NshbError) as e:
             ws_size(m, nshb.params(rho=0x30000002), op)
         assert e.value.status == nshb.NSHB_ERR_PARAM, op
+
+
+def test_misaligned_norm_output_is_refused():
+    lib = nshb.lib()
+    m = fake_mats([(64, 64)])
+    assert lib.nshb_fro_norms(m, 1, 0x30000002, 0x40000000, 1 << 20, None) == nshb.NSHB_ERR_SHAPE
+    assert lib.nshb_fro_norms_static(m, 1, 0x30000002, None) == nshb.NSHB_ERR_SHAPE
