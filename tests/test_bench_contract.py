@@ -5,8 +5,6 @@ for real on one bounded step."""
 import json
 import sys
 
-import pytest
-
 import bench
 from newton_schulz_hyperball_b200 import workloads as wl
 

@@ -5,7 +5,6 @@ scratch is a fixed array inside the library.  The GPU test checks it against the
 workspace-based nshb_fro_norms on two calls in a row (the shared scratch keeps the previous
 call's contents, which must not leak into the next result).  This file is collected last.
 """
-import ctypes
 
 import numpy as np
 import pytest
