@@ -357,3 +357,36 @@ def test_misaligned_norm_output_is_refused():
     m = fake_mats([(64, 64)])
     assert lib.nshb_fro_norms(m, 1, 0x30000002, 0x40000000, 1 << 20, None) == nshb.NSHB_ERR_SHAPE
     assert lib.nshb_fro_norms_static(m, 1, 0x30000002, None) == nshb.NSHB_ERR_SHAPE
+
+
+def _no_cuda_device():
+    import torch
+    return not torch.cuda.is_available()
+
+
+@pytest.mark.skipif(not _no_cuda_device(), reason="passes fake device pointers: only where no GPU exists")
+def test_chunk_partition_is_the_greedy_longest_prefix():
+    """nshb_step_chunked fixes its chunk boundaries on the host before its first CUDA call, so
+    on a machine without a GPU the partition is reported and the call then stops with
+    NSHB_ERR_CUDA.  Each chunk must be the longest run of matrices, from where the last one
+    ended, whose workspace fits (brute force over the sizes nshb_workspace_size reports)."""
+    shapes = [(768, 768), (3072, 768), (768, 3072), (256, 512), (768, 768), (1024, 256), (64, 64)]
+    mats = fake_mats(shapes)
+    p = nshb.params()
+
+    def need(i, k):
+        return nshb.workspace_size(fake_mats(shapes[i:i + k]), p, nshb.NSHB_OP_HYPERBALL)
+
+    least = nshb.workspace_size_min(mats, p, nshb.NSHB_OP_HYPERBALL)
+    full = nshb.workspace_size(mats, p, nshb.NSHB_OP_HYPERBALL)
+    for ws_bytes in sorted({least, (least + full) // 2 // 256 * 256, full - 256, full}):
+        expect, i = 0, 0
+        while i < len(shapes):
+            k = max(k for k in range(1, len(shapes) - i + 1) if need(i, k) <= ws_bytes)
+            expect, i = expect + 1, i + k
+        n = ctypes.c_int32(-1)
+        st = nshb.lib().nshb_step_chunked(nshb.NSHB_OP_HYPERBALL, mats, len(shapes), ctypes.byref(p), 0x40000000,
+                                          ws_bytes, None, ctypes.byref(n))
+        assert st == nshb.NSHB_ERR_CUDA
+        assert n.value == expect, (ws_bytes, n.value, expect)
+    assert expect == 1   # the whole set fits in `full`
