@@ -70,6 +70,19 @@ struct Plan {
   int nseg = 0, k1_total = 0, w_total = 0;
 };
 
+// Checks of one matrix that every planner makes, in this order: sizes, limits, pointers,
+// dtype, element alignment (W, G, O_out to their element; M and, when given, V to 4 bytes).
+nshb_status check_matrix(const nshb_matrix &d, const float *V = nullptr, bool need_v = false) {
+  if (d.rows <= 0 || d.cols <= 0 || d.ld < d.cols) return NSHB_ERR_SHAPE;
+  if (d.rows > (1LL << 20) || d.cols > (1LL << 20) || d.ld > (1LL << 30)) return NSHB_ERR_UNSUPPORTED;
+  if (!d.W || !d.G || !d.M || (need_v && !V)) return NSHB_ERR_NULL;
+  if (d.w_dtype != NSHB_BF16 && d.w_dtype != NSHB_F32) return NSHB_ERR_DTYPE;
+  const size_t esz = d.w_dtype == NSHB_F32 ? 4 : 2;
+  if (d.O_out && ((uintptr_t)d.O_out % esz) != 0) return NSHB_ERR_SHAPE;
+  if ((uintptr_t)d.W % esz || (uintptr_t)d.G % esz || (uintptr_t)d.M % 4 || (uintptr_t)V % 4) return NSHB_ERR_SHAPE;
+  return NSHB_OK;
+}
+
 nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p, int op, Plan &pl) {
   if (!p) return NSHB_ERR_NULL;
   if (n_mats < 0) return NSHB_ERR_SHAPE;
@@ -109,10 +122,8 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
   for (int i = 0; i < n_mats; ++i) {
     const nshb_matrix &d = mats[i];
     MatPlan &m = pl.mp[i];
-    if (d.rows <= 0 || d.cols <= 0 || d.ld < d.cols) return NSHB_ERR_SHAPE;
-    if (d.rows > (1LL << 20) || d.cols > (1LL << 20) || d.ld > (1LL << 30)) return NSHB_ERR_UNSUPPORTED;
-    if (!d.W || !d.G || !d.M) return NSHB_ERR_NULL;
-    if (d.w_dtype != NSHB_BF16 && d.w_dtype != NSHB_F32) return NSHB_ERR_DTYPE;
+    const nshb_status ce = check_matrix(d);
+    if (ce != NSHB_OK) return ce;
     m.m = d.rows;
     m.n = d.cols;
     m.ld = d.ld;
@@ -120,8 +131,6 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
     const size_t esz = wf32 ? 4 : 2;
     const bool vec = ((uintptr_t)d.W % 16 == 0) && ((uintptr_t)d.G % 16 == 0) && ((uintptr_t)d.M % 16 == 0) &&
                      ((d.ld * esz) % 16 == 0) && ((d.ld * 4) % 16 == 0);
-    if (d.O_out && ((uintptr_t)d.O_out % esz) != 0) return NSHB_ERR_SHAPE;
-    if ((uintptr_t)d.W % esz || (uintptr_t)d.G % esz || (uintptr_t)d.M % 4) return NSHB_ERR_SHAPE;
     m.f32 = pl.f32ns || (!pl.tiled && std::min(d.rows, d.cols) < kSmallNsF32);
     m.flags = (vec ? kVec : 0) | (wf32 ? kWF32 : 0) | (m.f32 ? kNsF32 : 0);
     if (pl.tiled) {
@@ -908,17 +917,12 @@ nshb_status plan_adamh(const nshb_matrix *mats, int n_mats, float *const *V, con
   for (int i = 0; i < n_mats; ++i) {
     const nshb_matrix &d = mats[i];
     MatPlan &m = pl.mp[i];
-    if (d.rows <= 0 || d.cols <= 0 || d.ld < d.cols) return NSHB_ERR_SHAPE;
-    if (d.rows > (1LL << 20) || d.cols > (1LL << 20) || d.ld > (1LL << 30)) return NSHB_ERR_UNSUPPORTED;
-    if (!d.W || !d.G || !d.M || !V[i]) return NSHB_ERR_NULL;
-    if (d.w_dtype != NSHB_BF16 && d.w_dtype != NSHB_F32) return NSHB_ERR_DTYPE;
+    const nshb_status ce = check_matrix(d, V[i], /*need_v=*/true);
+    if (ce != NSHB_OK) return ce;
     const bool wf32 = d.w_dtype == NSHB_F32;
     const size_t esz = wf32 ? 4 : 2;
     const bool vec = ((uintptr_t)d.W % 16 == 0) && ((uintptr_t)d.G % 16 == 0) && ((uintptr_t)d.M % 16 == 0) &&
                      ((uintptr_t)V[i] % 16 == 0) && ((d.ld * esz) % 16 == 0) && ((d.ld * 4) % 16 == 0);
-    if (d.O_out && ((uintptr_t)d.O_out % esz) != 0) return NSHB_ERR_SHAPE;
-    if ((uintptr_t)d.W % esz || (uintptr_t)d.G % esz || (uintptr_t)d.M % 4 || (uintptr_t)V[i] % 4)
-      return NSHB_ERR_SHAPE;
     m.m = d.rows;
     m.n = d.cols;
     m.ld = d.ld;
