@@ -1260,6 +1260,6 @@ nshb_status nshb_profile_read(int32_t n_kinds, float *ms, int32_t *launches) {
 
 int32_t nshb_last_cuda_error(void) { return g_last_cuda_error; }
 
-int32_t nshb_version(void) { return 100; }
+int32_t nshb_version(void) { return 200; }   // 0.2.0: AdamH, RelativeUpdate, chunked steps, alignment checks
 
 }  // extern "C"
