@@ -89,27 +89,30 @@ def momentum(M, G, beta: float, nesterov: bool = True):
 
 
 # --------------------------------------------------------------------------
-# Newton-Schulz (Muon explainer, Newton-Schulz section and newton_schulz5).
+# Newton-Schulz (Muon explainer, Newton-Schulz section: the odd quintic
+# phi(x) = a x + b x^3 + c x^5 applied to the matrix, i.e. to every singular value).
 # --------------------------------------------------------------------------
-def newton_schulz(G, steps: int = 5, eps: float = NS_EPS, coeffs=None):
-    """Approximate msgn(G) = U V^T by the odd-polynomial iteration.
+def quintic(X, a: float, b: float, c: float):
+    """The odd matrix polynomial phi(X) = a X + b (X X^T) X + c (X X^T)^2 X.
 
-    1. work on the wide side: if rows > cols, X = G^T;
-    2. X <- X / (||X||_F + eps);
-    3. repeat: A = X X^T; B = b A + c A A; X <- a X + B X;
-    4. transpose back if step 1 transposed.
-    """
-    X = _f64(G)
-    tall = X.shape[0] > X.shape[1]
-    if tall:
-        X = X.T
-    X = X / (fro(X) + eps)
+    Since (X X^T)^k X = X (X^T X)^k, phi(X) = q(X X^T) X = X q(X^T X) with the
+    polynomial q(S) = a I + b S + c S^2 of a Gram matrix.  The Gram matrix of the
+    shorter side is the smaller one: the left Gram X X^T when X has no more rows
+    than columns, the right Gram X^T X otherwise."""
+    if X.shape[0] <= X.shape[1]:
+        S = X @ X.T
+        return (a * np.eye(S.shape[0]) + b * S + c * (S @ S)) @ X
+    S = X.T @ X
+    return X @ (a * np.eye(S.shape[0]) + b * S + c * (S @ S))
+
+
+def newton_schulz(G, steps: int = 5, eps: float = NS_EPS, coeffs=None):
+    """Approximate msgn(G) = U V^T: scale G to (at most) unit Frobenius norm,
+    X_0 = G / (||G||_F + eps), then apply the quintic ``steps`` times,
+    X_{k+1} = phi_k(X_k) with the k-th (a, b, c) of the coefficient table."""
+    X = _f64(G) / (fro(G) + eps)
     for a, b, c in coeff_table(steps, coeffs):
-        A = X @ X.T
-        B = b * A + c * (A @ A)
-        X = a * X + B @ X
-    if tall:
-        X = X.T
+        X = quintic(X, a, b, c)
     return np.ascontiguousarray(X)
 
 
