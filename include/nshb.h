@@ -178,7 +178,7 @@ nshb_status himuon_step(const nshb_matrix *mats, int32_t n_mats, const nshb_para
  * n_tokens, 16-byte aligned); n_tokens (up to 2^24) and every z_rows[j] (up to 16384) must be
  * multiples of 64, else NSHB_ERR_SHAPE; matrix i uses Z[mats[i].z_index] (an index outside
  * [0, n_z) is NSHB_ERR_PARAM), which needs z_rows == cols (else NSHB_ERR_SHAPE).  Z and z_rows
- * are HOST arrays of n_z entries (1 <= n_z <= 192).  A pivot that is not positive in fp32 sets
+ * are HOST arrays of n_z entries (1 <= n_z <= 224).  A pivot that is not positive in fp32 sets
  * NSHB_DEV_NOT_SPD.  bf16 NS only. */
 nshb_status newton_muon_step(const nshb_matrix *mats, int32_t n_mats, const void *const *Z,
                              const int64_t *z_rows, int32_t n_z, int64_t n_tokens,
@@ -246,7 +246,11 @@ nshb_status nshb_fro_norms(const nshb_matrix *mats, int32_t n_mats, float *out, 
  * call on a device looks up that array's address (make it before any stream capture).
  * Limits: n_mats <= 192 and sum over matrices of ceil(rows/64) * ceil(cols/64) <= 174,240
  * (about 7.1e8 elements); larger requests return NSHB_ERR_WORKSPACE before any work is
- * queued.  Calls share the array, so calls that overlap on the GPU race. */
+ * queued.  Calls share the array, so calls that overlap on the GPU race.  The array's
+ * address is looked up once per device and kept, so resetting a device (cudaDeviceReset)
+ * after the first call on it is not supported.  There is no status word to read: a
+ * non-finite norm shows only as NaN or Inf in out.  A failed launch returns NSHB_ERR_CUDA
+ * and records the CUDA error for nshb_last_cuda_error. */
 #define NSHB_STATIC_SCRATCH_BYTES (4u << 20)
 nshb_status nshb_fro_norms_static(const nshb_matrix *mats, int32_t n_mats, float *out, nshb_stream stream);
 

@@ -13,7 +13,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libnshb.so")
-SOURCES = ["api.cu", "stream_kernels.cu", "ns_f32.cu", "ns_tc.cu", "ns_tc2.cu", "himuon_tile.cu", "newton.cu",
+SOURCES = ["api.cu", "stream_kernels.cu", "ns_f32.cu", "ns_tc2.cu", "himuon_tile.cu", "newton.cu",
            "norms_static.cu"]
 HEADERS = ["nshb_internal.h", "nshb_device.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

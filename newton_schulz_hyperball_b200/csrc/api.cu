@@ -17,6 +17,9 @@
 #include "nshb_internal.h"
 
 namespace nshb {
+
+thread_local int g_last_cuda_error = 0;   // last CUDA error seen by this thread's calls
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -46,6 +49,10 @@ struct MatPlan {
   int pr = 0, pc = 0;            // momentum block domain (W coordinates)
   int k1_blocks = 0, k1_begin = 0;
   int w_blocks = 0, w_begin = 0;
+  // (||O||^2, <W,O>, ||W||^2) records: from the last NS update's epilogue (fused: one per
+  // epilogue warp and output tile) or from the reduce pass (one per 64 x 64 block of W)
+  bool fused = false;
+  int rec_begin = 0, rec_count = 0;
 };
 
 struct Plan {
@@ -54,7 +61,6 @@ struct Plan {
   bool tiled = false;
   int bn = 256;
   int comp = 0;                  // compensated (hi/lo) iterations of the bf16 chain
-  bool pair = true;              // bf16 GEMMs on CTA pairs (256-row tiles); single CTAs for T = 128
   std::vector<MatPlan> mp;
   // Newton-Muon: per layer input Z
   struct ZPlan {
@@ -66,21 +72,14 @@ struct Plan {
   int64_t n_tokens = 0;
   std::vector<int64_t> r_off;         // per matrix: fp32 m x n buffer for U -> Y -> P
   std::vector<int> zidx;
-  size_t scal_off = 0, scale_off = 0, nu_off = 0, k1part_off = 0, wpart_off = 0, total = 0;
-  int nseg = 0, k1_total = 0, w_total = 0;
+  size_t scal_off = 0, scale_off = 0, nu_off = 0, k1part_off = 0, wpart_off = 0, xpart_off = 0, total = 0;
+  int nseg = 0, k1_total = 0, w_total = 0, rec_total = 0;
 };
 
-// Checks of one matrix that every planner makes, in this order: sizes, limits, pointers,
-// dtype, element alignment (W, G, O_out to their element; M and, when given, V to 4 bytes).
-nshb_status check_matrix(const nshb_matrix &d, const float *V = nullptr, bool need_v = false) {
-  if (d.rows <= 0 || d.cols <= 0 || d.ld < d.cols) return NSHB_ERR_SHAPE;
-  if (d.rows > (1LL << 20) || d.cols > (1LL << 20) || d.ld > (1LL << 30)) return NSHB_ERR_UNSUPPORTED;
-  if (!d.W || !d.G || !d.M || (need_v && !V)) return NSHB_ERR_NULL;
-  if (d.w_dtype != NSHB_BF16 && d.w_dtype != NSHB_F32) return NSHB_ERR_DTYPE;
-  const size_t esz = d.w_dtype == NSHB_F32 ? 4 : 2;
-  if (d.O_out && ((uintptr_t)d.O_out % esz) != 0) return NSHB_ERR_SHAPE;
-  if ((uintptr_t)d.W % esz || (uintptr_t)d.G % esz || (uintptr_t)d.M % 4 || (uintptr_t)V % 4) return NSHB_ERR_SHAPE;
-  return NSHB_OK;
+// Steps whose update rule needs (||O||^2, <W,O>, ||W||^2).
+bool needs_partials(int op) {
+  return op == NSHB_OP_HYPERBALL || op == NSHB_OP_RADIAL_BRAKE || op == NSHB_OP_RELATIVE_UPDATE ||
+         op == NSHB_OP_HIMUON || op == NSHB_OP_NEWTON_MUON;
 }
 
 nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p, int op, Plan &pl) {
@@ -113,7 +112,6 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
     if (pl.f32ns) return NSHB_ERR_UNSUPPORTED;
     if (p->tile != 128 && p->tile != 256 && p->tile != 512) return NSHB_ERR_PARAM;
     pl.bn = p->tile == 128 ? 128 : 256;
-    pl.pair = p->tile != 128;
   }
   if (op == NSHB_OP_NEWTON_MUON) {
     if (!(p->ridge_rel >= 0.f) || !std::isfinite(p->ridge_rel)) return NSHB_ERR_PARAM;
@@ -160,6 +158,21 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
     }
     m.k1_blocks = (m.pr / kBlk) * (m.pc / kBlk);
     m.w_blocks = (int)(((m.m + kBlk - 1) / kBlk) * ((m.n + kBlk - 1) / kBlk));
+    // The partials come from the epilogue that writes the final O wherever the NS runs on
+    // the tensor cores: the pair GEMM's last update (one record per epilogue warp and 256 x
+    // 256 output tile) or the tile-resident Hierarchical-Muon kernels (one per epilogue warp
+    // and tile: 16 for T = 256, 4 for T = 128).  The fp32 chain and fp32 weights leave them
+    // to the reduce pass.
+    m.fused = needs_partials(op) && !m.f32 && !wf32;
+    if (m.fused) {
+      int64_t recs;
+      if (!pl.tiled) recs = (m.Rp / 256) * (m.Sp / 256) * kPartsPerTile;
+      else if (m.T == 512) recs = (int64_t)m.ntiles * 4 * kPartsPerTile;
+      else recs = (int64_t)m.ntiles * (m.T == 256 ? kPartsPerTile : 4);
+      m.rec_count = (int)recs;
+    } else {
+      m.rec_count = m.w_blocks;
+    }
   }
   // Workspace layout.
   size_t off = kAlign;  // [0, 256): device status word
@@ -168,6 +181,7 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
   pl.nseg = 0;
   pl.k1_total = 0;
   pl.w_total = 0;
+  pl.rec_total = 0;
   for (auto &m : pl.mp) {
     m.seg_begin = pl.nseg;
     pl.nseg += m.nseg;
@@ -175,6 +189,8 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
     pl.k1_total += m.k1_blocks;
     m.w_begin = pl.w_total;
     pl.w_total += m.w_blocks;
+    m.rec_begin = pl.rec_total;
+    pl.rec_total += m.rec_count;
   }
   pl.scale_off = off;
   off = align_up(off + sizeof(float) * (size_t)pl.nseg);
@@ -183,7 +199,9 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
   pl.k1part_off = off;
   off = align_up(off + sizeof(double) * (size_t)pl.k1_total);
   pl.wpart_off = off;
-  off = align_up(off + 3 * sizeof(double) * (size_t)pl.w_total);
+  off = align_up(off + 3 * sizeof(double) * (size_t)pl.rec_total);
+  pl.xpart_off = off;
+  off = align_up(off + sizeof(double) * (size_t)pl.w_total);
   for (auto &m : pl.mp) {
     size_t xb, ab;
     if (pl.tiled) {
@@ -274,6 +292,7 @@ MatDesc make_desc(const nshb_matrix &d, const MatPlan &m, int idx, int64_t o_off
   r.seg_begin = m.seg_begin;
   r.tiles_c = m.tiles_c;
   r.mat = idx;
+  r.rec_begin = m.rec_begin;
   return r;
 }
 
@@ -298,8 +317,6 @@ int device_sms() {
   }
   return v;
 }
-
-thread_local int g_last_cuda_error = 0;   // last CUDA error seen by this thread's calls
 
 #define NSHB_CHECK_CUDA(x)                 \
   do {                                     \
@@ -431,7 +448,8 @@ void coeffs_for(const nshb_params *p, int it, float &a, float &b, float &c) {
 }
 
 // Hierarchical Muon with T = 256 or 128: every tile's whole chain in a tile-resident kernel.
-nshb_status run_himuon_tile(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t st) {
+nshb_status run_himuon_tile(const nshb_matrix *mats, const Plan &pl, const nshb_params *p, char *ws,
+                            cudaStream_t st) {
   const int n = (int)pl.mp.size();
   for (int c0 = 0; c0 < n; c0 += kMaxProb) {
     const int c1 = std::min(n, c0 + kMaxProb);
@@ -443,6 +461,7 @@ nshb_status run_himuon_tile(const Plan &pl, const nshb_params *p, char *ws, cuda
     hp.wait_limit = (p->debug_flags & 1u) ? kWaitLimitTest : kWaitLimit;
     hp.ns_steps = p->ns_steps;
     hp.comp = pl.comp;
+    hp.test_stall = (p->debug_flags & 2u) ? 1 : 0;
     for (int it = 0; it < p->ns_steps; ++it) coeffs_for(p, it, hp.coef[it][0], hp.coef[it][1], hp.coef[it][2]);
     int tiles = 0;
     for (int i = c0; i < c1; ++i) {
@@ -455,6 +474,18 @@ nshb_status run_himuon_tile(const Plan &pl, const nshb_params *p, char *ws, cuda
       q.tile_begin = tiles;
       q.ntiles = m.ntiles;
       q.seg_begin = m.seg_begin;
+      q.w_tiles_c = m.tiles_c;
+      q.w = nullptr;
+      if (m.fused) {
+        const nshb_matrix &d = mats[i];
+        q.w = d.W;
+        q.w_m = (int)m.m;
+        q.w_n = (int)m.n;
+        q.w_ld = (int)m.ld;
+        q.w_flags = (uintptr_t)d.W % 16 == 0 && (d.ld * 2) % 16 == 0 ? kPwVec : 0;   // bf16 W
+        q.part_begin = m.rec_begin;
+        hp.partials = reinterpret_cast<double *>(ws + pl.wpart_off);
+      }
       tiles += m.ntiles;
     }
     hp.nprob = c1 - c0;
@@ -467,14 +498,15 @@ nshb_status run_himuon_tile(const Plan &pl, const nshb_params *p, char *ws, cuda
 }
 
 // K iterations of the three NS phases.  Returns the offset of each matrix's O in `o_off`.
-nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t st, std::vector<int64_t> &o_off) {
+nshb_status run_ns(const nshb_matrix *mats, const Plan &pl, const nshb_params *p, char *ws, cudaStream_t st,
+                   std::vector<int64_t> &o_off) {
   const int n = (int)pl.mp.size();
   o_off.resize(n);
   const float *scales = reinterpret_cast<const float *>(ws + pl.scale_off);
   uint32_t *status = reinterpret_cast<uint32_t *>(ws);
   const long long limit = (p->debug_flags & 1u) ? kWaitLimitTest : kWaitLimit;
-  if (pl.tiled && (p->tile == 256 || p->tile == 128) && !p->debug_flags) {
-    const nshb_status e = run_himuon_tile(pl, p, ws, st);
+  if (pl.tiled && (p->tile == 256 || p->tile == 128)) {
+    const nshb_status e = run_himuon_tile(mats, pl, p, ws, st);
     if (e != NSHB_OK) return e;
     for (int i = 0; i < n; ++i) o_off[i] = (p->ns_steps % 2 == 0) ? pl.mp[i].x0 : pl.mp[i].x1;
     return NSHB_OK;
@@ -537,6 +569,8 @@ nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t 
           gp.test_stall = (p->debug_flags & 2u) ? 1 : 0;
           gp.mode = mode;
           gp.ca = ca; gp.cb = cb; gp.cc = cc;
+          const bool last_update = mode == kUpdate && it + 1 == p->ns_steps;
+          gp.partials = nullptr;
           // Longest-k problems first, so the static tile walk ends evenly.
           std::vector<std::pair<int64_t, int>> ord;
           for (int ii = c0; ii < c1; ++ii) {
@@ -554,18 +588,29 @@ nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t 
             GemmProb &q = gp.prob[k++];
             int64_t R, S;
             int batch;
-            int64_t xbs, abs_;
             if (pl.tiled) {
               R = m.T; S = m.T; batch = m.ntiles;
-              xbs = (int64_t)m.T * m.T * 2;
-              abs_ = xbs;
             } else {
               R = m.Rp; S = m.Sp; batch = 1;
-              xbs = 0; abs_ = 0;
             }
             q.batch = batch;
-            q.a_ph = q.b_ph = q.d_ph = (int)R;
-            q.mt = (int)(R / (pl.pair ? 256 : 128));
+            q.ph = (int)R;
+            // X, A and B of a tile share one stride (T x T bf16); a whole matrix is one batch
+            q.bs = pl.tiled ? (int64_t)m.T * m.T * 2 : 0;
+            q.w = nullptr;
+            if (last_update && m.fused) {
+              const nshb_matrix &d = mats[i];
+              const bool wvec = (uintptr_t)d.W % 16 == 0 && (d.ld * 2) % 16 == 0;   // bf16 W
+              q.w = d.W;
+              q.w_m = (int)m.m;
+              q.w_n = (int)m.n;
+              q.w_ld = (int)m.ld;
+              q.w_flags = (m.tall ? kPwTall : 0) | (pl.tiled ? kPwTiled : 0) | (wvec ? kPwVec : 0);
+              q.w_tiles_c = m.tiles_c;
+              q.part_begin = m.rec_begin;
+              gp.partials = reinterpret_cast<double *>(ws + pl.wpart_off);
+            }
+            q.mt = (int)(R / 256);
             q.c_lo = -1;
             q.d_lo = -1;
             if (mode == kUpdate && it < pl.comp) {
@@ -574,30 +619,23 @@ nshb_status run_ns(const Plan &pl, const nshb_params *p, char *ws, cudaStream_t 
             }
             if (mode == kGram) {
               q.a_off = xin; q.b_off = xin; q.c_off = m.a; q.d_off = m.a;
-              q.a_bs = xbs; q.b_bs = xbs; q.c_bs = abs_; q.d_bs = abs_;
               q.nt = (int)(R / pl.bn); q.kt = (int)(S / 64);
             } else if (mode == kPoly) {
               q.a_off = m.a; q.b_off = m.a; q.c_off = m.a; q.d_off = m.b;
-              q.a_bs = abs_; q.b_bs = abs_; q.c_bs = abs_; q.d_bs = abs_;
               q.nt = (int)(R / pl.bn); q.kt = (int)(R / 64);
             } else {
               q.a_off = m.b; q.b_off = xin; q.c_off = xin; q.d_off = xout;
-              q.a_bs = abs_; q.b_bs = xbs; q.c_bs = xbs; q.d_bs = xbs;
               q.nt = (int)(S / pl.bn); q.kt = (int)(R / 64);
             }
-            q.tiles_per_batch = gemm_tiles(mode, q.mt, q.nt, pl.pair ? 256 : 128, pl.bn);
+            q.tiles_per_batch = gemm_tiles(mode, q.mt, q.nt, 256, pl.bn);
             q.scale_idx = (it == 0 && mode != kPoly) ? m.seg_begin : -1;
             q.tile_begin = tiles;
             tiles += q.tiles_per_batch * q.batch;
           }
           gp.nprob = k;
           gp.total_tiles = tiles;
-          if (pl.pair) {
-            NSHB_CHECK_CUDA(encode_ws_tensor_map(&gp.tmap, ws, pl.total / 128 * 128));
-            NSHB_LAUNCH(NSHB_PROF_GRAM + mode, launch_gemm_tc2(gp, device_sms(), st));
-          } else {
-            NSHB_LAUNCH(NSHB_PROF_GRAM + mode, launch_gemm_tc(gp, pl.bn, device_sms(), st));
-          }
+          NSHB_CHECK_CUDA(encode_ws_tensor_map(&gp.tmap, ws, pl.total / 128 * 128));
+          NSHB_LAUNCH(NSHB_PROF_GRAM + mode, launch_gemm_tc2(gp, device_sms(), st));
         }
       }
     }
@@ -612,6 +650,7 @@ nshb_status run_apply(const nshb_matrix *mats, const Plan &pl, const nshb_params
   const int n = (int)pl.mp.size();
   MatScalars *scal = reinterpret_cast<MatScalars *>(ws + pl.scal_off);
   double *wpart = reinterpret_cast<double *>(ws + pl.wpart_off);
+  double *xpart = reinterpret_cast<double *>(ws + pl.xpart_off);
   uint32_t *status = reinterpret_cast<uint32_t *>(ws);
   for (int c0 = 0; c0 < n; c0 += kMaxMats) {
     const int c1 = std::min(n, c0 + kMaxMats);
@@ -622,6 +661,10 @@ nshb_status run_apply(const nshb_matrix *mats, const Plan &pl, const nshb_params
     ap.status = status;
     ap.op = apply_op;
     ap.nmat = c1 - c0;
+    // The reduce pass covers only the matrices whose records the NS epilogue did not write.
+    ApplyParams rp = ap;
+    rp.nmat = 0;
+    rp.partials = wpart;
     ApplyFinParams fp;
     std::memset(&fp, 0, sizeof(fp));
     fp.scal = scal;
@@ -636,23 +679,31 @@ nshb_status run_apply(const nshb_matrix *mats, const Plan &pl, const nshb_params
     fp.brake_out = p->brake_out;
     fp.brake_in = p->brake_in;
     fp.nmat = c1 - c0;
-    int nb = 0;
+    int nb = 0, rb = 0;
     for (int i = c0; i < c1; ++i) {
       const MatPlan &m = pl.mp[i];
       ap.mats[i - c0] = make_desc(mats[i], m, i, o_off.empty() ? 0 : o_off[i], nb, false);
+      if (!m.fused) {
+        rp.mats[rp.nmat] = make_desc(mats[i], m, i, o_off.empty() ? 0 : o_off[i], rb, false);
+        rp.nmat++;
+        rb += m.w_blocks;
+      }
+      fp.rec_begin[i - c0] = m.rec_begin;
       fp.blk_begin[i - c0] = nb;
       fp.mat[i - c0] = i;
       fp.m[i - c0] = (int)m.m;
       fp.n[i - c0] = (int)m.n;
       nb += m.w_blocks;
     }
+    fp.rec_begin[c1 - c0] = pl.mp[c1 - 1].rec_begin + pl.mp[c1 - 1].rec_count;
     fp.blk_begin[c1 - c0] = nb;
     ap.total_blocks = nb;
-    // One region for the whole call: chunk c0 uses the partials of its own blocks.
-    ap.partials = wpart + 3 * (int64_t)pl.mp[c0].w_begin;
-    fp.partials = ap.partials;
-    if (apply_op != kOpMuon && !have_partials) {
-      NSHB_LAUNCH(NSHB_PROF_REDUCE, launch_reduce(ap, st));
+    rp.total_blocks = rb;
+    fp.partials = wpart;                                   // records: absolute indices
+    ap.partials = xpart + pl.mp[c0].w_begin;               // exact-norm sums: one per block
+    fp.xpartials = ap.partials;
+    if (apply_op != kOpMuon && !have_partials && rp.nmat > 0) {
+      NSHB_LAUNCH(NSHB_PROF_REDUCE, launch_reduce(rp, st));
     }
     fp.stage = 0;
     NSHB_LAUNCH(NSHB_PROF_FINALIZE, launch_apply_finalize(fp, st));
@@ -775,8 +826,9 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
       q.a_off = q.b_off = z.zp;
       q.c_off = q.d_off = z.s;
       q.c_lo = q.d_lo = -1;
-      q.a_ph = q.b_ph = (int)z.Dp;
-      q.d_ph = (int)z.Dp;
+      q.ph = (int)z.Dp;
+      q.bs = 0;
+      q.w = nullptr;
       q.mt = (int)(z.Dp / 256);
       q.nt = (int)(z.Dp / 256);
       q.kt = (int)(pl.n_tokens / 64);
@@ -886,7 +938,7 @@ nshb_status do_step(const nshb_matrix *mats, int n_mats, const nshb_params *p, i
   e = run_momentum(mats, pl, p, w, st);
   if (e != NSHB_OK) return e;
   std::vector<int64_t> o_off;
-  e = run_ns(pl, p, w, st, o_off);
+  e = run_ns(mats, pl, p, w, st, o_off);
   if (e != NSHB_OK) return e;
   const int aop = op == NSHB_OP_MUON              ? kOpMuon
                   : op == NSHB_OP_RADIAL_BRAKE    ? kOpBrake
@@ -932,9 +984,14 @@ nshb_status plan_adamh(const nshb_matrix *mats, int n_mats, float *const *V, con
     m.w_blocks = (int)(((m.m + kBlk - 1) / kBlk) * ((m.n + kBlk - 1) / kBlk));
     m.w_begin = pl.w_total;
     pl.w_total += m.w_blocks;
+    m.rec_begin = m.w_begin;      // adam_kernel writes one record per block
+    m.rec_count = m.w_blocks;
   }
+  pl.rec_total = pl.w_total;
   pl.wpart_off = off;
   off = align_up(off + 3 * sizeof(double) * (size_t)pl.w_total);
+  pl.xpart_off = off;
+  off = align_up(off + sizeof(double) * (size_t)pl.w_total);
   for (auto &m : pl.mp) {
     m.x0 = off;
     const size_t ub = (m.flags & kWF32) ? (size_t)m.m * m.n * 4 : (size_t)m.Rp * round_up(m.n, kBlk) * 2;
@@ -974,6 +1031,29 @@ nshb_status run_adam(const nshb_matrix *mats, const Plan &pl, float *const *V, c
 }
 
 }  // namespace
+}  // namespace nshb
+
+namespace nshb {
+
+nshb_status check_matrix(const nshb_matrix &d, const float *V, bool need_v, bool w_only) {
+  if (d.rows <= 0 || d.cols <= 0 || d.ld < d.cols) return NSHB_ERR_SHAPE;
+  if (d.rows > (1LL << 20) || d.cols > (1LL << 20) || d.ld > (1LL << 30)) return NSHB_ERR_UNSUPPORTED;
+  if (!d.W) return NSHB_ERR_NULL;
+  if (!w_only && (!d.G || !d.M || (need_v && !V))) return NSHB_ERR_NULL;
+  if (d.w_dtype != NSHB_BF16 && d.w_dtype != NSHB_F32) return NSHB_ERR_DTYPE;
+  const size_t esz = d.w_dtype == NSHB_F32 ? 4 : 2;
+  if ((uintptr_t)d.W % esz) return NSHB_ERR_SHAPE;
+  if (w_only) return NSHB_OK;
+  if (d.O_out && ((uintptr_t)d.O_out % esz) != 0) return NSHB_ERR_SHAPE;
+  if ((uintptr_t)d.G % esz || (uintptr_t)d.M % 4 || (uintptr_t)V % 4) return NSHB_ERR_SHAPE;
+  return NSHB_OK;
+}
+
+void record_cuda_error(cudaError_t e) {
+  g_last_cuda_error = (int)e;
+  (void)cudaGetLastError();
+}
+
 }  // namespace nshb
 
 using namespace nshb;
@@ -1100,7 +1180,7 @@ nshb_status newton_muon_step(const nshb_matrix *mats, int32_t n_mats, const void
   e = run_momentum(mats, pl, p, w, st, /*from_p=*/true);
   if (e != NSHB_OK) return e;
   std::vector<int64_t> o_off;
-  e = run_ns(pl, p, w, st, o_off);
+  e = run_ns(mats, pl, p, w, st, o_off);
   if (e != NSHB_OK) return e;
   return run_apply(mats, pl, p, kOpHyperball, w, st, o_off, nullptr);
 }

@@ -160,6 +160,66 @@ __device__ __forceinline__ uint32_t col_chunk(int g, int jj) {
   return (uint32_t)((jj >> 6) * kPanel256 + g * 128 + ((((jj >> 3) & 7) ^ (g & 7)) << 4));
 }
 
+// The caller's bf16 W at row wr, columns wc .. wc+31 as 16 pairs in logical order (zero
+// outside the matrix; fp32 weights take the reduce pass).  Loaded a chunk ahead of use.
+__device__ __forceinline__ void w_load(const HmProb &q, int64_t wr, int64_t wc, uint32_t (&wv)[16]) {
+  const bool rin = wr < q.w_m;
+  const unsigned short *row = static_cast<const unsigned short *>(q.w) + wr * q.w_ld;
+  if (rin && wc + 31 < q.w_n && (q.w_flags & kPwVec)) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(row + wc);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const uint4 u = src[g];
+      wv[4 * g] = u.x; wv[4 * g + 1] = u.y; wv[4 * g + 2] = u.z; wv[4 * g + 3] = u.w;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint32_t lo = (rin && wc + 2 * e < q.w_n) ? (uint32_t)row[wc + 2 * e] : 0u;
+      const uint32_t hi = (rin && wc + 2 * e + 1 < q.w_n) ? (uint32_t)row[wc + 2 * e + 1] : 0u;
+      wv[e] = lo | (hi << 16);
+    }
+  }
+}
+
+// Adds the (||O||^2, <W,O>, ||W||^2) terms of 32 elements of a tile row: O as stored (bf16
+// pairs hw) and W (pairs wv, both in logical order).  fp32 terms over the 32 elements,
+// added to the thread's fp64 sums.
+__device__ __forceinline__ void w_partials(const uint32_t (&wv)[16], const uint32_t (&hw)[16], double &dom,
+                                           double &dde, double &dpi) {
+  float om = 0.f, de = 0.f, pi = 0.f;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const float w0 = bf16lo(wv[e]), w1 = bf16hi(wv[e]);
+    const float o0 = bf16lo(hw[e]), o1 = bf16hi(hw[e]);
+    om = fmaf(o0, o0, fmaf(o1, o1, om));
+    de = fmaf(w0, o0, fmaf(w1, o1, de));
+    pi = fmaf(w0, w0, fmaf(w1, w1, pi));
+  }
+  dom += (double)om;
+  dde += (double)de;
+  dpi += (double)pi;
+}
+
+// Pulls the thread's W row segment (ncol elements from column wc) into L2 ahead of use.
+__device__ __forceinline__ void w_prefetch(const HmProb &q, int64_t wr, int64_t wc, int ncol) {
+  if (wr >= q.w_m || wc >= q.w_n) return;
+  const char *base = static_cast<const char *>(q.w) + (wr * q.w_ld + wc) * 2;
+  for (int b = 0; b < ncol * 2; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(base + b));
+}
+
+// One (||O||^2, <W,O>, ||W||^2) record per epilogue warp: the warp's fp64 sums in fixed order.
+__device__ __forceinline__ void w_record(double *partials, int64_t rec, double dom, double dde, double dpi) {
+  dom = warp_sum(dom);
+  dde = warp_sum(dde);
+  dpi = warp_sum(dpi);
+  if ((threadIdx.x & 31) == 0) {
+    partials[3 * rec] = dom;
+    partials[3 * rec + 1] = dde;
+    partials[3 * rec + 2] = dpi;
+  }
+}
+
 __device__ __forceinline__ int find_prob(const HmParams &p, int tile) {
   int lo = 0, hi = p.nprob - 1;
   while (lo < hi) {
@@ -178,6 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
   const uint32_t bar_base = smem_u32(bars);
   const uint32_t xfull = bar_base, xfree = bar_base + 8, mmadone = bar_base + 16;
   const uint32_t xready = bar_base + 24, opnd = bar_base + 32;   // used in the leader only
+  const uint32_t stallbar = bar_base + 40;                        // test stall (leader only)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cta_rank();
@@ -189,6 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
     mbar_init(mmadone, 1);
     mbar_init(xready, 2);                 // both producers
     mbar_init(opnd, 2 * kEpiWarps);       // every epilogue warp of both CTAs
+    mbar_init(stallbar, 1);
     mbar_fence_init();
   }
   if (warp == 1) {
@@ -248,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
         ph_o ^= 1u;
         tc_fence_after();
       };
-      for (int tile = cid; ok && tile < p.total_tiles; tile += ncl) {
+      for (int tile = cid, tl = 0; ok && tile < p.total_tiles; tile += ncl, ++tl) {
         if (!mbar_wait(xready, ph_r, limit)) {
           set_status(p.status, kTimeoutBit);
           break;
@@ -266,7 +328,15 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
             const uint64_t d = smem_desc_sw128(sXown + kofs, 16, 1024);
             tc_mma2(tmem_base, d, d, idesc_k, k != 0);
           }
-          tc_commit2_mc(mmadone, 0x3);
+          if (p.test_stall && tl == 0 && it == 0) {
+            // Test stall: the epilogues never hear of this accumulator, so their bounded
+            // wait runs out.  The MMAs still complete (on a barrier of the leader only)
+            // before this thread goes on, so none is in flight when the CTAs leave.
+            tc_commit2_mc(stallbar, 0x1);
+            if (!mbar_wait(stallbar, 0, limit)) set_status(p.status, kTimeoutBit);
+          } else {
+            tc_commit2_mc(mmadone, 0x3);
+          }
           wait_opnd();     // epilogue 1 wrote A to sA
           if (!ok) break;
 #pragma unroll
@@ -324,6 +394,11 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
       const int t = tile - q.tile_begin;
       const int64_t toff = (int64_t)t * T * T * 2;
       const float s = p.scales[q.seg_begin + t];
+      // Hyperball partials: this thread's W row and the first column of its half
+      const bool wp = p.partials != nullptr && q.w != nullptr;
+      const int64_t wr = (int64_t)(t / q.w_tiles_c) * T + g;
+      const int64_t wc = (int64_t)(t % q.w_tiles_c) * T + 128 * half;
+      double dom = 0.0, dde = 0.0, dpi = 0.0;
       if (!mbar_wait(xfull, ph_x, limit)) {            // sXown holds X0 (read by epilogue 3)
         if (lane == 0) set_status(p.status, kTimeoutBit);
         break;
@@ -332,6 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
       for (int it = 0; ok && it < K; ++it) {
         const float ca = p.coef[it][0], cb = p.coef[it][1], cc = p.coef[it][2];
         const float s2 = it == 0 ? s * s : 1.0f, ks = it == 0 ? s : 1.0f;
+        if (wp && it + 1 == K) w_prefetch(q, wr, wc, 128);
         // ---- epilogue 1: A -> sA (bf16)
         wait_mma();
         if (!ok) break;
@@ -375,15 +451,20 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
         }
         report(false);
         // ---- epilogue 3: X' = s (a X + B X)
+        const bool last = it + 1 == K;
+        const bool wlast = wp && last;
+        uint32_t wv[16];
+        if (wlast) w_load(q, wr, wc, wv);       // in flight while the update MMAs run
         wait_mma();
         if (!ok) break;
-        const bool last = it + 1 == K;
         const char *clo = it < p.comp ? p.ws + ((it % 2 == 0) ? q.xl0 : q.xl1) + toff : nullptr;
         char *dlo = (it + 1 < p.comp) ? p.ws + ((it % 2 == 0) ? q.xl1 : q.xl0) + toff : nullptr;
         char *dout = last ? p.ws + q.xo + toff : nullptr;
 #pragma unroll 1
         for (int ch = 0; ch < 4; ++ch) {
           const int j0 = 128 * half + 32 * ch;
+          uint32_t wn[16];
+          if (wlast && ch < 3) w_load(q, wr, wc + 32 * (ch + 1), wn);
           uint32_t r[32];
           tmem_ld32(tmem_base + (uint32_t)j0 + lane_off, r);
           uint32_t xw[16], lw[16];
@@ -419,6 +500,11 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
               unswizzle_pair(in8, odd, w8);
               st_global_256(dout + panel_pair_off(g, j0 + 16 * k, T), w8);
             }
+            if (wp) {
+              w_partials(wv, hw, dom, dde, dpi);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) wv[e] = wn[e];
+            }
           } else {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -441,6 +527,9 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
         }
         report(!last);   // the partner's sXcol was written
       }
+      if (ok && wp)
+        w_record(p.partials, (int64_t)q.part_begin + (int64_t)t * (2 * kEpiWarps) + rank * kEpiWarps + (warp - 2),
+                 dom, dde, dpi);
     }
   }
 
@@ -480,12 +569,14 @@ __global__ void __launch_bounds__(kThreads1, kCtasPerSm1) himuon_tile128_kernel(
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
   const uint32_t bar_base = smem_u32(bars);
   const uint32_t xfull = bar_base, xfree = bar_base + 8, mmadone = bar_base + 16, opnd = bar_base + 24;
+  const uint32_t stallbar = bar_base + 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(xfull, 1);
     mbar_init(xfree, 1);
     mbar_init(mmadone, 1);
     mbar_init(opnd, 4);                   // the four epilogue warps
+    mbar_init(stallbar, 1);
     mbar_fence_init();
   }
   if (warp == 1) {
@@ -530,7 +621,7 @@ __global__ void __launch_bounds__(kThreads1, kCtasPerSm1) himuon_tile128_kernel(
         ph_o ^= 1u;
         tc_fence_after();
       };
-      for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+      for (int tile = blockIdx.x, tl = 0; ok && tile < p.total_tiles; tile += gridDim.x, ++tl) {
         if (!mbar_wait(xfull, ph_x, limit)) {
           set_status(p.status, kTimeoutBit);
           break;
@@ -548,7 +639,13 @@ __global__ void __launch_bounds__(kThreads1, kCtasPerSm1) himuon_tile128_kernel(
             const uint64_t d = smem_desc_sw128(sX + kofs, 16, 1024);
             tc_mma(tmem_base, d, d, idesc_k, k != 0);
           }
-          tc_commit(mmadone);
+          if (p.test_stall && tl == 0 && it == 0) {
+            // Test stall, as in the T = 256 kernel: the MMAs complete on a spare barrier.
+            tc_commit(stallbar);
+            if (!mbar_wait(stallbar, 0, limit)) set_status(p.status, kTimeoutBit);
+          } else {
+            tc_commit(mmadone);
+          }
           wait_opnd();
           if (!ok) break;
 #pragma unroll
@@ -601,6 +698,10 @@ __global__ void __launch_bounds__(kThreads1, kCtasPerSm1) himuon_tile128_kernel(
       const int t = tile - q.tile_begin;
       const int64_t toff = (int64_t)t * T1 * T1 * 2;
       const float s = p.scales[q.seg_begin + t];
+      const bool wp = p.partials != nullptr && q.w != nullptr;
+      const int64_t wr = (int64_t)(t / q.w_tiles_c) * T1 + rl;
+      const int64_t wc = (int64_t)(t % q.w_tiles_c) * T1;
+      double dom = 0.0, dde = 0.0, dpi = 0.0;
       if (!mbar_wait(xfull, ph_x, limit)) {
         if (lane == 0) set_status(p.status, kTimeoutBit);
         break;
@@ -609,6 +710,7 @@ __global__ void __launch_bounds__(kThreads1, kCtasPerSm1) himuon_tile128_kernel(
       for (int it = 0; ok && it < K; ++it) {
         const float ca = p.coef[it][0], cb = p.coef[it][1], cc = p.coef[it][2];
         const float s2 = it == 0 ? s * s : 1.0f, ks = it == 0 ? s : 1.0f;
+        if (wp && it + 1 == K) w_prefetch(q, wr, wc, 128);
         wait_mma();
         if (!ok) break;
 #pragma unroll 1
@@ -649,15 +751,20 @@ __global__ void __launch_bounds__(kThreads1, kCtasPerSm1) himuon_tile128_kernel(
           }
         }
         report();
+        const bool last = it + 1 == K;
+        const bool wlast = wp && last;
+        uint32_t wv[16];
+        if (wlast) w_load(q, wr, wc, wv);       // in flight while the update MMAs run
         wait_mma();
         if (!ok) break;
-        const bool last = it + 1 == K;
         const char *clo = it < p.comp ? p.ws + ((it % 2 == 0) ? q.xl0 : q.xl1) + toff : nullptr;
         char *dlo = (it + 1 < p.comp) ? p.ws + ((it % 2 == 0) ? q.xl1 : q.xl0) + toff : nullptr;
         char *dout = last ? p.ws + q.xo + toff : nullptr;
 #pragma unroll 1
         for (int ch = 0; ch < 4; ++ch) {
           const int j0 = 32 * ch;
+          uint32_t wn[16];
+          if (wlast && ch < 3) w_load(q, wr, wc + 32 * (ch + 1), wn);
           uint32_t r[32];
           tmem_ld32(tmem_base + (uint32_t)j0 + lane_off, r);
           uint32_t xw[16], lw[16];
@@ -693,6 +800,11 @@ __global__ void __launch_bounds__(kThreads1, kCtasPerSm1) himuon_tile128_kernel(
               unswizzle_pair(in8, odd, w8);
               st_global_256(dout + panel_pair_off(rl, j0 + 16 * k, T1), w8);
             }
+            if (wp) {
+              w_partials(wv, hw, dom, dde, dpi);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) wv[e] = wn[e];
+            }
           } else {
 #pragma unroll
             for (int c = 0; c < 4; ++c) st_shared_v4(sX + half_chunk(rl, j0 + 8 * c), hw + 4 * c);
@@ -710,6 +822,7 @@ __global__ void __launch_bounds__(kThreads1, kCtasPerSm1) himuon_tile128_kernel(
         }
         report();
       }
+      if (ok && wp) w_record(p.partials, (int64_t)q.part_begin + (int64_t)t * 4 + (warp - 2), dom, dde, dpi);
     }
   }
 

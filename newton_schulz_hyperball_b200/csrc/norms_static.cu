@@ -14,6 +14,9 @@
 // cudaGetSymbolAddress, with that device current, on the first call made on the device.
 // Every call shares the array: calls that overlap on the GPU (different streams, or
 // different host threads on one device) race and must be serialised by the caller.
+// The looked-up address is kept for the life of the process, so a device reset
+// (cudaDeviceReset) after the first call on that device is not supported.  A non-finite
+// norm shows only as a NaN or Inf in the output: there is no status word to read.
 #include <cuda_runtime.h>
 
 #include <cstring>
@@ -27,9 +30,11 @@ namespace {
 
 constexpr size_t kScratchBytes = NSHB_STATIC_SCRATCH_BYTES;
 constexpr size_t kStatusBytes = 256;                                  // status word + counter
-constexpr size_t kScalarsBytes = sizeof(MatScalars) * kMaxMats;       // per-matrix records
+constexpr int kStaticMaxMats = 192;                                   // matrices per call
+constexpr size_t kScalarsBytes = sizeof(MatScalars) * kStaticMaxMats; // per-matrix records
 constexpr size_t kPartialsOff = kStatusBytes + ((kScalarsBytes + 255) / 256) * 256;
 constexpr size_t kMaxBlocks = (kScratchBytes - kPartialsOff) / (3 * sizeof(double));
+static_assert(kStaticMaxMats <= kMaxMats, "one launch of the norm kernels");
 
 __device__ __align__(256) unsigned char g_norm_scratch[kScratchBytes];
 
@@ -39,16 +44,18 @@ char *g_addr[64] = {nullptr};
 // Device address of g_norm_scratch on the current device (looked up once per device).
 nshb_status scratch_address(char **out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) {
-    (void)cudaGetLastError();
+  const cudaError_t de = cudaGetDevice(&dev);
+  if (de != cudaSuccess) {
+    record_cuda_error(de);
     return NSHB_ERR_CUDA;
   }
   if (dev < 0 || dev >= 64) return NSHB_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> g(g_mu);
   if (!g_addr[dev]) {
     void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_norm_scratch) != cudaSuccess || !p) {
-      (void)cudaGetLastError();
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_norm_scratch);
+    if (e != cudaSuccess || !p) {
+      record_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
       return NSHB_ERR_CUDA;
     }
     g_addr[dev] = static_cast<char *>(p);
@@ -68,7 +75,7 @@ extern "C" nshb_status nshb_fro_norms_static(const nshb_matrix *mats, int32_t n_
   if (n_mats == 0) return NSHB_OK;
   if (!mats || !out) return NSHB_ERR_NULL;
   if ((uintptr_t)out % sizeof(float)) return NSHB_ERR_SHAPE;
-  if (n_mats > kMaxMats) return NSHB_ERR_WORKSPACE;
+  if (n_mats > kStaticMaxMats) return NSHB_ERR_WORKSPACE;
   ApplyParams ap;
   ApplyFinParams fp;
   std::memset(&ap, 0, sizeof(ap));
@@ -76,13 +83,10 @@ extern "C" nshb_status nshb_fro_norms_static(const nshb_matrix *mats, int32_t n_
   size_t blocks = 0;
   for (int i = 0; i < n_mats; ++i) {
     const nshb_matrix &d = mats[i];
-    if (d.rows <= 0 || d.cols <= 0 || d.ld < d.cols) return NSHB_ERR_SHAPE;
-    if (d.rows > (1LL << 20) || d.cols > (1LL << 20) || d.ld > (1LL << 30)) return NSHB_ERR_UNSUPPORTED;
-    if (!d.W) return NSHB_ERR_NULL;
-    if (d.w_dtype != NSHB_BF16 && d.w_dtype != NSHB_F32) return NSHB_ERR_DTYPE;
+    const nshb_status ce = check_matrix(d, nullptr, false, /*w_only=*/true);
+    if (ce != NSHB_OK) return ce;
     const bool wf32 = d.w_dtype == NSHB_F32;
     const size_t esz = wf32 ? 4 : 2;
-    if ((uintptr_t)d.W % esz) return NSHB_ERR_SHAPE;
     const bool vec = ((uintptr_t)d.W % 16 == 0) && ((d.ld * esz) % 16 == 0);
     MatDesc &md = ap.mats[i];
     md.W = d.W;
@@ -93,7 +97,9 @@ extern "C" nshb_status nshb_fro_norms_static(const nshb_matrix *mats, int32_t n_
     md.pr = (int)((d.rows + kBlk - 1) / kBlk * kBlk);
     md.pc = (int)((d.cols + kBlk - 1) / kBlk * kBlk);
     md.blk_begin = (int)blocks;
+    md.rec_begin = (int)blocks;
     md.mat = i;
+    fp.rec_begin[i] = (int)blocks;
     fp.blk_begin[i] = (int)blocks;
     fp.mat[i] = i;
     fp.m[i] = md.m;
@@ -102,6 +108,7 @@ extern "C" nshb_status nshb_fro_norms_static(const nshb_matrix *mats, int32_t n_
     if (blocks > kMaxBlocks) return NSHB_ERR_WORKSPACE;  // beyond the fixed scratch
   }
   fp.blk_begin[n_mats] = (int)blocks;
+  fp.rec_begin[n_mats] = (int)blocks;
 
   char *scratch = nullptr;
   nshb_status e = scratch_address(&scratch);
@@ -112,8 +119,9 @@ extern "C" nshb_status nshb_fro_norms_static(const nshb_matrix *mats, int32_t n_
   double *partials = reinterpret_cast<double *>(scratch + kPartialsOff);
   // The status word and the exact-pass counter start at zero; partials and records are
   // fully written by the kernels before they are read.
-  if (cudaMemsetAsync(status, 0, 2 * sizeof(uint32_t), st) != cudaSuccess) {
-    (void)cudaGetLastError();
+  cudaError_t ce = cudaMemsetAsync(status, 0, 2 * sizeof(uint32_t), st);
+  if (ce != cudaSuccess) {
+    record_cuda_error(ce);
     return NSHB_ERR_CUDA;
   }
   ap.ws = scratch;
@@ -131,7 +139,11 @@ extern "C" nshb_status nshb_fro_norms_static(const nshb_matrix *mats, int32_t n_
   fp.stage = 0;
   fp.hb_eps = 1e-8f;
   fp.nmat = n_mats;
-  if (launch_reduce(ap, st) != cudaSuccess) return NSHB_ERR_CUDA;
-  if (launch_apply_finalize(fp, st) != cudaSuccess) return NSHB_ERR_CUDA;
+  ce = launch_reduce(ap, st);
+  if (ce == cudaSuccess) ce = launch_apply_finalize(fp, st);
+  if (ce != cudaSuccess) {
+    record_cuda_error(ce);
+    return NSHB_ERR_CUDA;
+  }
   return NSHB_OK;
 }

@@ -42,6 +42,7 @@ constexpr int TMEM_COLS = 2 * BN;                 // two 128 x 256 fp32 accumula
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
+static_assert(2 * kEpiWarps == kPartsPerTile, "one partial record per epilogue warp of the pair");
 constexpr uint32_t kTimeoutBit = 0x4u;
 constexpr uint32_t kPeerMask = 0xFEFFFFFFu;       // clears the CTA-rank bit of a cluster address
 
@@ -168,7 +169,11 @@ __device__ __forceinline__ Tile decode2(const GemmParams &p, int tile) {
   return t;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
+// FUSE: the instance for the last update launch with Hyperball partials (W read in the
+// epilogue); the other launches use the instance without that code, whose register budget
+// it would otherwise raise.
+template <bool FUSE>
+__device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
@@ -218,8 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
       for (int tile = cid; ok && tile < p.total_tiles; tile += ncl) {
         const Tile t = decode2(p, tile);
         const GemmProb &q = p.prob[t.prob];
-        const int64_t a_row = (q.a_off + (int64_t)t.batch * q.a_bs) >> 7;   // 128-byte rows
-        const int64_t b_row = (q.b_off + (int64_t)t.batch * q.b_bs) >> 7;
+        const int64_t a_row = (q.a_off + (int64_t)t.batch * q.bs) >> 7;   // 128-byte rows
+        const int64_t b_row = (q.b_off + (int64_t)t.batch * q.bs) >> 7;
         const int am = t.m0 + 128 * (int)rank;     // this CTA's A rows
         const int bn = t.n0 + 128 * (int)rank;     // this CTA's B columns
         for (int kb = 0; kb < q.kt; kb += 2) {      // q.kt counts 64-deep panels
@@ -235,18 +240,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
             last_parity[stage] = (int)phase;
           }
           // K-major A: rows am .. am+127 of k panels kb and kb+1 (16 KB each)
-          const int64_t ya = a_row + (int64_t)kb * q.a_ph + am;
+          const int64_t ya = a_row + (int64_t)kb * q.ph + am;
           tma_load_2sm(sA, &p.tmap, 0, (int)ya, fb);
-          tma_load_2sm(sA + SLICE_BYTES, &p.tmap, 0, (int)(ya + q.a_ph), fb);
+          tma_load_2sm(sA + SLICE_BYTES, &p.tmap, 0, (int)(ya + q.ph), fb);
           if (p.mode != kUpdate) {
-            const int64_t yb = b_row + (int64_t)kb * q.b_ph + bn;
+            const int64_t yb = b_row + (int64_t)kb * q.ph + bn;
             tma_load_2sm(sB, &p.tmap, 0, (int)yb, fb);
-            tma_load_2sm(sB + SLICE_BYTES, &p.tmap, 0, (int)(yb + q.b_ph), fb);
+            tma_load_2sm(sB + SLICE_BYTES, &p.tmap, 0, (int)(yb + q.ph), fb);
           } else {
             // MN-major: the 128 columns are two 64-column panels, k rows kb*64 .. +127
-            const int64_t y0 = b_row + (int64_t)(bn >> 6) * q.b_ph + (int64_t)kb * 64;
+            const int64_t y0 = b_row + (int64_t)(bn >> 6) * q.ph + (int64_t)kb * 64;
             tma_load_2sm(sB, &p.tmap, 0, (int)y0, fb);
-            tma_load_2sm(sB + SLICE_BYTES, &p.tmap, 0, (int)(y0 + q.b_ph), fb);
+            tma_load_2sm(sB + SLICE_BYTES, &p.tmap, 0, (int)(y0 + q.ph), fb);
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -314,6 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
     const int row = 128 * (int)rank + quarter * 32 + lane;   // row of the 256-row tile
     const bool sym = sym_mode(p.mode);
     const bool needc = (p.mode == kPoly || p.mode == kUpdate);
+    const bool fuse = FUSE && p.mode == kUpdate && p.partials != nullptr;
     int tl = 0;
     for (int tile = cid; tile < p.total_tiles; tile += ncl, ++tl) {
       const Tile t = decode2(p, tile);
@@ -322,24 +328,91 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
       const uint32_t tph = (uint32_t)(tl >> 1) & 1u;
       const float s = q.scale_idx >= 0 ? p.scales[q.scale_idx + t.batch] : 1.0f;
       const float s2 = s * s;
-      const char *cbase = p.ws + q.c_off + (int64_t)t.batch * q.c_bs;
-      char *dbase = p.ws + q.d_off + (int64_t)t.batch * q.d_bs;
-      const char *clo = q.c_lo >= 0 ? p.ws + q.c_lo + (int64_t)t.batch * q.c_bs : nullptr;
-      char *dlo = q.d_lo >= 0 ? p.ws + q.d_lo + (int64_t)t.batch * q.d_bs : nullptr;
+      const char *cbase = p.ws + q.c_off + (int64_t)t.batch * q.bs;
+      char *dbase = p.ws + q.d_off + (int64_t)t.batch * q.bs;
+      const char *clo = q.c_lo >= 0 ? p.ws + q.c_lo + (int64_t)t.batch * q.bs : nullptr;
+      char *dlo = q.d_lo >= 0 ? p.ws + q.d_lo + (int64_t)t.batch * q.bs : nullptr;
       const int64_t i = t.m0 + row;
       const int ra = (int)(i >> 6);
       const int cc_end = (half + 1) * NCH;
+      // Hyperball partials of this problem: the caller's W next to O (X coordinates (i, c)
+      // are W's (i, c), or (c, i) for a matrix whose NS ran on the transpose, offset by the
+      // tile origin for a Hierarchical-Muon tile).
+      const bool wp = fuse && q.w != nullptr;
+      const bool wtall = wp && (q.w_flags & kPwTall);
+      int64_t wr0 = 0, wc0 = 0;
+      if (wp && (q.w_flags & kPwTiled)) {
+        wr0 = (int64_t)(t.batch / q.w_tiles_c) * q.ph;
+        wc0 = (int64_t)(t.batch % q.w_tiles_c) * q.ph;
+      }
+      // bf16 W of columns t.n0 + 32 cc .. +31 as pairs in logical order, zero outside W (the
+      // epilogue reads bf16 weights only; fp32 weights take the reduce pass).
+      auto load_w = [&](int cc, uint32_t (&wv)[16]) {
+        const int64_t xc0 = t.n0 + cc * 32;
+        const unsigned short *w16 = static_cast<const unsigned short *>(q.w);
+        if (wtall) {
+          const bool in = i < q.w_n;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int64_t r0 = xc0 + 2 * e;
+            const uint32_t lo = (in && r0 < q.w_m) ? (uint32_t)w16[r0 * q.w_ld + i] : 0u;
+            const uint32_t hi = (in && r0 + 1 < q.w_m) ? (uint32_t)w16[(r0 + 1) * q.w_ld + i] : 0u;
+            wv[e] = lo | (hi << 16);
+          }
+        } else {
+          const int64_t wr = wr0 + i, wc = wc0 + xc0;
+          if (wr < q.w_m && wc + 31 < q.w_n && (q.w_flags & kPwVec)) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(w16 + wr * q.w_ld + wc);
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const uint4 u = src[g];
+              wv[4 * g] = u.x; wv[4 * g + 1] = u.y; wv[4 * g + 2] = u.z; wv[4 * g + 3] = u.w;
+            }
+          } else {
+            const bool in = wr < q.w_m;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int64_t c = wc + 2 * e;
+              const uint32_t lo = (in && c < q.w_n) ? (uint32_t)w16[wr * q.w_ld + c] : 0u;
+              const uint32_t hi = (in && c + 1 < q.w_n) ? (uint32_t)w16[wr * q.w_ld + c + 1] : 0u;
+              wv[e] = lo | (hi << 16);
+            }
+          }
+        }
+      };
+      double dom = 0.0, dde = 0.0, dpi = 0.0;
+      // Pulls this thread's W elements of the tile into L2 while the MMAs run, so that the
+      // per-chunk loads below find them there.
+      auto prefetch_w = [&]() {
+        const int esz = 2;
+        const char *wb = static_cast<const char *>(q.w);
+        for (int c = half * NCH; c < cc_end; ++c) {
+          const int64_t xc0 = t.n0 + c * 32;
+          if (wtall) {
+            // the warp's lanes cover 32 consecutive columns of each W row: lane l pulls row xc0 + l
+            const int64_t r = xc0 + lane, c0w = i - lane;
+            if (r < q.w_m && c0w < q.w_n)
+              asm volatile("prefetch.global.L2 [%0];" ::"l"(wb + (r * q.w_ld + c0w) * esz));
+          } else {
+            const int64_t wr = wr0 + i, wc = wc0 + xc0;
+            if (wr < q.w_m && wc < q.w_n) {
+              asm volatile("prefetch.global.L2 [%0];" ::"l"(wb + (wr * q.w_ld + wc) * esz));
+            }
+          }
+        }
+      };
       auto live = [&](int cc) { return cc < cc_end && !(sym && ((t.n0 + cc * 32) >> 6) > ra); };
       const bool odd = i & 1;
       // C words of columns col0 .. col0+31 in logical order (two 32-byte sector reads).
+      // (The fused instance prefetches W instead of C's low part, which it reads in the chunk.)
       auto load_c = [&](int cc, uint32_t (&h)[16], uint32_t (&l)[16]) {
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
-          const size_t off = panel_pair_off(i, t.n0 + cc * 32 + 16 * k, q.d_ph);
+          const size_t off = panel_pair_off(i, t.n0 + cc * 32 + 16 * k, q.ph);
           uint32_t w[8];
           ld_global_256(cbase + off, w);
           unswizzle_pair(w, odd, h + 8 * k);
-          if (clo) {
+          if (!FUSE && clo) {
             ld_global_256(clo + off, w);
             unswizzle_pair(w, odd, l + 8 * k);
           } else {
@@ -349,8 +422,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
         }
       };
       int cc = half * NCH;
-      uint32_t ch[16], cl[16];
+      uint32_t ch[16], cl[16], wcur[16];
       if (needc && live(cc)) load_c(cc, ch, cl);
+      if (wp) {
+        prefetch_w();
+        load_w(cc, wcur);                    // in flight while the tile's MMAs finish
+      }
       if (!mbar_wait(tfull_bar(buf), tph, limit)) {
         set_status(p.status, kTimeoutBit);
         break;
@@ -360,14 +437,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
       for (; live(cc); ++cc) {
         const int col0 = t.n0 + cc * 32;
         const int ca = col0 >> 6;
-        uint32_t nh[16], nl[16];
+        uint32_t nh[16], nl[16], wn[16];
         if (needc && live(cc + 1)) load_c(cc + 1, nh, nl);
+        if (wp && live(cc + 1)) load_w(cc + 1, wn);
+        if (FUSE && clo) {
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            uint32_t w[8];
+            ld_global_256(clo + panel_pair_off(i, col0 + 16 * k, q.ph), w);
+            unswizzle_pair(w, odd, cl + 8 * k);
+          }
+        }
         uint32_t r[32];
         tmem_ld32(tmem_base + (uint32_t)(buf * BN + cc * 32) + ((uint32_t)(quarter * 32) << 16), r);
         tmem_ld_wait();
         float v[32];
         if (p.mode == kGramF32) {
-          float *drow = reinterpret_cast<float *>(dbase) + i * q.d_ph;
+          float *drow = reinterpret_cast<float *>(dbase) + i * q.ph;
 #pragma unroll
           for (int g = 0; g < 8; ++g)
             *reinterpret_cast<float4 *>(drow + col0 + 4 * g) =
@@ -376,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
           if (ca < ra) {
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              reinterpret_cast<float *>(dbase)[(int64_t)(col0 + e) * q.d_ph + i] = __uint_as_float(r[e]);
+              reinterpret_cast<float *>(dbase)[(int64_t)(col0 + e) * q.ph + i] = __uint_as_float(r[e]);
           }
           continue;
         }
@@ -398,12 +484,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
             }
           }
         }
+        float pom = 0.f, pde = 0.f, ppi = 0.f;   // this chunk's partials (32 terms, fp32)
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           uint32_t o[8], w[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) o[e] = pack_bf16(v[16 * k + 2 * e], v[16 * k + 2 * e + 1]);
-          const size_t off = panel_pair_off(i, col0 + 16 * k, q.d_ph);
+          if (wp) {
+            // of O as stored (bf16), which is what the apply pass reads
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float o0 = bf16lo(o[e]), o1 = bf16hi(o[e]);
+              const float w0 = bf16lo(wcur[8 * k + e]), w1 = bf16hi(wcur[8 * k + e]);
+              pom = fmaf(o0, o0, fmaf(o1, o1, pom));
+              pde = fmaf(w0, o0, fmaf(w1, o1, pde));
+              ppi = fmaf(w0, w0, fmaf(w1, w1, ppi));
+            }
+          }
+          const size_t off = panel_pair_off(i, col0 + 16 * k, q.ph);
           unswizzle_pair(o, odd, w);              // the same swap puts logical order back
           st_global_256(dbase + off, w);
           if (dlo) {
@@ -421,18 +519,37 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             __nv_bfloat16 h = __float2bfloat16_rn(v[e]);
-            *reinterpret_cast<__nv_bfloat16 *>(dbase + panel_chunk_off(col0 + e, ib, q.d_ph) + 2 * ie) = h;
+            *reinterpret_cast<__nv_bfloat16 *>(dbase + panel_chunk_off(col0 + e, ib, q.ph) + 2 * ie) = h;
           }
+        }
+        if (wp) {
+          dom += (double)pom;
+          dde += (double)pde;
+          dpi += (double)ppi;
         }
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           ch[e] = nh[e];
-          cl[e] = nl[e];
+          if (!FUSE) cl[e] = nl[e];
+          if (FUSE) wcur[e] = wn[e];
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) remote_arrive(mapa(tempty_bar(buf), 0));   // the leader's barrier
+      if (wp) {
+        // One record per epilogue warp and tile: fixed order, so the sums are deterministic.
+        dom = warp_sum(dom);
+        dde = warp_sum(dde);
+        dpi = warp_sum(dpi);
+        if (lane == 0) {
+          const int64_t rec = (int64_t)q.part_begin + (int64_t)(tile - q.tile_begin) * kPartsPerTile +
+                              (int64_t)rank * kEpiWarps + (warp - 2);
+          p.partials[3 * rec] = dom;
+          p.partials[3 * rec + 1] = dde;
+          p.partials[3 * rec + 2] = dpi;
+        }
+      }
     }
   }
 
@@ -444,6 +561,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
     tc_fence_after();
     tmem_dealloc2(tmem_base, TMEM_COLS);
   }
+}
+
+// 320 threads: three warps share one SM sub-partition's 16K registers, so 168 per thread is
+// the most a CTA can be given.
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
+  gemm_tc2_body<false>(p);
+}
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc2_fused_kernel(const __grid_constant__ GemmParams p) {
+  gemm_tc2_body<true>(p);
 }
 
 std::mutex g_tmap_mu;
@@ -478,9 +604,12 @@ cudaError_t launch_gemm_tc2(const GemmParams &p, int num_sms, cudaStream_t s) {
   cudaGetDevice(&dev);
   if (!attr_set.get(dev)) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemm_tc2_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set.set(dev, 1);
   }
+  const bool fused = p.mode == kUpdate && p.partials != nullptr;
   if (p.total_tiles <= 0) return cudaSuccess;
   // Pairs that can be resident at once (a GPC with an odd number of free SMs leaves one
   // idle), so that the persistent grid never spills into a second wave.
@@ -521,7 +650,7 @@ cudaError_t launch_gemm_tc2(const GemmParams &p, int num_sms, cudaStream_t s) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc2_kernel, p);
+  cudaError_t e = fused ? cudaLaunchKernelEx(&cfg, gemm_tc2_fused_kernel, p) : cudaLaunchKernelEx(&cfg, gemm_tc2_kernel, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

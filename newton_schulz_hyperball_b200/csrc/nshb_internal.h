@@ -8,6 +8,8 @@
 #include <atomic>
 #include <cstdint>
 
+#include "../../include/nshb.h"
+
 namespace nshb {
 
 // A once-per-device fact of a launcher (a kernel attribute already set, the CTAs that fit
@@ -22,8 +24,11 @@ struct PerDevice {
   }
 };
 
-constexpr int kMaxMats = 192;   // matrices per launch of a streaming kernel (host splits larger sets)
-constexpr int kMaxProb = 192;   // GEMM problems per launch
+// Matrices per launch of a streaming kernel and GEMM problems per launch (the host splits
+// larger sets).  224 keeps a whole 8B-width set (224 matrices) or Qwen3-style set (196) in
+// one launch per phase while every parameter block stays under the 32,764-byte limit.
+constexpr int kMaxMats = 224;
+constexpr int kMaxProb = 224;
 constexpr int kBlk = 64;        // streaming kernels work on 64 x 64 blocks
 
 // Matrix flags.
@@ -54,7 +59,7 @@ struct MatDesc {
   int32_t seg_begin; // first norm segment (matrix, or first tile when tiled)
   int32_t tiles_c;   // tiled: tiles per tile-row of the padded grid
   int32_t mat;       // index of the matrix in the whole call
-  int32_t pad_;
+  int32_t rec_begin; // reduce: first (||O||^2, <W,O>, ||W||^2) record of this matrix
 };
 
 // Momentum + U + per-block ||U||^2 partials.
@@ -96,7 +101,8 @@ struct MatScalars {
 enum ApplyOp { kOpMuon = 0, kOpHyperball = 1, kOpBrake = 2, kOpNorms = 3, kOpRelative = 4 };
 struct ApplyParams {
   char *ws;
-  double *partials;        // 3 doubles per block (reduce) or 1 (exact norm)
+  double *partials;        // reduce: 3 doubles per record (MatDesc::rec_begin + local block);
+                           // exact norm: 1 double per block of the launch
   MatScalars *scal;        // indexed by MatDesc::mat
   uint32_t *status;
   int32_t op;
@@ -104,7 +110,8 @@ struct ApplyParams {
   MatDesc mats[kMaxMats];
 };
 struct ApplyFinParams {
-  const double *partials;
+  const double *partials;  // stage 0: 3-double records; stage 1: exact-norm block sums
+  const double *xpartials;
   MatScalars *scal;
   uint32_t *status;
   const float *rho;        // device radii or NULL
@@ -112,7 +119,8 @@ struct ApplyFinParams {
   int32_t op, stage;       // stage 0: after the reduce; stage 1: after the exact-norm pass
   float lr, weight_decay, eta, hb_eps, brake_out, brake_in;
   int32_t nmat;
-  int32_t blk_begin[kMaxMats + 1];
+  int32_t rec_begin[kMaxMats + 1];  // stage 0: records of matrix k (contiguous)
+  int32_t blk_begin[kMaxMats + 1];  // stage 1: exact-norm blocks of matrix k
   int32_t mat[kMaxMats];
   int32_t m[kMaxMats], n[kMaxMats];
 };
@@ -132,16 +140,28 @@ struct AdamParams {
 };
 
 // One bf16 GEMM problem of a Newton-Schulz phase (possibly a batch of equal problems).
-// Operands live in the workspace in the panel layout (see panel_chunk_off).
+// Operands live in the workspace in the panel layout (see panel_chunk_off); every operand
+// of a problem has the same panel height and batch stride.
 struct GemmProb {
   int64_t a_off, b_off, c_off, d_off;  // byte offsets of batch 0
   int64_t c_lo, d_lo;                  // kUpdate: bf16 low parts of C (read) / D (written), or -1
-  int64_t a_bs, b_bs, c_bs, d_bs;      // byte strides between batches
-  int32_t a_ph, b_ph, d_ph;            // panel heights (C shares D's)
-  int32_t mt, nt, kt;                  // 128-row tiles, BN-column tiles, 64-deep k blocks
+  int64_t bs;                          // byte stride between batches (every operand)
+  int32_t ph;                          // panel height (padded rows) of every operand
+  int32_t mt, nt, kt;                  // 256-row tiles, BN-column tiles, 64-deep k blocks
   int32_t batch, tiles_per_batch, tile_begin;
   int32_t scale_idx;                   // scale of batch 0 in GemmParams::scales, or -1
+  // Hyperball partials of the last update (kUpdate with GemmParams::partials): the caller's
+  // weight W (rows w_m x w_n, leading dimension w_ld) read in the epilogue next to O.
+  const void *w;                       // NULL: no partials for this problem
+  int32_t w_m, w_n, w_ld;
+  int32_t w_flags;                     // kPwTall | kPwTiled | kPwVec (W is bf16)
+  int32_t w_tiles_c;                   // kPwTiled: tiles per tile-row (batch b = tile (b / tc, b % tc))
+  int32_t part_begin;                  // first partial record of this problem (16 per tile)
 };
+constexpr int kPwTall = 1;   // X = W^T: X element (r, c) is W element (c, r)
+constexpr int kPwTiled = 4;  // batch b is the T x T tile (b / w_tiles_c, b % w_tiles_c) of W
+constexpr int kPwVec = 8;    // W rows may be read with 16-byte loads
+constexpr int kPartsPerTile = 16;   // partial records per 256 x 256 tile (one per epilogue warp)
 enum GemmMode { kGram = 0, kPoly = 1, kUpdate = 2, kPlain = 3, kSub = 4, kGramF32 = 5 };
 struct GemmParams {
   CUtensorMap tmap;       // 2-SM kernel: the workspace seen as rows of 128 bytes (64 bf16),
@@ -149,6 +169,7 @@ struct GemmParams {
   char *ws;
   const float *scales;
   uint32_t *status;
+  double *partials;       // kUpdate: (||O||^2, <W,O>, ||W||^2) records of problems with w, or NULL
   long long wait_limit;   // clock cycles a role may wait on one mbarrier phase
   int32_t mode;           // kGram: D = s^2 acc (lower triangle + mirror)
                           // kPoly: D = cb C + cc acc (lower triangle + mirror)
@@ -170,6 +191,12 @@ struct HmProb {
   int32_t tile_begin;      // first tile of this matrix in the launch
   int32_t ntiles;
   int32_t seg_begin;       // scale of tile 0 in scales
+  int32_t w_tiles_c;       // tiles per tile-row of the matrix (tile t = (t / w_tiles_c, t % w_tiles_c))
+  // Hyperball partials (HmParams::partials): the caller's W read next to the final O.
+  const void *w;           // NULL: no partials for this matrix
+  int32_t w_m, w_n, w_ld;
+  int32_t w_flags;         // kPwVec (W is bf16)
+  int32_t part_begin;      // first record (one per epilogue warp and tile)
   int32_t pad_;
 };
 struct HmParams {
@@ -177,8 +204,12 @@ struct HmParams {
   char *ws;
   const float *scales;
   uint32_t *status;
+  double *partials;        // (||O||^2, <W,O>, ||W||^2) records, or NULL
   long long wait_limit;
   int32_t ns_steps, comp, nprob, total_tiles;
+  int32_t test_stall;      // tests only: the MMA warp withholds the first Gram commit of its
+                           // first tile, so the epilogues' bounded wait runs out
+  int32_t pad_;
   float coef[32][3];       // (a, b, c) of every iteration
   HmProb prob[kMaxProb];
 };
@@ -224,6 +255,13 @@ struct CholParams {          // one blocked-Cholesky step (column block k) for a
   int32_t n;
 };
 
+// Checks of one matrix that every entry point makes, in this order: sizes, limits, pointers,
+// dtype, element alignment (W, G, O_out to their element; M and, when given, V to 4 bytes).
+// w_only: only W is read (the norm entry points), so G, M and V are not looked at.
+nshb_status check_matrix(const nshb_matrix &d, const float *V = nullptr, bool need_v = false, bool w_only = false);
+// Records a CUDA error for nshb_last_cuda_error (per calling thread) and clears it.
+void record_cuda_error(cudaError_t e);
+
 // Launchers (defined in the .cu files); each returns cudaGetLastError().
 cudaError_t launch_momentum(const MomentumParams &p, cudaStream_t s);
 cudaError_t launch_norm_finalize(const NormFinParams &p, int nseg_total, cudaStream_t s);
@@ -232,7 +270,6 @@ cudaError_t launch_exact_norm(const ApplyParams &p, cudaStream_t s);
 cudaError_t launch_apply_finalize(const ApplyFinParams &p, cudaStream_t s);
 cudaError_t launch_apply(const ApplyParams &p, cudaStream_t s);
 cudaError_t launch_adam(const AdamParams &p, cudaStream_t s);
-cudaError_t launch_gemm_tc(const GemmParams &p, int bn, int num_sms, cudaStream_t s);
 // 2-SM (CTA pair) form: 256 x 256 tiles, tcgen05.mma.cta_group::2; p.tmap must be encoded.
 cudaError_t launch_gemm_tc2(const GemmParams &p, int num_sms, cudaStream_t s);
 // Tile-resident Hierarchical Muon for T = 256 (all iterations of a tile on one CTA pair).
@@ -245,5 +282,17 @@ cudaError_t launch_gemm_f32(const F32Params &p, cudaStream_t s);
 cudaError_t launch_pack_panels(const PackParams &p, cudaStream_t s);
 cudaError_t launch_ridge(const CholParams &p, cudaStream_t s);
 cudaError_t launch_potrf_block(const CholParams &p, cudaStream_t s);
+
+constexpr size_t kMaxParamBytes = 32764;   // kernel parameter limit (CUDA 12.1+, sm_70+)
+static_assert(sizeof(MomentumParams) <= kMaxParamBytes, "MomentumParams");
+static_assert(sizeof(NormFinParams) <= kMaxParamBytes, "NormFinParams");
+static_assert(sizeof(ApplyParams) <= kMaxParamBytes, "ApplyParams");
+static_assert(sizeof(ApplyFinParams) <= kMaxParamBytes, "ApplyFinParams");
+static_assert(sizeof(AdamParams) <= kMaxParamBytes, "AdamParams");
+static_assert(sizeof(GemmParams) <= kMaxParamBytes, "GemmParams");
+static_assert(sizeof(HmParams) <= kMaxParamBytes, "HmParams");
+static_assert(sizeof(F32Params) <= kMaxParamBytes, "F32Params");
+static_assert(sizeof(PackParams) <= kMaxParamBytes, "PackParams");
+static_assert(sizeof(CholParams) <= kMaxParamBytes, "CholParams");
 
 }  // namespace nshb

@@ -504,9 +504,10 @@ __device__ __forceinline__ void reduce_block(const ApplyParams &p, const MatDesc
   cta_sum<3>(a3, s, red, nred & 1);
   ++nred;
   if (threadIdx.x == 0) {
-    p.partials[3 * (int64_t)cblk + 0] = s[0];
-    p.partials[3 * (int64_t)cblk + 1] = s[1];
-    p.partials[3 * (int64_t)cblk + 2] = s[2];
+    const int64_t rec = (int64_t)d.rec_begin + (cblk - d.blk_begin);   // the matrix's own records
+    p.partials[3 * rec + 0] = s[0];
+    p.partials[3 * rec + 1] = s[1];
+    p.partials[3 * rec + 2] = s[2];
   }
 }
 
@@ -635,7 +636,9 @@ __global__ void apply_finalize_kernel(const __grid_constant__ ApplyFinParams p) 
   }
   double om = 0.0, de = 0.0, pi = 0.0, ex = 0.0;
   if (p.stage == 0) {
-    for (int b = p.blk_begin[k] + lane; b < p.blk_begin[k + 1]; b += 32) {
+    // (||O||^2, <W,O>, ||W||^2) records of this matrix: one per block of the reduce pass,
+    // or one per epilogue warp and tile of the last Newton-Schulz update
+    for (int b = p.rec_begin[k] + lane; b < p.rec_begin[k + 1]; b += 32) {
       om += p.partials[3 * (int64_t)b];
       de += p.partials[3 * (int64_t)b + 1];
       pi += p.partials[3 * (int64_t)b + 2];
@@ -644,7 +647,7 @@ __global__ void apply_finalize_kernel(const __grid_constant__ ApplyFinParams p) 
     de = warp_sum(de);
     pi = warp_sum(pi);
   } else if (s.need_exact) {
-    for (int b = p.blk_begin[k] + lane; b < p.blk_begin[k + 1]; b += 32) ex += p.partials[b];
+    for (int b = p.blk_begin[k] + lane; b < p.blk_begin[k + 1]; b += 32) ex += p.xpartials[b];
     ex = warp_sum(ex);
   }
   if (lane != 0) return;

@@ -134,8 +134,9 @@ def test_workspace_too_small_or_misaligned_is_rejected_before_launch():
     lib = nshb.lib()
     m = fake_mats([(64, 64)])
     p = nshb.params()
-    need = ws_size(m, p, nshb.NSHB_OP_HYPERBALL)
-    for fn in (lib.muon_step, lib.hyperball_step, lib.radial_brake_step):
+    for fn, op in ((lib.muon_step, nshb.NSHB_OP_MUON), (lib.hyperball_step, nshb.NSHB_OP_HYPERBALL),
+                   (lib.radial_brake_step, nshb.NSHB_OP_RADIAL_BRAKE)):
+        need = ws_size(m, p, op)
         assert fn(m, 1, ctypes.byref(p), 0x20000000, need - 256, None) == nshb.NSHB_ERR_WORKSPACE
         assert fn(m, 1, ctypes.byref(p), 0x20000010, need, None) == nshb.NSHB_ERR_WORKSPACE
         assert fn(m, 1, ctypes.byref(p), None, need, None) == nshb.NSHB_ERR_NULL
@@ -155,7 +156,8 @@ def test_adam_params_layout_defaults_and_argument_errors():
     p = nshb.params()
     n = nshb.workspace_size(mats, p, nshb.NSHB_OP_ADAMH)
     assert n > 0
-    assert nshb.workspace_size(mats, p, nshb.NSHB_OP_RELATIVE_UPDATE) == nshb.workspace_size(mats, p, nshb.NSHB_OP_MUON)
+    # RelativeUpdate adds the (||O||^2, <W,O>, ||W||^2) records to the Muon step's workspace
+    assert nshb.workspace_size(mats, p, nshb.NSHB_OP_RELATIVE_UPDATE) >= nshb.workspace_size(mats, p, nshb.NSHB_OP_MUON)
     V = [0x30000000, 0x31000000]
     ws = (0x40000000, n)
     for bad in (dict(step=0), dict(beta1=1.0), dict(beta2=-0.1), dict(eps=0.0)):

@@ -93,3 +93,29 @@ def test_himuon_tile_schedule_follows_oracle():
             Wr[i], Mr[i], Or, _ = o.himuon_step(Wr[i], Gs[i], Mr[i], tile=T, eta=0.02, rho=rhos[i])
             assert rel_fro(Mg[i], Mr[i]) <= 1e-6 * (step + 1), (step, i)
             assert rel_fro(Og[i], Or) <= 2e-2, (step, i, rel_fro(Og[i], Or))
+
+
+def test_chunked_step_keeps_a_flag_raised_in_the_first_chunk():
+    """A NaN gradient in the first chunk's matrix sets NSHB_DEV_NONFINITE; the later chunks
+    add their flags to the same status word without clearing it, so the flag is still there
+    when the call returns.  The matrix with the NaN keeps its weights, the others step."""
+    shapes = [(r, c) for _, r, c in wl.gpt2_small_shapes(3)]
+    W, G = device_set(shapes, 64)
+    G[0][3, 5] = float("nan")
+    W0 = [w.clone() for w in W]
+    M = [torch.zeros(w.shape, dtype=torch.float32, device=DEV) for w in W]
+    rho = torch.stack([w.float().norm() for w in W])
+    mats = nshb.matrices(W, G, M)
+    p = nshb.params(rho=rho, eta=0.02)
+    op = nshb.NSHB_OP_HYPERBALL
+    full = nshb.workspace_size(mats, p, op)
+    size = max(nshb.workspace_size_min(mats, p, op), int(full * 0.3) // 256 * 256)
+    ws = torch.empty(size, dtype=torch.uint8, device=DEV)
+    n = nshb.step_chunked(op, mats, p, ws)
+    assert n >= 3
+    flags = nshb.device_status(ws)
+    assert flags & nshb.NSHB_DEV_NONFINITE
+    assert torch.equal(W[0], W0[0])
+    assert not torch.equal(W[-1], W0[-1])
+    for w in W[1:]:
+        assert torch.isfinite(w.float()).all()

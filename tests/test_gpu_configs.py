@@ -120,11 +120,13 @@ def test_qwen3_1b_full_set(kind):
 @pytest.mark.parametrize("tile,layers", [(256, 32), (512, 32), (128, 4)])
 def test_8b_width_himuon(tile, layers):
     """8B-width matrices (32 layers: 224 matrices, 6.98B parameters) with every T x T tile
-    batched in one himuon_step; a 4096^2 and a 1024x4096 matrix of layer 0 checked tile by
-    tile against the oracle, the radius of every matrix checked."""
+    batched in one himuon_step.  Checked tile by tile against the oracle: one matrix of every
+    shape of layer 0 (4096^2, 1024x4096, 14336x4096, 4096x14336) and two of the last layer
+    (its 1024x4096 and 4096x14336); the radius of every matrix checked."""
     cfg = wl.CFG_8B_WIDTH
     shapes = [(r, c) for _, r, c in wl.width_8b_shapes(layers)]
-    sampled = {0, 2}
+    last = 7 * (layers - 1)
+    sampled = {0, 2, 4, 6, last + 3, last + 6}
     W, M, O, rho, flags, w0 = run_set(shapes, sampled, cfg, "himuon", tile=tile, eta=0.02)
     assert flags == 0
     check_sampled(shapes, sampled, cfg, "himuon", W, M, O, rho, w0, tile=tile, eta=0.02)
