@@ -13,7 +13,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libnshb.so")
-SOURCES = ["api.cu", "stream_kernels.cu", "ns_f32.cu", "ns_tc2.cu", "himuon_tile.cu", "newton.cu",
+SOURCES = ["api.cu", "stream_kernels.cu", "ns_f32.cu", "ns_tc2.cu", "himuon_tile.cu", "newton.cu", "newton_tc.cu",
            "norms_static.cu"]
 HEADERS = ["nshb_internal.h", "nshb_device.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -30,7 +30,7 @@ def nvcc_path() -> str:
 
 
 def _inputs():
-    srcs = [os.path.join(CSRC, s) for s in SOURCES if os.path.exists(os.path.join(CSRC, s))]
+    srcs = [os.path.join(CSRC, s) for s in SOURCES]
     deps = srcs + [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(ROOT, "include", "nshb.h")]
     return srcs, deps
 
@@ -48,8 +48,9 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     srcs, _ = _inputs()
     tmp = LIB + ".tmp"
+    # --no-undefined: a symbol that no source defines fails the build instead of the first call
     cmd = [nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
-           "-I", os.path.join(ROOT, "include"), "-o", tmp, *srcs]
+           "-Xlinker", "--no-undefined", "-I", os.path.join(ROOT, "include"), "-o", tmp, *srcs]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd))

@@ -62,15 +62,21 @@ struct Plan {
   int bn = 256;
   int comp = 0;                  // compensated (hi/lo) iterations of the bf16 chain
   std::vector<MatPlan> mp;
-  // Newton-Muon: per layer input Z
+  // Newton-Muon: per layer input Z (d rows, padded to Dp = a multiple of 256)
   struct ZPlan {
     int64_t d = 0, Dp = 0;
     const void *src = nullptr;
-    int64_t zp = 0, s = 0, inv = 0;   // panel copy of Z, S / L (fp32 Dp x Dp), diagonal-block inverses
+    int64_t zp = 0;                   // panel copy of Z (Dp x n_tokens bf16)
+    int64_t s = 0;                    // S = Z Z^T + lambda I, fp32 Dp x Dp, updated in place
+    int64_t sh = 0, sl = 0;           // bf16 hi / lo panels of S (operands of the panel products)
+    int64_t lh = 0, ll = 0;           // bf16 hi / lo panels of the Cholesky factor L
+    int64_t dh = 0, dl = 0;           // hi / lo panels of the stacked diagonal-block inverses (Dp x 256)
   };
   std::vector<ZPlan> zp;
   int64_t n_tokens = 0;
-  std::vector<int64_t> r_off;         // per matrix: fp32 m x n buffer for U -> Y -> P
+  std::vector<int64_t> r_off;         // per matrix: fp32 m x n, U (momentum) and then P
+  std::vector<int64_t> y32, yh, yl;   // per matrix: fp32 Mp x Dp U -> Y, and its hi / lo panels
+  std::vector<int64_t> mpad;          // per matrix: rows padded to 256
   std::vector<int> zidx;
   size_t scal_off = 0, scale_off = 0, nu_off = 0, k1part_off = 0, wpart_off = 0, xpart_off = 0, total = 0;
   int nseg = 0, k1_total = 0, w_total = 0, rec_total = 0;
@@ -197,7 +203,7 @@ nshb_status plan_step(const nshb_matrix *mats, int n_mats, const nshb_params *p,
   pl.nu_off = off;
   off = align_up(off + sizeof(double) * (size_t)pl.nseg);
   pl.k1part_off = off;
-  off = align_up(off + sizeof(double) * (size_t)pl.k1_total);
+  off = align_up(off + kK1PartsPerBlock * sizeof(double) * (size_t)pl.k1_total);
   pl.wpart_off = off;
   off = align_up(off + 3 * sizeof(double) * (size_t)pl.rec_total);
   pl.xpart_off = off;
@@ -244,19 +250,33 @@ nshb_status plan_newton(const nshb_matrix *mats, int n_mats, const void *const *
     z.src = Z ? Z[j] : nullptr;
     if (Z && (!z.src || (uintptr_t)z.src % 16 != 0)) return !z.src ? NSHB_ERR_NULL : NSHB_ERR_SHAPE;
     z.Dp = round_up(z.d, 256);
+    const size_t sq = (size_t)z.Dp * z.Dp;
     z.zp = off; off = align_up(off + (size_t)z.Dp * n_tokens * 2);
-    z.s = off;  off = align_up(off + (size_t)z.Dp * z.Dp * 4);
-    z.inv = off; off = align_up(off + (size_t)(z.d / 64) * 64 * 64 * 4);
+    z.s = off;  off = align_up(off + sq * 4);
+    z.sh = off; off = align_up(off + sq * 2);
+    z.sl = off; off = align_up(off + sq * 2);
+    z.lh = off; off = align_up(off + sq * 2);
+    z.ll = off; off = align_up(off + sq * 2);
+    z.dh = off; off = align_up(off + (size_t)z.Dp * 256 * 2);
+    z.dl = off; off = align_up(off + (size_t)z.Dp * 256 * 2);
   }
   pl.r_off.resize(n_mats);
+  pl.y32.resize(n_mats);
+  pl.yh.resize(n_mats);
+  pl.yl.resize(n_mats);
+  pl.mpad.resize(n_mats);
   pl.zidx.resize(n_mats);
   for (int i = 0; i < n_mats; ++i) {
     const int zi = mats[i].z_index;
     if (zi < 0 || zi >= n_z) return NSHB_ERR_PARAM;
     if (pl.zp[zi].d != mats[i].cols) return NSHB_ERR_SHAPE;
     pl.zidx[i] = zi;
-    pl.r_off[i] = off;
-    off = align_up(off + (size_t)mats[i].rows * mats[i].cols * 4);
+    const int64_t Mp = round_up(mats[i].rows, 256), Dp = pl.zp[zi].Dp;
+    pl.mpad[i] = Mp;
+    pl.r_off[i] = off; off = align_up(off + (size_t)mats[i].rows * mats[i].cols * 4);
+    pl.y32[i] = off;   off = align_up(off + (size_t)Mp * Dp * 4);
+    pl.yh[i] = off;    off = align_up(off + (size_t)Mp * Dp * 2);
+    pl.yl[i] = off;    off = align_up(off + (size_t)Mp * Dp * 2);
   }
   pl.total = off;
   return NSHB_OK;
@@ -300,7 +320,7 @@ MatDesc make_desc(const nshb_matrix &d, const MatPlan &m, int idx, int64_t o_off
 // those that touch the lower triangle (BM-row block mi needs the BN-wide column tiles
 // that start at or before its last row).
 int gemm_tiles(int mode, int mt, int nt, int bm, int bn) {
-  if (mode == kUpdate || mode == kPlain) return mt * nt;
+  if (mode == kUpdate) return mt * nt;
   int cnt = 0;
   for (int mi = 0; mi < mt; ++mi) cnt += std::min(nt, (bm * mi + bm - 1) / bn + 1);
   return cnt;
@@ -394,7 +414,7 @@ nshb_status run_momentum(const nshb_matrix *mats, const Plan &pl, const nshb_par
     MomentumParams mp;
     std::memset(&mp, 0, sizeof(mp));
     mp.ws = ws;
-    mp.partials = k1part + pl.mp[c0].k1_begin;
+    mp.partials = k1part + kK1PartsPerBlock * (int64_t)pl.mp[c0].k1_begin;
     mp.status = reinterpret_cast<uint32_t *>(ws);
     mp.beta = p->beta;
     mp.nesterov = p->nesterov ? 1 : 0;
@@ -413,7 +433,7 @@ nshb_status run_momentum(const nshb_matrix *mats, const Plan &pl, const nshb_par
 
     NormFinParams nf;
     std::memset(&nf, 0, sizeof(nf));
-    nf.partials = k1part + pl.mp[c0].k1_begin;
+    nf.partials = k1part + kK1PartsPerBlock * (int64_t)pl.mp[c0].k1_begin;
     const int seg0 = pl.mp[c0].seg_begin;
     nf.scales = reinterpret_cast<float *>(ws + pl.scale_off) + seg0;
     nf.nus = reinterpret_cast<double *>(ws + pl.nu_off) + seg0;
@@ -424,8 +444,8 @@ nshb_status run_momentum(const nshb_matrix *mats, const Plan &pl, const nshb_par
     for (int i = c0; i < c1; ++i) {
       const MatPlan &m = pl.mp[i];
       nf.seg_begin[i - c0] = segs;
-      nf.blk_begin[i - c0] = blks;
-      nf.bps[i - c0] = m.k1_blocks / m.nseg;
+      nf.blk_begin[i - c0] = kK1PartsPerBlock * blks;             // partial records
+      nf.bps[i - c0] = kK1PartsPerBlock * (m.k1_blocks / m.nseg);  // records per segment
       segs += m.nseg;
       blks += m.k1_blocks;
     }
@@ -718,46 +738,49 @@ nshb_status run_apply(const nshb_matrix *mats, const Plan &pl, const nshb_params
   return NSHB_OK;
 }
 
-// F32 GEMM problem helper.
-// Output tiles of an fp32 GEMM problem (all, or those on and below the diagonal).
-int f32_tiles(const F32Prob &q) {
-  const int tm = (q.M + kF32Tile - 1) / kF32Tile;
-  if (!q.lower) return tm * q.tiles_n;
-  int cnt = 0;
-  for (int mi = 0; mi < tm; ++mi) cnt += std::min(mi + 1, q.tiles_n);
-  return cnt;
-}
-
-F32Prob f32prob(int64_t a, int lda, int64_t b, int ldb, int bt, int64_t c, int64_t d, int ldc, int M, int N, int K) {
-  F32Prob q;
+NwProb nw_prob() {
+  NwProb q;
   std::memset(&q, 0, sizeof(q));
-  q.a_off = a; q.lda = lda;
-  q.b_off = b; q.ldb = ldb; q.b_trans = bt;
-  q.c_off = c; q.d_off = d; q.ldc = ldc;
-  q.M = M; q.N = N; q.K = K;
-  q.scale_idx = -1;
-  q.tiles_n = (N + kF32Tile - 1) / kF32Tile;
+  q.c32 = q.d32 = q.dhi = q.dlo = -1;
+  q.kt = 4;                        // every product is 256 deep (one block column)
   return q;
 }
 
-// Launches the fp32 GEMM on a list of problems (split into launches of kMaxProb).
-nshb_status run_f32(const std::vector<F32Prob> &probs, int mode, char *ws, cudaStream_t st) {
-  for (size_t c0 = 0; c0 < probs.size(); c0 += kMaxProb) {
-    const size_t c1 = std::min(probs.size(), c0 + kMaxProb);
-    F32Params fp;
-    std::memset(&fp, 0, sizeof(fp));
-    fp.ws = ws;
-    fp.mode = mode;
+// Launches the split-precision products of `probs` (in launches of kMaxNwProb).
+nshb_status run_nw(NwParams &np, const std::vector<NwProb> &probs, cudaStream_t st) {
+  for (size_t c0 = 0; c0 < probs.size(); c0 += kMaxNwProb) {
+    const size_t c1 = std::min(probs.size(), c0 + (size_t)kMaxNwProb);
     int tiles = 0;
     for (size_t i = c0; i < c1; ++i) {
-      F32Prob q = probs[i];
+      NwProb q = probs[i];
       q.tile_begin = tiles;
-      tiles += f32_tiles(q);
-      fp.prob[i - c0] = q;
+      tiles += (q.flags & kNwLower) ? q.mt * (q.mt + 1) / 2 : q.mt * q.nt;
+      np.prob[i - c0] = q;
     }
-    fp.nprob = (int)(c1 - c0);
-    fp.total_tiles = tiles;
-    NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_gemm_f32(fp, st));
+    np.nprob = (int)(c1 - c0);
+    np.total_tiles = tiles;
+    NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_newton_gemm(np, device_sms(), st));
+  }
+  return NSHB_OK;
+}
+
+// fp32 -> bf16 hi / lo panels for a list of regions (in launches of kMaxMats).
+nshb_status run_split(const std::vector<SplitItem> &items, char *ws, cudaStream_t st) {
+  for (size_t c0 = 0; c0 < items.size(); c0 += kMaxMats) {
+    const size_t c1 = std::min(items.size(), c0 + (size_t)kMaxMats);
+    SplitParams sp;
+    std::memset(&sp, 0, sizeof(sp));
+    sp.ws = ws;
+    int nb = 0;
+    for (size_t i = c0; i < c1; ++i) {
+      SplitItem it = items[i];
+      it.blk_begin = nb;
+      nb += (it.prow / 64) * (it.pcol / 64);
+      sp.item[i - c0] = it;
+    }
+    sp.n = (int)(c1 - c0);
+    sp.total_blocks = nb;
+    NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_split(sp, st));
   }
   return NSHB_OK;
 }
@@ -844,9 +867,9 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
     NSHB_CHECK_CUDA(encode_ws_tensor_map(&gp.tmap, ws, pl.total / 128 * 128));
     NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_gemm_tc2(gp, device_sms(), st));
   }
-  // 3. blocked Cholesky, all layer inputs at once
-  int64_t dmax = 0;
-  for (auto &z : pl.zp) dmax = std::max(dmax, z.d);
+  // 3. ridge (and a unit diagonal on the padding), then the operands of the first step as
+  //    bf16 hi / lo panels: S's first column block and every U (with an fp32 copy padded to
+  //    Mp x Dp, the running Y of the forward solve)
   for (int c0 = 0; c0 < nz; c0 += kMaxMats) {
     const int c1 = std::min(nz, c0 + kMaxMats);
     CholParams cp;
@@ -857,58 +880,154 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
     cp.n = c1 - c0;
     for (int j = c0; j < c1; ++j) {
       cp.s_off[j - c0] = pl.zp[j].s;
-      cp.inv_off[j - c0] = pl.zp[j].inv;
       cp.ld[j - c0] = (int)pl.zp[j].Dp;
       cp.d[j - c0] = (int)pl.zp[j].d;
     }
     NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_ridge(cp, st));
-    for (int64_t k = 0; k < dmax; k += 64) {
-      cp.k = (int)k;
-      NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_potrf_block(cp, st));
-      std::vector<F32Prob> panel, trail;
-      for (int j = c0; j < c1; ++j) {
-        const Plan::ZPlan &z = pl.zp[j];
-        if (k + 64 >= z.d) continue;
-        const int ld = (int)z.Dp, rest = (int)(z.d - k - 64);
-        const int64_t pan = z.s + ((k + 64) * z.Dp + k) * 4;
-        panel.push_back(f32prob(pan, ld, z.inv + (k / 64) * 64 * 64 * 4, 64, 1, pan, pan, ld, rest, 64, 64));
-        const int64_t tr = z.s + ((k + 64) * z.Dp + (k + 64)) * 4;
-        trail.push_back(f32prob(pan, ld, pan, ld, 1, tr, tr, ld, rest, rest, 64));
-        trail.back().lower = 1;   // symmetric update: the factorisation reads the lower triangle only
-      }
-      nshb_status e = run_f32(panel, kPlain, ws, st);
-      if (e != NSHB_OK) return e;
-      e = run_f32(trail, kSub, ws, st);
-      if (e != NSHB_OK) return e;
-    }
   }
-  // 4. P = U L^-T L^-1 by right-looking block solves, in place on the fp32 buffer
-  int max_blocks = 0;
-  for (int i = 0; i < n; ++i) max_blocks = std::max(max_blocks, (int)(pl.mp[i].n / 64));
-  for (int pass = 0; pass < 2; ++pass) {
-    for (int sidx = 0; sidx < max_blocks; ++sidx) {
-      std::vector<F32Prob> solve, upd;
-      for (int i = 0; i < n; ++i) {
-        const Plan::ZPlan &z = pl.zp[pl.zidx[i]];
-        const int d = (int)pl.mp[i].n, m = (int)pl.mp[i].m, nb = d / 64;
-        if (sidx >= nb) continue;
-        const int kb = pass == 0 ? sidx : nb - 1 - sidx;
-        const int64_t k = (int64_t)kb * 64;
-        const int64_t R = pl.r_off[i];
-        const int64_t inv = z.inv + (int64_t)kb * 64 * 64 * 4;
-        solve.push_back(f32prob(R + k * 4, d, inv, 64, pass == 0 ? 1 : 0, R + k * 4, R + k * 4, d, m, 64, 64));
-        if (pass == 0 && k + 64 < d) {
-          upd.push_back(f32prob(R + k * 4, d, z.s + ((k + 64) * z.Dp + k) * 4, (int)z.Dp, 1, R + (k + 64) * 4,
-                                R + (k + 64) * 4, d, m, (int)(d - k - 64), 64));
-        } else if (pass == 1 && k > 0) {
-          upd.push_back(f32prob(R + k * 4, d, z.s + (k * z.Dp) * 4, (int)z.Dp, 0, R, R, d, m, (int)k, 64));
-        }
-      }
-      nshb_status e = run_f32(solve, kPlain, ws, st);
-      if (e != NSHB_OK) return e;
-      e = run_f32(upd, kSub, ws, st);
-      if (e != NSHB_OK) return e;
+  {
+    std::vector<SplitItem> items;
+    for (auto &z : pl.zp) {
+      SplitItem it;
+      std::memset(&it, 0, sizeof(it));
+      it.src32 = z.s;
+      it.dst32 = -1;
+      it.dhi = z.sh;
+      it.dlo = z.sl;
+      it.src_ld = (int)z.Dp;
+      it.rows = it.prow = (int)z.Dp;
+      it.cols = it.pcol = 256;
+      it.d_ph = (int)z.Dp;
+      items.push_back(it);
     }
+    for (int i = 0; i < n; ++i) {
+      const Plan::ZPlan &z = pl.zp[pl.zidx[i]];
+      SplitItem it;
+      std::memset(&it, 0, sizeof(it));
+      it.src32 = pl.r_off[i];
+      it.dst32 = pl.y32[i];
+      it.dhi = pl.yh[i];
+      it.dlo = pl.yl[i];
+      it.src_ld = (int)pl.mp[i].n;
+      it.dst_ld = (int)z.Dp;
+      it.rows = (int)pl.mp[i].m;
+      it.cols = (int)pl.mp[i].n;
+      it.prow = (int)pl.mpad[i];
+      it.pcol = (int)z.Dp;
+      it.d_ph = (int)pl.mpad[i];
+      items.push_back(it);
+    }
+    nshb_status e = run_split(items, ws, st);
+    if (e != NSHB_OK) return e;
+  }
+  NwParams np;
+  std::memset(&np, 0, sizeof(np));
+  np.ws = ws;
+  np.status = status;
+  np.wait_limit = limit;
+  NSHB_CHECK_CUDA(encode_ws_tensor_map(&np.tmap, ws, pl.total / 128 * 128));
+  int64_t dmax = 0;
+  for (auto &z : pl.zp) dmax = std::max(dmax, z.Dp);
+  const int nb = (int)(dmax / 256);
+  // 4. forward: blocked right-looking Cholesky S = L L^T with the rows of every U carried
+  //    along, so that block column k of Y = U L^-T is final after step k
+  for (int k = 0; k < nb; ++k) {
+    const int64_t k0 = 256LL * k, k1 = k0 + 256;
+    for (int c0 = 0; c0 < nz; c0 += kMaxMats) {
+      const int c1 = std::min(nz, c0 + kMaxMats);
+      DiagParams dp;
+      std::memset(&dp, 0, sizeof(dp));
+      dp.ws = ws;
+      dp.status = status;
+      dp.k = k;
+      for (int j = c0; j < c1; ++j) {
+        if (pl.zp[j].Dp <= k0) continue;
+        dp.s32[dp.n] = pl.zp[j].s;
+        dp.dhi[dp.n] = pl.zp[j].dh;
+        dp.dlo[dp.n] = pl.zp[j].dl;
+        dp.ld[dp.n] = (int)pl.zp[j].Dp;
+        dp.n++;
+      }
+      if (dp.n) NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_potrf_diag(dp, st));
+    }
+    // panel: L[k1:, k] = S[k1:, k] D_k^T and Y[:, k] = U[:, k] D_k^T
+    std::vector<NwProb> panel, trail;
+    for (auto &z : pl.zp) {
+      if (z.Dp <= k1) continue;
+      NwProb q = nw_prob();
+      q.a_hi = z.sh; q.a_lo = z.sl; q.a_ph = (int)z.Dp; q.a_r0 = (int)k1; q.a_k0 = (int)k0;
+      q.b_hi = z.dh; q.b_lo = z.dl; q.b_ph = (int)z.Dp; q.b_r0 = (int)k0; q.b_k0 = 0;
+      q.dhi = z.lh; q.dlo = z.ll; q.d_ph = (int)z.Dp; q.d_r0 = (int)k1; q.d_c0 = (int)k0;
+      q.mt = (int)((z.Dp - k1) / 256); q.nt = 1;
+      panel.push_back(q);
+      // trailing: S[k1:, k1:] -= L[k1:, k] L[k1:, k]^T (lower tiles), fp32 and panels
+      NwProb t = nw_prob();
+      t.a_hi = z.lh; t.a_lo = z.ll; t.a_ph = (int)z.Dp; t.a_r0 = (int)k1; t.a_k0 = (int)k0;
+      t.b_hi = z.lh; t.b_lo = z.ll; t.b_ph = (int)z.Dp; t.b_r0 = (int)k1; t.b_k0 = (int)k0;
+      t.c32 = t.d32 = z.s + (k1 * z.Dp + k1) * 4; t.ld32 = (int)z.Dp;
+      t.m_valid = t.n_valid = (int)(z.Dp - k1);
+      t.dhi = z.sh; t.dlo = z.sl; t.d_ph = (int)z.Dp; t.d_r0 = (int)k1; t.d_c0 = (int)k1;
+      t.mt = t.nt = (int)((z.Dp - k1) / 256);
+      t.flags = kNwLower;
+      trail.push_back(t);
+    }
+    for (int i = 0; i < n; ++i) {
+      const Plan::ZPlan &z = pl.zp[pl.zidx[i]];
+      if (z.Dp <= k0) continue;
+      NwProb q = nw_prob();
+      q.a_hi = pl.yh[i]; q.a_lo = pl.yl[i]; q.a_ph = (int)pl.mpad[i]; q.a_r0 = 0; q.a_k0 = (int)k0;
+      q.b_hi = z.dh; q.b_lo = z.dl; q.b_ph = (int)z.Dp; q.b_r0 = (int)k0; q.b_k0 = 0;
+      q.d32 = pl.y32[i] + k0 * 4; q.ld32 = (int)z.Dp; q.m_valid = (int)pl.mpad[i]; q.n_valid = 256;
+      q.dhi = pl.yh[i]; q.dlo = pl.yl[i]; q.d_ph = (int)pl.mpad[i]; q.d_r0 = 0; q.d_c0 = (int)k0;
+      q.mt = (int)(pl.mpad[i] / 256); q.nt = 1;
+      panel.push_back(q);
+      if (z.Dp <= k1) continue;
+      // U[:, k1:] -= Y[:, k] L[k1:, k]^T
+      NwProb t = nw_prob();
+      t.a_hi = pl.yh[i]; t.a_lo = pl.yl[i]; t.a_ph = (int)pl.mpad[i]; t.a_r0 = 0; t.a_k0 = (int)k0;
+      t.b_hi = z.lh; t.b_lo = z.ll; t.b_ph = (int)z.Dp; t.b_r0 = (int)k1; t.b_k0 = (int)k0;
+      t.c32 = t.d32 = pl.y32[i] + k1 * 4; t.ld32 = (int)z.Dp;
+      t.m_valid = (int)pl.mpad[i]; t.n_valid = (int)(z.Dp - k1);
+      t.dhi = pl.yh[i]; t.dlo = pl.yl[i]; t.d_ph = (int)pl.mpad[i]; t.d_r0 = 0; t.d_c0 = (int)k1;
+      t.mt = (int)(pl.mpad[i] / 256); t.nt = (int)((z.Dp - k1) / 256);
+      trail.push_back(t);
+    }
+    nshb_status e = run_nw(np, panel, st);
+    if (e != NSHB_OK) return e;
+    e = run_nw(np, trail, st);
+    if (e != NSHB_OK) return e;
+  }
+  // 5. backward: P L = Y, right-looking from the last block: P[:, k] = Y[:, k] D_k (fp32 into
+  //    the m x n buffer the momentum pass reads, and panels), then Y[:, :k] -= P[:, k] L[k, :k]
+  for (int k = nb - 1; k >= 0; --k) {
+    const int64_t k0 = 256LL * k;
+    std::vector<NwProb> solve, upd;
+    for (int i = 0; i < n; ++i) {
+      const Plan::ZPlan &z = pl.zp[pl.zidx[i]];
+      if (z.Dp <= k0) continue;
+      const int d = (int)pl.mp[i].n, m = (int)pl.mp[i].m;
+      NwProb q = nw_prob();
+      q.a_hi = pl.yh[i]; q.a_lo = pl.yl[i]; q.a_ph = (int)pl.mpad[i]; q.a_r0 = 0; q.a_k0 = (int)k0;
+      q.b_hi = z.dh; q.b_lo = z.dl; q.b_ph = (int)z.Dp; q.b_r0 = 0; q.b_k0 = (int)k0;
+      q.flags = kNwBMn;
+      q.d32 = pl.r_off[i] + k0 * 4; q.ld32 = d; q.m_valid = m; q.n_valid = (int)std::max<int64_t>(0, d - k0);
+      q.dhi = pl.yh[i]; q.dlo = pl.yl[i]; q.d_ph = (int)pl.mpad[i]; q.d_r0 = 0; q.d_c0 = (int)k0;
+      q.mt = (int)(pl.mpad[i] / 256); q.nt = 1;
+      solve.push_back(q);
+      if (k == 0) continue;
+      NwProb t = nw_prob();
+      t.a_hi = pl.yh[i]; t.a_lo = pl.yl[i]; t.a_ph = (int)pl.mpad[i]; t.a_r0 = 0; t.a_k0 = (int)k0;
+      t.b_hi = z.lh; t.b_lo = z.ll; t.b_ph = (int)z.Dp; t.b_r0 = 0; t.b_k0 = (int)k0;
+      t.flags = kNwBMn;
+      t.c32 = t.d32 = pl.y32[i]; t.ld32 = (int)z.Dp; t.m_valid = (int)pl.mpad[i]; t.n_valid = (int)k0;
+      t.dhi = pl.yh[i]; t.dlo = pl.yl[i]; t.d_ph = (int)pl.mpad[i]; t.d_r0 = 0; t.d_c0 = 0;
+      t.mt = (int)(pl.mpad[i] / 256); t.nt = k;
+      upd.push_back(t);
+    }
+    nshb_status e = run_nw(np, solve, st);
+    if (e != NSHB_OK) return e;
+    e = run_nw(np, upd, st);
+    if (e != NSHB_OK) return e;
   }
   return NSHB_OK;
 }

@@ -48,32 +48,6 @@ constexpr int kHalf = 4 * kPanel128;            // 64 KB
 constexpr int SMEM_BYTES = 3 * kHalf + 1024 + 256;
 constexpr uint32_t kTimeoutBit = 0x4u;
 
-__device__ __forceinline__ uint32_t cta_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t cluster_id() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t num_clusters() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
 // 2-D TMA load into this CTA's shared memory, completing on this CTA's barrier.
 __device__ __forceinline__ void tma_load_local(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
   asm volatile(
@@ -81,30 +55,6 @@ __device__ __forceinline__ void tma_load_local(uint32_t dst, const CUtensorMap *
           "r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
       : "memory");
-}
-__device__ __forceinline__ void tmem_alloc2(uint32_t dst, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst), "r"(ncols) : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish2() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-__device__ __forceinline__ void tc_mma2(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.u32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void tc_commit2_mc(uint32_t bar, uint16_t mask) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::
-                   "r"(bar),
-               "h"(mask)
-               : "memory");
 }
 // Generic-proxy shared-memory writes become visible to the tensor core (async proxy): this
 // CTA's shared memory, or any shared memory of the cluster (writes into the partner's).
@@ -125,28 +75,6 @@ __device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t *w) {
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
                : "r"(addr)
-               : "memory");
-}
-// 32-byte global accesses of two logically adjacent 16-byte chunks of a panel row (the
-// 128-byte swizzle keeps chunks {c, c+1}, c even, in one sector, swapped on odd rows).
-__device__ __forceinline__ size_t panel_pair_off(int64_t row, int64_t col, int64_t ph) {
-  return ((size_t)((col >> 6) * ph + row) << 7) + ((size_t)(((col >> 4) & 3) ^ ((row >> 1) & 3)) << 5);
-}
-__device__ __forceinline__ void unswizzle_pair(const uint32_t (&w)[8], bool odd, uint32_t *out) {
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    out[e] = odd ? w[4 + e] : w[e];
-    out[4 + e] = odd ? w[e] : w[4 + e];
-  }
-}
-__device__ __forceinline__ void ld_global_256(const void *p, uint32_t (&w)[8]) {
-  asm volatile("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
-               : "l"(p));
-}
-__device__ __forceinline__ void st_global_256(void *p, const uint32_t (&w)[8]) {
-  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
-               "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
                : "memory");
 }
 

@@ -4,11 +4,11 @@
 //   pack_panels   layer input Z (bf16 row-major d x n) -> the tensor-core panel layout,
 //                 so that S = Z Z^T runs on the grouped tcgen05 GEMM (fp32 output);
 //   ridge         lambda = ridge_rel tr(S) / d, S += lambda I (one CTA per Z, fixed order);
-//   potrf_block   Cholesky of the 64 x 64 diagonal block at column k (lower factor, in
-//                 place) and the inverse of that factor, which turns each panel and
-//                 block solve into a small GEMM.
-// The panel solves, the trailing updates and the triangular solves for P = U S^-1 run on
-// the fp32 GEMM kernel; the host sequences them.
+//   split         fp32 regions -> bf16 hi / lo panels, the operands of the split products;
+//   potrf_diag    Cholesky factor of a 256 x 256 diagonal block and its inverse, which
+//                 turns every panel and block solve into a product.
+// The panel products, the trailing updates and the triangular solves for P = U S^-1 run
+// on the split-precision tensor-core GEMM (newton_tc.cu); the host sequences them.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -41,6 +41,9 @@ __global__ void __launch_bounds__(256) pack_panels_kernel(const __grid_constant_
   }
 }
 
+// lambda = ridge_rel tr(S) / d added to the diagonal.  The padded rows and columns of S
+// (d .. ld-1, zero from the Gram) get a unit diagonal, so the padded matrix factors as
+// [L 0; 0 I] and the padded columns of every solve stay zero.
 __global__ void __launch_bounds__(256) ridge_kernel(const __grid_constant__ CholParams p) {
   __shared__ double red[8];
   const int z = blockIdx.x;
@@ -51,57 +54,195 @@ __global__ void __launch_bounds__(256) ridge_kernel(const __grid_constant__ Chol
   block_sum<1>(v, red);
   const float lam = (float)((double)p.ridge_rel * v[0] / (double)d);
   for (int i = threadIdx.x; i < d; i += blockDim.x) S[(int64_t)i * ld + i] += lam;
+  for (int i = d + threadIdx.x; i < ld; i += blockDim.x) S[(int64_t)i * ld + i] = 1.f;
 }
 
-// Right-looking unblocked Cholesky of the 64 x 64 diagonal block in shared memory, then
-// the inverse of the lower factor by forward substitution (one column per thread).
-__global__ void __launch_bounds__(256) potrf_block_kernel(const __grid_constant__ CholParams p) {
-  __shared__ float A[64][65];
-  __shared__ float Li[64][65];
+// fp32 regions -> bf16 hi/lo panels (X_hi = bf16(X), X_lo = bf16(X - X_hi)), one 64 x 64
+// block per CTA; thread t handles row t/4 (+ 64 (t/256)) ... columns 16 (t % 4) .. +15.
+__global__ void __launch_bounds__(256) split_kernel(const __grid_constant__ SplitParams p) {
+  pdl_trigger();
+  pdl_wait();
+  const int blk = blockIdx.x;
+  if (blk >= p.total_blocks) return;
+  int lo = 0, hi = p.n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.item[mid].blk_begin <= blk) lo = mid; else hi = mid - 1;
+  }
+  const SplitItem &it = p.item[lo];
+  const int lb = blk - it.blk_begin, bc = it.pcol / 64;
+  const int r0 = (lb / bc) * 64, c0 = (lb % bc) * 64;
+  const float *src = reinterpret_cast<const float *>(p.ws + it.src32);
+  float *dst = it.dst32 >= 0 ? reinterpret_cast<float *>(p.ws + it.dst32) : nullptr;
+  for (int q = threadIdx.x; q < 64 * 8; q += blockDim.x) {
+    const int r = r0 + (q >> 3), c = c0 + 8 * (q & 7);
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = (r < it.rows && c + e < it.cols) ? src[(int64_t)r * it.src_ld + c + e] : 0.f;
+    if (dst) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dst[(int64_t)r * it.dst_ld + c + e] = v[e];
+    }
+    uint4 h, l;
+    uint32_t *hp = &h.x, *lp = &l.x;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      hp[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+      lp[e] = pack_bf16(v[2 * e] - bf16lo(hp[e]), v[2 * e + 1] - bf16hi(hp[e]));
+    }
+    const size_t off = panel_chunk_off(it.d_r0 + r, it.d_c0 + c, it.d_ph);
+    *reinterpret_cast<uint4 *>(p.ws + it.dhi + off) = h;
+    *reinterpret_cast<uint4 *>(p.ws + it.dlo + off) = l;
+  }
+}
+
+// ------------------------------------------------ diagonal block of the factorisation
+// One 256 x 256 diagonal block of S per layer input, factored as two 128-column halves in
+// shared memory (three 128 x 128 fp32 tiles), then inverted:
+//   L11 = chol(A11);  D11 = L11^-1;  L21 = A21 D11^T;  L22 = chol(A22 - L21 L21^T);
+//   D22 = L22^-1;  D21 = -D22 (L21 D11);
+// the inverse D = [D11 0; D21 D22] goes out as bf16 hi/lo panels (block k of the stack).
+constexpr int kT = 128, kTP = 129;       // tile size, padded row stride (floats)
+constexpr int kDiagThreads = 512;
+constexpr int kDiagSmem = 3 * kT * kTP * 4;
+
+// In-place lower Cholesky factor of a 128 x 128 tile (only its lower triangle is read).
+// Column j: every thread takes the pivot a = T[j][j], updates its share of the trailing
+// lower part with T[i][c] -= T[i][j] T[c][j] / a (four threads per row i, interleaved
+// columns), and scales column j - 1 by 1 / sqrt of that column's pivot.  A pivot that is
+// not positive is flagged (NSHB_DEV_NOT_SPD) and replaced by 1e-30.
+__device__ __forceinline__ float pivot(float a) { return a > 0.f ? a : 1e-30f; }
+
+__device__ void chol_tile(float *T, uint32_t *status) {
+  const int tid = threadIdx.x, rr = tid >> 2, cpart = tid & 3;
+  for (int j = 0; j < kT; ++j) {
+    const float a0 = T[j * kTP + j];
+    if (!(a0 > 0.f) && tid == 0) set_status(status, 0x10u);   // not positive definite in fp32
+    const float a = pivot(a0);
+    if (j > 0) {                                  // finish column j - 1
+      const float rs = rsqrtf(pivot(T[(j - 1) * kTP + (j - 1)]));
+      for (int i = j + tid; i < kT; i += kDiagThreads) T[i * kTP + (j - 1)] *= rs;
+    }
+    __syncthreads();
+    if (tid == 0 && j > 0) T[(j - 1) * kTP + (j - 1)] = sqrtf(pivot(T[(j - 1) * kTP + (j - 1)]));
+    const int i = j + 1 + rr;                     // one row per group of four threads
+    if (i < kT) {
+      const float li = T[i * kTP + j] / a;
+      for (int c = j + 1 + cpart; c <= i; c += 4) T[i * kTP + c] = fmaf(-li, T[c * kTP + j], T[i * kTP + c]);
+    }
+    __syncthreads();
+  }
+  if (tid == 0) T[(kT - 1) * kTP + (kT - 1)] = sqrtf(pivot(T[(kT - 1) * kTP + (kT - 1)]));
+  __syncthreads();
+}
+
+// D = L^-1 of a lower-triangular tile (D lower).  Warp w solves columns 8w .. 8w+7, four
+// lanes per column: D[i][c] = (delta_ic - sum_{c <= q < i} L[i][q] D[q][c]) / L[i][i].
+__device__ void inv_tile(const float *L, float *D) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = 8 * warp + (lane >> 2), part = lane & 3;
+  for (int i = 0; i < kT; ++i) {
+    float acc = 0.f;
+    if (i > c)
+      for (int q = c + part; q < i; q += 4) acc = fmaf(L[i * kTP + q], D[q * kTP + c], acc);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    if (part == 0) D[i * kTP + c] = i < c ? 0.f : ((i == c ? 1.f : 0.f) - acc) / L[i * kTP + i];
+    __syncwarp();
+  }
+  __syncthreads();
+}
+
+// acc[e] = sum_q X[r][q] Y'[q][c_e] for row r = tid / 4 and the interleaved columns
+// c_e = tid % 4 + 4 e (Y' = Y, or Y^T when ytrans): the four threads of a row read four
+// different banks.
+__device__ __forceinline__ void row_products(const float *X, const float *Y, bool ytrans, float (&acc)[32]) {
+  const int tid = threadIdx.x, r = tid >> 2, cp = tid & 3;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+  for (int q = 0; q < kT; ++q) {
+    const float x = X[r * kTP + q];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) acc[e] = fmaf(x, ytrans ? Y[(cp + 4 * e) * kTP + q] : Y[q * kTP + cp + 4 * e], acc[e]);
+  }
+}
+
+// Out = sgn * X Y' (128 x 128 tiles); Out may be X (every row of X is read first).
+__device__ void mul_tile(const float *X, const float *Y, float *Out, float sgn, bool ytrans) {
+  const int tid = threadIdx.x, r = tid >> 2, cp = tid & 3;
+  float acc[32];
+  row_products(X, Y, ytrans, acc);
+  __syncthreads();
+#pragma unroll
+  for (int e = 0; e < 32; ++e) Out[r * kTP + cp + 4 * e] = sgn * acc[e];
+  __syncthreads();
+}
+
+// Writes a 128 x 128 tile into the hi / lo panels of the inverse stack at (r0, c0).
+__device__ void store_tile_panels(const float *T, char *hi, char *lo, int ph, int r0, int c0) {
+  for (int q = threadIdx.x; q < kT * kT / 8; q += kDiagThreads) {
+    const int r = q >> 4, c = 8 * (q & 15);
+    uint4 h, l;
+    uint32_t *hp = &h.x, *lp = &l.x;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float v0 = T[r * kTP + c + 2 * e], v1 = T[r * kTP + c + 2 * e + 1];
+      hp[e] = pack_bf16(v0, v1);
+      lp[e] = pack_bf16(v0 - bf16lo(hp[e]), v1 - bf16hi(hp[e]));
+    }
+    const size_t off = panel_chunk_off(r0 + r, c0 + c, ph);
+    *reinterpret_cast<uint4 *>(hi + off) = h;
+    *reinterpret_cast<uint4 *>(lo + off) = l;
+  }
+}
+
+__device__ void load_tile(const float *S, int ld, int r0, int c0, float *T) {
+  for (int q = threadIdx.x; q < kT * kT; q += kDiagThreads) {
+    const int r = q >> 7, c = q & 127;
+    T[r * kTP + c] = S[(int64_t)(r0 + r) * ld + c0 + c];
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kDiagThreads, 1) potrf_diag_kernel(const __grid_constant__ DiagParams p) {
+  extern __shared__ float tsm[];
+  float *T0 = tsm, *T1 = tsm + kT * kTP, *T2 = tsm + 2 * kT * kTP;
+  pdl_trigger();
+  pdl_wait();
   const int z = blockIdx.x;
-  if (p.k >= p.d[z]) return;
-  float *S = reinterpret_cast<float *>(p.ws + p.s_off[z]);
-  float *inv = reinterpret_cast<float *>(p.ws + p.inv_off[z]) + (int64_t)(p.k / 64) * 64 * 64;
-  const int ld = p.ld[z], k = p.k;
-  for (int e = threadIdx.x; e < 64 * 64; e += 256) {
-    const int r = e >> 6, c = e & 63;
-    A[r][c] = S[(int64_t)(k + r) * ld + k + c];
-  }
-  __syncthreads();
-  for (int j = 0; j < 64; ++j) {
-    if (threadIdx.x == 0) {
-      float a = A[j][j];
-      if (!(a > 0.f)) {           // not positive definite in fp32: flag it, keep going
-        set_status(p.status, 0x10u);
-        a = 1e-30f;
-      }
-      A[j][j] = sqrtf(a);
-    }
-    __syncthreads();
-    const float djj = A[j][j];
-    for (int i = j + 1 + threadIdx.x; i < 64; i += 256) A[i][j] /= djj;
-    __syncthreads();
-    const int rem = 63 - j;
-    for (int e = threadIdx.x; e < rem * rem; e += 256) {
-      const int i = j + 1 + e / rem, c = j + 1 + e % rem;
-      if (c <= i) A[i][c] = fmaf(-A[i][j], A[c][j], A[i][c]);
-    }
+  if (z >= p.n) return;
+  const int ld = p.ld[z], k0 = 256 * p.k;
+  if (k0 >= ld) return;
+  const float *S = reinterpret_cast<const float *>(p.ws + p.s32[z]);
+  char *hi = p.ws + p.dhi[z], *lo = p.ws + p.dlo[z];
+  load_tile(S, ld, k0, k0, T0);                 // A11
+  chol_tile(T0, p.status);                       // L11
+  inv_tile(T0, T2);                              // D11
+  load_tile(S, ld, k0 + kT, k0, T1);             // A21
+  mul_tile(T1, T2, T1, 1.f, true);               // L21 = A21 D11^T
+  load_tile(S, ld, k0 + kT, k0 + kT, T0);        // A22
+  // A22 -= L21 L21^T (the upper part is computed too and never read)
+  {
+    const int tid = threadIdx.x, r = tid >> 2, cp = tid & 3;
+    float acc[32];
+    row_products(T1, T1, true, acc);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) T0[r * kTP + cp + 4 * e] -= acc[e];
     __syncthreads();
   }
-  // Inverse of the lower-triangular factor: L X = I, column c per thread.
-  if (threadIdx.x < 64) {
-    const int c = threadIdx.x;
-    for (int i = 0; i < 64; ++i) {
-      float acc = (i == c) ? 1.f : 0.f;
-      for (int q = c; q < i; ++q) acc = fmaf(-A[i][q], Li[q][c], acc);
-      Li[i][c] = (i >= c) ? acc / A[i][i] : 0.f;
-    }
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < 64 * 64; e += 256) {
-    const int r = e >> 6, c = e & 63;
-    S[(int64_t)(k + r) * ld + k + c] = (c <= r) ? A[r][c] : 0.f;
-    inv[e] = Li[r][c];
+  chol_tile(T0, p.status);                       // L22
+  store_tile_panels(T2, hi, lo, ld, k0, 0);      // D11
+  mul_tile(T1, T2, T1, 1.f, false);              // X = L21 D11
+  inv_tile(T0, T2);                              // D22
+  mul_tile(T2, T1, T0, -1.f, false);             // D21 = -D22 X
+  store_tile_panels(T0, hi, lo, ld, k0 + kT, 0);
+  store_tile_panels(T2, hi, lo, ld, k0 + kT, kT);
+  // the upper-right 128 x 128 of the block inverse is zero
+  for (int q = threadIdx.x; q < kT * kT / 8; q += kDiagThreads) {
+    const int r = q >> 4, c = 8 * (q & 15);
+    const size_t off = panel_chunk_off(k0 + r, kT + c, ld);
+    *reinterpret_cast<uint4 *>(hi + off) = make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4 *>(lo + off) = make_uint4(0, 0, 0, 0);
   }
 }
 
@@ -115,8 +256,20 @@ cudaError_t launch_ridge(const CholParams &p, cudaStream_t s) {
   if (p.n > 0) ridge_kernel<<<p.n, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
-cudaError_t launch_potrf_block(const CholParams &p, cudaStream_t s) {
-  if (p.n > 0) potrf_block_kernel<<<p.n, 256, 0, s>>>(p);
+cudaError_t launch_split(const SplitParams &p, cudaStream_t s) {
+  if (p.total_blocks > 0) return launch_pdl(split_kernel, p.total_blocks, 256, 0, s, p);
+  return cudaGetLastError();
+}
+cudaError_t launch_potrf_diag(const DiagParams &p, cudaStream_t s) {
+  static PerDevice attr_set;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr_set.get(dev)) {
+    cudaError_t e = cudaFuncSetAttribute(potrf_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDiagSmem);
+    if (e != cudaSuccess) return e;
+    attr_set.set(dev, 1);
+  }
+  if (p.n > 0) return launch_pdl(potrf_diag_kernel, p.n, kDiagThreads, kDiagSmem, s, p);
   return cudaGetLastError();
 }
 

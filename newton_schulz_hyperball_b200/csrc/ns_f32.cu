@@ -8,10 +8,7 @@
 //   kUpdate  X' = s (a X + B X)
 // where s = 1 / (||U|| + eps) on the first iteration (the normalisation folded into the
 // first Gram and update epilogues) and 1 afterwards ("Muon: the orthogonalized optimizer
-// explained", Newton-Schulz section and newton_schulz5).  The same kernel also computes the
-// plain product D = A B and the update D = C - A B of the Newton-Muon Cholesky
-// factorisation and triangular solves; a problem may ask for the output tiles on and
-// below the diagonal only (the symmetric trailing update of the factorisation).
+// explained", Newton-Schulz section and newton_schulz5).
 //
 // 128x128 output tiles, 8-deep k slices double-buffered in shared memory, 256 threads
 // with an 8x8 register tile each (rows ty*4 + {0..3, 64..67}, columns tx*4 + {0..3,
@@ -87,20 +84,10 @@ __device__ __forceinline__ void store_slice(const F32Prob &q, const Slice &s, fl
   }
 }
 
-// Tile (mi, ni) of local tile index lt: all tiles row by row, or only those with ni <= mi.
+// Tile (mi, ni) of local tile index lt, row by row.
 __device__ __forceinline__ void decode_tile(const F32Prob &q, int lt, int &mi, int &ni) {
-  if (!q.lower) {
-    mi = lt / q.tiles_n;
-    ni = lt % q.tiles_n;
-    return;
-  }
-  mi = 0;
-  for (;; ++mi) {
-    const int c = mi + 1 < q.tiles_n ? mi + 1 : q.tiles_n;
-    if (lt < c) break;
-    lt -= c;
-  }
-  ni = lt;
+  mi = lt / q.tiles_n;
+  ni = lt % q.tiles_n;
 }
 
 __global__ void __launch_bounds__(kThreads) gemm_f32_kernel(const __grid_constant__ F32Params p) {
@@ -171,9 +158,7 @@ __global__ void __launch_bounds__(kThreads) gemm_f32_kernel(const __grid_constan
         if (gj0 + y >= q.N) { v[y] = 0.f; continue; }
         if (p.mode == kGram) v[y] = (sc * sc) * a;
         else if (p.mode == kPoly) v[y] = fmaf(p.cb, C[o], p.cc * a);
-        else if (p.mode == kUpdate) v[y] = sc * fmaf(p.ca, C[o], a);
-        else if (p.mode == kSub) v[y] = C[o] - a;
-        else v[y] = a;
+        else v[y] = sc * fmaf(p.ca, C[o], a);   // kUpdate
       }
       const int64_t o0 = (int64_t)gi * q.ldc + gj0;
       if (vec_d && gj0 + 3 < q.N) {

@@ -62,10 +62,11 @@ struct MatDesc {
   int32_t rec_begin; // reduce: first (||O||^2, <W,O>, ||W||^2) record of this matrix
 };
 
-// Momentum + U + per-block ||U||^2 partials.
+// Momentum + U + ||U||^2 partials, one per warp of every block (kK1PartsPerBlock per block).
+constexpr int kK1PartsPerBlock = 8;
 struct MomentumParams {
   char *ws;
-  double *partials;  // one per block of the launch
+  double *partials;  // kK1PartsPerBlock per block of the launch
   uint32_t *status;
   float beta;
   int32_t nesterov;
@@ -82,8 +83,8 @@ struct NormFinParams {
   float ns_eps;
   int32_t nmat;
   int32_t seg_begin[kMaxMats + 1];  // segment prefix (segments of one matrix are contiguous)
-  int32_t blk_begin[kMaxMats];      // partial index of each matrix's first block
-  int32_t bps[kMaxMats];            // blocks per segment
+  int32_t blk_begin[kMaxMats];      // index of each matrix's first partial record
+  int32_t bps[kMaxMats];            // partial records per segment
 };
 
 // Per-matrix scalars kept in the workspace between the reduce, finalize and apply kernels.
@@ -162,7 +163,7 @@ constexpr int kPwTall = 1;   // X = W^T: X element (r, c) is W element (c, r)
 constexpr int kPwTiled = 4;  // batch b is the T x T tile (b / w_tiles_c, b % w_tiles_c) of W
 constexpr int kPwVec = 8;    // W rows may be read with 16-byte loads
 constexpr int kPartsPerTile = 16;   // partial records per 256 x 256 tile (one per epilogue warp)
-enum GemmMode { kGram = 0, kPoly = 1, kUpdate = 2, kPlain = 3, kSub = 4, kGramF32 = 5 };
+enum GemmMode { kGram = 0, kPoly = 1, kUpdate = 2, kGramF32 = 5 };
 struct GemmParams {
   CUtensorMap tmap;       // 2-SM kernel: the workspace seen as rows of 128 bytes (64 bf16),
                           // 64-row boxes, no swizzle (the data is stored pre-swizzled)
@@ -223,8 +224,6 @@ struct F32Prob {
   int32_t b_trans;         // 1: B element (k, j) at b[j * ldb + k]; 0: at b[k * ldb + j]
   int32_t tiles_n, tile_begin;
   int32_t scale_idx;
-  int32_t lower;           // 1: only the output tiles on and below the diagonal
-  int32_t pad_;
 };
 struct F32Params {
   char *ws;
@@ -244,14 +243,12 @@ struct PackParams {          // row-major bf16 (rows x cols, ld) -> panel layout
   char *ws;
   int32_t n;
 };
-struct CholParams {          // one blocked-Cholesky step (column block k) for a batch of matrices
+struct CholParams {          // the ridge of a batch of layer-input Gram matrices
   char *ws;
   uint32_t *status;
-  int64_t s_off[kMaxMats];   // fp32 row-major S / L (ld = ld[i])
-  int64_t inv_off[kMaxMats]; // fp32 64 x 64 inverse of each diagonal block, block b at +b*64*64
+  int64_t s_off[kMaxMats];   // fp32 row-major S (ld = ld[i], padded size)
   int32_t ld[kMaxMats], d[kMaxMats];
   float ridge_rel;
-  int32_t k;                 // first column of the block
   int32_t n;
 };
 
@@ -261,6 +258,64 @@ struct CholParams {          // one blocked-Cholesky step (column block k) for a
 nshb_status check_matrix(const nshb_matrix &d, const float *V = nullptr, bool need_v = false, bool w_only = false);
 // Records a CUDA error for nshb_last_cuda_error (per calling thread) and clears it.
 void record_cuda_error(cudaError_t e);
+
+// Split-precision (bf16 x 3) products of the Newton-Muon preconditioner (newton_tc.cu):
+// D = A B^T (B K-major), D = A B (B MN-major) or D = C - A B^(T), over 256 x 256 tiles of
+// one M x N region, with A = A_hi + A_lo and B = B_hi + B_lo held as bf16 panel matrices.
+constexpr int kNwBMn = 1;     // B MN-major
+constexpr int kNwLower = 2;   // only the output tiles on and below the diagonal
+constexpr int kMaxNwProb = 200;
+struct NwProb {
+  int64_t a_hi, a_lo, b_hi, b_lo;  // panel matrices of A and B (workspace byte offsets of panel 0)
+  int64_t c32, d32;                // fp32 row-major C / D: byte offset of the region's (0, 0), or -1
+  int64_t dhi, dlo;                // panel matrices of D (hi, lo), or -1
+  int32_t a_ph, b_ph, d_ph;        // panel heights
+  int32_t a_r0, a_k0;              // A region: first row, first k (multiple of 64)
+  int32_t b_r0, b_k0;              // B region: first n (row if K-major, column if MN-major), first k
+  int32_t d_r0, d_c0;              // D region within D's panels
+  int32_t ld32;                    // row stride (elements) of the fp32 C and D
+  int32_t m_valid, n_valid;        // rows / columns of the fp32 D region that exist
+  int32_t mt, nt, kt;              // 256-row tiles, 256-column tiles, 64-deep k panels (even)
+  int32_t flags;                   // kNwBMn | kNwLower
+  int32_t tile_begin;
+};
+struct NwParams {
+  CUtensorMap tmap;                // the workspace as 128-byte rows (see GemmParams)
+  char *ws;
+  uint32_t *status;
+  long long wait_limit;
+  int32_t nprob, total_tiles;
+  NwProb prob[kMaxNwProb];
+};
+
+// fp32 row-major regions -> bf16 hi/lo panel matrices (and optionally an fp32 copy with
+// another leading dimension), zero outside the source region up to the padded extents.
+struct SplitItem {
+  int64_t src32;                   // workspace byte offset of the source's (0, 0)
+  int64_t dst32;                   // fp32 copy's (0, 0), or -1
+  int64_t dhi, dlo;                // panel matrices (panel 0)
+  int32_t src_ld, dst_ld;          // elements
+  int32_t rows, cols;              // source extent
+  int32_t prow, pcol;              // padded extent written (multiples of 64)
+  int32_t d_ph, d_r0, d_c0;        // destination panels: height, region origin
+  int32_t blk_begin;               // first 64 x 64 block of this item in the launch
+};
+struct SplitParams {
+  char *ws;
+  int32_t n, total_blocks;
+  SplitItem item[kMaxMats];
+};
+
+// Cholesky factor and inverse of one 256 x 256 diagonal block per layer input (column
+// block k), written as the bf16 hi/lo panels of a stack of inverses (block k at rows 256 k).
+struct DiagParams {
+  char *ws;
+  uint32_t *status;
+  int32_t n, k;
+  int64_t s32[kMaxMats];           // fp32 S (row-major, ld[i])
+  int64_t dhi[kMaxMats], dlo[kMaxMats];
+  int32_t ld[kMaxMats];            // S row stride = panel height of the inverse stack
+};
 
 // Launchers (defined in the .cu files); each returns cudaGetLastError().
 cudaError_t launch_momentum(const MomentumParams &p, cudaStream_t s);
@@ -281,7 +336,9 @@ cudaError_t encode_ws_tensor_map(CUtensorMap *map, void *ws, size_t bytes);
 cudaError_t launch_gemm_f32(const F32Params &p, cudaStream_t s);
 cudaError_t launch_pack_panels(const PackParams &p, cudaStream_t s);
 cudaError_t launch_ridge(const CholParams &p, cudaStream_t s);
-cudaError_t launch_potrf_block(const CholParams &p, cudaStream_t s);
+cudaError_t launch_newton_gemm(const NwParams &p, int num_sms, cudaStream_t s);
+cudaError_t launch_split(const SplitParams &p, cudaStream_t s);
+cudaError_t launch_potrf_diag(const DiagParams &p, cudaStream_t s);
 
 constexpr size_t kMaxParamBytes = 32764;   // kernel parameter limit (CUDA 12.1+, sm_70+)
 static_assert(sizeof(MomentumParams) <= kMaxParamBytes, "MomentumParams");
@@ -294,5 +351,8 @@ static_assert(sizeof(HmParams) <= kMaxParamBytes, "HmParams");
 static_assert(sizeof(F32Params) <= kMaxParamBytes, "F32Params");
 static_assert(sizeof(PackParams) <= kMaxParamBytes, "PackParams");
 static_assert(sizeof(CholParams) <= kMaxParamBytes, "CholParams");
+static_assert(sizeof(NwParams) <= kMaxParamBytes, "NwParams");
+static_assert(sizeof(SplitParams) <= kMaxParamBytes, "SplitParams");
+static_assert(sizeof(DiagParams) <= kMaxParamBytes, "DiagParams");
 
 }  // namespace nshb

@@ -34,6 +34,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+static_assert(kWarps == kK1PartsPerBlock, "one ||U||^2 partial per warp of a momentum block");
 
 template <typename P>
 __device__ __forceinline__ int find_mat(const P &p, int blk) {
@@ -275,8 +276,7 @@ __device__ __forceinline__ void momentum_load(const MomentumParams &p, const Mat
 // One 64x64 block: momentum update, U into the NS operand storage, ||U||^2 partial.
 template <bool F32>
 __device__ __forceinline__ void momentum_block(const MomentumParams &p, const MatDesc &d, int cblk, int cr0,
-                                               int cc0, const MomIn &in, float (&sT)[2][kBlk][kBlk + 1],
-                                               double (*red)[kWarps], int &nred) {
+                                               int cc0, const MomIn &in, float (&sT)[2][kBlk][kBlk + 1]) {
   const int rq = threadIdx.x >> 3, cq = (threadIdx.x & 7) * 8;
   const bool f32 = F32 && (d.flags & kWF32), vec = d.flags & kVec;
   const bool from_p = F32 && (d.flags & kFromP);
@@ -289,6 +289,9 @@ __device__ __forceinline__ void momentum_block(const MomentumParams &p, const Ma
   const float beta = p.beta, omb = 1.0f - p.beta;
   const bool full = full_block(d, cr0, cc0);
   float acc = 0.f;
+  // Every thread has finished reading the previous block's transpose staging (tr is the
+  // same for the whole CTA, so the barrier is uniform).
+  if (tr && !urow) __syncthreads();
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int i = cr0 + rq + 32 * h, j = cc0 + cq;
@@ -345,11 +348,9 @@ __device__ __forceinline__ void momentum_block(const MomentumParams &p, const Ma
         }
       }
     }
-    const float a1[1] = {acc};
-    double s[1];
-    cta_sum<1>(a1, s, red, nred & 1);
-    ++nred;
-    if (threadIdx.x == 0) p.partials[cblk] = s[0];
+    // one partial per warp (fixed order within the warp), no block-wide barrier
+    const float w = warp_sum(acc);
+    if ((threadIdx.x & 31) == 0) p.partials[(int64_t)kWarps * cblk + (threadIdx.x >> 5)] = (double)w;
   }
 }
 
@@ -361,7 +362,6 @@ __global__ void __launch_bounds__(kThreads, F32 ? 2 : 3) momentum_kernel(const _
   pdl_trigger();
   pdl_wait();
   __shared__ float sT[2][kBlk][kBlk + 1];   // transpose staging (tall matrices): hi, lo
-  __shared__ double red[2][kWarps];
   int blk = blockIdx.x;
   if (blk >= p.total_blocks) return;
   int mi = find_mat(p, blk);
@@ -369,7 +369,6 @@ __global__ void __launch_bounds__(kThreads, F32 ? 2 : 3) momentum_kernel(const _
   block_origin(p.mats[mi], blk - p.mats[mi].blk_begin, r0, c0);
   MomIn nxt;
   momentum_load<F32>(p, p.mats[mi], r0, c0, nxt);
-  int nred = 0;
   for (;;) {
     const MomIn in = nxt;
     const int cblk = blk, cr0 = r0, cc0 = c0;
@@ -382,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, F32 ? 2 : 3) momentum_kernel(const _
       momentum_load<F32>(p, p.mats[nmi], r0, c0, nxt);
       mi = nmi;
     }
-    momentum_block<F32>(p, d, cblk, cr0, cc0, in, sT, red, nred);
+    momentum_block<F32>(p, d, cblk, cr0, cc0, in, sT);
     if (!more) break;
   }
 }

@@ -428,14 +428,18 @@ def test_tile_resident_himuon_wait_limit_reports_timeout(T):
 
 # ---------------------------------------------------------------- Newton-Muon
 def test_bf16_newton_muon_small():
-    """P = U (Z Z^T + lambda I)^-1 through the tensor-core Gram, fp32 blocked Cholesky and
-    block solves, then bf16 NS and Hyperball; against the oracle's plain linear solve."""
+    """P = U (Z Z^T + lambda I)^-1 through the tensor-core Gram, the blocked Cholesky with
+    256-wide diagonal blocks and split-precision products, and the block solves; then bf16
+    NS and Hyperball; against the oracle's plain linear solve.  Layer inputs of 128, 256, 320
+    and 576 rows (one to three diagonal blocks, the last one partly padding), matrices with
+    row counts that are not multiples of 256, wide and tall."""
     from gpu_harness import newton_step
     cfg = wl.CFG_NEWTON_GPT2
     n_tok = 512
-    Zs = [wl.layer_input(cfg, 0, 128, n_tok), wl.layer_input(cfg, 1, 256, n_tok)]
-    shapes = [(192, 128), (128, 256), (320, 256), (64, 128)]
-    zi = [0, 1, 1, 0]
+    Zs = [wl.layer_input(cfg, 0, 128, n_tok), wl.layer_input(cfg, 1, 256, n_tok),
+          wl.layer_input(cfg, 2, 320, n_tok), wl.layer_input(cfg, 3, 576, n_tok)]
+    shapes = [(192, 128), (128, 256), (320, 256), (64, 128), (100, 320), (700, 320), (600, 576)]
+    zi = [0, 1, 1, 0, 2, 2, 3]
     Ws = [wl.init_weight(cfg, 40 + i, r, c, bf16=True).astype(np.float64) for i, (r, c) in enumerate(shapes)]
     Gs = [wl.gradient(cfg, 40 + i, 0, r, c, bf16=True).astype(np.float64) for i, (r, c) in enumerate(shapes)]
     rhos = [o.fro(w) for w in Ws]
