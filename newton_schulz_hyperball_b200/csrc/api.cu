@@ -299,7 +299,7 @@ MatDesc make_desc(const nshb_matrix &d, const MatPlan &m, int idx, int64_t o_off
   r.flags = m.flags;
   if (m.flags & kTiled) r.ph = m.T;
   else if (m.flags & kNsF32) r.ph = (int)m.s;
-  else r.ph = (int)m.Rp;
+  else r.ph = (int)(m.tall ? m.Sp : m.Rp);   // bf16 X = U as stored: m rows, padded
   if (k1) {
     r.pr = m.pr;
     r.pc = m.pc;
@@ -614,9 +614,12 @@ nshb_status run_ns(const nshb_matrix *mats, const Plan &pl, const nshb_params *p
               R = m.Rp; S = m.Sp; batch = 1;
             }
             q.batch = batch;
-            q.ph = (int)R;
             // X, A and B of a tile share one stride (T x T bf16); a whole matrix is one batch
             q.bs = pl.tiled ? (int64_t)m.T * m.T * 2 : 0;
+            // A tall matrix keeps X = U (S rows, R columns): its Gram X^T X reads X MN-major on
+            // both sides, its update X B reads X and B K-major.  Everything else is R rows.
+            const bool tall = !pl.tiled && m.tall;
+            const int64_t xph = tall ? S : R;
             q.w = nullptr;
             if (last_update && m.fused) {
               const nshb_matrix &d = mats[i];
@@ -625,12 +628,11 @@ nshb_status run_ns(const nshb_matrix *mats, const Plan &pl, const nshb_params *p
               q.w_m = (int)m.m;
               q.w_n = (int)m.n;
               q.w_ld = (int)m.ld;
-              q.w_flags = (m.tall ? kPwTall : 0) | (pl.tiled ? kPwTiled : 0) | (wvec ? kPwVec : 0);
+              q.w_flags = (pl.tiled ? kPwTiled : 0) | (wvec ? kPwVec : 0);
               q.w_tiles_c = m.tiles_c;
               q.part_begin = m.rec_begin;
               gp.partials = reinterpret_cast<double *>(ws + pl.wpart_off);
             }
-            q.mt = (int)(R / 256);
             q.c_lo = -1;
             q.d_lo = -1;
             if (mode == kUpdate && it < pl.comp) {
@@ -639,13 +641,26 @@ nshb_status run_ns(const nshb_matrix *mats, const Plan &pl, const nshb_params *p
             }
             if (mode == kGram) {
               q.a_off = xin; q.b_off = xin; q.c_off = m.a; q.d_off = m.a;
-              q.nt = (int)(R / pl.bn); q.kt = (int)(S / 64);
+              q.a_ph = q.b_ph = (int)xph; q.d_ph = (int)R;
+              q.major = tall ? (kAMn | kBMn) : 0;
+              q.mt = (int)(R / 256); q.nt = (int)(R / pl.bn); q.kt = (int)(S / 64);
             } else if (mode == kPoly) {
               q.a_off = m.a; q.b_off = m.a; q.c_off = m.a; q.d_off = m.b;
-              q.nt = (int)(R / pl.bn); q.kt = (int)(R / 64);
-            } else {
+              q.a_ph = q.b_ph = q.d_ph = (int)R;
+              q.major = 0;
+              q.mt = (int)(R / 256); q.nt = (int)(R / pl.bn); q.kt = (int)(R / 64);
+            } else if (!tall) {
+              // X' = s (a X + B X): A = B (K-major), B operand = X (MN-major)
               q.a_off = m.b; q.b_off = xin; q.c_off = xin; q.d_off = xout;
-              q.nt = (int)(S / pl.bn); q.kt = (int)(R / 64);
+              q.a_ph = q.b_ph = q.d_ph = (int)R;
+              q.major = kBMn;
+              q.mt = (int)(R / 256); q.nt = (int)(S / pl.bn); q.kt = (int)(R / 64);
+            } else {
+              // X' = s (a X + X B): A = X (K-major, S rows), B operand = B (symmetric, K-major)
+              q.a_off = xin; q.b_off = m.b; q.c_off = xin; q.d_off = xout;
+              q.a_ph = q.d_ph = (int)S; q.b_ph = (int)R;
+              q.major = 0;
+              q.mt = (int)(S / 256); q.nt = (int)(R / pl.bn); q.kt = (int)(R / 64);
             }
             q.tiles_per_batch = gemm_tiles(mode, q.mt, q.nt, 256, pl.bn);
             q.scale_idx = (it == 0 && mode != kPoly) ? m.seg_begin : -1;
@@ -849,7 +864,8 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
       q.a_off = q.b_off = z.zp;
       q.c_off = q.d_off = z.s;
       q.c_lo = q.d_lo = -1;
-      q.ph = (int)z.Dp;
+      q.a_ph = q.b_ph = q.d_ph = (int)z.Dp;
+      q.major = 0;
       q.bs = 0;
       q.w = nullptr;
       q.mt = (int)(z.Dp / 256);

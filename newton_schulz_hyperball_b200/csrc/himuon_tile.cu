@@ -162,11 +162,14 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sXown = smem_u32(smem), sXcol = sXown + kHalf, sA = sXcol + kHalf;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 3 * kHalf);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 12);   // after the nine barriers
   const uint32_t bar_base = smem_u32(bars);
   const uint32_t xfull = bar_base, xfree = bar_base + 8, mmadone = bar_base + 16;
-  const uint32_t xready = bar_base + 24, opnd = bar_base + 32;   // used in the leader only
-  const uint32_t stallbar = bar_base + 40;                        // test stall (leader only)
+  const uint32_t xready = bar_base + 24;                          // used in the leader only
+  const uint32_t stallbar = bar_base + 32;                        // test stall (leader only)
+  // pready[p]: the epilogues have written 64-column panel p of the next phase's operand
+  // (in the leader only; four warps of each CTA write a panel)
+  auto pready = [&](int pnl) { return bar_base + 40 + 8u * pnl; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cta_rank();
@@ -177,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
     mbar_init(xfree, 1);
     mbar_init(mmadone, 1);
     mbar_init(xready, 2);                 // both producers
-    mbar_init(opnd, 2 * kEpiWarps);       // every epilogue warp of both CTAs
+    for (int pnl = 0; pnl < 4; ++pnl) mbar_init(pready(pnl), kEpiWarps);   // 4 warps x 2 CTAs
     mbar_init(stallbar, 1);
     mbar_fence_init();
   }
@@ -227,16 +230,25 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ------------------------------------------------------------ MMA issuer (leader)
-      const uint32_t idesc_k = idesc_bf16(2 * 128, T, 0), idesc_mn = idesc_bf16(2 * 128, T, 1);
-      uint32_t ph_r = 0, ph_o = 0;
+      const uint32_t idesc_k = idesc_bf16(2 * 128, T, 0, 0), idesc_mn = idesc_bf16(2 * 128, T, 0, 1);
+      // A phase's MMAs go panel by panel (64 k columns: 4 MMAs) in the order the epilogue
+      // warps finish them: warps of column half 0 write panels 0 then 1, those of half 1
+      // panels 2 then 3.  Accumulators alternate between TMEM columns [0, 256) and
+      // [256, 512) from phase to phase, so a phase never writes what the epilogue of the
+      // previous phase is still reading.
+      constexpr int kOrder[4] = {0, 2, 1, 3};
+      uint32_t ph_r = 0, ph_p = 0;
       bool ok = true;
-      auto wait_opnd = [&]() {
-        if (!mbar_wait(opnd, ph_o, limit)) {
+      auto wait_panel = [&](int pnl) {
+        if (!mbar_wait(pready(pnl), ph_p, limit)) {
           set_status(p.status, kTimeoutBit);
           ok = false;
         }
-        ph_o ^= 1u;
         tc_fence_after();
+      };
+      auto wait_all_panels = [&]() {
+        for (int pnl = 0; ok && pnl < 4; ++pnl) wait_panel(pnl);
+        ph_p ^= 1u;
       };
       for (int tile = cid, tl = 0; ok && tile < p.total_tiles; tile += ncl, ++tl) {
         if (!mbar_wait(xready, ph_r, limit)) {
@@ -246,16 +258,23 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
         ph_r ^= 1u;
         tc_fence_after();
         for (int it = 0; ok && it < K; ++it) {
-          if (it > 0) {
-            wait_opnd();   // epilogue 3 of the previous iteration wrote X'
+          const uint32_t dg = tmem_base + (uint32_t)(((3 * it) & 1) * T);
+          const uint32_t dq = tmem_base + (uint32_t)(((3 * it + 1) & 1) * T);
+          const uint32_t du = tmem_base + (uint32_t)(((3 * it + 2) & 1) * T);
+          // Gram: A = X X^T (X' of the previous epilogue 3, or X0 from the producer)
+          for (int o = 0; ok && o < 4; ++o) {
+            const int pnl = kOrder[o];
+            if (it > 0) wait_panel(pnl);
             if (!ok) break;
-          }
 #pragma unroll
-          for (int k = 0; k < T / 16; ++k) {   // Gram: A = X X^T
-            const uint32_t kofs = (uint32_t)(k >> 2) * kPanel128 + 32u * (k & 3);
-            const uint64_t d = smem_desc_sw128(sXown + kofs, 16, 1024);
-            tc_mma2(tmem_base, d, d, idesc_k, k != 0);
+            for (int k = 4 * pnl; k < 4 * pnl + 4; ++k) {
+              const uint32_t kofs = (uint32_t)(k >> 2) * kPanel128 + 32u * (k & 3);
+              const uint64_t d = smem_desc_sw128(sXown + kofs, 16, 1024);
+              tc_mma2(dg, d, d, idesc_k, k != 0);
+            }
           }
+          if (it > 0) ph_p ^= 1u;
+          if (!ok) break;
           if (p.test_stall && tl == 0 && it == 0) {
             // Test stall: the epilogues never hear of this accumulator, so their bounded
             // wait runs out.  The MMAs still complete (on a barrier of the leader only)
@@ -265,28 +284,41 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
           } else {
             tc_commit2_mc(mmadone, 0x3);
           }
-          wait_opnd();     // epilogue 1 wrote A to sA
-          if (!ok) break;
+          // A^2 = A A^T (A symmetric), panel by panel as epilogue 1 writes A to sA
+          for (int o = 0; ok && o < 4; ++o) {
+            const int pnl = kOrder[o];
+            wait_panel(pnl);
+            if (!ok) break;
 #pragma unroll
-          for (int k = 0; k < T / 16; ++k) {   // A^2 = A A^T (A symmetric)
-            const uint32_t kofs = (uint32_t)(k >> 2) * kPanel128 + 32u * (k & 3);
-            const uint64_t d = smem_desc_sw128(sA + kofs, 16, 1024);
-            tc_mma2(tmem_base + T, d, d, idesc_k, k != 0);
+            for (int k = 4 * pnl; k < 4 * pnl + 4; ++k) {
+              const uint32_t kofs = (uint32_t)(k >> 2) * kPanel128 + 32u * (k & 3);
+              const uint64_t d = smem_desc_sw128(sA + kofs, 16, 1024);
+              tc_mma2(dq, d, d, idesc_k, k != 0);
+            }
           }
+          ph_p ^= 1u;
+          if (!ok) break;
           tc_commit2_mc(mmadone, 0x3);
-          wait_opnd();     // epilogue 2 wrote B to sA
-          if (!ok) break;
+          // B X: B K-major (panels of sA as epilogue 2 writes them), X MN-major (16 rows of
+          // sXcol per step)
+          for (int o = 0; ok && o < 4; ++o) {
+            const int pnl = kOrder[o];
+            wait_panel(pnl);
+            if (!ok) break;
 #pragma unroll
-          for (int k = 0; k < T / 16; ++k) {   // B X: B K-major, X MN-major (16 rows per step)
-            const uint32_t kofs = (uint32_t)(k >> 2) * kPanel128 + 32u * (k & 3);
-            const uint64_t ad = smem_desc_sw128(sA + kofs, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(sXcol + 2048u * k, kPanel256, 1024);
-            tc_mma2(tmem_base, ad, bd, idesc_mn, k != 0);
+            for (int k = 4 * pnl; k < 4 * pnl + 4; ++k) {
+              const uint32_t kofs = (uint32_t)(k >> 2) * kPanel128 + 32u * (k & 3);
+              const uint64_t ad = smem_desc_sw128(sA + kofs, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(sXcol + 2048u * k, kPanel256, 1024);
+              tc_mma2(du, ad, bd, idesc_mn, k != 0);
+            }
           }
+          ph_p ^= 1u;
+          if (!ok) break;
           tc_commit2_mc(mmadone, 0x3);
         }
         if (!ok) break;
-        wait_opnd();       // the tile's last epilogue is done with sXown and the TMEM
+        wait_all_panels();   // the tile's last epilogue is done with sXown and the TMEM
         if (!ok) break;
         remote_arrive(mapa(xfree, 0));
         remote_arrive(mapa(xfree, 1));
@@ -311,11 +343,13 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
       ph_m ^= 1u;
       tc_fence_after();
     };
-    auto report = [&](bool partner_smem) {
+    // This warp's rows of panel pnl are written (shared memory of this CTA, or also the
+    // partner's): the MMA issuer may read the panel.
+    auto report = [&](int pnl, bool partner_smem) {
       if (partner_smem) fence_proxy_async_cluster(); else fence_proxy_async_cta();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) remote_arrive(mapa(opnd, 0));
+      if (lane == 0) remote_arrive(mapa(pready(pnl), 0));
     };
     for (int tile = cid; ok && tile < p.total_tiles; tile += ncl) {
       const HmProb &q = p.prob[find_prob(p, tile)];
@@ -335,6 +369,9 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
       for (int it = 0; ok && it < K; ++it) {
         const float ca = p.coef[it][0], cb = p.coef[it][1], cc = p.coef[it][2];
         const float s2 = it == 0 ? s * s : 1.0f, ks = it == 0 ? s : 1.0f;
+        // TMEM columns of this iteration's three accumulators (they alternate by phase)
+        const uint32_t rg = (uint32_t)(((3 * it) & 1) * T), rq0 = (uint32_t)(((3 * it + 1) & 1) * T);
+        const uint32_t ru = (uint32_t)(((3 * it + 2) & 1) * T);
         if (wp && it + 1 == K) w_prefetch(q, wr, wc, 128);
         // ---- epilogue 1: A -> sA (bf16)
         wait_mma();
@@ -343,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
         for (int ch = 0; ch < 4; ++ch) {
           const int j0 = 128 * half + 32 * ch;
           uint32_t r[32];
-          tmem_ld32(tmem_base + (uint32_t)j0 + lane_off, r);
+          tmem_ld32(tmem_base + rg + (uint32_t)j0 + lane_off, r);
           tmem_ld_wait();
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -353,17 +390,19 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
               w[e] = pack_bf16(s2 * __uint_as_float(r[8 * c + 2 * e]), s2 * __uint_as_float(r[8 * c + 2 * e + 1]));
             st_shared_v4(sA + half_chunk(rl, j0 + 8 * c), w);
           }
+          if (ch & 1) report(2 * half + (ch >> 1), false);
         }
-        report(false);
-        // ---- epilogue 2: B = b A + c A^2 -> sA (bf16), A and A^2 from TMEM in fp32
+        // ---- epilogue 2: B = b A + c A^2 -> sA (bf16); A is the bf16 copy this thread wrote
+        // to sA (the TMEM copy is being overwritten by the update), A^2 from TMEM in fp32
         wait_mma();
         if (!ok) break;
 #pragma unroll 1
         for (int ch = 0; ch < 4; ++ch) {
           const int j0 = 128 * half + 32 * ch;
-          uint32_t ra[32], rq[32];
-          tmem_ld32(tmem_base + (uint32_t)j0 + lane_off, ra);
-          tmem_ld32(tmem_base + (uint32_t)(T + j0) + lane_off, rq);
+          uint32_t rq[32], aw[16];
+          tmem_ld32(tmem_base + rq0 + (uint32_t)j0 + lane_off, rq);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) ld_shared_v4(sA + half_chunk(rl, j0 + 8 * c), aw + 4 * c);
           tmem_ld_wait();
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -371,13 +410,13 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int i0 = 8 * c + 2 * e;
-              w[e] = pack_bf16(fmaf(cb * s2, __uint_as_float(ra[i0]), cc * __uint_as_float(rq[i0])),
-                               fmaf(cb * s2, __uint_as_float(ra[i0 + 1]), cc * __uint_as_float(rq[i0 + 1])));
+              w[e] = pack_bf16(fmaf(cb, bf16lo(aw[4 * c + e]), cc * __uint_as_float(rq[i0])),
+                               fmaf(cb, bf16hi(aw[4 * c + e]), cc * __uint_as_float(rq[i0 + 1])));
             }
             st_shared_v4(sA + half_chunk(rl, j0 + 8 * c), w);
           }
+          if (ch & 1) report(2 * half + (ch >> 1), false);
         }
-        report(false);
         // ---- epilogue 3: X' = s (a X + B X)
         const bool last = it + 1 == K;
         const bool wlast = wp && last;
@@ -394,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
           uint32_t wn[16];
           if (wlast && ch < 3) w_load(q, wr, wc + 32 * (ch + 1), wn);
           uint32_t r[32];
-          tmem_ld32(tmem_base + (uint32_t)j0 + lane_off, r);
+          tmem_ld32(tmem_base + ru + (uint32_t)j0 + lane_off, r);
           uint32_t xw[16], lw[16];
 #pragma unroll
           for (int c = 0; c < 4; ++c) ld_shared_v4(sXown + half_chunk(rl, j0 + 8 * c), xw + 4 * c);
@@ -452,8 +491,8 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
               }
             }
           }
+          if (ch & 1) report(2 * half + (ch >> 1), !last);   // (the partner's sXcol was written)
         }
-        report(!last);   // the partner's sXcol was written
       }
       if (ok && wp)
         w_record(p.partials, (int64_t)q.part_begin + (int64_t)t * (2 * kEpiWarps) + rank * kEpiWarps + (warp - 2),
@@ -538,7 +577,7 @@ __global__ void __launch_bounds__(kThreads1, kCtasPerSm1) himuon_tile128_kernel(
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc_k = idesc_bf16(T1, T1, 0), idesc_mn = idesc_bf16(T1, T1, 1);
+      const uint32_t idesc_k = idesc_bf16(T1, T1, 0, 0), idesc_mn = idesc_bf16(T1, T1, 0, 1);
       uint32_t ph_x = 0, ph_o = 0;
       bool ok = true;
       auto wait_opnd = [&]() {

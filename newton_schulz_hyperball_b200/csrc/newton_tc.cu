@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1) newton_gemm_kernel(const __grid_c
         const NwTile t = nw_decode(p, tile);
         const NwProb &q = p.prob[t.prob];
         const bool bmn = q.flags & kNwBMn;
-        const uint32_t idesc = idesc_bf16(BM, BN, bmn ? 1 : 0);
+        const uint32_t idesc = idesc_bf16(BM, BN, 0, bmn ? 1 : 0);
         const int buf = tl & 1;
         const uint32_t tph = (uint32_t)(tl >> 1) & 1u;
         if (!mbar_wait(tempty_bar(buf), tph ^ 1u, limit)) {

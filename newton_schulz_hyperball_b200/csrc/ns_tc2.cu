@@ -151,19 +151,25 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
             mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
             last_parity[stage] = (int)phase;
           }
-          // K-major A: rows am .. am+127 of k panels kb and kb+1 (16 KB each)
-          const int64_t ya = a_row + (int64_t)kb * q.ph + am;
-          tma_load_2sm(sA, &p.tmap, 0, (int)ya, fb);
-          tma_load_2sm(sA + SLICE_BYTES, &p.tmap, 0, (int)(ya + q.ph), fb);
-          if (p.mode != kUpdate) {
-            const int64_t yb = b_row + (int64_t)kb * q.ph + bn;
-            tma_load_2sm(sB, &p.tmap, 0, (int)yb, fb);
-            tma_load_2sm(sB + SLICE_BYTES, &p.tmap, 0, (int)(yb + q.ph), fb);
+          // K-major: rows am .. am+127 of k panels kb and kb+1 (16 KB each); MN-major: the 128
+          // rows (columns of the stored matrix) are two 64-column panels, k rows kb*64 .. +127.
+          if (!(q.major & kAMn)) {
+            const int64_t ya = a_row + (int64_t)kb * q.a_ph + am;
+            tma_load_2sm(sA, &p.tmap, 0, (int)ya, fb);
+            tma_load_2sm(sA + SLICE_BYTES, &p.tmap, 0, (int)(ya + q.a_ph), fb);
           } else {
-            // MN-major: the 128 columns are two 64-column panels, k rows kb*64 .. +127
-            const int64_t y0 = b_row + (int64_t)(bn >> 6) * q.ph + (int64_t)kb * 64;
+            const int64_t y0 = a_row + (int64_t)(am >> 6) * q.a_ph + (int64_t)kb * 64;
+            tma_load_2sm(sA, &p.tmap, 0, (int)y0, fb);
+            tma_load_2sm(sA + SLICE_BYTES, &p.tmap, 0, (int)(y0 + q.a_ph), fb);
+          }
+          if (!(q.major & kBMn)) {
+            const int64_t yb = b_row + (int64_t)kb * q.b_ph + bn;
+            tma_load_2sm(sB, &p.tmap, 0, (int)yb, fb);
+            tma_load_2sm(sB + SLICE_BYTES, &p.tmap, 0, (int)(yb + q.b_ph), fb);
+          } else {
+            const int64_t y0 = b_row + (int64_t)(bn >> 6) * q.b_ph + (int64_t)kb * 64;
             tma_load_2sm(sB, &p.tmap, 0, (int)y0, fb);
-            tma_load_2sm(sB + SLICE_BYTES, &p.tmap, 0, (int)(y0 + q.ph), fb);
+            tma_load_2sm(sB + SLICE_BYTES, &p.tmap, 0, (int)(y0 + q.b_ph), fb);
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -180,7 +186,6 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ------------------------------------------------------------ MMA issuer (leader)
-      const uint32_t idesc = idesc_bf16(BM, BN, p.mode == kUpdate ? 1 : 0);
       int stage = 0;
       uint32_t phase = 0;
       int tl = 0;
@@ -188,6 +193,8 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
       for (int tile = cid; ok && tile < p.total_tiles; tile += ncl, ++tl) {
         const Tile t = decode2(p, tile);
         const GemmProb &q = p.prob[t.prob];
+        const bool amn = q.major & kAMn, bmn = q.major & kBMn;
+        const uint32_t idesc = idesc_bf16(BM, BN, amn ? 1 : 0, bmn ? 1 : 0);
         const int buf = tl & 1;
         const uint32_t tph = (uint32_t)(tl >> 1) & 1u;
         if (!mbar_wait(tempty_bar(buf), tph ^ 1u, limit)) {
@@ -209,9 +216,10 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
             // K-major: panel k/4, 32-byte step k%4 inside the 128-byte swizzled rows.
             // MN-major: 16 k rows (2 KB) per step; the two 64-column chunks are 16 KB apart.
             const uint32_t kofs = (uint32_t)(k >> 2) * SLICE_BYTES + 32u * (k & 3);
-            const uint64_t ad = smem_desc_sw128(sA + kofs, 16, 1024);
-            const uint64_t bd = (p.mode == kUpdate) ? smem_desc_sw128(sB + 2048u * k, SLICE_BYTES, 1024)
-                                                    : smem_desc_sw128(sB + kofs, 16, 1024);
+            const uint64_t ad = amn ? smem_desc_sw128(sA + 2048u * k, SLICE_BYTES, 1024)
+                                    : smem_desc_sw128(sA + kofs, 16, 1024);
+            const uint64_t bd = bmn ? smem_desc_sw128(sB + 2048u * k, SLICE_BYTES, 1024)
+                                    : smem_desc_sw128(sB + kofs, 16, 1024);
             tc_mma2(d_tmem, ad, bd, idesc, (kb | k) != 0);
           }
           tc_commit2_mc(empty_bar(stage), 0x3);
@@ -248,30 +256,19 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
       const int ra = (int)(i >> 6);
       const int cc_end = (half + 1) * NCH;
       // Hyperball partials of this problem: the caller's W next to O (X coordinates (i, c)
-      // are W's (i, c), or (c, i) for a matrix whose NS ran on the transpose, offset by the
-      // tile origin for a Hierarchical-Muon tile).
+      // are W's (i, c), offset by the tile origin for a Hierarchical-Muon tile).
       const bool wp = fuse && q.w != nullptr;
-      const bool wtall = wp && (q.w_flags & kPwTall);
       int64_t wr0 = 0, wc0 = 0;
       if (wp && (q.w_flags & kPwTiled)) {
-        wr0 = (int64_t)(t.batch / q.w_tiles_c) * q.ph;
-        wc0 = (int64_t)(t.batch % q.w_tiles_c) * q.ph;
+        wr0 = (int64_t)(t.batch / q.w_tiles_c) * q.d_ph;
+        wc0 = (int64_t)(t.batch % q.w_tiles_c) * q.d_ph;
       }
       // bf16 W of columns t.n0 + 32 cc .. +31 as pairs in logical order, zero outside W (the
       // epilogue reads bf16 weights only; fp32 weights take the reduce pass).
       auto load_w = [&](int cc, uint32_t (&wv)[16]) {
         const int64_t xc0 = t.n0 + cc * 32;
         const unsigned short *w16 = static_cast<const unsigned short *>(q.w);
-        if (wtall) {
-          const bool in = i < q.w_n;
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int64_t r0 = xc0 + 2 * e;
-            const uint32_t lo = (in && r0 < q.w_m) ? (uint32_t)w16[r0 * q.w_ld + i] : 0u;
-            const uint32_t hi = (in && r0 + 1 < q.w_m) ? (uint32_t)w16[(r0 + 1) * q.w_ld + i] : 0u;
-            wv[e] = lo | (hi << 16);
-          }
-        } else {
+        {
           const int64_t wr = wr0 + i, wc = wc0 + xc0;
           if (wr < q.w_m && wc + 31 < q.w_n && (q.w_flags & kPwVec)) {
             const uint4 *src = reinterpret_cast<const uint4 *>(w16 + wr * q.w_ld + wc);
@@ -299,18 +296,8 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
         const int esz = 2;
         const char *wb = static_cast<const char *>(q.w);
         for (int c = half * NCH; c < cc_end; ++c) {
-          const int64_t xc0 = t.n0 + c * 32;
-          if (wtall) {
-            // the warp's lanes cover 32 consecutive columns of each W row: lane l pulls row xc0 + l
-            const int64_t r = xc0 + lane, c0w = i - lane;
-            if (r < q.w_m && c0w < q.w_n)
-              asm volatile("prefetch.global.L2 [%0];" ::"l"(wb + (r * q.w_ld + c0w) * esz));
-          } else {
-            const int64_t wr = wr0 + i, wc = wc0 + xc0;
-            if (wr < q.w_m && wc < q.w_n) {
-              asm volatile("prefetch.global.L2 [%0];" ::"l"(wb + (wr * q.w_ld + wc) * esz));
-            }
-          }
+          const int64_t wr = wr0 + i, wc = wc0 + t.n0 + c * 32;
+          if (wr < q.w_m && wc < q.w_n) asm volatile("prefetch.global.L2 [%0];" ::"l"(wb + (wr * q.w_ld + wc) * esz));
         }
       };
       auto live = [&](int cc) { return cc < cc_end && !(sym && ((t.n0 + cc * 32) >> 6) > ra); };
@@ -320,7 +307,7 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
       auto load_c = [&](int cc, uint32_t (&h)[16], uint32_t (&l)[16]) {
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
-          const size_t off = panel_pair_off(i, t.n0 + cc * 32 + 16 * k, q.ph);
+          const size_t off = panel_pair_off(i, t.n0 + cc * 32 + 16 * k, q.d_ph);
           uint32_t w[8];
           ld_global_256(cbase + off, w);
           unswizzle_pair(w, odd, h + 8 * k);
@@ -356,7 +343,7 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
             uint32_t w[8];
-            ld_global_256(clo + panel_pair_off(i, col0 + 16 * k, q.ph), w);
+            ld_global_256(clo + panel_pair_off(i, col0 + 16 * k, q.d_ph), w);
             unswizzle_pair(w, odd, cl + 8 * k);
           }
         }
@@ -365,7 +352,7 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
         tmem_ld_wait();
         float v[32];
         if (p.mode == kGramF32) {
-          float *drow = reinterpret_cast<float *>(dbase) + i * q.ph;
+          float *drow = reinterpret_cast<float *>(dbase) + i * q.d_ph;
 #pragma unroll
           for (int g = 0; g < 8; ++g)
             *reinterpret_cast<float4 *>(drow + col0 + 4 * g) =
@@ -374,7 +361,7 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
           if (ca < ra) {
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              reinterpret_cast<float *>(dbase)[(int64_t)(col0 + e) * q.ph + i] = __uint_as_float(r[e]);
+              reinterpret_cast<float *>(dbase)[(int64_t)(col0 + e) * q.d_ph + i] = __uint_as_float(r[e]);
           }
           continue;
         }
@@ -413,7 +400,7 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
               ppi = fmaf(w0, w0, fmaf(w1, w1, ppi));
             }
           }
-          const size_t off = panel_pair_off(i, col0 + 16 * k, q.ph);
+          const size_t off = panel_pair_off(i, col0 + 16 * k, q.d_ph);
           unswizzle_pair(o, odd, w);              // the same swap puts logical order back
           st_global_256(dbase + off, w);
           if (dlo) {
@@ -431,7 +418,7 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             __nv_bfloat16 h = __float2bfloat16_rn(v[e]);
-            *reinterpret_cast<__nv_bfloat16 *>(dbase + panel_chunk_off(col0 + e, ib, q.ph) + 2 * ie) = h;
+            *reinterpret_cast<__nv_bfloat16 *>(dbase + panel_chunk_off(col0 + e, ib, q.d_ph) + 2 * ie) = h;
           }
         }
         if (wp) {

@@ -32,7 +32,8 @@ constexpr int kMaxProb = 224;
 constexpr int kBlk = 64;        // streaming kernels work on 64 x 64 blocks
 
 // Matrix flags.
-constexpr int kTall = 1;        // rows > cols: the NS works on U^T (wide side)
+constexpr int kTall = 1;        // rows > cols: the fp32 chain works on U^T (the wide side); the
+                                // bf16 chain keeps X = U and takes the right Gram X^T X
 constexpr int kVec = 2;         // 16-byte vector access is legal for W/G/M rows
 constexpr int kWF32 = 4;        // W and G are fp32 (else bf16)
 constexpr int kTiled = 8;       // Hierarchical Muon: X is a grid of T x T tiles
@@ -142,12 +143,18 @@ struct AdamParams {
 
 // One bf16 GEMM problem of a Newton-Schulz phase (possibly a batch of equal problems).
 // Operands live in the workspace in the panel layout (see panel_chunk_off); every operand
-// of a problem has the same panel height and batch stride.
+// of a problem has the same batch stride.  An operand is K-major (its rows are the M or N
+// index, k runs along the panel rows) or MN-major (M or N runs along the panel rows, k down
+// the rows), which lets the chain run on a tall matrix as stored: its Gram X^T X takes both
+// operands MN-major, its update X B both K-major.
+constexpr int kAMn = 1;   // GemmProb::major: A MN-major
+constexpr int kBMn = 2;   // B MN-major
 struct GemmProb {
   int64_t a_off, b_off, c_off, d_off;  // byte offsets of batch 0
   int64_t c_lo, d_lo;                  // kUpdate: bf16 low parts of C (read) / D (written), or -1
   int64_t bs;                          // byte stride between batches (every operand)
-  int32_t ph;                          // panel height (padded rows) of every operand
+  int32_t a_ph, b_ph, d_ph;            // panel heights (padded rows) of A, B and C / D
+  int32_t major;                       // kAMn | kBMn
   int32_t mt, nt, kt;                  // 256-row tiles, BN-column tiles, 64-deep k blocks
   int32_t batch, tiles_per_batch, tile_begin;
   int32_t scale_idx;                   // scale of batch 0 in GemmParams::scales, or -1
@@ -155,11 +162,10 @@ struct GemmProb {
   // weight W (rows w_m x w_n, leading dimension w_ld) read in the epilogue next to O.
   const void *w;                       // NULL: no partials for this problem
   int32_t w_m, w_n, w_ld;
-  int32_t w_flags;                     // kPwTall | kPwTiled | kPwVec (W is bf16)
+  int32_t w_flags;                     // kPwTiled | kPwVec (W is bf16; X has W's orientation)
   int32_t w_tiles_c;                   // kPwTiled: tiles per tile-row (batch b = tile (b / tc, b % tc))
   int32_t part_begin;                  // first partial record of this problem (16 per tile)
 };
-constexpr int kPwTall = 1;   // X = W^T: X element (r, c) is W element (c, r)
 constexpr int kPwTiled = 4;  // batch b is the T x T tile (b / w_tiles_c, b % w_tiles_c) of W
 constexpr int kPwVec = 8;    // W rows may be read with 16-byte loads
 constexpr int kPartsPerTile = 16;   // partial records per 256 x 256 tile (one per epilogue warp)

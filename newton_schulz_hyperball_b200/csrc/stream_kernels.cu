@@ -283,7 +283,7 @@ __device__ __forceinline__ void momentum_block(const MomentumParams &p, const Ma
   const bool urow = F32 && (d.flags & kURow);
   const bool round_bf16 = !F32 || !(d.flags & (kNsF32 | kURow));
   const bool lo_part = round_bf16 && d.xlo_off >= 0;
-  const bool tr = (d.flags & kTall) && !(d.flags & kTiled);
+  const bool tr = F32 && (d.flags & kTall) && (d.flags & kNsF32);   // the fp32 chain takes U^T
   char *xbase = p.ws + d.x_off;
   char *lbase = lo_part ? p.ws + d.xlo_off : nullptr;
   const float beta = p.beta, omb = 1.0f - p.beta;
@@ -417,13 +417,14 @@ struct WoIn {
   Raw8 w[2], o[2];
 };
 
-__device__ __forceinline__ bool o_transposed(const MatDesc &d) { return (d.flags & kTall) && !(d.flags & kTiled); }
+// Only the fp32 chain runs on the transpose of a tall matrix; the bf16 chain keeps U's orientation.
+__device__ __forceinline__ bool o_transposed(const MatDesc &d) { return (d.flags & kTall) && (d.flags & kNsF32); }
 
 template <bool F32>
 __device__ __forceinline__ void wo_load(const ApplyParams &p, const MatDesc &d, int r0, int c0, bool want_o,
                                         WoIn &in) {
   const int rq = threadIdx.x >> 3, cq = (threadIdx.x & 7) * 8;
-  const bool tr = o_transposed(d);
+  const bool tr = F32 && o_transposed(d);
   const char *xbase = p.ws + d.o_off;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
@@ -445,7 +446,7 @@ __device__ __forceinline__ void wo_values(const MatDesc &d, int r0, int c0, cons
   const bool of32 = F32 && (d.flags & kNsF32);
 #pragma unroll
   for (int h = 0; h < 2; ++h) raw_cvt8(in.w[h], F32 && (d.flags & kWF32), w[h]);
-  if (o_transposed(d)) {
+  if (F32 && o_transposed(d)) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       float v[8];
