@@ -48,6 +48,9 @@ E2E_PIPELINE = "H2D of step k+1 on a second stream during step k (2 device buffe
 # says what was captured.
 CSRC = os.path.join(ROOT, "newton_schulz_hyperball_b200", "csrc")
 TRAFFIC = {
+    "gemm_qwen3": {"source": "ns_tc2.cu", "sha256_prefix": "74854940da1bdbdc", "bytes_per_launch": 5284000000,
+                   "case": "4 of the 28 Qwen3-style layers (28 matrices), one step's 15 launches: 11.32 GB "
+                           "DRAM read + write, 0.755 GB per launch, x7 for the 28 identical layers"},
     "gemm_gpt2": {"source": "ns_tc2.cu", "sha256_prefix": "3b2c50016d8520e6", "bytes_per_launch": 372400725,
                   "case": "GPT-2-small set, 15 launches of one step averaged"},
     "adam_gpt2": {"source": "stream_kernels.cu", "sha256_prefix": "705031530c8503d1",
@@ -793,7 +796,9 @@ def report(args, w: Workload, r, world, cpu):
             kinds, kname = ("gram", "poly", "update"), "gemm_tc2_kernel (NS Gram / polynomial / update, CTA pairs)"
         g_ms, g_n = kms(*kinds), klaunch(*kinds)
         tf = flops / (g_ms * 1e-3) / 1e12 if g_ms > 0 else None
-        traffic = traffic_for("gemm_gpt2") if (w.key == "gpt2" and not args.layers) else None
+        traffic = None
+        if not args.layers and w.key in ("gpt2", "qwen3", "qwen3-brake"):
+            traffic = traffic_for("gemm_gpt2" if w.key == "gpt2" else "gemm_qwen3")
         line["ns_tflops"] = None if tf is None else round(tf, 1)
         line["ns_frac_of_bf16_peak"] = None if tf is None else round(tf / peak_tf, 4)
         if w.step != "himuon" and g_ms > 0:

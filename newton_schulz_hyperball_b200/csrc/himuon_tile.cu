@@ -373,6 +373,13 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
         const uint32_t rg = (uint32_t)(((3 * it) & 1) * T), rq0 = (uint32_t)(((3 * it + 1) & 1) * T);
         const uint32_t ru = (uint32_t)(((3 * it + 2) & 1) * T);
         if (wp && it + 1 == K) w_prefetch(q, wr, wc, 128);
+        if (it < p.comp) {
+          // epilogue 3 reads this thread's row of X's low part: pull it into L2 now
+          const char *lo = p.ws + ((it % 2 == 0) ? q.xl0 : q.xl1) + toff;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(lo + panel_pair_off(g, 128 * half + 32 * k, T)));
+        }
         // ---- epilogue 1: A -> sA (bf16)
         wait_mma();
         if (!ok) break;
@@ -491,7 +498,10 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
               }
             }
           }
-          if (ch & 1) report(2 * half + (ch >> 1), !last);   // (the partner's sXcol was written)
+          // sXown (own CTA) is what the next Gram reads; the partner's sXcol, written in every
+          // chunk, is read by the next update, after this warp's second report: one
+          // cluster-scope fence before that report covers it.
+          if (ch & 1) report(2 * half + (ch >> 1), !last && ch == 3);
         }
       }
       if (ok && wp)
@@ -678,6 +688,13 @@ __global__ void __launch_bounds__(kThreads1, kCtasPerSm1) himuon_tile128_kernel(
         const float ca = p.coef[it][0], cb = p.coef[it][1], cc = p.coef[it][2];
         const float s2 = it == 0 ? s * s : 1.0f, ks = it == 0 ? s : 1.0f;
         if (wp && it + 1 == K) w_prefetch(q, wr, wc, 128);
+        if (it < p.comp) {
+          // epilogue 3 reads this thread's row of X's low part: pull it into L2 now
+          const char *lo = p.ws + ((it % 2 == 0) ? q.xl0 : q.xl1) + toff;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(lo + panel_pair_off(rl, 32 * k, T1)));
+        }
         wait_mma();
         if (!ok) break;
 #pragma unroll 1

@@ -99,10 +99,11 @@ __global__ void __launch_bounds__(256) split_kernel(const __grid_constant__ Spli
 // ------------------------------------------------ diagonal block of the factorisation
 // One 256 x 256 diagonal block of S per layer input, factored as two 128-column halves in
 // shared memory (three 128 x 128 fp32 tiles), then inverted:
-//   L11 = chol(A11);  D11 = L11^-1;  L21 = A21 D11^T;  L22 = chol(A22 - L21 L21^T);
+//   L11 = chol(A11);  D11 = L11^-1;  L21^T = D11 A12 (A12 = A21^T: the trailing update
+//   keeps the whole diagonal block current);  L22 = chol(A22 - L21 L21^T);
 //   D22 = L22^-1;  D21 = -D22 (L21 D11);
 // the inverse D = [D11 0; D21 D22] goes out as bf16 hi/lo panels (block k of the stack).
-constexpr int kT = 128, kTP = 129;       // tile size, padded row stride (floats)
+constexpr int kT = 128, kTP = 132;       // tile size, row stride (floats; rows 16-byte aligned)
 constexpr int kDiagThreads = 512;
 constexpr int kDiagSmem = 3 * kT * kTP * 4;
 
@@ -153,28 +154,57 @@ __device__ void inv_tile(const float *L, float *D) {
   __syncthreads();
 }
 
-// acc[e] = sum_q X[r][q] Y'[q][c_e] for row r = tid / 4 and the interleaved columns
-// c_e = tid % 4 + 4 e (Y' = Y, or Y^T when ytrans): the four threads of a row read four
-// different banks.
-__device__ __forceinline__ void row_products(const float *X, const float *Y, bool ytrans, float (&acc)[32]) {
-  const int tid = threadIdx.x, r = tid >> 2, cp = tid & 3;
+// acc[i][e] = sum_q A'[r0 + i][q] Y[q][c0 + e] over a 4 x 8 block per thread (r0 = 4 (t / 16),
+// c0 = 8 (t % 16)), with A' = A, or A^T when atrans.  Four k steps at a time: A' as four
+// float4 reads (rows of A, or rows of A^T = four consecutive rows of A' at one k), Y as
+// eight; a warp's reads hit distinct banks or broadcast.
+__device__ __forceinline__ void tile_products(const float *A, const float *Y, bool atrans, float (&acc)[4][8]) {
+  const int tid = threadIdx.x, r0 = 4 * (tid >> 4), c0 = 8 * (tid & 15);
 #pragma unroll
-  for (int e = 0; e < 32; ++e) acc[e] = 0.f;
-  for (int q = 0; q < kT; ++q) {
-    const float x = X[r * kTP + q];
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int e = 0; e < 32; ++e) acc[e] = fmaf(x, ytrans ? Y[(cp + 4 * e) * kTP + q] : Y[q * kTP + cp + 4 * e], acc[e]);
+    for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
+  for (int q = 0; q < kT; q += 4) {
+    float a[4][4];   // a[i][j] = A'[r0 + i][q + j]
+    if (!atrans) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 v = *reinterpret_cast<const float4 *>(A + (r0 + i) * kTP + q);
+        a[i][0] = v.x; a[i][1] = v.y; a[i][2] = v.z; a[i][3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 v = *reinterpret_cast<const float4 *>(A + (q + j) * kTP + r0);
+        a[0][j] = v.x; a[1][j] = v.y; a[2][j] = v.z; a[3][j] = v.w;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 y0 = *reinterpret_cast<const float4 *>(Y + (q + j) * kTP + c0);
+      const float4 y1 = *reinterpret_cast<const float4 *>(Y + (q + j) * kTP + c0 + 4);
+      const float y[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[i][e] = fmaf(a[i][j], y[e], acc[i][e]);
+    }
   }
 }
 
-// Out = sgn * X Y' (128 x 128 tiles); Out may be X (every row of X is read first).
-__device__ void mul_tile(const float *X, const float *Y, float *Out, float sgn, bool ytrans) {
-  const int tid = threadIdx.x, r = tid >> 2, cp = tid & 3;
-  float acc[32];
-  row_products(X, Y, ytrans, acc);
+// Out = sgn * A' Y (128 x 128 tiles); Out may be A or Y (every read happens first).
+__device__ void mul_tile(const float *A, const float *Y, float *Out, float sgn, bool atrans) {
+  const int tid = threadIdx.x, r0 = 4 * (tid >> 4), c0 = 8 * (tid & 15);
+  float acc[4][8];
+  tile_products(A, Y, atrans, acc);
   __syncthreads();
 #pragma unroll
-  for (int e = 0; e < 32; ++e) Out[r * kTP + cp + 4 * e] = sgn * acc[e];
+  for (int i = 0; i < 4; ++i) {
+    *reinterpret_cast<float4 *>(Out + (r0 + i) * kTP + c0) =
+        make_float4(sgn * acc[i][0], sgn * acc[i][1], sgn * acc[i][2], sgn * acc[i][3]);
+    *reinterpret_cast<float4 *>(Out + (r0 + i) * kTP + c0 + 4) =
+        make_float4(sgn * acc[i][4], sgn * acc[i][5], sgn * acc[i][6], sgn * acc[i][7]);
+  }
   __syncthreads();
 }
 
@@ -197,15 +227,15 @@ __device__ void store_tile_panels(const float *T, char *hi, char *lo, int ph, in
 }
 
 __device__ void load_tile(const float *S, int ld, int r0, int c0, float *T) {
-  for (int q = threadIdx.x; q < kT * kT; q += kDiagThreads) {
-    const int r = q >> 7, c = q & 127;
-    T[r * kTP + c] = S[(int64_t)(r0 + r) * ld + c0 + c];
+  for (int q = threadIdx.x; q < kT * kT / 4; q += kDiagThreads) {
+    const int r = q >> 5, c = 4 * (q & 31);
+    *reinterpret_cast<float4 *>(T + r * kTP + c) = *reinterpret_cast<const float4 *>(S + (int64_t)(r0 + r) * ld + c0 + c);
   }
   __syncthreads();
 }
 
 __global__ void __launch_bounds__(kDiagThreads, 1) potrf_diag_kernel(const __grid_constant__ DiagParams p) {
-  extern __shared__ float tsm[];
+  extern __shared__ __align__(16) float tsm[];
   float *T0 = tsm, *T1 = tsm + kT * kTP, *T2 = tsm + 2 * kT * kTP;
   pdl_trigger();
   pdl_wait();
@@ -218,21 +248,23 @@ __global__ void __launch_bounds__(kDiagThreads, 1) potrf_diag_kernel(const __gri
   load_tile(S, ld, k0, k0, T0);                 // A11
   chol_tile(T0, p.status);                       // L11
   inv_tile(T0, T2);                              // D11
-  load_tile(S, ld, k0 + kT, k0, T1);             // A21
-  mul_tile(T1, T2, T1, 1.f, true);               // L21 = A21 D11^T
+  load_tile(S, ld, k0, k0 + kT, T1);             // A12 = A21^T
+  mul_tile(T2, T1, T1, 1.f, false);              // L21^T = D11 A12
   load_tile(S, ld, k0 + kT, k0 + kT, T0);        // A22
-  // A22 -= L21 L21^T (the upper part is computed too and never read)
   {
-    const int tid = threadIdx.x, r = tid >> 2, cp = tid & 3;
-    float acc[32];
-    row_products(T1, T1, true, acc);
+    // A22 -= L21 L21^T: [r][c] -= sum_q L21^T[q][r] L21^T[q][c] (the upper part is never read)
+    const int tid = threadIdx.x, r0 = 4 * (tid >> 4), c0 = 8 * (tid & 15);
+    float acc[4][8];
+    tile_products(T1, T1, true, acc);
 #pragma unroll
-    for (int e = 0; e < 32; ++e) T0[r * kTP + cp + 4 * e] -= acc[e];
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) T0[(r0 + i) * kTP + c0 + e] -= acc[i][e];
     __syncthreads();
   }
   chol_tile(T0, p.status);                       // L22
   store_tile_panels(T2, hi, lo, ld, k0, 0);      // D11
-  mul_tile(T1, T2, T1, 1.f, false);              // X = L21 D11
+  mul_tile(T1, T2, T1, 1.f, true);               // X = L21 D11
   inv_tile(T0, T2);                              // D22
   mul_tile(T2, T1, T0, -1.f, false);             // D21 = -D22 X
   store_tile_panels(T0, hi, lo, ld, k0 + kT, 0);

@@ -232,6 +232,16 @@ __global__ void __launch_bounds__(kThreads, 1) newton_gemm_kernel(const __grid_c
       const float *crow = sub ? reinterpret_cast<const float *>(p.ws + q.c32) + i * q.ld32 + t.n0 : nullptr;
       float *drow = q.d32 >= 0 ? reinterpret_cast<float *>(p.ws + q.d32) + i * q.ld32 + t.n0 : nullptr;
       const bool valid = i < q.m_valid;                   // rows past the valid region are not written
+      // C of columns col0 .. col0+31 (issued a chunk ahead of its use)
+      auto load_c = [&](int col0, float (&c)[32]) {
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const float4 v = *reinterpret_cast<const float4 *>(crow + col0 + 4 * g);
+          c[4 * g] = v.x; c[4 * g + 1] = v.y; c[4 * g + 2] = v.z; c[4 * g + 3] = v.w;
+        }
+      };
+      float c[32];
+      if (sub) load_c(half * 128, c);                      // in flight while the MMAs finish
       if (!mbar_wait(tfull_bar(buf), tph, limit)) {
         set_status(p.status, kTimeoutBit);
         break;
@@ -240,14 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1) newton_gemm_kernel(const __grid_c
 #pragma unroll 1
       for (int cc = half * 4; cc < half * 4 + 4; ++cc) {
         const int col0 = cc * 32;                           // column within the tile
-        float c[32];
-        if (sub) {
-#pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            const float4 v = *reinterpret_cast<const float4 *>(crow + col0 + 4 * g);
-            c[4 * g] = v.x; c[4 * g + 1] = v.y; c[4 * g + 2] = v.z; c[4 * g + 3] = v.w;
-          }
-        }
+        float cn[32];
+        if (sub && cc + 1 < half * 4 + 4) load_c(col0 + 32, cn);
         uint32_t r[32];
         tmem_ld32(tmem_base + (uint32_t)(buf * BN + col0) + ((uint32_t)(quarter * 32) << 16), r);
         tmem_ld_wait();
@@ -284,6 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1) newton_gemm_kernel(const __grid_c
             st_global_256(p.ws + q.dlo + off, w);
           }
         }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) c[e] = cn[e];
       }
       tc_fence_before();
       __syncwarp();
