@@ -416,6 +416,7 @@ nshb_status run_momentum(const nshb_matrix *mats, const Plan &pl, const nshb_par
     mp.ws = ws;
     mp.partials = k1part + kK1PartsPerBlock * (int64_t)pl.mp[c0].k1_begin;
     mp.status = reinterpret_cast<uint32_t *>(ws);
+    mp.wait_limit = (p->debug_flags & 1u) ? kWaitLimitTest : kWaitLimit;
     mp.beta = p->beta;
     mp.nesterov = p->nesterov ? 1 : 0;
     mp.nmat = c1 - c0;
@@ -758,11 +759,12 @@ NwProb nw_prob() {
   std::memset(&q, 0, sizeof(q));
   q.c32 = q.d32 = q.dhi = q.dlo = -1;
   q.kt = 4;                        // every product is 256 deep (one block column)
+  q.hl_n0 = -1;
   return q;
 }
 
 // Launches the split-precision products of `probs` (in launches of kMaxNwProb).
-nshb_status run_nw(NwParams &np, const std::vector<NwProb> &probs, cudaStream_t st) {
+nshb_status run_nw(NwParams &np, const std::vector<NwProb> &probs, cudaStream_t st, int reserve_pairs = 0) {
   for (size_t c0 = 0; c0 < probs.size(); c0 += kMaxNwProb) {
     const size_t c1 = std::min(probs.size(), c0 + (size_t)kMaxNwProb);
     int tiles = 0;
@@ -774,7 +776,7 @@ nshb_status run_nw(NwParams &np, const std::vector<NwProb> &probs, cudaStream_t 
     }
     np.nprob = (int)(c1 - c0);
     np.total_tiles = tiles;
-    NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_newton_gemm(np, device_sms(), st));
+    NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_newton_gemm(np, device_sms(), st, reserve_pairs));
   }
   return NSHB_OK;
 }
@@ -814,6 +816,7 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
     mp.ws = ws;
     mp.partials = reinterpret_cast<double *>(ws + pl.k1part_off);
     mp.status = status;
+    mp.wait_limit = limit;
     mp.beta = p->beta;
     mp.nesterov = p->nesterov ? 1 : 0;
     mp.nmat = c1 - c0;
@@ -946,9 +949,11 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
   for (auto &z : pl.zp) dmax = std::max(dmax, z.Dp);
   const int nb = (int)(dmax / 256);
   // 4. forward: blocked right-looking Cholesky S = L L^T with the rows of every U carried
-  //    along, so that block column k of Y = U L^-T is final after step k
-  for (int k = 0; k < nb; ++k) {
-    const int64_t k0 = 256LL * k, k1 = k0 + 256;
+  //    along, so that block column k of Y = U L^-T is final after step k.  The diagonal
+  //    block of step k + 1 needs only step k's update of S, so it is factored while step k's
+  //    update of U runs: launches diag(0), then per step panel(k), S(k), diag(k + 1), U(k).
+  auto run_diag = [&](int k) -> nshb_status {
+    const int64_t k0 = 256LL * k;
     for (int c0 = 0; c0 < nz; c0 += kMaxMats) {
       const int c1 = std::min(nz, c0 + kMaxMats);
       DiagParams dp;
@@ -966,8 +971,14 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
       }
       if (dp.n) NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_potrf_diag(dp, st));
     }
+    return NSHB_OK;
+  };
+  nshb_status ed = run_diag(0);
+  if (ed != NSHB_OK) return ed;
+  for (int k = 0; k < nb; ++k) {
+    const int64_t k0 = 256LL * k, k1 = k0 + 256;
     // panel: L[k1:, k] = S[k1:, k] D_k^T and Y[:, k] = U[:, k] D_k^T
-    std::vector<NwProb> panel, trail;
+    std::vector<NwProb> panel, trail_s, trail_u;
     for (auto &z : pl.zp) {
       if (z.Dp <= k1) continue;
       NwProb q = nw_prob();
@@ -985,7 +996,8 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
       t.dhi = z.sh; t.dlo = z.sl; t.d_ph = (int)z.Dp; t.d_r0 = (int)k1; t.d_c0 = (int)k1;
       t.mt = t.nt = (int)((z.Dp - k1) / 256);
       t.flags = kNwLower;
-      trail.push_back(t);
+      t.hl_n0 = 0;                 // the next panel reads block column k + 1 only
+      trail_s.push_back(t);
     }
     for (int i = 0; i < n; ++i) {
       const Plan::ZPlan &z = pl.zp[pl.zidx[i]];
@@ -1006,11 +1018,23 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
       t.m_valid = (int)pl.mpad[i]; t.n_valid = (int)(z.Dp - k1);
       t.dhi = pl.yh[i]; t.dlo = pl.yl[i]; t.d_ph = (int)pl.mpad[i]; t.d_r0 = 0; t.d_c0 = (int)k1;
       t.mt = (int)(pl.mpad[i] / 256); t.nt = (int)((z.Dp - k1) / 256);
-      trail.push_back(t);
+      t.hl_n0 = 0;
+      trail_u.push_back(t);
     }
     nshb_status e = run_nw(np, panel, st);
     if (e != NSHB_OK) return e;
-    e = run_nw(np, trail, st);
+    e = run_nw(np, trail_s, st);
+    if (e != NSHB_OK) return e;
+    if (k + 1 == nb) continue;
+    e = run_diag(k + 1);
+    if (e != NSHB_OK) return e;
+    // beside the diagonal blocks: one SM per block is taken, and a few pairs more for the
+    // SMs that the pairing leaves single
+    int ndiag = 0;
+    for (auto &z : pl.zp) ndiag += z.Dp > k1 ? 1 : 0;
+    np.late_wait = 1;
+    e = run_nw(np, trail_u, st, (ndiag + 1) / 2 + 4);
+    np.late_wait = 0;
     if (e != NSHB_OK) return e;
   }
   // 5. backward: P L = Y, right-looking from the last block: P[:, k] = Y[:, k] D_k (fp32 into
@@ -1038,6 +1062,7 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
       t.c32 = t.d32 = pl.y32[i]; t.ld32 = (int)z.Dp; t.m_valid = (int)pl.mpad[i]; t.n_valid = (int)k0;
       t.dhi = pl.yh[i]; t.dlo = pl.yl[i]; t.d_ph = (int)pl.mpad[i]; t.d_r0 = 0; t.d_c0 = 0;
       t.mt = (int)(pl.mpad[i] / 256); t.nt = k;
+      t.hl_n0 = (int)(k0 - 256);   // the next solve reads block column k - 1 only
       upd.push_back(t);
     }
     nshb_status e = run_nw(np, solve, st);

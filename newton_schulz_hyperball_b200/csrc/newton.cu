@@ -58,7 +58,8 @@ __global__ void __launch_bounds__(256) ridge_kernel(const __grid_constant__ Chol
 }
 
 // fp32 regions -> bf16 hi/lo panels (X_hi = bf16(X), X_lo = bf16(X - X_hi)), one 64 x 64
-// block per CTA; thread t handles row t/4 (+ 64 (t/256)) ... columns 16 (t % 4) .. +15.
+// block per CTA; thread t handles 8 columns 8 (t % 8) .. +7 of rows t / 8 and 32 + t / 8 (two
+// 16-byte loads each where the row is whole and 16-byte aligned).
 __global__ void __launch_bounds__(256) split_kernel(const __grid_constant__ SplitParams p) {
   pdl_trigger();
   pdl_wait();
@@ -74,21 +75,43 @@ __global__ void __launch_bounds__(256) split_kernel(const __grid_constant__ Spli
   const int r0 = (lb / bc) * 64, c0 = (lb % bc) * 64;
   const float *src = reinterpret_cast<const float *>(p.ws + it.src32);
   float *dst = it.dst32 >= 0 ? reinterpret_cast<float *>(p.ws + it.dst32) : nullptr;
-  for (int q = threadIdx.x; q < 64 * 8; q += blockDim.x) {
+  const bool vsrc = (it.src_ld & 3) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+  const bool vdst = dst && (it.dst_ld & 3) == 0 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0;
+  float v[2][8];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {                     // both loads in flight before any store
+    const int q = threadIdx.x + 256 * u;
     const int r = r0 + (q >> 3), c = c0 + 8 * (q & 7);
-    float v[8];
+    const float *s = src + (int64_t)r * it.src_ld + c;
+    if (vsrc && r < it.rows && c + 8 <= it.cols) {
+      const float4 a = *reinterpret_cast<const float4 *>(s), b = *reinterpret_cast<const float4 *>(s + 4);
+      v[u][0] = a.x; v[u][1] = a.y; v[u][2] = a.z; v[u][3] = a.w;
+      v[u][4] = b.x; v[u][5] = b.y; v[u][6] = b.z; v[u][7] = b.w;
+    } else {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = (r < it.rows && c + e < it.cols) ? src[(int64_t)r * it.src_ld + c + e] : 0.f;
+      for (int e = 0; e < 8; ++e) v[u][e] = (r < it.rows && c + e < it.cols) ? s[e] : 0.f;
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int q = threadIdx.x + 256 * u;
+    const int r = r0 + (q >> 3), c = c0 + 8 * (q & 7);
     if (dst) {
+      float *d = dst + (int64_t)r * it.dst_ld + c;
+      if (vdst) {
+        *reinterpret_cast<float4 *>(d) = make_float4(v[u][0], v[u][1], v[u][2], v[u][3]);
+        *reinterpret_cast<float4 *>(d + 4) = make_float4(v[u][4], v[u][5], v[u][6], v[u][7]);
+      } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) dst[(int64_t)r * it.dst_ld + c + e] = v[e];
+        for (int e = 0; e < 8; ++e) d[e] = v[u][e];
+      }
     }
     uint4 h, l;
     uint32_t *hp = &h.x, *lp = &l.x;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      hp[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
-      lp[e] = pack_bf16(v[2 * e] - bf16lo(hp[e]), v[2 * e + 1] - bf16hi(hp[e]));
+      hp[e] = pack_bf16(v[u][2 * e], v[u][2 * e + 1]);
+      lp[e] = pack_bf16(v[u][2 * e] - bf16lo(hp[e]), v[u][2 * e + 1] - bf16hi(hp[e]));
     }
     const size_t off = panel_chunk_off(it.d_r0 + r, it.d_c0 + c, it.d_ph);
     *reinterpret_cast<uint4 *>(p.ws + it.dhi + off) = h;
@@ -97,184 +120,241 @@ __global__ void __launch_bounds__(256) split_kernel(const __grid_constant__ Spli
 }
 
 // ------------------------------------------------ diagonal block of the factorisation
-// One 256 x 256 diagonal block of S per layer input, factored as two 128-column halves in
-// shared memory (three 128 x 128 fp32 tiles), then inverted:
-//   L11 = chol(A11);  D11 = L11^-1;  L21^T = D11 A12 (A12 = A21^T: the trailing update
-//   keeps the whole diagonal block current);  L22 = chol(A22 - L21 L21^T);
-//   D22 = L22^-1;  D21 = -D22 (L21 D11);
-// the inverse D = [D11 0; D21 D22] goes out as bf16 hi/lo panels (block k of the stack).
-constexpr int kT = 128, kTP = 132;       // tile size, row stride (floats; rows 16-byte aligned)
-constexpr int kDiagThreads = 512;
-constexpr int kDiagSmem = 3 * kT * kTP * 4;
+// One 256 x 256 diagonal block A of S per layer input (one CTA each), factored A = L L^T and
+// inverted, D = L^-1, in one left-to-right sweep over eight 32-wide block columns.  The lower
+// triangle lives in shared memory as 36 blocks of 32 x 32 (block (i, k), i >= k); every
+// block is overwritten in turn by L and then by D.  Step j:
+//   A  one warp factors the diagonal block, A_jj = L_jj L_jj^T, and inverts it, D_jj =
+//      L_jj^-1 (L_jj itself is needed by nothing else);  the other warps meanwhile finish
+//      block row j - 1 of D (below);
+//   B  panel L_ij = A_ij D_jj^T (i > j), and X_jm = D_jj L_jm (m < j: block row j of L is
+//      no longer read by the factorisation);
+//   C  trailing update A_ik -= L_ij L_kj^T (j < k <= i);
+// and block row j of D is  D_jk = -sum_{k <= m < j} X_jm D_mk  (from D L = I), computed
+// during step j + 1 (row 7 at the end).  The result goes out as bf16 hi / lo panels (block k
+// of the inverse stack), with zeros above the diagonal.  A pivot that is not positive in
+// fp32 is flagged (NSHB_DEV_NOT_SPD) and replaced by 1e-30.
+constexpr int kNB = 8;                    // block columns
+constexpr int kBS = 36;                   // row stride of a block (floats): conflict-free float4 rows
+constexpr int kBlk = 32 * kBS + 4;        // block stride (floats): consecutive blocks start 4 banks apart
+constexpr int kNBlk = kNB * (kNB + 1) / 2;
+constexpr int kDiagThreads = 512, kDiagWarps = kDiagThreads / 32;
+constexpr int kDiagSmem = kNBlk * kBlk * 4;
+static_assert(kDiagSmem <= 227 * 1024, "diagonal block does not fit in shared memory");
 
-// In-place lower Cholesky factor of a 128 x 128 tile (only its lower triangle is read).
-// Column j: every thread takes the pivot a = T[j][j], updates its share of the trailing
-// lower part with T[i][c] -= T[i][j] T[c][j] / a (four threads per row i, interleaved
-// columns), and scales column j - 1 by 1 / sqrt of that column's pivot.  A pivot that is
-// not positive is flagged (NSHB_DEV_NOT_SPD) and replaced by 1e-30.
-__device__ __forceinline__ float pivot(float a) { return a > 0.f ? a : 1e-30f; }
+__device__ __forceinline__ float *blk(float *sm, int i, int k) { return sm + (i * (i + 1) / 2 + k) * kBlk; }
 
-__device__ void chol_tile(float *T, uint32_t *status) {
-  const int tid = threadIdx.x, rr = tid >> 2, cpart = tid & 3;
-  for (int j = 0; j < kT; ++j) {
-    const float a0 = T[j * kTP + j];
-    if (!(a0 > 0.f) && tid == 0) set_status(status, 0x10u);   // not positive definite in fp32
-    const float a = pivot(a0);
-    if (j > 0) {                                  // finish column j - 1
-      const float rs = rsqrtf(pivot(T[(j - 1) * kTP + (j - 1)]));
-      for (int i = j + tid; i < kT; i += kDiagThreads) T[i * kTP + (j - 1)] *= rs;
-    }
-    __syncthreads();
-    if (tid == 0 && j > 0) T[(j - 1) * kTP + (j - 1)] = sqrtf(pivot(T[(j - 1) * kTP + (j - 1)]));
-    const int i = j + 1 + rr;                     // one row per group of four threads
-    if (i < kT) {
-      const float li = T[i * kTP + j] / a;
-      for (int c = j + 1 + cpart; c <= i; c += 4) T[i * kTP + c] = fmaf(-li, T[c * kTP + j], T[i * kTP + c]);
-    }
-    __syncthreads();
-  }
-  if (tid == 0) T[(kT - 1) * kTP + (kT - 1)] = sqrtf(pivot(T[(kT - 1) * kTP + (kT - 1)]));
-  __syncthreads();
-}
-
-// D = L^-1 of a lower-triangular tile (D lower).  Warp w solves columns 8w .. 8w+7, four
-// lanes per column: D[i][c] = (delta_ic - sum_{c <= q < i} L[i][q] D[q][c]) / L[i][i].
-__device__ void inv_tile(const float *L, float *D) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c = 8 * warp + (lane >> 2), part = lane & 3;
-  for (int i = 0; i < kT; ++i) {
-    float acc = 0.f;
-    if (i > c)
-      for (int q = c + part; q < i; q += 4) acc = fmaf(L[i * kTP + q], D[q * kTP + c], acc);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    if (part == 0) D[i * kTP + c] = i < c ? 0.f : ((i == c ? 1.f : 0.f) - acc) / L[i * kTP + i];
-    __syncwarp();
-  }
-  __syncthreads();
-}
-
-// acc[i][e] = sum_q A'[r0 + i][q] Y[q][c0 + e] over a 4 x 8 block per thread (r0 = 4 (t / 16),
-// c0 = 8 (t % 16)), with A' = A, or A^T when atrans.  Four k steps at a time: A' as four
-// float4 reads (rows of A, or rows of A^T = four consecutive rows of A' at one k), Y as
-// eight; a warp's reads hit distinct banks or broadcast.
-__device__ __forceinline__ void tile_products(const float *A, const float *Y, bool atrans, float (&acc)[4][8]) {
-  const int tid = threadIdx.x, r0 = 4 * (tid >> 4), c0 = 8 * (tid & 15);
+// acc[x][e] += sum_q A[g + 8x][q] B[h + 4e][q]   (A B^T;  g = lane / 4, h = lane % 4)
+__device__ __forceinline__ void nt_acc(const float *A, const float *B, float (&acc)[4][8]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, h = lane & 3;
+#pragma unroll 2
+  for (int q = 0; q < 32; q += 4) {
+    float4 a[4], b[8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+    for (int x = 0; x < 4; ++x) a[x] = *reinterpret_cast<const float4 *>(A + (g + 8 * x) * kBS + q);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
-  for (int q = 0; q < kT; q += 4) {
-    float a[4][4];   // a[i][j] = A'[r0 + i][q + j]
-    if (!atrans) {
+    for (int e = 0; e < 8; ++e) b[e] = *reinterpret_cast<const float4 *>(B + (h + 4 * e) * kBS + q);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 v = *reinterpret_cast<const float4 *>(A + (r0 + i) * kTP + q);
-        a[i][0] = v.x; a[i][1] = v.y; a[i][2] = v.z; a[i][3] = v.w;
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float t = acc[x][e];
+        t = fmaf(a[x].x, b[e].x, t);
+        t = fmaf(a[x].y, b[e].y, t);
+        t = fmaf(a[x].z, b[e].z, t);
+        acc[x][e] = fmaf(a[x].w, b[e].w, t);
       }
-    } else {
+  }
+}
+
+// acc[x][e] += sum_q A[g + 8x][q] B[q][8h + e]   (A B)
+__device__ __forceinline__ void nn_acc(const float *A, const float *B, float (&acc)[4][8]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, h = lane & 3;
+#pragma unroll 2
+  for (int q = 0; q < 32; q += 4) {
+    float4 a[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float4 v = *reinterpret_cast<const float4 *>(A + (q + j) * kTP + r0);
-        a[0][j] = v.x; a[1][j] = v.y; a[2][j] = v.z; a[3][j] = v.w;
+    for (int x = 0; x < 4; ++x) a[x] = *reinterpret_cast<const float4 *>(A + (g + 8 * x) * kBS + q);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const float4 b0 = *reinterpret_cast<const float4 *>(B + (q + t) * kBS + 8 * h);
+      const float4 b1 = *reinterpret_cast<const float4 *>(B + (q + t) * kBS + 8 * h + 4);
+      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const float av = t == 0 ? a[x].x : t == 1 ? a[x].y : t == 2 ? a[x].z : a[x].w;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[x][e] = fmaf(av, b[e], acc[x][e]);
       }
     }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float4 y0 = *reinterpret_cast<const float4 *>(Y + (q + j) * kTP + c0);
-      const float4 y1 = *reinterpret_cast<const float4 *>(Y + (q + j) * kTP + c0 + 4);
-      const float y[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[i][e] = fmaf(a[i][j], y[e], acc[i][e]);
-    }
   }
 }
 
-// Out = sgn * A' Y (128 x 128 tiles); Out may be A or Y (every read happens first).
-__device__ void mul_tile(const float *A, const float *Y, float *Out, float sgn, bool atrans) {
-  const int tid = threadIdx.x, r0 = 4 * (tid >> 4), c0 = 8 * (tid & 15);
+__device__ __forceinline__ void zero_acc(float (&acc)[4][8]) {
+#pragma unroll
+  for (int x = 0; x < 4; ++x)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[x][e] = 0.f;
+}
+
+// Stores sgn * acc into a block, in the element order of nt_acc (nt) or nn_acc.
+__device__ __forceinline__ void put_acc(float *C, const float (&acc)[4][8], float sgn, bool nt) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, h = lane & 3;
+#pragma unroll
+  for (int x = 0; x < 4; ++x)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) C[(g + 8 * x) * kBS + (nt ? h + 4 * e : 8 * h + e)] = sgn * acc[x][e];
+}
+
+// One warp: block B (32 x 32, lower triangle read) is replaced by D = L^-1, where B = L L^T.
+// Cholesky with row r in lane r's registers (pivot and column broadcast by shuffles); then L^T
+// goes to B (reciprocal on the diagonal) and lane c solves column c of D by forward
+// substitution, D[q][c] = (e_c - sum_{p < q} L[q][p] D[p][c]) / L[q][q].
+__device__ void chol_inv_block(float *B, uint32_t *status) {
+  const int lane = threadIdx.x & 31;
+  float a[32];
+#pragma unroll
+  for (int c = 0; c < 32; c += 4) {
+    const float4 v = *reinterpret_cast<const float4 *>(B + lane * kBS + c);
+    a[c] = v.x; a[c + 1] = v.y; a[c + 2] = v.z; a[c + 3] = v.w;
+  }
+  bool bad = false;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    float piv = __shfl_sync(0xffffffffu, a[j], j);
+    bad |= !(piv > 0.f);
+    piv = piv > 0.f ? piv : 1e-30f;
+    const float l = lane > j ? a[j] * rsqrtf(piv) : lane == j ? piv * rsqrtf(piv) : 0.f;
+    a[j] = l;
+#pragma unroll
+    for (int c = j + 1; c < 32; ++c) a[c] = fmaf(-l, __shfl_sync(0xffffffffu, l, c), a[c]);
+  }
+  if (bad && lane == 0) set_status(status, 0x10u);
+  __syncwarp();
+#pragma unroll
+  for (int c = 0; c < 32; ++c) B[c * kBS + lane] = c < lane ? a[c] : c == lane ? 1.f / a[c] : 0.f;
+  __syncwarp();
+  float d[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) d[i] = i == lane ? 1.f : 0.f;
+#pragma unroll
+  for (int q = 0; q < 32; ++q) {
+    const float *lt = B + q * kBS;                      // row q of L^T: L[i][q] at i
+    d[q] *= lt[q];
+#pragma unroll
+    for (int i4 = (q + 1) & ~3; i4 < 32; i4 += 4) {
+      const float4 v = *reinterpret_cast<const float4 *>(lt + i4);
+      const float w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (i4 + u > q) d[i4 + u] = fmaf(-w[u], d[q], d[i4 + u]);
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) B[i * kBS + lane] = d[i];
+  __syncwarp();
+}
+
+// Block row J of D over `nw` warps starting at warp w0 (J <= 7 < nw: at most one block each):
+// D_Jk = -sum_{k <= m < J} X_Jm D_mk, written in place of X_Jk once every participating warp
+// has read its operands (named barrier 1 over the nw warps).
+__device__ void drow(float *sm, int J, int w0, int nw) {
+  const int k = (int)(threadIdx.x >> 5) - w0;
   float acc[4][8];
-  tile_products(A, Y, atrans, acc);
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    *reinterpret_cast<float4 *>(Out + (r0 + i) * kTP + c0) =
-        make_float4(sgn * acc[i][0], sgn * acc[i][1], sgn * acc[i][2], sgn * acc[i][3]);
-    *reinterpret_cast<float4 *>(Out + (r0 + i) * kTP + c0 + 4) =
-        make_float4(sgn * acc[i][4], sgn * acc[i][5], sgn * acc[i][6], sgn * acc[i][7]);
-  }
-  __syncthreads();
+  zero_acc(acc);
+  if (k < J)
+    for (int m = k; m < J; ++m) nn_acc(blk(sm, J, m), blk(sm, m, k), acc);
+  asm volatile("bar.sync 1, %0;" ::"r"(nw * 32) : "memory");
+  if (k < J) put_acc(blk(sm, J, k), acc, -1.f, false);
 }
 
-// Writes a 128 x 128 tile into the hi / lo panels of the inverse stack at (r0, c0).
-__device__ void store_tile_panels(const float *T, char *hi, char *lo, int ph, int r0, int c0) {
-  for (int q = threadIdx.x; q < kT * kT / 8; q += kDiagThreads) {
-    const int r = q >> 4, c = 8 * (q & 15);
-    uint4 h, l;
-    uint32_t *hp = &h.x, *lp = &l.x;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float v0 = T[r * kTP + c + 2 * e], v1 = T[r * kTP + c + 2 * e + 1];
-      hp[e] = pack_bf16(v0, v1);
-      lp[e] = pack_bf16(v0 - bf16lo(hp[e]), v1 - bf16hi(hp[e]));
-    }
-    const size_t off = panel_chunk_off(r0 + r, c0 + c, ph);
-    *reinterpret_cast<uint4 *>(hi + off) = h;
-    *reinterpret_cast<uint4 *>(lo + off) = l;
-  }
-}
-
-__device__ void load_tile(const float *S, int ld, int r0, int c0, float *T) {
-  for (int q = threadIdx.x; q < kT * kT / 4; q += kDiagThreads) {
-    const int r = q >> 5, c = 4 * (q & 31);
-    *reinterpret_cast<float4 *>(T + r * kTP + c) = *reinterpret_cast<const float4 *>(S + (int64_t)(r0 + r) * ld + c0 + c);
-  }
-  __syncthreads();
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 
 __global__ void __launch_bounds__(kDiagThreads, 1) potrf_diag_kernel(const __grid_constant__ DiagParams p) {
-  extern __shared__ __align__(16) float tsm[];
-  float *T0 = tsm, *T1 = tsm + kT * kTP, *T2 = tsm + 2 * kT * kTP;
-  pdl_trigger();
+  extern __shared__ __align__(16) float sm[];
+  // Wait first, then let the next kernel start: it may run beside this one (the update of U by
+  // the previous step does not touch S), and everything before this kernel is complete.
   pdl_wait();
+  pdl_trigger();
   const int z = blockIdx.x;
   if (z >= p.n) return;
   const int ld = p.ld[z], k0 = 256 * p.k;
   if (k0 >= ld) return;
   const float *S = reinterpret_cast<const float *>(p.ws + p.s32[z]);
   char *hi = p.ws + p.dhi[z], *lo = p.ws + p.dlo[z];
-  load_tile(S, ld, k0, k0, T0);                 // A11
-  chol_tile(T0, p.status);                       // L11
-  inv_tile(T0, T2);                              // D11
-  load_tile(S, ld, k0, k0 + kT, T1);             // A12 = A21^T
-  mul_tile(T2, T1, T1, 1.f, false);              // L21^T = D11 A12
-  load_tile(S, ld, k0 + kT, k0 + kT, T0);        // A22
-  {
-    // A22 -= L21 L21^T: [r][c] -= sum_q L21^T[q][r] L21^T[q][c] (the upper part is never read)
-    const int tid = threadIdx.x, r0 = 4 * (tid >> 4), c0 = 8 * (tid & 15);
-    float acc[4][8];
-    tile_products(T1, T1, true, acc);
+  const int warp = threadIdx.x >> 5;
+  // the 36 lower blocks: 32 rows of eight 16-byte pieces each
+  for (int q = threadIdx.x; q < kNBlk * 256; q += kDiagThreads) {
+    const int b = q >> 8, r = (q >> 3) & 31, c4 = q & 7;
+    int i = 0, k = b;
+    while (k > i) k -= ++i;
+    cp_async16(sm + b * kBlk + r * kBS + 4 * c4, S + (int64_t)(k0 + 32 * i + r) * ld + k0 + 32 * k + 4 * c4);
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
+  for (int j = 0; j < kNB; ++j) {
+    // A: factor and invert the diagonal block; finish block row j - 1 of D beside it
+    if (warp == 0) chol_inv_block(blk(sm, j, j), p.status);
+    else if (j >= 2) drow(sm, j - 1, 1, kDiagWarps - 1);
+    __syncthreads();
+    // B: the panel below (7 - j blocks) and block row j of X (j blocks), one block per warp
+    if (warp < kNB - 1) {
+      float acc[4][8];
+      zero_acc(acc);
+      float *C;
+      const bool panel = warp < kNB - 1 - j;
+      if (panel) {
+        C = blk(sm, j + 1 + warp, j);
+        nt_acc(C, blk(sm, j, j), acc);                  // L_ij = A_ij D_jj^T
+      } else {
+        C = blk(sm, j, warp - (kNB - 1 - j));
+        nn_acc(blk(sm, j, j), C, acc);                  // X_jm = D_jj L_jm
+      }
+      __syncwarp();
+      put_acc(C, acc, 1.f, panel);
+    }
+    __syncthreads();
+    // C: trailing update of the blocks right of and below the panel
+    const int n = kNB - 1 - j;
+    for (int t = warp; t < n * (n + 1) / 2; t += kDiagWarps) {
+      int ii = 0, kk = t;
+      while (kk > ii) kk -= ++ii;
+      const int i = j + 1 + ii, k = j + 1 + kk;
+      float acc[4][8];
+      zero_acc(acc);
+      nt_acc(blk(sm, i, j), blk(sm, k, j), acc);
+      float *C = blk(sm, i, k);
+      const int lane = threadIdx.x & 31, g = lane >> 2, h = lane & 3;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+      for (int x = 0; x < 4; ++x)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) T0[(r0 + i) * kTP + c0 + e] -= acc[i][e];
+        for (int e = 0; e < 8; ++e) C[(g + 8 * x) * kBS + h + 4 * e] -= acc[x][e];
+    }
     __syncthreads();
   }
-  chol_tile(T0, p.status);                       // L22
-  store_tile_panels(T2, hi, lo, ld, k0, 0);      // D11
-  mul_tile(T1, T2, T1, 1.f, true);               // X = L21 D11
-  inv_tile(T0, T2);                              // D22
-  mul_tile(T2, T1, T0, -1.f, false);             // D21 = -D22 X
-  store_tile_panels(T0, hi, lo, ld, k0 + kT, 0);
-  store_tile_panels(T2, hi, lo, ld, k0 + kT, kT);
-  // the upper-right 128 x 128 of the block inverse is zero
-  for (int q = threadIdx.x; q < kT * kT / 8; q += kDiagThreads) {
-    const int r = q >> 4, c = 8 * (q & 15);
-    const size_t off = panel_chunk_off(k0 + r, kT + c, ld);
-    *reinterpret_cast<uint4 *>(hi + off) = make_uint4(0, 0, 0, 0);
-    *reinterpret_cast<uint4 *>(lo + off) = make_uint4(0, 0, 0, 0);
+  drow(sm, kNB - 1, 0, kDiagWarps);
+  __syncthreads();
+  // out: rows k0 .. k0+255, columns 0 .. 255 of the stack, eight columns per 16-byte piece
+  for (int q = threadIdx.x; q < 256 * 32; q += kDiagThreads) {
+    const int r = q >> 5, c = 8 * (q & 31), i = r >> 5, k = c >> 5;
+    uint4 h = make_uint4(0, 0, 0, 0), l = h;
+    if (k <= i) {
+      const float *src = blk(sm, i, k) + (r & 31) * kBS + (c & 31);
+      const float4 v0 = *reinterpret_cast<const float4 *>(src), v1 = *reinterpret_cast<const float4 *>(src + 4);
+      const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      uint32_t *hp = &h.x, *lp = &l.x;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        hp[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+        lp[e] = pack_bf16(v[2 * e] - bf16lo(hp[e]), v[2 * e + 1] - bf16hi(hp[e]));
+      }
+    }
+    const size_t off = panel_chunk_off(k0 + r, c, ld);
+    *reinterpret_cast<uint4 *>(hi + off) = h;
+    *reinterpret_cast<uint4 *>(lo + off) = l;
   }
 }
 

@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1) newton_gemm_kernel(const __grid_c
   const uint32_t tmem_base = *tmem_slot;
   const long long limit = p.wait_limit;
   pdl_trigger();
-  pdl_wait();
+  if (!p.late_wait) pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1) newton_gemm_kernel(const __grid_c
           for (int e = 0; e < 32; ++e)
             if (e < cvalid) drow[col0 + e] = v[e];
         }
-        if (q.dhi >= 0) {
+        if (q.dhi >= 0 && (q.hl_n0 < 0 || t.n0 == q.hl_n0)) {
           const int64_t pr = q.d_r0 + i;                    // row and column in D's panels
           const int64_t pc = q.d_c0 + t.n0 + col0;
           const bool odd = pr & 1;
@@ -304,11 +304,14 @@ __global__ void __launch_bounds__(kThreads, 1) newton_gemm_kernel(const __grid_c
     tc_fence_after();
     tmem_dealloc2(tmem_base, TMEM_COLS);
   }
+  // Ran beside the previous kernel: finish only after it, so that the next kernel's wait
+  // covers both.
+  if (p.late_wait) pdl_wait();
 }
 
 }  // namespace
 
-cudaError_t launch_newton_gemm(const NwParams &p, int num_sms, cudaStream_t s) {
+cudaError_t launch_newton_gemm(const NwParams &p, int num_sms, cudaStream_t s, int reserve_pairs) {
   static PerDevice attr_set;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -342,7 +345,8 @@ cudaError_t launch_newton_gemm(const NwParams &p, int num_sms, cudaStream_t s) {
     mp = n < num_sms / 2 ? n : num_sms / 2;
     max_pairs.set(dev, mp);
   }
-  const int clusters = p.total_tiles < mp ? p.total_tiles : mp;
+  const int avail = mp - reserve_pairs > 1 ? mp - reserve_pairs : 1;
+  const int clusters = p.total_tiles < avail ? p.total_tiles : avail;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);

@@ -69,6 +69,7 @@ struct MomentumParams {
   char *ws;
   double *partials;  // kK1PartsPerBlock per block of the launch
   uint32_t *status;
+  long long wait_limit;  // clock cycles per mbarrier phase (bulk-copy variant)
   float beta;
   int32_t nesterov;
   int32_t nmat, total_blocks;
@@ -284,6 +285,8 @@ struct NwProb {
   int32_t mt, nt, kt;              // 256-row tiles, 256-column tiles, 64-deep k panels (even)
   int32_t flags;                   // kNwBMn | kNwLower
   int32_t tile_begin;
+  int32_t hl_n0;                   // >= 0: hi / lo panels only for the tiles at this column of the
+                                   // region (the only ones read before they are rewritten); -1: all
 };
 struct NwParams {
   CUtensorMap tmap;                // the workspace as 128-byte rows (see GemmParams)
@@ -291,6 +294,9 @@ struct NwParams {
   uint32_t *status;
   long long wait_limit;
   int32_t nprob, total_tiles;
+  int32_t late_wait;               // 1: the inputs were complete when the previous kernel let this
+                                   // one start, so it runs beside that kernel and waits for it at the end
+  int32_t pad_;
   NwProb prob[kMaxNwProb];
 };
 
@@ -342,7 +348,9 @@ cudaError_t encode_ws_tensor_map(CUtensorMap *map, void *ws, size_t bytes);
 cudaError_t launch_gemm_f32(const F32Params &p, cudaStream_t s);
 cudaError_t launch_pack_panels(const PackParams &p, cudaStream_t s);
 cudaError_t launch_ridge(const CholParams &p, cudaStream_t s);
-cudaError_t launch_newton_gemm(const NwParams &p, int num_sms, cudaStream_t s);
+// reserve_pairs: SM pairs left to a kernel that runs beside this one (the grid is that much
+// smaller, so that every CTA pair is resident from the start).
+cudaError_t launch_newton_gemm(const NwParams &p, int num_sms, cudaStream_t s, int reserve_pairs = 0);
 cudaError_t launch_split(const SplitParams &p, cudaStream_t s);
 cudaError_t launch_potrf_diag(const DiagParams &p, cudaStream_t s);
 
