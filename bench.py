@@ -765,8 +765,9 @@ def report(args, w: Workload, r, world, cpu):
     })
     if w.tile:
         line["config"]["tile"] = w.tile
-    # Streaming kernels: algorithmic HBM bytes momentum 12 B/elem (G 2 + M 4 + 4 + U 2),
-    # apply 6 B/elem (W 2 + 2, O 2); the partials pass (reduce) re-reads W and O.
+    # Streaming kernels: algorithmic HBM bytes momentum 14 B/elem (G 2 + M 4 + 4 + U 4: the NS
+    # input X0 is written as a bf16 hi + lo pair, the compensated chain's fp32-accurate start),
+    # apply 6 B/elem (W 2 + 2, O 2); reduce (fp32 weights only) re-reads W and O.
     mom_ms, apply_ms, red_ms = kms("momentum"), kms("apply"), kms("reduce")
     if w.step == "adamh":
         adam_ms = kms("adam")
@@ -782,10 +783,11 @@ def report(args, w: Workload, r, world, cpu):
         line["fused_gbs"] = None if fused is None else round(fused, 1)
     else:
         fused_ms = mom_ms + apply_ms + red_ms
-        fused = 18.0 * n / (fused_ms * 1e-3) / 1e9 if fused_ms > 0 else None
+        fused = 20.0 * n / (fused_ms * 1e-3) / 1e9 if fused_ms > 0 else None
         line["fused_gbs"] = None if fused is None else round(fused, 1)
         line["fused_frac_of_hbm"] = None if fused is None else round(fused / peak_bw, 4)
-        line["momentum_gbs"] = round(12.0 * n / (mom_ms * 1e-3) / 1e9, 1) if mom_ms > 0 else None
+        line["momentum_gbs"] = round(14.0 * n / (mom_ms * 1e-3) / 1e9, 1) if mom_ms > 0 else None
+        line["apply_gbs"] = round(6.0 * n / (apply_ms * 1e-3) / 1e9, 1) if apply_ms > 0 else None
         flops = work_flops(w)
         if w.step == "himuon" and w.tile in (128, 256):
             kinds, kname = ("gram",), f"himuon_tile{'128' if w.tile == 128 else ''}_kernel (tile-resident NS, T={w.tile})"

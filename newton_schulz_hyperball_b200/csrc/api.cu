@@ -416,7 +416,6 @@ nshb_status run_momentum(const nshb_matrix *mats, const Plan &pl, const nshb_par
     mp.ws = ws;
     mp.partials = k1part + kK1PartsPerBlock * (int64_t)pl.mp[c0].k1_begin;
     mp.status = reinterpret_cast<uint32_t *>(ws);
-    mp.wait_limit = (p->debug_flags & 1u) ? kWaitLimitTest : kWaitLimit;
     mp.beta = p->beta;
     mp.nesterov = p->nesterov ? 1 : 0;
     mp.nmat = c1 - c0;
@@ -816,7 +815,6 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
     mp.ws = ws;
     mp.partials = reinterpret_cast<double *>(ws + pl.k1part_off);
     mp.status = status;
-    mp.wait_limit = limit;
     mp.beta = p->beta;
     mp.nesterov = p->nesterov ? 1 : 0;
     mp.nmat = c1 - c0;

@@ -139,23 +139,29 @@ constexpr int kBS = 36;                   // row stride of a block (floats): con
 constexpr int kBlk = 32 * kBS + 4;        // block stride (floats): consecutive blocks start 4 banks apart
 constexpr int kNBlk = kNB * (kNB + 1) / 2;
 constexpr int kDiagThreads = 512, kDiagWarps = kDiagThreads / 32;
-constexpr int kDiagSmem = kNBlk * kBlk * 4;
+constexpr int kLtStride = 64;             // L^T scratch of the diagonal factor: 32 shifted rows
+constexpr int kPartSlots = 10;            // partial sums of the split block-row products (at most 10)
+constexpr int kDiagSmem = (kNBlk * kBlk + 32 * kLtStride + 128 + kPartSlots * 1024) * 4;
 static_assert(kDiagSmem <= 227 * 1024, "diagonal block does not fit in shared memory");
 
 __device__ __forceinline__ float *blk(float *sm, int i, int k) { return sm + (i * (i + 1) / 2 + k) * kBlk; }
 
-// acc[x][e] += sum_q A[g + 8x][q] B[h + 4e][q]   (A B^T;  g = lane / 4, h = lane % 4)
-__device__ __forceinline__ void nt_acc(const float *A, const float *B, float (&acc)[4][8]) {
+// Block products on one warp.  The warp computes rows r0 + g + 8x (x < NX; g = lane / 4) of a
+// 32 x 32 output, NX rows and eight columns per lane (NX = 4, r0 = 0: a whole block).  Reads
+// are 16-byte rows of distinct banks, or broadcasts.
+// acc[x][e] += sum_q A[r0 + g + 8x][q] B[h + 4e][q]   (A B^T;  h = lane % 4)
+template <int NX>
+__device__ __forceinline__ void nt_acc(const float *A, const float *B, float (&acc)[NX][8], int r0 = 0) {
   const int lane = threadIdx.x & 31, g = lane >> 2, h = lane & 3;
 #pragma unroll 2
   for (int q = 0; q < 32; q += 4) {
-    float4 a[4], b[8];
+    float4 a[NX], b[8];
 #pragma unroll
-    for (int x = 0; x < 4; ++x) a[x] = *reinterpret_cast<const float4 *>(A + (g + 8 * x) * kBS + q);
+    for (int x = 0; x < NX; ++x) a[x] = *reinterpret_cast<const float4 *>(A + (r0 + g + 8 * x) * kBS + q);
 #pragma unroll
     for (int e = 0; e < 8; ++e) b[e] = *reinterpret_cast<const float4 *>(B + (h + 4 * e) * kBS + q);
 #pragma unroll
-    for (int x = 0; x < 4; ++x)
+    for (int x = 0; x < NX; ++x)
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         float t = acc[x][e];
@@ -167,21 +173,22 @@ __device__ __forceinline__ void nt_acc(const float *A, const float *B, float (&a
   }
 }
 
-// acc[x][e] += sum_q A[g + 8x][q] B[q][8h + e]   (A B)
-__device__ __forceinline__ void nn_acc(const float *A, const float *B, float (&acc)[4][8]) {
+// acc[x][e] += sum_q A[r0 + g + 8x][q] B[q][8h + e]   (A B)
+template <int NX>
+__device__ __forceinline__ void nn_acc(const float *A, const float *B, float (&acc)[NX][8], int r0 = 0) {
   const int lane = threadIdx.x & 31, g = lane >> 2, h = lane & 3;
 #pragma unroll 2
   for (int q = 0; q < 32; q += 4) {
-    float4 a[4];
+    float4 a[NX];
 #pragma unroll
-    for (int x = 0; x < 4; ++x) a[x] = *reinterpret_cast<const float4 *>(A + (g + 8 * x) * kBS + q);
+    for (int x = 0; x < NX; ++x) a[x] = *reinterpret_cast<const float4 *>(A + (r0 + g + 8 * x) * kBS + q);
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       const float4 b0 = *reinterpret_cast<const float4 *>(B + (q + t) * kBS + 8 * h);
       const float4 b1 = *reinterpret_cast<const float4 *>(B + (q + t) * kBS + 8 * h + 4);
       const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int x = 0; x < 4; ++x) {
+      for (int x = 0; x < NX; ++x) {
         const float av = t == 0 ? a[x].x : t == 1 ? a[x].y : t == 2 ? a[x].z : a[x].w;
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[x][e] = fmaf(av, b[e], acc[x][e]);
@@ -190,27 +197,36 @@ __device__ __forceinline__ void nn_acc(const float *A, const float *B, float (&a
   }
 }
 
-__device__ __forceinline__ void zero_acc(float (&acc)[4][8]) {
+template <int NX>
+__device__ __forceinline__ void zero_acc(float (&acc)[NX][8]) {
 #pragma unroll
-  for (int x = 0; x < 4; ++x)
+  for (int x = 0; x < NX; ++x)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[x][e] = 0.f;
 }
 
 // Stores sgn * acc into a block, in the element order of nt_acc (nt) or nn_acc.
-__device__ __forceinline__ void put_acc(float *C, const float (&acc)[4][8], float sgn, bool nt) {
+template <int NX>
+__device__ __forceinline__ void put_acc(float *C, const float (&acc)[NX][8], float sgn, bool nt, int r0 = 0) {
   const int lane = threadIdx.x & 31, g = lane >> 2, h = lane & 3;
 #pragma unroll
-  for (int x = 0; x < 4; ++x)
+  for (int x = 0; x < NX; ++x)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) C[(g + 8 * x) * kBS + (nt ? h + 4 * e : 8 * h + e)] = sgn * acc[x][e];
+    for (int e = 0; e < 8; ++e) C[(r0 + g + 8 * x) * kBS + (nt ? h + 4 * e : 8 * h + e)] = sgn * acc[x][e];
 }
 
 // One warp: block B (32 x 32, lower triangle read) is replaced by D = L^-1, where B = L L^T.
-// Cholesky with row r in lane r's registers (pivot and column broadcast by shuffles); then L^T
-// goes to B (reciprocal on the diagonal) and lane c solves column c of D by forward
-// substitution, D[q][c] = (e_c - sum_{p < q} L[q][p] D[p][c]) / L[q][q].
-__device__ void chol_inv_block(float *B, uint32_t *status) {
+// Right-looking Cholesky with row r in lane r's registers, shifted by one column per step so
+// that the current column is always a[0] and the loop body is the same for every step.  The
+// column of L that every lane needs is exchanged through shared memory (each lane stores its
+// entry already shifted, so the reads are eight aligned 16-byte broadcasts) instead of 31
+// dependent shuffles; the lane that holds the next pivot computes it from its own L entry as
+// soon as it has one (the same fma as its update below), so only one shuffle per step sits on
+// the chain of pivots.  Row j of L^T is kept shifted the same way in LT (LT[j][k] = L[j + k][j],
+// LT[j][0] = 1 / L[j][j], which is the pivot's rsqrt; entries past row 31 are never used), and
+// lane c then solves column c
+// of D by forward substitution, D[q][c] = (e_c - sum_{p < q} L[q][p] D[p][c]) / L[q][q].
+__device__ void chol_inv_block(float *B, float *LT, float *xv, uint32_t *status) {
   const int lane = threadIdx.x & 31;
   float a[32];
 #pragma unroll
@@ -219,54 +235,92 @@ __device__ void chol_inv_block(float *B, uint32_t *status) {
     a[c] = v.x; a[c + 1] = v.y; a[c + 2] = v.z; a[c + 3] = v.w;
   }
   bool bad = false;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    float piv = __shfl_sync(0xffffffffu, a[j], j);
+  float pn = a[0];                                      // lane j's pivot at step j
+#pragma unroll 1
+  for (int j = 0; j < 32; ++j) {                       // a[k] = current A[lane][j + k]
+    float piv = __shfl_sync(0xffffffffu, pn, j);
     bad |= !(piv > 0.f);
     piv = piv > 0.f ? piv : 1e-30f;
-    const float l = lane > j ? a[j] * rsqrtf(piv) : lane == j ? piv * rsqrtf(piv) : 0.f;
-    a[j] = l;
+    const float rs = rsqrtf(piv);
+    const float l = lane > j ? a[0] * rs : lane == j ? piv * rs : 0.f;   // L[lane][j]
+    pn = fmaf(-l, l, a[1]);       // this lane's a[0] after the update below: lane j + 1's next pivot
+    float *v = xv + 64 * (j & 1);                       // two buffers: step j + 1 writes the other
+    v[(lane - j - 1) & 63] = l;                         // v[c - 1] = L[j + c][j]
+    LT[j * kLtStride + ((lane - j) & 63)] = lane == j ? rs : l;   // 1 / L[j][j] = rsqrt(pivot)
+    __syncwarp();
 #pragma unroll
-    for (int c = j + 1; c < 32; ++c) a[c] = fmaf(-l, __shfl_sync(0xffffffffu, l, c), a[c]);
+    for (int c4 = 0; c4 < 32; c4 += 4) {
+      const float4 w = *reinterpret_cast<const float4 *>(v + c4);
+      const float wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (c4 + u < 31) a[c4 + u] = fmaf(-l, wv[u], a[c4 + u + 1]);
+    }
+    a[31] = 0.f;
   }
   if (bad && lane == 0) set_status(status, 0x10u);
   __syncwarp();
-#pragma unroll
-  for (int c = 0; c < 32; ++c) B[c * kBS + lane] = c < lane ? a[c] : c == lane ? 1.f / a[c] : 0.f;
-  __syncwarp();
-  float d[32];
+  float d[32];                                          // d[k] = pending D[q + k][lane]
 #pragma unroll
   for (int i = 0; i < 32; ++i) d[i] = i == lane ? 1.f : 0.f;
-#pragma unroll
+#pragma unroll 1
   for (int q = 0; q < 32; ++q) {
-    const float *lt = B + q * kBS;                      // row q of L^T: L[i][q] at i
-    d[q] *= lt[q];
+    const float *lt = LT + q * kLtStride;
+    float w[32];
 #pragma unroll
-    for (int i4 = (q + 1) & ~3; i4 < 32; i4 += 4) {
-      const float4 v = *reinterpret_cast<const float4 *>(lt + i4);
-      const float w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (i4 + u > q) d[i4 + u] = fmaf(-w[u], d[q], d[i4 + u]);
+    for (int k4 = 0; k4 < 32; k4 += 4) {
+      const float4 t = *reinterpret_cast<const float4 *>(lt + k4);
+      w[k4] = t.x; w[k4 + 1] = t.y; w[k4 + 2] = t.z; w[k4 + 3] = t.w;
     }
-  }
-  __syncwarp();
+    const float dq = d[0] * w[0];
+    B[q * kBS + lane] = dq;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) B[i * kBS + lane] = d[i];
+    for (int k = 1; k < 32; ++k) d[k - 1] = fmaf(-w[k], dq, d[k]);
+    d[31] = 0.f;
+  }
   __syncwarp();
 }
 
-// Block row J of D over `nw` warps starting at warp w0 (J <= 7 < nw: at most one block each):
-// D_Jk = -sum_{k <= m < J} X_Jm D_mk, written in place of X_Jk once every participating warp
-// has read its operands (named barrier 1 over the nw warps).
-__device__ void drow(float *sm, int J, int w0, int nw) {
-  const int k = (int)(threadIdx.x >> 5) - w0;
+// Block row J of D over `nw` warps starting at warp w0: D_Jk = -sum_{k <= m < J} X_Jm D_mk,
+// each sum cut into pieces of one product (when the J (J + 1) / 2 products fit the warps) or
+// two, k-major, one piece per warp (at most 16 pieces for J <= 7).  The pieces after the first
+// of a sum leave their partial in a scratch slot; after every participating warp has read its
+// operands (named barrier 1 over the nw warps), the first piece adds them in order and writes
+// the block in place of X_Jk.
+__device__ void drow(float *sm, float *part, int J, int w0, int nw) {
+  const int w = (int)(threadIdx.x >> 5) - w0, lane = threadIdx.x & 31;
+  const int sz = J * (J + 1) / 2 <= nw ? 1 : 2;
+  int k = 0, p = 0, first = 0, np = 0;                  // this warp's piece: sum k, piece p of np
+  bool mine = false;
+  for (int kk = 0, idx = 0; kk < J; ++kk) {
+    const int n = (J - kk + sz - 1) / sz;
+    if (w >= idx && w < idx + n) {
+      k = kk; p = w - idx; first = idx; np = n; mine = true;
+    }
+    idx += n;
+  }
   float acc[4][8];
   zero_acc(acc);
-  if (k < J)
-    for (int m = k; m < J; ++m) nn_acc(blk(sm, J, m), blk(sm, m, k), acc);
+  if (mine)
+    for (int m = k + sz * p; m < min(J, k + sz * p + sz); ++m) nn_acc(blk(sm, J, m), blk(sm, m, k), acc);
+  if (mine && p > 0) {
+    float *slot = part + (first + p - (k + 1)) * 1024;
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) slot[(8 * x + e) * 32 + lane] = acc[x][e];
+  }
   asm volatile("bar.sync 1, %0;" ::"r"(nw * 32) : "memory");
-  if (k < J) put_acc(blk(sm, J, k), acc, -1.f, false);
+  if (mine && p == 0) {
+    for (int q = 1; q < np; ++q) {
+      const float *slot = part + (first + q - (k + 1)) * 1024;
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[x][e] += slot[(8 * x + e) * 32 + lane];
+    }
+    put_acc(blk(sm, J, k), acc, -1.f, false);
+  }
 }
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
@@ -286,19 +340,27 @@ __global__ void __launch_bounds__(kDiagThreads, 1) potrf_diag_kernel(const __gri
   const float *S = reinterpret_cast<const float *>(p.ws + p.s32[z]);
   char *hi = p.ws + p.dhi[z], *lo = p.ws + p.dlo[z];
   const int warp = threadIdx.x >> 5;
-  // the 36 lower blocks: 32 rows of eight 16-byte pieces each
-  for (int q = threadIdx.x; q < kNBlk * 256; q += kDiagThreads) {
-    const int b = q >> 8, r = (q >> 3) & 31, c4 = q & 7;
-    int i = 0, k = b;
+  float *LT = sm + kNBlk * kBlk, *xv = LT + 32 * kLtStride, *part = xv + 128;
+  // the 36 lower blocks, 32 rows of eight 16-byte pieces each: block column 0 first (all that
+  // step 0's factor and panel read), the other 28 blocks as a second group that lands while
+  // the first diagonal block is factored
+  auto load_blk = [&](int i, int k, int r, int c4) {
+    cp_async16(blk(sm, i, k) + r * kBS + 4 * c4, S + (int64_t)(k0 + 32 * i + r) * ld + k0 + 32 * k + 4 * c4);
+  };
+  for (int q = threadIdx.x; q < kNB * 256; q += kDiagThreads) load_blk(q >> 8, 0, (q >> 3) & 31, q & 7);
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  for (int q = threadIdx.x; q < (kNBlk - kNB) * 256; q += kDiagThreads) {
+    int i = 0, k = q >> 8;
     while (k > i) k -= ++i;
-    cp_async16(sm + b * kBlk + r * kBS + 4 * c4, S + (int64_t)(k0 + 32 * i + r) * ld + k0 + 32 * k + 4 * c4);
+    load_blk(i + 1, k + 1, (q >> 3) & 31, q & 7);
   }
-  asm volatile("cp.async.wait_all;" ::: "memory");
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
   __syncthreads();
   for (int j = 0; j < kNB; ++j) {
     // A: factor and invert the diagonal block; finish block row j - 1 of D beside it
-    if (warp == 0) chol_inv_block(blk(sm, j, j), p.status);
-    else if (j >= 2) drow(sm, j - 1, 1, kDiagWarps - 1);
+    if (warp == 0) chol_inv_block(blk(sm, j, j), LT, xv, p.status);
+    else if (j >= 2) drow(sm, part, j - 1, 1, kDiagWarps - 1);
     __syncthreads();
     // B: the panel below (7 - j blocks) and block row j of X (j blocks), one block per warp
     if (warp < kNB - 1) {
@@ -316,6 +378,7 @@ __global__ void __launch_bounds__(kDiagThreads, 1) potrf_diag_kernel(const __gri
       __syncwarp();
       put_acc(C, acc, 1.f, panel);
     }
+    if (j == 0) asm volatile("cp.async.wait_group 0;" ::: "memory");   // the trailing blocks
     __syncthreads();
     // C: trailing update of the blocks right of and below the panel
     const int n = kNB - 1 - j;
@@ -335,7 +398,7 @@ __global__ void __launch_bounds__(kDiagThreads, 1) potrf_diag_kernel(const __gri
     }
     __syncthreads();
   }
-  drow(sm, kNB - 1, 0, kDiagWarps);
+  drow(sm, part, kNB - 1, 0, kDiagWarps);
   __syncthreads();
   // out: rows k0 .. k0+255, columns 0 .. 255 of the stack, eight columns per 16-byte piece
   for (int q = threadIdx.x; q < 256 * 32; q += kDiagThreads) {

@@ -69,7 +69,6 @@ struct MomentumParams {
   char *ws;
   double *partials;  // kK1PartsPerBlock per block of the launch
   uint32_t *status;
-  long long wait_limit;  // clock cycles per mbarrier phase (bulk-copy variant)
   float beta;
   int32_t nesterov;
   int32_t nmat, total_blocks;

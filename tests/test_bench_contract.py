@@ -67,9 +67,11 @@ def test_default_line_is_the_qwen3_muonh_set(monkeypatch, capsys):
     gemm_ms = 12.0 + 9.0 + 27.0
     assert abs(bench.ns_flops(QWEN) / 1e12 - 47.80) < 0.01
     assert abs(line["ns_tflops"] - bench.ns_flops(QWEN) / (gemm_ms * 1e-3) / 1e12) < 0.1
-    # fused streaming bytes: 18 B/elem over momentum + reduce + apply
+    # fused streaming bytes: 20 B/elem (momentum 14 with X0's low part, apply 6) over
+    # momentum + reduce + apply
     n = 1409286144
-    assert abs(line["fused_gbs"] - 18.0 * n / ((2.5 + 1.4 + 1.3) * 1e-3) / 1e9) < 1.0
+    assert abs(line["fused_gbs"] - 20.0 * n / ((2.5 + 1.4 + 1.3) * 1e-3) / 1e9) < 1.0
+    assert abs(line["momentum_gbs"] - 14.0 * n / (2.5e-3) / 1e9) < 1.0
     assert line["gpu_launches"] == 22 * 20
     assert line["clocks"]["reasons"] == ["sw_power_cap"]
     assert line["e2e"]["h2d_bytes_per_step"] == 2 * n and line["e2e"]["d2h_bytes_per_step"] == 4

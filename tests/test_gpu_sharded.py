@@ -65,3 +65,28 @@ def test_sharded_step_equals_unsharded_bitwise(kind, kw):
     assert one.device_status() == 0
     for i in range(len(shapes)):
         assert torch.equal(Wb[i], Wa[i]), i
+
+
+@pytest.mark.parametrize("kind,kw", [("hyperball", {}), ("himuon", {"tile": 256})])
+def test_a_ragged_neighbour_does_not_change_a_matrix_bitwise(kind, kw):
+    """A matrix's step does not depend on the other matrices of its call: adding a ragged
+    matrix (element-wise loads and masked blocks in the same launches) leaves the results of
+    the aligned ones bit for bit unchanged, momentum buffers included."""
+    aligned = [(768, 768), (3072, 768), (768, 3072), (1024, 4096)]
+    W, G = device_set(aligned + [(300, 700)], 73)
+    rho = torch.stack([w.float().norm() for w in W])
+    op = nshb.NSHB_OP_HYPERBALL if kind == "hyperball" else nshb.NSHB_OP_HIMUON
+    outs = []
+    for n in (len(aligned), len(aligned) + 1):
+        Wc = [w.clone() for w in W[:n]]
+        Mc = [torch.zeros(w.shape, dtype=torch.float32, device=DEV) for w in W[:n]]
+        mats = nshb.matrices(Wc, G[:n], Mc)
+        p = nshb.params(rho=rho[:n].contiguous(), **kw)
+        ws = nshb.workspace(mats, p, op)
+        for _ in range(2):
+            getattr(nshb, kind + "_step")(mats, p, ws)
+        assert nshb.device_status(ws) == 0
+        outs.append((Wc, Mc))
+    for i in range(len(aligned)):
+        assert torch.equal(outs[0][1][i], outs[1][1][i]), i
+        assert torch.equal(outs[0][0][i], outs[1][0][i]), i
