@@ -1027,11 +1027,15 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
     e = run_diag(k + 1);
     if (e != NSHB_OK) return e;
     // beside the diagonal blocks: one SM per block is taken, and a few pairs more for the
-    // SMs that the pairing leaves single
+    // SMs that the pairing leaves single.  When that would take more than a quarter of the
+    // pairs, nothing is reserved: the pairs that find no SM start when the diagonal blocks
+    // end, which costs what running the two in turn costs.
     int ndiag = 0;
     for (auto &z : pl.zp) ndiag += z.Dp > k1 ? 1 : 0;
+    int reserve = (ndiag + 1) / 2 + 4;
+    if (4 * reserve > device_sms() / 2) reserve = 0;
     np.late_wait = 1;
-    e = run_nw(np, trail_u, st, (ndiag + 1) / 2 + 4);
+    e = run_nw(np, trail_u, st, reserve);
     np.late_wait = 0;
     if (e != NSHB_OK) return e;
   }

@@ -232,12 +232,16 @@ __global__ void __launch_bounds__(kThreads, 1) newton_gemm_kernel(const __grid_c
       const float *crow = sub ? reinterpret_cast<const float *>(p.ws + q.c32) + i * q.ld32 + t.n0 : nullptr;
       float *drow = q.d32 >= 0 ? reinterpret_cast<float *>(p.ws + q.d32) + i * q.ld32 + t.n0 : nullptr;
       const bool valid = i < q.m_valid;                   // rows past the valid region are not written
-      // C of columns col0 .. col0+31 (issued a chunk ahead of its use)
+      // C of columns col0 .. col0+31 (issued a chunk ahead of its use).  A thread owns one row,
+      // so a warp access touches 32 lines: 32-byte accesses move twice the bytes per L1
+      // wavefront of 16-byte ones (rows and tiles are 32-byte aligned).
       auto load_c = [&](int col0, float (&c)[32]) {
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const float4 v = *reinterpret_cast<const float4 *>(crow + col0 + 4 * g);
-          c[4 * g] = v.x; c[4 * g + 1] = v.y; c[4 * g + 2] = v.z; c[4 * g + 3] = v.w;
+        for (int g = 0; g < 4; ++g) {
+          uint32_t w[8];
+          ld_global_256(crow + col0 + 8 * g, w);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) c[8 * g + e] = __uint_as_float(w[e]);
         }
       };
       float c[32];
@@ -261,8 +265,12 @@ __global__ void __launch_bounds__(kThreads, 1) newton_gemm_kernel(const __grid_c
         const int cvalid = q.n_valid - (t.n0 + col0);       // columns of this chunk that exist
         if (drow && valid && cvalid >= 32) {
 #pragma unroll
-          for (int g = 0; g < 8; ++g)
-            *reinterpret_cast<float4 *>(drow + col0 + 4 * g) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+          for (int g = 0; g < 4; ++g) {
+            uint32_t w[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w[e] = __float_as_uint(v[8 * g + e]);
+            st_global_256(drow + col0 + 8 * g, w);
+          }
         } else if (drow && valid) {
 #pragma unroll
           for (int e = 0; e < 32; ++e)
