@@ -946,10 +946,15 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
   int64_t dmax = 0;
   for (auto &z : pl.zp) dmax = std::max(dmax, z.Dp);
   const int nb = (int)(dmax / 256);
-  // 4. forward: blocked right-looking Cholesky S = L L^T with the rows of every U carried
-  //    along, so that block column k of Y = U L^-T is final after step k.  The diagonal
-  //    block of step k + 1 needs only step k's update of S, so it is factored while step k's
-  //    update of U runs: launches diag(0), then per step panel(k), S(k), diag(k + 1), U(k).
+  // 4. forward, left-looking by block columns of 256.  Block column k of S is brought up to
+  //    date by one product over every earlier column of L, T = S[k0:, k] - L[k0:, :k] L[k, :k]^T;
+  //    its diagonal block is factored and inverted (D_k); the panel L[k1:, k] = T[k1:] D_k^T
+  //    follows.  The rows of every U are carried along the same way: V = U[:, k] - Y[:, :k]
+  //    L[k, :k]^T, Y[:, k] = V D_k^T.  Every fp32 element of S and U is read and written once
+  //    (a right-looking order rewrites the whole trailing matrix at every step).  Launches per
+  //    step: S column (k > 0), diagonal blocks, U column (k > 0; it needs only earlier columns,
+  //    so it runs beside the diagonal blocks, starting without waiting and waiting for them at
+  //    its end), panel.
   auto run_diag = [&](int k) -> nshb_status {
     const int64_t k0 = 256LL * k;
     for (int c0 = 0; c0 < nz; c0 += kMaxMats) {
@@ -971,35 +976,50 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
     }
     return NSHB_OK;
   };
-  nshb_status ed = run_diag(0);
-  if (ed != NSHB_OK) return ed;
   for (int k = 0; k < nb; ++k) {
     const int64_t k0 = 256LL * k, k1 = k0 + 256;
-    // panel: L[k1:, k] = S[k1:, k] D_k^T and Y[:, k] = U[:, k] D_k^T
-    std::vector<NwProb> panel, trail_s, trail_u;
+    std::vector<NwProb> col_s, col_u, panel;
+    int ndiag = 0;
     for (auto &z : pl.zp) {
+      if (z.Dp <= k0) continue;
+      ++ndiag;
+      if (k > 0) {
+        // T = S[k0:, k] - L[k0:, :k] L[k0:k1, :k]^T, fp32 in place and as hi / lo panels
+        NwProb t = nw_prob();
+        t.a_hi = z.lh; t.a_lo = z.ll; t.a_ph = (int)z.Dp; t.a_r0 = (int)k0; t.a_k0 = 0;
+        t.b_hi = z.lh; t.b_lo = z.ll; t.b_ph = (int)z.Dp; t.b_r0 = (int)k0; t.b_k0 = 0;
+        t.kt = (int)(k0 / 64);
+        t.c32 = t.d32 = z.s + (k0 * z.Dp + k0) * 4; t.ld32 = (int)z.Dp;
+        t.m_valid = (int)(z.Dp - k0); t.n_valid = 256;
+        t.dhi = z.sh; t.dlo = z.sl; t.d_ph = (int)z.Dp; t.d_r0 = (int)k0; t.d_c0 = (int)k0;
+        t.mt = (int)((z.Dp - k0) / 256); t.nt = 1;
+        col_s.push_back(t);
+      }
       if (z.Dp <= k1) continue;
+      // L[k1:, k] = T[k1:] D_k^T
       NwProb q = nw_prob();
       q.a_hi = z.sh; q.a_lo = z.sl; q.a_ph = (int)z.Dp; q.a_r0 = (int)k1; q.a_k0 = (int)k0;
       q.b_hi = z.dh; q.b_lo = z.dl; q.b_ph = (int)z.Dp; q.b_r0 = (int)k0; q.b_k0 = 0;
       q.dhi = z.lh; q.dlo = z.ll; q.d_ph = (int)z.Dp; q.d_r0 = (int)k1; q.d_c0 = (int)k0;
       q.mt = (int)((z.Dp - k1) / 256); q.nt = 1;
       panel.push_back(q);
-      // trailing: S[k1:, k1:] -= L[k1:, k] L[k1:, k]^T (lower tiles), fp32 and panels
-      NwProb t = nw_prob();
-      t.a_hi = z.lh; t.a_lo = z.ll; t.a_ph = (int)z.Dp; t.a_r0 = (int)k1; t.a_k0 = (int)k0;
-      t.b_hi = z.lh; t.b_lo = z.ll; t.b_ph = (int)z.Dp; t.b_r0 = (int)k1; t.b_k0 = (int)k0;
-      t.c32 = t.d32 = z.s + (k1 * z.Dp + k1) * 4; t.ld32 = (int)z.Dp;
-      t.m_valid = t.n_valid = (int)(z.Dp - k1);
-      t.dhi = z.sh; t.dlo = z.sl; t.d_ph = (int)z.Dp; t.d_r0 = (int)k1; t.d_c0 = (int)k1;
-      t.mt = t.nt = (int)((z.Dp - k1) / 256);
-      t.flags = kNwLower;
-      t.hl_n0 = 0;                 // the next panel reads block column k + 1 only
-      trail_s.push_back(t);
     }
     for (int i = 0; i < n; ++i) {
       const Plan::ZPlan &z = pl.zp[pl.zidx[i]];
       if (z.Dp <= k0) continue;
+      if (k > 0) {
+        // V = U[:, k] - Y[:, :k] L[k0:k1, :k]^T, fp32 in place and as hi / lo panels
+        NwProb t = nw_prob();
+        t.a_hi = pl.yh[i]; t.a_lo = pl.yl[i]; t.a_ph = (int)pl.mpad[i]; t.a_r0 = 0; t.a_k0 = 0;
+        t.b_hi = z.lh; t.b_lo = z.ll; t.b_ph = (int)z.Dp; t.b_r0 = (int)k0; t.b_k0 = 0;
+        t.kt = (int)(k0 / 64);
+        t.c32 = t.d32 = pl.y32[i] + k0 * 4; t.ld32 = (int)z.Dp;
+        t.m_valid = (int)pl.mpad[i]; t.n_valid = 256;
+        t.dhi = pl.yh[i]; t.dlo = pl.yl[i]; t.d_ph = (int)pl.mpad[i]; t.d_r0 = 0; t.d_c0 = (int)k0;
+        t.mt = (int)(pl.mpad[i] / 256); t.nt = 1;
+        col_u.push_back(t);
+      }
+      // Y[:, k] = V D_k^T
       NwProb q = nw_prob();
       q.a_hi = pl.yh[i]; q.a_lo = pl.yl[i]; q.a_ph = (int)pl.mpad[i]; q.a_r0 = 0; q.a_k0 = (int)k0;
       q.b_hi = z.dh; q.b_lo = z.dl; q.b_ph = (int)z.Dp; q.b_r0 = (int)k0; q.b_k0 = 0;
@@ -1007,47 +1027,47 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
       q.dhi = pl.yh[i]; q.dlo = pl.yl[i]; q.d_ph = (int)pl.mpad[i]; q.d_r0 = 0; q.d_c0 = (int)k0;
       q.mt = (int)(pl.mpad[i] / 256); q.nt = 1;
       panel.push_back(q);
-      if (z.Dp <= k1) continue;
-      // U[:, k1:] -= Y[:, k] L[k1:, k]^T
-      NwProb t = nw_prob();
-      t.a_hi = pl.yh[i]; t.a_lo = pl.yl[i]; t.a_ph = (int)pl.mpad[i]; t.a_r0 = 0; t.a_k0 = (int)k0;
-      t.b_hi = z.lh; t.b_lo = z.ll; t.b_ph = (int)z.Dp; t.b_r0 = (int)k1; t.b_k0 = (int)k0;
-      t.c32 = t.d32 = pl.y32[i] + k1 * 4; t.ld32 = (int)z.Dp;
-      t.m_valid = (int)pl.mpad[i]; t.n_valid = (int)(z.Dp - k1);
-      t.dhi = pl.yh[i]; t.dlo = pl.yl[i]; t.d_ph = (int)pl.mpad[i]; t.d_r0 = 0; t.d_c0 = (int)k1;
-      t.mt = (int)(pl.mpad[i] / 256); t.nt = (int)((z.Dp - k1) / 256);
-      t.hl_n0 = 0;
-      trail_u.push_back(t);
     }
-    nshb_status e = run_nw(np, panel, st);
+    nshb_status e = run_nw(np, col_s, st);
     if (e != NSHB_OK) return e;
-    e = run_nw(np, trail_s, st);
+    e = run_diag(k);
     if (e != NSHB_OK) return e;
-    if (k + 1 == nb) continue;
-    e = run_diag(k + 1);
-    if (e != NSHB_OK) return e;
-    // beside the diagonal blocks: one SM per block is taken, and a few pairs more for the
-    // SMs that the pairing leaves single.  When that would take more than a quarter of the
-    // pairs, nothing is reserved: the pairs that find no SM start when the diagonal blocks
-    // end, which costs what running the two in turn costs.
-    int ndiag = 0;
-    for (auto &z : pl.zp) ndiag += z.Dp > k1 ? 1 : 0;
+    // beside the diagonal blocks: one SM per block is taken, and a few pairs more for the SMs
+    // that the pairing leaves single.  When that would take more than a quarter of the pairs,
+    // nothing is reserved: the pairs that find no SM start when the diagonal blocks end, which
+    // costs what running the two in turn costs.
     int reserve = (ndiag + 1) / 2 + 4;
     if (4 * reserve > device_sms() / 2) reserve = 0;
     np.late_wait = 1;
-    e = run_nw(np, trail_u, st, reserve);
+    e = run_nw(np, col_u, st, reserve);
     np.late_wait = 0;
     if (e != NSHB_OK) return e;
+    e = run_nw(np, panel, st);
+    if (e != NSHB_OK) return e;
   }
-  // 5. backward: P L = Y, right-looking from the last block: P[:, k] = Y[:, k] D_k (fp32 into
-  //    the m x n buffer the momentum pass reads, and panels), then Y[:, :k] -= P[:, k] L[k, :k]
+  // 5. backward, P L = Y by block columns from the last, left-looking as well:
+  //    W = Y[:, k] - P[:, k1:] L[k1:, k] (one product over every later column of P; only its
+  //    hi / lo panels are kept, in place of Y[:, k]), then P[:, k] = W D_k (fp32 into the m x n
+  //    buffer the momentum pass reads, and hi / lo panels in place of W).
   for (int k = nb - 1; k >= 0; --k) {
-    const int64_t k0 = 256LL * k;
-    std::vector<NwProb> solve, upd;
+    const int64_t k0 = 256LL * k, k1 = k0 + 256;
+    std::vector<NwProb> col_p, solve;
     for (int i = 0; i < n; ++i) {
       const Plan::ZPlan &z = pl.zp[pl.zidx[i]];
       if (z.Dp <= k0) continue;
       const int d = (int)pl.mp[i].n, m = (int)pl.mp[i].m;
+      if (z.Dp > k1) {
+        NwProb t = nw_prob();
+        t.a_hi = pl.yh[i]; t.a_lo = pl.yl[i]; t.a_ph = (int)pl.mpad[i]; t.a_r0 = 0; t.a_k0 = (int)k1;
+        t.b_hi = z.lh; t.b_lo = z.ll; t.b_ph = (int)z.Dp; t.b_r0 = (int)k0; t.b_k0 = (int)k1;
+        t.kt = (int)((z.Dp - k1) / 64);
+        t.flags = kNwBMn;
+        t.c32 = pl.y32[i] + k0 * 4; t.ld32 = (int)z.Dp;
+        t.m_valid = (int)pl.mpad[i]; t.n_valid = 256;
+        t.dhi = pl.yh[i]; t.dlo = pl.yl[i]; t.d_ph = (int)pl.mpad[i]; t.d_r0 = 0; t.d_c0 = (int)k0;
+        t.mt = (int)(pl.mpad[i] / 256); t.nt = 1;
+        col_p.push_back(t);
+      }
       NwProb q = nw_prob();
       q.a_hi = pl.yh[i]; q.a_lo = pl.yl[i]; q.a_ph = (int)pl.mpad[i]; q.a_r0 = 0; q.a_k0 = (int)k0;
       q.b_hi = z.dh; q.b_lo = z.dl; q.b_ph = (int)z.Dp; q.b_r0 = 0; q.b_k0 = (int)k0;
@@ -1056,20 +1076,10 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
       q.dhi = pl.yh[i]; q.dlo = pl.yl[i]; q.d_ph = (int)pl.mpad[i]; q.d_r0 = 0; q.d_c0 = (int)k0;
       q.mt = (int)(pl.mpad[i] / 256); q.nt = 1;
       solve.push_back(q);
-      if (k == 0) continue;
-      NwProb t = nw_prob();
-      t.a_hi = pl.yh[i]; t.a_lo = pl.yl[i]; t.a_ph = (int)pl.mpad[i]; t.a_r0 = 0; t.a_k0 = (int)k0;
-      t.b_hi = z.lh; t.b_lo = z.ll; t.b_ph = (int)z.Dp; t.b_r0 = 0; t.b_k0 = (int)k0;
-      t.flags = kNwBMn;
-      t.c32 = t.d32 = pl.y32[i]; t.ld32 = (int)z.Dp; t.m_valid = (int)pl.mpad[i]; t.n_valid = (int)k0;
-      t.dhi = pl.yh[i]; t.dlo = pl.yl[i]; t.d_ph = (int)pl.mpad[i]; t.d_r0 = 0; t.d_c0 = 0;
-      t.mt = (int)(pl.mpad[i] / 256); t.nt = k;
-      t.hl_n0 = (int)(k0 - 256);   // the next solve reads block column k - 1 only
-      upd.push_back(t);
     }
-    nshb_status e = run_nw(np, solve, st);
+    nshb_status e = run_nw(np, col_p, st);
     if (e != NSHB_OK) return e;
-    e = run_nw(np, upd, st);
+    e = run_nw(np, solve, st);
     if (e != NSHB_OK) return e;
   }
   return NSHB_OK;
