@@ -758,7 +758,6 @@ NwProb nw_prob() {
   std::memset(&q, 0, sizeof(q));
   q.c32 = q.d32 = q.dhi = q.dlo = -1;
   q.kt = 4;                        // every product is 256 deep (one block column)
-  q.hl_n0 = -1;
   return q;
 }
 

@@ -125,15 +125,15 @@ __global__ void __launch_bounds__(256) split_kernel(const __grid_constant__ Spli
 // triangle lives in shared memory as 36 blocks of 32 x 32 (block (i, k), i >= k); every
 // block is overwritten in turn by L and then by D.  Step j:
 //   A  one warp factors the diagonal block, A_jj = L_jj L_jj^T, and inverts it, D_jj =
-//      L_jj^-1 (L_jj itself is needed by nothing else);  the other warps meanwhile finish
-//      block row j - 1 of D (below);
+//      L_jj^-1 (L_jj itself is needed by nothing else);
 //   B  panel L_ij = A_ij D_jj^T (i > j), and X_jm = D_jj L_jm (m < j: block row j of L is
 //      no longer read by the factorisation);
-//   C  trailing update A_ik -= L_ij L_kj^T (j < k <= i);
-// and block row j of D is  D_jk = -sum_{k <= m < j} X_jm D_mk  (from D L = I), computed
-// during step j + 1 (row 7 at the end).  The result goes out as bf16 hi / lo panels (block k
-// of the inverse stack), with zeros above the diagonal.  A pivot that is not positive in
-// fp32 is flagged (NSHB_DEV_NOT_SPD) and replaced by 1e-30.
+//   C  trailing update A_ik -= L_ij L_kj^T (j < k <= i), and block row j of D,
+//      D_jk = -sum_{k <= m < j} X_jm D_mk  (from D L = I).
+// Step j + 1's A runs inside step j's C: the warp that updates block (j + 1, j + 1) factors
+// it right away while the other warps finish the rest of C.  The result goes out as bf16
+// hi / lo panels (block k of the inverse stack), with zeros above the diagonal.  A pivot that
+// is not positive in fp32 is flagged (NSHB_DEV_NOT_SPD) and replaced by 1e-30.
 constexpr int kNB = 8;                    // block columns
 constexpr int kBS = 36;                   // row stride of a block (floats): conflict-free float4 rows
 constexpr int kBlk = 32 * kBS + 4;        // block stride (floats): consecutive blocks start 4 banks apart
@@ -281,15 +281,20 @@ __device__ void chol_inv_block(float *B, float *LT, float *xv, uint32_t *status)
   __syncwarp();
 }
 
-// Block row J of D over `nw` warps starting at warp w0: D_Jk = -sum_{k <= m < J} X_Jm D_mk,
-// each sum cut into pieces of one product (when the J (J + 1) / 2 products fit the warps) or
-// two, k-major, one piece per warp (at most 16 pieces for J <= 7).  The pieces after the first
+// Block row J of D over `nw` warps (this one is number w of them): D_Jk = -sum_{k <= m < J} X_Jm D_mk,
+// each sum cut into pieces of the fewest products that give every piece a warp (k-major, one
+// piece per warp; at most 10 partial slots for J <= 7 and nw >= 12).  The pieces after the first
 // of a sum leave their partial in a scratch slot; after every participating warp has read its
 // operands (named barrier 1 over the nw warps), the first piece adds them in order and writes
 // the block in place of X_Jk.
-__device__ void drow(float *sm, float *part, int J, int w0, int nw) {
-  const int w = (int)(threadIdx.x >> 5) - w0, lane = threadIdx.x & 31;
-  const int sz = J * (J + 1) / 2 <= nw ? 1 : 2;
+__device__ void drow(float *sm, float *part, int J, int w, int nw) {
+  const int lane = threadIdx.x & 31;
+  int sz = 1;                                           // smallest piece size whose pieces fit the warps
+  for (;; ++sz) {
+    int cnt = 0;
+    for (int kk = 0; kk < J; ++kk) cnt += (J - kk + sz - 1) / sz;
+    if (cnt <= nw) break;
+  }
   int k = 0, p = 0, first = 0, np = 0;                  // this warp's piece: sum k, piece p of np
   bool mine = false;
   for (int kk = 0, idx = 0; kk < J; ++kk) {
@@ -357,11 +362,21 @@ __global__ void __launch_bounds__(kDiagThreads, 1) potrf_diag_kernel(const __gri
   asm volatile("cp.async.commit_group;" ::: "memory");
   asm volatile("cp.async.wait_group 1;" ::: "memory");
   __syncthreads();
+  if (warp == 0) chol_inv_block(blk(sm, 0, 0), LT, xv, p.status);
+  __syncthreads();
+  // A_ik -= L_ij L_kj^T for one block
+  auto trail = [&](int j, int i, int k) {
+    float acc[4][8];
+    zero_acc(acc);
+    nt_acc(blk(sm, i, j), blk(sm, k, j), acc);
+    float *C = blk(sm, i, k);
+    const int lane = threadIdx.x & 31, g = lane >> 2, h = lane & 3;
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) C[(g + 8 * x) * kBS + h + 4 * e] -= acc[x][e];
+  };
   for (int j = 0; j < kNB; ++j) {
-    // A: factor and invert the diagonal block; finish block row j - 1 of D beside it
-    if (warp == 0) chol_inv_block(blk(sm, j, j), LT, xv, p.status);
-    else if (j >= 2) drow(sm, part, j - 1, 1, kDiagWarps - 1);
-    __syncthreads();
     // B: the panel below (7 - j blocks) and block row j of X (j blocks), one block per warp
     if (warp < kNB - 1) {
       float acc[4][8];
@@ -380,26 +395,30 @@ __global__ void __launch_bounds__(kDiagThreads, 1) potrf_diag_kernel(const __gri
     }
     if (j == 0) asm volatile("cp.async.wait_group 0;" ::: "memory");   // the trailing blocks
     __syncthreads();
-    // C: trailing update of the blocks right of and below the panel
+    // C: the trailing update.  Warp 0 updates the next diagonal block first and factors and
+    // inverts it at once (look-ahead: the next step needs nothing else from this one to start
+    // its factor); warps 1..15 update the other blocks and then finish block row j of D.
+    // The other warps of warp 0's sub-partition (4, 8, 12) stay idle, so that its chain of
+    // dependent steps gets every issue slot there.
     const int n = kNB - 1 - j;
-    for (int t = warp; t < n * (n + 1) / 2; t += kDiagWarps) {
-      int ii = 0, kk = t;
-      while (kk > ii) kk -= ++ii;
-      const int i = j + 1 + ii, k = j + 1 + kk;
-      float acc[4][8];
-      zero_acc(acc);
-      nt_acc(blk(sm, i, j), blk(sm, k, j), acc);
-      float *C = blk(sm, i, k);
-      const int lane = threadIdx.x & 31, g = lane >> 2, h = lane & 3;
-#pragma unroll
-      for (int x = 0; x < 4; ++x)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) C[(g + 8 * x) * kBS + h + 4 * e] -= acc[x][e];
+    constexpr int kHelpers = kDiagWarps - kDiagWarps / 4;    // warps 1-3, 5-7, 9-11, 13-15
+    if (warp == 0) {
+      if (n > 0) {
+        trail(j, j + 1, j + 1);
+        __syncwarp();
+        chol_inv_block(blk(sm, j + 1, j + 1), LT, xv, p.status);
+      }
+    } else if (warp & 3) {
+      const int w = warp - warp / 4 - 1;                     // 0 .. kHelpers - 1
+      for (int t = 1 + w; t < n * (n + 1) / 2; t += kHelpers) {   // task 0 is warp 0's block
+        int ii = 0, kk = t;
+        while (kk > ii) kk -= ++ii;
+        trail(j, j + 1 + ii, j + 1 + kk);
+      }
+      if (j >= 1) drow(sm, part, j, w, kHelpers);
     }
     __syncthreads();
   }
-  drow(sm, part, kNB - 1, 0, kDiagWarps);
-  __syncthreads();
   // out: rows k0 .. k0+255, columns 0 .. 255 of the stack, eight columns per 16-byte piece
   for (int q = threadIdx.x; q < 256 * 32; q += kDiagThreads) {
     const int r = q >> 5, c = 8 * (q & 31), i = r >> 5, k = c >> 5;

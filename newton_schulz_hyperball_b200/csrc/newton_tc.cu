@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1) newton_gemm_kernel(const __grid_c
           for (int e = 0; e < 32; ++e)
             if (e < cvalid) drow[col0 + e] = v[e];
         }
-        if (q.dhi >= 0 && (q.hl_n0 < 0 || t.n0 == q.hl_n0)) {
+        if (q.dhi >= 0) {
           const int64_t pr = q.d_r0 + i;                    // row and column in D's panels
           const int64_t pc = q.d_c0 + t.n0 + col0;
           const bool odd = pr & 1;

@@ -284,8 +284,6 @@ struct NwProb {
   int32_t mt, nt, kt;              // 256-row tiles, 256-column tiles, 64-deep k panels (even)
   int32_t flags;                   // kNwBMn | kNwLower
   int32_t tile_begin;
-  int32_t hl_n0;                   // >= 0: hi / lo panels only for the tiles at this column of the
-                                   // region (the only ones read before they are rewritten); -1: all
 };
 struct NwParams {
   CUtensorMap tmap;                // the workspace as 128-byte rows (see GemmParams)
