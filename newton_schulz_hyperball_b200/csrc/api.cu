@@ -946,14 +946,16 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
   for (auto &z : pl.zp) dmax = std::max(dmax, z.Dp);
   const int nb = (int)(dmax / 256);
   // 4. forward, left-looking by block columns of 256.  Block column k of S is brought up to
-  //    date by one product over every earlier column of L, T = S[k0:, k] - L[k0:, :k] L[k, :k]^T;
+  //    date by products over every earlier column of L, T = S[k0:, k] - L[k0:, :k] L[k, :k]^T;
   //    its diagonal block is factored and inverted (D_k); the panel L[k1:, k] = T[k1:] D_k^T
   //    follows.  The rows of every U are carried along the same way: V = U[:, k] - Y[:, :k]
-  //    L[k, :k]^T, Y[:, k] = V D_k^T.  Every fp32 element of S and U is read and written once
-  //    (a right-looking order rewrites the whole trailing matrix at every step).  Launches per
-  //    step: S column (k > 0), diagonal blocks, U column (k > 0; it needs only earlier columns,
-  //    so it runs beside the diagonal blocks, starting without waiting and waiting for them at
-  //    its end), panel.
+  //    L[k, :k]^T, Y[:, k] = V D_k^T.  Every fp32 element of S and U is read and written about
+  //    once (a right-looking order rewrites the whole trailing matrix at every step).  Only the
+  //    last term of T, from column k - 1, waits for the previous panel: the rest of column k's
+  //    update runs beside step k - 1's diagonal blocks, with the update of U's column (both
+  //    need only earlier columns; that launch starts without waiting and waits for the
+  //    diagonal blocks at its end).  Launches per step: T's last term (k > 0), diagonal blocks,
+  //    [V and the next column's early terms], panel.
   auto run_diag = [&](int k) -> nshb_status {
     const int64_t k0 = 256LL * k;
     for (int c0 = 0; c0 < nz; c0 += kMaxMats) {
@@ -983,11 +985,12 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
       if (z.Dp <= k0) continue;
       ++ndiag;
       if (k > 0) {
-        // T = S[k0:, k] - L[k0:, :k] L[k0:k1, :k]^T, fp32 in place and as hi / lo panels
+        // T = S[k0:, k] - L[k0:, k-1] L[k0:k1, k-1]^T, the last term of the column's update
+        // (the others were applied beside the previous step's diagonal blocks), fp32 in place
+        // and as hi / lo panels
         NwProb t = nw_prob();
-        t.a_hi = z.lh; t.a_lo = z.ll; t.a_ph = (int)z.Dp; t.a_r0 = (int)k0; t.a_k0 = 0;
-        t.b_hi = z.lh; t.b_lo = z.ll; t.b_ph = (int)z.Dp; t.b_r0 = (int)k0; t.b_k0 = 0;
-        t.kt = (int)(k0 / 64);
+        t.a_hi = z.lh; t.a_lo = z.ll; t.a_ph = (int)z.Dp; t.a_r0 = (int)k0; t.a_k0 = (int)(k0 - 256);
+        t.b_hi = z.lh; t.b_lo = z.ll; t.b_ph = (int)z.Dp; t.b_r0 = (int)k0; t.b_k0 = (int)(k0 - 256);
         t.c32 = t.d32 = z.s + (k0 * z.Dp + k0) * 4; t.ld32 = (int)z.Dp;
         t.m_valid = (int)(z.Dp - k0); t.n_valid = 256;
         t.dhi = z.sh; t.dlo = z.sl; t.d_ph = (int)z.Dp; t.d_r0 = (int)k0; t.d_c0 = (int)k0;
@@ -995,6 +998,17 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
         col_s.push_back(t);
       }
       if (z.Dp <= k1) continue;
+      if (k > 0) {
+        // beside the diagonal blocks: S[k1:, k + 1] -= L[k1:, :k] L[k1:k1+256, :k]^T (fp32 only)
+        NwProb t = nw_prob();
+        t.a_hi = z.lh; t.a_lo = z.ll; t.a_ph = (int)z.Dp; t.a_r0 = (int)k1; t.a_k0 = 0;
+        t.b_hi = z.lh; t.b_lo = z.ll; t.b_ph = (int)z.Dp; t.b_r0 = (int)k1; t.b_k0 = 0;
+        t.kt = (int)(k0 / 64);
+        t.c32 = t.d32 = z.s + (k1 * z.Dp + k1) * 4; t.ld32 = (int)z.Dp;
+        t.m_valid = (int)(z.Dp - k1); t.n_valid = 256;
+        t.mt = (int)((z.Dp - k1) / 256); t.nt = 1;
+        col_u.push_back(t);
+      }
       // L[k1:, k] = T[k1:] D_k^T
       NwProb q = nw_prob();
       q.a_hi = z.sh; q.a_lo = z.sl; q.a_ph = (int)z.Dp; q.a_r0 = (int)k1; q.a_k0 = (int)k0;
