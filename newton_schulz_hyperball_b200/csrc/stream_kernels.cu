@@ -354,12 +354,13 @@ __device__ __forceinline__ void momentum_block(const MomentumParams &p, const Ma
   }
 }
 
-// The inputs of the next two blocks are prefetched into registers while the current one is
-// processed, so loads stay in flight through the block's arithmetic and stores even when a
-// power-capped SM clock stretches them (two CTAs per SM; 12 % faster than one block ahead
-// with three CTAs, and 8 % under the 1 kW cap).
+// The inputs of the next two blocks (bf16 instance; one for fp32) are prefetched into
+// registers while the current one is processed, so loads stay in flight through the block's
+// arithmetic and stores even when a power-capped SM clock stretches them (two CTAs per SM;
+// 12 % faster than one block ahead with three CTAs, and 8 % under the 1 kW cap).
 template <bool F32>
 __global__ void __launch_bounds__(kThreads, 2) momentum_kernel(const __grid_constant__ MomentumParams p) {
+  constexpr bool kTwoAhead = !F32;          // the fp32 instance has no registers for a second block
   pdl_trigger();
   pdl_wait();
   __shared__ float sT[2][kBlk][kBlk + 1];   // transpose staging (tall matrices): hi, lo
@@ -370,20 +371,30 @@ __global__ void __launch_bounds__(kThreads, 2) momentum_kernel(const __grid_cons
   block_origin(p.mats[mi], blk - p.mats[mi].blk_begin, r0, c0);
   MomIn n1, n2;
   momentum_load<F32>(p, p.mats[mi], r0, c0, n1);
+  const int ahead = kTwoAhead ? 2 : 1;
   int blk2 = blk + gridDim.x, mi2 = mi, r2 = 0, c2 = 0;
-  if (blk2 < p.total_blocks) {
+  if (kTwoAhead && blk2 < p.total_blocks) {
     mi2 = advance_mat(p, mi, blk2);
     block_origin(p.mats[mi2], blk2 - p.mats[mi2].blk_begin, r2, c2);
     momentum_load<F32>(p, p.mats[mi2], r2, c2, n2);
   }
   for (;;) {
     const MomIn in = n1;
-    n1 = n2;
     const int cblk = blk, cr0 = r0, cc0 = c0;
     const MatDesc &d = p.mats[mi];
-    blk = blk2; mi = mi2; r0 = r2; c0 = c2;
-    blk2 = blk + gridDim.x;
-    if (blk2 < p.total_blocks) {
+    if (kTwoAhead) {
+      n1 = n2;
+      blk = blk2; mi = mi2; r0 = r2; c0 = c2;
+    } else {
+      blk += gridDim.x;
+      if (blk < p.total_blocks) {
+        mi = advance_mat(p, mi, blk);
+        block_origin(p.mats[mi], blk - p.mats[mi].blk_begin, r0, c0);
+        momentum_load<F32>(p, p.mats[mi], r0, c0, n1);
+      }
+    }
+    blk2 = blk + (ahead - 1) * gridDim.x;
+    if (kTwoAhead && blk2 < p.total_blocks) {
       mi2 = advance_mat(p, mi, blk2);
       block_origin(p.mats[mi2], blk2 - p.mats[mi2].blk_begin, r2, c2);
       momentum_load<F32>(p, p.mats[mi2], r2, c2, n2);
