@@ -172,8 +172,10 @@ nshb_status himuon_step(const nshb_matrix *mats, int32_t n_mats, const nshb_para
                         size_t ws_bytes, nshb_stream stream);
 
 /* Newton-Muon wrapped by Hyperball: P = U (Z Z^T + lambda I)^-1 with
- * lambda = ridge_rel tr(Z Z^T) / d_in, solved through an fp32 Cholesky factorisation,
- * then O = NS_K(P) and the Hyperball rule (U is the Nesterov momentum update).  Z[j] is a
+ * lambda = ridge_rel tr(Z Z^T) / d_in, solved through a blocked Cholesky factorisation (the
+ * 256 x 256 diagonal blocks factored and inverted in fp32; every other product on the tensor
+ * cores with each operand split into two bf16 parts, three products per output, fp32
+ * accumulation), then O = NS_K(P) and the Hyperball rule (U is the Nesterov momentum update).  Z[j] is a
  * DEVICE pointer to a bf16 row-major z_rows[j] x n_tokens matrix (leading dimension
  * n_tokens, 16-byte aligned); n_tokens (up to 2^24) and every z_rows[j] (up to 16384) must be
  * multiples of 64, else NSHB_ERR_SHAPE; matrix i uses Z[mats[i].z_index] (an index outside

@@ -7,8 +7,9 @@
 //   split         fp32 regions -> bf16 hi / lo panels, the operands of the split products;
 //   potrf_diag    Cholesky factor of a 256 x 256 diagonal block and its inverse, which
 //                 turns every panel and block solve into a product.
-// The panel products, the trailing updates and the triangular solves for P = U S^-1 run
-// on the split-precision tensor-core GEMM (newton_tc.cu); the host sequences them.
+// The column updates, the panels and the triangular solves for P = U S^-1 (a left-looking
+// blocked Cholesky) run on the split-precision tensor-core GEMM (newton_tc.cu); the host
+// sequences them.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
