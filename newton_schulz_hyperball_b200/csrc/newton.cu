@@ -147,22 +147,20 @@ static_assert(kDiagSmem <= 227 * 1024, "diagonal block does not fit in shared me
 
 __device__ __forceinline__ float *blk(float *sm, int i, int k) { return sm + (i * (i + 1) / 2 + k) * kBlk; }
 
-// Block products on one warp.  The warp computes rows r0 + g + 8x (x < NX; g = lane / 4) of a
-// 32 x 32 output, NX rows and eight columns per lane (NX = 4, r0 = 0: a whole block).  Reads
-// are 16-byte rows of distinct banks, or broadcasts.
-// acc[x][e] += sum_q A[r0 + g + 8x][q] B[h + 4e][q]   (A B^T;  h = lane % 4)
-template <int NX>
-__device__ __forceinline__ void nt_acc(const float *A, const float *B, float (&acc)[NX][8], int r0 = 0) {
+// Block products on one warp: a 32 x 32 output, four rows (g + 8x, g = lane / 4) and eight
+// columns per lane.  Reads are 16-byte rows of distinct banks, or broadcasts.
+// acc[x][e] += sum_q A[g + 8x][q] B[h + 4e][q]   (A B^T;  h = lane % 4)
+__device__ __forceinline__ void nt_acc(const float *A, const float *B, float (&acc)[4][8]) {
   const int lane = threadIdx.x & 31, g = lane >> 2, h = lane & 3;
 #pragma unroll 2
   for (int q = 0; q < 32; q += 4) {
-    float4 a[NX], b[8];
+    float4 a[4], b[8];
 #pragma unroll
-    for (int x = 0; x < NX; ++x) a[x] = *reinterpret_cast<const float4 *>(A + (r0 + g + 8 * x) * kBS + q);
+    for (int x = 0; x < 4; ++x) a[x] = *reinterpret_cast<const float4 *>(A + (g + 8 * x) * kBS + q);
 #pragma unroll
     for (int e = 0; e < 8; ++e) b[e] = *reinterpret_cast<const float4 *>(B + (h + 4 * e) * kBS + q);
 #pragma unroll
-    for (int x = 0; x < NX; ++x)
+    for (int x = 0; x < 4; ++x)
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         float t = acc[x][e];
@@ -174,22 +172,21 @@ __device__ __forceinline__ void nt_acc(const float *A, const float *B, float (&a
   }
 }
 
-// acc[x][e] += sum_q A[r0 + g + 8x][q] B[q][8h + e]   (A B)
-template <int NX>
-__device__ __forceinline__ void nn_acc(const float *A, const float *B, float (&acc)[NX][8], int r0 = 0) {
+// acc[x][e] += sum_q A[g + 8x][q] B[q][8h + e]   (A B)
+__device__ __forceinline__ void nn_acc(const float *A, const float *B, float (&acc)[4][8]) {
   const int lane = threadIdx.x & 31, g = lane >> 2, h = lane & 3;
 #pragma unroll 2
   for (int q = 0; q < 32; q += 4) {
-    float4 a[NX];
+    float4 a[4];
 #pragma unroll
-    for (int x = 0; x < NX; ++x) a[x] = *reinterpret_cast<const float4 *>(A + (r0 + g + 8 * x) * kBS + q);
+    for (int x = 0; x < 4; ++x) a[x] = *reinterpret_cast<const float4 *>(A + (g + 8 * x) * kBS + q);
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       const float4 b0 = *reinterpret_cast<const float4 *>(B + (q + t) * kBS + 8 * h);
       const float4 b1 = *reinterpret_cast<const float4 *>(B + (q + t) * kBS + 8 * h + 4);
       const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int x = 0; x < NX; ++x) {
+      for (int x = 0; x < 4; ++x) {
         const float av = t == 0 ? a[x].x : t == 1 ? a[x].y : t == 2 ? a[x].z : a[x].w;
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[x][e] = fmaf(av, b[e], acc[x][e]);
@@ -198,22 +195,20 @@ __device__ __forceinline__ void nn_acc(const float *A, const float *B, float (&a
   }
 }
 
-template <int NX>
-__device__ __forceinline__ void zero_acc(float (&acc)[NX][8]) {
+__device__ __forceinline__ void zero_acc(float (&acc)[4][8]) {
 #pragma unroll
-  for (int x = 0; x < NX; ++x)
+  for (int x = 0; x < 4; ++x)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[x][e] = 0.f;
 }
 
 // Stores sgn * acc into a block, in the element order of nt_acc (nt) or nn_acc.
-template <int NX>
-__device__ __forceinline__ void put_acc(float *C, const float (&acc)[NX][8], float sgn, bool nt, int r0 = 0) {
+__device__ __forceinline__ void put_acc(float *C, const float (&acc)[4][8], float sgn, bool nt) {
   const int lane = threadIdx.x & 31, g = lane >> 2, h = lane & 3;
 #pragma unroll
-  for (int x = 0; x < NX; ++x)
+  for (int x = 0; x < 4; ++x)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) C[(r0 + g + 8 * x) * kBS + (nt ? h + 4 * e : 8 * h + e)] = sgn * acc[x][e];
+    for (int e = 0; e < 8; ++e) C[(g + 8 * x) * kBS + (nt ? h + 4 * e : 8 * h + e)] = sgn * acc[x][e];
 }
 
 // One warp: block B (32 x 32, lower triangle read) is replaced by D = L^-1, where B = L L^T.
