@@ -977,6 +977,49 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
     }
     return NSHB_OK;
   };
+  // 5. backward, P L = Y by block columns from the last, left-looking as well:
+  //    W = Y[:, k] - P[:, k1:] L[k1:, k] (one product over every later column of P; only its
+  //    hi / lo panels are kept, in place of Y[:, k]), then P[:, k] = W D_k (fp32 into the m x n
+  //    buffer the momentum pass reads, and hi / lo panels in place of W).  A matrix whose layer
+  //    input has g block columns runs 2g - 1 stages (solve g-1, column g-2, solve g-2, ..., solve
+  //    0); its stages start as soon as its forward sweep is over, one per launch, so the matrices
+  //    of narrow layer inputs finish theirs inside the forward sweep of the wide ones (in the
+  //    launches beside the diagonal blocks) and the rest continue after it.
+  auto bwd_stage = [&](int i, int s, std::vector<NwProb> &out) {
+    const Plan::ZPlan &z = pl.zp[pl.zidx[i]];
+    const int g = (int)(z.Dp / 256);
+    const int kk = g - 1 - (s + 1) / 2;
+    const int64_t k0 = 256LL * kk, k1 = k0 + 256;
+    if (s % 2 == 1) {
+      NwProb t = nw_prob();
+      t.a_hi = pl.yh[i]; t.a_lo = pl.yl[i]; t.a_ph = (int)pl.mpad[i]; t.a_r0 = 0; t.a_k0 = (int)k1;
+      t.b_hi = z.lh; t.b_lo = z.ll; t.b_ph = (int)z.Dp; t.b_r0 = (int)k0; t.b_k0 = (int)k1;
+      t.kt = (int)((z.Dp - k1) / 64);
+      t.flags = kNwBMn;
+      t.c32 = pl.y32[i] + k0 * 4; t.ld32 = (int)z.Dp;
+      t.m_valid = (int)pl.mpad[i]; t.n_valid = 256;
+      t.dhi = pl.yh[i]; t.dlo = pl.yl[i]; t.d_ph = (int)pl.mpad[i]; t.d_r0 = 0; t.d_c0 = (int)k0;
+      t.mt = (int)(pl.mpad[i] / 256); t.nt = 1;
+      out.push_back(t);
+    } else {
+      const int d = (int)pl.mp[i].n, m = (int)pl.mp[i].m;
+      NwProb q = nw_prob();
+      q.a_hi = pl.yh[i]; q.a_lo = pl.yl[i]; q.a_ph = (int)pl.mpad[i]; q.a_r0 = 0; q.a_k0 = (int)k0;
+      q.b_hi = z.dh; q.b_lo = z.dl; q.b_ph = (int)z.Dp; q.b_r0 = 0; q.b_k0 = (int)k0;
+      q.flags = kNwBMn;
+      q.d32 = pl.r_off[i] + k0 * 4; q.ld32 = d; q.m_valid = m; q.n_valid = (int)std::max<int64_t>(0, d - k0);
+      q.dhi = pl.yh[i]; q.dlo = pl.yl[i]; q.d_ph = (int)pl.mpad[i]; q.d_r0 = 0; q.d_c0 = (int)k0;
+      q.mt = (int)(pl.mpad[i] / 256); q.nt = 1;
+      out.push_back(q);
+    }
+  };
+  // stage k - g of every matrix whose g block columns are done by step k (0 <= k - g <= 2g - 2)
+  auto bwd_stages = [&](int k, std::vector<NwProb> &out) {
+    for (int i = 0; i < n; ++i) {
+      const int g = (int)(pl.zp[pl.zidx[i]].Dp / 256), s = k - g;
+      if (s >= 0 && s <= 2 * g - 2) bwd_stage(i, s, out);
+    }
+  };
   for (int k = 0; k < nb; ++k) {
     const int64_t k0 = 256LL * k, k1 = k0 + 256;
     std::vector<NwProb> col_s, col_u, panel;
@@ -1051,6 +1094,7 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
     // costs what running the two in turn costs.
     int reserve = (ndiag + 1) / 2 + 4;
     if (4 * reserve > device_sms() / 2) reserve = 0;
+    bwd_stages(k, col_u);                 // backward stages of the matrices already done
     np.late_wait = 1;
     e = run_nw(np, col_u, st, reserve);
     np.late_wait = 0;
@@ -1058,41 +1102,11 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
     e = run_nw(np, panel, st);
     if (e != NSHB_OK) return e;
   }
-  // 5. backward, P L = Y by block columns from the last, left-looking as well:
-  //    W = Y[:, k] - P[:, k1:] L[k1:, k] (one product over every later column of P; only its
-  //    hi / lo panels are kept, in place of Y[:, k]), then P[:, k] = W D_k (fp32 into the m x n
-  //    buffer the momentum pass reads, and hi / lo panels in place of W).
-  for (int k = nb - 1; k >= 0; --k) {
-    const int64_t k0 = 256LL * k, k1 = k0 + 256;
-    std::vector<NwProb> col_p, solve;
-    for (int i = 0; i < n; ++i) {
-      const Plan::ZPlan &z = pl.zp[pl.zidx[i]];
-      if (z.Dp <= k0) continue;
-      const int d = (int)pl.mp[i].n, m = (int)pl.mp[i].m;
-      if (z.Dp > k1) {
-        NwProb t = nw_prob();
-        t.a_hi = pl.yh[i]; t.a_lo = pl.yl[i]; t.a_ph = (int)pl.mpad[i]; t.a_r0 = 0; t.a_k0 = (int)k1;
-        t.b_hi = z.lh; t.b_lo = z.ll; t.b_ph = (int)z.Dp; t.b_r0 = (int)k0; t.b_k0 = (int)k1;
-        t.kt = (int)((z.Dp - k1) / 64);
-        t.flags = kNwBMn;
-        t.c32 = pl.y32[i] + k0 * 4; t.ld32 = (int)z.Dp;
-        t.m_valid = (int)pl.mpad[i]; t.n_valid = 256;
-        t.dhi = pl.yh[i]; t.dlo = pl.yl[i]; t.d_ph = (int)pl.mpad[i]; t.d_r0 = 0; t.d_c0 = (int)k0;
-        t.mt = (int)(pl.mpad[i] / 256); t.nt = 1;
-        col_p.push_back(t);
-      }
-      NwProb q = nw_prob();
-      q.a_hi = pl.yh[i]; q.a_lo = pl.yl[i]; q.a_ph = (int)pl.mpad[i]; q.a_r0 = 0; q.a_k0 = (int)k0;
-      q.b_hi = z.dh; q.b_lo = z.dl; q.b_ph = (int)z.Dp; q.b_r0 = 0; q.b_k0 = (int)k0;
-      q.flags = kNwBMn;
-      q.d32 = pl.r_off[i] + k0 * 4; q.ld32 = d; q.m_valid = m; q.n_valid = (int)std::max<int64_t>(0, d - k0);
-      q.dhi = pl.yh[i]; q.dlo = pl.yl[i]; q.d_ph = (int)pl.mpad[i]; q.d_r0 = 0; q.d_c0 = (int)k0;
-      q.mt = (int)(pl.mpad[i] / 256); q.nt = 1;
-      solve.push_back(q);
-    }
-    nshb_status e = run_nw(np, col_p, st);
-    if (e != NSHB_OK) return e;
-    e = run_nw(np, solve, st);
+  // the remaining backward stages, one launch per stage index
+  for (int k = nb; k <= 3 * nb - 2; ++k) {
+    std::vector<NwProb> stage;
+    bwd_stages(k, stage);
+    nshb_status e = run_nw(np, stage, st);
     if (e != NSHB_OK) return e;
   }
   return NSHB_OK;
