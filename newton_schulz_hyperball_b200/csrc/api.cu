@@ -769,7 +769,7 @@ nshb_status run_nw(NwParams &np, const std::vector<NwProb> &probs, cudaStream_t 
     for (size_t i = c0; i < c1; ++i) {
       NwProb q = probs[i];
       q.tile_begin = tiles;
-      tiles += (q.flags & kNwLower) ? q.mt * (q.mt + 1) / 2 : q.mt * q.nt;
+      tiles += q.mt * q.nt;
       np.prob[i - c0] = q;
     }
     np.nprob = (int)(c1 - c0);

@@ -52,22 +52,11 @@ __device__ __forceinline__ NwTile nw_decode(const NwParams &p, int tile) {
     if (p.prob[mid].tile_begin <= tile) lo = mid; else hi = mid - 1;
   }
   const NwProb &q = p.prob[lo];
-  int l = tile - q.tile_begin;
+  const int l = tile - q.tile_begin;
   NwTile t;
   t.prob = lo;
-  if (q.flags & kNwLower) {
-    int mi = 0;
-    for (;; ++mi) {
-      const int c = (mi + 1 < q.nt) ? mi + 1 : q.nt;
-      if (l < c) break;
-      l -= c;
-    }
-    t.m0 = mi * BM;
-    t.n0 = l * BN;
-  } else {
-    t.m0 = (l / q.nt) * BM;
-    t.n0 = (l % q.nt) * BN;
-  }
+  t.m0 = (l / q.nt) * BM;
+  t.n0 = (l % q.nt) * BN;
   return t;
 }
 
