@@ -563,6 +563,55 @@ def test_step_captures_in_a_cuda_graph():
             assert np.array_equal(x, y)
 
 
+
+def test_newton_muon_step_captures_in_a_cuda_graph():
+    """The Newton-Muon step (its launches that run beside the diagonal blocks and wait for
+    them at their end included) can be captured once and replayed; the replay equals a direct
+    call on the same inputs bit for bit.  Layer inputs of 256 and 768 rows: one and three
+    diagonal blocks, so the staged backward of the narrow one runs inside the wide one's
+    forward sweep."""
+    cfg = wl.CFG_NEWTON_GPT2
+    n_tok = 512
+    Zs = [wl.layer_input(cfg, 10, 256, n_tok), wl.layer_input(cfg, 11, 768, n_tok)]
+    shapes = [(256, 256), (512, 768), (300, 256), (768, 768)]
+    zi = [0, 1, 0, 1]
+    Ws = [wl.init_weight(cfg, 60 + i, r, c, bf16=True).astype(np.float64) for i, (r, c) in enumerate(shapes)]
+    Gs = [wl.gradient(cfg, 60 + i, 0, r, c, bf16=True).astype(np.float64) for i, (r, c) in enumerate(shapes)]
+    rho = torch.tensor([o.fro(w) for w in Ws], dtype=torch.float32, device="cuda")
+    p = nshb.params(eta=0.02, rho=rho, ridge_rel=1e-3)
+    Zd = [torch.from_numpy(z.astype(np.float32)).to("cuda").to(torch.bfloat16) for z in Zs]
+    z_rows = [z.shape[0] for z in Zs]
+
+    def make_set():
+        gs = GpuSet(Ws, bf16=True)
+        for k in range(len(shapes)):
+            gs.mats[k].z_index = zi[k]
+        gs.set_grads(Gs)
+        need = nshb.workspace_size(gs.mats, p, nshb.NSHB_OP_NEWTON_MUON, z_rows, n_tok)
+        return gs, torch.empty(need, dtype=torch.uint8, device="cuda")
+
+    direct, ws_d = make_set()
+    nshb.newton_muon_step(direct.mats, Zd, n_tok, p, ws_d)
+    assert nshb.device_status(ws_d) == 0
+    graphed, ws = make_set()
+    nshb.newton_muon_step(graphed.mats, Zd, n_tok, p, ws)   # first call outside capture (module set-up)
+    torch.cuda.synchronize()
+    for w, w0 in zip(graphed.W, Ws):
+        w.copy_(torch.from_numpy(w0.astype(np.float32)).to("cuda").to(torch.bfloat16))
+    for m in graphed.M:
+        m.zero_()
+    s = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            nshb.newton_muon_step(graphed.mats, Zd, n_tok, p, ws, s)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert nshb.device_status(ws) == 0
+    for a, b in zip(direct.host(), graphed.host()):
+        for x, y in zip(a, b):
+            assert np.array_equal(x, y)
+
 def test_thirteen_shapes_in_one_call():
     """Thirteen distinct padded shapes in one call (every GEMM launch mixes problems of
     different sizes and k depths); every matrix against the oracle, and the first two run
