@@ -645,21 +645,23 @@ nshb_status run_ns(const nshb_matrix *mats, const Plan &pl, const nshb_params *p
               q.major = tall ? (kAMn | kBMn) : 0;
               q.mt = (int)(R / 256); q.nt = (int)(R / pl.bn); q.kt = (int)(S / 64);
             } else if (mode == kPoly) {
+              // A is stored on and below the diagonal only (as is every symmetric result)
               q.a_off = m.a; q.b_off = m.a; q.c_off = m.a; q.d_off = m.b;
               q.a_ph = q.b_ph = q.d_ph = (int)R;
-              q.major = 0;
+              q.major = kASym | kBSym;
               q.mt = (int)(R / 256); q.nt = (int)(R / pl.bn); q.kt = (int)(R / 64);
             } else if (!tall) {
-              // X' = s (a X + B X): A = B (K-major), B operand = X (MN-major)
+              // X' = s (a X + B X): A = B (K-major, lower triangle stored), B operand = X (MN-major)
               q.a_off = m.b; q.b_off = xin; q.c_off = xin; q.d_off = xout;
               q.a_ph = q.b_ph = q.d_ph = (int)R;
-              q.major = kBMn;
+              q.major = kBMn | kASym;
               q.mt = (int)(R / 256); q.nt = (int)(S / pl.bn); q.kt = (int)(R / 64);
             } else {
-              // X' = s (a X + X B): A = X (K-major, S rows), B operand = B (symmetric, K-major)
+              // X' = s (a X + X B): A = X (K-major, S rows), B operand = B (symmetric, K-major,
+              // lower triangle stored)
               q.a_off = xin; q.b_off = m.b; q.c_off = xin; q.d_off = xout;
               q.a_ph = q.d_ph = (int)S; q.b_ph = (int)R;
-              q.major = 0;
+              q.major = kBSym;
               q.mt = (int)(S / 256); q.nt = (int)(R / pl.bn); q.kt = (int)(R / 64);
             }
             q.tiles_per_batch = gemm_tiles(mode, q.mt, q.nt, 256, pl.bn);

@@ -1,7 +1,8 @@
 // Grouped bf16 Newton-Schulz GEMM on CTA pairs (tcgen05.mma.cta_group::2).
 //
 // Same phases and epilogues as the single-CTA kernel (ns_tc.cu): Gram A = s^2 X X^T and
-// polynomial B = b A + c A^2 (lower-triangle tiles + mirrored stores), update
+// polynomial B = b A + c A^2 (only the tiles on and below the diagonal are computed and
+// stored; a reader takes a block above the diagonal as the transpose of its mirror), update
 // X' = s (a X + B X) ("Muon: the orthogonalized optimizer explained", Newton-Schulz
 // section and newton_schulz5), plus the fp32 Gram of the Newton-Muon layer inputs.
 //
@@ -153,7 +154,11 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
           }
           // K-major: rows am .. am+127 of k panels kb and kb+1 (16 KB each); MN-major: the 128
           // rows (columns of the stored matrix) are two 64-column panels, k rows kb*64 .. +127.
-          if (!(q.major & kAMn)) {
+          // A symmetric operand stored below the diagonal only reads a block above it (k tile
+          // > the operand's row tile) MN-major from its mirror.
+          const bool a_mn = (q.major & kAMn) || ((q.major & kASym) && (kb >> 2) > (t.m0 >> 8));
+          const bool b_mn = (q.major & kBMn) || ((q.major & kBSym) && (kb >> 2) > (t.n0 >> 8));
+          if (!a_mn) {
             const int64_t ya = a_row + (int64_t)kb * q.a_ph + am;
             tma_load_2sm(sA, &p.tmap, 0, (int)ya, fb);
             tma_load_2sm(sA + SLICE_BYTES, &p.tmap, 0, (int)(ya + q.a_ph), fb);
@@ -162,7 +167,7 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
             tma_load_2sm(sA, &p.tmap, 0, (int)y0, fb);
             tma_load_2sm(sA + SLICE_BYTES, &p.tmap, 0, (int)(y0 + q.a_ph), fb);
           }
-          if (!(q.major & kBMn)) {
+          if (!b_mn) {
             const int64_t yb = b_row + (int64_t)kb * q.b_ph + bn;
             tma_load_2sm(sB, &p.tmap, 0, (int)yb, fb);
             tma_load_2sm(sB + SLICE_BYTES, &p.tmap, 0, (int)(yb + q.b_ph), fb);
@@ -193,8 +198,6 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
       for (int tile = cid; ok && tile < p.total_tiles; tile += ncl, ++tl) {
         const Tile t = decode2(p, tile);
         const GemmProb &q = p.prob[t.prob];
-        const bool amn = q.major & kAMn, bmn = q.major & kBMn;
-        const uint32_t idesc = idesc_bf16(BM, BN, amn ? 1 : 0, bmn ? 1 : 0);
         const int buf = tl & 1;
         const uint32_t tph = (uint32_t)(tl >> 1) & 1u;
         if (!mbar_wait(tempty_bar(buf), tph ^ 1u, limit)) {
@@ -211,6 +214,10 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
           }
           tc_fence_after();
           const uint32_t sA = smem_base + stage * STAGE_BYTES, sB = sA + HALF_BYTES;
+          // the majorness the producer loaded this stage with
+          const bool amn = (q.major & kAMn) || ((q.major & kASym) && (kb >> 2) > (t.m0 >> 8));
+          const bool bmn = (q.major & kBMn) || ((q.major & kBSym) && (kb >> 2) > (t.n0 >> 8));
+          const uint32_t idesc = idesc_bf16(BM, BN, amn ? 1 : 0, bmn ? 1 : 0);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             // K-major: panel k/4, 32-byte step k%4 inside the 128-byte swizzled rows.
@@ -237,7 +244,6 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
     const int row = 128 * (int)rank + quarter * 32 + lane;   // row of the 256-row tile
-    const bool sym = sym_mode(p.mode);
     const bool needc = (p.mode == kPoly || p.mode == kUpdate);
     const bool fuse = FUSE && p.mode == kUpdate && p.partials != nullptr;
     int tl = 0;
@@ -253,7 +259,6 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
       const char *clo = q.c_lo >= 0 ? p.ws + q.c_lo + (int64_t)t.batch * q.bs : nullptr;
       char *dlo = q.d_lo >= 0 ? p.ws + q.d_lo + (int64_t)t.batch * q.bs : nullptr;
       const int64_t i = t.m0 + row;
-      const int ra = (int)(i >> 6);
       const int cc_end = (half + 1) * NCH;
       // Hyperball partials of this problem: the caller's W next to O (X coordinates (i, c)
       // are W's (i, c), offset by the tile origin for a Hierarchical-Muon tile).
@@ -300,7 +305,9 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
           if (wr < q.w_m && wc < q.w_n) asm volatile("prefetch.global.L2 [%0];" ::"l"(wb + (wr * q.w_ld + wc) * esz));
         }
       };
-      auto live = [&](int cc) { return cc < cc_end && !(sym && ((t.n0 + cc * 32) >> 6) > ra); };
+      // every chunk of the tile, the diagonal tiles of a symmetric result whole (its readers
+      // take a block above the diagonal from the stored one below it)
+      auto live = [&](int cc) { return cc < cc_end; };
       const bool odd = i & 1;
       // C words of columns col0 .. col0+31 in logical order (two 32-byte sector reads).
       // (The fused instance prefetches W instead of C's low part, which it reads in the chunk.)
@@ -335,7 +342,6 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
 #pragma unroll 1
       for (; live(cc); ++cc) {
         const int col0 = t.n0 + cc * 32;
-        const int ca = col0 >> 6;
         uint32_t nh[16], nl[16], wn[16];
         if (needc && live(cc + 1)) load_c(cc + 1, nh, nl);
         if (wp && live(cc + 1)) load_w(cc + 1, wn);
@@ -358,11 +364,6 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
             *reinterpret_cast<float4 *>(drow + col0 + 4 * g) =
                 make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]), __uint_as_float(r[4 * g + 2]),
                             __uint_as_float(r[4 * g + 3]));
-          if (ca < ra) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              reinterpret_cast<float *>(dbase)[(int64_t)(col0 + e) * q.d_ph + i] = __uint_as_float(r[e]);
-          }
           continue;
         }
         if (p.mode == kGram) {
@@ -410,15 +411,6 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
               l[e] = pack_bf16(v[16 * k + 2 * e] - bf16lo(o[e]), v[16 * k + 2 * e + 1] - bf16hi(o[e]));
             unswizzle_pair(l, odd, w);
             st_global_256(dlo + off, w);
-          }
-        }
-        if (sym && ca < ra) {
-          const int64_t ib = i & ~7LL;
-          const int ie = (int)(i & 7);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            __nv_bfloat16 h = __float2bfloat16_rn(v[e]);
-            *reinterpret_cast<__nv_bfloat16 *>(dbase + panel_chunk_off(col0 + e, ib, q.d_ph) + 2 * ie) = h;
           }
         }
         if (wp) {

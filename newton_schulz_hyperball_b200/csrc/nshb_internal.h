@@ -149,12 +149,17 @@ struct AdamParams {
 // operands MN-major, its update X B both K-major.
 constexpr int kAMn = 1;   // GemmProb::major: A MN-major
 constexpr int kBMn = 2;   // B MN-major
+// The operand is a symmetric matrix of which only the 256 x 256 tiles on and below the
+// diagonal are stored: a block above the diagonal is read as the transpose of its mirror
+// (the same rows of the stored matrix, taken MN-major instead of K-major).
+constexpr int kASym = 4;
+constexpr int kBSym = 8;
 struct GemmProb {
   int64_t a_off, b_off, c_off, d_off;  // byte offsets of batch 0
   int64_t c_lo, d_lo;                  // kUpdate: bf16 low parts of C (read) / D (written), or -1
   int64_t bs;                          // byte stride between batches (every operand)
   int32_t a_ph, b_ph, d_ph;            // panel heights (padded rows) of A, B and C / D
-  int32_t major;                       // kAMn | kBMn
+  int32_t major;                       // kAMn | kBMn | kASym | kBSym
   int32_t mt, nt, kt;                  // 256-row tiles, BN-column tiles, 64-deep k blocks
   int32_t batch, tiles_per_batch, tile_begin;
   int32_t scale_idx;                   // scale of batch 0 in GemmParams::scales, or -1
