@@ -181,7 +181,8 @@ nshb_status himuon_step(const nshb_matrix *mats, int32_t n_mats, const nshb_para
  * multiples of 64, else NSHB_ERR_SHAPE; matrix i uses Z[mats[i].z_index] (an index outside
  * [0, n_z) is NSHB_ERR_PARAM), which needs z_rows == cols (else NSHB_ERR_SHAPE).  Z and z_rows
  * are HOST arrays of n_z entries (1 <= n_z <= 224).  A pivot that is not positive in fp32 sets
- * NSHB_DEV_NOT_SPD.  bf16 NS only. */
+ * NSHB_DEV_NOT_SPD.  bf16 NS only.  The tensor cores read every Z in place during the call
+ * (no copy in the workspace), so Z must stay unchanged until the step has run on the stream. */
 nshb_status newton_muon_step(const nshb_matrix *mats, int32_t n_mats, const void *const *Z,
                              const int64_t *z_rows, int32_t n_z, int64_t n_tokens,
                              const nshb_params *p, void *ws, size_t ws_bytes, nshb_stream stream);

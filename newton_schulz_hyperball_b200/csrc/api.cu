@@ -66,7 +66,6 @@ struct Plan {
   struct ZPlan {
     int64_t d = 0, Dp = 0;
     const void *src = nullptr;
-    int64_t zp = 0;                   // panel copy of Z (Dp x n_tokens bf16)
     int64_t s = 0;                    // S = Z Z^T + lambda I, fp32 Dp x Dp, updated in place
     int64_t sh = 0, sl = 0;           // bf16 hi / lo panels of S (operands of the panel products)
     int64_t lh = 0, ll = 0;           // bf16 hi / lo panels of the Cholesky factor L
@@ -251,7 +250,6 @@ nshb_status plan_newton(const nshb_matrix *mats, int n_mats, const void *const *
     if (Z && (!z.src || (uintptr_t)z.src % 16 != 0)) return !z.src ? NSHB_ERR_NULL : NSHB_ERR_SHAPE;
     z.Dp = round_up(z.d, 256);
     const size_t sq = (size_t)z.Dp * z.Dp;
-    z.zp = off; off = align_up(off + (size_t)z.Dp * n_tokens * 2);
     z.s = off;  off = align_up(off + sq * 4);
     z.sh = off; off = align_up(off + sq * 2);
     z.sl = off; off = align_up(off + sq * 2);
@@ -830,29 +828,10 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
     mp.total_blocks = nb;
     NSHB_LAUNCH(NSHB_PROF_MOMENTUM, launch_momentum(mp, st));
   }
-  // 2. Z -> panels, S = Z Z^T on the tensor cores (fp32 out), ridge
-  for (int c0 = 0; c0 < nz; c0 += kMaxMats) {
-    const int c1 = std::min(nz, c0 + kMaxMats);
-    PackParams pp;
-    std::memset(&pp, 0, sizeof(pp));
-    pp.ws = ws;
-    pp.n = c1 - c0;
-    int nb = 0;
-    for (int j = c0; j < c1; ++j) {
-      const Plan::ZPlan &z = pl.zp[j];
-      pp.src[j - c0] = z.src;
-      pp.dst_off[j - c0] = z.zp;
-      pp.rows[j - c0] = (int)z.d;
-      pp.cols[j - c0] = (int)pl.n_tokens;
-      pp.ld[j - c0] = (int)pl.n_tokens;
-      pp.ph[j - c0] = (int)z.Dp;
-      pp.blk_begin[j - c0] = nb;
-      nb += (int)(z.Dp / 64) * (int)(pl.n_tokens / 64);
-    }
-    pp.blk_begin[c1 - c0] = nb;
-    NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_pack_panels(pp, st));
-
-    GemmParams gp;
+  // 2. S = Z Z^T on the tensor cores (fp32 out), its operands read straight from each Z
+  for (int c0 = 0; c0 < nz; c0 += kMaxZMaps) {
+    const int c1 = std::min(nz, c0 + kMaxZMaps);
+    SyrkParams gp;
     std::memset(&gp, 0, sizeof(gp));
     gp.ws = ws;
     gp.status = status;
@@ -862,8 +841,9 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
     int tiles = 0, k = 0;
     for (int j = c0; j < c1; ++j) {
       const Plan::ZPlan &z = pl.zp[j];
+      NSHB_CHECK_CUDA(encode_z_tensor_map(&gp.zmap[k], z.src, z.d, pl.n_tokens));
       GemmProb &q = gp.prob[k++];
-      q.a_off = q.b_off = z.zp;
+      q.a_off = q.b_off = 0;
       q.c_off = q.d_off = z.s;
       q.c_lo = q.d_lo = -1;
       q.a_ph = q.b_ph = q.d_ph = (int)z.Dp;
@@ -883,7 +863,7 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
     gp.nprob = k;
     gp.total_tiles = tiles;
     NSHB_CHECK_CUDA(encode_ws_tensor_map(&gp.tmap, ws, pl.total / 128 * 128));
-    NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_gemm_tc2(gp, device_sms(), st));
+    NSHB_LAUNCH(NSHB_PROF_NEWTON, launch_gemm_syrk(gp, device_sms(), st));
   }
   // 3. ridge (and a unit diagonal on the padding), then the operands of the first step as
   //    bf16 hi / lo panels: S's first column block and every U (with an fp32 copy padded to

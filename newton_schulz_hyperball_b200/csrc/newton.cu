@@ -1,15 +1,14 @@
 // Newton-Muon preconditioner pieces ("The Newton-Muon Optimizer", abstract: the update
 // msgn(G (Z Z^T)^-1), here with a ridge lambda = ridge_rel tr(Z Z^T) / d_in).
 //
-//   pack_panels   layer input Z (bf16 row-major d x n) -> the tensor-core panel layout,
-//                 so that S = Z Z^T runs on the grouped tcgen05 GEMM (fp32 output);
 //   ridge         lambda = ridge_rel tr(S) / d, S += lambda I (one CTA per Z, fixed order);
 //   split         fp32 regions -> bf16 hi / lo panels, the operands of the split products;
 //   potrf_diag    Cholesky factor of a 256 x 256 diagonal block and its inverse, which
 //                 turns every panel and block solve into a product.
-// The column updates, the panels and the triangular solves for P = U S^-1 (a left-looking
-// blocked Cholesky) run on the split-precision tensor-core GEMM (newton_tc.cu); the host
-// sequences them.
+// S = Z Z^T itself runs on the grouped pair GEMM (ns_tc2.cu), reading each Z where the
+// caller keeps it.  The column updates, the panels and the triangular solves for
+// P = U S^-1 (a left-looking blocked Cholesky) run on the split-precision tensor-core GEMM
+// (newton_tc.cu); the host sequences them.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -18,29 +17,6 @@
 
 namespace nshb {
 namespace {
-
-__global__ void __launch_bounds__(256) pack_panels_kernel(const __grid_constant__ PackParams p) {
-  const int blk = blockIdx.x;
-  int lo = 0, hi = p.n - 1;
-  while (lo < hi) {
-    int mid = (lo + hi + 1) >> 1;
-    if (p.blk_begin[mid] <= blk) lo = mid; else hi = mid - 1;
-  }
-  const int lb = blk - p.blk_begin[lo];
-  const int rows = p.rows[lo], cols = p.cols[lo], ph = p.ph[lo];
-  const int bc = cols / 64;
-  const int r0 = (lb / bc) * 64, c0 = (lb % bc) * 64;
-  const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(p.src[lo]);
-  char *dst = p.ws + p.dst_off[lo];
-  // 64 x 64 block = 512 chunks of 16 bytes; two per thread.
-  for (int c = threadIdx.x; c < 512; c += 256) {
-    const int rr = c >> 3, q = c & 7;
-    const int r = r0 + rr, col = c0 + 8 * q;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r < rows) v = *reinterpret_cast<const uint4 *>(src + (int64_t)r * p.ld[lo] + col);
-    *reinterpret_cast<uint4 *>(dst + panel_chunk_off(r, col, ph)) = v;
-  }
-}
 
 // lambda = ridge_rel tr(S) / d added to the diagonal.  The padded rows and columns of S
 // (d .. ld-1, zero from the Gram) get a unit diagonal, so the padded matrix factors as
@@ -438,10 +414,6 @@ __global__ void __launch_bounds__(kDiagThreads, 1) potrf_diag_kernel(const __gri
 
 }  // namespace
 
-cudaError_t launch_pack_panels(const PackParams &p, cudaStream_t s) {
-  if (p.n > 0 && p.blk_begin[p.n] > 0) pack_panels_kernel<<<p.blk_begin[p.n], 256, 0, s>>>(p);
-  return cudaGetLastError();
-}
 cudaError_t launch_ridge(const CholParams &p, cudaStream_t s) {
   if (p.n > 0) ridge_kernel<<<p.n, 256, 0, s>>>(p);
   return cudaGetLastError();

@@ -1,10 +1,10 @@
 // Grouped bf16 Newton-Schulz GEMM on CTA pairs (tcgen05.mma.cta_group::2).
 //
-// Same phases and epilogues as the single-CTA kernel (ns_tc.cu): Gram A = s^2 X X^T and
-// polynomial B = b A + c A^2 (only the tiles on and below the diagonal are computed and
+// Phases: Gram A = s^2 X X^T and polynomial B = b A + c A^2 (only the tiles on and below the diagonal are computed and
 // stored; a reader takes a block above the diagonal as the transpose of its mirror), update
 // X' = s (a X + B X) ("Muon: the orthogonalized optimizer explained", Newton-Schulz
-// section and newton_schulz5), plus the fp32 Gram of the Newton-Muon layer inputs.
+// section), plus the fp32 Gram S = Z Z^T of the Newton-Muon layer inputs, whose operands are
+// loaded straight from the caller's row-major Z through one swizzling tensor map per input.
 //
 // Why pairs: with single-CTA 128 x 256 tiles every SM must stream 96 bytes of operands
 // per clock to keep its tensor core busy, more than the L2 delivers per SM.  A pair of
@@ -28,6 +28,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "nshb_device.cuh"
 #include "nshb_internal.h"
@@ -53,7 +54,8 @@ struct Tile {
 
 __device__ __forceinline__ bool sym_mode(int mode) { return mode == kGram || mode == kPoly || mode == kGramF32; }
 
-__device__ __forceinline__ Tile decode2(const GemmParams &p, int tile) {
+template <class P>
+__device__ __forceinline__ Tile decode2(const P &p, int tile) {
   int lo = 0, hi = p.nprob - 1;
   while (lo < hi) {
     int mid = (lo + hi + 1) >> 1;
@@ -85,8 +87,10 @@ __device__ __forceinline__ Tile decode2(const GemmParams &p, int tile) {
 // FUSE: the instance for the last update launch with Hyperball partials (W read in the
 // epilogue); the other launches use the instance without that code, whose register budget
 // it would otherwise raise.
-template <bool FUSE>
-__device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
+// RAW (SyrkParams): A and B of problem i are rows of the caller's Z through p.zmap[i].
+template <bool FUSE, class P>
+__device__ __forceinline__ void gemm_tc2_body(const P &p) {
+  constexpr bool RAW = std::is_same<P, SyrkParams>::value;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
@@ -158,7 +162,16 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
           // > the operand's row tile) MN-major from its mirror.
           const bool a_mn = (q.major & kAMn) || ((q.major & kASym) && (kb >> 2) > (t.m0 >> 8));
           const bool b_mn = (q.major & kBMn) || ((q.major & kBSym) && (kb >> 2) > (t.n0 >> 8));
-          if (!a_mn) {
+          if constexpr (RAW) {
+            // Columns kb*64 .. +127 of Z's rows am .. am+127 and bn .. bn+127; the tensor map
+            // swizzles them into the same image as a stored panel, and reads zeros past the
+            // last row or column.
+            const CUtensorMap *zm = &p.zmap[t.prob];
+            tma_load_2sm(sA, zm, kb * 64, am, fb);
+            tma_load_2sm(sA + SLICE_BYTES, zm, kb * 64 + 64, am, fb);
+            tma_load_2sm(sB, zm, kb * 64, bn, fb);
+            tma_load_2sm(sB + SLICE_BYTES, zm, kb * 64 + 64, bn, fb);
+          } else if (!a_mn) {
             const int64_t ya = a_row + (int64_t)kb * q.a_ph + am;
             tma_load_2sm(sA, &p.tmap, 0, (int)ya, fb);
             tma_load_2sm(sA + SLICE_BYTES, &p.tmap, 0, (int)(ya + q.a_ph), fb);
@@ -167,7 +180,8 @@ __device__ __forceinline__ void gemm_tc2_body(const GemmParams &p) {
             tma_load_2sm(sA, &p.tmap, 0, (int)y0, fb);
             tma_load_2sm(sA + SLICE_BYTES, &p.tmap, 0, (int)(y0 + q.a_ph), fb);
           }
-          if (!b_mn) {
+          if (RAW) {
+          } else if (!b_mn) {
             const int64_t yb = b_row + (int64_t)kb * q.b_ph + bn;
             tma_load_2sm(sB, &p.tmap, 0, (int)yb, fb);
             tma_load_2sm(sB + SLICE_BYTES, &p.tmap, 0, (int)(yb + q.b_ph), fb);
@@ -462,23 +476,31 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_kernel(const __grid_cons
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc2_fused_kernel(const __grid_constant__ GemmParams p) {
   gemm_tc2_body<true>(p);
 }
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc2_syrk_kernel(const __grid_constant__ SyrkParams p) {
+  gemm_tc2_body<false>(p);
+}
 
 std::mutex g_tmap_mu;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
+// The driver's tensor-map encoder, looked up once.
+cudaError_t load_encoder() {
+  std::lock_guard<std::mutex> g(g_tmap_mu);
+  if (!g_encode) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return e != cudaSuccess ? e : cudaErrorNotSupported;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  return cudaSuccess;
+}
+
 }  // namespace
 
 cudaError_t encode_ws_tensor_map(CUtensorMap *map, void *ws, size_t bytes) {
-  {
-    std::lock_guard<std::mutex> g(g_tmap_mu);
-    if (!g_encode) {
-      void *fn = nullptr;
-      cudaDriverEntryPointQueryResult q;
-      cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-      if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return e != cudaSuccess ? e : cudaErrorNotSupported;
-      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    }
-  }
+  cudaError_t e = load_encoder();
+  if (e != cudaSuccess) return e;
   const cuuint64_t dims[2] = {64, (cuuint64_t)(bytes / 128)};
   const cuuint64_t strides[1] = {128};
   const cuuint32_t box[2] = {64, 128};
@@ -489,21 +511,39 @@ cudaError_t encode_ws_tensor_map(CUtensorMap *map, void *ws, size_t bytes) {
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t launch_gemm_tc2(const GemmParams &p, int num_sms, cudaStream_t s) {
-  static PerDevice attr_set;  // the attribute is set once per device
-  int dev = 0;
-  cudaGetDevice(&dev);
+cudaError_t encode_z_tensor_map(CUtensorMap *map, const void *z, int64_t d, int64_t n) {
+  cudaError_t e = load_encoder();
+  if (e != cudaSuccess) return e;
+  if (d <= 0 || n <= 0 || n % 64 != 0 || reinterpret_cast<uintptr_t>(z) % 16 != 0) return cudaErrorInvalidValue;
+  const cuuint64_t dims[2] = {(cuuint64_t)n, (cuuint64_t)d};
+  const cuuint64_t strides[1] = {(cuuint64_t)n * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(z), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+namespace {
+
+int set_up_device(int dev, int num_sms, cudaError_t *err) {
+  static PerDevice attr_set;  // the attributes are set once per device
   if (!attr_set.get(dev)) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(gemm_tc2_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemm_tc2_syrk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) {
+      *err = e;
+      return 0;
+    }
     attr_set.set(dev, 1);
   }
-  const bool fused = p.mode == kUpdate && p.partials != nullptr;
-  if (p.total_tiles <= 0) return cudaSuccess;
   // Pairs that can be resident at once (a GPC with an odd number of free SMs leaves one
-  // idle), so that the persistent grid never spills into a second wave.
+  // idle), so that the persistent grid never spills into a second wave.  The three kernels
+  // have the same shape.
   static PerDevice max_pairs;
   int mp = max_pairs.get(dev);
   if (!mp) {
@@ -526,6 +566,17 @@ cudaError_t launch_gemm_tc2(const GemmParams &p, int num_sms, cudaStream_t s) {
     mp = n < num_sms / 2 ? n : num_sms / 2;
     max_pairs.set(dev, mp);
   }
+  return mp;
+}
+
+template <class P>
+cudaError_t launch_pairs(void (*kernel)(P), const P &p, int num_sms, cudaStream_t s) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaError_t err = cudaSuccess;
+  const int mp = set_up_device(dev, num_sms, &err);
+  if (!mp) return err;
+  if (p.total_tiles <= 0) return cudaSuccess;
   const int clusters = p.total_tiles < mp ? p.total_tiles : mp;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters, 1, 1);
@@ -541,9 +592,21 @@ cudaError_t launch_gemm_tc2(const GemmParams &p, int num_sms, cudaStream_t s) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  cudaError_t e = fused ? cudaLaunchKernelEx(&cfg, gemm_tc2_fused_kernel, p) : cudaLaunchKernelEx(&cfg, gemm_tc2_kernel, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc2(const GemmParams &p, int num_sms, cudaStream_t s) {
+  const bool fused = p.mode == kUpdate && p.partials != nullptr;
+  return launch_pairs(fused ? gemm_tc2_fused_kernel : gemm_tc2_kernel, p, num_sms, s);
+}
+
+cudaError_t launch_gemm_syrk(const SyrkParams &p, int num_sms, cudaStream_t s) {
+  if (p.mode != kGramF32) return cudaErrorInvalidValue;
+  return launch_pairs(gemm_tc2_syrk_kernel, p, num_sms, s);
 }
 
 }  // namespace nshb

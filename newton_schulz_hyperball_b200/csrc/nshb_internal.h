@@ -175,7 +175,7 @@ constexpr int kPwTiled = 4;  // batch b is the T x T tile (b / w_tiles_c, b % w_
 constexpr int kPwVec = 8;    // W rows may be read with 16-byte loads
 constexpr int kPartsPerTile = 16;   // partial records per 256 x 256 tile (one per epilogue warp)
 enum GemmMode { kGram = 0, kPoly = 1, kUpdate = 2, kGramF32 = 5 };
-struct GemmParams {
+struct GemmHead {
   CUtensorMap tmap;       // 2-SM kernel: the workspace seen as rows of 128 bytes (64 bf16),
                           // 64-row boxes, no swizzle (the data is stored pre-swizzled)
   char *ws;
@@ -183,15 +183,27 @@ struct GemmParams {
   uint32_t *status;
   double *partials;       // kUpdate: (||O||^2, <W,O>, ||W||^2) records of problems with w, or NULL
   long long wait_limit;   // clock cycles a role may wait on one mbarrier phase
-  int32_t mode;           // kGram: D = s^2 acc (lower triangle + mirror)
-                          // kPoly: D = cb C + cc acc (lower triangle + mirror)
+  int32_t mode;           // kGram: D = s^2 acc (tiles on and below the diagonal)
+                          // kPoly: D = cb C + cc acc (tiles on and below the diagonal)
                           // kUpdate: D = s (ca C + acc), B operand MN-major; C may be a
                           //          hi + lo pair and D may be written as one
+                          // kGramF32: D = acc in fp32 (tiles on and below the diagonal)
   float ca, cb, cc;
   int32_t nprob, total_tiles;
   int32_t test_stall;     // tests only: the MMA warp withholds its first accumulator commit,
                           // so the epilogue's bounded wait runs out (NSHB_DEV_TIMEOUT)
+};
+struct GemmParams : GemmHead {
   GemmProb prob[kMaxProb];
+};
+// The Gram S = Z Z^T of the Newton-Muon layer inputs, read straight from the caller's
+// row-major bf16 Z (d x n): problem i's A and B operands come through zmap[i] (128-byte
+// swizzled boxes of 64 columns x 128 rows, zeros outside Z), the fp32 result goes to the
+// workspace (c_off / d_off) as in kGramF32.
+constexpr int kMaxZMaps = 64;
+struct SyrkParams : GemmHead {
+  GemmProb prob[kMaxZMaps];
+  CUtensorMap zmap[kMaxZMaps];
 };
 
 // Tile-resident Hierarchical Muon (T = 256): one record per tiled matrix; its tiles are
@@ -246,14 +258,6 @@ struct F32Params {
 };
 
 // Newton-Muon helpers.
-struct PackParams {          // row-major bf16 (rows x cols, ld) -> panel layout (ph rows)
-  const void *src[kMaxMats];
-  int64_t dst_off[kMaxMats];
-  int32_t rows[kMaxMats], cols[kMaxMats], ld[kMaxMats], ph[kMaxMats];
-  int32_t blk_begin[kMaxMats + 1];
-  char *ws;
-  int32_t n;
-};
 struct CholParams {          // the ridge of a batch of layer-input Gram matrices
   char *ws;
   uint32_t *status;
@@ -340,14 +344,16 @@ cudaError_t launch_apply(const ApplyParams &p, cudaStream_t s);
 cudaError_t launch_adam(const AdamParams &p, cudaStream_t s);
 // 2-SM (CTA pair) form: 256 x 256 tiles, tcgen05.mma.cta_group::2; p.tmap must be encoded.
 cudaError_t launch_gemm_tc2(const GemmParams &p, int num_sms, cudaStream_t s);
+cudaError_t launch_gemm_syrk(const SyrkParams &p, int num_sms, cudaStream_t s);
 // Tile-resident Hierarchical Muon for T = 256 (all iterations of a tile on one CTA pair).
 cudaError_t launch_himuon_tile(const HmParams &p, int num_sms, cudaStream_t s);
 // The same for T = 128, one tile per CTA, two CTAs per SM.
 cudaError_t launch_himuon_tile128(const HmParams &p, int num_sms, cudaStream_t s);
 // Encodes p.tmap for a workspace of `bytes` bytes at `ws` (host; driver entry point).
 cudaError_t encode_ws_tensor_map(CUtensorMap *map, void *ws, size_t bytes);
+// Row-major bf16 d x n (n a multiple of 64, 16-byte aligned): 64 x 128 boxes, 128-byte swizzle.
+cudaError_t encode_z_tensor_map(CUtensorMap *map, const void *z, int64_t d, int64_t n);
 cudaError_t launch_gemm_f32(const F32Params &p, cudaStream_t s);
-cudaError_t launch_pack_panels(const PackParams &p, cudaStream_t s);
 cudaError_t launch_ridge(const CholParams &p, cudaStream_t s);
 // reserve_pairs: SM pairs left to a kernel that runs beside this one (the grid is that much
 // smaller, so that every CTA pair is resident from the start).
@@ -364,7 +370,7 @@ static_assert(sizeof(AdamParams) <= kMaxParamBytes, "AdamParams");
 static_assert(sizeof(GemmParams) <= kMaxParamBytes, "GemmParams");
 static_assert(sizeof(HmParams) <= kMaxParamBytes, "HmParams");
 static_assert(sizeof(F32Params) <= kMaxParamBytes, "F32Params");
-static_assert(sizeof(PackParams) <= kMaxParamBytes, "PackParams");
+static_assert(sizeof(SyrkParams) <= kMaxParamBytes, "SyrkParams");
 static_assert(sizeof(CholParams) <= kMaxParamBytes, "CholParams");
 static_assert(sizeof(NwParams) <= kMaxParamBytes, "NwParams");
 static_assert(sizeof(SplitParams) <= kMaxParamBytes, "SplitParams");

@@ -230,8 +230,9 @@ def test_newton_muon_workspace_and_step_checks_before_launch():
     m = newton_mats([768, 768, 3072], [0, 0, 1])
     a = nshb.workspace_size(m, p, nshb.NSHB_OP_NEWTON_MUON, z_rows=[768, 3072], n_tokens=4096)
     b = nshb.workspace_size(m, p, nshb.NSHB_OP_NEWTON_MUON, z_rows=[768, 3072], n_tokens=8192)
-    # the bf16 panel copy of every Z grows with the token count: (768 + 3072) x 4096 x 2 bytes more
-    assert b - a >= (768 + 3072) * 4096 * 2
+    # Z is read where the caller keeps it (no copy), so the workspace does not grow with the
+    # token count
+    assert b == a
     assert a > nshb.workspace_size(m, p, nshb.NSHB_OP_HYPERBALL)
     with pytest.raises(nshb.NshbError) as e:   # Newton-Muon runs the bf16 NS only
         nshb.workspace_size(m, nshb.params(ns_precision=nshb.NSHB_F32), nshb.NSHB_OP_NEWTON_MUON,

@@ -460,6 +460,34 @@ def test_bf16_newton_muon_small():
         assert abs(o.fro(Wg[i]) - rhos[i]) / rhos[i] <= radius_tol(Wg[i], True)
 
 
+def test_bf16_newton_muon_odd_token_panels():
+    """A token count of 320 (five 64-wide panels, so the last 128-deep stage of S = Z Z^T
+    runs past the end of Z, where the tensor map reads zeros) and layer inputs of 192 and
+    448 rows (the last 256-row tile of S partly past Z's rows)."""
+    from gpu_harness import newton_step
+    cfg = wl.CFG_NEWTON_GPT2
+    n_tok = 320
+    Zs = [wl.layer_input(cfg, 20, 192, n_tok), wl.layer_input(cfg, 21, 448, n_tok)]
+    shapes = [(256, 192), (130, 448), (448, 448)]
+    zi = [0, 1, 1]
+    Ws = [wl.init_weight(cfg, 80 + i, r, c, bf16=True).astype(np.float64) for i, (r, c) in enumerate(shapes)]
+    Gs = [wl.gradient(cfg, 80 + i, 0, r, c, bf16=True).astype(np.float64) for i, (r, c) in enumerate(shapes)]
+    rhos = [o.fro(w) for w in Ws]
+    gs = GpuSet(Ws, bf16=True)
+    for k in range(len(shapes)):
+        gs.mats[k].z_index = zi[k]
+    gs.set_grads(Gs)
+    rho_dev = torch.tensor(rhos, dtype=torch.float32, device="cuda")
+    p = nshb.params(eta=0.02, rho=rho_dev, ridge_rel=1e-3)
+    assert newton_step(gs, Zs, n_tok, p) == 0
+    Wg, Mg, Og = gs.host()
+    for i, W in enumerate(Ws):
+        Wr, Mr, Or, _ = o.newton_muon_step(W, Gs[i], np.zeros_like(W), Zs[zi[i]].astype(np.float64),
+                                           ridge_rel=1e-3, eta=0.02, rho=rhos[i])
+        assert rel_fro(Og[i], Or) <= 2e-2, (i, rel_fro(Og[i], Or))
+        assert abs(o.fro(Wg[i]) - rhos[i]) / rhos[i] <= radius_tol(Wg[i], True)
+
+
 # ------------------------------------------------- determinism, schedules, graphs
 def test_steps_are_bit_deterministic():
     """Fixed-order reductions, no float atomics: two runs on the same inputs agree bit for bit."""
