@@ -193,6 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1) himuon_tile_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const long long limit = p.wait_limit;
+  if (warp == 0 && lane == 0) prefetch_tmap(&p.tmap);
   pdl_trigger();
   pdl_wait();                             // X0, its low part and the scales are written
   const int K = p.ns_steps;
@@ -565,6 +566,7 @@ __global__ void __launch_bounds__(kThreads1, kCtasPerSm1) himuon_tile128_kernel(
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const long long limit = p.wait_limit;
+  if (warp == 0 && lane == 0) prefetch_tmap(&p.tmap);
   pdl_trigger();
   pdl_wait();
   const int K = p.ns_steps;

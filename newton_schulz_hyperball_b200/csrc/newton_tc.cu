@@ -96,6 +96,7 @@ __global__ void __launch_bounds__(kThreads, 1) newton_gemm_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const long long limit = p.wait_limit;
+  if (warp == 0 && lane == 0) prefetch_tmap(&p.tmap);
   pdl_trigger();
   if (!p.late_wait) pdl_wait();
 

@@ -126,6 +126,13 @@ __device__ __forceinline__ void gemm_tc2_body(const P &p) {
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const long long limit = p.wait_limit;
+  if (warp == 0 && lane == 0) {
+    if constexpr (RAW) {
+      if (cid < p.total_tiles) prefetch_tmap(&p.zmap[decode2(p, cid).prob]);
+    } else {
+      prefetch_tmap(&p.tmap);
+    }
+  }
   pdl_trigger();
   pdl_wait();                                      // the previous kernel's outputs are visible
 
