@@ -69,12 +69,15 @@ struct Plan {
     int64_t s = 0;                    // S = Z Z^T + lambda I, fp32 Dp x Dp, updated in place
     int64_t sh = 0, sl = 0;           // bf16 hi / lo panels of S (operands of the panel products)
     int64_t lh = 0, ll = 0;           // bf16 hi / lo panels of the Cholesky factor L
-    int64_t dh = 0, dl = 0;           // hi / lo panels of the stacked diagonal-block inverses (Dp x 256)
+    int64_t dh = 0, dl = 0;           // hi / lo panels of the stacked inverses of the 512 x 512 diagonal
+                                      // blocks (Dp x 512): rows 512 j .. +511 hold the inverse of
+                                      // L's diagonal block j of 512 (block k of 256 at columns 256 (k % 2))
   };
   std::vector<ZPlan> zp;
   int64_t n_tokens = 0;
   std::vector<int64_t> r_off;         // per matrix: fp32 m x n, U (momentum) and then P
   std::vector<int64_t> y32, yh, yl;   // per matrix: fp32 Mp x Dp U -> Y, and its hi / lo panels
+  std::vector<int64_t> ph, plo;       // per matrix: hi / lo panels of P (Mp x Dp), the backward's operand
   std::vector<int64_t> mpad;          // per matrix: rows padded to 256
   std::vector<int> zidx;
   size_t scal_off = 0, scale_off = 0, nu_off = 0, k1part_off = 0, wpart_off = 0, xpart_off = 0, total = 0;
@@ -255,13 +258,15 @@ nshb_status plan_newton(const nshb_matrix *mats, int n_mats, const void *const *
     z.sl = off; off = align_up(off + sq * 2);
     z.lh = off; off = align_up(off + sq * 2);
     z.ll = off; off = align_up(off + sq * 2);
-    z.dh = off; off = align_up(off + (size_t)z.Dp * 256 * 2);
-    z.dl = off; off = align_up(off + (size_t)z.Dp * 256 * 2);
+    z.dh = off; off = align_up(off + (size_t)z.Dp * 512 * 2);
+    z.dl = off; off = align_up(off + (size_t)z.Dp * 512 * 2);
   }
   pl.r_off.resize(n_mats);
   pl.y32.resize(n_mats);
   pl.yh.resize(n_mats);
   pl.yl.resize(n_mats);
+  pl.ph.resize(n_mats);
+  pl.plo.resize(n_mats);
   pl.mpad.resize(n_mats);
   pl.zidx.resize(n_mats);
   for (int i = 0; i < n_mats; ++i) {
@@ -275,6 +280,8 @@ nshb_status plan_newton(const nshb_matrix *mats, int n_mats, const void *const *
     pl.y32[i] = off;   off = align_up(off + (size_t)Mp * Dp * 4);
     pl.yh[i] = off;    off = align_up(off + (size_t)Mp * Dp * 2);
     pl.yl[i] = off;    off = align_up(off + (size_t)Mp * Dp * 2);
+    pl.ph[i] = off;    off = align_up(off + (size_t)Mp * Dp * 2);
+    pl.plo[i] = off;   off = align_up(off + (size_t)Mp * Dp * 2);
   }
   pl.total = off;
   return NSHB_OK;
@@ -959,56 +966,93 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
     }
     return NSHB_OK;
   };
-  // 5. backward, P L = Y by block columns from the last, left-looking as well:
-  //    W = Y[:, k] - P[:, k1:] L[k1:, k] (one product over every later column of P; only its
-  //    hi / lo panels are kept, in place of Y[:, k]), then P[:, k] = W D_k (fp32 into the m x n
-  //    buffer the momentum pass reads, and hi / lo panels in place of W).  A matrix whose layer
-  //    input has g block columns runs 2g - 1 stages (solve g-1, column g-2, solve g-2, ..., solve
-  //    0); its stages start as soon as its forward sweep is over, one per launch, so the matrices
-  //    of narrow layer inputs finish theirs inside the forward sweep of the wide ones (in the
-  //    launches beside the diagonal blocks) and the rest continue after it.
+  // 5. backward, P L = Y by block columns of 512 from the last, left-looking as well:
+  //    W = Y[:, K] - P[:, K1:] L[K1:, K] (one product over every later column of P; only its
+  //    hi / lo panels are kept, in place of Y[:, K]), then P[:, K] = W E_K with E_K the inverse
+  //    of L's 512 x 512 diagonal block K (fp32 into the m x n buffer the momentum pass reads, and
+  //    hi / lo panels of P).  E_K = [D_a 0; X D_b] for the 256-blocks a = 2j, b = 2j + 1, with
+  //    X = -D_b L_ba D_a formed during the forward sweep; a last block of 256 has E = D.  A
+  //    matrix whose layer input has G blocks of 512 runs 2G - 1 stages (solve G-1, column
+  //    G-2, solve G-2, ..., solve 0); its stages start as soon as its forward sweep is over,
+  //    one per launch, so the matrices of narrow layer inputs finish theirs inside the forward
+  //    sweep of the wide ones (in the launches beside the diagonal blocks) and the rest
+  //    continue after it.
+  auto n_super = [&](const Plan::ZPlan &z) { return (int)((z.Dp / 256 + 1) / 2); };
   auto bwd_stage = [&](int i, int s, std::vector<NwProb> &out) {
     const Plan::ZPlan &z = pl.zp[pl.zidx[i]];
-    const int g = (int)(z.Dp / 256);
-    const int kk = g - 1 - (s + 1) / 2;
-    const int64_t k0 = 256LL * kk, k1 = k0 + 256;
+    const int G = n_super(z);
+    const int jj = G - 1 - (s + 1) / 2;
+    const int64_t K0 = 512LL * jj, wj = std::min<int64_t>(512, z.Dp - K0), K1 = K0 + wj;
     if (s % 2 == 1) {
       NwProb t = nw_prob();
-      t.a_hi = pl.yh[i]; t.a_lo = pl.yl[i]; t.a_ph = (int)pl.mpad[i]; t.a_r0 = 0; t.a_k0 = (int)k1;
-      t.b_hi = z.lh; t.b_lo = z.ll; t.b_ph = (int)z.Dp; t.b_r0 = (int)k0; t.b_k0 = (int)k1;
-      t.kt = (int)((z.Dp - k1) / 64);
+      t.a_hi = pl.ph[i]; t.a_lo = pl.plo[i]; t.a_ph = (int)pl.mpad[i]; t.a_r0 = 0; t.a_k0 = (int)K1;
+      t.b_hi = z.lh; t.b_lo = z.ll; t.b_ph = (int)z.Dp; t.b_r0 = (int)K0; t.b_k0 = (int)K1;
+      t.kt = (int)((z.Dp - K1) / 64);
       t.flags = kNwBMn;
-      t.c32 = pl.y32[i] + k0 * 4; t.ld32 = (int)z.Dp;
-      t.m_valid = (int)pl.mpad[i]; t.n_valid = 256;
-      t.dhi = pl.yh[i]; t.dlo = pl.yl[i]; t.d_ph = (int)pl.mpad[i]; t.d_r0 = 0; t.d_c0 = (int)k0;
-      t.mt = (int)(pl.mpad[i] / 256); t.nt = 1;
+      t.c32 = pl.y32[i] + K0 * 4; t.ld32 = (int)z.Dp;
+      t.m_valid = (int)pl.mpad[i]; t.n_valid = (int)wj;
+      t.dhi = pl.yh[i]; t.dlo = pl.yl[i]; t.d_ph = (int)pl.mpad[i]; t.d_r0 = 0; t.d_c0 = (int)K0;
+      t.mt = (int)(pl.mpad[i] / 256); t.nt = (int)(wj / 256);
       out.push_back(t);
     } else {
       const int d = (int)pl.mp[i].n, m = (int)pl.mp[i].m;
       NwProb q = nw_prob();
-      q.a_hi = pl.yh[i]; q.a_lo = pl.yl[i]; q.a_ph = (int)pl.mpad[i]; q.a_r0 = 0; q.a_k0 = (int)k0;
-      q.b_hi = z.dh; q.b_lo = z.dl; q.b_ph = (int)z.Dp; q.b_r0 = 0; q.b_k0 = (int)k0;
+      q.a_hi = pl.yh[i]; q.a_lo = pl.yl[i]; q.a_ph = (int)pl.mpad[i]; q.a_r0 = 0; q.a_k0 = (int)K0;
+      q.b_hi = z.dh; q.b_lo = z.dl; q.b_ph = (int)z.Dp; q.b_r0 = 0; q.b_k0 = (int)K0;
+      q.kt = (int)(wj / 64);
       q.flags = kNwBMn;
-      q.d32 = pl.r_off[i] + k0 * 4; q.ld32 = d; q.m_valid = m; q.n_valid = (int)std::max<int64_t>(0, d - k0);
-      q.dhi = pl.yh[i]; q.dlo = pl.yl[i]; q.d_ph = (int)pl.mpad[i]; q.d_r0 = 0; q.d_c0 = (int)k0;
-      q.mt = (int)(pl.mpad[i] / 256); q.nt = 1;
+      q.d32 = pl.r_off[i] + K0 * 4; q.ld32 = d; q.m_valid = m; q.n_valid = (int)std::max<int64_t>(0, d - K0);
+      q.dhi = pl.ph[i]; q.dlo = pl.plo[i]; q.d_ph = (int)pl.mpad[i]; q.d_r0 = 0; q.d_c0 = (int)K0;
+      q.mt = (int)(pl.mpad[i] / 256); q.nt = (int)(wj / 256);
       out.push_back(q);
     }
   };
-  // stage k - g of every matrix whose g block columns are done by step k (0 <= k - g <= 2g - 2)
+  // A matrix whose forward sweep ends well before the last step (g + 2G - 2 < nb - 1) starts
+  // its stages 0 .. R-1 steps late, matrices in turn, so that the launches beside the diagonal
+  // blocks carry about 1/R of every stage instead of whole stages in a few of them.
+  std::vector<int> bwd_off(n, 0);
+  for (int i = 0, turn = 0; i < n; ++i) {
+    const Plan::ZPlan &z = pl.zp[pl.zidx[i]];
+    const int g = (int)(z.Dp / 256), R = std::min(6, nb - 1 - (g + 2 * n_super(z) - 2) + 1);
+    if (R > 1) bwd_off[i] = turn++ % R;
+  }
+  // stage k - g - off of every matrix whose g block columns of 256 are done by step k
+  // (0 <= k - g - off <= 2G - 2)
   auto bwd_stages = [&](int k, std::vector<NwProb> &out) {
     for (int i = 0; i < n; ++i) {
-      const int g = (int)(pl.zp[pl.zidx[i]].Dp / 256), s = k - g;
-      if (s >= 0 && s <= 2 * g - 2) bwd_stage(i, s, out);
+      const Plan::ZPlan &z = pl.zp[pl.zidx[i]];
+      const int g = (int)(z.Dp / 256), s = k - g - bwd_off[i];
+      if (s >= 0 && s <= 2 * n_super(z) - 2) bwd_stage(i, s, out);
     }
   };
   for (int k = 0; k < nb; ++k) {
     const int64_t k0 = 256LL * k, k1 = k0 + 256;
+    const int dcol = (k & 1) * 256;       // column of D_k in the stack of 512-wide inverses
     std::vector<NwProb> col_s, col_u, panel;
     int ndiag = 0;
     for (auto &z : pl.zp) {
       if (z.Dp <= k0) continue;
       ++ndiag;
+      if (k & 1) {
+        // the lower-left block X = -D_k L[k0:k1, k-1] D_{k-1} of the inverse of the 512 x 512
+        // diagonal block (k-1, k), in two products over the columns 0 .. 255 of block row k of
+        // the stack: T = L[k0:k1, k-1] D_{k-1} beside the diagonal blocks (both factors are
+        // done), then X = -D_k T after them (one tile, so T is read before X replaces it)
+        NwProb t = nw_prob();
+        t.a_hi = z.lh; t.a_lo = z.ll; t.a_ph = (int)z.Dp; t.a_r0 = (int)k0; t.a_k0 = (int)(k0 - 256);
+        t.b_hi = z.dh; t.b_lo = z.dl; t.b_ph = (int)z.Dp; t.b_r0 = 0; t.b_k0 = (int)(k0 - 256);
+        t.flags = kNwBMn;
+        t.dhi = z.dh; t.dlo = z.dl; t.d_ph = (int)z.Dp; t.d_r0 = (int)k0; t.d_c0 = 0;
+        t.mt = 1; t.nt = 1;
+        col_u.push_back(t);
+        NwProb x = nw_prob();
+        x.a_hi = z.dh; x.a_lo = z.dl; x.a_ph = (int)z.Dp; x.a_r0 = (int)k0; x.a_k0 = 256;
+        x.b_hi = z.dh; x.b_lo = z.dl; x.b_ph = (int)z.Dp; x.b_r0 = 0; x.b_k0 = (int)k0;
+        x.flags = kNwBMn | kNwNeg;
+        x.dhi = z.dh; x.dlo = z.dl; x.d_ph = (int)z.Dp; x.d_r0 = (int)k0; x.d_c0 = 0;
+        x.mt = 1; x.nt = 1;
+        panel.push_back(x);
+      }
       if (k > 0) {
         // T = S[k0:, k] - L[k0:, k-1] L[k0:k1, k-1]^T, the last term of the column's update
         // (the others were applied beside the previous step's diagonal blocks), fp32 in place
@@ -1037,7 +1081,7 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
       // L[k1:, k] = T[k1:] D_k^T
       NwProb q = nw_prob();
       q.a_hi = z.sh; q.a_lo = z.sl; q.a_ph = (int)z.Dp; q.a_r0 = (int)k1; q.a_k0 = (int)k0;
-      q.b_hi = z.dh; q.b_lo = z.dl; q.b_ph = (int)z.Dp; q.b_r0 = (int)k0; q.b_k0 = 0;
+      q.b_hi = z.dh; q.b_lo = z.dl; q.b_ph = (int)z.Dp; q.b_r0 = (int)k0; q.b_k0 = dcol;
       q.dhi = z.lh; q.dlo = z.ll; q.d_ph = (int)z.Dp; q.d_r0 = (int)k1; q.d_c0 = (int)k0;
       q.mt = (int)((z.Dp - k1) / 256); q.nt = 1;
       panel.push_back(q);
@@ -1060,7 +1104,7 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
       // Y[:, k] = V D_k^T
       NwProb q = nw_prob();
       q.a_hi = pl.yh[i]; q.a_lo = pl.yl[i]; q.a_ph = (int)pl.mpad[i]; q.a_r0 = 0; q.a_k0 = (int)k0;
-      q.b_hi = z.dh; q.b_lo = z.dl; q.b_ph = (int)z.Dp; q.b_r0 = (int)k0; q.b_k0 = 0;
+      q.b_hi = z.dh; q.b_lo = z.dl; q.b_ph = (int)z.Dp; q.b_r0 = (int)k0; q.b_k0 = dcol;
       q.d32 = pl.y32[i] + k0 * 4; q.ld32 = (int)z.Dp; q.m_valid = (int)pl.mpad[i]; q.n_valid = 256;
       q.dhi = pl.yh[i]; q.dlo = pl.yl[i]; q.d_ph = (int)pl.mpad[i]; q.d_r0 = 0; q.d_c0 = (int)k0;
       q.mt = (int)(pl.mpad[i] / 256); q.nt = 1;
@@ -1085,7 +1129,12 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
     if (e != NSHB_OK) return e;
   }
   // the remaining backward stages, one launch per stage index
-  for (int k = nb; k <= 3 * nb - 2; ++k) {
+  int k_end = 0;
+  for (int i = 0; i < n; ++i) {
+    const Plan::ZPlan &z = pl.zp[pl.zidx[i]];
+    k_end = std::max(k_end, (int)(z.Dp / 256) + bwd_off[i] + 2 * n_super(z) - 2);
+  }
+  for (int k = nb; k <= k_end; ++k) {
     std::vector<NwProb> stage;
     bwd_stages(k, stage);
     nshb_status e = run_nw(np, stage, st);

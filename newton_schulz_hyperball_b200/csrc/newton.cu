@@ -392,6 +392,7 @@ __global__ void __launch_bounds__(kDiagThreads, 1) potrf_diag_kernel(const __gri
     __syncthreads();
   }
   // out: rows k0 .. k0+255, columns 0 .. 255 of the stack, eight columns per 16-byte piece
+  const int cofs = (p.k & 1) * 256;
   for (int q = threadIdx.x; q < 256 * 32; q += kDiagThreads) {
     const int r = q >> 5, c = 8 * (q & 31), i = r >> 5, k = c >> 5;
     uint4 h = make_uint4(0, 0, 0, 0), l = h;
@@ -406,9 +407,17 @@ __global__ void __launch_bounds__(kDiagThreads, 1) potrf_diag_kernel(const __gri
         lp[e] = pack_bf16(v[2 * e] - bf16lo(hp[e]), v[2 * e + 1] - bf16hi(hp[e]));
       }
     }
-    const size_t off = panel_chunk_off(k0 + r, c, ld);
+    // block k's inverse goes to columns 256 (k % 2) .. +255 of the 512-wide stack; an even
+    // block also zeroes columns 256 .. 511 of its rows, the upper-right block of the inverse
+    // of the 512 x 512 diagonal block it forms with block k + 1
+    const size_t off = panel_chunk_off(k0 + r, cofs + c, ld);
     *reinterpret_cast<uint4 *>(hi + off) = h;
     *reinterpret_cast<uint4 *>(lo + off) = l;
+    if (cofs == 0) {
+      const size_t zo = panel_chunk_off(k0 + r, 256 + c, ld);
+      *reinterpret_cast<uint4 *>(hi + zo) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4 *>(lo + zo) = make_uint4(0, 0, 0, 0);
+    }
   }
 }
 

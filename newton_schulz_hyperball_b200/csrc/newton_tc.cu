@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1) newton_gemm_kernel(const __grid_c
       const int buf = tl & 1;
       const uint32_t tph = (uint32_t)(tl >> 1) & 1u;
       const int64_t i = t.m0 + row;                        // row of the output region
-      const bool sub = q.c32 >= 0;
+      const bool sub = q.c32 >= 0, neg = q.flags & kNwNeg;
       const float *crow = sub ? reinterpret_cast<const float *>(p.ws + q.c32) + i * q.ld32 + t.n0 : nullptr;
       float *drow = q.d32 >= 0 ? reinterpret_cast<float *>(p.ws + q.d32) + i * q.ld32 + t.n0 : nullptr;
       const bool valid = i < q.m_valid;                   // rows past the valid region are not written
@@ -251,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1) newton_gemm_kernel(const __grid_c
         tmem_ld_wait();
         float v[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = sub ? c[e] - __uint_as_float(r[e]) : __uint_as_float(r[e]);
+        for (int e = 0; e < 32; ++e) v[e] = sub ? c[e] - __uint_as_float(r[e]) : neg ? -__uint_as_float(r[e]) : __uint_as_float(r[e]);
         const int cvalid = q.n_valid - (t.n0 + col0);       // columns of this chunk that exist
         if (drow && valid && cvalid >= 32) {
 #pragma unroll

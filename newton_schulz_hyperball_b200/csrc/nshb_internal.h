@@ -278,6 +278,7 @@ void record_cuda_error(cudaError_t e);
 // D = A B^T (B K-major), D = A B (B MN-major) or D = C - A B^(T), over 256 x 256 tiles of
 // one M x N region, with A = A_hi + A_lo and B = B_hi + B_lo held as bf16 panel matrices.
 constexpr int kNwBMn = 1;     // B MN-major
+constexpr int kNwNeg = 2;     // D = -A B (no C)
 constexpr int kMaxNwProb = 200;
 struct NwProb {
   int64_t a_hi, a_lo, b_hi, b_lo;  // panel matrices of A and B (workspace byte offsets of panel 0)
@@ -290,7 +291,7 @@ struct NwProb {
   int32_t ld32;                    // row stride (elements) of the fp32 C and D
   int32_t m_valid, n_valid;        // rows / columns of the fp32 D region that exist
   int32_t mt, nt, kt;              // 256-row tiles, 256-column tiles, 64-deep k panels (even)
-  int32_t flags;                   // kNwBMn
+  int32_t flags;                   // kNwBMn | kNwNeg
   int32_t tile_begin;
 };
 struct NwParams {
