@@ -48,10 +48,10 @@ E2E_PIPELINE = "H2D of step k+1 on a second stream during step k (2 device buffe
 # says what was captured.
 CSRC = os.path.join(ROOT, "newton_schulz_hyperball_b200", "csrc")
 TRAFFIC = {
-    "gemm_qwen3": {"source": "ns_tc2.cu", "sha256_prefix": "f9696084335066a3", "bytes_per_launch": 4475861436,
-                   "case": "4 of the 28 Qwen3-style layers (28 matrices), one step's 15 launches: 9.59 GB "
+    "gemm_qwen3": {"source": "ns_tc2.cu", "sha256_prefix": "04b0c7ee8b4b7441", "bytes_per_launch": 4470472531,
+                   "case": "4 of the 28 Qwen3-style layers (28 matrices), one step's 15 launches: 9.58 GB "
                            "DRAM read + write, 0.639 GB per launch, x7 for the 28 identical layers"},
-    "gemm_gpt2": {"source": "ns_tc2.cu", "sha256_prefix": "f9696084335066a3", "bytes_per_launch": 260810957,
+    "gemm_gpt2": {"source": "ns_tc2.cu", "sha256_prefix": "04b0c7ee8b4b7441", "bytes_per_launch": 260381952,
                   "case": "GPT-2-small set, 15 launches of one step averaged"},
     "adam_gpt2": {"source": "stream_kernels.cu", "sha256_prefix": "1ac6016cf38009db",
                   "bytes_per_launch": 1813149184, "case": "GPT-2-small set, one launch"},
