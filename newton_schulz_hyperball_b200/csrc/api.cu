@@ -280,8 +280,18 @@ nshb_status plan_newton(const nshb_matrix *mats, int n_mats, const void *const *
     pl.y32[i] = off;   off = align_up(off + (size_t)Mp * Dp * 4);
     pl.yh[i] = off;    off = align_up(off + (size_t)Mp * Dp * 2);
     pl.yl[i] = off;    off = align_up(off + (size_t)Mp * Dp * 2);
-    pl.ph[i] = off;    off = align_up(off + (size_t)Mp * Dp * 2);
-    pl.plo[i] = off;   off = align_up(off + (size_t)Mp * Dp * 2);
+  }
+  // The backward solve writes P's hi / lo panels (Mp x Dp, the NS operand's layout: panel
+  // height round_up(m, 256), width round_up(n, 256), either orientation) straight into X0 and
+  // its low part.
+  for (int i = 0; i < n_mats; ++i) {
+    const int64_t Mp = pl.mpad[i], Dp = pl.zp[pl.zidx[i]].Dp;
+    pl.ph[i] = pl.mp[i].x0;
+    pl.plo[i] = pl.mp[i].xl0;
+    if (pl.plo[i] < 0) {   // no compensated NS iteration: the backward still needs P's low part
+      pl.plo[i] = off;
+      off = align_up(off + (size_t)Mp * Dp * 2);
+    }
   }
   pl.total = off;
   return NSHB_OK;
@@ -428,7 +438,9 @@ nshb_status run_momentum(const nshb_matrix *mats, const Plan &pl, const nshb_par
     for (int i = c0; i < c1; ++i) {
       mp.mats[i - c0] = make_desc(mats[i], pl.mp[i], i, 0, nb, true);
       if (from_p) {
-        mp.mats[i - c0].flags |= kFromP;
+        // P's hi / lo panels, which the backward solve wrote where the NS reads X0, already
+        // are the operand: the pass only forms the norm
+        mp.mats[i - c0].flags |= kFromP | kNoX;
         mp.mats[i - c0].u_off = pl.r_off[i];
       }
       nb += pl.mp[i].k1_blocks;

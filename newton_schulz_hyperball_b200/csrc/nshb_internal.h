@@ -41,6 +41,8 @@ constexpr int kNsF32 = 16;      // NS in fp32, X row-major fp32 (else bf16 panel
 constexpr int kTileMajor = 32;  // block list enumerates tile by tile (momentum of tiled matrices)
 constexpr int kFromP = 64;      // momentum kernel: take U from an fp32 row-major matrix (no momentum)
 constexpr int kURow = 128;      // momentum kernel: write U as fp32 row-major only (Newton-Muon input)
+constexpr int kNoX = 256;       // momentum kernel: the NS operand is already in place (Newton-Muon:
+                                // the backward solve wrote P's hi / lo panels), only the norm
 
 // Per-matrix record of a streaming launch (momentum, reductions, apply).
 struct MatDesc {

@@ -327,7 +327,7 @@ __device__ __forceinline__ void momentum_block(const MomentumParams &p, const Ma
         sT[0][rq + 32 * h][cq + e] = u[e];
         if (lo_part) sT[1][rq + 32 * h][cq + e] = ul[e];
       }
-    } else {
+    } else if (!(d.flags & kNoX)) {
       x_store8(xbase, d, i, j, u, F32);
       if (lo_part) x_store8(lbase, d, i, j, ul, F32);
     }
