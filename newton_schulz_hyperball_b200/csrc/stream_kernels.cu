@@ -158,17 +158,16 @@ __device__ __forceinline__ void store8(void *base, int64_t ld, int i, int j, int
   }
 }
 
-// Address of X element block for the tiled layout: tile (tr, tc) is a T x T panel matrix.
-__device__ __forceinline__ const char *tile_base(const char *xbase, const MatDesc &d, int r, int c) {
-  const int64_t T = d.ph;
-  const int64_t tl = (int64_t)(r / T) * d.tiles_c + (c / T);
-  return xbase + tl * T * T * 2;
-}
-
 // Byte offset (from xbase) of the 16-byte chunk holding X row xr, columns xc..xc+7 of a
-// bf16 X (panel layout, or a grid of T x T panel tiles when tiled).
+// bf16 X (panel layout, or a grid of T x T panel tiles when tiled: tile (tr, tc), a T x T
+// panel matrix, is tile tr * tiles_c + tc).  T (= ph) is 128, 256 or 512, so the tile and
+// the position in it come from shifts and masks rather than divisions.
 __device__ __forceinline__ const char *x_chunk(const char *xbase, const MatDesc &d, int xr, int xc) {
-  if (d.flags & kTiled) return tile_base(xbase, d, xr, xc) + panel_chunk_off(xr % d.ph, xc % d.ph, d.ph);
+  if (d.flags & kTiled) {
+    const int lg = __ffs(d.ph) - 1, mask = d.ph - 1;
+    const int64_t tl = (int64_t)(xr >> lg) * d.tiles_c + (xc >> lg);
+    return xbase + (tl << (2 * lg + 1)) + panel_chunk_off(xr & mask, xc & mask, d.ph);
+  }
   return xbase + panel_chunk_off(xr, xc, d.ph);
 }
 
