@@ -109,7 +109,8 @@ __global__ void __launch_bounds__(256) split_kernel(const __grid_constant__ Spli
 //      D_jk = -sum_{k <= m < j} X_jm D_mk  (from D L = I).
 // Step j + 1's A runs inside step j's C: the warp that updates block (j + 1, j + 1) factors
 // it right away while the other warps finish the rest of C.  The result goes out as bf16
-// hi / lo panels (block k of the inverse stack), with zeros above the diagonal.  A pivot that
+// hi / lo panels into the stack of 512-wide inverses (rows 256 k, columns 256 (k % 2)), with
+// zeros above the diagonal.  A pivot that
 // is not positive in fp32 is flagged (NSHB_DEV_NOT_SPD) and replaced by 1e-30.
 constexpr int kNB = 8;                    // block columns
 constexpr int kBS = 36;                   // row stride of a block (floats): conflict-free float4 rows

@@ -327,7 +327,9 @@ struct SplitParams {
 };
 
 // Cholesky factor and inverse of one 256 x 256 diagonal block per layer input (column
-// block k), written as the bf16 hi/lo panels of a stack of inverses (block k at rows 256 k).
+// block k), written as bf16 hi/lo panels into the stack of the 512 x 512 diagonal blocks'
+// inverses (Dp x 512): block k at rows 256 k, columns 256 (k % 2); an even block also
+// zeroes columns 256 .. 511 of its rows.
 struct DiagParams {
   char *ws;
   uint32_t *status;
