@@ -318,7 +318,7 @@ class Stepper:
                                        n_tokens=self.w.extra["n_tokens"])
         return self.nshb.workspace(mats, self.p, self.op, device=dev)
 
-    def __call__(self, mats, ws, stream):
+    def __call__(self, mats, ws, stream, Z=None):
         nshb, s = self.nshb, self.w.step
         if s == "hyperball":
             nshb.hyperball_step(mats, self.p, ws, stream)
@@ -327,22 +327,26 @@ class Stepper:
         elif s == "himuon":
             nshb.himuon_step(mats, self.p, ws, stream)
         elif s == "newton":
-            nshb.newton_muon_step(mats, self.Z, self.w.extra["n_tokens"], self.p, ws, stream)
+            nshb.newton_muon_step(mats, self.Z if Z is None else Z, self.w.extra["n_tokens"], self.p, ws, stream)
         else:
             self.count += 1
             nshb.adamh_step(mats, self.V, nshb.adam_params(step=self.count), self.p, ws, stream)
 
 
-def timed_e2e(Gh, stepper, ws, stream, ke, torch, dev):
-    """End to end through the public API with host buffers: every step's gradients are copied
-    host->device from pinned memory and the step's device status word is read back.  The copy
-    of step k+1 runs on a second stream while step k computes (two device buffers, events
-    in both directions), as an input pipeline would; all copies lie inside the timed region.
-    Gh: list of pinned host gradient sets (used in turn)."""
+def timed_e2e(Gh, stepper, ws, stream, ke, torch, dev, Zh=None):
+    """End to end through the public API with host buffers: every step's gradients (and, for
+    Newton-Muon, its layer inputs Z) are copied host->device from pinned memory and the step's
+    device status word is read back.  The copy of step k+1 runs on a second stream while step
+    k computes (two device buffers, events in both directions), as an input pipeline would;
+    all copies lie inside the timed region.
+    Gh: list of pinned host gradient sets (used in turn); Zh: pinned host layer inputs."""
     bufs = [[torch.empty(g.shape, dtype=g.dtype, device=dev) for g in Gh[0]] for _ in range(2)]
+    zbufs = [[torch.empty(z.shape, dtype=z.dtype, device=dev) for z in Zh] for _ in range(2)] if Zh else None
     mats_b = [stepper.mats(bufs[j]) for j in range(2)]
     st_host = torch.empty(1, dtype=torch.int32).pin_memory()
     h2d = sum(g.numel() * g.element_size() for g in Gh[0])
+    if Zh:
+        h2d += sum(z.numel() * z.element_size() for z in Zh)
     copy_stream = torch.cuda.Stream(device=dev)
     copied = [torch.cuda.Event() for _ in range(2)]
     consumed = [torch.cuda.Event() for _ in range(2)]
@@ -359,6 +363,9 @@ def timed_e2e(Gh, stepper, ws, stream, ke, torch, dev):
                 copy_stream.wait_event(consumed[j])
             for d, s_ in zip(bufs[j], Gh[k % len(Gh)]):
                 d.copy_(s_, non_blocking=True)
+            if zbufs:
+                for d, s_ in zip(zbufs[j], Zh):
+                    d.copy_(s_, non_blocking=True)
             copied[j].record(copy_stream)
 
     issue_copy(0)
@@ -367,13 +374,13 @@ def timed_e2e(Gh, stepper, ws, stream, ke, torch, dev):
             issue_copy(k + 1)
         j = k % 2
         stream.wait_event(copied[j])
-        stepper(mats_b[j], ws, stream)
+        stepper(mats_b[j], ws, stream, Z=zbufs[j] if zbufs else None)
         consumed[j].record(stream)
         st_host.copy_(ws[:4].view(torch.int32), non_blocking=True)
     t1.record(stream)
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / ke
-    del bufs, mats_b
+    del bufs, zbufs, mats_b
     return ms, h2d
 
 
@@ -464,11 +471,19 @@ def run_cuda(args, rank, world, local_rank, w: Workload):
                 h.copy_(g)
                 hs.append(h)
             Gh.append(hs)
+        Zh = None
+        if Z is not None:
+            # a training step's layer inputs arrive with its gradients
+            Zh = []
+            for z in Z:
+                h = torch.empty(z.shape, dtype=z.dtype, pin_memory=True)
+                h.copy_(z)
+                Zh.append(h)
         del Gd, mats
         torch.cuda.empty_cache()
         ke = max(5, min(args.steps, 20))
         barrier()
-        e2e_one, h2d = timed_e2e(Gh, stepper, ws, stream, ke, torch, dev)
+        e2e_one, h2d = timed_e2e(Gh, stepper, ws, stream, ke, torch, dev, Zh)
         barrier()
         e2e_ms = max_over_ranks(e2e_one)
         del Gh
