@@ -1019,14 +1019,48 @@ nshb_status run_newton_precond(const nshb_matrix *mats, const Plan &pl, const ns
       out.push_back(q);
     }
   };
-  // A matrix whose forward sweep ends well before the last step (g + 2G - 2 < nb - 1) starts
-  // its stages 0 .. R-1 steps late, matrices in turn, so that the launches beside the diagonal
-  // blocks carry about 1/R of every stage instead of whole stages in a few of them.
-  std::vector<int> bwd_off(n, 0);
-  for (int i = 0, turn = 0; i < n; ++i) {
+  // A matrix whose forward sweep ends well before the last step (g + 2G - 2 < nb - 1) may start
+  // its stages up to R - 1 steps late.  The delays are chosen greedily, largest matrices first,
+  // to even out the work of the launches beside the diagonal blocks: each launch's estimated
+  // cost (per 256 x 256 tile, its k panels times the three products plus an epilogue's worth)
+  // starts from the early terms of the next S column and the update of U's column, and every
+  // matrix takes the delay that leaves the largest launch its stages touch the smallest.
+  auto tile_cost = [](int64_t tiles, int64_t kt) { return (double)tiles * (double)(3 * kt + 24); };
+  std::vector<double> load(nb > 0 ? nb : 1, 0.0);
+  for (int k = 1; k < nb; ++k) {
+    const int64_t k0 = 256LL * k, k1 = k0 + 256;
+    for (auto &z : pl.zp)
+      if (z.Dp > k1) load[k] += tile_cost((z.Dp - k1) / 256, k0 / 64);
+    for (int i = 0; i < n; ++i)
+      if (pl.zp[pl.zidx[i]].Dp > k0) load[k] += tile_cost(pl.mpad[i] / 256, k0 / 64);
+  }
+  auto stage_cost = [&](int i, int s) {
     const Plan::ZPlan &z = pl.zp[pl.zidx[i]];
-    const int g = (int)(z.Dp / 256), R = std::min(6, nb - 1 - (g + 2 * n_super(z) - 2) + 1);
-    if (R > 1) bwd_off[i] = turn++ % R;
+    const int G = n_super(z), jj = G - 1 - (s + 1) / 2;
+    const int64_t K0 = 512LL * jj, wj = std::min<int64_t>(512, z.Dp - K0), K1 = K0 + wj;
+    const int64_t tiles = (pl.mpad[i] / 256) * (wj / 256);
+    return s % 2 == 1 ? tile_cost(tiles, (z.Dp - K1) / 64) : tile_cost(tiles, wj / 64);
+  };
+  std::vector<int> bwd_off(n, 0), order;
+  for (int i = 0; i < n; ++i) {
+    const Plan::ZPlan &z = pl.zp[pl.zidx[i]];
+    const int g = (int)(z.Dp / 256);
+    if (nb - g - 2 * n_super(z) + 2 > 1) order.push_back(i);
+  }
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return pl.mpad[a] > pl.mpad[b]; });
+  for (int i : order) {
+    const Plan::ZPlan &z = pl.zp[pl.zidx[i]];
+    const int g = (int)(z.Dp / 256), ns = 2 * n_super(z) - 1;
+    const int R = std::min(8, nb - g - ns + 1);
+    int best = 0;
+    double best_peak = 0.0;
+    for (int o = 0; o < R; ++o) {
+      double peak = 0.0;
+      for (int st = 0; st < ns; ++st) peak = std::max(peak, load[g + o + st] + stage_cost(i, st));
+      if (o == 0 || peak < best_peak) { best = o; best_peak = peak; }
+    }
+    bwd_off[i] = best;
+    for (int st = 0; st < ns; ++st) load[g + best + st] += stage_cost(i, st);
   }
   // stage k - g - off of every matrix whose g block columns of 256 are done by step k
   // (0 <= k - g - off <= 2G - 2)
