@@ -750,7 +750,7 @@ __device__ __forceinline__ void apply_block(const MatDesc &d, int cr0, int cc0, 
 
 // Register prefetch of the next block (F32 as for momentum_kernel).
 template <bool F32>
-__global__ void __launch_bounds__(kThreads, F32 ? 2 : 3) apply_kernel(const __grid_constant__ ApplyParams p) {
+__global__ void __launch_bounds__(kThreads, F32 ? 2 : 4) apply_kernel(const __grid_constant__ ApplyParams p) {
   pdl_trigger();
   pdl_wait();
   __shared__ float sO[kBlk][kBlk + 1];
