@@ -239,13 +239,13 @@ __device__ __forceinline__ void cluster_sync() {
 __device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
-// 2-D TMA load into this CTA's shared memory; the transaction bytes complete on the
-// barrier at cluster address `bar` (the leader's barrier).  No multicast.
 // Pulls a tensor map (a kernel parameter) into the TMA unit's descriptor cache ahead of its
 // first use, e.g. while the kernel waits for the previous one.
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
+// 2-D TMA load into this CTA's shared memory; the transaction bytes complete on the
+// barrier at cluster address `bar` (the leader's barrier).  No multicast.
 __device__ __forceinline__ void tma_load_2sm(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
