@@ -281,14 +281,21 @@ nshb_status plan_newton(const nshb_matrix *mats, int n_mats, const void *const *
     pl.yh[i] = off;    off = align_up(off + (size_t)Mp * Dp * 2);
     pl.yl[i] = off;    off = align_up(off + (size_t)Mp * Dp * 2);
   }
-  // The backward solve writes P's hi / lo panels (Mp x Dp, the NS operand's layout: panel
-  // height round_up(m, 256), width round_up(n, 256), either orientation) straight into X0 and
-  // its low part.
+  // The backward solve writes P's hi / lo panels (Mp x Dp) straight into X0 and its low part
+  // when they are the NS operand's layout (bf16 panels of height round_up(m, 256) and width
+  // round_up(n, 256), either orientation).  A matrix whose NS runs in fp32 (fewer than 32 rows)
+  // gets panels of its own, and the pass after the solve writes its X0 from the fp32 P.
   for (int i = 0; i < n_mats; ++i) {
+    const MatPlan &m = pl.mp[i];
     const int64_t Mp = pl.mpad[i], Dp = pl.zp[pl.zidx[i]].Dp;
-    pl.ph[i] = pl.mp[i].x0;
-    pl.plo[i] = pl.mp[i].xl0;
-    if (pl.plo[i] < 0) {   // no compensated NS iteration: the backward still needs P's low part
+    const bool in_place = !m.f32 && m.pr == Mp && m.pc == Dp;
+    pl.ph[i] = in_place ? m.x0 : -1;
+    pl.plo[i] = in_place ? m.xl0 : -1;
+    if (pl.ph[i] < 0) {
+      pl.ph[i] = off;
+      off = align_up(off + (size_t)Mp * Dp * 2);
+    }
+    if (pl.plo[i] < 0) {   // also when no compensated NS iteration keeps a low part of X0
       pl.plo[i] = off;
       off = align_up(off + (size_t)Mp * Dp * 2);
     }
@@ -438,9 +445,9 @@ nshb_status run_momentum(const nshb_matrix *mats, const Plan &pl, const nshb_par
     for (int i = c0; i < c1; ++i) {
       mp.mats[i - c0] = make_desc(mats[i], pl.mp[i], i, 0, nb, true);
       if (from_p) {
-        // P's hi / lo panels, which the backward solve wrote where the NS reads X0, already
-        // are the operand: the pass only forms the norm
-        mp.mats[i - c0].flags |= kFromP | kNoX;
+        // Where the backward solve wrote P's hi / lo panels into X0 they already are the
+        // operand, and the pass only forms the norm; otherwise it writes X0 from the fp32 P.
+        mp.mats[i - c0].flags |= kFromP | (pl.ph[i] == pl.mp[i].x0 ? kNoX : 0);
         mp.mats[i - c0].u_off = pl.r_off[i];
       }
       nb += pl.mp[i].k1_blocks;
